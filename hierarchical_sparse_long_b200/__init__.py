@@ -1,0 +1,11 @@
+"""B200-native Hierarchical Global Attention (HGA) layer.
+
+The compute lives in ``libhga.so`` (hand-written sm_100a CUDA, C ABI in
+include/hga.h); this package is its ctypes binding plus a small driver for
+segment-by-segment processing.
+"""
+from .binding import (  # noqa: F401
+    HGA_BF16, HGA_FP32, HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT, EXPORTED, HGAError, Params, lib,
+    hga_build_summaries, hga_route, hga_attn_fwd, hga_attn_bwd_workspace_size, hga_attn_bwd,
+    hga_fetch_tiered, hga_get_device_status,
+)

@@ -1,0 +1,182 @@
+"""Thin ctypes binding of ``libhga.so`` (the C ABI declared in include/hga.h).
+
+Argument marshalling only: every step of the layer runs in the library's
+CUDA kernels.  Tensors are torch tensors (device tensors on the current CUDA
+device, page-locked host tensors for the tiered history); the stream is the
+caller's current torch stream unless one is given.  A missing or unloadable
+library raises ``HGAError`` -- there is no other implementation to fall back
+to.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import os
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libhga.so")
+
+HGA_BF16, HGA_FP32 = 0, 1
+HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT = 1, 2
+STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3: "HGA_ERR_CUDA",
+          -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
+
+EXPORTED = ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
+            "hga_fetch_tiered", "hga_get_device_status", "hga_status_string", "hga_last_error")
+
+
+class HGAError(RuntimeError):
+    def __init__(self, code: int, what: str, detail: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {STATUS.get(code, code)}" + (f" ({detail})" if detail else ""))
+
+
+class CParams(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int), ("n_q_heads", ctypes.c_int), ("n_kv_heads", ctypes.c_int),
+                ("head_dim", ctypes.c_int), ("chunk", ctypes.c_int), ("q_block", ctypes.c_int),
+                ("topk", ctypes.c_int), ("seg_len", ctypes.c_int), ("n_hist_chunks", ctypes.c_int),
+                ("dtype", ctypes.c_int), ("hist_head_stride", ctypes.c_longlong),
+                ("seg_head_stride", ctypes.c_longlong), ("qblock_begin", ctypes.c_int),
+                ("qblock_end", ctypes.c_int)]
+
+
+@dataclasses.dataclass
+class Params:
+    """Mirror of ``hga_params_t`` (strides in tokens; 0/0 block range = all blocks)."""
+    batch: int
+    n_q_heads: int
+    n_kv_heads: int
+    head_dim: int
+    topk: int
+    seg_len: int
+    n_hist_chunks: int
+    dtype: int = HGA_BF16
+    hist_head_stride: int = -1  # -1: n_hist_chunks * chunk
+    seg_head_stride: int = -1   # -1: seg_len
+    chunk: int = 64
+    q_block: int = 64
+    qblock_begin: int = 0
+    qblock_end: int = 0
+
+    def c(self) -> CParams:
+        hs = self.hist_head_stride if self.hist_head_stride >= 0 else self.n_hist_chunks * self.chunk
+        ss = self.seg_head_stride if self.seg_head_stride >= 0 else self.seg_len
+        return CParams(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.chunk, self.q_block,
+                       self.topk, self.seg_len, self.n_hist_chunks, self.dtype, hs, ss, self.qblock_begin,
+                       self.qblock_end)
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Loads libhga.so (raises HGAError if it is missing)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise HGAError(-2, "libhga.so is not built",
+                           "run `python -m hierarchical_sparse_long_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, ll, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_longlong, ctypes.c_size_t
+        pp = ctypes.POINTER(CParams)
+        L.hga_build_summaries.argtypes = [vp, ll, i, i, i, i, i, i, i, vp, i, vp]
+        L.hga_route.argtypes = [pp, vp, vp, i, vp, vp]
+        L.hga_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.hga_attn_bwd_workspace_size.argtypes = [pp]
+        L.hga_attn_bwd_workspace_size.restype = sz
+        L.hga_attn_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
+        L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+        L.hga_status_string.argtypes = [i]
+        L.hga_status_string.restype = ctypes.c_char_p
+        L.hga_last_error.restype = ctypes.c_char_p
+        for f in ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_fetch_tiered",
+                  "hga_get_device_status"):
+            getattr(L, f).restype = ctypes.c_int
+        _lib = L
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != 0:
+        detail = lib().hga_last_error().decode() if rc == -3 else ""
+        raise HGAError(rc, what, detail)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def dtype_code(t) -> int:
+    import torch
+    if t.dtype == torch.bfloat16:
+        return HGA_BF16
+    if t.dtype == torch.float32:
+        return HGA_FP32
+    raise HGAError(-1, "unsupported tensor dtype", str(t.dtype))
+
+
+def hga_build_summaries(k, head_stride: int, batch: int, n_kv_heads: int, head_dim: int, chunk: int,
+                        first_chunk: int, n_chunks: int, summ, summ_cap_chunks: int, stream=None):
+    """Chunk summaries (mean of keys) for chunks [first_chunk, first_chunk + n_chunks)."""
+    _check(lib().hga_build_summaries(_ptr(k), head_stride, batch, n_kv_heads, head_dim, chunk, first_chunk,
+                                     n_chunks, dtype_code(k), _ptr(summ), summ_cap_chunks, _stream(stream)),
+           "hga_build_summaries")
+
+
+def hga_route(p: Params, q, summ, summ_cap_chunks: int, idx, stream=None):
+    """Top-k chunk routing per (batch, kv head, query block) into idx (int32)."""
+    cp = p.c()
+    _check(lib().hga_route(ctypes.byref(cp), _ptr(q), _ptr(summ), summ_cap_chunks, _ptr(idx), _stream(stream)),
+           "hga_route")
+
+
+def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stream=None):
+    """Exact-token attention forward over routed chunks + the causal segment."""
+    cp = p.c()
+    _check(lib().hga_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg),
+                              _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)), "hga_attn_fwd")
+
+
+def hga_attn_bwd_workspace_size(p: Params) -> int:
+    cp = p.c()
+    return int(lib().hga_attn_bwd_workspace_size(ctypes.byref(cp)))
+
+
+def hga_attn_bwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, dout, dq, dk_seg, dv_seg,
+                 workspace, stream=None):
+    """Backward with frozen routes: dq (history + segment keys), dk/dv of the segment only."""
+    cp = p.c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().hga_attn_bwd(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg),
+                              _ptr(idx), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk_seg), _ptr(dv_seg),
+                              _ptr(workspace), nbytes, _stream(stream)), "hga_attn_bwd")
+
+
+def hga_fetch_tiered(p: Params, host_k, host_v, idx, qblock_begin: int, qblock_end: int, stage_k, stage_v,
+                     stage_slots: int, slot_map, idx_remapped, n_fetched=None, copy_stream=None, done=None):
+    """Copies only the routed chunks' K/V tiles from pinned host memory into staging slots."""
+    cp = p.c()
+    ev = None if done is None else ctypes.c_void_p(done.cuda_event)
+    _check(lib().hga_fetch_tiered(ctypes.byref(cp), _ptr(host_k), _ptr(host_v), _ptr(idx), qblock_begin,
+                                  qblock_end, _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(slot_map),
+                                  _ptr(idx_remapped), _ptr(n_fetched), _stream(copy_stream), ev),
+           "hga_fetch_tiered")
+
+
+def hga_get_device_status(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the device status bits."""
+    bits = ctypes.c_uint(0)
+    rc = lib().hga_get_device_status(_stream(stream), ctypes.byref(bits))
+    if rc not in (0, -4, -5):
+        _check(rc, "hga_get_device_status")
+    return bits.value

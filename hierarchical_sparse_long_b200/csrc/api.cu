@@ -1,0 +1,197 @@
+// C ABI of the HGA library: argument validation, kernel selection and the
+// device status word.  Every check runs on the host before anything is
+// enqueued, so a rejected call leaves the stream untouched.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+
+namespace {
+
+__device__ unsigned int g_status_word;
+
+thread_local std::string t_last_error;
+
+constexpr int kMaxDevices = 64;
+unsigned *g_status_ptr[kMaxDevices];
+std::mutex g_status_mu;
+
+// Address of this device's status word (looked up once per device with the
+// device current, as the symbol's host-side name is not a device address).
+unsigned *status_ptr() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    std::lock_guard<std::mutex> lock(g_status_mu);
+    if (!g_status_ptr[dev]) {
+        void *ptr = nullptr;
+        if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
+        g_status_ptr[dev] = static_cast<unsigned *>(ptr);
+    }
+    return g_status_ptr[dev];
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape checks shared by route / fwd / bwd / fetch.
+hga_status_t check_params(const hga_params_t *p) {
+    if (!p) return HGA_ERR_INVALID_ARG;
+    if (p->batch < 1 || p->n_q_heads < 1 || p->n_kv_heads < 1) return HGA_ERR_INVALID_ARG;
+    if (p->n_q_heads % p->n_kv_heads) return HGA_ERR_INVALID_ARG;
+    if (p->dtype != HGA_BF16 && p->dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
+    if (p->head_dim != 64 && p->head_dim != 128) return HGA_ERR_UNSUPPORTED;
+    if (p->chunk != 64 || p->q_block != 64) return HGA_ERR_UNSUPPORTED;
+    if (p->topk < 1 || p->topk > 64) return HGA_ERR_INVALID_ARG;
+    if (p->seg_len < 1 || p->seg_len % p->q_block || p->seg_len % p->chunk) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks < 0) return HGA_ERR_INVALID_ARG;
+    if (p->seg_head_stride < p->seg_len) return HGA_ERR_INVALID_ARG;
+    if (p->hist_head_stride < 0) return HGA_ERR_INVALID_ARG;
+    if (p->hist_head_stride != 0 && p->hist_head_stride < (long long)p->n_hist_chunks * p->chunk)
+        return HGA_ERR_INVALID_ARG;
+    const int nqb = p->seg_len / p->q_block;
+    if (!(p->qblock_begin == 0 && p->qblock_end == 0)) {
+        if (p->qblock_begin < 0 || p->qblock_end <= p->qblock_begin || p->qblock_end > nqb)
+            return HGA_ERR_INVALID_ARG;
+    }
+    return HGA_OK;
+}
+
+}  // namespace
+
+namespace hga {
+hga_status_t record_cuda(cudaError_t e) {
+    if (e == cudaSuccess) return HGA_OK;
+    t_last_error = cudaGetErrorString(e);
+    return HGA_ERR_CUDA;
+}
+}  // namespace hga
+
+extern "C" {
+
+const char *hga_status_string(hga_status_t s) {
+    switch (s) {
+    case HGA_OK: return "HGA_OK";
+    case HGA_ERR_INVALID_ARG: return "HGA_ERR_INVALID_ARG";
+    case HGA_ERR_UNSUPPORTED: return "HGA_ERR_UNSUPPORTED";
+    case HGA_ERR_CUDA: return "HGA_ERR_CUDA";
+    case HGA_ERR_DEVICE_CHECK: return "HGA_ERR_DEVICE_CHECK";
+    case HGA_ERR_TIMEOUT: return "HGA_ERR_TIMEOUT";
+    }
+    return "HGA_ERR_UNKNOWN";
+}
+
+const char *hga_last_error(void) { return t_last_error.c_str(); }
+
+hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch, int n_kv_heads, int head_dim,
+                                 int chunk, int first_chunk, int n_chunks, hga_dtype_t dtype, float *summ,
+                                 int summ_cap_chunks, cudaStream_t stream) {
+    if (batch < 1 || n_kv_heads < 1 || n_chunks < 0 || first_chunk < 0 || chunk < 1) return HGA_ERR_INVALID_ARG;
+    if (dtype != HGA_BF16 && dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
+    if (head_dim != 64 && head_dim != 128) return HGA_ERR_UNSUPPORTED;
+    if ((long long)first_chunk + n_chunks > summ_cap_chunks) return HGA_ERR_INVALID_ARG;
+    if (head_stride < (long long)(first_chunk + n_chunks) * chunk) return HGA_ERR_INVALID_ARG;
+    if (n_chunks == 0) return HGA_OK;
+    if (!k || !summ || !aligned16(k) || !aligned16(summ)) return HGA_ERR_INVALID_ARG;
+    return hga::launch_summaries(k, head_stride, batch * n_kv_heads, head_dim, chunk, first_chunk, n_chunks, dtype,
+                                 summ, summ_cap_chunks, stream);
+}
+
+hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks, int32_t *idx,
+                       cudaStream_t stream) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (summ_cap_chunks < p->n_hist_chunks) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 16384) return HGA_ERR_UNSUPPORTED;
+    if (!q || !idx || !aligned16(q)) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!summ || !aligned16(summ))) return HGA_ERR_INVALID_ARG;
+    return hga::launch_route(*p, q, summ, summ_cap_chunks, idx, stream);
+}
+
+hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                          const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
+                          cudaStream_t stream) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (!q || !k_seg || !v_seg || !idx || !out || !lse) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {q, k_hist, v_hist, k_seg, v_seg, (const void *)out})
+        if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    if (hga::attn_fwd_tc_supported(*p))
+        return hga::launch_attn_fwd_tc(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status, stream);
+    return hga::launch_attn_fwd_simt(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status, stream);
+}
+
+size_t hga_attn_bwd_workspace_size(const hga_params_t *p) {
+    if (check_params(p) != HGA_OK) return 0;
+    const size_t rows = (size_t)p->batch * p->n_q_heads * p->seg_len;
+    return ((rows * sizeof(float)) + 255) & ~(size_t)255;
+}
+
+hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                          const void *k_seg, const void *v_seg, const int32_t *idx, const void *out,
+                          const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg, void *workspace,
+                          size_t workspace_bytes, cudaStream_t stream) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (p->qblock_begin != 0 || p->qblock_end != 0) return HGA_ERR_INVALID_ARG;
+    if (!q || !k_seg || !v_seg || !idx || !out || !lse || !dout || !dq || !dk_seg || !dv_seg || !workspace)
+        return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
+    if (workspace_bytes < hga_attn_bwd_workspace_size(p)) return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {q, k_hist, v_hist, k_seg, v_seg, out, dout, (const void *)dq, (const void *)dk_seg,
+                            (const void *)dv_seg, (const void *)workspace})
+        if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    return hga::launch_attn_bwd_simt(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, dout, dq, dk_seg, dv_seg,
+                                     static_cast<float *>(workspace), status, stream);
+}
+
+hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,
+                              int qblock_begin, int qblock_end, void *stage_k, void *stage_v, int stage_slots,
+                              int32_t *slot_map, int32_t *idx_remapped, int32_t *n_fetched, cudaStream_t copy_stream,
+                              cudaEvent_t done) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    const int nqb = p->seg_len / p->q_block;
+    if (qblock_begin < 0 || qblock_end <= qblock_begin || qblock_end > nqb) return HGA_ERR_INVALID_ARG;
+    if (p->hist_head_stride < (long long)p->n_hist_chunks * p->chunk) return HGA_ERR_INVALID_ARG;
+    if (!host_k || !host_v || !idx || !stage_k || !stage_v || !slot_map || !idx_remapped || stage_slots < 0)
+        return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {host_k, host_v, (const void *)stage_k, (const void *)stage_v})
+        if (!aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    const int keff = p->topk < p->n_hist_chunks ? p->topk : p->n_hist_chunks;
+    const long long worst = (long long)(qblock_end - qblock_begin) * p->batch * p->n_kv_heads * keff;
+    const long long distinct = (long long)p->batch * p->n_kv_heads * p->n_hist_chunks;
+    if ((worst < distinct ? worst : distinct) > stage_slots) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, qblock_begin, qblock_end, stage_k, stage_v, stage_slots,
+                                  slot_map, idx_remapped, n_fetched, status, copy_stream);
+    if (st != HGA_OK) return st;
+    if (done) return hga::record_cuda(cudaEventRecord(done, copy_stream));
+    return HGA_OK;
+}
+
+hga_status_t hga_get_device_status(cudaStream_t stream, unsigned int *bits) {
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    cudaError_t e = cudaStreamSynchronize(stream);
+    if (e != cudaSuccess) return hga::record_cuda(e);
+    unsigned v = 0;
+    e = cudaMemcpy(&v, status, sizeof(v), cudaMemcpyDeviceToHost);
+    if (e != cudaSuccess) return hga::record_cuda(e);
+    const unsigned zero = 0;
+    e = cudaMemcpy(status, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) return hga::record_cuda(e);
+    if (bits) *bits = v;
+    if (v & HGA_DEV_TIMEOUT) return HGA_ERR_TIMEOUT;
+    if (v) return HGA_ERR_DEVICE_CHECK;
+    return HGA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,76 @@
+// Shared device helpers of the HGA CUDA library (sm_100a).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "hga.h"
+
+namespace hga {
+
+// Device status word bits (mirrors HGA_DEV_* in hga.h).
+constexpr unsigned kDevBadIndex = HGA_DEV_BAD_INDEX;
+constexpr unsigned kDevTimeout = HGA_DEV_TIMEOUT;
+
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+template <typename T> __device__ __forceinline__ T from_f32(float x);
+template <> __device__ __forceinline__ float from_f32<float>(float x) { return x; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// Loads VEC = 16 / sizeof(T) consecutive elements (one 16-byte vector) as fp32.
+template <typename T> struct Vec16;
+template <> struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ __forceinline__ static void load(const float *p, float *out) {
+        float4 v = *reinterpret_cast<const float4 *>(p);
+        out[0] = v.x; out[1] = v.y; out[2] = v.z; out[3] = v.w;
+    }
+};
+template <> struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ __forceinline__ static void load(const __nv_bfloat16 *p, float *out) {
+        uint4 v = *reinterpret_cast<const uint4 *>(p);
+        const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            out[2 * i] = __uint_as_float(w[i] << 16);
+            out[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    }
+};
+
+}  // namespace hga
+
+// Host-side launchers (one translation unit each); all validate nothing --
+// the C ABI layer has already checked every argument.
+namespace hga {
+hga_status_t launch_summaries(const void *k, long long head_stride, int bh, int head_dim, int chunk,
+                              int first_chunk, int n_chunks, hga_dtype_t dtype, float *summ, int cap,
+                              cudaStream_t stream);
+hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
+                          cudaStream_t stream);
+hga_status_t launch_attn_fwd_simt(const hga_params_t &p, const void *q, const void *k_hist,
+                                  const void *v_hist, const void *k_seg, const void *v_seg,
+                                  const int32_t *idx, void *out, float *lse, unsigned *status,
+                                  cudaStream_t stream);
+hga_status_t launch_attn_bwd_simt(const hga_params_t &p, const void *q, const void *k_hist,
+                                  const void *v_hist, const void *k_seg, const void *v_seg,
+                                  const int32_t *idx, const void *out, const float *lse, const void *dout,
+                                  void *dq, void *dk_seg, void *dv_seg, float *delta, unsigned *status,
+                                  cudaStream_t stream);
+bool attn_fwd_tc_supported(const hga_params_t &p);
+hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *k_hist,
+                                const void *v_hist, const void *k_seg, const void *v_seg,
+                                const int32_t *idx, void *out, float *lse, unsigned *status,
+                                cudaStream_t stream);
+hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
+                                 const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
+                                 int stage_slots, int32_t *slot_map, int32_t *idx_remapped,
+                                 int32_t *n_fetched, unsigned *status, cudaStream_t stream);
+hga_status_t record_cuda(cudaError_t e);
+}  // namespace hga

@@ -1,0 +1,203 @@
+/*
+ * hga.h -- C ABI of the B200 (sm_100a) Hierarchical Global Attention layer.
+ *
+ * What the layer computes is described in "Long-Context Fine-Tuning with
+ * Limited VRAM" (Fedosov, Sazhin, Grinenko, Woernle; the gist.science
+ * technical summary, sections 2.1 "Hierarchical Global Attention" and 2.2
+ * "Segment-wise backward and tiered storage", and the author abstract):
+ * the context is cut into fixed 64-token chunks; a compact summary of every
+ * closed chunk stays resident on the GPU; each query block scores those
+ * summaries, keeps the best history chunks and attends, with exact softmax,
+ * to the exact keys/values of those chunks together with a local window;
+ * routing carries no gradient; training runs segment by segment and only the
+ * active segment is differentiable; detached history may live in host memory.
+ *
+ * Readings fixed by this library where the pages leave a step open:
+ *   chunk summary       = mean of the chunk's keys, per KV head (fp32);
+ *   query-block summary = mean of the block's queries over the G query heads
+ *                         of the KV group (q head h reads KV head h / G);
+ *   score               = fp32 dot(query-block summary, chunk summary)/sqrt(D);
+ *   selection           = the min(k, Nc) best chunks by (score descending,
+ *                         chunk index ascending), listed in ascending chunk
+ *                         order and padded with -1;
+ *   local window        = every active-segment token at or before the query;
+ *   no attention sink and no 8-token group stage.
+ * Query i of the active segment therefore attends exactly
+ * min(k, Nc) * chunk + i + 1 tokens.
+ *
+ * Conventions for every entry point:
+ *   - The caller owns all memory.  Device pointers are CUDA device (or
+ *     managed) addresses; "host" pointers are page-locked host memory.  The
+ *     library allocates and frees nothing.
+ *   - Every call is asynchronous on the given stream: it validates its
+ *     arguments on the host, enqueues kernels and returns.  Arguments are
+ *     checked before anything is launched; a bad argument returns
+ *     HGA_ERR_INVALID_ARG (or HGA_ERR_UNSUPPORTED for a valid shape this
+ *     build has no kernel for) and enqueues nothing.  HGA_ERR_CUDA reports
+ *     a launch failure (the CUDA error string is kept for hga_last_error()).
+ *   - Errors found by kernels (an out-of-range route index, a pipeline
+ *     wait that ran out of time) are OR-ed into a device status word that
+ *     hga_get_device_status() reads back; kernels never trap.
+ *   - Tensors are row-major with the head dimension D contiguous.  Token
+ *     strides between consecutive (batch, head) slices are given in tokens
+ *     so that history and segment K/V may be two views of one buffer.
+ */
+#ifndef HGA_H
+#define HGA_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    HGA_OK = 0,
+    HGA_ERR_INVALID_ARG = -1,
+    HGA_ERR_UNSUPPORTED = -2,
+    HGA_ERR_CUDA = -3,
+    HGA_ERR_DEVICE_CHECK = -4,
+    HGA_ERR_TIMEOUT = -5
+} hga_status_t;
+
+typedef enum { HGA_BF16 = 0, HGA_FP32 = 1 } hga_dtype_t;
+
+/* Device status bits (hga_get_device_status). */
+#define HGA_DEV_BAD_INDEX 1u   /* a route index outside [-1, Nc) was skipped */
+#define HGA_DEV_TIMEOUT   2u   /* a pipeline wait gave up; results are invalid */
+
+/* Shape of one HGA attention layer call.
+ *   batch B, n_q_heads Hq, n_kv_heads Hkv (Hq % Hkv == 0, G = Hq / Hkv),
+ *   head_dim D (64 or 128), chunk c (64), q_block (64), topk k (1..64),
+ *   seg_len S (multiple of q_block and chunk), n_hist_chunks Nc (T = Nc*c
+ *   history tokens routable), dtype of q/k/v/out/grads.
+ *   hist_head_stride: tokens between (b, g) slices of k_hist / v_hist; 0 is
+ *     allowed and means one shared slice (used for a staging buffer whose
+ *     route indices were remapped to slots by hga_fetch_tiered).
+ *   seg_head_stride: tokens between (b, g) slices of k_seg / v_seg (>= S).
+ *   qblock_begin / qblock_end: the range of query blocks hga_attn_fwd
+ *     processes; 0 / 0 means every block (0 .. S/q_block). */
+typedef struct {
+    int batch;
+    int n_q_heads;
+    int n_kv_heads;
+    int head_dim;
+    int chunk;
+    int q_block;
+    int topk;
+    int seg_len;
+    int n_hist_chunks;
+    hga_dtype_t dtype;
+    long long hist_head_stride;
+    long long seg_head_stride;
+    int qblock_begin;
+    int qblock_end;
+} hga_params_t;
+
+/* Chunk summaries (technical summary section 2.1: one compact vector per
+ * closed chunk, resident on the GPU; here the mean of the chunk's keys).
+ * For every (b, g) and chunk j in [first_chunk, first_chunk + n_chunks):
+ *   summ[((b*n_kv_heads + g)*summ_cap_chunks + j)*head_dim + d]
+ *     = (1/chunk) * sum_{r<chunk} k[((b*n_kv_heads + g)*head_stride + j*chunk + r)*head_dim + d]
+ * accumulated in fp32 in a fixed order, so an incremental append after each
+ * detached segment is bit-identical to a full rebuild.
+ *   k: device, dtype elements, [B][Hkv][head_stride][D] with token 0 of each
+ *      slice being history token 0.   summ: device fp32, capacity
+ *      summ_cap_chunks per (b, g) slice; first_chunk + n_chunks <= cap.
+ * n_chunks == 0 is a no-op. */
+hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch, int n_kv_heads,
+                                 int head_dim, int chunk, int first_chunk, int n_chunks,
+                                 hga_dtype_t dtype, float *summ, int summ_cap_chunks,
+                                 cudaStream_t stream);
+
+/* Routing (technical summary section 2.1: the current query block scores the
+ * chunk summaries and keeps the most relevant history chunks; no learned
+ * weights, no gradient).  For every (b, g, query block m):
+ *   qbar   = fp32 mean over the G heads of group g and the q_block queries of m;
+ *   s_j    = fp32 dot(qbar, summ[b][g][j]) / sqrt(D), j < Nc;
+ *   idx[((b*Hkv + g)*nqb + m)*k + a], a < k: the min(k, Nc) chunks with the
+ *            largest s_j (ties: lower j), ascending, then -1 padding.
+ *   q: device [B][Hq][S][D] dtype.  summ: device fp32 with summ_cap_chunks per
+ *   (b, g) slice (>= Nc).  idx: device int32 [B][Hkv][S/q_block][k]. */
+hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
+                       int32_t *idx, cudaStream_t stream);
+
+/* Exact-token attention forward (technical summary section 2.1; author
+ * abstract: a bounded set of exact historical tokens per query block).  For
+ * query (b, h, i) of a processed block m = i / q_block, g = h / G:
+ *   U = {history tokens of chunks idx[b][g][m][*] >= 0} u {segment tokens t <= i}
+ *   z_t = q . k_t / sqrt(D),  out = sum_t softmax(z)_t v_t,  lse = ln sum_t exp(z_t)
+ * History chunk j of head (b, g) is rows [j*c, j*c + c) of the slice at
+ * k_hist + (b*Hkv + g)*hist_head_stride*D.  bf16 inputs use tcgen05 tensor
+ * cores with fp32 accumulation (P is rounded to bf16 for the P.V product);
+ * fp32 inputs use fp32 CUDA-core arithmetic.
+ *   out: device [B][Hq][S][D] dtype; lse: device fp32 [B][Hq][S].  Rows of
+ *   blocks outside [qblock_begin, qblock_end) are not written.
+ * Route indices outside [-1, Nc) are skipped and flagged HGA_DEV_BAD_INDEX. */
+hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                          const void *k_seg, const void *v_seg, const int32_t *idx, void *out,
+                          float *lse, cudaStream_t stream);
+
+/* Bytes of device workspace hga_attn_bwd needs (fp32 row terms
+ * delta = rowsum(dO * O), [B][Hq][S]).  Returns 0 for an invalid p. */
+size_t hga_attn_bwd_workspace_size(const hga_params_t *p);
+
+/* Backward of the exact-token attention with routes frozen (technical
+ * summary sections 2.1 and 2.2: routing without gradient, gather and
+ * attention differentiable, history detached at the segment boundary).
+ * With P the softmax row of query (b, h, i) and delta_i = sum_d dO*O:
+ *   dS_t = P_t (dO . v_t - delta_i)
+ *   dq[b][h][i]      = sum_{t in U} dS_t k_t / sqrt(D)       (history and segment keys)
+ *   dk_seg[b][g][t] = sum_{h in g, i >= t} dS_t q_i / sqrt(D) (segment keys only)
+ *   dv_seg[b][g][t] = sum_{h in g, i >= t} P_t dO_i           (segment keys only)
+ * History K/V get no gradient.  out / lse are the forward's outputs for
+ * every block (qblock_begin/end must be 0/0).  dq, dk_seg, dv_seg: device,
+ * dtype, overwritten (dk_seg/dv_seg use seg_head_stride = S layout
+ * [B][Hkv][S][D]).  workspace: device, >= hga_attn_bwd_workspace_size(p)
+ * bytes, 16-byte aligned. */
+hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                          const void *k_seg, const void *v_seg, const int32_t *idx, const void *out,
+                          const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg,
+                          void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Tiered history (technical summary section 2.2: detached K/V live in host
+ * RAM, only the routed exact K/V are brought to the GPU).  For the query
+ * blocks [qblock_begin, qblock_end) of idx, gathers the distinct (b, g, chunk)
+ * tiles they route to, copies only those K and V tiles from page-locked host
+ * memory (host_k / host_v: [B][Hkv][hist_head_stride][D], dtype) into the
+ * device staging buffers stage_k / stage_v ([stage_slots][chunk][D]) and
+ * writes idx_remapped (same shape as idx) with each index replaced by its
+ * staging slot.  hga_attn_fwd over the same blocks with k_hist = stage_k,
+ * v_hist = stage_v, hist_head_stride = 0 and idx = idx_remapped gives output
+ * bit-identical to attending the history in device memory.
+ *   slot_map: device int32 scratch of at least B*Hkv*Nc + stage_slots + 1
+ *     entries (tile flags / slot numbers, then the slot -> tile list).
+ *   n_fetched (device int32, may be NULL): number of tiles fetched.
+ * The attention call over the staging buffer passes n_hist_chunks =
+ * stage_slots (route indices are now slot numbers).
+ * All work is enqueued on copy_stream; when done != NULL it is recorded on
+ * copy_stream after the last kernel.  Returns HGA_ERR_INVALID_ARG when the
+ * blocks can need more tiles than stage_slots. */
+hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v,
+                              const int32_t *idx, int qblock_begin, int qblock_end, void *stage_k,
+                              void *stage_v, int stage_slots, int32_t *slot_map, int32_t *idx_remapped,
+                              int32_t *n_fetched, cudaStream_t copy_stream, cudaEvent_t done);
+
+/* Reads (after synchronising stream) and clears the device status word of the
+ * current device; *bits gets the HGA_DEV_* bits seen since the last call.
+ * Returns HGA_ERR_DEVICE_CHECK or HGA_ERR_TIMEOUT when bits are set. */
+hga_status_t hga_get_device_status(cudaStream_t stream, unsigned int *bits);
+
+/* Human-readable name of a status code. */
+const char *hga_status_string(hga_status_t s);
+
+/* Text of the last CUDA error seen by this thread's calls (or ""). */
+const char *hga_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HGA_H */

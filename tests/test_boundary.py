@@ -1,0 +1,104 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every entry point include/hga.h declares, and rejects bad arguments on the
+host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import hierarchical_sparse_long_b200 as hga
+from hierarchical_sparse_long_b200 import binding
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from hierarchical_sparse_long_b200 import build
+    build.build()
+    return binding.lib()
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "hga.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hga_[a-z_]+)\s*\(", text)))
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert set(names) == set(binding.EXPORTED)
+
+
+def test_status_strings(L):
+    for code, name in binding.STATUS.items():
+        assert L.hga_status_string(code).decode() == name
+
+
+def _params(**kw):
+    base = dict(batch=1, n_q_heads=4, n_kv_heads=2, head_dim=128, topk=4, seg_len=128, n_hist_chunks=8)
+    base.update(kw)
+    return hga.Params(**base)
+
+
+BAD = [
+    dict(n_q_heads=3),            # Hq % Hkv
+    dict(topk=0),
+    dict(topk=65),
+    dict(seg_len=100),            # not a multiple of the block
+    dict(n_hist_chunks=-1),
+    dict(qblock_begin=1, qblock_end=1),
+    dict(qblock_begin=0, qblock_end=3),  # 3 > S/64 = 2
+    dict(seg_head_stride=64),
+    dict(hist_head_stride=100),   # < Nc * c
+]
+
+
+@pytest.mark.parametrize("kw", BAD)
+def test_bad_params_rejected_on_host(L, kw):
+    p = _params(**kw).c()
+    fake = ctypes.c_void_p(0x1000)
+    rc = L.hga_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None)
+    assert rc == -1
+    rc = L.hga_route(ctypes.byref(p), fake, fake, 64, fake, None)
+    assert rc == -1
+
+
+def test_unsupported_shapes(L):
+    fake = ctypes.c_void_p(0x1000)
+    for kw in (dict(head_dim=96), dict(chunk=32)):
+        p = _params(**kw).c()
+        assert L.hga_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None) == -2
+
+
+def test_null_and_misaligned_pointers(L):
+    p = _params().c()
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    assert L.hga_attn_fwd(ctypes.byref(p), None, fake, fake, fake, fake, fake, fake, fake, None) == -1
+    assert L.hga_attn_fwd(ctypes.byref(p), odd, fake, fake, fake, fake, fake, fake, fake, None) == -1
+    assert L.hga_attn_bwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake,
+                          fake, 0, None) == -1  # workspace too small
+    assert L.hga_build_summaries(fake, 64, 1, 1, 128, 64, 0, 2, 0, fake, 1, None) == -1  # capacity
+    assert L.hga_build_summaries(odd, 1024, 1, 1, 128, 64, 0, 2, 0, fake, 4, None) == -1
+    assert L.hga_build_summaries(fake, 1024, 1, 1, 128, 64, 0, 0, 0, fake, 4, None) == 0  # no-op
+
+
+def test_tiered_staging_capacity_checked_on_host(L):
+    p = _params(n_hist_chunks=32).c()
+    fake = ctypes.c_void_p(0x1000)
+    # 2 blocks x 2 kv heads x 4 routes = 16 tiles may be needed
+    rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 0, 2, fake, fake, 15, fake, fake, None, None, None)
+    assert rc == -1
+    rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 1, 1, fake, fake, 64, fake, fake, None, None, None)
+    assert rc == -1
+
+
+def test_workspace_size(L):
+    p = _params()
+    assert hga.hga_attn_bwd_workspace_size(p) >= 4 * 4 * 128
+    assert hga.hga_attn_bwd_workspace_size(_params(topk=0)) == 0

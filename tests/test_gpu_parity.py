@@ -1,0 +1,346 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 CPU oracle.
+
+Routes must be bit-exact except at oracle near-ties (relative gap of the k-th
+and (k+1)-th scores below 1e-5), which are counted and printed.  Attention is
+checked with the oracle's routes fed to both sides.  Tolerances: bf16 inputs
+max-abs 2e-2 and mean-abs 2e-3, fp32 inputs max-abs 1e-4.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from inputs import gen
+from tests import hga_cases as hc
+
+pytestmark = pytest.mark.gpu
+
+W = gen.WORKLOADS
+# mid-size bf16 layer: several key tiles per block, ragged route lists (Nc=13)
+MID = gen.custom("mid_bf16", n_q_heads=8, n_kv_heads=2, head_dim=128, topk=4, seg_len=256, seq_len=1088,
+                 seg_starts=(832,), dtype="bf16", seed=7, backward=True)
+EDGE = [
+    gen.custom("no_history", topk=4, seg_len=192, seq_len=192, seg_starts=(0,), dtype="bf16", head_dim=128,
+               n_q_heads=4, n_kv_heads=1, seed=11, backward=True),
+    gen.custom("k_above_nc", topk=9, seg_len=128, seq_len=320, seg_starts=(192,), dtype="bf16", head_dim=128,
+               n_q_heads=8, n_kv_heads=2, seed=12, backward=True),
+    gen.custom("d64_mha_b2", batch=2, topk=3, seg_len=128, seq_len=768, seg_starts=(640,), dtype="bf16",
+               head_dim=64, n_q_heads=2, n_kv_heads=2, seed=13, backward=True),
+    gen.custom("fp32_g4", topk=2, seg_len=128, seq_len=512, seg_starts=(384,), dtype="fp32", head_dim=128,
+               n_q_heads=8, n_kv_heads=2, seed=14, backward=True),
+    gen.custom("one_block", topk=1, seg_len=64, seq_len=192, seg_starts=(128,), dtype="bf16", head_dim=128,
+               n_q_heads=4, n_kv_heads=1, seed=15, backward=True),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _built():
+    hc.ensure_built()
+    assert torch.cuda.is_available()
+    yield
+    import hierarchical_sparse_long_b200 as hga
+    assert hga.hga_get_device_status() == 0
+
+
+def _full_fwd_check(w, seg=0):
+    arrs = hc.segment_arrays(w, seg)
+    g = hc.GpuSegment(w, arrs)
+    sh, summ_o, idx_o, gap = hc.oracle_route(w, arrs)
+    T = arrs["T"]
+    out_o, lse_o = oracle.attn_fwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                                   arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], idx_o)
+    out, lse = g.fwd(torch.from_numpy(idx_o).cuda())
+    torch.cuda.synchronize()
+    hc.compare(hc.f32(out), out_o, w.dtype, f"{w.name} out")
+    hc.compare(hc.f32(lse), lse_o, "fp32" if w.dtype == "fp32" else "bf16", f"{w.name} lse")
+    return g, arrs, sh, idx_o
+
+
+# ---------------------------------------------------------------- summaries
+
+@pytest.mark.parametrize("name", ["tiny_fp32", "qwen3_16k_fwd"])
+def test_summaries_match_oracle(name):
+    w = W[name]
+    arrs = hc.segment_arrays(w, 0)
+    g = hc.GpuSegment(w, arrs)
+    s = hc.f32(g.summaries())
+    want = oracle.summaries(arrs["k_all"][:, :, :arrs["T"]], w.chunk)
+    assert np.max(np.abs(s - want)) < 1e-5
+
+
+def test_summaries_incremental_equals_full_rebuild():
+    import hierarchical_sparse_long_b200 as hga
+    w = W["qwen3_16k_fwd"]
+    g = hc.GpuSegment(w, hc.segment_arrays(w, 0))
+    L = g.T + w.seg_len
+    nct = L // w.chunk
+    full = torch.zeros(1, 8, nct, 128, device="cuda")
+    inc = torch.full_like(full, float("nan"))
+    hga.hga_build_summaries(g.k_all, L, 1, 8, 128, 64, 0, nct, full, nct)
+    for first in range(0, nct, 32):  # one 2,048-token segment at a time
+        hga.hga_build_summaries(g.k_all, L, 1, 8, 128, 64, first, min(32, nct - first), inc, nct)
+    torch.cuda.synchronize()
+    assert torch.equal(full, inc)
+
+
+# ---------------------------------------------------------------- routing
+
+@pytest.mark.parametrize("name,seg", [("tiny_fp32", 0), ("qwen3_16k_fwd", 0), ("qwen3_128k_eval", 31),
+                                      ("qwen3_128k_eval", 1)])
+def test_route_matches_oracle(name, seg):
+    w = W[name]
+    arrs = hc.segment_arrays(w, seg)
+    g = hc.GpuSegment(w, arrs)
+    idx = hc.f32(g.route(g.summaries())).astype(np.int32)
+    _, _, idx_o, gap = hc.oracle_route(w, arrs)
+    hard, exempt = hc.route_mismatches(idx, idx_o, gap)
+    print(f"{name} seg {seg}: {idx.shape[2]} blocks x {idx.shape[1]} heads, near-tie exemptions {exempt}")
+    assert hard == 0
+
+
+def test_route_edge_cases():
+    for w in EDGE:
+        arrs = hc.segment_arrays(w, 0)
+        g = hc.GpuSegment(w, arrs)
+        idx = hc.f32(g.route(g.summaries())).astype(np.int32)
+        _, _, idx_o, gap = hc.oracle_route(w, arrs)
+        hard, _ = hc.route_mismatches(idx, idx_o, gap)
+        assert hard == 0, w.name
+
+
+# ---------------------------------------------------------------- forward
+
+def test_fwd_tiny_fp32_full():
+    _full_fwd_check(W["tiny_fp32"])
+
+
+def test_fwd_mid_bf16_full():
+    _full_fwd_check(MID)
+
+
+@pytest.mark.parametrize("w", EDGE, ids=[w.name for w in EDGE])
+def test_fwd_edge_cases(w):
+    _full_fwd_check(w)
+
+
+def _sampled_rows(w, n, seed):
+    r = np.random.default_rng(seed)
+    S = w.seg_len
+    rows = set()
+    # first and last rows of blocks, plus random rows, over random heads
+    for _ in range(n):
+        b = int(r.integers(0, w.batch))
+        h = int(r.integers(0, w.n_q_heads))
+        i = int(r.integers(0, S))
+        rows.add((b * w.n_q_heads + h) * S + i)
+    for h in (0, w.n_q_heads - 1):
+        for i in (0, 63, 64, S - 1):
+            rows.add(h * S + i)
+    return np.array(sorted(rows), dtype=np.int64)
+
+
+@pytest.mark.parametrize("name,seg,n", [("qwen3_16k_fwd", 0, 384), ("qwen3_128k_eval", 31, 160)])
+def test_fwd_full_size_sampled(name, seg, n):
+    w = W[name]
+    arrs = hc.segment_arrays(w, seg)
+    g = hc.GpuSegment(w, arrs)
+    sh, _, idx_o, _ = hc.oracle_route(w, arrs)
+    T = arrs["T"]
+    rows = _sampled_rows(w, n, seed=seg)
+    out_o, lse_o = oracle.attn_fwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                                   arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], idx_o, rows=rows)
+    out, lse = g.fwd(torch.from_numpy(idx_o).cuda())
+    D = w.head_dim
+    hc.compare(hc.f32(out).reshape(-1, D)[rows], out_o.reshape(-1, D)[rows], "bf16", f"{name} out")
+    hc.compare(hc.f32(lse).reshape(-1)[rows], lse_o.reshape(-1)[rows], "bf16", f"{name} lse")
+
+
+def test_fwd_attended_count_on_gpu():
+    # q = 0: every logit is 0 and lse_i = ln(min(k, Nc)*64 + i + 1) exactly
+    for w in (MID, EDGE[0], EDGE[1]):
+        arrs = dict(hc.segment_arrays(w, 0))
+        arrs["q"] = np.zeros_like(arrs["q"])
+        g = hc.GpuSegment(w, arrs)
+        idx = g.route(g.summaries())
+        _, lse = g.fwd(idx)
+        keff = min(w.topk, arrs["T"] // 64)
+        want = np.log(keff * 64 + np.arange(w.seg_len) + 1.0)
+        got = hc.f32(lse)
+        assert np.max(np.abs(got - want[None, None, :])) < 1e-5, w.name
+
+
+def test_fwd_bad_route_index_is_flagged_and_skipped():
+    import hierarchical_sparse_long_b200 as hga
+    w = MID
+    arrs = hc.segment_arrays(w, 0)
+    g = hc.GpuSegment(w, arrs)
+    sh, _, idx_o, _ = hc.oracle_route(w, arrs)
+    bad = idx_o.copy()
+    bad[0, 1, 2, 0] = 10_000
+    bad[0, 0, 3, 1] = -7
+    hga.hga_get_device_status()  # clear
+    out, lse = g.fwd(torch.from_numpy(bad).cuda())
+    bits = hga.hga_get_device_status()
+    assert bits & hga.HGA_DEV_BAD_INDEX
+    skipped = bad.copy()
+    skipped[(skipped < -1) | (skipped >= sh.n_hist_chunks)] = -1
+    T = arrs["T"]
+    out_o, _ = oracle.attn_fwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                               arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], skipped)
+    hc.compare(hc.f32(out), out_o, "bf16", "skipped index")
+
+
+def test_fwd_summaries_are_not_values():
+    # the attention output depends on the routes only, never on summary values
+    w = MID
+    arrs = hc.segment_arrays(w, 0)
+    g = hc.GpuSegment(w, arrs)
+    summ = g.summaries()
+    idx = g.route(summ)
+    out1, _ = g.fwd(idx)
+    idx2 = g.route(summ * 3.0)  # positive rescale keeps every ordering
+    out2, _ = g.fwd(idx2)
+    torch.cuda.synchronize()
+    assert torch.equal(idx, idx2) and torch.equal(out1, out2)
+
+
+# ---------------------------------------------------------------- backward
+
+def _full_bwd_check(w):
+    arrs = hc.segment_arrays(w, 0)
+    g = hc.GpuSegment(w, arrs)
+    sh, _, idx_o, _ = hc.oracle_route(w, arrs)
+    T = arrs["T"]
+    args = (sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T], arrs["k_all"][:, :, T:],
+            arrs["v_all"][:, :, T:], idx_o)
+    dq_o, dk_o, dv_o = oracle.attn_bwd(*args, arrs["dout"])
+    idx = torch.from_numpy(idx_o).cuda()
+    out, lse = g.fwd(idx)
+    dq, dk, dv = g.bwd(idx, out, lse)
+    torch.cuda.synchronize()
+    hc.compare(hc.f32(dq), dq_o, w.dtype, f"{w.name} dq")
+    hc.compare(hc.f32(dk), dk_o, w.dtype, f"{w.name} dk")
+    hc.compare(hc.f32(dv), dv_o, w.dtype, f"{w.name} dv")
+
+
+def test_bwd_tiny_fp32_full():
+    w = gen.custom("tiny_fp32_bwd", backward=True)
+    _full_bwd_check(w)
+
+
+def test_bwd_mid_bf16_full():
+    _full_bwd_check(MID)
+
+
+@pytest.mark.parametrize("w", EDGE, ids=[w.name for w in EDGE])
+def test_bwd_edge_cases(w):
+    _full_bwd_check(w)
+
+
+def test_bwd_full_size_sampled():
+    # the 16K training layer's last segment (T = 14,336): sampled dq rows and
+    # dk/dv rows of the last 64 active keys (every query that sees them is visited)
+    w = W["qwen3_16k_train"]
+    seg = 7
+    arrs = hc.segment_arrays(w, seg)
+    g = hc.GpuSegment(w, arrs)
+    sh, _, idx_o, _ = hc.oracle_route(w, arrs)
+    T, S, D = arrs["T"], w.seg_len, w.head_dim
+    q_need = np.zeros((1, w.n_q_heads, S), dtype=np.uint8)
+    r = np.random.default_rng(3)
+    for _ in range(64):
+        q_need[0, r.integers(0, w.n_q_heads), r.integers(S - 256, S)] = 1
+    key_need = np.zeros((1, w.n_kv_heads, S), dtype=np.uint8)
+    key_need[0, 0, S - 64:] = 1
+    key_need[0, 5, [S - 1, S - 30]] = 1
+    dq_o, dk_o, dv_o = oracle.attn_bwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                                       arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], idx_o, arrs["dout"],
+                                       q_need=q_need, key_need=key_need)
+    idx = torch.from_numpy(idx_o).cuda()
+    out, lse = g.fwd(idx)
+    dq, dk, dv = g.bwd(idx, out, lse)
+    qm, km = q_need.astype(bool), key_need.astype(bool)
+    hc.compare(hc.f32(dq)[qm], dq_o[qm], "bf16", "dq sampled")
+    hc.compare(hc.f32(dk)[km], dk_o[km], "bf16", "dk sampled")
+    hc.compare(hc.f32(dv)[km], dv_o[km], "bf16", "dv sampled")
+
+
+# ---------------------------------------------------------------- segment-wise training (8 segments)
+
+def test_train_segments_route_and_summary_append():
+    """8 consecutive 2,048-token segments: summaries appended as each segment
+    detaches must equal a rebuild, and every segment's routes match the oracle."""
+    import hierarchical_sparse_long_b200 as hga
+    w = W["qwen3_16k_train"]
+    L = w.seq_len
+    k_all = hc.to_dev(gen.keys(w, 0, L), w)
+    q_all = hc.to_dev(gen.queries(w, 0, L), w)
+    nct = L // 64
+    summ = torch.zeros(1, 8, nct, 128, device="cuda")
+    total_exempt = 0
+    for s, T in enumerate(w.seg_starts):
+        p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
+        q = q_all[:, :, T:T + w.seg_len].contiguous()
+        idx = torch.empty(1, 8, w.seg_len // 64, w.topk, device="cuda", dtype=torch.int32)
+        hga.hga_route(p, q, summ, nct, idx)
+        arrs = dict(T=T, q=hc.f32(q), k_all=hc.f32(k_all[:, :, :T + w.seg_len]))
+        _, _, idx_o, gap = hc.oracle_route(w, arrs)
+        hard, exempt = hc.route_mismatches(hc.f32(idx).astype(np.int32), idx_o, gap)
+        total_exempt += exempt
+        assert hard == 0, f"segment {s}"
+        # detach: append this segment's 32 chunks
+        hga.hga_build_summaries(k_all, L, 1, 8, 128, 64, T // 64, w.seg_len // 64, summ, nct)
+    full = torch.zeros_like(summ)
+    hga.hga_build_summaries(k_all, L, 1, 8, 128, 64, 0, nct, full, nct)
+    torch.cuda.synchronize()
+    assert torch.equal(full, summ)
+    print(f"near-tie exemptions over 8 segments: {total_exempt}")
+
+
+# ---------------------------------------------------------------- tiered history
+
+def _tiered_equals_resident(w, seg, wave):
+    import hierarchical_sparse_long_b200 as hga
+    arrs = hc.segment_arrays(w, seg)
+    g = hc.GpuSegment(w, arrs)
+    T, S = arrs["T"], w.seg_len
+    idx = g.route(g.summaries())
+    out_res, lse_res = g.fwd(idx)
+    # history only in pinned host memory
+    host_k = g.k_all[:, :, :T].contiguous().cpu().pin_memory()
+    host_v = g.v_all[:, :, :T].contiguous().cpu().pin_memory()
+    nc = T // 64
+    nqb = S // 64
+    keff = min(w.topk, nc)
+    slots = min(wave * w.batch * w.n_kv_heads * keff, w.batch * w.n_kv_heads * nc)
+    stage_k = torch.empty(max(slots, 1), 64, w.head_dim, device="cuda", dtype=g.q.dtype)
+    stage_v = torch.empty_like(stage_k)
+    slot_map = torch.empty(w.batch * w.n_kv_heads * nc + slots + 1, device="cuda", dtype=torch.int32)
+    idx_r = torch.full_like(idx, -1)
+    nf = torch.zeros(1, device="cuda", dtype=torch.int32)
+    out = torch.empty_like(out_res)
+    lse = torch.empty_like(lse_res)
+    p = hc.params(w, T, hist_head_stride=T, seg_head_stride=T + S)
+    fetched = 0
+    for b0 in range(0, nqb, wave):
+        b1 = min(b0 + wave, nqb)
+        hga.hga_fetch_tiered(p, host_k, host_v, idx, b0, b1, stage_k, stage_v, slots, slot_map, idx_r, nf)
+        pa = hc.params(w, T, hist_head_stride=0, seg_head_stride=T + S, n_hist_chunks=slots,
+                       qblock_begin=b0, qblock_end=b1)
+        hga.hga_attn_fwd(pa, g.q, stage_k, stage_v, g.k_seg, g.v_seg, idx_r, out, lse)
+        torch.cuda.synchronize()
+        fetched += int(nf.item())
+    assert torch.equal(out, out_res) and torch.equal(lse, lse_res)
+    return fetched
+
+
+def test_tiered_bitwise_small():
+    _tiered_equals_resident(MID, 0, wave=2)
+
+
+def test_tiered_bitwise_128k_last_segment():
+    w = W["qwen3_128k_tiered"]
+    fetched = _tiered_equals_resident(w, 31, wave=8)
+    print(f"tiles fetched for the last 4,096-token segment: {fetched}")
