@@ -170,8 +170,8 @@ class Layer:
         self.out = torch.empty(w.batch, w.n_q_heads, w.seg_len, w.head_dim, device="cuda", dtype=dt)
         self.lse = torch.empty(w.batch, w.n_q_heads, w.seg_len, device="cuda")
         if w.backward:
-            self.dq = torch.empty_like(self.out)
-            self.dk = torch.empty(w.batch, w.n_kv_heads, w.seg_len, w.head_dim, device="cuda", dtype=dt)
+            self.dq = torch.empty(self.out.shape, device="cuda", dtype=torch.float32)
+            self.dk = torch.empty(w.batch, w.n_kv_heads, w.seg_len, w.head_dim, device="cuda", dtype=torch.float32)
             self.dv = torch.empty_like(self.dk)
             p = self.params(w.seg_starts[-1])
             self.ws = torch.empty(hga.hga_attn_bwd_workspace_size(p) // 4 + 64, device="cuda")
@@ -403,7 +403,7 @@ def e2e_measure(layer, steps):
     h2d = qh.numel() * 2 + kh.numel() * 2 + vh.numel() * 2 + (doh.numel() * 2 if doh is not None else 0)
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
     if w.backward:
-        d2h += layer.dq.numel() * 2 + layer.dk.numel() * 2 + layer.dv.numel() * 2
+        d2h += layer.dq.numel() * 4 + layer.dk.numel() * 4 + layer.dv.numel() * 4
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     times = []
     for it in range(steps + 2):

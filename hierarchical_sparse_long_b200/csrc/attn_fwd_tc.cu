@@ -1,10 +1,446 @@
-// tcgen05 forward kernel (in progress).
-#include "common.cuh"
+// Exact-token HGA attention forward on the 5th-generation tensor cores
+// (tcgen05 / TMEM / TMA), bf16 inputs, fp32 accumulation, head_dim 128.
+//
+// "Long-Context Fine-Tuning with Limited VRAM", technical summary section 2.1
+// (exact K/V of the routed chunks attended with a local window; summaries
+// route only) and the author abstract (a bounded set of exact historical
+// tokens per query block).
+//
+// One CTA per (batch, kv head, query block).  The G query heads of the KV
+// group share every K/V tile, so the CTA holds all G*64 query rows as NH
+// M=128 halves (NH = G/2): each 64-token key tile (a routed history chunk,
+// then the active segment's causal tiles 0..m) is read once for G heads,
+// which is what lifts a history tile from 64 to 256 flop/byte.
+//
+// Warp roles (NH = 2: 384 threads):
+//   warp 0      TMA producer: Q once, then K/V tiles into a 3-stage ring
+//               (routed chunk j -> TMA row coordinate (b*Hkv+g)*stride + 64 j)
+//   warp 1      TMEM owner and single-thread UMMA issuer:
+//               S_h = Q_h K^T   (M128 N64 K128, K-major A and B, SW128)
+//               O_h += P_h V    (M128 N128 K64, P K-major, V MN-major)
+//               QK^T of tile j is issued before PV of tile j-1 so the tensor
+//               core works while the softmax warps run.
+//   warps 4+4h  softmax of half h: one TMEM lane (= query row) per thread;
+//               online softmax in the log2 domain, O rescaled in TMEM when
+//               the row max grows, P written as bf16 in the SW128 K-major
+//               layout the next UMMA reads.
+// TMEM (512 columns): O_h at 128h, S_h double-buffered at 256 + 128h + 64b.
+// Every wait is bounded; a timeout sets HGA_DEV_TIMEOUT and the CTA unwinds.
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "tc_ptx.cuh"
 
 namespace hga {
-bool attn_fwd_tc_supported(const hga_params_t &) { return false; }
-hga_status_t launch_attn_fwd_tc(const hga_params_t &, const void *, const void *, const void *, const void *,
-                                const void *, const int32_t *, void *, float *, unsigned *, cudaStream_t) {
-    return HGA_ERR_UNSUPPORTED;
+
+namespace {
+
+constexpr int D = 128;
+constexpr int TILE = 64;
+constexpr int NSTAGE = 3;
+constexpr uint32_t Q_HALF_BYTES = 128 * D * 2;   // 32 KiB: [2 col halves][128 rows][128 B]
+constexpr uint32_t KV_TILE_BYTES = TILE * D * 2; // 16 KiB: [2 col halves][64 rows][128 B]
+constexpr uint32_t P_BYTES = 128 * TILE * 2;     // 16 KiB: [128 rows][128 B]
+constexpr uint32_t IDESC_QK = tc::idesc_bf16(128, TILE, false, false);
+constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, D, false, true);
+
+template <int NH>
+struct Smem {
+    static constexpr uint32_t Q = 0;
+    static constexpr uint32_t KV = Q + NH * Q_HALF_BYTES;
+    static constexpr uint32_t P = KV + NSTAGE * 2 * KV_TILE_BYTES;
+    static constexpr uint32_t BAR = P + NH * P_BYTES;
+    static constexpr uint32_t TOTAL = BAR + 1024;  // barriers, tile list, flags
+    static constexpr uint32_t ALLOC = TOTAL + 1024; // + alignment slack
+};
+
+struct Bars {
+    uint64_t q_full;
+    uint64_t kv_full[NSTAGE];
+    uint64_t kv_empty[NSTAGE];
+    uint64_t s_full[2][2];
+    uint64_t s_free[2][2];
+    uint64_t p_full[2];
+    uint64_t o_done[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int n_hist;
+    int issued;
+    int tiles[64];
+};
+
+struct FwdArgs {
+    int batch, n_q_heads, n_kv_heads, seg_len, topk, n_hist_chunks;
+    long long hist_stride, seg_stride;
+    int qb0, n_blocks;
+    const int32_t *idx;
+    __nv_bfloat16 *out;
+    float *lse;
+    unsigned *status;
+    float scale_log2;  // log2(e) / sqrt(D)
+};
+
+template <int NH>
+__global__ void __launch_bounds__(128 + 128 * NH, 1)
+    attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
+                       const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
+                       const __grid_constant__ CUtensorMap tm_vs, const FwdArgs a) {
+    using L = Smem<NH>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    Bars *bars = reinterpret_cast<Bars *>(smem + L::BAR);
+    const uint32_t sbase = tc::smem_u32(smem);
+
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = 2 * NH;
+    const int nqb = a.seg_len / TILE;
+    const int n_bg = a.batch * a.n_kv_heads;
+    const int m = a.qb0 + a.n_blocks - 1 - (int)blockIdx.x / n_bg;  // longest (latest) blocks first
+    const int bg = (int)blockIdx.x % n_bg;
+    const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < NSTAGE; ++s) {
+            tc::mbar_init(&bars->kv_full[s], 1);
+            tc::mbar_init(&bars->kv_empty[s], 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            for (int bb = 0; bb < 2; ++bb) {
+                tc::mbar_init(&bars->s_full[h][bb], 1);
+                tc::mbar_init(&bars->s_free[h][bb], 4);
+            }
+            tc::mbar_init(&bars->p_full[h], 4);
+            tc::mbar_init(&bars->o_done[h], 1);
+        }
+        tc::mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 2 && lane == 0) {
+        // routed history chunks of this block; -1 is padding, anything else out of range is skipped
+        const int32_t *sel = a.idx + ((long long)bg * nqb + m) * a.topk;
+        int n = 0;
+        for (int i = 0; i < a.topk; ++i) {
+            const int j = sel[i];
+            if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
+            else if (j != -1) atomicOr(a.status, kDevBadIndex);
+        }
+        bars->n_hist = n;
+    }
+    if (warp == 1) tc::tmem_alloc<512>(&bars->tmem_base);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+    const int n_hist = bars->n_hist;
+    const int n_tiles = n_hist + m + 1;
+    volatile int *abort = &bars->abort;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- TMA producer
+            tc::tma_prefetch_desc(&tm_q);
+            tc::tma_prefetch_desc(&tm_kh);
+            tc::tma_prefetch_desc(&tm_ks);
+            tc::mbar_arrive_expect_tx(&bars->q_full, NH * Q_HALF_BYTES);
+            for (int hh = 0; hh < G; ++hh) {
+                const int qrow = (b * a.n_q_heads + g * G + hh) * a.seg_len + m * TILE;
+                uint8_t *dst = smem + L::Q + (hh >> 1) * Q_HALF_BYTES + (hh & 1) * (64 * 128);
+                tc::tma_load_2d(dst, &tm_q, 0, qrow, &bars->q_full);
+                tc::tma_load_2d(dst + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
+            }
+            int issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % NSTAGE, u = j / NSTAGE;
+                if (j >= NSTAGE && !tc::mbar_wait(&bars->kv_empty[s], (u - 1) & 1, abort, a.status)) break;
+                const bool hist = j < n_hist;
+                const CUtensorMap *mk = hist ? &tm_kh : &tm_ks;
+                const CUtensorMap *mv = hist ? &tm_vh : &tm_vs;
+                const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
+                                     : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+                uint8_t *kdst = smem + L::KV + s * 2 * KV_TILE_BYTES;
+                uint8_t *vdst = kdst + KV_TILE_BYTES;
+                tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * KV_TILE_BYTES);
+                tc::tma_load_2d(kdst, mk, 0, row, &bars->kv_full[s]);
+                tc::tma_load_2d(kdst + 64 * 128, mk, 64, row, &bars->kv_full[s]);
+                tc::tma_load_2d(vdst, mv, 0, row, &bars->kv_full[s]);
+                tc::tma_load_2d(vdst + 64 * 128, mv, 64, row, &bars->kv_full[s]);
+                ++issued;
+            }
+            bars->issued = issued;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            // ---------------------------------------------------------- UMMA issuer
+            const uint32_t q_base = sbase + L::Q;
+            const uint32_t p_base = sbase + L::P;
+            auto issue_pv = [&](int t) -> bool {
+                const int s = t % NSTAGE;
+                const uint32_t v_base = sbase + L::KV + s * 2 * KV_TILE_BYTES + KV_TILE_BYTES;
+                for (int h = 0; h < NH; ++h) {
+                    if (!tc::mbar_wait(&bars->p_full[h], t & 1, abort, a.status)) return false;
+                    tc::fence_after_sync();
+                    const uint32_t d = tmem + 128 * h;
+#pragma unroll
+                    for (int kk = 0; kk < TILE / 16; ++kk) {
+                        const uint64_t adesc = tc::desc_sw128(p_base + h * P_BYTES + kk * 32, 16, 1024);
+                        const uint64_t bdesc = tc::desc_sw128(v_base + kk * 2048, 8192, 1024);
+                        tc::mma_f16(d, adesc, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    tc::mma_commit(&bars->o_done[h]);
+                }
+                tc::mma_commit(&bars->kv_empty[s]);
+                return true;
+            };
+            bool ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int s = j % NSTAGE;
+                if (!tc::mbar_wait(&bars->kv_full[s], (j / NSTAGE) & 1, abort, a.status)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t k_base = sbase + L::KV + s * 2 * KV_TILE_BYTES;
+                const int bb = j & 1;
+                for (int h = 0; h < NH; ++h) {
+                    if (j >= 2 && !tc::mbar_wait(&bars->s_free[h][bb], ((j >> 1) - 1) & 1, abort, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    const uint32_t d = tmem + 256 + 128 * h + 64 * bb;
+#pragma unroll
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t kb = (kk & 3) * 32;
+                        const uint64_t adesc =
+                            tc::desc_sw128(q_base + h * Q_HALF_BYTES + (kk >> 2) * (128 * 128) + kb, 16, 1024);
+                        const uint64_t bdesc = tc::desc_sw128(k_base + (kk >> 2) * (64 * 128) + kb, 16, 1024);
+                        tc::mma_f16(d, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(&bars->s_full[h][bb]);
+                }
+                if (!ok) break;
+                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+            }
+            if (ok) issue_pv(n_tiles - 1);
+        }
+    } else if (warp >= 4) {
+        // -------------------------------------------------------------- softmax / epilogue
+        const int h = (warp - 4) >> 2;        // M half
+        const int quad = warp & 3;            // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;       // row within the half = TMEM lane
+        const int hh = 2 * h + (r >> 6);      // head within the group
+        const int i = r & 63;                 // query row within the block
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const uint32_t o_addr = tmem + lane_addr + 128 * h;
+        const uint32_t p_row = sbase + L::P + h * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
+        float m_run = -INFINITY, l_run = 0.f;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int bb = j & 1;
+            if (!tc::mbar_wait(&bars->s_full[h][bb], (j >> 1) & 1, abort, a.status)) { ok = false; break; }
+            tc::fence_after_sync();
+            uint32_t sr[64];
+            {
+                uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+                uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * h + 64 * bb;
+                tc::tmem_ld32(s_addr, lo);
+                tc::tmem_ld32(s_addr + 32, hi);
+                tc::tmem_wait_ld();
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->s_free[h][bb]);
+            float x[64];
+            const bool diag = (j == n_tiles - 1);  // the local tile of this block
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                float v = __uint_as_float(sr[c]) * a.scale_log2;
+                if (diag && c > i) v = -INFINITY;
+                x[c] = v;
+                mx = fmaxf(mx, v);
+            }
+            const float m_new = fmaxf(m_run, mx);
+            float sum = 0.f;
+#pragma unroll
+            for (int c = 0; c < 64; ++c) {
+                x[c] = tc::ex2(x[c] - m_new);
+                sum += x[c];
+            }
+            const float alpha = tc::ex2(m_run - m_new);
+            l_run = l_run * alpha + sum;
+            // PV of the previous tile must be done before P is overwritten and O rescaled
+            if (j >= 1) {
+                if (!tc::mbar_wait(&bars->o_done[h], (j - 1) & 1, abort, a.status)) { ok = false; break; }
+                tc::fence_after_sync();
+                if (m_new > m_run) {
+#pragma unroll 1
+                    for (int c0 = 0; c0 < D; c0 += 32) {
+                        uint32_t o[32];
+                        tc::tmem_ld32(o_addr + c0, o);
+                        tc::tmem_wait_ld();
+#pragma unroll
+                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                        tc::tmem_st32(o_addr + c0, o);
+                    }
+                    tc::tmem_wait_st();
+                }
+            }
+            m_run = m_new;
+#pragma unroll
+            for (int cc = 0; cc < 8; ++cc) {
+                const uint32_t addr = p_row + ((cc ^ (r & 7)) << 4);
+                tc::st_shared_v4(addr, tc::pack_bf16(x[8 * cc + 0], x[8 * cc + 1]),
+                                 tc::pack_bf16(x[8 * cc + 2], x[8 * cc + 3]),
+                                 tc::pack_bf16(x[8 * cc + 4], x[8 * cc + 5]),
+                                 tc::pack_bf16(x[8 * cc + 6], x[8 * cc + 7]));
+            }
+            tc::fence_proxy_async();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->p_full[h]);
+        }
+        if (ok && tc::mbar_wait(&bars->o_done[h], (n_tiles - 1) & 1, abort, a.status)) {
+            tc::fence_after_sync();
+            const long long row = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + m * TILE + i;
+            __nv_bfloat16 *orow = a.out + row * D;
+            const float inv_l = 1.f / l_run;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tc::tmem_ld32(o_addr + c0, o);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c += 8) {
+                    uint4 v;
+                    v.x = tc::pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+                    v.y = tc::pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
+                    v.z = tc::pack_bf16(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
+                    v.w = tc::pack_bf16(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
+                    *reinterpret_cast<uint4 *>(orow + c0 + c) = v;
+                }
+            }
+            a.lse[row] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (*abort) {
+        // a wait gave up: let the copies and UMMAs still in flight finish before
+        // shared memory and TMEM are released
+        int never = 0;
+        if (warp == 0 && lane == 0) {
+            const int issued = bars->issued;
+            for (int j = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; j < issued; ++j)
+                tc::mbar_wait(&bars->kv_full[j % NSTAGE], (j / NSTAGE) & 1, &never, a.status, 1ll << 28);
+            tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
+        }
+        if (warp == 1 && lane == 0) {
+            tc::mma_commit(&bars->drain);
+            tc::mbar_wait(&bars->drain, 0, &never, a.status, 1ll << 28);
+        }
+        __syncwarp();
+        tc::fence_after_sync();
+    }
+    if (warp == 1) tc::tmem_dealloc<512>(tmem);
 }
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+// 2D map over rows of D bf16 values (256 B each), 64 x 64 boxes, 128-byte swizzle.
+bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+template <int NH>
+hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
+                       const void *vs, const int32_t *idx, void *out, float *lse, unsigned *status,
+                       cudaStream_t stream) {
+    CUtensorMap mq, mkh, mvh, mks, mvs;
+    const long long n_bg = (long long)p.batch * p.n_kv_heads;
+    const unsigned long long q_rows = (unsigned long long)p.batch * p.n_q_heads * p.seg_len;
+    const long long hist_rows =
+        p.hist_head_stride > 0 ? (n_bg - 1) * p.hist_head_stride + (long long)p.n_hist_chunks * p.chunk
+                               : (long long)p.n_hist_chunks * p.chunk;
+    const unsigned long long seg_rows = (unsigned long long)((n_bg - 1) * p.seg_head_stride + p.seg_len);
+    if (!make_map(&mq, q, q_rows) || !make_map(&mks, ks, seg_rows) || !make_map(&mvs, vs, seg_rows))
+        return HGA_ERR_INVALID_ARG;
+    if (hist_rows > 0) {
+        if (!make_map(&mkh, kh, (unsigned long long)hist_rows) || !make_map(&mvh, vh, (unsigned long long)hist_rows))
+            return HGA_ERR_INVALID_ARG;
+    } else {
+        mkh = mks;  // never read: no routable history
+        mvh = mvs;
+    }
+    const int nqb = p.seg_len / p.q_block;
+    FwdArgs a;
+    a.batch = p.batch;
+    a.n_q_heads = p.n_q_heads;
+    a.n_kv_heads = p.n_kv_heads;
+    a.seg_len = p.seg_len;
+    a.topk = p.topk;
+    a.n_hist_chunks = p.n_hist_chunks;
+    a.hist_stride = p.hist_head_stride;
+    a.seg_stride = p.seg_head_stride;
+    a.qb0 = p.qblock_end > 0 ? p.qblock_begin : 0;
+    a.n_blocks = (p.qblock_end > 0 ? p.qblock_end : nqb) - a.qb0;
+    a.idx = idx;
+    a.out = static_cast<__nv_bfloat16 *>(out);
+    a.lse = lse;
+    a.status = status;
+    a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
+    const size_t smem = Smem<NH>::ALLOC;
+    auto kern = attn_fwd_tc_kernel<NH>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return record_cuda(e);
+    const unsigned grid = (unsigned)(a.n_blocks * n_bg);
+    if (grid == 0) return HGA_OK;
+    kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
+    return record_cuda(cudaGetLastError());
+}
+
+}  // namespace
+
+bool attn_fwd_tc_supported(const hga_params_t &p) {
+    const int G = p.n_q_heads / p.n_kv_heads;
+    if (p.dtype != HGA_BF16 || p.head_dim != 128 || p.chunk != 64 || p.q_block != 64) return false;
+    if (G != 2 && G != 4) return false;
+    // TMA row coordinates are 32-bit
+    const long long n_bg = (long long)p.batch * p.n_kv_heads;
+    if (n_bg * (p.hist_head_stride > p.seg_head_stride ? p.hist_head_stride : p.seg_head_stride) >= (1ll << 31))
+        return false;
+    if ((long long)p.batch * p.n_q_heads * p.seg_len >= (1ll << 31)) return false;
+    return get_encoder();
+}
+
+hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,
+                                const void *ks, const void *vs, const int32_t *idx, void *out, float *lse,
+                                unsigned *status, cudaStream_t stream) {
+    const int G = p.n_q_heads / p.n_kv_heads;
+    if (G == 4) return launch_nh<2>(p, q, kh, vh, ks, vs, idx, out, lse, status, stream);
+    return launch_nh<1>(p, q, kh, vh, ks, vs, idx, out, lse, status, stream);
+}
+
 }  // namespace hga

@@ -202,7 +202,7 @@ __global__ void __launch_bounds__(NT) bwd_dq_simt_kernel(hga_params_t p, const T
                                                          const T *__restrict__ k_seg, const T *__restrict__ v_seg,
                                                          const int32_t *__restrict__ idx, const float *__restrict__ lse,
                                                          const float *__restrict__ delta, const T *__restrict__ dout,
-                                                         T *__restrict__ dq, unsigned *status) {
+                                                         float *__restrict__ dq, unsigned *status) {
     constexpr int LD = D + 1;
     constexpr int DPT = D / 16;
     extern __shared__ float sm[];
@@ -290,7 +290,7 @@ __global__ void __launch_bounds__(NT) bwd_dq_simt_kernel(hga_params_t p, const T
 #pragma unroll
     for (int r = 0; r < 4; ++r)
 #pragma unroll
-        for (int c = 0; c < DPT; ++c) dq[(row0 + rg * 4 + r) * D + cg + 16 * c] = from_f32<T>(acc[r][c] * scale);
+        for (int c = 0; c < DPT; ++c) dq[(row0 + rg * 4 + r) * D + cg + 16 * c] = acc[r][c] * scale;
 }
 
 // dK/dV of the active segment: key-major, summing over the later query
@@ -299,8 +299,8 @@ template <typename T, int D>
 __global__ void __launch_bounds__(NT) bwd_dkdv_simt_kernel(hga_params_t p, const T *__restrict__ q,
                                                            const T *__restrict__ k_seg, const T *__restrict__ v_seg,
                                                            const float *__restrict__ lse, const float *__restrict__ delta,
-                                                           const T *__restrict__ dout, T *__restrict__ dk,
-                                                           T *__restrict__ dv) {
+                                                           const T *__restrict__ dout, float *__restrict__ dk,
+                                                           float *__restrict__ dv) {
     constexpr int LD = D + 1;
     constexpr int DPT = D / 16;
     extern __shared__ float sm[];
@@ -387,8 +387,8 @@ __global__ void __launch_bounds__(NT) bwd_dkdv_simt_kernel(hga_params_t p, const
     for (int r = 0; r < 4; ++r)
 #pragma unroll
         for (int c = 0; c < DPT; ++c) {
-            dk[out0 + (rg * 4 + r) * D + cg + 16 * c] = from_f32<T>(akk[r][c] * scale);
-            dv[out0 + (rg * 4 + r) * D + cg + 16 * c] = from_f32<T>(avv[r][c]);
+            dk[out0 + (rg * 4 + r) * D + cg + 16 * c] = akk[r][c] * scale;
+            dv[out0 + (rg * 4 + r) * D + cg + 16 * c] = avv[r][c];
         }
 }
 
@@ -428,7 +428,7 @@ static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, 
         if (e != cudaSuccess) return record_cuda(e);
         kern<<<(unsigned)(nqb * p.batch * p.n_q_heads), NT, smem, stream>>>(
             p, (const T *)q, (const T *)kh, (const T *)vh, (const T *)ks, (const T *)vs, idx, lse, delta,
-            (const T *)dout, (T *)dq, status);
+            (const T *)dout, (float *)dq, status);
         e = cudaGetLastError();
         if (e != cudaSuccess) return record_cuda(e);
     }
@@ -438,7 +438,7 @@ static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, 
         e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return record_cuda(e);
         kern<<<(unsigned)(nqb * p.batch * p.n_kv_heads), NT, smem, stream>>>(
-            p, (const T *)q, (const T *)ks, (const T *)vs, lse, delta, (const T *)dout, (T *)dk, (T *)dv);
+            p, (const T *)q, (const T *)ks, (const T *)vs, lse, delta, (const T *)dout, (float *)dk, (float *)dv);
         e = cudaGetLastError();
     }
     return record_cuda(e);

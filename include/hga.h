@@ -153,10 +153,11 @@ size_t hga_attn_bwd_workspace_size(const hga_params_t *p);
  *   dk_seg[b][g][t] = sum_{h in g, i >= t} dS_t q_i / sqrt(D) (segment keys only)
  *   dv_seg[b][g][t] = sum_{h in g, i >= t} P_t dO_i           (segment keys only)
  * History K/V get no gradient.  out / lse are the forward's outputs for
- * every block (qblock_begin/end must be 0/0).  dq, dk_seg, dv_seg: device,
- * dtype, overwritten (dk_seg/dv_seg use seg_head_stride = S layout
- * [B][Hkv][S][D]).  workspace: device, >= hga_attn_bwd_workspace_size(p)
- * bytes, 16-byte aligned. */
+ * every block (qblock_begin/end must be 0/0).  dq [B][Hq][S][D], dk_seg and
+ * dv_seg [B][Hkv][S][D]: device fp32 for every input dtype (gradients are
+ * sums over many rows; fp32 keeps them within the tolerance a bf16 store
+ * would exceed once |grad| >= 8), overwritten.  workspace: device, >=
+ * hga_attn_bwd_workspace_size(p) bytes, 16-byte aligned. */
 hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                           const void *k_seg, const void *v_seg, const int32_t *idx, const void *out,
                           const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg,

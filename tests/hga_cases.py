@@ -99,9 +99,9 @@ class GpuSegment:
     def bwd(self, idx, out, lse, dout=None):
         import hierarchical_sparse_long_b200 as hga
         dout = self.dout if dout is None else dout
-        dq = torch.empty_like(self.q)
+        dq = torch.empty(self.q.shape, device="cuda", dtype=torch.float32)
         w = self.w
-        dk = torch.empty(w.batch, w.n_kv_heads, w.seg_len, w.head_dim, device="cuda", dtype=self.q.dtype)
+        dk = torch.empty(w.batch, w.n_kv_heads, w.seg_len, w.head_dim, device="cuda", dtype=torch.float32)
         dv = torch.empty_like(dk)
         ws = torch.empty(hga.hga_attn_bwd_workspace_size(self.p) // 4 + 1, device="cuda", dtype=torch.float32)
         hga.hga_attn_bwd(self.p, self.q, self.k_all, self.v_all, self.k_seg, self.v_seg, idx, out, lse, dout, dq,
