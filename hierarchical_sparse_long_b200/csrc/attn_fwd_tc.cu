@@ -237,7 +237,11 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
             const int bb = j & 1;
-            if (!tc::mbar_wait(&bars->s_full[h][bb], (j >> 1) & 1, abort, a.status)) { ok = false; break; }
+            // tcgen05.ld/st below are warp-collective: keep every decision warp-uniform
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[h][bb], (j >> 1) & 1, abort, a.status))) {
+                ok = false;
+                break;
+            }
             tc::fence_after_sync();
             uint32_t sr[64];
             {
@@ -272,9 +276,13 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             l_run = l_run * alpha + sum;
             // PV of the previous tile must be done before P is overwritten and O rescaled
             if (j >= 1) {
-                if (!tc::mbar_wait(&bars->o_done[h], (j - 1) & 1, abort, a.status)) { ok = false; break; }
+                if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h], (j - 1) & 1, abort, a.status))) {
+                    ok = false;
+                    break;
+                }
                 tc::fence_after_sync();
-                if (m_new > m_run) {
+                // rows whose max did not grow have alpha == 1 and are rescaled by an exact no-op
+                if (__any_sync(0xffffffffu, m_new > m_run)) {
 #pragma unroll 1
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t o[32];
@@ -301,7 +309,7 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->p_full[h]);
         }
-        if (ok && tc::mbar_wait(&bars->o_done[h], (n_tiles - 1) & 1, abort, a.status)) {
+        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h], (n_tiles - 1) & 1, abort, a.status))) {
             tc::fence_after_sync();
             const long long row = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + m * TILE + i;
             __nv_bfloat16 *orow = a.out + row * D;
@@ -344,7 +352,10 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         __syncwarp();
         tc::fence_after_sync();
     }
-    if (warp == 1) tc::tmem_dealloc<512>(tmem);
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_dealloc<512>(tmem);
+    }
 }
 
 // ------------------------------------------------------------------ host side
