@@ -22,7 +22,8 @@ STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3:
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
 EXPORTED = ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
-            "hga_fetch_tiered", "hga_get_device_status", "hga_status_string", "hga_last_error")
+            "hga_attn_bwd_noalloc", "hga_fetch_tiered", "hga_get_device_status", "hga_status_string",
+            "hga_last_error")
 
 
 class HGAError(RuntimeError):
@@ -85,13 +86,14 @@ def lib() -> ctypes.CDLL:
         L.hga_attn_bwd_workspace_size.argtypes = [pp]
         L.hga_attn_bwd_workspace_size.restype = sz
         L.hga_attn_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.hga_attn_bwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hga_status_string.argtypes = [i]
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
-        for f in ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_fetch_tiered",
-                  "hga_get_device_status"):
+        for f in ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
+                  "hga_fetch_tiered", "hga_get_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -160,6 +162,18 @@ def hga_attn_bwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, dout
     _check(lib().hga_attn_bwd(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg),
                               _ptr(idx), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq), _ptr(dk_seg), _ptr(dv_seg),
                               _ptr(workspace), nbytes, _stream(stream)), "hga_attn_bwd")
+
+
+def hga_attn_bwd_noalloc(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, dout, dq, dk_seg, dv_seg,
+                         stream=None):
+    """hga_attn_bwd for callers that cannot allocate device memory: the
+    workspace is a fixed array inside the library (batch * q heads * segment
+    length <= 1,048,576).  Calls on one device share that array, so calls
+    that overlap on the GPU must be serialised by the caller."""
+    cp = p.c()
+    _check(lib().hga_attn_bwd_noalloc(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg),
+                                      _ptr(v_seg), _ptr(idx), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                      _ptr(dk_seg), _ptr(dv_seg), _stream(stream)), "hga_attn_bwd_noalloc")
 
 
 def hga_fetch_tiered(p: Params, host_k, host_v, idx, qblock_begin: int, qblock_end: int, stage_k, stage_v,

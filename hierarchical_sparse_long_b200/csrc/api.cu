@@ -66,6 +66,7 @@ hga_status_t record_cuda(cudaError_t e) {
     t_last_error = cudaGetErrorString(e);
     return HGA_ERR_CUDA;
 }
+void record_error(const char *msg) { t_last_error = msg; }
 }  // namespace hga
 
 extern "C" {

@@ -163,6 +163,29 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
                           const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg,
                           void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* hga_attn_bwd without a caller-supplied workspace.  The source pages have
+ * no counterpart to this call; it exists for callers that cannot allocate
+ * device memory themselves -- a plugin or serving runtime that owns every
+ * byte of device memory through its own pool and only hands the library
+ * tensors and a stream, or a hot path that must not call cudaMalloc.  It
+ * computes exactly what hga_attn_bwd computes, with the same arguments minus
+ * workspace / workspace_bytes, and allocates nothing: the fp32 row terms live
+ * in a fixed 4 MiB array inside the library, which every GPU that loads the
+ * library keeps until the process exits.
+ *   Limit: batch * n_q_heads * seg_len <= 1,048,576 query rows; larger
+ *   shapes return HGA_ERR_INVALID_ARG (message in hga_last_error()).
+ *   The first call on a device looks up that device's copy of the array
+ *   (with the device current); make that first call before any stream
+ *   capture.  All calls on a device share the one array: calls that overlap
+ *   on the GPU (different streams without ordering between them) race and
+ *   must be serialised by the caller.  The array keeps the last call's
+ *   contents; nothing in it needs clearing, as every call rewrites the row
+ *   terms before reading them. */
+hga_status_t hga_attn_bwd_noalloc(const hga_params_t *p, const void *q, const void *k_hist,
+                                  const void *v_hist, const void *k_seg, const void *v_seg,
+                                  const int32_t *idx, const void *out, const float *lse, const void *dout,
+                                  void *dq, void *dk_seg, void *dv_seg, cudaStream_t stream);
+
 /* Tiered history (technical summary section 2.2: detached K/V live in host
  * RAM, only the routed exact K/V are brought to the GPU).  For the query
  * blocks [qblock_begin, qblock_end) of idx, gathers the distinct (b, g, chunk)
