@@ -38,6 +38,7 @@ namespace {
 constexpr int D = 128;
 constexpr int TILE = 64;
 constexpr int NSTAGE = 3;
+constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold on the running max (log2 units)
 constexpr uint32_t Q_HALF_BYTES = 128 * D * 2;   // 32 KiB: [2 col halves][128 rows][128 B]
 constexpr uint32_t KV_TILE_BYTES = TILE * D * 2; // 16 KiB: [2 col halves][64 rows][128 B]
 constexpr uint32_t P_BYTES = 128 * TILE * 2;     // 16 KiB: [128 rows][128 B]
@@ -257,22 +258,30 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             if (lane == 0) tc::mbar_arrive(&bars->s_free[h][bb]);
             float x[64];
             const bool diag = (j == n_tiles - 1);  // the local tile of this block
-            float mx = -INFINITY;
+            float mpart[8];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
                 float v = __uint_as_float(sr[c]) * a.scale_log2;
                 if (diag && c > i) v = -INFINITY;
                 x[c] = v;
-                mx = fmaxf(mx, v);
+                mpart[c & 7] = (c < 8) ? v : fmaxf(mpart[c & 7], v);
             }
-            const float m_new = fmaxf(m_run, mx);
-            float sum = 0.f;
+            const float mx = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
+                                   fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7])));
+            // Lazy rescaling: the reference max only moves when the row max grows by
+            // more than kRescaleLog2, so P stays <= 2^kRescaleLog2 and O is rescaled
+            // in TMEM only on those (rare) tiles.
+            const bool grow = mx > m_run + kRescaleLog2;
+            const float m_use = grow ? mx : m_run;
+            const float alpha = grow ? tc::ex2(m_run - m_use) : 1.f;
+            float spart[8];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                x[c] = tc::ex2(x[c] - m_new);
-                sum += x[c];
+                x[c] = tc::ex2(x[c] - m_use);
+                spart[c & 7] = (c < 8) ? x[c] : spart[c & 7] + x[c];
             }
-            const float alpha = tc::ex2(m_run - m_new);
+            const float sum = ((spart[0] + spart[1]) + (spart[2] + spart[3])) +
+                              ((spart[4] + spart[5]) + (spart[6] + spart[7]));
             l_run = l_run * alpha + sum;
             // PV of the previous tile must be done before P is overwritten and O rescaled
             if (j >= 1) {
@@ -281,8 +290,8 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                // rows whose max did not grow have alpha == 1 and are rescaled by an exact no-op
-                if (__any_sync(0xffffffffu, m_new > m_run)) {
+                // rows that keep their reference max have alpha == 1: an exact no-op
+                if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
                     for (int c0 = 0; c0 < D; c0 += 32) {
                         uint32_t o[32];
@@ -295,7 +304,7 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                     tc::tmem_wait_st();
                 }
             }
-            m_run = m_new;
+            m_run = m_use;
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
                 const uint32_t addr = p_row + ((cc ^ (r & 7)) << 4);

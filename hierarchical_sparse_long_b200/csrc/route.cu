@@ -11,10 +11,10 @@
 //
 // One CTA per (batch, kv head, query block).  The CTA reads its G*q_block
 // query rows once with 16-byte coalesced loads (the kernel's HBM traffic),
-// scores the L2-resident summaries with one warp per chunk (fp32 FFMA and a
-// fixed butterfly, no tensor cores so the scores are exact fp32 dot
-// products), then ranks 64-bit keys (order-preserving score bits, inverted
-// chunk index) with a shared-memory bitonic sort.
+// scores the L2-resident summaries with one thread per chunk (fp32 FFMA, no
+// tensor cores, so every score is an fp32 dot product in a fixed order),
+// then ranks 64-bit keys (order-preserving score bits, inverted chunk index)
+// with a shared-memory bitonic sort.
 #include "common.cuh"
 
 namespace hga {
@@ -46,14 +46,29 @@ __global__ void __launch_bounds__(256) route_kernel(const T *__restrict__ q, con
     const int G = n_q_heads / n_kv_heads;
     const int tid = threadIdx.x;
 
-    // 1. block summary: mean over G heads x q_block rows, fixed order
+    // 1. block summary: mean over G heads x q_block rows, fixed order; every
+    //    thread keeps 8 independent 16-byte loads in flight
     {
         const int col = (tid % LPR) * VEC, slot = tid / LPR;
         float acc[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
         const int rows = G * q_block;
-        for (int r = slot; r < rows; r += NSLOT) {
+        int r = slot;
+        for (; r + 7 * NSLOT < rows; r += 8 * NSLOT) {
+            float v[8][VEC];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int rr = r + u * NSLOT;
+                const int h = g * G + rr / q_block, i = m * q_block + rr % q_block;
+                Vec16<T>::load(q + (((long long)b * n_q_heads + h) * seg_len + i) * D + col, v[u]);
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+#pragma unroll
+                for (int e = 0; e < VEC; ++e) acc[e] += v[u][e];
+        }
+        for (; r < rows; r += NSLOT) {
             const int h = g * G + r / q_block, i = m * q_block + r % q_block;
             float v[VEC];
             Vec16<T>::load(q + (((long long)b * n_q_heads + h) * seg_len + i) * D + col, v);
@@ -71,29 +86,22 @@ __global__ void __launch_bounds__(256) route_kernel(const T *__restrict__ q, con
     }
     __syncthreads();
 
-    // 2. scores -> rank keys; one warp per chunk
-    const int warp = tid >> 5, lane = tid & 31;
-    constexpr int PER_LANE = D / 32;
-    float qv[PER_LANE];
-#pragma unroll
-    for (int e = 0; e < PER_LANE; ++e) qv[e] = qbar[lane * PER_LANE + e];
+    // 2. scores -> rank keys; one thread per chunk, four interleaved partial
+    //    dot products over d (mod 4) summed in a fixed order
     const float *sb = summ + (long long)bg * cap * D;
-    for (int j = warp; j < n_chunks; j += 8) {
-        const float *row = sb + (long long)j * D + lane * PER_LANE;
-        float dot = 0.f;
-        if constexpr (PER_LANE == 4) {
-            float4 v = *reinterpret_cast<const float4 *>(row);
-            dot = fmaf(qv[0], v.x, dot);
-            dot = fmaf(qv[1], v.y, dot);
-            dot = fmaf(qv[2], v.z, dot);
-            dot = fmaf(qv[3], v.w, dot);
-        } else {
-#pragma unroll
-            for (int e = 0; e < PER_LANE; ++e) dot = fmaf(qv[e], row[e], dot);
+    for (int j = tid; j < n_chunks; j += 256) {
+        const float4 *row = reinterpret_cast<const float4 *>(sb + (long long)j * D);
+        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
+#pragma unroll 8
+        for (int e = 0; e < D / 4; ++e) {
+            const float4 v = row[e];
+            d0 = fmaf(qbar[4 * e + 0], v.x, d0);
+            d1 = fmaf(qbar[4 * e + 1], v.y, d1);
+            d2 = fmaf(qbar[4 * e + 2], v.z, d2);
+            d3 = fmaf(qbar[4 * e + 3], v.w, d3);
         }
-#pragma unroll
-        for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        if (lane == 0) keys[j] = rank_key(dot * inv_sqrt_d, j);
+        const float dot = (d0 + d1) + (d2 + d3);
+        keys[j] = rank_key(dot * inv_sqrt_d, j);
     }
     for (int j = n_chunks + tid; j < npow2; j += 256) keys[j] = 0ull;  // below every real key
     __syncthreads();

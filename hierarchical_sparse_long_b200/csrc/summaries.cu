@@ -6,11 +6,11 @@
 // the mean of the chunk's keys.
 //
 // HBM-bound: every key byte is read once with 16-byte coalesced loads and
-// D*4 bytes are written per chunk.  One warp reduces one chunk; each lane
-// owns 16 bytes of a row and walks every (32 / lanes_per_row)-th row, so a
-// warp instruction reads 512 contiguous bytes.  The reduction order is fixed
-// (per-lane sequential, then a fixed butterfly), so summaries built in one
-// pass and summaries appended segment by segment are bit-identical.
+// D*4 bytes are written per chunk.  One 256-thread CTA reduces one chunk:
+// each thread owns 16 bytes of a row and a fixed set of rows (all its loads
+// are in flight together), and the row slots are then summed through shared
+// memory in a fixed order, so summaries built in one pass and summaries
+// appended segment by segment are bit-identical.
 #include "common.cuh"
 
 namespace hga {
@@ -20,61 +20,53 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T *__restrict__ k,
                                                         int n_slices, int chunk, int first_chunk,
                                                         int n_chunks, float *__restrict__ summ, int cap) {
     constexpr int VEC = Vec16<T>::N;
-    constexpr int LPR = D / VEC;   // lanes per row
-    constexpr int RPI = 32 / LPR;  // rows per warp step
-    static_assert(LPR >= 1 && LPR <= 32 && 32 % LPR == 0, "unsupported head_dim");
-    const int lane = threadIdx.x & 31;
-    const long long task = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (task >= (long long)n_slices * n_chunks) return;
-    const int slice = (int)(task / n_chunks);
-    const int j = first_chunk + (int)(task % n_chunks);
-    const int col = (lane % LPR) * VEC;
-    const int rslot = lane / LPR;
+    constexpr int LPR = D / VEC;     // threads per row
+    constexpr int NSLOT = 256 / LPR; // row slots
+    static_assert(LPR >= 1 && LPR <= 256 && 256 % LPR == 0, "unsupported head_dim");
+    __shared__ float part[NSLOT][D + 1];
+    const int tid = threadIdx.x;
+    const int slice = (int)(blockIdx.x / n_chunks);
+    const int j = first_chunk + (int)(blockIdx.x % n_chunks);
+    const int col = (tid % LPR) * VEC;
+    const int rslot = tid / LPR;
     const T *base = k + ((long long)slice * head_stride + (long long)j * chunk) * D + col;
 
     float acc[VEC];
 #pragma unroll
     for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
     int r = rslot;
-    // 8 loads in flight per lane
-    for (; r + 7 * RPI < chunk; r += 8 * RPI) {
-        float v[8][VEC];
+    for (; r + 3 * NSLOT < chunk; r += 4 * NSLOT) {
+        float v[4][VEC];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) Vec16<T>::load(base + (long long)(r + u * RPI) * D, v[u]);
+        for (int u = 0; u < 4; ++u) Vec16<T>::load(base + (long long)(r + u * NSLOT) * D, v[u]);
 #pragma unroll
-        for (int u = 0; u < 8; ++u)
+        for (int u = 0; u < 4; ++u)
 #pragma unroll
             for (int e = 0; e < VEC; ++e) acc[e] += v[u][e];
     }
-    for (; r < chunk; r += RPI) {
+    for (; r < chunk; r += NSLOT) {
         float v[VEC];
         Vec16<T>::load(base + (long long)r * D, v);
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] += v[e];
     }
 #pragma unroll
-    for (int off = LPR; off < 32; off <<= 1)
+    for (int e = 0; e < VEC; ++e) part[rslot][col + e] = acc[e];
+    __syncthreads();
+    if (tid < D) {
+        float s = 0.f;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] += __shfl_xor_sync(0xffffffffu, acc[e], off);
-    if (rslot == 0) {
-        float *dst = summ + ((long long)slice * cap + j) * D + col;
-        const float n = (float)chunk;
-#pragma unroll
-        for (int e = 0; e < VEC; e += 4) {
-            float4 o = make_float4(acc[e] / n, acc[e + 1] / n, acc[e + 2] / n, acc[e + 3] / n);
-            *reinterpret_cast<float4 *>(dst + e) = o;
-        }
+        for (int sl = 0; sl < NSLOT; ++sl) s += part[sl][tid];
+        summ[((long long)slice * cap + j) * D + tid] = s / (float)chunk;
     }
 }
 
 template <typename T, int D>
 static hga_status_t launch_t(const void *k, long long head_stride, int bh, int chunk, int first_chunk,
                              int n_chunks, float *summ, int cap, cudaStream_t stream) {
-    const long long tasks = (long long)bh * n_chunks;
-    const int warps_per_block = 8;
-    const long long blocks = (tasks + warps_per_block - 1) / warps_per_block;
-    summaries_kernel<T, D><<<(unsigned)blocks, 32 * warps_per_block, 0, stream>>>(
-        static_cast<const T *>(k), head_stride, bh, chunk, first_chunk, n_chunks, summ, cap);
+    const long long blocks = (long long)bh * n_chunks;
+    summaries_kernel<T, D><<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const T *>(k), head_stride, bh,
+                                                                 chunk, first_chunk, n_chunks, summ, cap);
     return record_cuda(cudaGetLastError());
 }
 
