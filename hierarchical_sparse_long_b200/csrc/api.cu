@@ -144,12 +144,20 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
     if (p->n_hist_chunks > 0 && (!k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
     if (workspace_bytes < hga_attn_bwd_workspace_size(p)) return HGA_ERR_INVALID_ARG;
     for (const void *ptr : {q, k_hist, v_hist, k_seg, v_seg, out, dout, (const void *)dq, (const void *)dk_seg,
-                            (const void *)dv_seg, (const void *)workspace})
+                            (const void *)dv_seg, (const void *)workspace, (const void *)lse})
         if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    float *delta = static_cast<float *>(workspace);
+    if (hga::attn_bwd_tc_supported(*p)) {
+        st = hga::launch_bwd_delta(*p, out, dout, delta, stream);
+        if (st != HGA_OK) return st;
+        return hga::launch_attn_bwd_tc(*p, q, k_hist, v_hist, k_seg, v_seg, idx, lse, delta, dout,
+                                       static_cast<float *>(dq), static_cast<float *>(dk_seg),
+                                       static_cast<float *>(dv_seg), status, stream);
+    }
     return hga::launch_attn_bwd_simt(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, dout, dq, dk_seg, dv_seg,
-                                     static_cast<float *>(workspace), status, stream);
+                                     delta, status, stream);
 }
 
 hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,

@@ -1,0 +1,671 @@
+// Backward of the exact-token HGA attention on tcgen05 tensor cores (bf16
+// inputs, fp32 accumulation in TMEM, head_dim 128).
+//
+// "Long-Context Fine-Tuning with Limited VRAM", technical summary sections
+// 2.1 (routing without gradient; gather and attention differentiable) and 2.2
+// (segment-wise backward: history K/V detached at the segment boundary).
+// With P = softmax row of query i (recomputed from the forward's LSE) and
+// delta_i = rowsum(dO * O):
+//   dS = P * (dO V^T - delta)
+//   dQ = dS K / sqrt(D)                      over routed history and segment keys
+//   dK_seg = dS^T Q / sqrt(D), dV_seg = P^T dO   over segment keys only
+//
+// Two kernels, no atomics (results are deterministic):
+//   bwd_dq_tc  : query-major, one CTA per (batch, kv head, query block) holding
+//                the G heads of the group as M=128 halves (like the forward);
+//                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128), the
+//                dS rows in bf16 into shared memory, dQ += dS K (M128 N128 K64).
+//   bwd_dkdv_tc: key-major over the active segment, one CTA per (batch, kv
+//                head, 128 segment keys); for every later 64-query tile of
+//                every head of the group: S^T = K Q^T and dP^T = V dO^T
+//                (M128 N64 K128), P^T and dS^T in bf16 into shared memory,
+//                dV += P^T dO and dK += dS^T Q (M128 N128 K64).
+// Warp 0 issues TMA loads, warp 1 owns TMEM and issues the UMMAs from one
+// thread, the remaining warpgroups handle one TMEM lane (row) per thread.
+// Every wait is bounded and every warp-collective TMEM access is made from a
+// converged warp with warp-uniform decisions.
+#include <cudaTypedefs.h>
+#include <mutex>
+
+#include "tc_ptx.cuh"
+
+namespace hga {
+
+namespace {
+
+constexpr int D = 128;
+constexpr int TILE = 64;
+constexpr uint32_t HALF_BYTES = 128 * D * 2;    // 32 KiB: [2 col halves][128 rows][128 B]
+constexpr uint32_t TILE_BYTES = TILE * D * 2;   // 16 KiB: [2 col halves][64 rows][128 B]
+constexpr uint32_t ROWS128_K64 = 128 * TILE * 2; // 16 KiB: [128 rows][128 B] bf16, K = 64
+constexpr uint32_t IDESC_N64 = tc::idesc_bf16(128, TILE, false, false);
+constexpr uint32_t IDESC_N128_BMN = tc::idesc_bf16(128, D, false, true);
+
+struct BwdArgs {
+    int batch, n_q_heads, n_kv_heads, seg_len, topk, n_hist_chunks;
+    long long hist_stride, seg_stride;
+    const int32_t *idx;
+    const float *lse;
+    const float *delta;
+    float *dq;
+    float *dk;
+    float *dv;
+    unsigned *status;
+    float scale_log2;  // log2(e) / sqrt(D)
+    float scale;       // 1 / sqrt(D)
+};
+
+// S = A B^T over D = 128 (K-major A rows at a_base with 128-row halves, K-major
+// 64-row B tile at b_base): 8 UMMA steps of K = 16.
+__device__ __forceinline__ void mma_rows_x_tile(uint32_t d, uint32_t a_base, uint32_t b_base) {
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const uint32_t kb = (kk & 3) * 32;
+        const uint64_t adesc = tc::desc_sw128(a_base + (kk >> 2) * (128 * 128) + kb, 16, 1024);
+        const uint64_t bdesc = tc::desc_sw128(b_base + (kk >> 2) * (64 * 128) + kb, 16, 1024);
+        tc::mma_f16(d, adesc, bdesc, IDESC_N64, kk > 0 ? 1u : 0u);
+    }
+}
+
+// D(+)= A B with A = 128 rows x 64 (K-major, bf16 written by the threads) and
+// B = a 64-row tile read MN-major (N = D = 128): 4 UMMA steps of K = 16.
+__device__ __forceinline__ void mma_k64_x_tile(uint32_t d, uint32_t a_base, uint32_t b_base, bool accumulate) {
+#pragma unroll
+    for (int kk = 0; kk < TILE / 16; ++kk) {
+        const uint64_t adesc = tc::desc_sw128(a_base + kk * 32, 16, 1024);
+        const uint64_t bdesc = tc::desc_sw128(b_base + kk * 2048, 8192, 1024);
+        tc::mma_f16(d, adesc, bdesc, IDESC_N128_BMN, (accumulate || kk > 0) ? 1u : 0u);
+    }
+}
+
+// Writes 32 packed bf16 pairs (64 values) of row r as a 128-byte SW128 row.
+__device__ __forceinline__ void store_row_sw128(uint32_t row_addr, int r, const uint32_t (&pk)[32]) {
+#pragma unroll
+    for (int cc = 0; cc < 8; ++cc)
+        tc::st_shared_v4(row_addr + ((cc ^ (r & 7)) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
+                         pk[4 * cc + 3]);
+}
+
+// ============================================================ dQ kernel
+template <int NH>
+struct DqSmem {
+    static constexpr int NSTAGE = 2;
+    static constexpr uint32_t Q = 0;
+    static constexpr uint32_t DO = Q + NH * HALF_BYTES;
+    static constexpr uint32_t KV = DO + NH * HALF_BYTES;
+    static constexpr uint32_t DS = KV + NSTAGE * 2 * TILE_BYTES;
+    static constexpr uint32_t BAR = DS + NH * ROWS128_K64;
+    static constexpr uint32_t ALLOC = BAR + 1024 + 1024;
+};
+
+struct DqBars {
+    uint64_t q_full;
+    uint64_t kv_full[2];
+    uint64_t kv_empty[2];
+    uint64_t sdp_full[2];
+    uint64_t sdp_free[2];
+    uint64_t ds_full[2];
+    uint64_t dq_done[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int n_hist;
+    int issued;
+    int tiles[64];
+};
+
+template <int NH>
+__global__ void __launch_bounds__(128 + 128 * NH, 1)
+    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                     const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
+                     const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                     const BwdArgs a) {
+    using L = DqSmem<NH>;
+    constexpr int NST = L::NSTAGE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    DqBars *bars = reinterpret_cast<DqBars *>(smem + L::BAR);
+    const uint32_t sbase = tc::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = 2 * NH;
+    const int nqb = a.seg_len / TILE;
+    const int n_bg = a.batch * a.n_kv_heads;
+    const int m = nqb - 1 - (int)blockIdx.x / n_bg;
+    const int bg = (int)blockIdx.x % n_bg;
+    const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars->q_full, 1);
+        for (int s = 0; s < NST; ++s) {
+            tc::mbar_init(&bars->kv_full[s], 1);
+            tc::mbar_init(&bars->kv_empty[s], 1);
+        }
+        for (int h = 0; h < 2; ++h) {
+            tc::mbar_init(&bars->sdp_full[h], 1);
+            tc::mbar_init(&bars->sdp_free[h], 4);
+            tc::mbar_init(&bars->ds_full[h], 4);
+            tc::mbar_init(&bars->dq_done[h], 1);
+        }
+        tc::mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        bars->issued = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 2 && lane == 0) {
+        const int32_t *sel = a.idx + ((long long)bg * nqb + m) * a.topk;
+        int n = 0;
+        for (int i = 0; i < a.topk; ++i) {
+            const int j = sel[i];
+            if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
+        }
+        bars->n_hist = n;
+    }
+    if (warp == 1) tc::tmem_alloc<512>(&bars->tmem_base);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+    const int n_hist = bars->n_hist;
+    const int n_tiles = n_hist + m + 1;
+    volatile int *abort = &bars->abort;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            tc::mbar_arrive_expect_tx(&bars->q_full, 2 * NH * HALF_BYTES);
+            for (int hh = 0; hh < G; ++hh) {
+                const int qrow = (b * a.n_q_heads + g * G + hh) * a.seg_len + m * TILE;
+                const uint32_t off = (hh >> 1) * HALF_BYTES + (hh & 1) * (64 * 128);
+                tc::tma_load_2d(smem + L::Q + off, &tm_q, 0, qrow, &bars->q_full);
+                tc::tma_load_2d(smem + L::Q + off + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
+                tc::tma_load_2d(smem + L::DO + off, &tm_do, 0, qrow, &bars->q_full);
+                tc::tma_load_2d(smem + L::DO + off + 128 * 128, &tm_do, 64, qrow, &bars->q_full);
+            }
+            int issued = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % NST, u = j / NST;
+                if (j >= NST && !tc::mbar_wait(&bars->kv_empty[s], (u - 1) & 1, abort, a.status)) break;
+                const bool hist = j < n_hist;
+                const CUtensorMap *mk = hist ? &tm_kh : &tm_ks;
+                const CUtensorMap *mv = hist ? &tm_vh : &tm_vs;
+                const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
+                                     : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+                uint8_t *kdst = smem + L::KV + s * 2 * TILE_BYTES;
+                uint8_t *vdst = kdst + TILE_BYTES;
+                tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * TILE_BYTES);
+                tc::tma_load_2d(kdst, mk, 0, row, &bars->kv_full[s]);
+                tc::tma_load_2d(kdst + 64 * 128, mk, 64, row, &bars->kv_full[s]);
+                tc::tma_load_2d(vdst, mv, 0, row, &bars->kv_full[s]);
+                tc::tma_load_2d(vdst + 64 * 128, mv, 64, row, &bars->kv_full[s]);
+                ++issued;
+            }
+            bars->issued = issued;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            auto issue_dq = [&](int t) -> bool {
+                const int s = t % NST;
+                const uint32_t k_base = sbase + L::KV + s * 2 * TILE_BYTES;
+                for (int h = 0; h < NH; ++h) {
+                    if (!tc::mbar_wait(&bars->ds_full[h], t & 1, abort, a.status)) return false;
+                    tc::fence_after_sync();
+                    mma_k64_x_tile(tmem + 128 * h, sbase + L::DS + h * ROWS128_K64, k_base, t > 0);
+                    tc::mma_commit(&bars->dq_done[h]);
+                }
+                tc::mma_commit(&bars->kv_empty[s]);
+                return true;
+            };
+            bool ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
+            for (int j = 0; ok && j < n_tiles; ++j) {
+                const int s = j % NST;
+                if (!tc::mbar_wait(&bars->kv_full[s], (j / NST) & 1, abort, a.status)) { ok = false; break; }
+                tc::fence_after_sync();
+                const uint32_t k_base = sbase + L::KV + s * 2 * TILE_BYTES;
+                for (int h = 0; h < NH; ++h) {
+                    if (j >= 1 && !tc::mbar_wait(&bars->sdp_free[h], (j - 1) & 1, abort, a.status)) {
+                        ok = false;
+                        break;
+                    }
+                    tc::fence_after_sync();
+                    mma_rows_x_tile(tmem + 256 + 128 * h, sbase + L::Q + h * HALF_BYTES, k_base);
+                    mma_rows_x_tile(tmem + 256 + 128 * h + 64, sbase + L::DO + h * HALF_BYTES, k_base + TILE_BYTES);
+                    tc::mma_commit(&bars->sdp_full[h]);
+                }
+                if (!ok) break;
+                if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
+            }
+            if (ok) issue_dq(n_tiles - 1);
+        }
+    } else if (warp >= 4) {
+        const int h = (warp - 4) >> 2;
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;
+        const int hh = 2 * h + (r >> 6);
+        const int i = r & 63;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const long long row = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + m * TILE + i;
+        const float lse2 = a.lse[row] * 1.4426950408889634f;
+        const float dlt = a.delta[row];
+        const uint32_t ds_row = sbase + L::DS + h * ROWS128_K64 + (r >> 3) * 1024 + (r & 7) * 128;
+        bool ok = true;
+        for (int j = 0; j < n_tiles; ++j) {
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[h], j & 1, abort, a.status))) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const bool diag = (j == n_tiles - 1);
+            uint32_t pk[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32], dpv[32];
+                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * h + 32 * half;
+                tc::tmem_ld32(s_addr, sv);
+                tc::tmem_ld32(s_addr + 64, dpv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const int c0 = 32 * half + c;
+                    float p0 = tc::ex2(__uint_as_float(sv[c]) * a.scale_log2 - lse2);
+                    float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2);
+                    if (diag && c0 > i) p0 = 0.f;
+                    if (diag && c0 + 1 > i) p1 = 0.f;
+                    pk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt),
+                                                          p1 * (__uint_as_float(dpv[c + 1]) - dlt));
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[h]);
+            if (j >= 1 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->dq_done[h], (j - 1) & 1, abort, a.status))) {
+                ok = false;
+                break;
+            }
+            store_row_sw128(ds_row, r, pk);
+            tc::fence_proxy_async();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->ds_full[h]);
+        }
+        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->dq_done[h], (n_tiles - 1) & 1, abort, a.status))) {
+            tc::fence_after_sync();
+            float *out = a.dq + row * D;
+#pragma unroll 1
+            for (int c0 = 0; c0 < D; c0 += 32) {
+                uint32_t o[32];
+                tc::tmem_ld32(tmem + lane_addr + 128 * h + c0, o);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c += 4)
+                    *reinterpret_cast<float4 *>(out + c0 + c) =
+                        make_float4(__uint_as_float(o[c]) * a.scale, __uint_as_float(o[c + 1]) * a.scale,
+                                    __uint_as_float(o[c + 2]) * a.scale, __uint_as_float(o[c + 3]) * a.scale);
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (*abort) {
+        int never = 0;
+        if (warp == 0 && lane == 0) {
+            const int issued = bars->issued;
+            for (int j = issued - NST < 0 ? 0 : issued - NST; j < issued; ++j)
+                tc::mbar_wait(&bars->kv_full[j % NST], (j / NST) & 1, &never, a.status, 1ll << 28);
+            tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
+        }
+        if (warp == 1 && lane == 0) {
+            tc::mma_commit(&bars->drain);
+            tc::mbar_wait(&bars->drain, 0, &never, a.status, 1ll << 28);
+        }
+        __syncwarp();
+        tc::fence_after_sync();
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_dealloc<512>(tmem);
+    }
+}
+
+// ============================================================ dK/dV kernel
+struct DkvSmem {
+    static constexpr int NSTAGE = 3;
+    static constexpr uint32_t K = 0;                          // 128 keys, K-major
+    static constexpr uint32_t V = K + HALF_BYTES;
+    static constexpr uint32_t RING = V + HALF_BYTES;          // per stage: Q tile, dO tile
+    static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
+    static constexpr uint32_t PT = RING + NSTAGE * STAGE_BYTES;  // P^T  [128 keys][64 q] bf16
+    static constexpr uint32_t DST = PT + ROWS128_K64;          // dS^T
+    static constexpr uint32_t ROWT = DST + ROWS128_K64;        // per stage: lse2[64], delta[64]
+    static constexpr uint32_t BAR = ROWT + NSTAGE * 512;
+    static constexpr uint32_t ALLOC = BAR + 1024 + 1024;
+};
+
+struct DkvBars {
+    uint64_t kv_full;
+    uint64_t ring_full[3];
+    uint64_t ring_empty[3];
+    uint64_t sdp_full[2];
+    uint64_t sdp_free[2];
+    uint64_t pds_full;
+    uint64_t pds_free;
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort;
+    int issued;
+};
+
+__global__ void __launch_bounds__(256, 1)
+    bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                       const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                       const BwdArgs a) {
+    using L = DkvSmem;
+    constexpr int NST = L::NSTAGE;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    DkvBars *bars = reinterpret_cast<DkvBars *>(smem + L::BAR);
+    const uint32_t sbase = tc::smem_u32(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int nqb = a.seg_len / TILE;
+    const int n_bg = a.batch * a.n_kv_heads;
+    const int n = (int)blockIdx.x / n_bg;  // 128-key tile, earliest (most work) first
+    const int bg = (int)blockIdx.x % n_bg;
+    const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+    const int key0 = 128 * n;
+    const int m0 = key0 / TILE;
+    const int n_steps = G * (nqb - m0);  // (head, query tile) pairs, head-major
+
+    if (threadIdx.x == 0) {
+        tc::mbar_init(&bars->kv_full, 1);
+        for (int s = 0; s < NST; ++s) {
+            tc::mbar_init(&bars->ring_full[s], 1);
+            tc::mbar_init(&bars->ring_empty[s], 1);
+        }
+        for (int bb = 0; bb < 2; ++bb) {
+            tc::mbar_init(&bars->sdp_full[bb], 1);
+            tc::mbar_init(&bars->sdp_free[bb], 4);
+        }
+        tc::mbar_init(&bars->pds_full, 4);
+        tc::mbar_init(&bars->pds_free, 1);
+        tc::mbar_init(&bars->drain, 1);
+        bars->abort = 0;
+        bars->issued = 0;
+        tc::fence_mbar_init();
+    }
+    if (warp == 1) tc::tmem_alloc<512>(&bars->tmem_base);
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    const uint32_t tmem = bars->tmem_base;
+    volatile int *abort = &bars->abort;
+
+    if (warp == 0) {
+        if (lane == 0) {
+            // the CTA's 128 keys and values (rows past the segment read as zero or are never written back)
+            const int krow = (int)((long long)bg * a.seg_stride + key0);
+            tc::mbar_arrive_expect_tx(&bars->kv_full, 2 * HALF_BYTES);
+            for (int part = 0; part < 2; ++part) {
+                const uint32_t off = part * (64 * 128);
+                tc::tma_load_2d(smem + L::K + off, &tm_ks, 0, krow + 64 * part, &bars->kv_full);
+                tc::tma_load_2d(smem + L::K + off + 128 * 128, &tm_ks, 64, krow + 64 * part, &bars->kv_full);
+                tc::tma_load_2d(smem + L::V + off, &tm_vs, 0, krow + 64 * part, &bars->kv_full);
+                tc::tma_load_2d(smem + L::V + off + 128 * 128, &tm_vs, 64, krow + 64 * part, &bars->kv_full);
+            }
+            int issued = 0;
+            for (int t = 0; t < n_steps; ++t) {
+                const int s = t % NST, u = t / NST;
+                if (t >= NST && !tc::mbar_wait(&bars->ring_empty[s], (u - 1) & 1, abort, a.status)) break;
+                const int hh = t / (nqb - m0), mq = m0 + t % (nqb - m0);
+                const long long qrow = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + (long long)mq * TILE;
+                uint8_t *qdst = smem + L::RING + s * L::STAGE_BYTES;
+                uint8_t *gdst = qdst + TILE_BYTES;
+                tc::mbar_arrive_expect_tx(&bars->ring_full[s], 2 * TILE_BYTES + 512);
+                tc::tma_load_2d(qdst, &tm_q, 0, (int)qrow, &bars->ring_full[s]);
+                tc::tma_load_2d(qdst + 64 * 128, &tm_q, 64, (int)qrow, &bars->ring_full[s]);
+                tc::tma_load_2d(gdst, &tm_do, 0, (int)qrow, &bars->ring_full[s]);
+                tc::tma_load_2d(gdst + 64 * 128, &tm_do, 64, (int)qrow, &bars->ring_full[s]);
+                tc::bulk_load(smem + L::ROWT + s * 512, a.lse + qrow, 256, &bars->ring_full[s]);
+                tc::bulk_load(smem + L::ROWT + s * 512 + 256, a.delta + qrow, 256, &bars->ring_full[s]);
+                ++issued;
+            }
+            bars->issued = issued;
+        }
+    } else if (warp == 1) {
+        if (lane == 0) {
+            auto issue_grads = [&](int t) -> bool {
+                const int s = t % NST;
+                if (!tc::mbar_wait(&bars->pds_full, t & 1, abort, a.status)) return false;
+                tc::fence_after_sync();
+                const uint32_t q_base = sbase + L::RING + s * L::STAGE_BYTES;
+                mma_k64_x_tile(tmem, sbase + L::PT, q_base + TILE_BYTES, t > 0);   // dV += P^T dO
+                mma_k64_x_tile(tmem + 128, sbase + L::DST, q_base, t > 0);         // dK += dS^T Q
+                tc::mma_commit(&bars->pds_free);
+                tc::mma_commit(&bars->ring_empty[s]);
+                return true;
+            };
+            bool ok = tc::mbar_wait(&bars->kv_full, 0, abort, a.status);
+            for (int t = 0; ok && t < n_steps; ++t) {
+                const int s = t % NST, bb = t & 1;
+                if (!tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status)) { ok = false; break; }
+                if (t >= 2 && !tc::mbar_wait(&bars->sdp_free[bb], ((t >> 1) - 1) & 1, abort, a.status)) {
+                    ok = false;
+                    break;
+                }
+                tc::fence_after_sync();
+                const uint32_t q_base = sbase + L::RING + s * L::STAGE_BYTES;
+                mma_rows_x_tile(tmem + 256 + 128 * bb, sbase + L::K, q_base);                   // S^T
+                mma_rows_x_tile(tmem + 256 + 128 * bb + 64, sbase + L::V, q_base + TILE_BYTES); // dP^T
+                tc::mma_commit(&bars->sdp_full[bb]);
+                if (t >= 1 && !issue_grads(t - 1)) { ok = false; break; }
+            }
+            if (ok && n_steps > 0) issue_grads(n_steps - 1);
+        }
+    } else if (warp >= 4) {
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;  // key row = TMEM lane
+        const int key = key0 + r;
+        const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
+        const uint32_t pt_row = sbase + L::PT + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t dst_row = sbase + L::DST + (r >> 3) * 1024 + (r & 7) * 128;
+        bool ok = true;
+        for (int t = 0; t < n_steps; ++t) {
+            const int s = t % NST, bb = t & 1;
+            const int mq = m0 + t % (nqb - m0);
+            // the stage's lse / delta rows (TMA-written) and this step's S^T, dP^T in TMEM
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status) &&
+                                             tc::mbar_wait(&bars->sdp_full[bb], (t >> 1) & 1, abort, a.status))) {
+                ok = false;
+                break;
+            }
+            tc::fence_after_sync();
+            const float *lse2 = reinterpret_cast<const float *>(smem + L::ROWT + s * 512);
+            const float *dlt = lse2 + 64;
+            const int q0 = mq * TILE;  // first query position of the tile
+            uint32_t ppk[32], dpk[32];
+#pragma unroll
+            for (int half = 0; half < 2; ++half) {
+                uint32_t sv[32], dpv[32];
+                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * bb + 32 * half;
+                tc::tmem_ld32(s_addr, sv);
+                tc::tmem_ld32(s_addr + 64, dpv);
+                tc::tmem_wait_ld();
+#pragma unroll
+                for (int c = 0; c < 32; c += 2) {
+                    const int c0 = 32 * half + c;
+                    float p0 = tc::ex2(__uint_as_float(sv[c]) * a.scale_log2 - lse2[c0] * 1.4426950408889634f);
+                    float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2[c0 + 1] * 1.4426950408889634f);
+                    if (key > q0 + c0) p0 = 0.f;      // causal: the key comes after the query
+                    if (key > q0 + c0 + 1) p1 = 0.f;
+                    ppk[16 * half + c / 2] = tc::pack_bf16(p0, p1);
+                    dpk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
+                                                           p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
+                }
+            }
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[bb]);
+            if (t >= 1 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->pds_free, (t - 1) & 1, abort, a.status))) {
+                ok = false;
+                break;
+            }
+            store_row_sw128(pt_row, r, ppk);
+            store_row_sw128(dst_row, r, dpk);
+            tc::fence_proxy_async();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->pds_full);
+        }
+        const bool done = ok && (n_steps == 0 ||
+                                 __all_sync(0xffffffffu, tc::mbar_wait(&bars->pds_free, (n_steps - 1) & 1, abort,
+                                                                       a.status)));
+        if (done && n_steps > 0) {
+            tc::fence_after_sync();
+            const bool valid = key < a.seg_len;
+            const long long orow = (long long)bg * a.seg_len + key;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+                float *out = (which ? a.dk : a.dv) + orow * D;
+                const float sc = which ? a.scale : 1.f;
+#pragma unroll 1
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(tmem + lane_addr + 128 * which + c0, o);
+                    tc::tmem_wait_ld();
+                    if (valid) {
+#pragma unroll
+                        for (int c = 0; c < 32; c += 4)
+                            *reinterpret_cast<float4 *>(out + c0 + c) =
+                                make_float4(__uint_as_float(o[c]) * sc, __uint_as_float(o[c + 1]) * sc,
+                                            __uint_as_float(o[c + 2]) * sc, __uint_as_float(o[c + 3]) * sc);
+                    }
+                }
+            }
+        }
+    }
+    tc::fence_before_sync();
+    __syncthreads();
+    tc::fence_after_sync();
+    if (*abort) {
+        int never = 0;
+        if (warp == 0 && lane == 0) {
+            const int issued = bars->issued;
+            for (int t = issued - NST < 0 ? 0 : issued - NST; t < issued; ++t)
+                tc::mbar_wait(&bars->ring_full[t % NST], (t / NST) & 1, &never, a.status, 1ll << 28);
+            tc::mbar_wait(&bars->kv_full, 0, &never, a.status, 1ll << 28);
+        }
+        if (warp == 1 && lane == 0) {
+            tc::mma_commit(&bars->drain);
+            tc::mbar_wait(&bars->drain, 0, &never, a.status, 1ll << 28);
+        }
+        __syncwarp();
+        tc::fence_after_sync();
+    }
+    if (warp == 1) {
+        __syncwarp();
+        tc::tmem_dealloc<512>(tmem);
+    }
+}
+
+// ------------------------------------------------------------------ host side
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+bool get_encoder() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
+    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int NH>
+hga_status_t launch_dq(const hga_params_t &p, const CUtensorMap &mq, const CUtensorMap &mdo,
+                       const CUtensorMap &mkh, const CUtensorMap &mvh, const CUtensorMap &mks,
+                       const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
+    auto kern = bwd_dq_tc_kernel<NH>;
+    const size_t smem = DqSmem<NH>::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return record_cuda(e);
+    const unsigned grid = (unsigned)((p.seg_len / p.q_block) * p.batch * p.n_kv_heads);
+    kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mdo, mkh, mvh, mks, mvs, a);
+    return record_cuda(cudaGetLastError());
+}
+
+}  // namespace
+
+bool attn_bwd_tc_supported(const hga_params_t &p) {
+    const int G = p.n_q_heads / p.n_kv_heads;
+    if (p.dtype != HGA_BF16 || p.head_dim != 128 || p.chunk != 64 || p.q_block != 64) return false;
+    if (G != 2 && G != 4) return false;
+    const long long n_bg = (long long)p.batch * p.n_kv_heads;
+    if (n_bg * (p.hist_head_stride > p.seg_head_stride ? p.hist_head_stride : p.seg_head_stride) >= (1ll << 31))
+        return false;
+    if ((long long)p.batch * p.n_q_heads * p.seg_len >= (1ll << 31)) return false;
+    return get_encoder();
+}
+
+hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,
+                                const void *ks, const void *vs, const int32_t *idx, const float *lse,
+                                const float *delta, const void *dout, float *dq, float *dk, float *dv,
+                                unsigned *status, cudaStream_t stream) {
+    CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
+    const long long n_bg = (long long)p.batch * p.n_kv_heads;
+    const unsigned long long q_rows = (unsigned long long)p.batch * p.n_q_heads * p.seg_len;
+    const long long hist_rows =
+        p.hist_head_stride > 0 ? (n_bg - 1) * p.hist_head_stride + (long long)p.n_hist_chunks * p.chunk
+                               : (long long)p.n_hist_chunks * p.chunk;
+    const unsigned long long seg_rows = (unsigned long long)((n_bg - 1) * p.seg_head_stride + p.seg_len);
+    if (!make_map(&mq, q, q_rows) || !make_map(&mdo, dout, q_rows) || !make_map(&mks, ks, seg_rows) ||
+        !make_map(&mvs, vs, seg_rows))
+        return HGA_ERR_INVALID_ARG;
+    if (hist_rows > 0) {
+        if (!make_map(&mkh, kh, (unsigned long long)hist_rows) || !make_map(&mvh, vh, (unsigned long long)hist_rows))
+            return HGA_ERR_INVALID_ARG;
+    } else {
+        mkh = mks;
+        mvh = mvs;
+    }
+    BwdArgs a;
+    a.batch = p.batch;
+    a.n_q_heads = p.n_q_heads;
+    a.n_kv_heads = p.n_kv_heads;
+    a.seg_len = p.seg_len;
+    a.topk = p.topk;
+    a.n_hist_chunks = p.n_hist_chunks;
+    a.hist_stride = p.hist_head_stride;
+    a.seg_stride = p.seg_head_stride;
+    a.idx = idx;
+    a.lse = lse;
+    a.delta = delta;
+    a.dq = dq;
+    a.dk = dk;
+    a.dv = dv;
+    a.status = status;
+    a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
+    a.scale = (float)(1.0 / __builtin_sqrt((double)D));
+    const int G = p.n_q_heads / p.n_kv_heads;
+    hga_status_t st = G == 4 ? launch_dq<2>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream)
+                             : launch_dq<1>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream);
+    if (st != HGA_OK) return st;
+    const size_t smem = DkvSmem::ALLOC;
+    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return record_cuda(e);
+    const unsigned grid = (unsigned)(((p.seg_len + 127) / 128) * n_bg);
+    bwd_dkdv_tc_kernel<<<grid, 256, smem, stream>>>(mq, mdo, mks, mvs, a);
+    return record_cuda(cudaGetLastError());
+}
+
+}  // namespace hga

@@ -444,6 +444,28 @@ static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, 
     return record_cuda(e);
 }
 
+hga_status_t launch_bwd_delta(const hga_params_t &p, const void *out, const void *dout, float *delta,
+                              cudaStream_t stream) {
+    const long long rows = (long long)p.batch * p.n_q_heads * p.seg_len;
+    const unsigned grid = (unsigned)((rows + 7) / 8);
+    if (p.dtype == HGA_BF16) {
+        if (p.head_dim == 128)
+            bwd_delta_kernel<__nv_bfloat16, 128><<<grid, 256, 0, stream>>>(
+                (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, delta, rows);
+        else
+            bwd_delta_kernel<__nv_bfloat16, 64><<<grid, 256, 0, stream>>>(
+                (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, delta, rows);
+    } else {
+        if (p.head_dim == 128)
+            bwd_delta_kernel<float, 128><<<grid, 256, 0, stream>>>((const float *)out, (const float *)dout, delta,
+                                                                   rows);
+        else
+            bwd_delta_kernel<float, 64><<<grid, 256, 0, stream>>>((const float *)out, (const float *)dout, delta,
+                                                                  rows);
+    }
+    return record_cuda(cudaGetLastError());
+}
+
 hga_status_t launch_attn_fwd_simt(const hga_params_t &p, const void *q, const void *kh, const void *vh,
                                   const void *ks, const void *vs, const int32_t *idx, void *out, float *lse,
                                   unsigned *status, cudaStream_t stream) {

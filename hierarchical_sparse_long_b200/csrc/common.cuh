@@ -63,6 +63,13 @@ hga_status_t launch_attn_bwd_simt(const hga_params_t &p, const void *q, const vo
                                   const int32_t *idx, const void *out, const float *lse, const void *dout,
                                   void *dq, void *dk_seg, void *dv_seg, float *delta, unsigned *status,
                                   cudaStream_t stream);
+hga_status_t launch_bwd_delta(const hga_params_t &p, const void *out, const void *dout, float *delta,
+                              cudaStream_t stream);
+bool attn_bwd_tc_supported(const hga_params_t &p);
+hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void *k_hist, const void *v_hist,
+                                const void *k_seg, const void *v_seg, const int32_t *idx, const float *lse,
+                                const float *delta, const void *dout, float *dq, float *dk, float *dv,
+                                unsigned *status, cudaStream_t stream);
 bool attn_fwd_tc_supported(const hga_params_t &p);
 hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *k_hist,
                                 const void *v_hist, const void *k_seg, const void *v_seg,
