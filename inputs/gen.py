@@ -215,3 +215,88 @@ def custom(name: str, **kw) -> Workload:
                 seg_len=256, seq_len=1280, seg_starts=(1024,), dtype="fp32", seed=0)
     base.update(kw)
     return Workload(name=name, **base)
+
+
+# ---------------------------------------------------------------------------
+# The same recipe drawn with torch (int64 arithmetic wraps modulo 2**64), so a
+# benchmark can draw long sequences directly on the GPU.  Logical right shifts
+# are arithmetic shifts with the sign-extended top bits masked off.  float64
+# log/cos may differ from numpy's in the last bit, which almost never survives
+# the rounding to float32/bf16.
+
+def _to_i64(u: int) -> int:
+    return u - (1 << 64) if u >= (1 << 63) else u
+
+
+_GAMMA_I = _to_i64(0x9E3779B97F4A7C15)
+_M1_I = _to_i64(0xBF58476D1CE4E5B9)
+_M2_I = _to_i64(0x94D049BB133111EB)
+
+
+def _shr(z, k: int):
+    return (z >> k) & ((1 << (64 - k)) - 1)
+
+
+def _mix_t(z):
+    z = z ^ _shr(z, 30)
+    z = z * _M1_I
+    z = z ^ _shr(z, 27)
+    z = z * _M2_I
+    return z ^ _shr(z, 31)
+
+
+def draw_torch(seed: int, tag: int, shape_full: tuple, t0: int, t1: int, device):
+    """torch (float64) version of ``draw`` for tokens [t0, t1) of axis 2."""
+    import torch
+    key = _to_i64(int(stream_key(seed, tag)))
+    dims = list(shape_full)
+    strides = [int(s) for s in np.cumprod([1] + dims[::-1][:-1])[::-1]]
+    ar = lambda n, s, ax: (torch.arange(n[0], n[1], device=device, dtype=torch.int64) * s).reshape(
+        [-1 if a == ax else 1 for a in range(len(dims))])
+    flat = ar((0, dims[0]), strides[0], 0) + ar((0, dims[1]), strides[1], 1) + ar((t0, t1), strides[2], 2) + \
+        ar((0, dims[3]), strides[3], 3)
+    n2 = flat * 2
+
+    def uni(n):
+        r = _mix_t(key + (n + 1) * _GAMMA_I)
+        return (_shr(r, 11).to(torch.float64) + 0.5) * (2.0 ** -53)
+    return torch.sqrt(-2.0 * torch.log(uni(n2))) * torch.cos(2.0 * np.pi * uni(n2 + 1))
+
+
+def _finish_t(x, dtype: str):
+    import torch
+    x32 = x.to(torch.float32)
+    return x32.to(torch.bfloat16) if dtype == "bf16" else x32
+
+
+def keys_torch(w: Workload, t0: int, t1: int, device):
+    c = w.chunk
+    nck = w.seq_len // c
+    parts = []
+    for a in range(t0, t1, PIECE):
+        b = min(a + PIECE, t1)
+        k = draw_torch(w.seed, TAG_K, (w.batch, w.n_kv_heads, w.seq_len, w.head_dim), a, b, device)
+        u = draw_torch(w.seed, TAG_OFFSET, (w.batch, w.n_kv_heads, nck, w.head_dim), a // c, b // c, device)
+        off = 2.0 * u / u.norm(dim=-1, keepdim=True)
+        parts.append(_finish_t(k + off.repeat_interleave(c, dim=2), w.dtype))
+    import torch
+    return torch.cat(parts, dim=2)
+
+
+def _plain_torch(w: Workload, tag: int, heads: int, t0: int, t1: int, device):
+    import torch
+    return torch.cat([_finish_t(draw_torch(w.seed, tag, (w.batch, heads, w.seq_len, w.head_dim), a,
+                                           min(a + PIECE, t1), device), w.dtype)
+                      for a in range(t0, t1, PIECE)], dim=2)
+
+
+def values_torch(w: Workload, t0: int, t1: int, device):
+    return _plain_torch(w, TAG_V, w.n_kv_heads, t0, t1, device)
+
+
+def queries_torch(w: Workload, t0: int, t1: int, device):
+    return _plain_torch(w, TAG_Q, w.n_q_heads, t0, t1, device)
+
+
+def grad_out_torch(w: Workload, t0: int, t1: int, device):
+    return _plain_torch(w, TAG_DO, w.n_q_heads, t0, t1, device)

@@ -357,3 +357,13 @@ def test_generator_slices_agree_and_offsets_have_norm_two():
 def test_generator_normal_moments():
     z = gen.normals(gen.stream_key(7, 1), np.arange(200000))
     assert abs(z.mean()) < 0.01 and abs(z.std() - 1.0) < 0.01
+
+
+def test_torch_generator_matches_numpy_recipe():
+    w = gen.custom("t", seq_len=512, seg_starts=(256,), dtype="bf16", head_dim=32, n_q_heads=4, n_kv_heads=2)
+    for fn_np, fn_t in ((gen.keys, gen.keys_torch), (gen.values, gen.values_torch),
+                        (gen.queries, gen.queries_torch)):
+        a = fn_np(w, 128, 384)
+        b = fn_t(w, 128, 384, "cpu").float().numpy()
+        mismatch = np.mean(a != b)
+        assert mismatch < 1e-3 and np.max(np.abs(a - b)) < 1e-2, (fn_np.__name__, mismatch)
