@@ -13,20 +13,25 @@
 // which is what lifts a history tile from 64 to 256 flop/byte.
 //
 // Warp roles (NH = 2: 384 threads):
-//   warp 0      TMA producer: Q once, then K/V tiles into a 3-stage ring
-//               (routed chunk j -> TMA row coordinate (b*Hkv+g)*stride + 64 j)
-//   warp 1      TMEM owner and single-thread UMMA issuer:
+//   warps 0, 2  TMA producers: Q once and the K tiles (warp 0), the V tiles
+//               (warp 2), each into its own 3-stage ring (routed chunk j ->
+//               TMA row coordinate (b*Hkv+g)*stride + 64 j); a K stage is
+//               released as soon as QK^T of its tile completes, a V stage
+//               after PV, so K loads run well ahead of the softmax.
+//   warps 1, 3  UMMA issuers, one thread per M half (warp 1 also owns TMEM):
 //               S_h = Q_h K^T   (M128 N64 K128, K-major A and B, SW128)
 //               O_h += P_h V    (M128 N128 K64, P K-major, V MN-major)
 //               QK^T of tile j is issued before PV of tile j-1 so the tensor
 //               core works while the softmax warps run.
 //   warps 4+4h  softmax of half h: one TMEM lane (= query row) per thread;
 //               online softmax in the log2 domain, O rescaled in TMEM when
-//               the row max grows, P written as bf16 in the SW128 K-major
-//               layout the next UMMA reads.
+//               the row max grows by more than 2^8, P written as bf16 in the
+//               SW128 K-major layout the next UMMA reads, into one of two
+//               buffers so tile j+1's softmax never waits for PV(j).
 // TMEM (512 columns): O_h at 128h, S_h double-buffered at 256 + 128h + 64b.
 // Every wait is bounded; a timeout sets HGA_DEV_TIMEOUT and the CTA unwinds.
 #include <cudaTypedefs.h>
+#include <cstdlib>
 #include <mutex>
 
 #include "tc_ptx.cuh"
@@ -41,33 +46,37 @@ constexpr int NSTAGE = 3;
 constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold on the running max (log2 units)
 constexpr uint32_t Q_HALF_BYTES = 128 * D * 2;   // 32 KiB: [2 col halves][128 rows][128 B]
 constexpr uint32_t KV_TILE_BYTES = TILE * D * 2; // 16 KiB: [2 col halves][64 rows][128 B]
-constexpr uint32_t P_BYTES = 128 * TILE * 2;     // 16 KiB: [128 rows][128 B]
+constexpr uint32_t P_BYTES = 128 * TILE * 2;     // 16 KiB: [128 rows][128 B] (one P buffer)
 constexpr uint32_t IDESC_QK = tc::idesc_bf16(128, TILE, false, false);
 constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, D, false, true);
 
 template <int NH>
 struct Smem {
     static constexpr uint32_t Q = 0;
-    static constexpr uint32_t KV = Q + NH * Q_HALF_BYTES;
-    static constexpr uint32_t P = KV + NSTAGE * 2 * KV_TILE_BYTES;
-    static constexpr uint32_t BAR = P + NH * P_BYTES;
+    static constexpr uint32_t K = Q + NH * Q_HALF_BYTES;      // K ring
+    static constexpr uint32_t V = K + NSTAGE * KV_TILE_BYTES; // V ring
+    static constexpr uint32_t P = V + NSTAGE * KV_TILE_BYTES;
+    static constexpr uint32_t BAR = P + NH * 2 * P_BYTES;  // P double-buffered per half
     static constexpr uint32_t TOTAL = BAR + 1024;  // barriers, tile list, flags
     static constexpr uint32_t ALLOC = TOTAL + 1024; // + alignment slack
 };
 
 struct Bars {
     uint64_t q_full;
-    uint64_t kv_full[NSTAGE];
-    uint64_t kv_empty[NSTAGE];
+    uint64_t k_full[NSTAGE];
+    uint64_t k_empty[NSTAGE];  // released once QK^T of the tile completes
+    uint64_t v_full[NSTAGE];
+    uint64_t v_empty[NSTAGE];  // released once PV of the tile completes
     uint64_t s_full[2][2];
     uint64_t s_free[2][2];
-    uint64_t p_full[2];
-    uint64_t o_done[2];
-    uint64_t drain;
+    uint64_t p_full[2][2];  // [half][P buffer]
+    uint64_t o_done[2][2];  // [half][P buffer of the PV that completed]
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
     int n_hist;
-    int issued;
+    int issued_k;
+    int issued_v;
     int tiles[64];
 };
 
@@ -82,7 +91,7 @@ struct FwdArgs {
     float scale_log2;  // log2(e) / sqrt(D)
 };
 
-template <int NH>
+template <int NH, int POLY>
 __global__ void __launch_bounds__(128 + 128 * NH, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                        const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
@@ -104,18 +113,25 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->q_full, 1);
         for (int s = 0; s < NSTAGE; ++s) {
-            tc::mbar_init(&bars->kv_full[s], 1);
-            tc::mbar_init(&bars->kv_empty[s], 1);
+            tc::mbar_init(&bars->k_full[s], 1);
+            tc::mbar_init(&bars->k_empty[s], NH);
+            tc::mbar_init(&bars->v_full[s], 1);
+            tc::mbar_init(&bars->v_empty[s], NH);
         }
+        bars->issued_k = 0;
+        bars->issued_v = 0;
         for (int h = 0; h < 2; ++h) {
             for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->s_full[h][bb], 1);
                 tc::mbar_init(&bars->s_free[h][bb], 4);
             }
-            tc::mbar_init(&bars->p_full[h], 4);
-            tc::mbar_init(&bars->o_done[h], 1);
+            for (int bb = 0; bb < 2; ++bb) {
+                tc::mbar_init(&bars->p_full[h][bb], 4);
+                tc::mbar_init(&bars->o_done[h][bb], 1);
+            }
         }
-        tc::mbar_init(&bars->drain, 1);
+        tc::mbar_init(&bars->drain[0], 1);
+        tc::mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         tc::fence_mbar_init();
     }
@@ -139,9 +155,34 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
     const int n_tiles = n_hist + m + 1;
     volatile int *abort = &bars->abort;
 
+    // TMA producer of one ring: K tiles (released after QK^T) or V tiles
+    // (released after PV); each routed chunk j is row (b*Hkv+g)*stride + 64 j.
+    auto produce = [&](bool key) {
+        const CUtensorMap *mh = key ? &tm_kh : &tm_vh;
+        const CUtensorMap *ms = key ? &tm_ks : &tm_vs;
+        uint64_t *full = key ? bars->k_full : bars->v_full;
+        uint64_t *empty = key ? bars->k_empty : bars->v_empty;
+        uint8_t *ring = smem + (key ? L::K : L::V);
+        int issued = 0;
+        for (int j = 0; j < n_tiles; ++j) {
+            const int s = j % NSTAGE, u = j / NSTAGE;
+            if (j >= NSTAGE && !tc::mbar_wait(&empty[s], (u - 1) & 1, abort, a.status)) break;
+            const bool hist = j < n_hist;
+            const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
+                                 : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+            uint8_t *dst = ring + s * KV_TILE_BYTES;
+            tc::mbar_arrive_expect_tx(&full[s], KV_TILE_BYTES);
+            tc::tma_load_2d(dst, hist ? mh : ms, 0, row, &full[s]);
+            tc::tma_load_2d(dst + 64 * 128, hist ? mh : ms, 64, row, &full[s]);
+            ++issued;
+        }
+        if (key) bars->issued_k = issued;
+        else bars->issued_v = issued;
+    };
+
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------------------------------------------------- TMA producer
+            // ---------------------------------------------------------- TMA producer (Q, K)
             tc::tma_prefetch_desc(&tm_q);
             tc::tma_prefetch_desc(&tm_kh);
             tc::tma_prefetch_desc(&tm_ks);
@@ -152,74 +193,60 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                 tc::tma_load_2d(dst, &tm_q, 0, qrow, &bars->q_full);
                 tc::tma_load_2d(dst + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
             }
-            int issued = 0;
-            for (int j = 0; j < n_tiles; ++j) {
-                const int s = j % NSTAGE, u = j / NSTAGE;
-                if (j >= NSTAGE && !tc::mbar_wait(&bars->kv_empty[s], (u - 1) & 1, abort, a.status)) break;
-                const bool hist = j < n_hist;
-                const CUtensorMap *mk = hist ? &tm_kh : &tm_ks;
-                const CUtensorMap *mv = hist ? &tm_vh : &tm_vs;
-                const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
-                                     : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
-                uint8_t *kdst = smem + L::KV + s * 2 * KV_TILE_BYTES;
-                uint8_t *vdst = kdst + KV_TILE_BYTES;
-                tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * KV_TILE_BYTES);
-                tc::tma_load_2d(kdst, mk, 0, row, &bars->kv_full[s]);
-                tc::tma_load_2d(kdst + 64 * 128, mk, 64, row, &bars->kv_full[s]);
-                tc::tma_load_2d(vdst, mv, 0, row, &bars->kv_full[s]);
-                tc::tma_load_2d(vdst + 64 * 128, mv, 64, row, &bars->kv_full[s]);
-                ++issued;
-            }
-            bars->issued = issued;
+            produce(true);
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
-            // ---------------------------------------------------------- UMMA issuer
-            const uint32_t q_base = sbase + L::Q;
-            const uint32_t p_base = sbase + L::P;
+    } else if (warp == 2) {
+        if (lane == 0) produce(false);  // V tiles, independent of the K ring
+    } else if (warp == 1 || warp == 3) {
+        // ------------------------------------------------------------ UMMA issuers
+        // One issuing thread per 128-row half (warp 1: half 0, warp 3: half 1):
+        // a single thread can only issue a tcgen05.mma every ~100 cycles, so the
+        // halves' MMAs are issued by two threads that the tensor core serves
+        // concurrently.
+        const int h = warp == 1 ? 0 : 1;
+        if (lane == 0 && h < NH) {
+            // Descriptors are built once; a K-step, stage or buffer offset is added
+            // to the start-address field (addresses stay below 2^18, so no carry).
+            const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * Q_HALF_BYTES, 16, 1024);
+            const uint64_t k_desc = tc::desc_sw128(sbase + L::K, 16, 1024);
+            const uint64_t v_desc = tc::desc_sw128(sbase + L::V, 8192, 1024);
+            const uint64_t p_desc = tc::desc_sw128(sbase + L::P + 2 * h * P_BYTES, 16, 1024);
+            const uint32_t o_tmem = tmem + 128 * h;
+            // O_h += P_h(t) V(t) once the softmax of tile t has written P buffer t&1
             auto issue_pv = [&](int t) -> bool {
-                const int s = t % NSTAGE;
-                const uint32_t v_base = sbase + L::KV + s * 2 * KV_TILE_BYTES + KV_TILE_BYTES;
-                for (int h = 0; h < NH; ++h) {
-                    if (!tc::mbar_wait(&bars->p_full[h], t & 1, abort, a.status)) return false;
-                    tc::fence_after_sync();
-                    const uint32_t d = tmem + 128 * h;
+                const int s = t % NSTAGE, pb = t & 1;
+                if (!tc::mbar_wait(&bars->v_full[s], (t / NSTAGE) & 1, abort, a.status)) return false;
+                if (!tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort, a.status)) return false;
+                tc::fence_after_sync();
+                const uint64_t vd = v_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
+                const uint64_t pd = p_desc + (uint64_t)((pb * P_BYTES) >> 4);
 #pragma unroll
-                    for (int kk = 0; kk < TILE / 16; ++kk) {
-                        const uint64_t adesc = tc::desc_sw128(p_base + h * P_BYTES + kk * 32, 16, 1024);
-                        const uint64_t bdesc = tc::desc_sw128(v_base + kk * 2048, 8192, 1024);
-                        tc::mma_f16(d, adesc, bdesc, IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-                    }
-                    tc::mma_commit(&bars->o_done[h]);
-                }
-                tc::mma_commit(&bars->kv_empty[s]);
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    tc::mma_f16(o_tmem, pd + (kk * 32 >> 4), vd + (kk * 2048 >> 4), IDESC_PV,
+                                (t > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&bars->o_done[h][pb]);
+                tc::mma_commit(&bars->v_empty[s]);  // one arrival per half
                 return true;
             };
             bool ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
             for (int j = 0; ok && j < n_tiles; ++j) {
-                const int s = j % NSTAGE;
-                if (!tc::mbar_wait(&bars->kv_full[s], (j / NSTAGE) & 1, abort, a.status)) { ok = false; break; }
-                tc::fence_after_sync();
-                const uint32_t k_base = sbase + L::KV + s * 2 * KV_TILE_BYTES;
-                const int bb = j & 1;
-                for (int h = 0; h < NH; ++h) {
-                    if (j >= 2 && !tc::mbar_wait(&bars->s_free[h][bb], ((j >> 1) - 1) & 1, abort, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
-                    const uint32_t d = tmem + 256 + 128 * h + 64 * bb;
-#pragma unroll
-                    for (int kk = 0; kk < D / 16; ++kk) {
-                        const uint32_t kb = (kk & 3) * 32;
-                        const uint64_t adesc =
-                            tc::desc_sw128(q_base + h * Q_HALF_BYTES + (kk >> 2) * (128 * 128) + kb, 16, 1024);
-                        const uint64_t bdesc = tc::desc_sw128(k_base + (kk >> 2) * (64 * 128) + kb, 16, 1024);
-                        tc::mma_f16(d, adesc, bdesc, IDESC_QK, kk > 0 ? 1u : 0u);
-                    }
-                    tc::mma_commit(&bars->s_full[h][bb]);
+                const int s = j % NSTAGE, bb = j & 1;
+                if (!tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)) { ok = false; break; }
+                if (j >= 2 && !tc::mbar_wait(&bars->s_free[h][bb], ((j >> 1) - 1) & 1, abort, a.status)) {
+                    ok = false;
+                    break;
                 }
-                if (!ok) break;
+                tc::fence_after_sync();
+                const uint64_t kd = k_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t koff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+                    const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                    tc::mma_f16(tmem + 256 + 128 * h + 64 * bb, q_desc + qoff, kd + koff, IDESC_QK,
+                                kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&bars->s_full[h][bb]);
+                tc::mma_commit(&bars->k_empty[s]);  // one arrival per half
                 if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
             }
             if (ok) issue_pv(n_tiles - 1);
@@ -233,7 +260,7 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         const int i = r & 63;                 // query row within the block
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const uint32_t o_addr = tmem + lane_addr + 128 * h;
-        const uint32_t p_row = sbase + L::P + h * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t p_rows = sbase + L::P + 2 * h * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
@@ -257,17 +284,21 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->s_free[h][bb]);
             float x[64];
-            const bool diag = (j == n_tiles - 1);  // the local tile of this block
+            const bool diag = (j == n_tiles - 1);  // the local tile of this block (warp-uniform)
+#pragma unroll
+            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (c > i) x[c] = -INFINITY;
+            }
+            // row max of the raw scores (the scale is positive), 8 independent chains
             float mpart[8];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                float v = __uint_as_float(sr[c]) * a.scale_log2;
-                if (diag && c > i) v = -INFINITY;
-                x[c] = v;
-                mpart[c & 7] = (c < 8) ? v : fmaxf(mpart[c & 7], v);
-            }
+            for (int c = 0; c < 64; ++c) mpart[c & 7] = (c < 8) ? x[c] : fmaxf(mpart[c & 7], x[c]);
             const float mx = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
-                                   fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7])));
+                                   fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7]))) *
+                             a.scale_log2;
             // Lazy rescaling: the reference max only moves when the row max grows by
             // more than kRescaleLog2, so P stays <= 2^kRescaleLog2 and O is rescaled
             // in TMEM only on those (rare) tiles.
@@ -277,34 +308,49 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             float spart[8];
 #pragma unroll
             for (int c = 0; c < 64; ++c) {
-                x[c] = tc::ex2(x[c] - m_use);
+                // p = 2^(s * log2(e)/sqrt(D) - m); a share of them on the FMA pipe
+                const float arg = fmaf(x[c], a.scale_log2, -m_use);
+                const bool poly = (POLY == 1 && (c & 3) == 3) || (POLY == 2 && (c & 1));
+                x[c] = poly ? tc::ex2_poly(arg) : tc::ex2(arg);
                 spart[c & 7] = (c < 8) ? x[c] : spart[c & 7] + x[c];
+            }
+            if (POLY != 0 && diag) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (c > i) x[c] = 0.f;  // the cubic maps -inf to ~2^-125, not 0
             }
             const float sum = ((spart[0] + spart[1]) + (spart[2] + spart[3])) +
                               ((spart[4] + spart[5]) + (spart[6] + spart[7]));
             l_run = l_run * alpha + sum;
-            // PV of the previous tile must be done before P is overwritten and O rescaled
-            if (j >= 1) {
-                if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h], (j - 1) & 1, abort, a.status))) {
+            const int pb = j & 1;
+            // P buffer pb was last read by PV(j-2)
+            if (j >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][pb], ((j >> 1) - 1) & 1, abort,
+                                                                  a.status))) {
+                ok = false;
+                break;
+            }
+            // a rescale needs O complete up to tile j-1 (PV(j-1) done) before PV(j) adds to it;
+            // rows that keep their reference max have alpha == 1, an exact no-op
+            if (j >= 1 && __any_sync(0xffffffffu, grow)) {
+                if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][pb ^ 1], ((j - 1) >> 1) & 1, abort,
+                                                            a.status))) {
                     ok = false;
                     break;
                 }
                 tc::fence_after_sync();
-                // rows that keep their reference max have alpha == 1: an exact no-op
-                if (__any_sync(0xffffffffu, grow)) {
 #pragma unroll 1
-                    for (int c0 = 0; c0 < D; c0 += 32) {
-                        uint32_t o[32];
-                        tc::tmem_ld32(o_addr + c0, o);
-                        tc::tmem_wait_ld();
+                for (int c0 = 0; c0 < D; c0 += 32) {
+                    uint32_t o[32];
+                    tc::tmem_ld32(o_addr + c0, o);
+                    tc::tmem_wait_ld();
 #pragma unroll
-                        for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
-                        tc::tmem_st32(o_addr + c0, o);
-                    }
-                    tc::tmem_wait_st();
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                    tc::tmem_st32(o_addr + c0, o);
                 }
+                tc::tmem_wait_st();
             }
             m_run = m_use;
+            const uint32_t p_row = p_rows + pb * P_BYTES;
 #pragma unroll
             for (int cc = 0; cc < 8; ++cc) {
                 const uint32_t addr = p_row + ((cc ^ (r & 7)) << 4);
@@ -316,9 +362,10 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->p_full[h]);
+            if (lane == 0) tc::mbar_arrive(&bars->p_full[h][pb]);
         }
-        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h], (n_tiles - 1) & 1, abort, a.status))) {
+        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][(n_tiles - 1) & 1],
+                                                        ((n_tiles - 1) >> 1) & 1, abort, a.status))) {
             tc::fence_after_sync();
             const long long row = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + m * TILE + i;
             __nv_bfloat16 *orow = a.out + row * D;
@@ -348,15 +395,17 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         // a wait gave up: let the copies and UMMAs still in flight finish before
         // shared memory and TMEM are released
         int never = 0;
-        if (warp == 0 && lane == 0) {
-            const int issued = bars->issued;
+        if ((warp == 0 || warp == 2) && lane == 0) {
+            const bool key = warp == 0;
+            const int issued = key ? bars->issued_k : bars->issued_v;
+            uint64_t *full = key ? bars->k_full : bars->v_full;
             for (int j = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; j < issued; ++j)
-                tc::mbar_wait(&bars->kv_full[j % NSTAGE], (j / NSTAGE) & 1, &never, a.status, 1ll << 28);
-            tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
+                tc::mbar_wait(&full[j % NSTAGE], (j / NSTAGE) & 1, &never, a.status, 1ll << 28);
+            if (key) tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
         }
-        if (warp == 1 && lane == 0) {
-            tc::mma_commit(&bars->drain);
-            tc::mbar_wait(&bars->drain, 0, &never, a.status, 1ll << 28);
+        if ((warp == 1 || (warp == 3 && NH == 2)) && lane == 0) {
+            tc::mma_commit(&bars->drain[warp == 3]);
+            tc::mbar_wait(&bars->drain[warp == 3], 0, &never, a.status, 1ll << 28);
         }
         __syncwarp();
         tc::fence_after_sync();
@@ -432,7 +481,12 @@ hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, con
     a.status = status;
     a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
     const size_t smem = Smem<NH>::ALLOC;
-    auto kern = attn_fwd_tc_kernel<NH>;
+    static const int poly = [] {
+        const char *e = getenv("HGA_FWD_EXP2_POLY");
+        return e ? atoi(e) : 0;
+    }();
+    auto kern = poly == 2 ? attn_fwd_tc_kernel<NH, 2> : poly == 0 ? attn_fwd_tc_kernel<NH, 0>
+                                                                   : attn_fwd_tc_kernel<NH, 1>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const unsigned grid = (unsigned)(a.n_blocks * n_bg);
