@@ -20,8 +20,10 @@
 //                every head of the group: S^T = K Q^T and dP^T = V dO^T
 //                (M128 N64 K128), P^T and dS^T in bf16 into shared memory,
 //                dV += P^T dO and dK += dS^T Q (M128 N128 K64).
-// Warp 0 issues TMA loads, warp 1 owns TMEM and issues the UMMAs from one
-// thread, the remaining warpgroups handle one TMEM lane (row) per thread.
+// Warp 0 issues TMA loads, warps 1 and 3 issue the UMMAs (one thread each:
+// a single thread can issue a tcgen05.mma only every ~100 cycles), warp 1
+// owns TMEM, and the remaining warpgroups handle one TMEM lane (row) per
+// thread.
 // Every wait is bounded and every warp-collective TMEM access is made from a
 // converged warp with warp-uniform decisions.
 #include <cudaTypedefs.h>
@@ -55,29 +57,6 @@ struct BwdArgs {
     float scale;       // 1 / sqrt(D)
 };
 
-// S = A B^T over D = 128 (K-major A rows at a_base with 128-row halves, K-major
-// 64-row B tile at b_base): 8 UMMA steps of K = 16.
-__device__ __forceinline__ void mma_rows_x_tile(uint32_t d, uint32_t a_base, uint32_t b_base) {
-#pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const uint32_t kb = (kk & 3) * 32;
-        const uint64_t adesc = tc::desc_sw128(a_base + (kk >> 2) * (128 * 128) + kb, 16, 1024);
-        const uint64_t bdesc = tc::desc_sw128(b_base + (kk >> 2) * (64 * 128) + kb, 16, 1024);
-        tc::mma_f16(d, adesc, bdesc, IDESC_N64, kk > 0 ? 1u : 0u);
-    }
-}
-
-// D(+)= A B with A = 128 rows x 64 (K-major, bf16 written by the threads) and
-// B = a 64-row tile read MN-major (N = D = 128): 4 UMMA steps of K = 16.
-__device__ __forceinline__ void mma_k64_x_tile(uint32_t d, uint32_t a_base, uint32_t b_base, bool accumulate) {
-#pragma unroll
-    for (int kk = 0; kk < TILE / 16; ++kk) {
-        const uint64_t adesc = tc::desc_sw128(a_base + kk * 32, 16, 1024);
-        const uint64_t bdesc = tc::desc_sw128(b_base + kk * 2048, 8192, 1024);
-        tc::mma_f16(d, adesc, bdesc, IDESC_N128_BMN, (accumulate || kk > 0) ? 1u : 0u);
-    }
-}
-
 // Writes 32 packed bf16 pairs (64 values) of row r as a 128-byte SW128 row.
 __device__ __forceinline__ void store_row_sw128(uint32_t row_addr, int r, const uint32_t (&pk)[32]) {
 #pragma unroll
@@ -106,7 +85,7 @@ struct DqBars {
     uint64_t sdp_free[2];
     uint64_t ds_full[2];
     uint64_t dq_done[2];
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
     int n_hist;
@@ -138,7 +117,7 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         tc::mbar_init(&bars->q_full, 1);
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(&bars->kv_full[s], 1);
-            tc::mbar_init(&bars->kv_empty[s], 1);
+            tc::mbar_init(&bars->kv_empty[s], NH);
         }
         for (int h = 0; h < 2; ++h) {
             tc::mbar_init(&bars->sdp_full[h], 1);
@@ -146,7 +125,8 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             tc::mbar_init(&bars->ds_full[h], 4);
             tc::mbar_init(&bars->dq_done[h], 1);
         }
-        tc::mbar_init(&bars->drain, 1);
+        tc::mbar_init(&bars->drain[0], 1);
+        tc::mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         bars->issued = 0;
         tc::fence_mbar_init();
@@ -200,37 +180,45 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             }
             bars->issued = issued;
         }
-    } else if (warp == 1) {
-        if (lane == 0) {
+    } else if (warp == 1 || warp == 3) {
+        // one UMMA issuing thread per 128-row half (a thread issues one MMA per ~100 cycles)
+        const int h = warp == 1 ? 0 : 1;
+        if (lane == 0 && h < NH) {
+            const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * HALF_BYTES, 16, 1024);
+            const uint64_t do_desc = tc::desc_sw128(sbase + L::DO + h * HALF_BYTES, 16, 1024);
+            const uint64_t kv_desc = tc::desc_sw128(sbase + L::KV, 16, 1024);
+            const uint64_t kmn_desc = tc::desc_sw128(sbase + L::KV, 8192, 1024);
+            const uint64_t ds_desc = tc::desc_sw128(sbase + L::DS + h * ROWS128_K64, 16, 1024);
             auto issue_dq = [&](int t) -> bool {
                 const int s = t % NST;
-                const uint32_t k_base = sbase + L::KV + s * 2 * TILE_BYTES;
-                for (int h = 0; h < NH; ++h) {
-                    if (!tc::mbar_wait(&bars->ds_full[h], t & 1, abort, a.status)) return false;
-                    tc::fence_after_sync();
-                    mma_k64_x_tile(tmem + 128 * h, sbase + L::DS + h * ROWS128_K64, k_base, t > 0);
-                    tc::mma_commit(&bars->dq_done[h]);
-                }
-                tc::mma_commit(&bars->kv_empty[s]);
+                if (!tc::mbar_wait(&bars->ds_full[h], t & 1, abort, a.status)) return false;
+                tc::fence_after_sync();
+                const uint64_t kd = kmn_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    tc::mma_f16(tmem + 128 * h, ds_desc + (kk * 32 >> 4), kd + (kk * 2048 >> 4), IDESC_N128_BMN,
+                                (t > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&bars->dq_done[h]);
+                tc::mma_commit(&bars->kv_empty[s]);  // one arrival per half
                 return true;
             };
             bool ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % NST;
                 if (!tc::mbar_wait(&bars->kv_full[s], (j / NST) & 1, abort, a.status)) { ok = false; break; }
+                if (j >= 1 && !tc::mbar_wait(&bars->sdp_free[h], (j - 1) & 1, abort, a.status)) { ok = false; break; }
                 tc::fence_after_sync();
-                const uint32_t k_base = sbase + L::KV + s * 2 * TILE_BYTES;
-                for (int h = 0; h < NH; ++h) {
-                    if (j >= 1 && !tc::mbar_wait(&bars->sdp_free[h], (j - 1) & 1, abort, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    tc::fence_after_sync();
-                    mma_rows_x_tile(tmem + 256 + 128 * h, sbase + L::Q + h * HALF_BYTES, k_base);
-                    mma_rows_x_tile(tmem + 256 + 128 * h + 64, sbase + L::DO + h * HALF_BYTES, k_base + TILE_BYTES);
-                    tc::mma_commit(&bars->sdp_full[h]);
+                const uint64_t kd = kv_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
+                const uint64_t vd = kd + (uint64_t)(TILE_BYTES >> 4);
+                // S = Q K^T and dP = dO V^T: two independent accumulators, interleaved
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                    const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+                    tc::mma_f16(tmem + 256 + 128 * h, q_desc + aoff, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                    tc::mma_f16(tmem + 256 + 128 * h + 64, do_desc + aoff, vd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
                 }
-                if (!ok) break;
+                tc::mma_commit(&bars->sdp_full[h]);
                 if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
             }
             if (ok) issue_dq(n_tiles - 1);
@@ -313,9 +301,9 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                 tc::mbar_wait(&bars->kv_full[j % NST], (j / NST) & 1, &never, a.status, 1ll << 28);
             tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
         }
-        if (warp == 1 && lane == 0) {
-            tc::mma_commit(&bars->drain);
-            tc::mbar_wait(&bars->drain, 0, &never, a.status, 1ll << 28);
+        if ((warp == 1 || (warp == 3 && NH == 2)) && lane == 0) {
+            tc::mma_commit(&bars->drain[warp == 3]);
+            tc::mbar_wait(&bars->drain[warp == 3], 0, &never, a.status, 1ll << 28);
         }
         __syncwarp();
         tc::fence_after_sync();
@@ -348,7 +336,7 @@ struct DkvBars {
     uint64_t sdp_free[2];
     uint64_t pds_full;
     uint64_t pds_free;
-    uint64_t drain;
+    uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
     int issued;
@@ -379,15 +367,16 @@ __global__ void __launch_bounds__(256, 1)
         tc::mbar_init(&bars->kv_full, 1);
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(&bars->ring_full[s], 1);
-            tc::mbar_init(&bars->ring_empty[s], 1);
+            tc::mbar_init(&bars->ring_empty[s], 2);
         }
         for (int bb = 0; bb < 2; ++bb) {
-            tc::mbar_init(&bars->sdp_full[bb], 1);
+            tc::mbar_init(&bars->sdp_full[bb], 2);  // S^T and dP^T issuers
             tc::mbar_init(&bars->sdp_free[bb], 4);
         }
         tc::mbar_init(&bars->pds_full, 4);
-        tc::mbar_init(&bars->pds_free, 1);
-        tc::mbar_init(&bars->drain, 1);
+        tc::mbar_init(&bars->pds_free, 2);  // dV and dK issuers
+        tc::mbar_init(&bars->drain[0], 1);
+        tc::mbar_init(&bars->drain[1], 1);
         bars->abort = 0;
         bars->issued = 0;
         tc::fence_mbar_init();
@@ -430,17 +419,30 @@ __global__ void __launch_bounds__(256, 1)
             }
             bars->issued = issued;
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || warp == 3) {
+        // two UMMA issuing threads (a thread issues one MMA per ~100 cycles):
+        // warp 1 issues S^T = K Q^T and dV += P^T dO, warp 3 dP^T = V dO^T and dK += dS^T Q
+        const bool first = warp == 1;
         if (lane == 0) {
+            const uint64_t kv_desc = tc::desc_sw128(sbase + (first ? L::K : L::V), 16, 1024);
+            const uint64_t ring_desc = tc::desc_sw128(sbase + L::RING, 16, 1024);
+            const uint64_t ring_mn_desc = tc::desc_sw128(sbase + L::RING, 8192, 1024);
+            const uint64_t a_desc = tc::desc_sw128(sbase + (first ? L::PT : L::DST), 16, 1024);
+            // stage operand of each issuer: Q tile for S^T / dK, dO tile for dP^T / dV
+            const uint32_t s_op = first ? 0u : TILE_BYTES;     // S^T uses Q, dP^T uses dO
+            const uint32_t g_op = first ? TILE_BYTES : 0u;     // dV uses dO, dK uses Q
+            const uint32_t acc = first ? 0u : 128u;            // dV at 0, dK at 128
             auto issue_grads = [&](int t) -> bool {
                 const int s = t % NST;
                 if (!tc::mbar_wait(&bars->pds_full, t & 1, abort, a.status)) return false;
                 tc::fence_after_sync();
-                const uint32_t q_base = sbase + L::RING + s * L::STAGE_BYTES;
-                mma_k64_x_tile(tmem, sbase + L::PT, q_base + TILE_BYTES, t > 0);   // dV += P^T dO
-                mma_k64_x_tile(tmem + 128, sbase + L::DST, q_base, t > 0);         // dK += dS^T Q
-                tc::mma_commit(&bars->pds_free);
-                tc::mma_commit(&bars->ring_empty[s]);
+                const uint64_t bd = ring_mn_desc + (uint64_t)((s * L::STAGE_BYTES + g_op) >> 4);
+#pragma unroll
+                for (int kk = 0; kk < TILE / 16; ++kk)
+                    tc::mma_f16(tmem + acc, a_desc + (kk * 32 >> 4), bd + (kk * 2048 >> 4), IDESC_N128_BMN,
+                                (t > 0 || kk > 0) ? 1u : 0u);
+                tc::mma_commit(&bars->pds_free);       // one arrival per issuer
+                tc::mma_commit(&bars->ring_empty[s]);  // one arrival per issuer
                 return true;
             };
             bool ok = tc::mbar_wait(&bars->kv_full, 0, abort, a.status);
@@ -452,10 +454,15 @@ __global__ void __launch_bounds__(256, 1)
                     break;
                 }
                 tc::fence_after_sync();
-                const uint32_t q_base = sbase + L::RING + s * L::STAGE_BYTES;
-                mma_rows_x_tile(tmem + 256 + 128 * bb, sbase + L::K, q_base);                   // S^T
-                mma_rows_x_tile(tmem + 256 + 128 * bb + 64, sbase + L::V, q_base + TILE_BYTES); // dP^T
-                tc::mma_commit(&bars->sdp_full[bb]);
+                const uint64_t bd = ring_desc + (uint64_t)((s * L::STAGE_BYTES + s_op) >> 4);
+                const uint32_t d = tmem + 256 + 128 * bb + (first ? 0u : 64u);
+#pragma unroll
+                for (int kk = 0; kk < D / 16; ++kk) {
+                    const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                    const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+                    tc::mma_f16(d, kv_desc + aoff, bd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                }
+                tc::mma_commit(&bars->sdp_full[bb]);  // one arrival per issuer
                 if (t >= 1 && !issue_grads(t - 1)) { ok = false; break; }
             }
             if (ok && n_steps > 0) issue_grads(n_steps - 1);
@@ -553,9 +560,9 @@ __global__ void __launch_bounds__(256, 1)
                 tc::mbar_wait(&bars->ring_full[t % NST], (t / NST) & 1, &never, a.status, 1ll << 28);
             tc::mbar_wait(&bars->kv_full, 0, &never, a.status, 1ll << 28);
         }
-        if (warp == 1 && lane == 0) {
-            tc::mma_commit(&bars->drain);
-            tc::mbar_wait(&bars->drain, 0, &never, a.status, 1ll << 28);
+        if ((warp == 1 || warp == 3) && lane == 0) {
+            tc::mma_commit(&bars->drain[warp == 3]);
+            tc::mbar_wait(&bars->drain[warp == 3], 0, &never, a.status, 1ll << 28);
         }
         __syncwarp();
         tc::fence_after_sync();
