@@ -10,12 +10,12 @@
 //   dQ = dS K / sqrt(D)                      over routed history and segment keys
 //   dK_seg = dS^T Q / sqrt(D), dV_seg = P^T dO   over segment keys only
 //
-// Two kernels, no atomics (results are deterministic):
-//   bwd_dq_tc  : query-major, one CTA per (batch, kv head, query block) holding
+// Two block types in one launch, no atomics (results are deterministic):
+//   dQ blocks  : query-major, one CTA per (batch, kv head, query block) holding
 //                the G heads of the group as M=128 halves (like the forward);
 //                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128), the
 //                dS rows in bf16 into shared memory, dQ += dS K (M128 N128 K64).
-//   bwd_dkdv_tc: key-major over the active segment, one CTA per (batch, kv
+//   dK/dV blocks: key-major over the active segment, one CTA per (batch, kv
 //                head, 128 segment keys); for every later 64-query tile of
 //                every head of the group: S^T = K Q^T and dP^T = V dO^T
 //                (M128 N64 K128), P^T and dS^T in bf16 into shared memory,
@@ -94,14 +94,11 @@ struct DqBars {
 };
 
 template <int NH>
-__global__ void __launch_bounds__(128 + 128 * NH, 1)
-    bwd_dq_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                     const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
-                     const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
-                     const BwdArgs a) {
+__device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_q,
+                                        const CUtensorMap &tm_do, const CUtensorMap &tm_kh, const CUtensorMap &tm_vh,
+                                        const CUtensorMap &tm_ks, const CUtensorMap &tm_vs, const BwdArgs &a) {
     using L = DqSmem<NH>;
     constexpr int NST = L::NSTAGE;
-    extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     DqBars *bars = reinterpret_cast<DqBars *>(smem + L::BAR);
     const uint32_t sbase = tc::smem_u32(smem);
@@ -109,8 +106,8 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
     const int G = 2 * NH;
     const int nqb = a.seg_len / TILE;
     const int n_bg = a.batch * a.n_kv_heads;
-    const int m = nqb - 1 - (int)blockIdx.x / n_bg;
-    const int bg = (int)blockIdx.x % n_bg;
+    const int m = nqb - 1 - blk / n_bg;
+    const int bg = blk % n_bg;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
 
     if (threadIdx.x == 0) {
@@ -342,13 +339,11 @@ struct DkvBars {
     int issued;
 };
 
-__global__ void __launch_bounds__(256, 1)
-    bwd_dkdv_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
-                       const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
-                       const BwdArgs a) {
+__device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_q,
+                                          const CUtensorMap &tm_do, const CUtensorMap &tm_ks,
+                                          const CUtensorMap &tm_vs, const BwdArgs &a) {
     using L = DkvSmem;
     constexpr int NST = L::NSTAGE;
-    extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     DkvBars *bars = reinterpret_cast<DkvBars *>(smem + L::BAR);
     const uint32_t sbase = tc::smem_u32(smem);
@@ -356,8 +351,8 @@ __global__ void __launch_bounds__(256, 1)
     const int G = a.n_q_heads / a.n_kv_heads;
     const int nqb = a.seg_len / TILE;
     const int n_bg = a.batch * a.n_kv_heads;
-    const int n = (int)blockIdx.x / n_bg;  // 128-key tile, earliest (most work) first
-    const int bg = (int)blockIdx.x % n_bg;
+    const int n = blk / n_bg;  // 128-key tile, earliest (most work) first
+    const int bg = blk % n_bg;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
     const int key0 = 128 * n;
     const int m0 = key0 / TILE;
@@ -467,7 +462,7 @@ __global__ void __launch_bounds__(256, 1)
             }
             if (ok && n_steps > 0) issue_grads(n_steps - 1);
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         const int quad = warp & 3;
         const int r = quad * 32 + lane;  // key row = TMEM lane
         const int key = key0 + r;
@@ -478,9 +473,12 @@ __global__ void __launch_bounds__(256, 1)
         for (int t = 0; t < n_steps; ++t) {
             const int s = t % NST, bb = t & 1;
             const int mq = m0 + t % (nqb - m0);
-            // the stage's lse / delta rows (TMA-written) and this step's S^T, dP^T in TMEM
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status) &&
-                                             tc::mbar_wait(&bars->sdp_full[bb], (t >> 1) & 1, abort, a.status))) {
+            // the stage's lse / delta rows (TMA-written), this step's S^T, dP^T in TMEM,
+            // and the P^T / dS^T buffers free again (the previous step's dV, dK done)
+            if (!__all_sync(0xffffffffu,
+                            tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status) &&
+                                tc::mbar_wait(&bars->sdp_full[bb], (t >> 1) & 1, abort, a.status) &&
+                                (t == 0 || tc::mbar_wait(&bars->pds_free, (t - 1) & 1, abort, a.status)))) {
                 ok = false;
                 break;
             }
@@ -488,7 +486,6 @@ __global__ void __launch_bounds__(256, 1)
             const float *lse2 = reinterpret_cast<const float *>(smem + L::ROWT + s * 512);
             const float *dlt = lse2 + 64;
             const int q0 = mq * TILE;  // first query position of the tile
-            uint32_t ppk[32], dpk[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t sv[32], dpv[32];
@@ -496,6 +493,7 @@ __global__ void __launch_bounds__(256, 1)
                 tc::tmem_ld32(s_addr, sv);
                 tc::tmem_ld32(s_addr + 64, dpv);
                 tc::tmem_wait_ld();
+                uint32_t ppk[16], dpk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const int c0 = 32 * half + c;
@@ -503,24 +501,26 @@ __global__ void __launch_bounds__(256, 1)
                     float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2[c0 + 1] * 1.4426950408889634f);
                     if (key > q0 + c0) p0 = 0.f;      // causal: the key comes after the query
                     if (key > q0 + c0 + 1) p1 = 0.f;
-                    ppk[16 * half + c / 2] = tc::pack_bf16(p0, p1);
-                    dpk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
-                                                           p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
+                    ppk[c / 2] = tc::pack_bf16(p0, p1);
+                    dpk[c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
+                                               p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
+                }
+#pragma unroll
+                for (int cc = 0; cc < 4; ++cc) {
+                    const int chunk = 4 * half + cc;
+                    tc::st_shared_v4(pt_row + ((chunk ^ (r & 7)) << 4), ppk[4 * cc], ppk[4 * cc + 1], ppk[4 * cc + 2],
+                                     ppk[4 * cc + 3]);
+                    tc::st_shared_v4(dst_row + ((chunk ^ (r & 7)) << 4), dpk[4 * cc], dpk[4 * cc + 1],
+                                     dpk[4 * cc + 2], dpk[4 * cc + 3]);
                 }
             }
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[bb]);
-            if (t >= 1 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->pds_free, (t - 1) & 1, abort, a.status))) {
-                ok = false;
-                break;
-            }
-            store_row_sw128(pt_row, r, ppk);
-            store_row_sw128(dst_row, r, dpk);
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->pds_full);
+            if (lane == 0) {
+                tc::mbar_arrive(&bars->sdp_free[bb]);
+                tc::mbar_arrive(&bars->pds_full);
+            }
         }
         const bool done = ok && (n_steps == 0 ||
                                  __all_sync(0xffffffffu, tc::mbar_wait(&bars->pds_free, (n_steps - 1) & 1, abort,
@@ -598,16 +598,35 @@ bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// One launch for both gradient passes: the first n_kv_ctas blocks run the
+// key-major dK/dV body (most work first), the rest the query-major dQ body.
+// The causal dK/dV blocks are very uneven (the first key tile is seen by
+// every later query tile), so the dQ blocks fill the SMs around them.
 template <int NH>
-hga_status_t launch_dq(const hga_params_t &p, const CUtensorMap &mq, const CUtensorMap &mdo,
-                       const CUtensorMap &mkh, const CUtensorMap &mvh, const CUtensorMap &mks,
-                       const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
-    auto kern = bwd_dq_tc_kernel<NH>;
-    const size_t smem = DqSmem<NH>::ALLOC;
+__global__ void __launch_bounds__(128 + 128 * NH, 1)
+    bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
+                  const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
+                  const BwdArgs a, const int n_kv_ctas) {
+    extern __shared__ uint8_t smem_raw[];
+    if ((int)blockIdx.x < n_kv_ctas)
+        dkdv_body((int)blockIdx.x, smem_raw, tm_q, tm_do, tm_ks, tm_vs, a);
+    else
+        dq_body<NH>((int)blockIdx.x - n_kv_ctas, smem_raw, tm_q, tm_do, tm_kh, tm_vh, tm_ks, tm_vs, a);
+}
+
+template <int NH>
+hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUtensorMap &mdo,
+                        const CUtensorMap &mkh, const CUtensorMap &mvh, const CUtensorMap &mks,
+                        const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
+    auto kern = bwd_tc_kernel<NH>;
+    const size_t smem = DqSmem<NH>::ALLOC > DkvSmem::ALLOC ? DqSmem<NH>::ALLOC : DkvSmem::ALLOC;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
-    const unsigned grid = (unsigned)((p.seg_len / p.q_block) * p.batch * p.n_kv_heads);
-    kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mdo, mkh, mvh, mks, mvs, a);
+    const int n_bg = p.batch * p.n_kv_heads;
+    const int n_kv_ctas = ((p.seg_len + 127) / 128) * n_bg;
+    const unsigned grid = (unsigned)(n_kv_ctas + (p.seg_len / p.q_block) * n_bg);
+    kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mdo, mkh, mvh, mks, mvs, a, n_kv_ctas);
     return record_cuda(cudaGetLastError());
 }
 
@@ -664,15 +683,8 @@ hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void
     a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
     a.scale = (float)(1.0 / __builtin_sqrt((double)D));
     const int G = p.n_q_heads / p.n_kv_heads;
-    hga_status_t st = G == 4 ? launch_dq<2>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream)
-                             : launch_dq<1>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream);
-    if (st != HGA_OK) return st;
-    const size_t smem = DkvSmem::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(bwd_dkdv_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return record_cuda(e);
-    const unsigned grid = (unsigned)(((p.seg_len + 127) / 128) * n_bg);
-    bwd_dkdv_tc_kernel<<<grid, 256, smem, stream>>>(mq, mdo, mks, mvs, a);
-    return record_cuda(cudaGetLastError());
+    return G == 4 ? launch_bwd<2>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream)
+                  : launch_bwd<1>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream);
 }
 
 }  // namespace hga
