@@ -358,6 +358,22 @@ def flush_l2(buf):
     buf.add_(1)
 
 
+def max_over_ranks(ms, world, device):
+    """The slowest rank's device time (every rank calls this, in the same order)."""
+    if world <= 1:
+        return ms
+    import torch
+    t = torch.tensor([ms], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_step, steps, world, total_ms):
+    """Whole-job query tokens/s: every rank processes its own layer instance
+    (weak scaling), timed by the slowest rank."""
+    return tokens_per_step * steps * world / (total_ms / 1000.0)
+
+
 # ------------------------------------------------------------------ CPU oracle sample
 def oracle_sample(w, target_seconds):
     """Times the CPU oracle on a bounded sample of the workload; returns (tok/s, desc, cores)."""
@@ -484,13 +500,8 @@ def run_hga(args, rank, world, local):
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
-    total_ms = sum(a.elapsed_time(b) for a, b in zip(starts, ends))
-    if world > 1:
-        t = torch.tensor([total_ms], device="cuda")
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
-    tokens_per_step = w.seg_len * w.batch * len(w.seg_starts)
-    value = tokens_per_step * args.steps * world / (total_ms / 1000.0)
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, "cuda")
+    value = job_throughput(w.seg_len * w.batch * len(w.seg_starts), args.steps, world, total_ms)
     status = hga.hga_get_device_status()
 
     # per-kernel device time over the timed steps (events on the launching stream)

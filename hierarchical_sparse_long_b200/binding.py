@@ -22,8 +22,8 @@ STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3:
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
 EXPORTED = ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
-            "hga_attn_bwd_noalloc", "hga_fetch_tiered", "hga_get_device_status", "hga_status_string",
-            "hga_last_error")
+            "hga_attn_bwd_noalloc", "hga_fetch_tiered", "hga_get_device_status", "hga_selftest_wait_timeout",
+            "hga_status_string", "hga_last_error")
 
 
 class HGAError(RuntimeError):
@@ -89,6 +89,8 @@ def lib() -> ctypes.CDLL:
         L.hga_attn_bwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
+        L.hga_selftest_wait_timeout.argtypes = [ll, vp]
+        L.hga_selftest_wait_timeout.restype = ctypes.c_int
         L.hga_status_string.argtypes = [i]
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
@@ -185,6 +187,12 @@ def hga_fetch_tiered(p: Params, host_k, host_v, idx, qblock_begin: int, qblock_e
                                   qblock_end, _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(slot_map),
                                   _ptr(idx_remapped), _ptr(n_fetched), _stream(copy_stream), ev),
            "hga_fetch_tiered")
+
+
+def hga_selftest_wait_timeout(wait_cycles: int, stream=None):
+    """Launches a wait that can never complete, bounded to wait_cycles; the device
+    status then carries HGA_DEV_TIMEOUT (see hga_get_device_status)."""
+    _check(lib().hga_selftest_wait_timeout(wait_cycles, _stream(stream)), "hga_selftest_wait_timeout")
 
 
 def hga_get_device_status(stream=None) -> int:

@@ -186,6 +186,13 @@ hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const v
     return HGA_OK;
 }
 
+hga_status_t hga_selftest_wait_timeout(long long wait_cycles, cudaStream_t stream) {
+    if (wait_cycles < 1000 || wait_cycles > (1ll << 32)) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    return hga::launch_selftest_wait_timeout(wait_cycles, status, stream);
+}
+
 hga_status_t hga_get_device_status(cudaStream_t stream, unsigned int *bits) {
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);

@@ -42,11 +42,10 @@ namespace {
 
 constexpr int D = 128;
 constexpr int TILE = 64;
-constexpr int NSTAGE = 3;
+constexpr int NSTAGE = 5;
 constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold on the running max (log2 units)
 constexpr uint32_t Q_HALF_BYTES = 128 * D * 2;   // 32 KiB: [2 col halves][128 rows][128 B]
 constexpr uint32_t KV_TILE_BYTES = TILE * D * 2; // 16 KiB: [2 col halves][64 rows][128 B]
-constexpr uint32_t P_BYTES = 128 * TILE * 2;     // 16 KiB: [128 rows][128 B] (one P buffer)
 constexpr uint32_t IDESC_QK = tc::idesc_bf16(128, TILE, false, false);
 constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, D, false, true);
 
@@ -55,11 +54,21 @@ struct Smem {
     static constexpr uint32_t Q = 0;
     static constexpr uint32_t K = Q + NH * Q_HALF_BYTES;      // K ring
     static constexpr uint32_t V = K + NSTAGE * KV_TILE_BYTES; // V ring
-    static constexpr uint32_t P = V + NSTAGE * KV_TILE_BYTES;
-    static constexpr uint32_t BAR = P + NH * 2 * P_BYTES;  // P double-buffered per half
+    static constexpr uint32_t BAR = V + NSTAGE * KV_TILE_BYTES;
     static constexpr uint32_t TOTAL = BAR + 1024;  // barriers, tile list, flags
     static constexpr uint32_t ALLOC = TOTAL + 1024; // + alignment slack
 };
+
+// D[tmem] (+)= A[tmem] * B[smem] for one K=16 step of kind::f16 (A read from TMEM).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
 
 struct Bars {
     uint64_t q_full;
@@ -68,9 +77,8 @@ struct Bars {
     uint64_t v_full[NSTAGE];
     uint64_t v_empty[NSTAGE];  // released once PV of the tile completes
     uint64_t s_full[2][2];
-    uint64_t s_free[2][2];
-    uint64_t p_full[2][2];  // [half][P buffer]
-    uint64_t o_done[2][2];  // [half][P buffer of the PV that completed]
+    uint64_t p_full[2][2];  // [half][S/P buffer]: P of the buffer's tile written to TMEM
+    uint64_t o_done[2][2];  // [half][S/P buffer]: PV of the buffer's tile completed
     uint64_t drain[2];
     uint32_t tmem_base;
     int abort;
@@ -123,7 +131,6 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         for (int h = 0; h < 2; ++h) {
             for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->s_full[h][bb], 1);
-                tc::mbar_init(&bars->s_free[h][bb], 4);
             }
             for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->p_full[h][bb], 4);
@@ -210,7 +217,6 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * Q_HALF_BYTES, 16, 1024);
             const uint64_t k_desc = tc::desc_sw128(sbase + L::K, 16, 1024);
             const uint64_t v_desc = tc::desc_sw128(sbase + L::V, 8192, 1024);
-            const uint64_t p_desc = tc::desc_sw128(sbase + L::P + 2 * h * P_BYTES, 16, 1024);
             const uint32_t o_tmem = tmem + 128 * h;
             // O_h += P_h(t) V(t) once the softmax of tile t has written P buffer t&1
             auto issue_pv = [&](int t) -> bool {
@@ -219,11 +225,11 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                 if (!tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort, a.status)) return false;
                 tc::fence_after_sync();
                 const uint64_t vd = v_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
-                const uint64_t pd = p_desc + (uint64_t)((pb * P_BYTES) >> 4);
+                // P(t) as bf16 pairs in the first 32 columns of S buffer pb: 8 columns per K step
+                const uint32_t pa = tmem + 256 + 128 * h + 64 * pb;
 #pragma unroll
                 for (int kk = 0; kk < TILE / 16; ++kk)
-                    tc::mma_f16(o_tmem, pd + (kk * 32 >> 4), vd + (kk * 2048 >> 4), IDESC_PV,
-                                (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_f16_ts(o_tmem, pa + 8 * kk, vd + (kk * 2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
                 tc::mma_commit(&bars->o_done[h][pb]);
                 tc::mma_commit(&bars->v_empty[s]);  // one arrival per half
                 return true;
@@ -232,7 +238,8 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             for (int j = 0; ok && j < n_tiles; ++j) {
                 const int s = j % NSTAGE, bb = j & 1;
                 if (!tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)) { ok = false; break; }
-                if (j >= 2 && !tc::mbar_wait(&bars->s_free[h][bb], ((j >> 1) - 1) & 1, abort, a.status)) {
+                // S buffer bb is free once PV(j-2), which read P(j-2) from it, has completed
+                if (j >= 2 && !tc::mbar_wait(&bars->o_done[h][bb], ((j >> 1) - 1) & 1, abort, a.status)) {
                     ok = false;
                     break;
                 }
@@ -260,7 +267,6 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         const int i = r & 63;                 // query row within the block
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const uint32_t o_addr = tmem + lane_addr + 128 * h;
-        const uint32_t p_rows = sbase + L::P + 2 * h * P_BYTES + (r >> 3) * 1024 + (r & 7) * 128;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
@@ -280,9 +286,6 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                 tc::tmem_ld32(s_addr + 32, hi);
                 tc::tmem_wait_ld();
             }
-            tc::fence_before_sync();
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->s_free[h][bb]);
             float x[64];
             const bool diag = (j == n_tiles - 1);  // the local tile of this block (warp-uniform)
 #pragma unroll
@@ -323,12 +326,6 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                               ((spart[4] + spart[5]) + (spart[6] + spart[7]));
             l_run = l_run * alpha + sum;
             const int pb = j & 1;
-            // P buffer pb was last read by PV(j-2)
-            if (j >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][pb], ((j >> 1) - 1) & 1, abort,
-                                                                  a.status))) {
-                ok = false;
-                break;
-            }
             // a rescale needs O complete up to tile j-1 (PV(j-1) done) before PV(j) adds to it;
             // rows that keep their reference max have alpha == 1, an exact no-op
             if (j >= 1 && __any_sync(0xffffffffu, grow)) {
@@ -350,16 +347,15 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                 tc::tmem_wait_st();
             }
             m_run = m_use;
-            const uint32_t p_row = p_rows + pb * P_BYTES;
+            // P as bf16 pairs over the first 32 columns of this tile's S buffer (already
+            // read into registers); PV reads it from there as its A operand
+            {
+                uint32_t pk[32];
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
-                const uint32_t addr = p_row + ((cc ^ (r & 7)) << 4);
-                tc::st_shared_v4(addr, tc::pack_bf16(x[8 * cc + 0], x[8 * cc + 1]),
-                                 tc::pack_bf16(x[8 * cc + 2], x[8 * cc + 3]),
-                                 tc::pack_bf16(x[8 * cc + 4], x[8 * cc + 5]),
-                                 tc::pack_bf16(x[8 * cc + 6], x[8 * cc + 7]));
+                for (int c = 0; c < 32; ++c) pk[c] = tc::pack_bf16(x[2 * c], x[2 * c + 1]);
+                tc::tmem_st32(tmem + lane_addr + 256 + 128 * h + 64 * pb, pk);
+                tc::tmem_wait_st();
             }
-            tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->p_full[h][pb]);

@@ -79,6 +79,7 @@ hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, cons
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
                                  int stage_slots, int32_t *slot_map, int32_t *idx_remapped,
                                  int32_t *n_fetched, unsigned *status, cudaStream_t stream);
+hga_status_t launch_selftest_wait_timeout(long long wait_cycles, unsigned *status, cudaStream_t stream);
 hga_status_t record_cuda(cudaError_t e);
 void record_error(const char *msg);
 }  // namespace hga

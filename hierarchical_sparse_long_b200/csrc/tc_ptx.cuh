@@ -191,6 +191,15 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     return *reinterpret_cast<uint32_t *>(&v);
 }
 
+// bf16x2 of two non-negative finite floats, round-to-nearest-even, on the
+// integer pipe (add 0x7FFF plus the kept LSB, keep the high halves).
+__device__ __forceinline__ uint32_t pack_bf16_rne_int(float lo, float hi) {
+    const uint32_t a = __float_as_uint(lo), b = __float_as_uint(hi);
+    const uint32_t ra = a + 0x7FFFu + ((a >> 16) & 1u);
+    const uint32_t rb = b + 0x7FFFu + ((b >> 16) & 1u);
+    return __byte_perm(ra, rb, 0x7632);
+}
+
 __device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }

@@ -209,6 +209,15 @@ hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const v
                               void *stage_v, int stage_slots, int32_t *slot_map, int32_t *idx_remapped,
                               int32_t *n_fetched, cudaStream_t copy_stream, cudaEvent_t done);
 
+/* Self-test of the bounded waits (the source pages have no counterpart): every
+ * pipeline wait in the tensor-core kernels gives up after a cycle limit instead
+ * of hanging, sets HGA_DEV_TIMEOUT and lets the kernel end.  This launches one
+ * CTA whose only thread waits on an mbarrier nothing ever arrives at, with a
+ * limit of wait_cycles (1e3 .. 2^32 SM cycles); afterwards
+ * hga_get_device_status() reports HGA_ERR_TIMEOUT and the context stays usable.
+ * Returns HGA_ERR_INVALID_ARG for a limit outside that range. */
+hga_status_t hga_selftest_wait_timeout(long long wait_cycles, cudaStream_t stream);
+
 /* Reads (after synchronising stream) and clears the device status word of the
  * current device; *bits gets the HGA_DEV_* bits seen since the last call.
  * Returns HGA_ERR_DEVICE_CHECK or HGA_ERR_TIMEOUT when bits are set. */
