@@ -160,10 +160,12 @@ def attn_bwd_flops(w, T):
 
 
 def route_bytes(w, T):
-    """Q read once + the routable summaries read per (b, g, block)."""
+    """Algorithmic bytes of one route: the queries read once, every routable
+    summary read once, the route table written."""
     nqb = w.seg_len // w.q_block
     return (w.batch * w.n_q_heads * w.seg_len * w.head_dim * 2 +
-            w.batch * w.n_kv_heads * nqb * (T // w.chunk) * w.head_dim * 4)
+            w.batch * w.n_kv_heads * (T // w.chunk) * w.head_dim * 4 +
+            w.batch * w.n_kv_heads * nqb * w.topk * 4)
 
 
 def summaries_bytes(w):

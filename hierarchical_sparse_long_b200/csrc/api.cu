@@ -107,7 +107,9 @@ hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, 
     if (p->n_hist_chunks > 16384) return HGA_ERR_UNSUPPORTED;
     if (!q || !idx || !aligned16(q)) return HGA_ERR_INVALID_ARG;
     if (p->n_hist_chunks > 0 && (!summ || !aligned16(summ))) return HGA_ERR_INVALID_ARG;
-    return hga::launch_route(*p, q, summ, summ_cap_chunks, idx, stream);
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    return hga::launch_route(*p, q, summ, summ_cap_chunks, idx, status, stream);
 }
 
 hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,

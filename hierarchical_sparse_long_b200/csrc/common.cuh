@@ -53,7 +53,7 @@ hga_status_t launch_summaries(const void *k, long long head_stride, int bh, int 
                               int first_chunk, int n_chunks, hga_dtype_t dtype, float *summ, int cap,
                               cudaStream_t stream);
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
-                          cudaStream_t stream);
+                          unsigned *status, cudaStream_t stream);
 hga_status_t launch_attn_fwd_simt(const hga_params_t &p, const void *q, const void *k_hist,
                                   const void *v_hist, const void *k_seg, const void *v_seg,
                                   const int32_t *idx, void *out, float *lse, unsigned *status,

@@ -9,16 +9,83 @@
 // fp32 dot / sqrt(D), and the k best chunks are taken by (score descending,
 // chunk index ascending) and listed in ascending chunk order.
 //
-// One CTA per (batch, kv head, query block).  The CTA reads its G*q_block
-// query rows once with 16-byte coalesced loads (the kernel's HBM traffic),
-// scores the L2-resident summaries with one thread per chunk (fp32 FFMA, no
-// tensor cores, so every score is an fp32 dot product in a fixed order),
-// then finds the k-th largest score by a 4-pass 8-bit radix select on the
-// order-preserving score bits and collects the chunks above it plus the
-// lowest-index chunks tied with it.
+// One CTA per (batch, kv head, query block); CL consecutive query blocks of
+// one (batch, kv head) form a thread-block cluster.
+//   1. Summary tiles start streaming at once by bulk copies into a 4-slot
+//      shared-memory ring, while every thread loads its share of the block's
+//      G x q_block query rows straight into registers (16-byte loads, all in
+//      flight together) and the CTA sums them in a fixed order: the block
+//      summary qbar (fp32).
+//   2. The cluster's CL summaries are exchanged through distributed shared
+//      memory; each CTA scores its 1/CL slice of the chunks against all CL
+//      of them, so every chunk summary crosses L2 -> SM once per cluster.
+//      16 lanes share one chunk row (coalesced reads), fp32 FFMA only (no
+//      tensor cores), and the lane partials fold by shuffles in a fixed
+//      tree, so every score is a deterministic fp32 dot product.
+//   3. Each CTA gathers its own query block's full score row from the
+//      cluster and selects with all its threads: a lower bound of the k-th
+//      best score from the per-thread maxima, the few chunks at or above it,
+//      and their exact ranks by (score, then the lower chunk index).
+#include <algorithm>
+
 #include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace hga {
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kRing = 4;         // bulk-copy ring slots
+constexpr int kCandCap = 1024;   // candidate list of the selecting warp
+constexpr int kMaxSmem = 227 * 1024 - 1024;
+constexpr unsigned kFull = 0xffffffffu;
+
+// Byte offsets of the dynamic shared-memory regions (host computed).
+struct RouteLayout {
+    int ring, part, qown, qall, sc, row, tmax, key, cj, hist, misc, bar, total;
+};
+
+struct RouteArgs {
+    const void *q;
+    const float *summ;
+    int32_t *idx;
+    unsigned *status;
+    long long cap;  // summary rows per (b, g)
+    int n_q_heads, n_kv_heads, seg_len, n, topk;
+    int ns;  // chunks per cluster rank (multiple of 4)
+    float inv_sqrt_d;
+    RouteLayout L;
+};
+
+constexpr int kTileBytes = 16 * 1024;  // one ring slot: a tile of summary rows
+constexpr int kQBlock = 64;            // queries per block (the only size the API accepts)
+constexpr int kWarps = kThreads / 32;
+
+int round4(int x) { return (x + 3) & ~3; }
+
+RouteLayout route_layout(int D, int esize, int cl, int ns, int n) {
+    RouteLayout L{};
+    int off = 0;
+    auto take = [&](int bytes) {
+        const int at = off;
+        off += (bytes + 15) & ~15;
+        return at;
+    };
+    L.ring = take(kRing * kTileBytes);
+    L.part = take((kThreads / (D * esize / 16)) * D * 4);
+    L.qown = take(D * 4);
+    L.qall = take(cl * D * 4);
+    L.sc = take(cl * ns * 4);
+    L.row = take(cl > 1 ? round4(n) * 4 : 0);
+    L.tmax = take(kThreads * 4);
+    L.key = take(kCandCap * 8);
+    L.cj = take(kCandCap * 4);
+    L.hist = take(256 * 4);
+    L.misc = take(16 * 4);
+    L.bar = take(kRing * 8);
+    L.total = off;
+    return L;
+}
 
 // Order-preserving 32-bit image of an fp32 score (larger score -> larger
 // value; -0 and +0 map to the same value).
@@ -28,217 +95,491 @@ __device__ __forceinline__ uint32_t ordered_bits(float s) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-template <typename T, int D>
-__global__ void __launch_bounds__(256) route_kernel(const T *__restrict__ q, const float *__restrict__ summ,
-                                                    int cap, int32_t *__restrict__ idx, int n_q_heads,
-                                                    int n_kv_heads, int seg_len, int q_block, int n_chunks,
-                                                    int topk, float inv_sqrt_d) {
-    constexpr int VEC = Vec16<T>::N;
-    constexpr int LPR = D / VEC;
-    constexpr int NSLOT = 256 / LPR;
-    extern __shared__ uint32_t ord[];  // n_chunks ordered score images
-    __shared__ float part[NSLOT][D + 1];
-    __shared__ float qbar[D];
-    __shared__ int hist[256];
-    __shared__ int chosen[64];
-    __shared__ int n_chosen;
-    __shared__ uint32_t sel_prefix;
-    __shared__ int sel_remaining;
-    __shared__ int warp_ties[8];
-    __shared__ int ties_before;
+// 64-bit selection key: score image, then the lower chunk index first.
+__device__ __forceinline__ uint64_t sel_key(uint32_t ord, int j) {
+    return (static_cast<uint64_t>(ord) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(j));
+}
 
-    const int nqb = seg_len / q_block;
-    const int m = blockIdx.x % nqb;
-    const int bg = blockIdx.x / nqb;  // b * Hkv + g
-    const int b = bg / n_kv_heads, g = bg % n_kv_heads;
-    const int G = n_q_heads / n_kv_heads;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+// acc[e] += element e of one 16-byte unit (8 bf16 or 4 fp32).
+template <typename T> __device__ __forceinline__ void add_unit(const uint4 &w, float *acc);
+template <> __device__ __forceinline__ void add_unit<float>(const uint4 &w, float *acc) {
+    acc[0] += __uint_as_float(w.x);
+    acc[1] += __uint_as_float(w.y);
+    acc[2] += __uint_as_float(w.z);
+    acc[3] += __uint_as_float(w.w);
+}
+template <> __device__ __forceinline__ void add_unit<__nv_bfloat16>(const uint4 &w, float *acc) {
+    const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        acc[2 * i] += __uint_as_float(v[i] << 16);
+        acc[2 * i + 1] += __uint_as_float(v[i] & 0xFFFF0000u);
+    }
+}
 
-    // 1. block summary: mean over G heads x q_block rows, fixed order; every
-    //    thread keeps 8 independent 16-byte loads in flight
-    {
-        const int col = (tid % LPR) * VEC, slot = tid / LPR;
-        float acc[VEC];
-#pragma unroll
-        for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
-        const int rows = G * q_block;
-        int r = slot;
-        for (; r + 7 * NSLOT < rows; r += 8 * NSLOT) {
-            float v[8][VEC];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const int rr = r + u * NSLOT;
-                const int h = g * G + rr / q_block, i = m * q_block + rr % q_block;
-                Vec16<T>::load(q + (((long long)b * n_q_heads + h) * seg_len + i) * D + col, v[u]);
+// One warp, the whole row: the k (< n) best chunks of row[0, n) by (score
+// image descending, chunk index ascending), written to out[0, k) in ascending
+// chunk order.  Radix select (4 passes of 8 bits, most significant first) of
+// the k-th largest image, then every chunk above it and the lowest-index
+// chunks equal to it.  Used when the candidate list of select_cta overflows.
+__device__ void select_warp_radix(const uint32_t *row, int n, int k, int32_t *out, int *hist, int lane) {
+    const unsigned lt = (1u << lane) - 1u;
+    uint32_t prefix = 0u, mask = 0u;
+    int rem = k;
+    for (int shift = 24; shift >= 0; shift -= 8) {
+        for (int b = lane; b < 256; b += 32) hist[b] = 0;
+        __syncwarp();
+        for (int base = 0; base < n; base += 32) {
+            const int p = base + lane;
+            const uint32_t v = p < n ? row[p] : 0u;
+            const bool in = p < n && (v & mask) == prefix;
+            const int bin = static_cast<int>((v >> shift) & 255u);
+            const unsigned act = __ballot_sync(kFull, in);
+            if (act) {
+                // one shared atomic when every active lane hits the same bin
+                const int leader = __ffs(act) - 1;
+                const int b0 = __shfl_sync(kFull, bin, leader);
+                if (__ballot_sync(kFull, in && bin != b0) == 0) {
+                    if (lane == leader) atomicAdd(&hist[b0], __popc(act));
+                } else if (in) {
+                    atomicAdd(&hist[bin], 1);
+                }
             }
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-#pragma unroll
-                for (int e = 0; e < VEC; ++e) acc[e] += v[u][e];
         }
-        for (; r < rows; r += NSLOT) {
-            const int h = g * G + r / q_block, i = m * q_block + r % q_block;
-            float v[VEC];
-            Vec16<T>::load(q + (((long long)b * n_q_heads + h) * seg_len + i) * D + col, v);
+        __syncwarp();
+        // lane l holds bins 8l .. 8l+7; scan from the top bin down
+        int cnt[8], tot = 0;
 #pragma unroll
-            for (int e = 0; e < VEC; ++e) acc[e] += v[e];
+        for (int e = 0; e < 8; ++e) {
+            cnt[e] = hist[8 * lane + e];
+            tot += cnt[e];
         }
+        int suf = tot;
 #pragma unroll
-        for (int e = 0; e < VEC; ++e) part[slot][col + e] = acc[e];
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_down_sync(kFull, suf, o);
+            if (lane + o < 32) suf += y;
+        }
+        int above = suf - tot, fbin = -1, frem = 0;
+#pragma unroll
+        for (int e = 7; e >= 0; --e) {
+            if (fbin < 0 && above < rem && above + cnt[e] >= rem) {
+                fbin = 8 * lane + e;
+                frem = rem - above;
+            }
+            above += cnt[e];
+        }
+        const unsigned fb = __ballot_sync(kFull, fbin >= 0);
+        const int src = fb ? __ffs(fb) - 1 : 0;
+        fbin = __shfl_sync(kFull, fbin, src);
+        frem = __shfl_sync(kFull, frem, src);
+        if (fbin < 0) {  // unreachable: the bins count every chunk matching the prefix
+            fbin = 0;
+            frem = rem;
+        }
+        prefix |= static_cast<uint32_t>(fbin) << shift;
+        mask |= 255u << shift;
+        rem = frem;
+        __syncwarp();
     }
-    __syncthreads();
-    if (tid < D) {
-        float s = 0.f;
-        for (int sl = 0; sl < NSLOT; ++sl) s += part[sl][tid];
-        qbar[tid] = s / (float)(G * q_block);
+    int written = 0, ties = 0;
+    for (int base = 0; base < n && written < k; base += 32) {
+        const int p = base + lane;
+        const uint32_t v = p < n ? row[p] : 0u;
+        const bool tie = p < n && v == prefix;
+        const unsigned tb = __ballot_sync(kFull, tie);
+        const bool take = p < n && (v > prefix || (tie && ties + __popc(tb & lt) < rem));
+        const unsigned kb = __ballot_sync(kFull, take);
+        if (take) out[written + __popc(kb & lt)] = p;
+        written += __popc(kb);
+        ties += __popc(tb);
     }
-    if (tid == 0) n_chosen = 0;
-    __syncthreads();
+}
 
-    // 2. scores; one thread per chunk, four interleaved partial dot products
-    //    over d (mod 4) summed in a fixed order
-    const float *sb = summ + (long long)bg * cap * D;
-    for (int j = tid; j < n_chunks; j += 256) {
-        const float4 *row = reinterpret_cast<const float4 *>(sb + (long long)j * D);
-        float d0 = 0.f, d1 = 0.f, d2 = 0.f, d3 = 0.f;
-#pragma unroll 8
-        for (int e = 0; e < D / 4; ++e) {
-            const float4 v = row[e];
-            d0 = fmaf(qbar[4 * e + 0], v.x, d0);
-            d1 = fmaf(qbar[4 * e + 1], v.y, d1);
-            d2 = fmaf(qbar[4 * e + 2], v.z, d2);
-            d3 = fmaf(qbar[4 * e + 3], v.w, d3);
+struct SelScratch {
+    uint32_t *tmax;  // [kThreads] per-thread maxima
+    uint64_t *key;   // [kCandCap] candidate keys
+    int *cj;         // [kCandCap] chosen candidates' chunk index, else INT_MAX
+    int *hist;       // [256] (whole-row fallback)
+    int *misc;       // [16]: candidate count, per-warp minima
+};
+
+// The whole CTA: the k (< n) best chunks of row[0, n) by (score image
+// descending, chunk index ascending), written to out[0, k) ascending.
+//   bound: thr = k-th largest of the kThreads per-thread maxima (thread t
+//          takes chunks t, t + kThreads, ...); they are distinct chunks, so
+//          at least k chunks have an image >= thr and so do all k best;
+//   candidates: the chunks with image >= thr (warp-aggregated append);
+//   rank of each candidate among the candidates by its 64-bit key (image,
+//   then the lower chunk index); the k of rank < k are the answer and each
+//   lands at the count of chosen candidates with a lower chunk index.
+__device__ void select_cta(const uint32_t *row, int n, int k, int32_t *out, const SelScratch &s, int tid) {
+    const int lane = tid & 31, warp = tid >> 5;
+    const unsigned lt = (1u << lane) - 1u;
+    uint32_t mx = 0u;  // 0 is below every real score image
+    for (int j = tid; j < n; j += kThreads) mx = max(mx, row[j]);
+    s.tmax[tid] = mx;
+    if (tid == 0) s.misc[0] = 0;
+    __syncthreads();
+    int gp[4] = {0, 0, 0, 0};  // independent partial counts (short dependency chains)
+#pragma unroll 4
+    for (int u = 0; u < kThreads; u += 16) {
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(s.tmax + u + 4 * h);
+            gp[h] += (v.x > mx) + (v.y > mx) + (v.z > mx) + (v.w > mx);
         }
-        ord[j] = ordered_bits(((d0 + d1) + (d2 + d3)) * inv_sqrt_d);
+    }
+    const int greater = (gp[0] + gp[1]) + (gp[2] + gp[3]);
+    uint32_t thr = greater < k ? mx : 0xFFFFFFFFu;
+#pragma unroll
+    for (int o = 16; o; o >>= 1) thr = min(thr, __shfl_xor_sync(kFull, thr, o));
+    if (lane == 0) s.misc[8 + warp] = static_cast<int>(thr);
+    __syncthreads();
+    thr = static_cast<uint32_t>(s.misc[8]);
+#pragma unroll
+    for (int w = 1; w < kThreads / 32; ++w) thr = min(thr, static_cast<uint32_t>(s.misc[8 + w]));
+
+    for (int base = 0; base < n; base += kThreads) {  // warp-uniform trip count
+        const int j = base + tid;
+        const bool in = j < n && row[j] >= thr;
+        const unsigned bal = __ballot_sync(kFull, in);
+        int wbase = 0;
+        if (lane == 0 && bal) wbase = atomicAdd(&s.misc[0], __popc(bal));
+        wbase = __shfl_sync(kFull, wbase, 0);
+        const int pos = wbase + __popc(bal & lt);
+        if (in && pos < kCandCap) s.key[pos] = sel_key(row[j], j);
     }
     __syncthreads();
+    const int C = s.misc[0];
+    if (C > kCandCap) {  // too many chunks at the bound: radix select on the whole row
+        if (warp == 0) select_warp_radix(row, n, k, out, s.hist, lane);
+        return;
+    }
+    for (int c = tid; c < C; c += kThreads) {
+        const uint64_t kc = s.key[c];
+        int r = 0;
+        for (int u = 0; u < C; ++u) r += s.key[u] > kc;
+        s.cj[c] = r < k ? static_cast<int>(~static_cast<uint32_t>(kc)) : 0x7FFFFFFF;
+    }
+    __syncthreads();
+    for (int c = tid; c < C; c += kThreads) {
+        const int j = s.cj[c];
+        if (j != 0x7FFFFFFF) {
+            int pos = 0;
+            for (int u = 0; u < C; ++u) pos += s.cj[u] < j;
+            out[pos] = j;
+        }
+    }
+}
 
-    int32_t *out = idx + ((long long)bg * nqb + m) * topk;
-    const int keff = topk < n_chunks ? topk : n_chunks;
-    if (keff == n_chunks) {
-        // every chunk is routed
-        for (int a = tid; a < topk; a += 256) out[a] = a < n_chunks ? a : -1;
+// Waits, with a fresh bound, for bulk copies still in flight after an abort.
+__device__ void drain_ring(uint64_t *bar, int from, int to) {
+    for (int i = from; i < to; ++i) {
+        const long long t0 = clock64();
+        while (!tc::mbar_try_wait(&bar[i % kRing], (i / kRing) & 1) && clock64() - t0 < (1ll << 31)) {
+        }
+    }
+}
+
+template <typename T, int D, int CL>
+__global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    __shared__ int abort_flag;
+    const RouteLayout &L = a.L;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nqb = a.seg_len / kQBlock;
+    const int m = blockIdx.x % nqb, bg = blockIdx.x / nqb;
+    const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int n = a.n;
+    int32_t *out = a.idx + ((long long)bg * nqb + m) * a.topk;
+    if (n <= a.topk) {  // every chunk is routed (the same branch for the whole grid)
+        for (int t = tid; t < a.topk; t += kThreads) out[t] = t < n ? t : -1;
         return;
     }
 
-    // 3. radix select (4 passes of 8 bits, most significant first) of the
-    //    keff-th largest score image: sel_prefix ends as that value and
-    //    sel_remaining as how many chunks equal to it are taken
+    const int rank = CL > 1 ? static_cast<int>(tc::cluster_ctarank()) : 0;  // == m % CL
+    const int c_begin = rank * a.ns;
+    const int n_slice = max(0, min(n, c_begin + a.ns) - c_begin);
+    constexpr int TCN = kTileBytes / (D * 4);  // chunks per summary tile
+    const int ntiles = (n_slice + TCN - 1) / TCN;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + L.bar);
+    const float *sbase = a.summ + ((long long)bg * a.cap + c_begin) * D;
+
+    auto issue = [&](int t) {
+        const int slot = t % kRing;
+        const uint32_t bytes = static_cast<uint32_t>(min(TCN, n_slice - t * TCN) * D * 4);
+        tc::mbar_arrive_expect_tx(&bar[slot], bytes);
+        tc::bulk_load(smem + L.ring + slot * kTileBytes, sbase + (long long)t * TCN * D, bytes, &bar[slot]);
+    };
+
     if (tid == 0) {
-        sel_prefix = 0u;
-        sel_remaining = keff;
+        abort_flag = 0;
+        for (int s = 0; s < kRing; ++s) tc::mbar_init(&bar[s], 1);
+        tc::fence_mbar_init();
     }
-    uint32_t mask = 0u;
-    for (int shift = 24; shift >= 0; shift -= 8) {
-        hist[tid] = 0;
-        __syncthreads();
-        const uint32_t prefix = sel_prefix;
-        for (int base = 0; base < n_chunks; base += 256) {  // warp-uniform trip count
-            const int j = base + tid;
-            const uint32_t v = j < n_chunks ? ord[j] : 0u;
-            const bool in = j < n_chunks && (v & mask) == prefix;
-            const int bin = (int)((v >> shift) & 255u);
-            // one shared atomic per distinct bin of the warp
-            const unsigned act = __ballot_sync(0xffffffffu, in);
-            if (in) {
-                const unsigned peers = __match_any_sync(act, bin);
-                if ((__ffs(peers) - 1) == lane) atomicAdd(&hist[bin], __popc(peers));
-            }
-        }
-        __syncthreads();
-        if (warp == 0) {
-            // bins from the top: find the bin holding the remaining-th largest
-            int rem = sel_remaining;
-            int above = 0;  // count in bins above the current 32-bin group
-            for (int grp = 7; grp >= 0; --grp) {
-                const int c = hist[grp * 32 + lane];
-                // inclusive suffix sum within the group (higher bins first)
-                int suf = c;
+    __syncthreads();
+    int issued = 0;  // thread 0's count of issued tiles
+    if (tid == 0)
+        for (; issued < min(kRing, ntiles); ++issued) issue(issued);
+
+    // 1. block summary.  Thread (rs, cu) sums the 16-byte column unit cu of
+    //    rows rs, rs + NRS, ... of the G x q_block rows (head-major), in order;
+    //    the NRS row slots are then added in order.
+    constexpr int VEC = Vec16<T>::N;  // elements per 16-byte unit
+    constexpr int UPR = D / VEC;      // units per row
+    constexpr int NRS = kThreads / UPR;
+    constexpr int BATCH = 16;         // loads in flight per thread
+    {
+        const int cu = tid % UPR, rs = tid / UPR;
+        const T *qbase = static_cast<const T *>(a.q) +
+                         (((long long)b * a.n_q_heads + (long long)g * G) * a.seg_len + (long long)m * kQBlock) * D +
+                         cu * VEC;
+        const int rows = G * kQBlock;
+        float acc[VEC];
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const int y = __shfl_down_sync(0xffffffffu, suf, off);
-                    if (lane + off < 32) suf += y;
+        for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
+        for (int r0 = rs; r0 < rows; r0 += BATCH * NRS) {
+            uint4 raw[BATCH];
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) {
+                const int r = r0 + u * NRS;
+                if (r < rows) {
+                    const int hh = r / kQBlock, i = r % kQBlock;
+                    raw[u] = *reinterpret_cast<const uint4 *>(qbase + ((long long)hh * a.seg_len + i) * D);
+                } else {
+                    raw[u] = make_uint4(0u, 0u, 0u, 0u);
                 }
-                const int total = __shfl_sync(0xffffffffu, suf, 0);
-                if (above + total >= rem) {
-                    // the bin is the highest lane whose suffix (>= itself) reaches rem
-                    const unsigned hit = __ballot_sync(0xffffffffu, above + suf >= rem);
-                    const int bl = 31 - __clz(hit);
-                    const int above_bin = above + __shfl_sync(0xffffffffu, suf, bl) -
-                                          __shfl_sync(0xffffffffu, c, bl);
-                    if (lane == 0) {
-                        sel_prefix = prefix | ((uint32_t)(grp * 32 + bl) << shift);
-                        sel_remaining = rem - above_bin;
+            }
+#pragma unroll
+            for (int u = 0; u < BATCH; ++u) add_unit<T>(raw[u], acc);
+        }
+        float *part = reinterpret_cast<float *>(smem + L.part);
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) part[rs * D + cu * VEC + e] = acc[e];
+    }
+    __syncthreads();
+    float *qown = reinterpret_cast<float *>(smem + L.qown);
+    if (tid < D) {
+        const float *part = reinterpret_cast<const float *>(smem + L.part);
+        float s = 0.f;
+        for (int sl = 0; sl < NRS; ++sl) s += part[sl * D + tid];
+        qown[tid] = s / static_cast<float>(G * kQBlock);
+    }
+
+    // 2. the cluster's CL block summaries, then this rank's slice of scores
+    const float *qall = qown;
+    if constexpr (CL > 1) {
+        tc::cluster_arrive();
+        tc::cluster_wait();
+        float *qa = reinterpret_cast<float *>(smem + L.qall);
+        constexpr int V4 = D / 4;
+        for (int t = tid; t < CL * V4; t += kThreads) {
+            const int r = t / V4, o = t % V4;
+            *reinterpret_cast<uint4 *>(qa + r * D + 4 * o) =
+                tc::ld_dsmem_v4(tc::mapa_shared(tc::smem_u32(qown + 4 * o), static_cast<uint32_t>(r)));
+        }
+        qall = qa;
+    }
+    __syncthreads();
+
+    constexpr int NV = D / 64;  // float4 per lane per chunk row
+    constexpr int LOGCL = CL == 8 ? 3 : CL == 4 ? 2 : CL == 2 ? 1 : 0;
+    const int half = lane >> 4, s16 = lane & 15;
+    float4 qr[CL][NV];
+#pragma unroll
+    for (int mb = 0; mb < CL; ++mb)
+#pragma unroll
+        for (int u = 0; u < NV; ++u) qr[mb][u] = *reinterpret_cast<const float4 *>(qall + mb * D + 4 * s16 + 64 * u);
+    uint32_t *sc = reinterpret_cast<uint32_t *>(smem + L.sc);  // [CL][ns] score images of the slice
+    const int my_mb = s16 >> (4 - LOGCL);
+    const bool writer = (s16 & ((1 << (4 - LOGCL)) - 1)) == 0;
+    bool ok = true;
+    int done = 0;  // tiles this thread waited for successfully
+    // rounds of up to kRing tiles: the round's chunks sit contiguously in the
+    // ring, every warp takes chunk pairs warp, warp + kWarps, ... of the round
+    constexpr int UNR = CL >= 8 ? 1 : 2;  // chunk pairs in flight per warp
+    for (int t0 = 0; t0 < ntiles; t0 += kRing) {
+        const int t1 = min(ntiles, t0 + kRing);
+        for (int t = t0; t < t1; ++t) {
+            ok = ok && tc::mbar_wait(&bar[t % kRing], (t / kRing) & 1, &abort_flag, a.status);
+            done += ok;
+        }
+        if (ok) {
+            const float *chunks = reinterpret_cast<const float *>(smem + L.ring);
+            const int rows = min((t1 - t0) * TCN, n_slice - t0 * TCN);
+            const int npairs = (rows + 1) >> 1;
+            for (int pr0 = warp; pr0 < npairs; pr0 += UNR * kWarps) {  // warp-uniform
+                float v[UNR][CL];
+#pragma unroll
+                for (int q = 0; q < UNR; ++q) {
+                    const int cl = 2 * (pr0 + q * kWarps) + half;
+                    const bool valid = cl < rows;
+                    float4 x[NV];
+#pragma unroll
+                    for (int u = 0; u < NV; ++u)
+                        x[u] = valid ? *reinterpret_cast<const float4 *>(chunks + cl * D + 4 * s16 + 64 * u)
+                                     : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int mb = 0; mb < CL; ++mb) {
+                        float acc = 0.f;
+#pragma unroll
+                        for (int u = 0; u < NV; ++u) {
+                            acc = fmaf(qr[mb][u].x, x[u].x, acc);
+                            acc = fmaf(qr[mb][u].y, x[u].y, acc);
+                            acc = fmaf(qr[mb][u].z, x[u].z, acc);
+                            acc = fmaf(qr[mb][u].w, x[u].w, acc);
+                        }
+                        v[q][mb] = acc;
                     }
-                    break;
                 }
-                above += total;
+                // fold the 16 lanes of each chunk (xor 8, 4, 2, 1): while several
+                // query blocks remain, each step halves them between lane pairs
+#pragma unroll
+                for (int st = 0; st < 4; ++st) {
+                    const int o = 8 >> st;
+                    const int w = CL >> st;
+#pragma unroll
+                    for (int q = 0; q < UNR; ++q) {
+                        if (w > 1) {
+                            const bool up = (s16 & o) != 0;
+#pragma unroll
+                            for (int e = 0; e < w / 2; ++e) {
+                                const float send = up ? v[q][e] : v[q][e + w / 2];
+                                const float keep = up ? v[q][e + w / 2] : v[q][e];
+                                v[q][e] = keep + __shfl_xor_sync(kFull, send, o);
+                            }
+                        } else {
+                            v[q][0] += __shfl_xor_sync(kFull, v[q][0], o);
+                        }
+                    }
+                }
+#pragma unroll
+                for (int q = 0; q < UNR; ++q) {
+                    const int cl = 2 * (pr0 + q * kWarps) + half;
+                    if (cl < rows && writer)
+                        sc[my_mb * a.ns + t0 * TCN + cl] = ordered_bits(v[q][0] * a.inv_sqrt_d);
+                }
             }
         }
-        mask |= 255u << shift;
         __syncthreads();
+        if (tid == 0 && issued < ntiles && !abort_flag) {
+            tc::fence_proxy_async();
+            for (; issued < min(ntiles, t1 + kRing); ++issued) issue(issued);
+        }
     }
-    const uint32_t thr = sel_prefix;
-    const int take_ties = sel_remaining;
 
-    // 4. collect: every chunk above the threshold, then the lowest-index
-    //    take_ties chunks equal to it (ties go to the lower chunk index)
-    for (int j = tid; j < n_chunks; j += 256)
-        if (ord[j] > thr) chosen[atomicAdd(&n_chosen, 1)] = j;
-    if (tid == 0) ties_before = 0;
-    __syncthreads();
-    for (int base = 0; base < n_chunks; base += 256) {
-        const int j = base + tid;
-        const bool tie = j < n_chunks && ord[j] == thr;
-        const unsigned bal = __ballot_sync(0xffffffffu, tie);
-        if (lane == 0) warp_ties[warp] = __popc(bal);
-        __syncthreads();
-        int rank = ties_before + __popc(bal & ((1u << lane) - 1u));
-        for (int w = 0; w < warp; ++w) rank += warp_ties[w];
-        if (tie && rank < take_ties) chosen[keff - take_ties + rank] = j;
-        __syncthreads();
-        if (tid == 0)
-            for (int w = 0; w < 8; ++w) ties_before += warp_ties[w];
-        __syncthreads();
-        if (ties_before >= take_ties) break;
+    // 3. this query block's full score row, then the CTA selects
+    const uint32_t *row = sc;
+    if constexpr (CL > 1) {
+        tc::cluster_arrive();
+        tc::cluster_wait();
+        uint32_t *rw = reinterpret_cast<uint32_t *>(smem + L.row);
+        const int n4 = a.ns / 4;
+        for (int t = tid; t < CL * n4; t += kThreads) {
+            const int r = t / n4, o = t % n4;
+            const int j = r * a.ns + 4 * o;
+            if (j < n)
+                *reinterpret_cast<uint4 *>(rw + j) = tc::ld_dsmem_v4(
+                    tc::mapa_shared(tc::smem_u32(sc + rank * a.ns + 4 * o), static_cast<uint32_t>(r)));
+        }
+        tc::cluster_arrive();  // done reading the peers' shared memory
+        row = rw;
     }
     __syncthreads();
-
-    // 5. the keff chosen chunks in ascending order, then -1 padding
-    if (tid < keff) {
-        const int me = chosen[tid];
-        int rank = 0;
-        for (int a = 0; a < keff; ++a) rank += chosen[a] < me;
-        out[rank] = me;
-    } else if (tid < topk) {
-        out[tid] = -1;
+    if (!abort_flag) {
+        SelScratch ss;
+        ss.tmax = reinterpret_cast<uint32_t *>(smem + L.tmax);
+        ss.key = reinterpret_cast<uint64_t *>(smem + L.key);
+        ss.cj = reinterpret_cast<int *>(smem + L.cj);
+        ss.hist = reinterpret_cast<int *>(smem + L.hist);
+        ss.misc = reinterpret_cast<int *>(smem + L.misc);
+        select_cta(row, n, a.topk, out, ss, tid);
     }
+    if (tid == 0 && abort_flag) drain_ring(bar, done, issued);
+    if constexpr (CL > 1) tc::cluster_wait();  // peers may still read this CTA's slice
+}
+
+template <typename T, int D, int CL>
+cudaError_t launch_cl(const RouteArgs &a, unsigned grid, cudaStream_t stream) {
+    auto kern = route_kernel<T, D, CL>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.L.total);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = static_cast<size_t>(a.L.total);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CL;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = CL > 1 ? 1 : 0;
+    return cudaLaunchKernelEx(&cfg, kern, a);
 }
 
 template <typename T, int D>
-static hga_status_t launch_t(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
-                             cudaStream_t stream) {
-    const size_t smem = sizeof(uint32_t) * (p.n_hist_chunks > 0 ? p.n_hist_chunks : 1);
-    auto kern = route_kernel<T, D>;
-    if (smem > 32 * 1024) {
-        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-        if (e != cudaSuccess) return record_cuda(e);
+cudaError_t launch_t(const RouteArgs &a, int cl, unsigned grid, cudaStream_t stream) {
+    switch (cl) {
+    case 8: return launch_cl<T, D, 8>(a, grid, stream);
+    case 4: return launch_cl<T, D, 4>(a, grid, stream);
+    case 2: return launch_cl<T, D, 2>(a, grid, stream);
+    default: return launch_cl<T, D, 1>(a, grid, stream);
     }
-    const int nqb = p.seg_len / p.q_block;
-    const unsigned grid = (unsigned)(p.batch * p.n_kv_heads * nqb);
-    const float inv_sqrt_d = (float)(1.0 / __builtin_sqrt((double)p.head_dim));
-    kern<<<grid, 256, smem, stream>>>(static_cast<const T *>(q), summ, cap, idx, p.n_q_heads, p.n_kv_heads,
-                                       p.seg_len, p.q_block, p.n_hist_chunks, p.topk, inv_sqrt_d);
-    return record_cuda(cudaGetLastError());
 }
 
+}  // namespace
+
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
-                          cudaStream_t stream) {
+                          unsigned *status, cudaStream_t stream) {
+    const int n = p.n_hist_chunks, D = p.head_dim;
+    const int nqb = p.seg_len / kQBlock;
+    const int esize = p.dtype == HGA_BF16 ? 2 : 4;
+    // cluster size: the smallest that lets one CTA's slice of the chunk list
+    // sit in the ring at once (one round of bulk copies), else the largest
+    const int ring_chunks = kRing * (kTileBytes / (D * 4));
+    int cl = 1;
+    RouteLayout L = route_layout(D, esize, 1, round4(n), n);
+    if (n > p.topk) {
+        for (int c : {1, 2, 4, 8}) {
+            if (nqb % c) continue;
+            const RouteLayout Lc = route_layout(D, esize, c, c > 1 ? round4((n + c - 1) / c) : round4(n), n);
+            if (Lc.total > kMaxSmem) continue;
+            cl = c;
+            L = Lc;
+            if ((n + c - 1) / c <= ring_chunks) break;
+        }
+    }
+    if (L.total > kMaxSmem) {
+        record_error("hga_route: shared-memory layout exceeds the per-CTA limit");
+        return HGA_ERR_UNSUPPORTED;
+    }
+    RouteArgs a{};
+    a.q = q;
+    a.summ = summ;
+    a.idx = idx;
+    a.status = status;
+    a.cap = cap;
+    a.n_q_heads = p.n_q_heads;
+    a.n_kv_heads = p.n_kv_heads;
+    a.seg_len = p.seg_len;
+    a.n = n;
+    a.topk = p.topk;
+    a.ns = cl > 1 ? round4((n + cl - 1) / cl) : round4(n);
+    a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
+    a.L = L;
+    const unsigned grid = static_cast<unsigned>(p.batch * p.n_kv_heads * nqb);
+    cudaError_t e;
     if (p.dtype == HGA_BF16)
-        return p.head_dim == 128 ? launch_t<__nv_bfloat16, 128>(p, q, summ, cap, idx, stream)
-                                 : launch_t<__nv_bfloat16, 64>(p, q, summ, cap, idx, stream);
-    return p.head_dim == 128 ? launch_t<float, 128>(p, q, summ, cap, idx, stream)
-                             : launch_t<float, 64>(p, q, summ, cap, idx, stream);
+        e = D == 128 ? launch_t<__nv_bfloat16, 128>(a, cl, grid, stream)
+                     : launch_t<__nv_bfloat16, 64>(a, cl, grid, stream);
+    else
+        e = D == 128 ? launch_t<float, 128>(a, cl, grid, stream) : launch_t<float, 64>(a, cl, grid, stream);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return record_cuda(e);
 }
 
 }  // namespace hga

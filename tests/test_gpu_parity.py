@@ -110,6 +110,75 @@ def test_route_edge_cases():
         assert hard == 0, w.name
 
 
+# route shapes reaching every selection and cluster path: k > 32 (two keys per
+# lane in the bound), and a chunk list split over clusters of 2, 4 and 8 query
+# blocks (fp32 and D = 64 included)
+ROUTE_SHAPES = [
+    gen.custom("k48_n300", topk=48, seg_len=256, seq_len=300 * 64 + 256, seg_starts=(300 * 64,), dtype="bf16",
+               head_dim=128, n_q_heads=8, n_kv_heads=2, seed=21),
+    gen.custom("k64_n65", topk=64, seg_len=128, seq_len=65 * 64 + 128, seg_starts=(65 * 64,), dtype="bf16",
+               head_dim=128, n_q_heads=4, n_kv_heads=1, seed=22),
+    gen.custom("cl2_n1100", topk=32, seg_len=128, seq_len=1100 * 64 + 128, seg_starts=(1100 * 64,),
+               dtype="bf16", head_dim=128, n_q_heads=8, n_kv_heads=2, seed=23),
+    gen.custom("cl4_n600_d64", topk=16, seg_len=256, seq_len=600 * 64 + 256, seg_starts=(600 * 64,),
+               dtype="bf16", head_dim=64, n_q_heads=4, n_kv_heads=2, seed=24),
+    gen.custom("cl8_n1100_fp32", topk=24, seg_len=512, seq_len=1100 * 64 + 512, seg_starts=(1100 * 64,),
+               dtype="fp32", head_dim=128, n_q_heads=4, n_kv_heads=1, seed=25),
+]
+
+
+def _route_only(w, q, summ):
+    """Route of one segment from host queries and fp32 summaries (device call)."""
+    import hierarchical_sparse_long_b200 as hga
+    T = w.seg_starts[0]
+    nc = T // w.chunk
+    idx = torch.full((w.batch, w.n_kv_heads, w.seg_len // w.q_block, w.topk), -7, device="cuda",
+                     dtype=torch.int32)
+    hga.hga_route(hc.params(w, T), hc.to_dev(q, w), summ, nc, idx)
+    torch.cuda.synchronize()
+    return hc.f32(idx).astype(np.int32)
+
+
+@pytest.mark.parametrize("w", ROUTE_SHAPES, ids=[w.name for w in ROUTE_SHAPES])
+def test_route_selection_and_cluster_paths(w):
+    import hierarchical_sparse_long_b200 as hga
+    T, S = w.seg_starts[0], w.seg_len
+    q = gen.queries(w, T, T + S)
+    k = gen.keys(w, 0, T)
+    nc = T // w.chunk
+    summ = torch.zeros(w.batch, w.n_kv_heads, nc, w.head_dim, device="cuda")
+    hga.hga_build_summaries(hc.to_dev(k, w), T, w.batch, w.n_kv_heads, w.head_dim, w.chunk, 0, nc, summ, nc)
+    idx = _route_only(w, q, summ)
+    _, _, idx_o, gap = hc.oracle_route(w, dict(T=T, q=q, k_all=k))
+    hard, exempt = hc.route_mismatches(idx, idx_o, gap)
+    print(f"{w.name}: near-tie exemptions {exempt}")
+    assert hard == 0
+
+
+def test_route_banded_and_equal_scores():
+    """Scores banded by chunk index mod 256 leave hundreds of chunks at or
+    above the selection's per-thread-maximum bound (several candidates per
+    thread); all-equal summaries tie every chunk at the bound, so the
+    selection falls back to the whole-row radix select and must route the
+    lowest chunk indices."""
+    n = 4096
+    w = gen.custom("banded", topk=32, seg_len=128, seq_len=n * 64 + 128, seg_starts=(n * 64,),
+                   dtype="bf16", head_dim=128, n_q_heads=4, n_kv_heads=1)
+    q = np.zeros((1, 4, 128, 128), np.float32)
+    q[..., 0] = 1.0  # block summary = e_0, so score_j = summ[j][0] / sqrt(D)
+    rng = np.random.default_rng(5)
+    summ = np.zeros((1, 1, n, 128), np.float32)
+    summ[..., 0] = (np.arange(n) % 256) + rng.permutation(n) / n * 0.5  # distinct, banded
+    idx = _route_only(w, q, torch.from_numpy(summ).cuda())
+    idx_o, gap, _ = oracle.route(hc.oracle_shape(w, n * 64), q, summ)
+    assert np.array_equal(idx, idx_o)
+    assert np.all(np.sort(summ[0, 0, idx[0, 0, 0], 0]) == np.sort(summ[0, 0, :, 0])[-32:])
+
+    same = np.broadcast_to(rng.standard_normal(128).astype(np.float32), (1, 1, n, 128)).copy()
+    idx = _route_only(w, q, torch.from_numpy(same).cuda())
+    assert np.array_equal(idx, np.broadcast_to(np.arange(32, dtype=np.int32), idx.shape))
+
+
 # ---------------------------------------------------------------- forward
 
 def test_fwd_tiny_fp32_full():
