@@ -22,6 +22,8 @@ with the recipe of inputs/gen.py):
 
 Metric: query tokens/s (active query tokens processed per second, all heads),
 device-timed with CUDA events, L2 flushed (256 MiB write) before every step.
+Device-resident workloads capture one step as a CUDA graph and replay it (the
+phase events are recorded inside the graph); the tiered workload runs eagerly.
 Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle.
 """
 from __future__ import annotations
@@ -336,15 +338,18 @@ class Layer:
 
 
 class PhaseEvents:
-    """CUDA events on the launching (current) stream between the phases of a step."""
+    """CUDA events on the launching (current) stream between the phases of a
+    step.  With external=True the events become event-record nodes when the
+    step is captured into a CUDA graph, and every replay re-records them."""
 
-    def __init__(self):
+    def __init__(self, external=False):
         import torch
         self.torch = torch
+        self.external = external
         self.marks = []
 
     def record(self, name):
-        e = self.torch.cuda.Event(enable_timing=True)
+        e = self.torch.cuda.Event(enable_timing=True, external=self.external)
         e.record()
         self.marks.append((name, e))
 
@@ -481,6 +486,18 @@ def run_hga(args, rank, world, local):
     torch.cuda.synchronize()
     if hga.hga_get_device_status() != 0:
         raise RuntimeError("device status reported an error during warm-up")
+    # Device-resident workloads replay one step captured as a CUDA graph (one
+    # host launch per step, phase events recorded inside the graph); the tiered
+    # workload drives its copy stream from the host and stays eager.
+    graph, gev = None, None
+    if not w.tiered:
+        gev = PhaseEvents(external=True)
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph):
+            graph_launches = layer.step(ev=gev)
+        flush_l2(flush)
+        graph.replay()
+        torch.cuda.synchronize()
     sampler = ClockSampler(local)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -493,11 +510,19 @@ def run_hga(args, rank, world, local):
     time.sleep(0.3)
     for s in range(args.steps):
         flush_l2(flush)
-        ev = PhaseEvents()
-        starts[s].record()
-        launches += layer.step(ev=ev)
-        ends[s].record()
-        phases.append(ev)
+        if graph is not None:
+            starts[s].record()
+            graph.replay()
+            ends[s].record()
+            launches += graph_launches
+            ends[s].synchronize()  # outside the timed window: read this replay's phase events
+            phases.append(gev.totals())
+        else:
+            ev = PhaseEvents()
+            starts[s].record()
+            launches += layer.step(ev=ev)
+            ends[s].record()
+            phases.append(ev)
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
@@ -509,7 +534,7 @@ def run_hga(args, rank, world, local):
     # per-kernel device time over the timed steps (events on the launching stream)
     ph = {}
     for ev in phases:
-        for k, v in ev.totals().items():
+        for k, v in (ev if isinstance(ev, dict) else ev.totals()).items():
             ph[k] = ph.get(k, 0.0) + v
     n_seg = len(w.seg_starts) * args.steps
     peaks, peak_src = measured_peaks()
@@ -550,7 +575,8 @@ def run_hga(args, rank, world, local):
                        "chunk": w.chunk, "q_block": w.q_block, "segments_per_step": len(w.seg_starts),
                        "backward": w.backward, "tiered": w.tiered,
                        "parallelism": f"one independent layer per GPU x{world}",
-                       "l2": "flushed before every timed step (256 MiB write)"},
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "launch": "one CUDA graph replay per step" if graph is not None else "eager"},
             "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
             "device_status": status}
     if w.tiered:

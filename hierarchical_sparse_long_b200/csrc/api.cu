@@ -1,6 +1,7 @@
 // C ABI of the HGA library: argument validation, kernel selection and the
 // device status word.  Every check runs on the host before anything is
 // enqueued, so a rejected call leaves the stream untouched.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -16,7 +17,7 @@ __device__ unsigned int g_status_word;
 thread_local std::string t_last_error;
 
 constexpr int kMaxDevices = 64;
-unsigned *g_status_ptr[kMaxDevices];
+std::atomic<unsigned *> g_status_ptr[kMaxDevices];
 std::mutex g_status_mu;
 
 // Address of this device's status word (looked up once per device with the
@@ -24,13 +25,14 @@ std::mutex g_status_mu;
 unsigned *status_ptr() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+    if (unsigned *p = g_status_ptr[dev].load(std::memory_order_acquire)) return p;
     std::lock_guard<std::mutex> lock(g_status_mu);
-    if (!g_status_ptr[dev]) {
+    if (!g_status_ptr[dev].load(std::memory_order_relaxed)) {
         void *ptr = nullptr;
         if (cudaGetSymbolAddress(&ptr, g_status_word) != cudaSuccess) return nullptr;
-        g_status_ptr[dev] = static_cast<unsigned *>(ptr);
+        g_status_ptr[dev].store(static_cast<unsigned *>(ptr), std::memory_order_release);
     }
-    return g_status_ptr[dev];
+    return g_status_ptr[dev].load(std::memory_order_relaxed);
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

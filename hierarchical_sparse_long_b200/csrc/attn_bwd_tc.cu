@@ -27,7 +27,6 @@
 // Every wait is bounded and every warp-collective TMEM access is made from a
 // converged warp with warp-uniform decisions.
 #include <cudaTypedefs.h>
-#include <mutex>
 
 #include "tc_ptx.cuh"
 
@@ -574,28 +573,8 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool get_encoder() {
-    std::call_once(g_encode_once, [] {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    return g_encode != nullptr;
-}
-
 bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, 64};
-    const cuuint32_t estr[2] = {1, 1};
-    return g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
-                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    return tma_rows_map(map, base, rows);
 }
 
 // One launch for both gradient passes: the first n_kv_ctas blocks run the
@@ -621,7 +600,7 @@ hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUte
                         const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
     auto kern = bwd_tc_kernel<NH>;
     const size_t smem = DqSmem<NH>::ALLOC > DkvSmem::ALLOC ? DqSmem<NH>::ALLOC : DkvSmem::ALLOC;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const int n_bg = p.batch * p.n_kv_heads;
     const int n_kv_ctas = ((p.seg_len + 127) / 128) * n_bg;
@@ -640,7 +619,7 @@ bool attn_bwd_tc_supported(const hga_params_t &p) {
     if (n_bg * (p.hist_head_stride > p.seg_head_stride ? p.hist_head_stride : p.seg_head_stride) >= (1ll << 31))
         return false;
     if ((long long)p.batch * p.n_q_heads * p.seg_len >= (1ll << 31)) return false;
-    return get_encoder();
+    return tma_encoder_available();
 }
 
 hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,

@@ -12,27 +12,28 @@
 // then the active segment's causal tiles 0..m) is read once for G heads,
 // which is what lifts a history tile from 64 to 256 flop/byte.
 //
-// Warp roles (NH = 2: 384 threads):
-//   warps 0, 2  TMA producers: Q once and the K tiles (warp 0), the V tiles
-//               (warp 2), each into its own 3-stage ring (routed chunk j ->
-//               TMA row coordinate (b*Hkv+g)*stride + 64 j); a K stage is
-//               released as soon as QK^T of its tile completes, a V stage
-//               after PV, so K loads run well ahead of the softmax.
-//   warps 1, 3  UMMA issuers, one thread per M half (warp 1 also owns TMEM):
-//               S_h = Q_h K^T   (M128 N64 K128, K-major A and B, SW128)
-//               O_h += P_h V    (M128 N128 K64, P K-major, V MN-major)
-//               QK^T of tile j is issued before PV of tile j-1 so the tensor
-//               core works while the softmax warps run.
-//   warps 4+4h  softmax of half h: one TMEM lane (= query row) per thread;
+// Warp roles (NH = 2: 512 threads, warps 5-7 idle):
+//   warp 0      TMA producer: Q once, then K and V of every tile, each into
+//               its own 5-stage ring (routed chunk j -> TMA row coordinate
+//               (b*Hkv+g)*stride + 64 j); a K stage is released as soon as
+//               QK^T of its tile completes, a V stage after PV.
+//   warps 1, 3  QK issuers, one thread per M half (warp 1 also owns TMEM):
+//               S_h = Q_h K^T   (M128 N64 K128, K-major A and B, SW128), into
+//               one of two S buffers once PV two tiles back has read the P
+//               stored there.
+//   warps 2, 4  PV issuers, one thread per M half:
+//               O_h += P_h V    (M128 N128 K64, P from TMEM, V MN-major),
+//               issued as soon as the softmax has written P.  One thread
+//               issues a tcgen05.mma only about every 100 cycles, so the four
+//               issue streams run in separate threads.
+//   warps 8+4h  softmax of half h: one TMEM lane (= query row) per thread;
 //               online softmax in the log2 domain, O rescaled in TMEM when
-//               the row max grows by more than 2^8, P written as bf16 in the
-//               SW128 K-major layout the next UMMA reads, into one of two
-//               buffers so tile j+1's softmax never waits for PV(j).
+//               the row max grows by more than 2^8, P written as bf16 pairs
+//               into the tile's S buffer, where the PV issue reads it.
 // TMEM (512 columns): O_h at 128h, S_h double-buffered at 256 + 128h + 64b.
 // Every wait is bounded; a timeout sets HGA_DEV_TIMEOUT and the CTA unwinds.
 #include <cudaTypedefs.h>
 #include <cstdlib>
-#include <mutex>
 
 #include "tc_ptx.cuh"
 
@@ -73,18 +74,19 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
 struct Bars {
     uint64_t q_full;
     uint64_t k_full[NSTAGE];
-    uint64_t k_empty[NSTAGE];  // released once QK^T of the tile completes
+    uint64_t k_empty[NSTAGE];  // released once QK^T of the tile completes (both halves)
     uint64_t v_full[NSTAGE];
-    uint64_t v_empty[NSTAGE];  // released once PV of the tile completes
-    uint64_t s_full[2][2];
+    uint64_t v_empty[NSTAGE];  // released once PV of the tile completes (both halves)
+    uint64_t s_full[2][2];  // [half][S/P buffer]: S of the buffer's tile in TMEM
     uint64_t p_full[2][2];  // [half][S/P buffer]: P of the buffer's tile written to TMEM
     uint64_t o_done[2][2];  // [half][S/P buffer]: PV of the buffer's tile completed
-    uint64_t drain[2];
+    uint64_t drain[4];      // one per issuing thread (abort path)
     uint32_t tmem_base;
     int abort;
     int n_hist;
-    int issued_k;
+    int issued_k;  // K / V tiles the producer issued
     int issued_v;
+    int sm0_tiles;  // tiles whose softmax half 0 has finished (scheduling hint)
     int tiles[64];
 };
 
@@ -99,8 +101,33 @@ struct FwdArgs {
     float scale_log2;  // log2(e) / sqrt(D)
 };
 
+// Two control warpgroups (producer, QK0, PV0, QK1, PV1, three idle warps) and
+// NH softmax warpgroups.  With NH = 2 the 512 threads launch at 128 registers
+// each; the control warpgroups give registers back and the softmax
+// warpgroups take them: 8 x 32 x 56 + 8 x 32 x 200 = 65,536, the launch total.
+// Bounded wait until the shared counter reaches `target` (same contract as mbar_wait).
+__device__ __forceinline__ bool wait_count(int *counter, int target, volatile int *abort, unsigned *status) {
+    volatile int *c = counter;
+    if (*c >= target) return true;
+    const long long t0 = clock64();
+    while (*c < target) {
+        if (*abort) return false;
+        if (clock64() - t0 > (1ll << 31)) {
+            *abort = 1;
+            atomicOr(status, kDevTimeout);
+            return false;
+        }
+    }
+    return true;
+}
+
+constexpr int kCtrlWarps = 8;
+constexpr int kCtrlRegs = 56;
+constexpr int kSoftmaxRegs = 200;
+static_assert(8 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs == 512 * 128, "register split must match the launch");
+
 template <int NH, int POLY>
-__global__ void __launch_bounds__(128 + 128 * NH, 1)
+__global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                        const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
                        const __grid_constant__ CUtensorMap tm_vs, const FwdArgs a) {
@@ -126,19 +153,16 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             tc::mbar_init(&bars->v_full[s], 1);
             tc::mbar_init(&bars->v_empty[s], NH);
         }
-        bars->issued_k = 0;
-        bars->issued_v = 0;
-        for (int h = 0; h < 2; ++h) {
+        for (int h = 0; h < 2; ++h)
             for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->s_full[h][bb], 1);
-            }
-            for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->p_full[h][bb], 4);
                 tc::mbar_init(&bars->o_done[h][bb], 1);
             }
-        }
-        tc::mbar_init(&bars->drain[0], 1);
-        tc::mbar_init(&bars->drain[1], 1);
+        for (int d = 0; d < 4; ++d) tc::mbar_init(&bars->drain[d], 1);
+        bars->issued_k = 0;
+        bars->issued_v = 0;
+        bars->sm0_tiles = 0;
         bars->abort = 0;
         tc::fence_mbar_init();
     }
@@ -162,37 +186,16 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
     const int n_tiles = n_hist + m + 1;
     volatile int *abort = &bars->abort;
 
-    // TMA producer of one ring: K tiles (released after QK^T) or V tiles
-    // (released after PV); each routed chunk j is row (b*Hkv+g)*stride + 64 j.
-    auto produce = [&](bool key) {
-        const CUtensorMap *mh = key ? &tm_kh : &tm_vh;
-        const CUtensorMap *ms = key ? &tm_ks : &tm_vs;
-        uint64_t *full = key ? bars->k_full : bars->v_full;
-        uint64_t *empty = key ? bars->k_empty : bars->v_empty;
-        uint8_t *ring = smem + (key ? L::K : L::V);
-        int issued = 0;
-        for (int j = 0; j < n_tiles; ++j) {
-            const int s = j % NSTAGE, u = j / NSTAGE;
-            if (j >= NSTAGE && !tc::mbar_wait(&empty[s], (u - 1) & 1, abort, a.status)) break;
-            const bool hist = j < n_hist;
-            const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
-                                 : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
-            uint8_t *dst = ring + s * KV_TILE_BYTES;
-            tc::mbar_arrive_expect_tx(&full[s], KV_TILE_BYTES);
-            tc::tma_load_2d(dst, hist ? mh : ms, 0, row, &full[s]);
-            tc::tma_load_2d(dst + 64 * 128, hist ? mh : ms, 64, row, &full[s]);
-            ++issued;
-        }
-        if (key) bars->issued_k = issued;
-        else bars->issued_v = issued;
-    };
-
+    if (warp < kCtrlWarps) {
+        if constexpr (NH == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (warp == 0) {
         if (lane == 0) {
-            // ---------------------------------------------------------- TMA producer (Q, K)
+            // ------------------------------------------------------------ TMA producer
             tc::tma_prefetch_desc(&tm_q);
             tc::tma_prefetch_desc(&tm_kh);
             tc::tma_prefetch_desc(&tm_ks);
+            tc::tma_prefetch_desc(&tm_vh);
+            tc::tma_prefetch_desc(&tm_vs);
             tc::mbar_arrive_expect_tx(&bars->q_full, NH * Q_HALF_BYTES);
             for (int hh = 0; hh < G; ++hh) {
                 const int qrow = (b * a.n_q_heads + g * G + hh) * a.seg_len + m * TILE;
@@ -200,71 +203,93 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
                 tc::tma_load_2d(dst, &tm_q, 0, qrow, &bars->q_full);
                 tc::tma_load_2d(dst + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
             }
-            produce(true);
+            // K(j), then V(j): a K stage frees once QK^T(j - NSTAGE) completes, a V
+            // stage once PV(j - NSTAGE) does; routed chunk j is row (b*Hkv+g)*stride + 64 j
+            int nk = 0, nv = 0;
+            for (int j = 0; j < n_tiles; ++j) {
+                const int s = j % NSTAGE, u = j / NSTAGE;
+                const bool hist = j < n_hist;
+                const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
+                                     : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+                if (j >= NSTAGE && !tc::mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort, a.status)) break;
+                uint8_t *kdst = smem + L::K + s * KV_TILE_BYTES;
+                tc::mbar_arrive_expect_tx(&bars->k_full[s], KV_TILE_BYTES);
+                tc::tma_load_2d(kdst, hist ? &tm_kh : &tm_ks, 0, row, &bars->k_full[s]);
+                tc::tma_load_2d(kdst + 64 * 128, hist ? &tm_kh : &tm_ks, 64, row, &bars->k_full[s]);
+                nk = j + 1;
+                if (j >= NSTAGE && !tc::mbar_wait(&bars->v_empty[s], (u - 1) & 1, abort, a.status)) break;
+                uint8_t *vdst = smem + L::V + s * KV_TILE_BYTES;
+                tc::mbar_arrive_expect_tx(&bars->v_full[s], KV_TILE_BYTES);
+                tc::tma_load_2d(vdst, hist ? &tm_vh : &tm_vs, 0, row, &bars->v_full[s]);
+                tc::tma_load_2d(vdst + 64 * 128, hist ? &tm_vh : &tm_vs, 64, row, &bars->v_full[s]);
+                nv = j + 1;
+            }
+            bars->issued_k = nk;
+            bars->issued_v = nv;
         }
-    } else if (warp == 2) {
-        if (lane == 0) produce(false);  // V tiles, independent of the K ring
-    } else if (warp == 1 || warp == 3) {
+    } else if (warp < kCtrlWarps) {
         // ------------------------------------------------------------ UMMA issuers
-        // One issuing thread per 128-row half (warp 1: half 0, warp 3: half 1):
-        // a single thread can only issue a tcgen05.mma every ~100 cycles, so the
-        // halves' MMAs are issued by two threads that the tensor core serves
-        // concurrently.
-        const int h = warp == 1 ? 0 : 1;
-        if (lane == 0 && h < NH) {
+        const int h = (warp - 1) >> 1;      // M half
+        const bool qk = (warp & 1) != 0;    // warps 1, 3: QK^T; warps 2, 4: PV
+        if (lane == 0 && warp <= 4 && h < NH) {
             // Descriptors are built once; a K-step, stage or buffer offset is added
             // to the start-address field (addresses stay below 2^18, so no carry).
-            const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * Q_HALF_BYTES, 16, 1024);
-            const uint64_t k_desc = tc::desc_sw128(sbase + L::K, 16, 1024);
-            const uint64_t v_desc = tc::desc_sw128(sbase + L::V, 8192, 1024);
-            const uint32_t o_tmem = tmem + 128 * h;
-            // O_h += P_h(t) V(t) once the softmax of tile t has written P buffer t&1
-            auto issue_pv = [&](int t) -> bool {
-                const int s = t % NSTAGE, pb = t & 1;
-                if (!tc::mbar_wait(&bars->v_full[s], (t / NSTAGE) & 1, abort, a.status)) return false;
-                if (!tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort, a.status)) return false;
-                tc::fence_after_sync();
-                const uint64_t vd = v_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
-                // P(t) as bf16 pairs in the first 32 columns of S buffer pb: 8 columns per K step
-                const uint32_t pa = tmem + 256 + 128 * h + 64 * pb;
+            bool ok = true;
+            if (qk) {
+                const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * Q_HALF_BYTES, 16, 1024);
+                const uint64_t k_desc = tc::desc_sw128(sbase + L::K, 16, 1024);
+                ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
+                for (int j = 0; ok && j < n_tiles; ++j) {
+                    const int s = j % NSTAGE, bb = j & 1;
+                    if (!tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)) break;
+                    // S buffer bb is free once PV(j-2), which read P(j-2) from it, has completed
+                    if (j >= 2 && !tc::mbar_wait(&bars->o_done[h][bb], ((j >> 1) - 1) & 1, abort, a.status))
+                        break;
+                    // half 1 runs half a tile behind half 0: its S(j) lands while half 0
+                    // is in the exp phase of tile j, so the two softmax groups take
+                    // turns on the MUFU instead of stalling on it together
+                    if (h == 1 && j >= 1 && !wait_count(&bars->sm0_tiles, j, abort, a.status)) break;
+                    tc::fence_after_sync();
+                    const uint64_t kd = k_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    mma_f16_ts(o_tmem, pa + 8 * kk, vd + (kk * 2048 >> 4), IDESC_PV, (t > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&bars->o_done[h][pb]);
-                tc::mma_commit(&bars->v_empty[s]);  // one arrival per half
-                return true;
-            };
-            bool ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int s = j % NSTAGE, bb = j & 1;
-                if (!tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)) { ok = false; break; }
-                // S buffer bb is free once PV(j-2), which read P(j-2) from it, has completed
-                if (j >= 2 && !tc::mbar_wait(&bars->o_done[h][bb], ((j >> 1) - 1) & 1, abort, a.status)) {
-                    ok = false;
-                    break;
+                    for (int kk = 0; kk < D / 16; ++kk) {
+                        const uint32_t koff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+                        const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                        tc::mma_f16(tmem + 256 + 128 * h + 64 * bb, q_desc + qoff, kd + koff, IDESC_QK,
+                                    kk > 0 ? 1u : 0u);
+                    }
+                    tc::mma_commit(&bars->s_full[h][bb]);
+                    tc::mma_commit(&bars->k_empty[s]);  // one arrival per half
                 }
-                tc::fence_after_sync();
-                const uint64_t kd = k_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
+            } else {
+                const uint64_t v_desc = tc::desc_sw128(sbase + L::V, 8192, 1024);
+                const uint32_t o_tmem = tmem + 128 * h;
+                for (int t = 0; t < n_tiles; ++t) {
+                    const int s = t % NSTAGE, pb = t & 1;
+                    if (!tc::mbar_wait(&bars->v_full[s], (t / NSTAGE) & 1, abort, a.status)) break;
+                    if (!tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort, a.status)) break;
+                    tc::fence_after_sync();
+                    const uint64_t vd = v_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
+                    // P(t) as bf16 pairs in the first 32 columns of S buffer pb: 8 columns per K step
+                    const uint32_t pa = tmem + 256 + 128 * h + 64 * pb;
 #pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t koff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
-                    const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                    tc::mma_f16(tmem + 256 + 128 * h + 64 * bb, q_desc + qoff, kd + koff, IDESC_QK,
-                                kk > 0 ? 1u : 0u);
+                    for (int kk = 0; kk < TILE / 16; ++kk)
+                        mma_f16_ts(o_tmem, pa + 8 * kk, vd + (kk * 2048 >> 4), IDESC_PV,
+                                   (t > 0 || kk > 0) ? 1u : 0u);
+                    tc::mma_commit(&bars->o_done[h][pb]);
+                    tc::mma_commit(&bars->v_empty[s]);  // one arrival per half
                 }
-                tc::mma_commit(&bars->s_full[h][bb]);
-                tc::mma_commit(&bars->k_empty[s]);  // one arrival per half
-                if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
             }
-            if (ok) issue_pv(n_tiles - 1);
         }
-    } else if (warp >= 4) {
+    }
+    } else {
         // -------------------------------------------------------------- softmax / epilogue
-        const int h = (warp - 4) >> 2;        // M half
-        const int quad = warp & 3;            // TMEM lane quadrant this warp may access
-        const int r = quad * 32 + lane;       // row within the half = TMEM lane
-        const int hh = 2 * h + (r >> 6);      // head within the group
-        const int i = r & 63;                 // query row within the block
+        if constexpr (NH == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
+        const int h = (warp - kCtrlWarps) >> 2;  // M half
+        const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;          // row within the half = TMEM lane
+        const int hh = 2 * h + (r >> 6);         // head within the group
+        const int i = r & 63;                    // query row within the block
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const uint32_t o_addr = tmem + lane_addr + 128 * h;
         float m_run = -INFINITY, l_run = 0.f;
@@ -359,6 +384,7 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->p_full[h][pb]);
+            if (NH == 2 && warp == kCtrlWarps && lane == 0) *reinterpret_cast<volatile int *>(&bars->sm0_tiles) = j + 1;
         }
         if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][(n_tiles - 1) & 1],
                                                         ((n_tiles - 1) >> 1) & 1, abort, a.status))) {
@@ -391,17 +417,18 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
         // a wait gave up: let the copies and UMMAs still in flight finish before
         // shared memory and TMEM are released
         int never = 0;
-        if ((warp == 0 || warp == 2) && lane == 0) {
-            const bool key = warp == 0;
-            const int issued = key ? bars->issued_k : bars->issued_v;
-            uint64_t *full = key ? bars->k_full : bars->v_full;
-            for (int j = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; j < issued; ++j)
-                tc::mbar_wait(&full[j % NSTAGE], (j / NSTAGE) & 1, &never, a.status, 1ll << 28);
-            if (key) tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
+        if (warp == 0 && lane == 0) {
+            for (int pass = 0; pass < 2; ++pass) {
+                const int issued = pass == 0 ? bars->issued_k : bars->issued_v;
+                uint64_t *full = pass == 0 ? bars->k_full : bars->v_full;
+                for (int j = issued - NSTAGE < 0 ? 0 : issued - NSTAGE; j < issued; ++j)
+                    tc::mbar_wait(&full[j % NSTAGE], (j / NSTAGE) & 1, &never, a.status, 1ll << 28);
+            }
+            tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
         }
-        if ((warp == 1 || (warp == 3 && NH == 2)) && lane == 0) {
-            tc::mma_commit(&bars->drain[warp == 3]);
-            tc::mbar_wait(&bars->drain[warp == 3], 0, &never, a.status, 1ll << 28);
+        if (warp >= 1 && warp <= 4 && lane == 0 && ((warp - 1) >> 1) < NH) {
+            tc::mma_commit(&bars->drain[warp - 1]);
+            tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
         }
         __syncwarp();
         tc::fence_after_sync();
@@ -413,30 +440,8 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
 }
 
 // ------------------------------------------------------------------ host side
-PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
-std::once_flag g_encode_once;
-
-bool get_encoder() {
-    std::call_once(g_encode_once, [] {
-        void *fn = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
-    });
-    return g_encode != nullptr;
-}
-
-// 2D map over rows of D bf16 values (256 B each), 64 x 64 boxes, 128-byte swizzle.
 bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
-    const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows};
-    const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
-    const cuuint32_t box[2] = {64, 64};
-    const cuuint32_t estr[2] = {1, 1};
-    CUresult r = g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
-                          estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                          CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return tma_rows_map(map, base, rows);
 }
 
 template <int NH>
@@ -483,11 +488,11 @@ hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, con
     }();
     auto kern = poly == 2 ? attn_fwd_tc_kernel<NH, 2> : poly == 0 ? attn_fwd_tc_kernel<NH, 0>
                                                                    : attn_fwd_tc_kernel<NH, 1>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const unsigned grid = (unsigned)(a.n_blocks * n_bg);
     if (grid == 0) return HGA_OK;
-    kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
+    kern<<<grid, 32 * kCtrlWarps + 128 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
     return record_cuda(cudaGetLastError());
 }
 
@@ -502,7 +507,7 @@ bool attn_fwd_tc_supported(const hga_params_t &p) {
     if (n_bg * (p.hist_head_stride > p.seg_head_stride ? p.hist_head_stride : p.seg_head_stride) >= (1ll << 31))
         return false;
     if ((long long)p.batch * p.n_q_heads * p.seg_len >= (1ll << 31)) return false;
-    return get_encoder();
+    return tma_encoder_available();
 }
 
 hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,

@@ -399,7 +399,7 @@ static hga_status_t fwd_t(const hga_params_t &p, const void *q, const void *kh, 
                           cudaStream_t stream) {
     const size_t smem = sizeof(float) * (3 * TILE * (D + 1) + TILE * 65);
     auto kern = fwd_simt_kernel<T, D>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const int nqb = p.seg_len / p.q_block;
     const int qb0 = p.qblock_end > 0 ? p.qblock_begin : 0;
@@ -424,7 +424,7 @@ static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, 
     {
         const size_t smem = sizeof(float) * (4 * TILE * (D + 1) + TILE * 65);
         auto kern = bwd_dq_simt_kernel<T, D>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
         if (e != cudaSuccess) return record_cuda(e);
         kern<<<(unsigned)(nqb * p.batch * p.n_q_heads), NT, smem, stream>>>(
             p, (const T *)q, (const T *)kh, (const T *)vh, (const T *)ks, (const T *)vs, idx, lse, delta,
@@ -435,7 +435,7 @@ static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, 
     {
         const size_t smem = sizeof(float) * (4 * TILE * (D + 1) + 2 * TILE * 65);
         auto kern = bwd_dkdv_simt_kernel<T, D>;
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
         if (e != cudaSuccess) return record_cuda(e);
         kern<<<(unsigned)(nqb * p.batch * p.n_kv_heads), NT, smem, stream>>>(
             p, (const T *)q, (const T *)ks, (const T *)vs, lse, delta, (const T *)dout, (float *)dk, (float *)dv);

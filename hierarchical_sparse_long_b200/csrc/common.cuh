@@ -2,6 +2,7 @@
 #pragma once
 
 #include <cstdint>
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
@@ -82,4 +83,12 @@ hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, cons
 hga_status_t launch_selftest_wait_timeout(long long wait_cycles, unsigned *status, cudaStream_t stream);
 hga_status_t record_cuda(cudaError_t e);
 void record_error(const char *msg);
+
+// Host helpers shared by the launchers (host.cu).
+bool tma_encoder_available();
+// 2-D TMA map over `rows` rows of 128 bf16 values (256 B), 64 x 64 boxes,
+// 128-byte swizzle; maps are cached per thread by (base, rows).
+bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows);
+// cudaFuncAttributeMaxDynamicSharedMemorySize, set once per kernel and device.
+cudaError_t set_max_dynamic_smem(const void *kernel, int bytes);
 }  // namespace hga

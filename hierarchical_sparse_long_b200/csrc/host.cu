@@ -1,0 +1,84 @@
+// Host-side helpers shared by the launchers: TMA tensor maps over rows of
+// 128 bf16 values (cached per thread, since encoding one is a driver call on
+// every launch otherwise) and the per-device dynamic shared-memory attribute
+// of a kernel (set once per kernel and device).
+#include <cudaTypedefs.h>
+#include <mutex>
+#include <utility>
+#include <vector>
+
+#include "common.cuh"
+
+namespace hga {
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+std::once_flag g_encode_once;
+
+struct MapEntry {
+    const void *base;
+    unsigned long long rows;
+    CUtensorMap map;
+};
+constexpr int kMapCache = 16;
+thread_local MapEntry t_maps[kMapCache];
+thread_local int t_map_next = 0;
+
+std::mutex g_attr_mu;
+std::vector<std::pair<std::pair<const void *, int>, int>> g_attr;  // (kernel, device) -> bytes set
+
+}  // namespace
+
+bool tma_encoder_available() {
+    std::call_once(g_encode_once, [] {
+        void *fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+    });
+    return g_encode != nullptr;
+}
+
+bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows) {
+    for (const MapEntry &e : t_maps)
+        if (e.base == base && e.rows == rows && base != nullptr) {
+            *map = e.map;
+            return true;
+        }
+    if (!tma_encoder_available()) return false;
+    const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    const cuuint64_t strides[1] = {128 * 2};
+    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t estr[2] = {1, 1};
+    if (g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    MapEntry &slot = t_maps[t_map_next];
+    t_map_next = (t_map_next + 1) % kMapCache;
+    slot.base = base;
+    slot.rows = rows;
+    slot.map = *map;
+    return true;
+}
+
+cudaError_t set_max_dynamic_smem(const void *kernel, int bytes) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(g_attr_mu);
+    for (auto &kv : g_attr)
+        if (kv.first.first == kernel && kv.first.second == dev) {
+            if (kv.second >= bytes) return cudaSuccess;
+            e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+            if (e == cudaSuccess) kv.second = bytes;
+            return e;
+        }
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) g_attr.push_back({{kernel, dev}, bytes});
+    return e;
+}
+
+}  // namespace hga

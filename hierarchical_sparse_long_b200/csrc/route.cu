@@ -504,7 +504,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
 template <typename T, int D, int CL>
 cudaError_t launch_cl(const RouteArgs &a, unsigned grid, cudaStream_t stream) {
     auto kern = route_kernel<T, D, CL>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, a.L.total);
+    cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), a.L.total);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(grid);
