@@ -46,7 +46,7 @@ CSRC = "hierarchical_sparse_long_b200/csrc/"
 KERNEL_SOURCES = {
     "attn_fwd": [CSRC + "attn_fwd_tc.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
     "attn_bwd": [CSRC + "attn_bwd_tc.cu", CSRC + "attn_simt.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
-    "route": [CSRC + "route.cu", CSRC + "common.cuh"],
+    "route": [CSRC + "route.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
     "summaries": [CSRC + "summaries.cu", CSRC + "common.cuh"],
     "fetch": [CSRC + "tiered.cu", CSRC + "common.cuh"],
 }
