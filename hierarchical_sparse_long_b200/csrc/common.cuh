@@ -86,9 +86,10 @@ void record_error(const char *msg);
 
 // Host helpers shared by the launchers (host.cu).
 bool tma_encoder_available();
-// 2-D TMA map over `rows` rows of 128 bf16 values (256 B), 64 x 64 boxes,
-// 128-byte swizzle; maps are cached per thread by (base, rows).
-bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows);
+// 2-D TMA map over `rows` rows of 128 bf16 values (256 B), boxes of 64 values
+// x box_rows rows, 128-byte swizzle; maps are cached per thread by
+// (base, rows, box_rows).
+bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows, unsigned box_rows = 64);
 // cudaFuncAttributeMaxDynamicSharedMemorySize, set once per kernel and device.
 cudaError_t set_max_dynamic_smem(const void *kernel, int bytes);
 }  // namespace hga

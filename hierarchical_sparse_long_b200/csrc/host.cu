@@ -19,6 +19,7 @@ std::once_flag g_encode_once;
 struct MapEntry {
     const void *base;
     unsigned long long rows;
+    unsigned box_rows;
     CUtensorMap map;
 };
 constexpr int kMapCache = 16;
@@ -41,16 +42,16 @@ bool tma_encoder_available() {
     return g_encode != nullptr;
 }
 
-bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows) {
+bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows, unsigned box_rows) {
     for (const MapEntry &e : t_maps)
-        if (e.base == base && e.rows == rows && base != nullptr) {
+        if (e.base == base && e.rows == rows && e.box_rows == box_rows && base != nullptr) {
             *map = e.map;
             return true;
         }
     if (!tma_encoder_available()) return false;
     const cuuint64_t dims[2] = {128, (cuuint64_t)rows};
     const cuuint64_t strides[1] = {128 * 2};
-    const cuuint32_t box[2] = {64, 64};
+    const cuuint32_t box[2] = {64, box_rows};
     const cuuint32_t estr[2] = {1, 1};
     if (g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box, estr,
                  CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -60,6 +61,7 @@ bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows) {
     t_map_next = (t_map_next + 1) % kMapCache;
     slot.base = base;
     slot.rows = rows;
+    slot.box_rows = box_rows;
     slot.map = *map;
     return true;
 }
