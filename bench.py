@@ -24,6 +24,8 @@ Metric: query tokens/s (active query tokens processed per second, all heads),
 device-timed with CUDA events, L2 flushed (256 MiB write) before every step.
 Device-resident workloads capture one step as a CUDA graph and replay it (the
 phase events are recorded inside the graph); the tiered workload runs eagerly.
+Each segment's summary append, which reads only the segment's keys, runs on a
+side stream next to the segment's route (``--serial-append``: after attention).
 Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle.
 """
 from __future__ import annotations
@@ -61,6 +63,9 @@ def parse():
     ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
     ap.add_argument("--workload", default="qwen3_16k_fwd", choices=WORKLOADS)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--serial-append", action="store_true",
+                    help="run each segment's summary append after its attention on the main stream "
+                         "(default: on a side stream, overlapped with the route)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     return ap.parse_args()
 
@@ -211,6 +216,8 @@ class Layer:
             self.dv = torch.empty_like(self.dk)
             self.ws = torch.empty(hga.hga_attn_bwd_workspace_size(self.params(w.seg_starts[-1])) // 4 + 64,
                                   device=dev)
+        self.side = torch.cuda.Stream()
+        self.side_append = False
         if w.tiered:
             self._init_tiered()
         self.reset()
@@ -235,12 +242,27 @@ class Layer:
 
     def segment(self, T, ev=None, q=None, do=None):
         """Route, attend [, backward], detach with history in device memory;
-        returns the number of library kernels launched."""
-        hga, w = self.hga, self.w
+        returns the number of library kernels launched.
+
+        With side_append the detach-time summary append (it reads only the
+        segment's keys and writes summaries of chunks this segment's route
+        never reads) runs on a side stream next to the route, whose grid leaves
+        SMs free, and is joined before the segment ends."""
+        torch, hga, w = self.torch, self.hga, self.w
         p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
         rec = ev.record if ev is not None else (lambda name: None)
+        main = torch.cuda.current_stream()
+        if self.side_append:
+            self.side.wait_stream(main)
+            with torch.cuda.stream(self.side):
+                if ev is not None:
+                    ev.record("summaries")
+                hga.hga_build_summaries(self.k, self.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
+                                        w.seg_len // w.chunk, self.summ, self.nct)
+                if ev is not None:
+                    ev.record(None)
         rec("route")
         hga.hga_route(p, q, self.summ, self.nct, self.idx)
         rec("attn_fwd")
@@ -251,10 +273,14 @@ class Layer:
             hga.hga_attn_bwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse,
                              self.do[T] if do is None else do, self.dq, self.dk, self.dv, self.ws)
             launches += 3
-        rec("summaries")
-        hga.hga_build_summaries(self.k, self.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
-                                w.seg_len // w.chunk, self.summ, self.nct)
-        rec(None)
+        if self.side_append:
+            rec(None)
+            main.wait_stream(self.side)
+        else:
+            rec("summaries")
+            hga.hga_build_summaries(self.k, self.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
+                                    w.seg_len // w.chunk, self.summ, self.nct)
+            rec(None)
         return launches + 1
 
     def _init_tiered(self):
@@ -346,18 +372,20 @@ class PhaseEvents:
         import torch
         self.torch = torch
         self.external = external
-        self.marks = []
+        self.marks = {}  # per stream: [(phase name or None, event)]
 
     def record(self, name):
+        stream = self.torch.cuda.current_stream()
         e = self.torch.cuda.Event(enable_timing=True, external=self.external)
-        e.record()
-        self.marks.append((name, e))
+        e.record(stream)
+        self.marks.setdefault(stream.cuda_stream, []).append((name, e))
 
     def totals(self):
         out = {}
-        for (name, a), (_, b) in zip(self.marks, self.marks[1:]):
-            if name is not None:
-                out[name] = out.get(name, 0.0) + a.elapsed_time(b)
+        for marks in self.marks.values():
+            for (name, a), (_, b) in zip(marks, marks[1:]):
+                if name is not None:
+                    out[name] = out.get(name, 0.0) + a.elapsed_time(b)
         return out
 
 
@@ -479,6 +507,7 @@ def run_hga(args, rank, world, local):
     hga.lib()
     w = gen.WORKLOADS[args.workload]
     layer = Layer(w)
+    layer.side_append = not args.serial_append and not w.tiered
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda", dtype=torch.float32)
     for _ in range(args.warmup):
         flush_l2(flush)
@@ -548,6 +577,8 @@ def run_hga(args, rank, world, local):
         "summaries": {"bound": "hbm", "ms_per_launch": ph["summaries"] / n_seg,
                       "achieved": summaries_bytes(w) * n_seg / (ph["summaries"] / 1e3) / 1e9, "unit": "GB/s"},
     }
+    if layer.side_append:
+        kernels["summaries"]["note"] = "on a side stream, timed while it overlaps the route"
     if w.tiered:
         kernels["attn_fwd"]["note"] = "includes waits for the wave fetches it cannot hide"
         kernels["summaries"]["note"] = "includes the segment K/V copy to host memory"
@@ -576,7 +607,8 @@ def run_hga(args, rank, world, local):
                        "backward": w.backward, "tiered": w.tiered,
                        "parallelism": f"one independent layer per GPU x{world}",
                        "l2": "flushed before every timed step (256 MiB write)",
-                       "launch": "one CUDA graph replay per step" if graph is not None else "eager"},
+                       "launch": "one CUDA graph replay per step" if graph is not None else "eager",
+                       "append": "side stream, overlapped with the route" if layer.side_append else "in order"},
             "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
             "device_status": status}
     if w.tiered:

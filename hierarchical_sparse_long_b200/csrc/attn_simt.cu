@@ -181,18 +181,42 @@ __global__ void __launch_bounds__(NT) fwd_simt_kernel(hga_params_t p, const T *_
 }
 
 // ---------------------------------------------------------------- backward
-// delta_i = sum_d dO_i,d * O_i,d (one warp per row)
+// delta_i = sum_d dO_i,d * O_i,d.  TPR threads per row, each one 16-byte
+// vector of O and of dO (8 bf16 or 4 fp32), DELTA_ROWS rows per thread with
+// every load in flight; the TPR partial dots are added by a fixed shuffle tree.
+constexpr int kDeltaThreads = 256;
+constexpr int kDeltaRows = 4;
 template <typename T, int D>
-__global__ void bwd_delta_kernel(const T *__restrict__ out, const T *__restrict__ dout, float *__restrict__ delta,
-                                 long long rows) {
-    const long long row = (long long)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int lane = threadIdx.x & 31;
-    if (row >= rows) return;
-    float s = 0.f;
-    for (int d = lane; d < D; d += 32) s = fmaf(to_f32(out[row * D + d]), to_f32(dout[row * D + d]), s);
+__global__ void __launch_bounds__(kDeltaThreads) bwd_delta_kernel(const T *__restrict__ out,
+                                                                   const T *__restrict__ dout,
+                                                                   float *__restrict__ delta, long long rows) {
+    constexpr int VEC = Vec16<T>::N;
+    constexpr int TPR = D / VEC;                 // 8 .. 32
+    constexpr int RPP = kDeltaThreads / TPR;     // rows per pass of the block
+    const int sub = threadIdx.x % TPR, rl = threadIdx.x / TPR;
+    const long long base = (long long)blockIdx.x * RPP * kDeltaRows + rl;
+    float o[kDeltaRows][VEC], g[kDeltaRows][VEC];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
-    if (lane == 0) delta[row] = s;
+    for (int u = 0; u < kDeltaRows; ++u) {
+        const long long row = base + (long long)u * RPP;
+        if (row < rows) {
+            Vec16<T>::load(out + row * D + sub * VEC, o[u]);
+            Vec16<T>::load(dout + row * D + sub * VEC, g[u]);
+        } else {
+#pragma unroll
+            for (int e = 0; e < VEC; ++e) o[u][e] = g[u][e] = 0.f;
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < kDeltaRows; ++u) {
+        float s = 0.f;
+#pragma unroll
+        for (int e = 0; e < VEC; ++e) s = fmaf(o[u][e], g[u][e], s);
+#pragma unroll
+        for (int off = TPR / 2; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+        const long long row = base + (long long)u * RPP;
+        if (sub == 0 && row < rows) delta[row] = s;
+    }
 }
 
 // dQ: query-major over the block's history and local tiles.
@@ -415,11 +439,9 @@ template <typename T, int D>
 static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
                           const void *vs, const int32_t *idx, const void *out, const float *lse, const void *dout,
                           void *dq, void *dk, void *dv, float *delta, unsigned *status, cudaStream_t stream) {
-    const long long rows = (long long)p.batch * p.n_q_heads * p.seg_len;
-    bwd_delta_kernel<T, D><<<(unsigned)((rows + 7) / 8), 256, 0, stream>>>((const T *)out, (const T *)dout, delta,
-                                                                          rows);
-    cudaError_t e = cudaGetLastError();
-    if (e != cudaSuccess) return record_cuda(e);
+    hga_status_t st = launch_bwd_delta(p, out, dout, delta, stream);
+    if (st != HGA_OK) return st;
+    cudaError_t e = cudaSuccess;
     const int nqb = p.seg_len / p.q_block;
     {
         const size_t smem = sizeof(float) * (4 * TILE * (D + 1) + TILE * 65);
@@ -447,20 +469,22 @@ static hga_status_t bwd_t(const hga_params_t &p, const void *q, const void *kh, 
 hga_status_t launch_bwd_delta(const hga_params_t &p, const void *out, const void *dout, float *delta,
                               cudaStream_t stream) {
     const long long rows = (long long)p.batch * p.n_q_heads * p.seg_len;
-    const unsigned grid = (unsigned)((rows + 7) / 8);
+    const int tpr = p.head_dim / (p.dtype == HGA_BF16 ? 8 : 4);
+    const long long per_block = (long long)(kDeltaThreads / tpr) * kDeltaRows;
+    const unsigned grid = (unsigned)((rows + per_block - 1) / per_block);
     if (p.dtype == HGA_BF16) {
         if (p.head_dim == 128)
-            bwd_delta_kernel<__nv_bfloat16, 128><<<grid, 256, 0, stream>>>(
+            bwd_delta_kernel<__nv_bfloat16, 128><<<grid, kDeltaThreads, 0, stream>>>(
                 (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, delta, rows);
         else
-            bwd_delta_kernel<__nv_bfloat16, 64><<<grid, 256, 0, stream>>>(
+            bwd_delta_kernel<__nv_bfloat16, 64><<<grid, kDeltaThreads, 0, stream>>>(
                 (const __nv_bfloat16 *)out, (const __nv_bfloat16 *)dout, delta, rows);
     } else {
         if (p.head_dim == 128)
-            bwd_delta_kernel<float, 128><<<grid, 256, 0, stream>>>((const float *)out, (const float *)dout, delta,
+            bwd_delta_kernel<float, 128><<<grid, kDeltaThreads, 0, stream>>>((const float *)out, (const float *)dout, delta,
                                                                    rows);
         else
-            bwd_delta_kernel<float, 64><<<grid, 256, 0, stream>>>((const float *)out, (const float *)dout, delta,
+            bwd_delta_kernel<float, 64><<<grid, kDeltaThreads, 0, stream>>>((const float *)out, (const float *)dout, delta,
                                                                   rows);
     }
     return record_cuda(cudaGetLastError());
