@@ -14,6 +14,8 @@ with the recipe of inputs/gen.py):
   dK/dV of the segment) + summary append.
 * ``qwen3_128k_eval``: one step = a 131,072-token evaluation as 32 segments of
   4,096 tokens, top-32 chunks, each route + forward + summary append.
+* ``qwen3_16k_fwd_sink``: ``qwen3_16k_fwd`` with a one-chunk attention-sink
+  window (history chunk 0 always routed, the other 15 slots by score).
 * ``qwen3_128k_tiered``: the 128K evaluation with detached history K/V in
   pinned host memory: each segment routes, fetches only the routed chunks
   (waves of 8 query blocks, double-buffered staging on a side stream
@@ -52,7 +54,7 @@ KERNEL_SOURCES = {
     "summaries": [CSRC + "summaries.cu", CSRC + "common.cuh"],
     "fetch": [CSRC + "tiered.cu", CSRC + "common.cuh"],
 }
-WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered")
+WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_16k_fwd_sink")
 
 
 def parse():
@@ -235,7 +237,8 @@ class Layer:
         w = self.w
         p = self.hga.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
                             topk=w.topk, seg_len=w.seg_len, n_hist_chunks=T // w.chunk, dtype=self.hga.HGA_BF16,
-                            hist_head_stride=self.L, seg_head_stride=self.L, chunk=w.chunk, q_block=w.q_block)
+                            hist_head_stride=self.L, seg_head_stride=self.L, chunk=w.chunk, q_block=w.q_block,
+                            sink_chunks=w.sink_chunks)
         for k, v in kw.items():
             setattr(p, k, v)
         return p
@@ -422,7 +425,8 @@ def oracle_sample(w, target_seconds):
     q = gen.queries_torch(w, T, T + S, "cpu").float().numpy()
     k_all = gen.keys_torch(w, 0, T + S, "cpu").float().numpy()
     v_all = gen.values_torch(w, 0, T + S, "cpu").float().numpy()
-    sh = oracle.shape(w.batch, w.n_q_heads, w.n_kv_heads, D, w.chunk, w.q_block, w.topk, S, T // w.chunk)
+    sh = oracle.shape(w.batch, w.n_q_heads, w.n_kv_heads, D, w.chunk, w.q_block, w.topk, S, T // w.chunk,
+                      w.sink_chunks)
     t0 = time.perf_counter()
     oracle.summaries(k_all[:, :, T:], w.chunk)  # detach-time summaries of the segment
     t_summ = time.perf_counter() - t0
@@ -603,6 +607,7 @@ def run_hga(args, rank, world, local):
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": w.name, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
                        "head_dim": w.head_dim, "context": w.seq_len, "seg_len": w.seg_len, "topk": w.topk,
+                       "sink_chunks": w.sink_chunks,
                        "chunk": w.chunk, "q_block": w.q_block, "segments_per_step": len(w.seg_starts),
                        "backward": w.backward, "tiered": w.tiered,
                        "parallelism": f"one independent layer per GPU x{world}",

@@ -38,7 +38,7 @@ class CParams(ctypes.Structure):
                 ("topk", ctypes.c_int), ("seg_len", ctypes.c_int), ("n_hist_chunks", ctypes.c_int),
                 ("dtype", ctypes.c_int), ("hist_head_stride", ctypes.c_longlong),
                 ("seg_head_stride", ctypes.c_longlong), ("qblock_begin", ctypes.c_int),
-                ("qblock_end", ctypes.c_int)]
+                ("qblock_end", ctypes.c_int), ("sink_chunks", ctypes.c_int)]
 
 
 @dataclasses.dataclass
@@ -58,13 +58,14 @@ class Params:
     q_block: int = 64
     qblock_begin: int = 0
     qblock_end: int = 0
+    sink_chunks: int = 0  # attention-sink window: chunks always routed
 
     def c(self) -> CParams:
         hs = self.hist_head_stride if self.hist_head_stride >= 0 else self.n_hist_chunks * self.chunk
         ss = self.seg_head_stride if self.seg_head_stride >= 0 else self.seg_len
         return CParams(self.batch, self.n_q_heads, self.n_kv_heads, self.head_dim, self.chunk, self.q_block,
                        self.topk, self.seg_len, self.n_hist_chunks, self.dtype, hs, ss, self.qblock_begin,
-                       self.qblock_end)
+                       self.qblock_end, self.sink_chunks)
 
 
 _lib = None

@@ -47,6 +47,7 @@ hga_status_t check_params(const hga_params_t *p) {
     if (p->head_dim != 64 && p->head_dim != 128) return HGA_ERR_UNSUPPORTED;
     if (p->chunk != 64 || p->q_block != 64) return HGA_ERR_UNSUPPORTED;
     if (p->topk < 1 || p->topk > 64) return HGA_ERR_INVALID_ARG;
+    if (p->sink_chunks < 0 || p->sink_chunks > p->topk) return HGA_ERR_INVALID_ARG;
     if (p->seg_len < 1 || p->seg_len % p->q_block || p->seg_len % p->chunk) return HGA_ERR_INVALID_ARG;
     if (p->n_hist_chunks < 0) return HGA_ERR_INVALID_ARG;
     if (p->seg_head_stride < p->seg_len) return HGA_ERR_INVALID_ARG;

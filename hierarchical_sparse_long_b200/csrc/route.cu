@@ -52,6 +52,7 @@ struct RouteArgs {
     unsigned *status;
     long long cap;  // summary rows per (b, g)
     int n_q_heads, n_kv_heads, seg_len, n, topk;
+    int sink;  // chunks 0 .. sink-1 are always routed (attention-sink window)
     int ns;  // chunks per cluster rank (multiple of 4)
     float inv_sqrt_d;
     RouteLayout L;
@@ -471,7 +472,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     }
 
     // 3. this query block's full score row, then the CTA selects
-    const uint32_t *row = sc;
+    uint32_t *row = sc;
     if constexpr (CL > 1) {
         tc::cluster_arrive();
         tc::cluster_wait();
@@ -488,6 +489,12 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
         row = rw;
     }
     __syncthreads();
+    if (a.sink > 0) {
+        // the sink chunks outrank every score (the largest image; ties among them
+        // go to the lower index, so they are listed first)
+        for (int j = tid; j < a.sink && j < n; j += kThreads) row[j] = 0xFFFFFFFFu;
+        __syncthreads();
+    }
     if (!abort_flag) {
         SelScratch ss;
         ss.tmax = reinterpret_cast<uint32_t *>(smem + L.tmax);
@@ -568,6 +575,7 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     a.seg_len = p.seg_len;
     a.n = n;
     a.topk = p.topk;
+    a.sink = p.sink_chunks;
     a.ns = cl > 1 ? round4((n + cl - 1) / cl) : round4(n);
     a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
     a.L = L;

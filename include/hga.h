@@ -78,7 +78,13 @@ typedef enum { HGA_BF16 = 0, HGA_FP32 = 1 } hga_dtype_t;
  *     route indices were remapped to slots by hga_fetch_tiered).
  *   seg_head_stride: tokens between (b, g) slices of k_seg / v_seg (>= S).
  *   qblock_begin / qblock_end: the range of query blocks hga_attn_fwd
- *     processes; 0 / 0 means every block (0 .. S/q_block). */
+ *     processes; 0 / 0 means every block (0 .. S/q_block).
+ *   sink_chunks: attention-sink window (0 .. topk; 0 = none): hga_route
+ *     always routes history chunks 0 .. min(sink_chunks, k_eff) - 1 and fills
+ *     the remaining slots by score ("Long-Context Fine-Tuning with Limited
+ *     VRAM", technical summary section 2.1: fixed sink and local windows next
+ *     to the routed chunks; the width is not given there, 1 chunk = 64 tokens
+ *     is the reading used by the benchmarks). */
 typedef struct {
     int batch;
     int n_q_heads;
@@ -94,6 +100,7 @@ typedef struct {
     long long seg_head_stride;
     int qblock_begin;
     int qblock_end;
+    int sink_chunks;
 } hga_params_t;
 
 /* Chunk summaries (technical summary section 2.1: one compact vector per
@@ -118,7 +125,9 @@ hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch
  *   qbar   = fp32 mean over the G heads of group g and the q_block queries of m;
  *   s_j    = fp32 dot(qbar, summ[b][g][j]) / sqrt(D), j < Nc;
  *   idx[((b*Hkv + g)*nqb + m)*k + a], a < k: the min(k, Nc) chunks with the
- *            largest s_j (ties: lower j), ascending, then -1 padding.
+ *            largest s_j (ties: lower j), ascending, then -1 padding; with
+ *            sink_chunks = s the chunks j < min(s, min(k, Nc)) are taken
+ *            first and the rest of the slots by score.
  *   q: device [B][Hq][S][D] dtype.  summ: device fp32 with summ_cap_chunks per
  *   (b, g) slice (>= Nc).  idx: device int32 [B][Hkv][S/q_block][k]. */
 hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,

@@ -113,6 +113,7 @@ class Workload:
     seed: int
     backward: bool = False
     tiered: bool = False
+    sink_chunks: int = 0  # attention-sink window: history chunks always routed
 
     @property
     def group(self) -> int:
@@ -137,6 +138,9 @@ WORKLOADS = {
     # the same evaluation with detached history K/V in pinned host memory
     "qwen3_128k_tiered": Workload("qwen3_128k_tiered", 1, 32, 8, 128, 64, 64, 32, 4096, 131072,
                                   _segs(0, 4096, 32), "bf16", 3, tiered=True),
+    # the 16K forward with a one-chunk attention-sink window (chunk 0 always routed)
+    "qwen3_16k_fwd_sink": Workload("qwen3_16k_fwd_sink", 1, 32, 8, 128, 64, 64, 16, 2048, 16384, (14336,),
+                                   "bf16", 1, sink_chunks=1),
 }
 
 

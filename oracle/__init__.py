@@ -25,7 +25,7 @@ _ip = ctypes.POINTER(ctypes.c_int)
 class Shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "head_dim", "chunk", "q_block", "topk", "seg_len",
-        "n_hist_chunks")]
+        "n_hist_chunks", "sink_chunks")]
 
 
 def build(force: bool = False) -> str:
@@ -72,8 +72,10 @@ def _check(rc: int, what: str):
         raise RuntimeError(f"{what} failed with code {rc}")
 
 
-def shape(batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks) -> Shape:
-    return Shape(batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks)
+def shape(batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks,
+          sink_chunks=0) -> Shape:
+    return Shape(batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks,
+                 sink_chunks)
 
 
 def summaries(k, chunk: int, n_chunks: int | None = None) -> np.ndarray:

@@ -47,6 +47,7 @@
 
 typedef struct {
     int batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks;
+    int sink_chunks; /* attention-sink window: history chunks 0..sink_chunks-1 are always routed */
 } oracle_shape_t;
 
 static long long ix4(long long a, long long A1, long long b, long long B1, long long c, long long C1, long long d)
@@ -100,7 +101,11 @@ static int ranks_before(double sa, int a, double sb, int b)
  * summary and keep the k best.  idx gets the chosen chunk ids in ascending
  * order, padded with -1 when k > Nc.  gap (optional) gets, per query block,
  * the relative distance between the k-th and (k+1)-th best scores, or
- * +inf when every chunk is taken.  scores (optional) gets all Nc scores. */
+ * +inf when every chunk is taken.  scores (optional) gets all Nc scores.
+ * [TS2.1, the fixed sink window] with sink_chunks = s > 0 the first
+ * min(s, k_eff) chunks are taken before any score is looked at and the
+ * remaining slots go to the best of the other chunks; gap then compares the
+ * last chunk taken by score with the next one (+inf if none is). */
 int oracle_route(const oracle_shape_t *p, const double *q, const double *summ,
                  int *idx, double *gap, double *scores)
 {
@@ -123,10 +128,16 @@ int oracle_route(const oracle_shape_t *p, const double *q, const double *summ,
                     s[j] = dot / sqrt((double)D);
                     if (scores) scores[ix4(b, Hkv, g, nqb, m, Nc, j)] = s[j];
                 }
-                /* plain selection: pick the best remaining chunk k_eff+1 times */
+                /* plain selection: the sink chunks first, then the best remaining
+                 * chunk until k_eff chunks (and one more, for the gap) are ranked */
                 memset(taken, 0, Nc > 0 ? Nc : 1);
+                const int n_sink = p->sink_chunks < keff ? (p->sink_chunks > 0 ? p->sink_chunks : 0) : keff;
+                for (int r = 0; r < n_sink; ++r) {
+                    order[r] = r;
+                    taken[r] = 1;
+                }
                 int n_rank = keff + (Nc > keff ? 1 : 0);
-                for (int r = 0; r < n_rank; ++r) {
+                for (int r = n_sink; r < n_rank; ++r) {
                     int best = -1;
                     for (int j = 0; j < Nc; ++j)
                         if (!taken[j] && (best < 0 || ranks_before(s[j], j, s[best], best))) best = j;
@@ -141,7 +152,7 @@ int oracle_route(const oracle_shape_t *p, const double *q, const double *summ,
                 for (; w < K; ++w) out[w] = -1;
                 if (gap) {
                     double g_rel = INFINITY;
-                    if (Nc > keff) {
+                    if (Nc > keff && keff > n_sink) {
                         double a = s[order[keff - 1]], c = s[order[keff]];
                         double den = fabs(a) > fabs(c) ? fabs(a) : fabs(c);
                         if (den < 1e-30) den = 1e-30;

@@ -46,7 +46,7 @@ def params(w, T, **kw):
                    topk=w.topk, seg_len=w.seg_len, n_hist_chunks=T // w.chunk,
                    dtype=hga.HGA_BF16 if w.dtype == "bf16" else hga.HGA_FP32,
                    hist_head_stride=T + w.seg_len, seg_head_stride=T + w.seg_len, chunk=w.chunk,
-                   q_block=w.q_block)
+                   q_block=w.q_block, sink_chunks=w.sink_chunks)
     for k, v in kw.items():
         setattr(p, k, v)
     return p
@@ -111,7 +111,7 @@ class GpuSegment:
 
 def oracle_shape(w, T):
     return oracle.shape(w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim, w.chunk, w.q_block, w.topk, w.seg_len,
-                        T // w.chunk)
+                        T // w.chunk, w.sink_chunks)
 
 
 def oracle_route(w, arrs):

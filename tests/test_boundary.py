@@ -55,6 +55,8 @@ BAD = [
     dict(qblock_begin=0, qblock_end=3),  # 3 > S/64 = 2
     dict(seg_head_stride=64),
     dict(hist_head_stride=100),   # < Nc * c
+    dict(sink_chunks=-1),
+    dict(sink_chunks=5),          # > topk
 ]
 
 

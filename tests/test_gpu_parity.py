@@ -88,7 +88,7 @@ def test_summaries_incremental_equals_full_rebuild():
 # ---------------------------------------------------------------- routing
 
 @pytest.mark.parametrize("name,seg", [("tiny_fp32", 0), ("qwen3_16k_fwd", 0), ("qwen3_128k_eval", 31),
-                                      ("qwen3_128k_eval", 1)])
+                                      ("qwen3_128k_eval", 1), ("qwen3_16k_fwd_sink", 0)])
 def test_route_matches_oracle(name, seg):
     w = W[name]
     arrs = hc.segment_arrays(w, seg)
@@ -124,6 +124,13 @@ ROUTE_SHAPES = [
                dtype="bf16", head_dim=64, n_q_heads=4, n_kv_heads=2, seed=24),
     gen.custom("cl8_n1100_fp32", topk=24, seg_len=512, seq_len=1100 * 64 + 512, seg_starts=(1100 * 64,),
                dtype="fp32", head_dim=128, n_q_heads=4, n_kv_heads=1, seed=25),
+    # attention-sink window: 1 chunk, 4 chunks under a cluster of 8, and every slot a sink chunk
+    gen.custom("sink1_n300", topk=16, sink_chunks=1, seg_len=256, seq_len=300 * 64 + 256,
+               seg_starts=(300 * 64,), dtype="bf16", head_dim=128, n_q_heads=8, n_kv_heads=2, seed=41),
+    gen.custom("sink4_cl8_n1100", topk=24, sink_chunks=4, seg_len=512, seq_len=1100 * 64 + 512,
+               seg_starts=(1100 * 64,), dtype="bf16", head_dim=128, n_q_heads=4, n_kv_heads=1, seed=42),
+    gen.custom("sink_all_d64", topk=3, sink_chunks=3, seg_len=128, seq_len=40 * 64 + 128, seg_starts=(40 * 64,),
+               dtype="fp32", head_dim=64, n_q_heads=2, n_kv_heads=2, seed=43),
 ]
 
 

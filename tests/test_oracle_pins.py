@@ -367,3 +367,53 @@ def test_torch_generator_matches_numpy_recipe():
         b = fn_t(w, 128, 384, "cpu").float().numpy()
         mismatch = np.mean(a != b)
         assert mismatch < 1e-3 and np.max(np.abs(a - b)) < 1e-2, (fn_np.__name__, mismatch)
+
+
+# ---------------------------------------------------------------- attention-sink window
+
+def _expected_sink_route(scores, k, sink):
+    """The rule written out with numpy: chunks 0..min(sink, k_eff)-1 first, then the
+    best of the others by (score descending, chunk index ascending); ascending, -1 padded."""
+    nc = scores.shape[-1]
+    keff = min(k, nc)
+    ns = min(sink, keff)
+    rest = np.arange(ns, nc)
+    order = rest[np.lexsort((rest, -scores[ns:]))]  # primary: score desc; then index asc
+    chosen = sorted(list(range(ns)) + list(order[:keff - ns]))
+    return chosen + [-1] * (k - keff)
+
+
+def test_route_sink_window_rule():
+    """The technical summary (section 2.1) puts a fixed sink window next to the routed
+    chunks; with sink_chunks = s the first s chunks are routed whatever their score and
+    the remaining slots go to the best other chunks."""
+    rng = np.random.default_rng(31)
+    B, Hq, Hkv, D, c, qb, S, nc, k = 2, 4, 2, 16, 16, 16, 48, 13, 5
+    q = rng.standard_normal((B, Hq, S, D))
+    summ = rng.standard_normal((B, Hkv, nc, D))
+    for sink in (0, 1, 2, 5):
+        sh = oracle.shape(B, Hq, Hkv, D, c, qb, k, S, nc, sink)
+        idx, gap, scores = oracle.route(sh, q, summ, with_scores=True)
+        for b in range(B):
+            for g in range(Hkv):
+                for m in range(S // qb):
+                    want = _expected_sink_route(scores[b, g, m], k, sink)
+                    assert list(idx[b, g, m]) == want, (sink, b, g, m)
+        if sink == k:
+            assert np.all(np.isinf(gap))  # no slot is decided by score
+
+
+def test_route_sink_keeps_a_low_scoring_first_chunk():
+    # chunk 0's summary points away from the queries: without a sink it is never routed
+    D, c, qb, S, nc, k = 8, 8, 8, 8, 6, 2
+    q = np.zeros((1, 2, S, D))
+    q[..., 0] = 1.0
+    summ = np.zeros((1, 1, nc, D))
+    summ[0, 0, :, 0] = [-5.0, 1.0, 2.0, 3.0, 4.0, 0.5]
+    idx0, _, _ = oracle.route(oracle.shape(1, 2, 1, D, c, qb, k, S, nc, 0), q, summ)
+    idx1, _, _ = oracle.route(oracle.shape(1, 2, 1, D, c, qb, k, S, nc, 1), q, summ)
+    assert list(idx0[0, 0, 0]) == [3, 4]
+    assert list(idx1[0, 0, 0]) == [0, 4]
+    # k >= Nc: every chunk is routed with or without the sink
+    idx2, _, _ = oracle.route(oracle.shape(1, 2, 1, D, c, qb, 8, S, nc, 1), q, summ)
+    assert list(idx2[0, 0, 0]) == [0, 1, 2, 3, 4, 5, -1, -1]
