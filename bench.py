@@ -14,6 +14,10 @@ with the recipe of inputs/gen.py):
   dK/dV of the segment) + summary append.
 * ``qwen3_128k_eval``: one step = a 131,072-token evaluation as 32 segments of
   4,096 tokens, top-32 chunks, each route + forward + summary append.
+* ``qwen3_128k_decode``: generation at 128K context: 16 sequences each add one
+  token after 131,008 detached history tokens; a step routes the 16 tokens
+  (one-token query blocks) and runs the split-K decode attention over their 32
+  routed chunks and 64-token local windows (query tok/s = tokens generated).
 * ``qwen3_16k_fwd_sink``: ``qwen3_16k_fwd`` with a one-chunk attention-sink
   window (history chunk 0 always routed, the other 15 slots by score).
 * ``qwen3_128k_tiered``: the 128K evaluation with detached history K/V in
@@ -53,8 +57,10 @@ KERNEL_SOURCES = {
     "route": [CSRC + "route.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
     "summaries": [CSRC + "summaries.cu", CSRC + "common.cuh"],
     "fetch": [CSRC + "tiered.cu", CSRC + "common.cuh"],
+    "attn_decode": [CSRC + "decode.cu", CSRC + "common.cuh"],
 }
-WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_16k_fwd_sink")
+WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_16k_fwd_sink",
+             "qwen3_128k_decode")
 
 
 def parse():
@@ -413,8 +419,48 @@ def job_throughput(tokens_per_step, steps, world, total_ms):
 
 
 # ------------------------------------------------------------------ CPU oracle sample
+def tokens_per_step(w):
+    """Query tokens a step processes: one per sequence when decoding."""
+    return w.batch if w.decode else w.seg_len * w.batch * len(w.seg_starts)
+
+
+def decode_oracle_sample(w, target_seconds):
+    """The oracle on the decode token of sequence 0 (its inputs drawn alone with the same
+    generator): its route (the oracle routes every token of the local window as a one-token
+    block; that time is divided by the window length) and its attention."""
+    import dataclasses
+
+    import numpy as np
+
+    import oracle
+    from inputs import gen
+    w1 = dataclasses.replace(w, batch=1)  # element n of sequence 0 is the same in a batch-1 draw
+    T, L, D = w.seg_starts[0], w.seg_len, w.head_dim
+    q = gen.queries_torch(w1, T, T + L, "cpu").float().numpy()
+    k_all = gen.keys_torch(w1, 0, T + L, "cpu").float().numpy()
+    v_all = gen.values_torch(w1, 0, T + L, "cpu").float().numpy()
+    sh = oracle.shape(1, w.n_q_heads, w.n_kv_heads, D, w.chunk, 1, w.topk, L, T // w.chunk, w.sink_chunks)
+    summ = oracle.summaries(k_all[:, :, :T], w.chunk)
+    reps, t_route, t_attn = 0, 0.0, 0.0
+    while reps == 0 or (t_route + t_attn < target_seconds and reps < 50):
+        t0 = time.perf_counter()
+        idx, _, _ = oracle.route(sh, q, summ)
+        t_route += (time.perf_counter() - t0) / L
+        rows = np.array([h * L + L - 1 for h in range(w.n_q_heads)], dtype=np.int64)
+        t0 = time.perf_counter()
+        oracle.attn_fwd(sh, q, k_all[:, :, :T], v_all[:, :, :T], k_all[:, :, T:], v_all[:, :, T:], idx, rows=rows)
+        t_attn += time.perf_counter() - t0
+        reps += 1
+    per_token = (t_route + t_attn) / reps
+    desc = (f"oracle fp64 single-thread, decode token of sequence 0 ({T} history tokens, {L}-token window): "
+            f"route (window routes / {L}) + attention, {reps} repetitions; history summaries not counted")
+    return 1.0 / per_token, desc, 1
+
+
 def oracle_sample(w, target_seconds):
     """Times the CPU oracle on a bounded sample of the workload; returns (tok/s, desc, cores)."""
+    if w.decode:
+        return decode_oracle_sample(w, target_seconds)
     import numpy as np
 
     import oracle
@@ -471,7 +517,7 @@ def run_reference(args, rank):
         if s >= args.warmup:
             per_step.append(tok_s)
     v = statistics.median(per_step)
-    ms = w.seg_len * w.batch * len(w.seg_starts) / v * 1000
+    ms = tokens_per_step(w) / v * 1000
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -676,14 +722,191 @@ def e2e_measure(layer, steps):
             "scope": "every segment of the step through the C ABI from pinned host buffers"}
 
 
+class DecodeLayer:
+    """Device state of a decode step: the sequences' K/V (history and local window
+    in one buffer per head), the history's chunk summaries and each sequence's new
+    token (the last of its local window)."""
+
+    def __init__(self, w):
+        import torch
+        from inputs import gen
+        import hierarchical_sparse_long_b200 as hga
+        self.w, self.hga, self.torch = w, hga, torch
+        dev = torch.device("cuda")
+        self.T, self.n_local, self.Ltot = w.seg_starts[0], w.seg_len, w.seq_len
+        self.k = gen.keys_torch(w, 0, self.Ltot, dev).contiguous()
+        self.v = gen.values_torch(w, 0, self.Ltot, dev).contiguous()
+        self.q = gen.queries_torch(w, self.Ltot - 1, self.Ltot, dev).contiguous()  # [B][Hq][1][D]
+        self.nc = self.T // w.chunk
+        self.summ = torch.zeros(w.batch, w.n_kv_heads, self.nc, w.head_dim, device=dev)
+        hga.hga_build_summaries(self.k, self.Ltot, w.batch, w.n_kv_heads, w.head_dim, w.chunk, 0, self.nc,
+                                self.summ, self.nc)
+        self.p = hga.Params(batch=w.batch, n_q_heads=w.n_q_heads, n_kv_heads=w.n_kv_heads, head_dim=w.head_dim,
+                            topk=w.topk, seg_len=1, n_hist_chunks=self.nc, dtype=hga.HGA_BF16,
+                            hist_head_stride=self.Ltot, seg_head_stride=self.Ltot, chunk=w.chunk, q_block=1,
+                            sink_chunks=w.sink_chunks)
+        self.idx = torch.empty(w.batch, w.n_kv_heads, 1, w.topk, device=dev, dtype=torch.int32)
+        self.out = torch.empty(w.batch, w.n_q_heads, 1, w.head_dim, device=dev, dtype=torch.bfloat16)
+        self.lse = torch.empty(w.batch, w.n_q_heads, 1, device=dev)
+        self.ws = torch.empty(hga.hga_attn_decode_workspace_size(self.p, self.n_local) // 4 + 64, device=dev)
+        torch.cuda.synchronize()
+
+    def step(self, ev=None, q=None):
+        rec = ev.record if ev is not None else (lambda name: None)
+        q = self.q if q is None else q
+        T = self.T
+        rec("route")
+        self.hga.hga_route(self.p, q, self.summ, self.nc, self.idx)
+        rec("attn_decode")
+        self.hga.hga_attn_decode(self.p, q, self.k, self.v, self.k[:, :, T:], self.v[:, :, T:], self.n_local,
+                                 self.idx, self.out, self.lse, self.ws)
+        rec(None)
+        return 3
+
+
+def run_decode(args, rank, world, local):
+    """bench.py for a decode workload: one step = route + decode attention of one new
+    token per sequence (query tok/s = tokens generated per second)."""
+    import torch
+    from inputs import gen
+    import hierarchical_sparse_long_b200 as hga
+    from hierarchical_sparse_long_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    hga.lib()
+    w = gen.WORKLOADS[args.workload]
+    layer = DecodeLayer(w)
+    flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda", dtype=torch.float32)
+    for _ in range(args.warmup):
+        flush_l2(flush)
+        layer.step()
+    torch.cuda.synchronize()
+    if hga.hga_get_device_status() != 0:
+        raise RuntimeError("device status reported an error during warm-up")
+    gev = PhaseEvents(external=True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        graph_launches = layer.step(ev=gev)
+    flush_l2(flush)
+    graph.replay()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    phases, launches = [], 0
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    sampler.start()
+    time.sleep(0.3)
+    for s_ in range(args.steps):
+        flush_l2(flush)
+        starts[s_].record()
+        graph.replay()
+        ends[s_].record()
+        launches += graph_launches
+        ends[s_].synchronize()  # outside the timed window: read this replay's phase events
+        phases.append(gev.totals())
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop()
+    total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, "cuda")
+    value = job_throughput(tokens_per_step(w), args.steps, world, total_ms)
+    status = hga.hga_get_device_status()
+    ph = {}
+    for ev in phases:
+        for k, v in ev.items():
+            ph[k] = ph.get(k, 0.0) + v
+    peaks, peak_src = measured_peaks()
+    B, Hq, Hkv, D = w.batch, w.n_q_heads, w.n_kv_heads, w.head_dim
+    keff = min(w.topk, layer.nc)
+    route_b = B * Hkv * layer.nc * D * 4 + B * Hq * D * 2 + B * Hkv * w.topk * 4
+    dec_b = B * Hkv * (keff * w.chunk + layer.n_local) * D * 2 * 2 + 2 * B * Hq * D * 2 + B * Hkv * w.topk * 4
+    kernels = {
+        "route": {"bound": "hbm", "ms_per_launch": ph["route"] / args.steps,
+                  "achieved": route_b * args.steps / (ph["route"] / 1e3) / 1e9, "unit": "GB/s"},
+        "attn_decode": {"bound": "hbm", "ms_per_launch": ph["attn_decode"] / args.steps,
+                        "achieved": dec_b * args.steps / (ph["attn_decode"] / 1e3) / 1e9, "unit": "GB/s"},
+    }
+    for k, v in kernels.items():
+        v["frac"] = round(v["achieved"] / peaks["hbm_gbs"], 4)
+        v["achieved"] = round(v["achieved"], 2)
+        v["ms_per_launch"] = round(v["ms_per_launch"], 4)
+    kd = kernels["attn_decode"]
+    roof = {"bound": "hbm", "kernel": "hga_attn_decode", "achieved": kd["achieved"], "peak": peaks["hbm_gbs"],
+            "unit": "GB/s", "frac": kd["frac"], "traffic": kernel_traffic("attn_decode", w.name),
+            "peak_source": f"{peak_src}: MEASURED_PEAKS.json hbm_gbs",
+            "units_per_launch": "K and V of the routed chunks and the local window once per (sequence, kv head), "
+                                "plus q, O and the route table"}
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": D,
+                       "context": w.seq_len, "history_tokens": layer.T, "local_window": layer.n_local,
+                       "topk": w.topk, "sink_chunks": w.sink_chunks, "chunk": w.chunk, "decode": True,
+                       "tokens_per_step": tokens_per_step(w),
+                       "parallelism": f"one independent layer per GPU x{world}",
+                       "l2": "flushed before every timed step (256 MiB write)",
+                       "launch": "one CUDA graph replay per step"},
+            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
+            "device_status": status}
+    line["e2e"] = decode_e2e(layer, max(2, min(args.steps, 5)))
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tok_s, desc, cores = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def decode_e2e(layer, steps):
+    """The decode step through the C ABI from pinned host buffers: the new tokens' q, k
+    and v copied in (k / v into the last slot of each local window), route and decode,
+    O and LSE copied back, all inside the timed region."""
+    import torch
+    w, T, Lt = layer.w, layer.T, layer.Ltot
+    host_q = layer.q.cpu().pin_memory()
+    host_k = layer.k[:, :, Lt - 1:Lt].cpu().pin_memory()
+    host_v = layer.v[:, :, Lt - 1:Lt].cpu().pin_memory()
+    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (layer.out, layer.lse)]
+    q_d = torch.empty_like(layer.q)
+    h2d = sum(t.numel() * t.element_size() for t in (host_q, host_k, host_v))
+    d2h = sum(t.numel() * t.element_size() for t in (layer.out, layer.lse))
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    times = []
+    for it in range(steps + 1):
+        torch.cuda.synchronize()
+        s.record()
+        q_d.copy_(host_q, non_blocking=True)
+        layer.k[:, :, Lt - 1:Lt].copy_(host_k, non_blocking=True)
+        layer.v[:, :, Lt - 1:Lt].copy_(host_v, non_blocking=True)
+        layer.step(q=q_d)
+        host_out[0].copy_(layer.out, non_blocking=True)
+        host_out[1].copy_(layer.lse, non_blocking=True)
+        e.record()
+        e.synchronize()
+        if it >= 1:
+            times.append(s.elapsed_time(e))
+    ms = statistics.mean(times)
+    return {"value": tokens_per_step(w) / (ms / 1000.0), "unit": UNIT, "h2d_bytes_per_step": h2d,
+            "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "scope": "the decode step through the C ABI from pinned host buffers"}
+
+
 def main():
     args = parse()
     if args.impl == "reference":
         run_reference(args, int(os.environ.get("RANK", "0")))
         return
     rank, world, local = dist_setup()
+    from inputs import gen
     try:
-        run_hga(args, rank, world, local)
+        if gen.WORKLOADS[args.workload].decode:
+            run_decode(args, rank, world, local)
+        else:
+            run_hga(args, rank, world, local)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -22,8 +22,8 @@ STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3:
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
 EXPORTED = ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
-            "hga_attn_bwd_noalloc", "hga_fetch_tiered", "hga_get_device_status", "hga_selftest_wait_timeout",
-            "hga_status_string", "hga_last_error")
+            "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_fetch_tiered",
+            "hga_get_device_status", "hga_selftest_wait_timeout", "hga_status_string", "hga_last_error")
 
 
 class HGAError(RuntimeError):
@@ -88,6 +88,9 @@ def lib() -> ctypes.CDLL:
         L.hga_attn_bwd_workspace_size.restype = sz
         L.hga_attn_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.hga_attn_bwd_noalloc.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.hga_attn_decode_workspace_size.argtypes = [pp, i]
+        L.hga_attn_decode_workspace_size.restype = sz
+        L.hga_attn_decode.argtypes = [pp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, sz, vp]
         L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hga_selftest_wait_timeout.argtypes = [ll, vp]
@@ -96,7 +99,7 @@ def lib() -> ctypes.CDLL:
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
         for f in ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-                  "hga_fetch_tiered", "hga_get_device_status"):
+                  "hga_attn_decode", "hga_fetch_tiered", "hga_get_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -150,6 +153,21 @@ def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stre
     cp = p.c()
     _check(lib().hga_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg),
                               _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)), "hga_attn_fwd")
+
+
+def hga_attn_decode_workspace_size(p: Params, n_local: int) -> int:
+    cp = p.c()
+    return int(lib().hga_attn_decode_workspace_size(ctypes.byref(cp), n_local))
+
+
+def hga_attn_decode(p: Params, q, k_hist, v_hist, k_local, v_local, n_local: int, idx, out, lse, workspace,
+                    stream=None):
+    """One new token per sequence: attention over its routed chunks and its n_local-token local window."""
+    cp = p.c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().hga_attn_decode(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_local),
+                                 _ptr(v_local), n_local, _ptr(idx), _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
+                                 _stream(stream)), "hga_attn_decode")
 
 
 def hga_attn_bwd_workspace_size(p: Params) -> int:

@@ -45,10 +45,12 @@ hga_status_t check_params(const hga_params_t *p) {
     if (p->n_q_heads % p->n_kv_heads) return HGA_ERR_INVALID_ARG;
     if (p->dtype != HGA_BF16 && p->dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
     if (p->head_dim != 64 && p->head_dim != 128) return HGA_ERR_UNSUPPORTED;
-    if (p->chunk != 64 || p->q_block != 64) return HGA_ERR_UNSUPPORTED;
+    // query blocks of 64, or a one-token segment (decode: seg_len = q_block = 1)
+    if (p->chunk != 64 || !(p->q_block == 64 || (p->q_block == 1 && p->seg_len == 1))) return HGA_ERR_UNSUPPORTED;
     if (p->topk < 1 || p->topk > 64) return HGA_ERR_INVALID_ARG;
     if (p->sink_chunks < 0 || p->sink_chunks > p->topk) return HGA_ERR_INVALID_ARG;
-    if (p->seg_len < 1 || p->seg_len % p->q_block || p->seg_len % p->chunk) return HGA_ERR_INVALID_ARG;
+    if (p->seg_len < 1 || p->seg_len % p->q_block || (p->q_block > 1 && p->seg_len % p->chunk))
+        return HGA_ERR_INVALID_ARG;
     if (p->n_hist_chunks < 0) return HGA_ERR_INVALID_ARG;
     if (p->seg_head_stride < p->seg_len) return HGA_ERR_INVALID_ARG;
     if (p->hist_head_stride < 0) return HGA_ERR_INVALID_ARG;
@@ -121,6 +123,7 @@ hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hi
                           cudaStream_t stream) {
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
+    if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
     if (!q || !k_seg || !v_seg || !idx || !out || !lse) return HGA_ERR_INVALID_ARG;
     if (p->n_hist_chunks > 0 && (!k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
     for (const void *ptr : {q, k_hist, v_hist, k_seg, v_seg, (const void *)out})
@@ -144,6 +147,7 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
                           size_t workspace_bytes, cudaStream_t stream) {
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
+    if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
     if (p->qblock_begin != 0 || p->qblock_end != 0) return HGA_ERR_INVALID_ARG;
     if (!q || !k_seg || !v_seg || !idx || !out || !lse || !dout || !dq || !dk_seg || !dv_seg || !workspace)
         return HGA_ERR_INVALID_ARG;
@@ -166,12 +170,37 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
                                      delta, status, stream);
 }
 
+size_t hga_attn_decode_workspace_size(const hga_params_t *p, int n_local) {
+    if (check_params(p) != HGA_OK || p->seg_len != 1 || n_local < 1) return 0;
+    return hga::decode_workspace_bytes(*p, n_local);
+}
+
+hga_status_t hga_attn_decode(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                             const void *k_local, const void *v_local, int n_local, const int32_t *idx, void *out,
+                             float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (p->seg_len != 1 || p->q_block != 1 || n_local < 1 || p->seg_head_stride < n_local)
+        return HGA_ERR_INVALID_ARG;
+    if (p->n_q_heads / p->n_kv_heads > 8) return HGA_ERR_UNSUPPORTED;
+    if (!q || !k_local || !v_local || !idx || !out || !lse || !workspace) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {q, k_hist, v_hist, k_local, v_local, (const void *)out, (const void *)workspace})
+        if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    if (workspace_bytes < hga::decode_workspace_bytes(*p, n_local)) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    return hga::launch_decode(*p, q, k_hist, v_hist, k_local, v_local, n_local, idx, out, lse,
+                              static_cast<float *>(workspace), status, stream);
+}
+
 hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,
                               int qblock_begin, int qblock_end, void *stage_k, void *stage_v, int stage_slots,
                               int32_t *slot_map, int32_t *idx_remapped, int32_t *n_fetched, cudaStream_t copy_stream,
                               cudaEvent_t done) {
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
+    if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
     const int nqb = p->seg_len / p->q_block;
     if (qblock_begin < 0 || qblock_end <= qblock_begin || qblock_end > nqb) return HGA_ERR_INVALID_ARG;
     if (p->hist_head_stride < (long long)p->n_hist_chunks * p->chunk) return HGA_ERR_INVALID_ARG;

@@ -76,6 +76,10 @@ hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void
                                 const void *v_hist, const void *k_seg, const void *v_seg,
                                 const int32_t *idx, void *out, float *lse, unsigned *status,
                                 cudaStream_t stream);
+size_t decode_workspace_bytes(const hga_params_t &p, int n_local);
+hga_status_t launch_decode(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *kl,
+                           const void *vl, int n_local, const int32_t *idx, void *out, float *lse, float *ws,
+                           unsigned *status, cudaStream_t stream);
 hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
                                  int stage_slots, int32_t *slot_map, int32_t *idx_remapped,

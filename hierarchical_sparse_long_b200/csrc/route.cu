@@ -51,7 +51,7 @@ struct RouteArgs {
     int32_t *idx;
     unsigned *status;
     long long cap;  // summary rows per (b, g)
-    int n_q_heads, n_kv_heads, seg_len, n, topk;
+    int n_q_heads, n_kv_heads, seg_len, q_block, n, topk;  // q_block: 64, or 1 for a decode token
     int sink;  // chunks 0 .. sink-1 are always routed (attention-sink window)
     int ns;  // chunks per cluster rank (multiple of 4)
     float inv_sqrt_d;
@@ -59,7 +59,6 @@ struct RouteArgs {
 };
 
 constexpr int kTileBytes = 16 * 1024;  // one ring slot: a tile of summary rows
-constexpr int kQBlock = 64;            // queries per block (the only size the API accepts)
 constexpr int kWarps = kThreads / 32;
 
 int round4(int x) { return (x + 3) & ~3; }
@@ -289,7 +288,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     __shared__ int abort_flag;
     const RouteLayout &L = a.L;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int nqb = a.seg_len / kQBlock;
+    const int nqb = a.seg_len / a.q_block;
     const int m = blockIdx.x % nqb, bg = blockIdx.x / nqb;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
     const int G = a.n_q_heads / a.n_kv_heads;
@@ -335,9 +334,9 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     {
         const int cu = tid % UPR, rs = tid / UPR;
         const T *qbase = static_cast<const T *>(a.q) +
-                         (((long long)b * a.n_q_heads + (long long)g * G) * a.seg_len + (long long)m * kQBlock) * D +
+                         (((long long)b * a.n_q_heads + (long long)g * G) * a.seg_len + (long long)m * a.q_block) * D +
                          cu * VEC;
-        const int rows = G * kQBlock;
+        const int rows = G * a.q_block;
         float acc[VEC];
 #pragma unroll
         for (int e = 0; e < VEC; ++e) acc[e] = 0.f;
@@ -347,7 +346,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
             for (int u = 0; u < BATCH; ++u) {
                 const int r = r0 + u * NRS;
                 if (r < rows) {
-                    const int hh = r / kQBlock, i = r % kQBlock;
+                    const int hh = r / a.q_block, i = r - hh * a.q_block;
                     raw[u] = *reinterpret_cast<const uint4 *>(qbase + ((long long)hh * a.seg_len + i) * D);
                 } else {
                     raw[u] = make_uint4(0u, 0u, 0u, 0u);
@@ -366,7 +365,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
         const float *part = reinterpret_cast<const float *>(smem + L.part);
         float s = 0.f;
         for (int sl = 0; sl < NRS; ++sl) s += part[sl * D + tid];
-        qown[tid] = s / static_cast<float>(G * kQBlock);
+        qown[tid] = s / static_cast<float>(G * a.q_block);
     }
 
     // 2. the cluster's CL block summaries, then this rank's slice of scores
@@ -543,7 +542,7 @@ cudaError_t launch_t(const RouteArgs &a, int cl, unsigned grid, cudaStream_t str
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
                           unsigned *status, cudaStream_t stream) {
     const int n = p.n_hist_chunks, D = p.head_dim;
-    const int nqb = p.seg_len / kQBlock;
+    const int nqb = p.seg_len / p.q_block;
     const int esize = p.dtype == HGA_BF16 ? 2 : 4;
     // cluster size: the smallest that lets one CTA's slice of the chunk list
     // sit in the ring at once (one round of bulk copies), else the largest
@@ -575,6 +574,7 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     a.seg_len = p.seg_len;
     a.n = n;
     a.topk = p.topk;
+    a.q_block = p.q_block;
     a.sink = p.sink_chunks;
     a.ns = cl > 1 ? round4((n + cl - 1) / cl) : round4(n);
     a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));

@@ -195,6 +195,28 @@ hga_status_t hga_attn_bwd_noalloc(const hga_params_t *p, const void *q, const vo
                                   const int32_t *idx, const void *out, const float *lse, const void *dout,
                                   void *dq, void *dk_seg, void *dv_seg, cudaStream_t stream);
 
+/* Single-query decode (generation: one new token per sequence).  The token's
+ * route comes from hga_route over a one-token segment (seg_len = q_block = 1:
+ * its block summary is the mean of its G query heads); it then attends, with
+ * exact softmax, the tokens of its routed history chunks and the n_local
+ * tokens of its local window (the not-yet-detached tokens, itself last):
+ * technical summary section 2.1, routed exact chunks next to a local window.
+ *   p: seg_len = q_block = 1, n_q_heads / n_kv_heads <= 8; seg_head_stride =
+ *     tokens between (b, g) slices of k_local / v_local (>= n_local);
+ *     hist_head_stride / n_hist_chunks / topk as for hga_attn_fwd.
+ *   q: device [B][Hq][1][D] dtype.  k_local, v_local: device [B][Hkv][*][D].
+ *   idx: device int32 [B][Hkv][1][k] (from hga_route).
+ *   out: device [B][Hq][1][D] dtype.  lse: device fp32 [B][Hq][1] (natural log).
+ *   workspace: device, at least hga_attn_decode_workspace_size(p, n_local)
+ *     bytes, 16-byte aligned (per-split partial results; nothing in it needs
+ *     clearing).
+ * Two kernels on stream (split-K partial attention, then the merge); nothing
+ * is allocated.  Out-of-range route indices are skipped and flagged. */
+size_t hga_attn_decode_workspace_size(const hga_params_t *p, int n_local);
+hga_status_t hga_attn_decode(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                             const void *k_local, const void *v_local, int n_local, const int32_t *idx,
+                             void *out, float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Tiered history (technical summary section 2.2: detached K/V live in host
  * RAM, only the routed exact K/V are brought to the GPU).  For the query
  * blocks [qblock_begin, qblock_end) of idx, gathers the distinct (b, g, chunk)

@@ -114,6 +114,7 @@ class Workload:
     backward: bool = False
     tiered: bool = False
     sink_chunks: int = 0  # attention-sink window: history chunks always routed
+    decode: bool = False  # one new token per sequence; seg_len is then its local window
 
     @property
     def group(self) -> int:
@@ -138,6 +139,10 @@ WORKLOADS = {
     # the same evaluation with detached history K/V in pinned host memory
     "qwen3_128k_tiered": Workload("qwen3_128k_tiered", 1, 32, 8, 128, 64, 64, 32, 4096, 131072,
                                   _segs(0, 4096, 32), "bf16", 3, tiered=True),
+    # decode at 128K context: 16 sequences, each adds one token after 131,008 detached history
+    # tokens and closes a 64-token local window; top-32 chunks
+    "qwen3_128k_decode": Workload("qwen3_128k_decode", 16, 32, 8, 128, 64, 64, 32, 64, 131072, (131008,),
+                                  "bf16", 4, decode=True),
     # the 16K forward with a one-chunk attention-sink window (chunk 0 always routed)
     "qwen3_16k_fwd_sink": Workload("qwen3_16k_fwd_sink", 1, 32, 8, 128, 64, 64, 16, 2048, 16384, (14336,),
                                    "bf16", 1, sink_chunks=1),

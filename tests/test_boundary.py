@@ -104,3 +104,17 @@ def test_workspace_size(L):
     p = _params()
     assert hga.hga_attn_bwd_workspace_size(p) >= 4 * 4 * 128
     assert hga.hga_attn_bwd_workspace_size(_params(topk=0)) == 0
+
+
+def test_decode_shape_checked_on_host(L):
+    """A decode call is a one-token segment (seg_len = q_block = 1); other one-token
+    shapes and an empty local window are rejected before any launch."""
+    ok = _params(seg_len=1, q_block=1).c()
+    assert L.hga_attn_decode_workspace_size(ctypes.byref(ok), 64) > 0
+    for bad in (dict(seg_len=2, q_block=1), dict(seg_len=64, q_block=1), dict(seg_len=1, q_block=64)):
+        p = _params(**bad).c()
+        assert L.hga_attn_decode_workspace_size(ctypes.byref(p), 64) == 0, bad
+    assert L.hga_attn_decode_workspace_size(ctypes.byref(ok), 0) == 0
+    fake = ctypes.c_void_p(0x1000)
+    # one-token segments are for hga_attn_decode only
+    assert L.hga_attn_fwd(ctypes.byref(ok), fake, fake, fake, fake, fake, fake, fake, fake, None) == -2

@@ -417,3 +417,32 @@ def test_route_sink_keeps_a_low_scoring_first_chunk():
     # k >= Nc: every chunk is routed with or without the sink
     idx2, _, _ = oracle.route(oracle.shape(1, 2, 1, D, c, qb, 8, S, nc, 1), q, summ)
     assert list(idx2[0, 0, 0]) == [0, 1, 2, 3, 4, 5, -1, -1]
+
+
+# ---------------------------------------------------------------- single-query decode
+
+def test_decode_token_equals_masked_attention():
+    """A decode token is a one-token query block (q_block = 1): its route uses the mean of
+    its G query heads, and its output is exact attention over the routed chunks and the
+    local window up to itself (torch, fp64, explicit mask; routes from the oracle)."""
+    rng = np.random.default_rng(51)
+    B, Hq, Hkv, D, c, L, nc, k = 2, 4, 2, 16, 8, 11, 9, 3
+    sh = oracle.shape(B, Hq, Hkv, D, c, 1, k, L, nc)
+    q = rng.standard_normal((B, Hq, L, D))
+    kh, vh = rng.standard_normal((B, Hkv, nc * c, D)), rng.standard_normal((B, Hkv, nc * c, D))
+    ks, vs = rng.standard_normal((B, Hkv, L, D)), rng.standard_normal((B, Hkv, L, D))
+    summ = oracle.summaries(kh, c)
+    idx, _, scores = oracle.route(sh, q, summ, with_scores=True)
+    # the last token's route: top-k of its own block summary's scores (ties -> lower index)
+    for b in range(B):
+        for g in range(Hkv):
+            qbar = q[b, g * 2:(g + 1) * 2, L - 1].mean(axis=0)
+            s = summ[b, g] @ qbar / np.sqrt(D)
+            assert np.allclose(scores[b, g, L - 1], s, rtol=1e-12, atol=1e-12)
+            want = sorted(np.lexsort((np.arange(nc), -s))[:k])
+            assert list(idx[b, g, L - 1]) == want
+    rows = np.array([(b * Hq + h) * L + L - 1 for b in range(B) for h in range(Hq)])
+    out, lse = oracle.attn_fwd(sh, q, kh, vh, ks, vs, idx, rows=rows)
+    ref_out, ref_lse = _sdpa(sh, q, kh, vh, ks, vs, _allowed_mask(sh, idx))
+    assert np.allclose(out[:, :, L - 1], ref_out[:, :, L - 1], atol=1e-12)
+    assert np.allclose(lse[:, :, L - 1], ref_lse[:, :, L - 1], atol=1e-12)
