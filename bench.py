@@ -18,6 +18,8 @@ with the recipe of inputs/gen.py):
   token after 131,008 detached history tokens; a step routes the 16 tokens
   (one-token query blocks) and runs the split-K decode attention over their 32
   routed chunks and 64-token local windows (query tok/s = tokens generated).
+* ``qwen3_32k_decode``: the same decode step after 32,704 history tokens (the
+  decode grid of the 128K case on 2.1 GB of K/V; used for counter captures).
 * ``qwen3_16k_fwd_sink``: ``qwen3_16k_fwd`` with a one-chunk attention-sink
   window (history chunk 0 always routed, the other 15 slots by score).
 * ``qwen3_128k_tiered``: the 128K evaluation with detached history K/V in
@@ -57,10 +59,10 @@ KERNEL_SOURCES = {
     "route": [CSRC + "route.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
     "summaries": [CSRC + "summaries.cu", CSRC + "common.cuh"],
     "fetch": [CSRC + "tiered.cu", CSRC + "common.cuh"],
-    "attn_decode": [CSRC + "decode.cu", CSRC + "common.cuh"],
+    "attn_decode": [CSRC + "decode.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
 }
 WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_16k_fwd_sink",
-             "qwen3_128k_decode")
+             "qwen3_128k_decode", "qwen3_32k_decode")
 
 
 def parse():

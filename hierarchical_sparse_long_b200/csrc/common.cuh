@@ -94,6 +94,13 @@ bool tma_encoder_available();
 // x box_rows rows, 128-byte swizzle; maps are cached per thread by
 // (base, rows, box_rows).
 bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows, unsigned box_rows = 64);
+// 3-D TMA map over `groups` groups of `rows` rows of D (64 or 128) bf16 values,
+// group g starting group_stride_rows rows after group g - 1; boxes of 64 values
+// x 64 rows x 1 group, 128-byte swizzle; rows past `rows` read as zeros.
+bool tma_group_rows_map(CUtensorMap *map, const void *base, int D, unsigned long long rows,
+                        unsigned long long groups, unsigned long long group_stride_rows);
 // cudaFuncAttributeMaxDynamicSharedMemorySize, set once per kernel and device.
 cudaError_t set_max_dynamic_smem(const void *kernel, int bytes);
+// Streaming multiprocessors of the current device (148 when it cannot be queried).
+int sm_count();
 }  // namespace hga

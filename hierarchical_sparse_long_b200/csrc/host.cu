@@ -1,5 +1,5 @@
 // Host-side helpers shared by the launchers: TMA tensor maps over rows of
-// 128 bf16 values (cached per thread, since encoding one is a driver call on
+// bf16 values (cached per thread, since encoding one is a driver call on
 // every launch otherwise) and the per-device dynamic shared-memory attribute
 // of a kernel (set once per kernel and device).
 #include <cudaTypedefs.h>
@@ -25,6 +25,15 @@ struct MapEntry {
 constexpr int kMapCache = 16;
 thread_local MapEntry t_maps[kMapCache];
 thread_local int t_map_next = 0;
+
+struct GroupMapEntry {
+    const void *base;
+    int D;
+    unsigned long long rows, groups, stride;
+    CUtensorMap map;
+};
+thread_local GroupMapEntry t_gmaps[kMapCache];
+thread_local int t_gmap_next = 0;
 
 std::mutex g_attr_mu;
 std::vector<std::pair<std::pair<const void *, int>, int>> g_attr;  // (kernel, device) -> bytes set
@@ -66,6 +75,34 @@ bool tma_rows_map(CUtensorMap *map, const void *base, unsigned long long rows, u
     return true;
 }
 
+bool tma_group_rows_map(CUtensorMap *map, const void *base, int D, unsigned long long rows,
+                        unsigned long long groups, unsigned long long group_stride_rows) {
+    for (const GroupMapEntry &e : t_gmaps)
+        if (e.base == base && e.D == D && e.rows == rows && e.groups == groups && e.stride == group_stride_rows &&
+            base != nullptr) {
+            *map = e.map;
+            return true;
+        }
+    if (!tma_encoder_available() || rows == 0 || groups == 0 || (D != 64 && D != 128)) return false;
+    const cuuint64_t dims[3] = {(cuuint64_t)D, (cuuint64_t)rows, (cuuint64_t)groups};
+    const cuuint64_t strides[2] = {(cuuint64_t)D * 2, (cuuint64_t)(group_stride_rows * D * 2)};
+    const cuuint32_t box[3] = {64, 64, 1};
+    const cuuint32_t estr[3] = {1, 1, 1};
+    if (g_encode(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box, estr,
+                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        return false;
+    GroupMapEntry &slot = t_gmaps[t_gmap_next];
+    t_gmap_next = (t_gmap_next + 1) % kMapCache;
+    slot.base = base;
+    slot.D = D;
+    slot.rows = rows;
+    slot.groups = groups;
+    slot.stride = group_stride_rows;
+    slot.map = *map;
+    return true;
+}
+
 cudaError_t set_max_dynamic_smem(const void *kernel, int bytes) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -81,6 +118,16 @@ cudaError_t set_max_dynamic_smem(const void *kernel, int bytes) {
     e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e == cudaSuccess) g_attr.push_back({{kernel, dev}, bytes});
     return e;
+}
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1) {
+        cudaGetLastError();
+        return 148;
+    }
+    return n;
 }
 
 }  // namespace hga

@@ -35,7 +35,7 @@ namespace hga {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kRing = 4;         // bulk-copy ring slots
+constexpr int kRound = 4;        // summary tiles scored per round (contiguous in the ring)
 constexpr int kCandCap = 1024;   // candidate list of the selecting warp
 constexpr int kMaxSmem = 227 * 1024 - 1024;
 constexpr unsigned kFull = 0xffffffffu;
@@ -54,6 +54,7 @@ struct RouteArgs {
     int n_q_heads, n_kv_heads, seg_len, q_block, n, topk;  // q_block: 64, or 1 for a decode token
     int sink;  // chunks 0 .. sink-1 are always routed (attention-sink window)
     int ns;  // chunks per cluster rank (multiple of 4)
+    int slots;  // ring slots: kRound, or 2 * kRound (the next round in flight while one is scored)
     float inv_sqrt_d;
     RouteLayout L;
 };
@@ -63,7 +64,7 @@ constexpr int kWarps = kThreads / 32;
 
 int round4(int x) { return (x + 3) & ~3; }
 
-RouteLayout route_layout(int D, int esize, int cl, int ns, int n) {
+RouteLayout route_layout(int D, int esize, int cl, int ns, int n, int slots) {
     RouteLayout L{};
     int off = 0;
     auto take = [&](int bytes) {
@@ -71,7 +72,7 @@ RouteLayout route_layout(int D, int esize, int cl, int ns, int n) {
         off += (bytes + 15) & ~15;
         return at;
     };
-    L.ring = take(kRing * kTileBytes);
+    L.ring = take(slots * kTileBytes);
     L.part = take((kThreads / (D * esize / 16)) * D * 4);
     L.qown = take(D * 4);
     L.qall = take(cl * D * 4);
@@ -82,7 +83,7 @@ RouteLayout route_layout(int D, int esize, int cl, int ns, int n) {
     L.cj = take(kCandCap * 4);
     L.hist = take(256 * 4);
     L.misc = take(16 * 4);
-    L.bar = take(kRing * 8);
+    L.bar = take(slots * 8);
     L.total = off;
     return L;
 }
@@ -274,10 +275,10 @@ __device__ void select_cta(const uint32_t *row, int n, int k, int32_t *out, cons
 }
 
 // Waits, with a fresh bound, for bulk copies still in flight after an abort.
-__device__ void drain_ring(uint64_t *bar, int from, int to) {
+__device__ void drain_ring(uint64_t *bar, int from, int to, int slots) {
     for (int i = from; i < to; ++i) {
         const long long t0 = clock64();
-        while (!tc::mbar_try_wait(&bar[i % kRing], (i / kRing) & 1) && clock64() - t0 < (1ll << 31)) {
+        while (!tc::mbar_try_wait(&bar[i % slots], (i / slots) & 1) && clock64() - t0 < (1ll << 31)) {
         }
     }
 }
@@ -308,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     const float *sbase = a.summ + ((long long)bg * a.cap + c_begin) * D;
 
     auto issue = [&](int t) {
-        const int slot = t % kRing;
+        const int slot = t % a.slots;
         const uint32_t bytes = static_cast<uint32_t>(min(TCN, n_slice - t * TCN) * D * 4);
         tc::mbar_arrive_expect_tx(&bar[slot], bytes);
         tc::bulk_load(smem + L.ring + slot * kTileBytes, sbase + (long long)t * TCN * D, bytes, &bar[slot]);
@@ -316,13 +317,13 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
 
     if (tid == 0) {
         abort_flag = 0;
-        for (int s = 0; s < kRing; ++s) tc::mbar_init(&bar[s], 1);
+        for (int s = 0; s < a.slots; ++s) tc::mbar_init(&bar[s], 1);
         tc::fence_mbar_init();
     }
     __syncthreads();
     int issued = 0;  // thread 0's count of issued tiles
     if (tid == 0)
-        for (; issued < min(kRing, ntiles); ++issued) issue(issued);
+        for (; issued < min(a.slots, ntiles); ++issued) issue(issued);
 
     // 1. block summary.  Thread (rs, cu) sums the 16-byte column unit cu of
     //    rows rs, rs + NRS, ... of the G x q_block rows (head-major), in order;
@@ -397,17 +398,18 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     const bool writer = (s16 & ((1 << (4 - LOGCL)) - 1)) == 0;
     bool ok = true;
     int done = 0;  // tiles this thread waited for successfully
-    // rounds of up to kRing tiles: the round's chunks sit contiguously in the
-    // ring, every warp takes chunk pairs warp, warp + kWarps, ... of the round
+    // rounds of up to kRound tiles: the round's chunks sit contiguously in the
+    // ring, every warp takes chunk pairs warp, warp + kWarps, ... of the round;
+    // with 2 * kRound slots the next round's copies are in flight meanwhile
     constexpr int UNR = CL >= 8 ? 1 : 2;  // chunk pairs in flight per warp
-    for (int t0 = 0; t0 < ntiles; t0 += kRing) {
-        const int t1 = min(ntiles, t0 + kRing);
+    for (int t0 = 0; t0 < ntiles; t0 += kRound) {
+        const int t1 = min(ntiles, t0 + kRound);
         for (int t = t0; t < t1; ++t) {
-            ok = ok && tc::mbar_wait(&bar[t % kRing], (t / kRing) & 1, &abort_flag, a.status);
+            ok = ok && tc::mbar_wait(&bar[t % a.slots], (t / a.slots) & 1, &abort_flag, a.status);
             done += ok;
         }
         if (ok) {
-            const float *chunks = reinterpret_cast<const float *>(smem + L.ring);
+            const float *chunks = reinterpret_cast<const float *>(smem + L.ring + (t0 % a.slots) * kTileBytes);
             const int rows = min((t1 - t0) * TCN, n_slice - t0 * TCN);
             const int npairs = (rows + 1) >> 1;
             for (int pr0 = warp; pr0 < npairs; pr0 += UNR * kWarps) {  // warp-uniform
@@ -466,7 +468,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
         __syncthreads();
         if (tid == 0 && issued < ntiles && !abort_flag) {
             tc::fence_proxy_async();
-            for (; issued < min(ntiles, t1 + kRing); ++issued) issue(issued);
+            for (; issued < min(ntiles, t1 + a.slots); ++issued) issue(issued);
         }
     }
 
@@ -503,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
         ss.misc = reinterpret_cast<int *>(smem + L.misc);
         select_cta(row, n, a.topk, out, ss, tid);
     }
-    if (tid == 0 && abort_flag) drain_ring(bar, done, issued);
+    if (tid == 0 && abort_flag) drain_ring(bar, done, issued, a.slots);
     if constexpr (CL > 1) tc::cluster_wait();  // peers may still read this CTA's slice
 }
 
@@ -545,19 +547,30 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     const int nqb = p.seg_len / p.q_block;
     const int esize = p.dtype == HGA_BF16 ? 2 : 4;
     // cluster size: the smallest that lets one CTA's slice of the chunk list
-    // sit in the ring at once (one round of bulk copies), else the largest
-    const int ring_chunks = kRing * (kTileBytes / (D * 4));
-    int cl = 1;
-    RouteLayout L = route_layout(D, esize, 1, round4(n), n);
-    if (n > p.topk) {
-        for (int c : {1, 2, 4, 8}) {
-            if (nqb % c) continue;
-            const RouteLayout Lc = route_layout(D, esize, c, c > 1 ? round4((n + c - 1) / c) : round4(n), n);
-            if (Lc.total > kMaxSmem) continue;
-            cl = c;
-            L = Lc;
-            if ((n + c - 1) / c <= ring_chunks) break;
+    // fit one round of bulk copies, else the largest
+    const int ring_chunks = kRound * (kTileBytes / (D * 4));
+    // a grid of less than one CTA per SM keeps two rounds in flight (two CTAs
+    // per SM overlap each other's copies otherwise) when that layout fits
+    const bool small_grid = (long long)p.batch * p.n_kv_heads * nqb < sm_count();
+    int cl = 1, slots = kRound;
+    RouteLayout L{};
+    for (int sl : {2 * kRound, kRound}) {
+        if (sl > kRound && !small_grid) continue;
+        slots = sl;
+        cl = 1;
+        L = route_layout(D, esize, 1, round4(n), n, sl);
+        if (n > p.topk) {
+            for (int c : {1, 2, 4, 8}) {
+                if (nqb % c) continue;
+                const RouteLayout Lc =
+                    route_layout(D, esize, c, c > 1 ? round4((n + c - 1) / c) : round4(n), n, sl);
+                if (Lc.total > kMaxSmem) continue;
+                cl = c;
+                L = Lc;
+                if ((n + c - 1) / c <= ring_chunks) break;
+            }
         }
+        if (L.total <= kMaxSmem) break;
     }
     if (L.total > kMaxSmem) {
         record_error("hga_route: shared-memory layout exceeds the per-CTA limit");
@@ -577,6 +590,7 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     a.q_block = p.q_block;
     a.sink = p.sink_chunks;
     a.ns = cl > 1 ? round4((n + cl - 1) / cl) : round4(n);
+    a.slots = slots;
     a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
     a.L = L;
     const unsigned grid = static_cast<unsigned>(p.batch * p.n_kv_heads * nqb);

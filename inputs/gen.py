@@ -143,6 +143,10 @@ WORKLOADS = {
     # tokens and closes a 64-token local window; top-32 chunks
     "qwen3_128k_decode": Workload("qwen3_128k_decode", 16, 32, 8, 128, 64, 64, 32, 64, 131072, (131008,),
                                   "bf16", 4, decode=True),
+    # the same decode at 32K context (same grid and routed-chunk count; 2.1 GB of K/V on the
+    # device, the size used for counter captures)
+    "qwen3_32k_decode": Workload("qwen3_32k_decode", 16, 32, 8, 128, 64, 64, 32, 64, 32768, (32704,),
+                                 "bf16", 4, decode=True),
     # the 16K forward with a one-chunk attention-sink window (chunk 0 always routed)
     "qwen3_16k_fwd_sink": Workload("qwen3_16k_fwd_sink", 1, 32, 8, 128, 64, 64, 16, 2048, 16384, (14336,),
                                    "bf16", 1, sink_chunks=1),

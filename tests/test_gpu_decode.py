@@ -33,6 +33,12 @@ CASES = [
                 seq_len=30 * 64 + 70, seg_starts=(30 * 64,), seed=66), 70, 0),
     (gen.custom("dec_128k", dtype="bf16", head_dim=128, n_q_heads=8, n_kv_heads=2, topk=32, seg_len=64,
                 seq_len=131072, seg_starts=(131072 - 64,), seed=67), 64, 0),
+    # bf16 D 64 with 8 heads per KV head; the window ends in a 2-token piece
+    (gen.custom("dec_d64_g8_bf16", dtype="bf16", head_dim=64, n_q_heads=16, n_kv_heads=2, topk=6, seg_len=130,
+                seq_len=50 * 64 + 130, seg_starts=(50 * 64,), batch=2, seed=69), 130, 0),
+    # one query head per KV head
+    (gen.custom("dec_g1_bf16", dtype="bf16", head_dim=128, n_q_heads=4, n_kv_heads=4, topk=5, seg_len=33,
+                seq_len=20 * 64 + 33, seg_starts=(20 * 64,), seed=70), 33, 0),
     # 300 routable chunks (more than one pass of the route's tile ring) and a sink chunk
     (gen.custom("dec_split_fp32_sink", dtype="fp32", head_dim=64, n_q_heads=4, n_kv_heads=2, topk=6, seg_len=10,
                 seq_len=300 * 64 + 10, seg_starts=(300 * 64,), seed=68), 10, 1),
