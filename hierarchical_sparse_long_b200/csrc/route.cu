@@ -26,6 +26,10 @@
 //      cluster and selects with all its threads: a lower bound of the k-th
 //      best score from the per-thread maxima, the few chunks at or above it,
 //      and their exact ranks by (score, then the lower chunk index).
+// A segment of one query block (a decode token) has no neighbours to share
+// its cluster with; there the CL CTAs of a cluster split that block's chunk
+// list (SPLIT): each scores only its slice for the one summary, and rank 0
+// gathers the row and selects.
 #include <algorithm>
 
 #include "common.cuh"
@@ -64,7 +68,7 @@ constexpr int kWarps = kThreads / 32;
 
 int round4(int x) { return (x + 3) & ~3; }
 
-RouteLayout route_layout(int D, int esize, int cl, int ns, int n, int slots) {
+RouteLayout route_layout(int D, int esize, int cl, int ns, int n, int slots, int rows) {
     RouteLayout L{};
     int off = 0;
     auto take = [&](int bytes) {
@@ -76,7 +80,7 @@ RouteLayout route_layout(int D, int esize, int cl, int ns, int n, int slots) {
     L.part = take((kThreads / (D * esize / 16)) * D * 4);
     L.qown = take(D * 4);
     L.qall = take(cl * D * 4);
-    L.sc = take(cl * ns * 4);
+    L.sc = take(rows * ns * 4);
     L.row = take(cl > 1 ? round4(n) * 4 : 0);
     L.tmax = take(kThreads * 4);
     L.key = take(kCandCap * 8);
@@ -283,14 +287,16 @@ __device__ void drain_ring(uint64_t *bar, int from, int to, int slots) {
     }
 }
 
-template <typename T, int D, int CL>
+template <typename T, int D, int CL, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
+    constexpr int R = SPLIT ? 1 : CL;  // query blocks scored by this CTA
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int abort_flag;
     const RouteLayout &L = a.L;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int nqb = a.seg_len / a.q_block;
-    const int m = blockIdx.x % nqb, bg = blockIdx.x / nqb;
+    const int m = SPLIT ? 0 : (int)blockIdx.x % nqb;
+    const int bg = SPLIT ? (int)blockIdx.x / CL : (int)blockIdx.x / nqb;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
     const int G = a.n_q_heads / a.n_kv_heads;
     const int n = a.n;
@@ -300,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
         return;
     }
 
-    const int rank = CL > 1 ? static_cast<int>(tc::cluster_ctarank()) : 0;  // == m % CL
+    const int rank = CL > 1 ? static_cast<int>(tc::cluster_ctarank()) : 0;  // m % CL, or the slice (SPLIT)
     const int c_begin = rank * a.ns;
     const int n_slice = max(0, min(n, c_begin + a.ns) - c_begin);
     constexpr int TCN = kTileBytes / (D * 4);  // chunks per summary tile
@@ -371,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
 
     // 2. the cluster's CL block summaries, then this rank's slice of scores
     const float *qall = qown;
-    if constexpr (CL > 1) {
+    if constexpr (CL > 1 && !SPLIT) {
         tc::cluster_arrive();
         tc::cluster_wait();
         float *qa = reinterpret_cast<float *>(smem + L.qall);
@@ -386,22 +392,22 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     __syncthreads();
 
     constexpr int NV = D / 64;  // float4 per lane per chunk row
-    constexpr int LOGCL = CL == 8 ? 3 : CL == 4 ? 2 : CL == 2 ? 1 : 0;
+    constexpr int LOGR = R == 8 ? 3 : R == 4 ? 2 : R == 2 ? 1 : 0;
     const int half = lane >> 4, s16 = lane & 15;
-    float4 qr[CL][NV];
+    float4 qr[R][NV];
 #pragma unroll
-    for (int mb = 0; mb < CL; ++mb)
+    for (int mb = 0; mb < R; ++mb)
 #pragma unroll
         for (int u = 0; u < NV; ++u) qr[mb][u] = *reinterpret_cast<const float4 *>(qall + mb * D + 4 * s16 + 64 * u);
-    uint32_t *sc = reinterpret_cast<uint32_t *>(smem + L.sc);  // [CL][ns] score images of the slice
-    const int my_mb = s16 >> (4 - LOGCL);
-    const bool writer = (s16 & ((1 << (4 - LOGCL)) - 1)) == 0;
+    uint32_t *sc = reinterpret_cast<uint32_t *>(smem + L.sc);  // [R][ns] score images of the slice
+    const int my_mb = s16 >> (4 - LOGR);
+    const bool writer = (s16 & ((1 << (4 - LOGR)) - 1)) == 0;
     bool ok = true;
     int done = 0;  // tiles this thread waited for successfully
     // rounds of up to kRound tiles: the round's chunks sit contiguously in the
     // ring, every warp takes chunk pairs warp, warp + kWarps, ... of the round;
-    // with 2 * kRound slots the next round's copies are in flight meanwhile
-    constexpr int UNR = CL >= 8 ? 1 : 2;  // chunk pairs in flight per warp
+    // with more slots the next rounds' copies are in flight meanwhile
+    constexpr int UNR = R >= 8 ? 1 : R >= 2 ? 2 : 4;  // chunk pairs in flight per warp
     for (int t0 = 0; t0 < ntiles; t0 += kRound) {
         const int t1 = min(ntiles, t0 + kRound);
         for (int t = t0; t < t1; ++t) {
@@ -413,7 +419,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
             const int rows = min((t1 - t0) * TCN, n_slice - t0 * TCN);
             const int npairs = (rows + 1) >> 1;
             for (int pr0 = warp; pr0 < npairs; pr0 += UNR * kWarps) {  // warp-uniform
-                float v[UNR][CL];
+                float v[UNR][R];
 #pragma unroll
                 for (int q = 0; q < UNR; ++q) {
                     const int cl = 2 * (pr0 + q * kWarps) + half;
@@ -424,7 +430,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
                         x[u] = valid ? *reinterpret_cast<const float4 *>(chunks + cl * D + 4 * s16 + 64 * u)
                                      : make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                    for (int mb = 0; mb < CL; ++mb) {
+                    for (int mb = 0; mb < R; ++mb) {
                         float acc = 0.f;
 #pragma unroll
                         for (int u = 0; u < NV; ++u) {
@@ -441,7 +447,7 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
 #pragma unroll
                 for (int st = 0; st < 4; ++st) {
                     const int o = 8 >> st;
-                    const int w = CL >> st;
+                    const int w = R >> st;
 #pragma unroll
                     for (int q = 0; q < UNR; ++q) {
                         if (w > 1) {
@@ -472,31 +478,36 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
         }
     }
 
-    // 3. this query block's full score row, then the CTA selects
+    // 3. this query block's full score row, then the CTA selects (SPLIT: rank 0
+    //    gathers the one block's row and selects)
+    const bool selector = !SPLIT || rank == 0;
     uint32_t *row = sc;
     if constexpr (CL > 1) {
         tc::cluster_arrive();
         tc::cluster_wait();
         uint32_t *rw = reinterpret_cast<uint32_t *>(smem + L.row);
         const int n4 = a.ns / 4;
-        for (int t = tid; t < CL * n4; t += kThreads) {
-            const int r = t / n4, o = t % n4;
-            const int j = r * a.ns + 4 * o;
-            if (j < n)
-                *reinterpret_cast<uint4 *>(rw + j) = tc::ld_dsmem_v4(
-                    tc::mapa_shared(tc::smem_u32(sc + rank * a.ns + 4 * o), static_cast<uint32_t>(r)));
+        const int my_row = SPLIT ? 0 : rank;  // this block's row in every peer's score slices
+        if (selector) {
+            for (int t = tid; t < CL * n4; t += kThreads) {
+                const int r = t / n4, o = t % n4;
+                const int j = r * a.ns + 4 * o;
+                if (j < n)
+                    *reinterpret_cast<uint4 *>(rw + j) = tc::ld_dsmem_v4(
+                        tc::mapa_shared(tc::smem_u32(sc + my_row * a.ns + 4 * o), static_cast<uint32_t>(r)));
+            }
         }
         tc::cluster_arrive();  // done reading the peers' shared memory
         row = rw;
     }
     __syncthreads();
-    if (a.sink > 0) {
+    if (a.sink > 0 && selector) {
         // the sink chunks outrank every score (the largest image; ties among them
         // go to the lower index, so they are listed first)
         for (int j = tid; j < a.sink && j < n; j += kThreads) row[j] = 0xFFFFFFFFu;
-        __syncthreads();
     }
-    if (!abort_flag) {
+    __syncthreads();
+    if (!abort_flag && selector) {
         SelScratch ss;
         ss.tmax = reinterpret_cast<uint32_t *>(smem + L.tmax);
         ss.key = reinterpret_cast<uint64_t *>(smem + L.key);
@@ -509,9 +520,9 @@ __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
     if constexpr (CL > 1) tc::cluster_wait();  // peers may still read this CTA's slice
 }
 
-template <typename T, int D, int CL>
+template <typename T, int D, int CL, bool SPLIT>
 cudaError_t launch_cl(const RouteArgs &a, unsigned grid, cudaStream_t stream) {
-    auto kern = route_kernel<T, D, CL>;
+    auto kern = route_kernel<T, D, CL, SPLIT>;
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), a.L.total);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
@@ -530,12 +541,19 @@ cudaError_t launch_cl(const RouteArgs &a, unsigned grid, cudaStream_t stream) {
 }
 
 template <typename T, int D>
-cudaError_t launch_t(const RouteArgs &a, int cl, unsigned grid, cudaStream_t stream) {
+cudaError_t launch_t(const RouteArgs &a, int cl, bool split, unsigned grid, cudaStream_t stream) {
+    if (split) {
+        switch (cl) {
+        case 8: return launch_cl<T, D, 8, true>(a, grid, stream);
+        case 4: return launch_cl<T, D, 4, true>(a, grid, stream);
+        default: return launch_cl<T, D, 2, true>(a, grid, stream);
+        }
+    }
     switch (cl) {
-    case 8: return launch_cl<T, D, 8>(a, grid, stream);
-    case 4: return launch_cl<T, D, 4>(a, grid, stream);
-    case 2: return launch_cl<T, D, 2>(a, grid, stream);
-    default: return launch_cl<T, D, 1>(a, grid, stream);
+    case 8: return launch_cl<T, D, 8, false>(a, grid, stream);
+    case 4: return launch_cl<T, D, 4, false>(a, grid, stream);
+    case 2: return launch_cl<T, D, 2, false>(a, grid, stream);
+    default: return launch_cl<T, D, 1, false>(a, grid, stream);
     }
 }
 
@@ -550,7 +568,9 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     // fit one round of bulk copies, else the largest
     const int ring_chunks = kRound * (kTileBytes / (D * 4));
     // a grid of less than one CTA per SM keeps two rounds in flight (two CTAs
-    // per SM overlap each other's copies otherwise) when that layout fits
+    // per SM overlap each other's copies otherwise) when that layout fits; more
+    // slots do not help: one SM's bulk copies stream at about 40 GB/s however
+    // many are in flight
     const bool small_grid = (long long)p.batch * p.n_kv_heads * nqb < sm_count();
     int cl = 1, slots = kRound;
     RouteLayout L{};
@@ -558,12 +578,12 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
         if (sl > kRound && !small_grid) continue;
         slots = sl;
         cl = 1;
-        L = route_layout(D, esize, 1, round4(n), n, sl);
+        L = route_layout(D, esize, 1, round4(n), n, sl, 1);
         if (n > p.topk) {
             for (int c : {1, 2, 4, 8}) {
                 if (nqb % c) continue;
                 const RouteLayout Lc =
-                    route_layout(D, esize, c, c > 1 ? round4((n + c - 1) / c) : round4(n), n, sl);
+                    route_layout(D, esize, c, c > 1 ? round4((n + c - 1) / c) : round4(n), n, sl, c);
                 if (Lc.total > kMaxSmem) continue;
                 cl = c;
                 L = Lc;
@@ -571,6 +591,27 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
             }
         }
         if (L.total <= kMaxSmem) break;
+    }
+    // one query block per (b, g) and more chunks than one round: a cluster of the
+    // largest size that keeps the grid within one CTA per SM splits the chunk
+    // list (rank 0 selects)
+    bool split = false;
+    if (nqb == 1 && n > p.topk && n > ring_chunks) {
+        const long long groups = (long long)p.batch * p.n_kv_heads;
+        const int sms = sm_count();
+        int c_best = 1;
+        for (int c : {2, 4, 8})
+            if (groups * c <= sms && (n + c - 1) / c >= ring_chunks / 2) c_best = c;
+        if (c_best > 1) {
+            const int sl = 2 * kRound;
+            const RouteLayout Lc = route_layout(D, esize, c_best, round4((n + c_best - 1) / c_best), n, sl, 1);
+            if (Lc.total <= kMaxSmem) {
+                split = true;
+                cl = c_best;
+                slots = sl;
+                L = Lc;
+            }
+        }
     }
     if (L.total > kMaxSmem) {
         record_error("hga_route: shared-memory layout exceeds the per-CTA limit");
@@ -593,13 +634,13 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     a.slots = slots;
     a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
     a.L = L;
-    const unsigned grid = static_cast<unsigned>(p.batch * p.n_kv_heads * nqb);
+    const unsigned grid = static_cast<unsigned>(p.batch * p.n_kv_heads * (split ? cl : nqb));
     cudaError_t e;
     if (p.dtype == HGA_BF16)
-        e = D == 128 ? launch_t<__nv_bfloat16, 128>(a, cl, grid, stream)
-                     : launch_t<__nv_bfloat16, 64>(a, cl, grid, stream);
+        e = D == 128 ? launch_t<__nv_bfloat16, 128>(a, cl, split, grid, stream)
+                     : launch_t<__nv_bfloat16, 64>(a, cl, split, grid, stream);
     else
-        e = D == 128 ? launch_t<float, 128>(a, cl, grid, stream) : launch_t<float, 64>(a, cl, grid, stream);
+        e = D == 128 ? launch_t<float, 128>(a, cl, split, grid, stream) : launch_t<float, 64>(a, cl, split, grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
     return record_cuda(e);
 }

@@ -209,9 +209,12 @@ hga_status_t hga_attn_bwd_noalloc(const hga_params_t *p, const void *q, const vo
  *   out: device [B][Hq][1][D] dtype.  lse: device fp32 [B][Hq][1] (natural log).
  *   workspace: device, at least hga_attn_decode_workspace_size(p, n_local)
  *     bytes, 16-byte aligned (per-split partial results; nothing in it needs
- *     clearing).
+ *     clearing).  The size depends on the current device's SM count (the
+ *     split count fills one wave): query it with that device current.
  * Two kernels on stream (split-K partial attention, then the merge); nothing
- * is allocated.  Out-of-range route indices are skipped and flagged. */
+ * is allocated.  Out-of-range route indices are skipped and flagged.  bf16
+ * reads K/V through TMA tensor maps: HGA_ERR_UNSUPPORTED when they cannot be
+ * encoded (no driver entry point). */
 size_t hga_attn_decode_workspace_size(const hga_params_t *p, int n_local);
 hga_status_t hga_attn_decode(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                              const void *k_local, const void *v_local, int n_local, const int32_t *idx,
