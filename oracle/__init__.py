@@ -25,7 +25,7 @@ _ip = ctypes.POINTER(ctypes.c_int)
 class Shape(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in (
         "batch", "n_q_heads", "n_kv_heads", "head_dim", "chunk", "q_block", "topk", "seg_len",
-        "n_hist_chunks", "sink_chunks")]
+        "n_hist_chunks", "sink_chunks", "group", "topg")]
 
 
 def build(force: bool = False) -> str:
@@ -53,8 +53,9 @@ def lib():
         _lib.oracle_attn_bwd.argtypes = [ctypes.POINTER(Shape), _dp, _dp, _dp, _dp, _dp, _ip, _dp,
                                          ctypes.c_void_p, ctypes.c_void_p, _dp, _dp, _dp]
         _lib.oracle_dense_causal.argtypes = [ctypes.POINTER(Shape), _dp, _dp, _dp, _dp, _dp]
+        _lib.oracle_route_groups.argtypes = [ctypes.POINTER(Shape), _dp, _dp, _ip, _ip, _dp]
         for f in ("oracle_summaries", "oracle_route", "oracle_attn_fwd", "oracle_attn_bwd",
-                  "oracle_dense_causal"):
+                  "oracle_dense_causal", "oracle_route_groups"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -73,9 +74,11 @@ def _check(rc: int, what: str):
 
 
 def shape(batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks,
-          sink_chunks=0) -> Shape:
+          sink_chunks=0, group=0, topg=0) -> Shape:
+    """group > 0 turns on the group stage: attention reads group routes (topg
+    groups of `group` tokens per query block) instead of chunk routes."""
     return Shape(batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks,
-                 sink_chunks)
+                 sink_chunks, group, topg)
 
 
 def summaries(k, chunk: int, n_chunks: int | None = None) -> np.ndarray:
@@ -101,6 +104,22 @@ def route(sh: Shape, q, summ, with_scores: bool = False):
     if scores is not None:
         scores = scores[..., :sh.n_hist_chunks]
     return idx, gap, scores
+
+
+def route_groups(sh: Shape, q, gsumm, idx):
+    """Second routing stage: (gidx int32 [B][Hkv][nqb][topg], gap [B][Hkv][nqb]).
+
+    gsumm: group summaries [B][Hkv][Nc * chunk / group][D] (``summaries(k, group)``);
+    idx: the chunk routes of ``route``.
+    """
+    q, gsumm = _f64(q), _f64(gsumm)
+    idx = np.ascontiguousarray(idx, dtype=np.int32)
+    nqb = sh.seg_len // sh.q_block
+    gidx = np.zeros((sh.batch, sh.n_kv_heads, nqb, sh.topg), dtype=np.int32)
+    gap = np.zeros((sh.batch, sh.n_kv_heads, nqb), dtype=np.float64)
+    _check(lib().oracle_route_groups(ctypes.byref(sh), _p(q), _p(gsumm), idx.ctypes.data_as(_ip),
+                                     gidx.ctypes.data_as(_ip), _p(gap)), "oracle_route_groups")
+    return gidx, gap
 
 
 def attn_fwd(sh: Shape, q, k_hist, v_hist, k_seg, v_seg, idx, rows=None):

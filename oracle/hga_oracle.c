@@ -31,7 +31,14 @@
  *   selection = the min(k, Nc) best chunks by (score descending, chunk index
  *     ascending), emitted in ascending chunk order, padded with -1;
  *   local window = every active-segment token at or before the query;
- *   no attention sink and no 8-token group stage.
+ *   sink window (sink_chunks = s): the first s history chunks are always
+ *     chosen, inside the k slots;
+ *   group stage (group = gs > 0) [TS2.1, group selection]: each chosen chunk
+ *     is split into c / gs groups of gs consecutive tokens; group summary =
+ *     mean of its gs keys; group score = dot(query-block summary, group
+ *     summary) / sqrt(D); the block keeps the topg best groups of its chosen
+ *     chunks by (score descending, group index ascending), emitted in
+ *     ascending group order and padded with -1, and attends their tokens.
  *
  * Layouts (row-major, D contiguous):
  *   q, dout, out, dq   [B][Hq][S][D]
@@ -48,6 +55,8 @@
 typedef struct {
     int batch, n_q_heads, n_kv_heads, head_dim, chunk, q_block, topk, seg_len, n_hist_chunks;
     int sink_chunks; /* attention-sink window: history chunks 0..sink_chunks-1 are always routed */
+    int group;       /* group stage: tokens per group (divides chunk); 0 = attend whole chunks */
+    int topg;        /* group stage: groups kept per query block */
 } oracle_shape_t;
 
 static long long ix4(long long a, long long A1, long long b, long long B1, long long c, long long C1, long long d)
@@ -165,21 +174,102 @@ int oracle_route(const oracle_shape_t *p, const double *q, const double *summ,
     return 0;
 }
 
+/* [TS2.1, group selection] second routing stage: for each query block, the
+ * groups of gs = p->group tokens inside its chosen chunks (idx, from
+ * oracle_route) are scored against the same query-block summary with their
+ * group summaries gsumm ([B][Hkv][Nc * c / gs][D], the mean of each group's
+ * keys), and the topg best (score descending, group index ascending) are
+ * kept.  gidx ([B][Hkv][S/q_block][topg]) gets the global group ids
+ * (chunk * c / gs + group within the chunk) in ascending order, padded with
+ * -1 when the chosen chunks hold fewer than topg groups.  gap (optional) gets
+ * the relative distance between the topg-th and (topg+1)-th best group
+ * scores, +inf when every candidate group is kept. */
+int oracle_route_groups(const oracle_shape_t *p, const double *q, const double *gsumm, const int *idx,
+                        int *gidx, double *gap)
+{
+    const int B = p->batch, Hkv = p->n_kv_heads, D = p->head_dim, Nc = p->n_hist_chunks, K = p->topk;
+    const int gs = p->group, KG = p->topg;
+    if (p->n_q_heads % Hkv || p->seg_len % p->q_block || K <= 0 || gs <= 0 || p->chunk % gs || KG <= 0)
+        return -1;
+    const int gpc = p->chunk / gs;  /* groups per chunk */
+    const int Ng = Nc * gpc;        /* groups in the history */
+    const int nqb = p->seg_len / p->q_block;
+    const int ncand_max = K * gpc;
+    double *qbar = (double *)malloc(sizeof(double) * D);
+    double *s = (double *)malloc(sizeof(double) * ncand_max);
+    int *cand = (int *)malloc(sizeof(int) * ncand_max);
+    int *order = (int *)malloc(sizeof(int) * (ncand_max + 1));
+    char *taken = (char *)malloc(ncand_max);
+    if (!qbar || !s || !cand || !order || !taken) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < Hkv; ++g)
+            for (int m = 0; m < nqb; ++m) {
+                query_block_summary(p, q, b, g, m, qbar);
+                /* the candidate groups: every group of every chosen chunk, ascending */
+                const int *sel = idx + ix4(b, Hkv, g, nqb, m, K, 0);
+                int nc = 0;
+                for (int a = 0; a < K; ++a) {
+                    const int j = sel[a];
+                    if (j < 0 || j >= Nc) continue;
+                    for (int u = 0; u < gpc; ++u) cand[nc++] = j * gpc + u;
+                }
+                for (int c = 0; c < nc; ++c) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += qbar[d] * gsumm[ix4(b, Hkv, g, Ng, cand[c], D, d)];
+                    s[c] = dot / sqrt((double)D);
+                }
+                /* plain selection of the best remaining candidate, kg times (and one
+                 * more for the gap) */
+                const int kg = KG < nc ? KG : nc;
+                memset(taken, 0, ncand_max);
+                const int n_rank = kg + (nc > kg ? 1 : 0);
+                for (int r = 0; r < n_rank; ++r) {
+                    int best = -1;
+                    for (int c = 0; c < nc; ++c)
+                        if (!taken[c] && (best < 0 || ranks_before(s[c], cand[c], s[best], cand[best]))) best = c;
+                    order[r] = best;
+                    if (r < kg) taken[best] = 1;
+                }
+                int *out = gidx + ix4(b, Hkv, g, nqb, m, KG, 0);
+                int w = 0;
+                for (int c = 0; c < nc; ++c) /* candidates are in ascending group order */
+                    if (taken[c]) out[w++] = cand[c];
+                for (; w < KG; ++w) out[w] = -1;
+                if (gap) {
+                    double g_rel = INFINITY;
+                    if (nc > kg && kg > 0) {
+                        double a = s[order[kg - 1]], c2 = s[order[kg]];
+                        double den = fabs(a) > fabs(c2) ? fabs(a) : fabs(c2);
+                        if (den < 1e-30) den = 1e-30;
+                        g_rel = (a - c2) / den;
+                    }
+                    gap[(b * Hkv + g) * nqb + m] = g_rel;
+                }
+            }
+    free(qbar); free(s); free(cand); free(order); free(taken);
+    return 0;
+}
+
 /* The key set U_i of query (b, h, i) [TS2.1, ABS]: the tokens of the routed
- * history chunks followed by the active-segment tokens 0..i.  Returns the
- * count and fills pointers to each key and value row. */
+ * history chunks (with the group stage: of the routed groups) followed by the
+ * active-segment tokens 0..i.  Returns the count and fills pointers to each
+ * key and value row. */
 static int gather_keys(const oracle_shape_t *p, const double *k_hist, const double *v_hist,
                        const double *k_seg, const double *v_seg, const int *idx,
                        int b, int g, int i, const double **kr, const double **vr, int *seg_pos)
 {
-    const int Hkv = p->n_kv_heads, D = p->head_dim, c = p->chunk, S = p->seg_len, K = p->topk;
+    const int Hkv = p->n_kv_heads, D = p->head_dim, S = p->seg_len;
+    /* routing unit: a chunk, or a group of the group stage */
+    const int c = p->group > 0 ? p->group : p->chunk;
+    const int K = p->group > 0 ? p->topg : p->topk;
+    const int n_units = p->group > 0 ? p->n_hist_chunks * (p->chunk / p->group) : p->n_hist_chunks;
     const int nqb = S / p->q_block, m = i / p->q_block;
-    const long long T = (long long)p->n_hist_chunks * c;
+    const long long T = (long long)p->n_hist_chunks * p->chunk;
     int n = 0;
     const int *sel = idx + ix4(b, Hkv, g, nqb, m, K, 0);
     for (int a = 0; a < K; ++a) {
         int j = sel[a];
-        if (j < 0 || j >= p->n_hist_chunks) continue;
+        if (j < 0 || j >= n_units) continue;
         for (int r = 0; r < c; ++r) {
             long long t = (long long)j * c + r;
             kr[n] = k_hist + (((long long)b * Hkv + g) * T + t) * D;
@@ -230,7 +320,8 @@ int oracle_attn_fwd(const oracle_shape_t *p, const double *q, const double *k_hi
     const int Hq = p->n_q_heads, Hkv = p->n_kv_heads, D = p->head_dim, S = p->seg_len;
     if (Hq % Hkv || S % p->q_block) return -1;
     const int G = Hq / Hkv;
-    const long long cap = (long long)p->topk * p->chunk + S;
+    const long long hist_cap = p->group > 0 ? (long long)p->topg * p->group : (long long)p->topk * p->chunk;
+    const long long cap = hist_cap + S;
     const double **kr = (const double **)malloc(sizeof(double *) * cap);
     const double **vr = (const double **)malloc(sizeof(double *) * cap);
     int *pos = (int *)malloc(sizeof(int) * cap);
@@ -268,7 +359,8 @@ int oracle_attn_bwd(const oracle_shape_t *p, const double *q, const double *k_hi
     const int B = p->batch, Hq = p->n_q_heads, Hkv = p->n_kv_heads, D = p->head_dim, S = p->seg_len;
     if (Hq % Hkv || S % p->q_block) return -1;
     const int G = Hq / Hkv;
-    const long long cap = (long long)p->topk * p->chunk + S;
+    const long long hist_cap = p->group > 0 ? (long long)p->topg * p->group : (long long)p->topk * p->chunk;
+    const long long cap = hist_cap + S;
     const double **kr = (const double **)malloc(sizeof(double *) * cap);
     const double **vr = (const double **)malloc(sizeof(double *) * cap);
     int *pos = (int *)malloc(sizeof(int) * cap);

@@ -446,3 +446,167 @@ def test_decode_token_equals_masked_attention():
     ref_out, ref_lse = _sdpa(sh, q, kh, vh, ks, vs, _allowed_mask(sh, idx))
     assert np.allclose(out[:, :, L - 1], ref_out[:, :, L - 1], atol=1e-12)
     assert np.allclose(lse[:, :, L - 1], ref_lse[:, :, L - 1], atol=1e-12)
+
+
+# ------------------------------------------------- group-level second-stage routing
+
+def _group_mask(sh, gidx):
+    """Boolean [B][Hkv][S][T+S]: routed groups' tokens + the causal segment."""
+    T = sh.n_hist_chunks * sh.chunk
+    S = sh.seg_len
+    mask = np.zeros((sh.batch, sh.n_kv_heads, S, T + S), dtype=bool)
+    for b in range(sh.batch):
+        for g in range(sh.n_kv_heads):
+            for i in range(S):
+                for u in gidx[b, g, i // sh.q_block]:
+                    if u >= 0:
+                        mask[b, g, i, u * sh.group:(u + 1) * sh.group] = True
+                mask[b, g, i, T:T + i + 1] = True
+    return mask
+
+
+def test_group_summaries_average_to_the_chunk_summary():
+    """A chunk's summary (mean of its c keys) is the mean of its c / gs group summaries
+    (means of equal-size parts), and a linear ramp K[t] = t v gives group j the summary
+    (gs j + (gs - 1) / 2) v."""
+    rng = np.random.default_rng(61)
+    k = rng.standard_normal((2, 3, 5 * 64, 16))
+    chunk = oracle.summaries(k, 64)
+    groups = oracle.summaries(k, 8)
+    assert groups.shape == (2, 3, 40, 16)
+    assert np.allclose(groups.reshape(2, 3, 5, 8, 16).mean(axis=3), chunk, rtol=1e-13, atol=1e-13)
+    v = rng.standard_normal(16)
+    ramp = np.arange(128, dtype=np.float64)[None, None, :, None] * v
+    g = oracle.summaries(ramp, 8)
+    for j in range(16):
+        assert np.allclose(g[0, 0, j], (8 * j + 3.5) * v, rtol=1e-14, atol=1e-12)
+
+
+def test_route_groups_constructed_scores_stay_inside_the_chosen_chunks():
+    """Group scores built so the order is known: q-bar = e0 and group summaries whose
+    first coordinate is the score times sqrt(D).  The best groups of the chosen chunks
+    win (equal scores go to the lower group index); a higher-scoring group of an
+    unchosen chunk is never taken."""
+    D, c, gs, qb, S, nc = 4, 16, 8, 8, 16, 4
+    q = np.zeros((1, 2, S, D))
+    q[..., 0] = 1.0
+    gsumm = np.zeros((1, 1, nc * c // gs, D))
+    # groups 0..7: chunk j holds groups 2j, 2j + 1
+    gsumm[0, 0, :, 0] = np.array([1.0, 5.0, 9.0, 2.0, 4.0, 4.0, 3.0, 0.5]) * 2.0
+    idx = np.array([[[[0, 2, 3], [1, 2, -1]]]], dtype=np.int32)  # block 0: chunks 0, 2, 3; block 1: 1, 2
+    sh = oracle.shape(1, 2, 1, D, c, qb, 3, S, nc, 0, gs, 3)
+    gidx, gap = oracle.route_groups(sh, q, gsumm, idx)
+    # block 0 candidates: groups 0, 1 (1, 5), 4, 5 (4, 4), 6, 7 (3, 0.5): best 1, then 4 and 5 tie
+    assert list(gidx[0, 0, 0]) == [1, 4, 5]
+    # block 1 candidates: 2, 3 (9, 2), 4, 5 (4, 4): 2, 4, 5; group 1 of chunk 0 (5) is not a candidate
+    assert list(gidx[0, 0, 1]) == [2, 4, 5]
+    # the 3rd and 4th best of block 0 are 4 (group 5) and 3 (group 6): gap (4 - 3) / 4
+    assert gap[0, 0, 0] == pytest.approx(0.25, rel=1e-14)
+    # a tie at the budget edge goes to the lower index: topg = 2 keeps groups 1 and 4
+    sh2 = oracle.shape(1, 2, 1, D, c, qb, 3, S, nc, 0, gs, 2)
+    gidx2, gap2 = oracle.route_groups(sh2, q, gsumm, idx)
+    assert list(gidx2[0, 0, 0]) == [1, 4]
+    assert gap2[0, 0, 0] == 0.0
+    # topg = 1: the best group alone, gap between the best (5) and the runner-up (4)
+    sh1 = oracle.shape(1, 2, 1, D, c, qb, 3, S, nc, 0, gs, 1)
+    gidx1, gap1 = oracle.route_groups(sh1, q, gsumm, idx)
+    assert list(gidx1[0, 0, 0]) == [1] and list(gidx1[0, 0, 1]) == [2]
+    assert gap1[0, 0, 0] == pytest.approx(0.2, rel=1e-14)
+
+
+def test_route_groups_matches_a_numpy_ranking():
+    """Random layers: the group route is the top-topg of the candidate groups by
+    (score descending, group index ascending) (numpy lexsort over the candidates)."""
+    rng = np.random.default_rng(62)
+    B, Hq, Hkv, D, c, gs, qb, S, nc, k, kg = 2, 4, 2, 8, 16, 4, 8, 24, 7, 3, 5
+    sh = oracle.shape(B, Hq, Hkv, D, c, qb, k, S, nc, 0, gs, kg)
+    q = rng.standard_normal((B, Hq, S, D))
+    kh = rng.standard_normal((B, Hkv, nc * c, D))
+    idx, _, _ = oracle.route(sh, q, oracle.summaries(kh, c))
+    gsumm = oracle.summaries(kh, gs)
+    gidx, _ = oracle.route_groups(sh, q, gsumm, idx)
+    G = Hq // Hkv
+    for b in range(B):
+        for g in range(Hkv):
+            for m in range(S // qb):
+                qbar = q[b, g * G:(g + 1) * G, m * qb:(m + 1) * qb].mean(axis=(0, 1))
+                cand = np.array([j * (c // gs) + u for j in idx[b, g, m] if j >= 0 for u in range(c // gs)])
+                s = gsumm[b, g, cand] @ qbar / np.sqrt(D)
+                best = cand[np.lexsort((cand, -s))[:kg]]
+                assert list(gidx[b, g, m]) == sorted(best.tolist())
+
+
+def test_route_groups_pads_when_the_budget_exceeds_the_candidates():
+    rng = np.random.default_rng(63)
+    D, c, gs, qb, S, nc = 8, 16, 8, 16, 16, 3
+    sh = oracle.shape(1, 2, 1, D, c, qb, 2, S, nc, 0, gs, 6)  # 2 chunks x 2 groups < 6
+    q = rng.standard_normal((1, 2, S, D))
+    gsumm = rng.standard_normal((1, 1, nc * 2, D))
+    idx = np.array([[[[0, 2]]]], dtype=np.int32)
+    gidx, gap = oracle.route_groups(sh, q, gsumm, idx)
+    assert list(gidx[0, 0, 0]) == [0, 1, 4, 5, -1, -1]
+    assert np.isinf(gap[0, 0, 0])
+
+
+def test_all_groups_of_the_chosen_chunks_equal_the_chunk_route():
+    """topg = k c / gs keeps every group of every chosen chunk: the same tokens in the
+    same order, so forward and backward equal the chunk-routed ones bit for bit."""
+    sh = _shape(Hq=4, Hkv=2, D=16, c=16, qb=16, k=2, S=48, Nc=5)
+    q, kh, vh, ks, vs = _random_layer(sh, seed=64)
+    idx, _, _ = oracle.route(sh, q, oracle.summaries(kh, 16))
+    shg = oracle.shape(1, 4, 2, 16, 16, 16, 2, 48, 5, 0, 4, 8)
+    gidx, gap = oracle.route_groups(shg, q, oracle.summaries(kh, 4), idx)
+    assert np.all(np.isinf(gap))
+    for b, g, m in np.ndindex(*idx.shape[:3]):
+        assert list(gidx[b, g, m]) == [4 * j + u for j in idx[b, g, m] for u in range(4)]
+    out, lse = oracle.attn_fwd(sh, q, kh, vh, ks, vs, idx)
+    outg, lseg = oracle.attn_fwd(shg, q, kh, vh, ks, vs, gidx)
+    assert np.array_equal(out, outg) and np.array_equal(lse, lseg)
+    dout = _rng(65).standard_normal(q.shape)
+    grads = oracle.attn_bwd(sh, q, kh, vh, ks, vs, idx, dout)
+    gradsg = oracle.attn_bwd(shg, q, kh, vh, ks, vs, gidx, dout)
+    for a, bb in zip(grads, gradsg):
+        assert np.array_equal(a, bb)
+
+
+def test_group_routes_equal_masked_attention_and_autograd():
+    """Attention over routed groups = torch attention (fp64) over an explicit mask of
+    the groups' tokens and the causal segment; the backward = torch autograd of it."""
+    sh = _shape(Hq=4, Hkv=2, D=16, c=16, qb=16, k=3, S=48, Nc=6)
+    q, kh, vh, ks, vs = _random_layer(sh, seed=66)
+    idx, _, _ = oracle.route(sh, q, oracle.summaries(kh, 16))
+    shg = oracle.shape(1, 4, 2, 16, 16, 16, 3, 48, 6, 0, 4, 5)
+    gidx, _ = oracle.route_groups(shg, q, oracle.summaries(kh, 4), idx)
+    mask = _group_mask(shg, gidx)
+    out, lse = oracle.attn_fwd(shg, q, kh, vh, ks, vs, gidx)
+    o_ref, lse_ref = _sdpa(shg, q, kh, vh, ks, vs, mask)
+    assert np.max(np.abs(out - o_ref)) < 1e-12
+    assert np.max(np.abs(lse - lse_ref)) < 1e-12
+    dout = _rng(67).standard_normal(q.shape)
+    dq, dk, dv = oracle.attn_bwd(shg, q, kh, vh, ks, vs, gidx, dout)
+    G = 2
+    qt = torch.from_numpy(q).requires_grad_()
+    kst = torch.from_numpy(ks).requires_grad_()
+    vst = torch.from_numpy(vs).requires_grad_()
+    k_all = torch.cat([torch.from_numpy(kh), kst], 2).repeat_interleave(G, 1)
+    v_all = torch.cat([torch.from_numpy(vh), vst], 2).repeat_interleave(G, 1)
+    m = torch.from_numpy(mask).repeat_interleave(G, dim=1)
+    o = torch.nn.functional.scaled_dot_product_attention(qt, k_all, v_all, attn_mask=m)
+    (o * torch.from_numpy(dout)).sum().backward()
+    assert np.max(np.abs(dq - qt.grad.numpy())) < 1e-12
+    assert np.max(np.abs(dk - kst.grad.numpy())) < 1e-12
+    assert np.max(np.abs(dv - vst.grad.numpy())) < 1e-12
+
+
+def test_group_attended_count():
+    """q = 0 makes every logit 0, so LSE = ln(#attended keys) = ln(gs * #routed groups + i + 1)."""
+    sh = oracle.shape(1, 2, 1, 8, 16, 8, 2, 24, 4, 0, 4, 3)
+    rng = np.random.default_rng(68)
+    q = np.zeros((1, 2, 24, 8))
+    kh, vh = rng.standard_normal((1, 1, 64, 8)), rng.standard_normal((1, 1, 64, 8))
+    ks, vs = rng.standard_normal((1, 1, 24, 8)), rng.standard_normal((1, 1, 24, 8))
+    gidx = np.array([[[[0, 5, 9], [2, -1, -1], [-1, -1, -1]]]], dtype=np.int32)
+    _, lse = oracle.attn_fwd(sh, q, kh, vh, ks, vs, gidx)
+    for i in range(24):
+        n_groups = (gidx[0, 0, i // 8] >= 0).sum()
+        assert lse[0, 0, i] == pytest.approx(math.log(4 * n_groups + i + 1), rel=1e-14)
