@@ -54,8 +54,9 @@ def lib():
                                          ctypes.c_void_p, ctypes.c_void_p, _dp, _dp, _dp]
         _lib.oracle_dense_causal.argtypes = [ctypes.POINTER(Shape), _dp, _dp, _dp, _dp, _dp]
         _lib.oracle_route_groups.argtypes = [ctypes.POINTER(Shape), _dp, _dp, _ip, _ip, _dp]
+        _lib.oracle_route_causal.argtypes = [ctypes.POINTER(Shape), _dp, _dp, _ip, _dp]
         for f in ("oracle_summaries", "oracle_route", "oracle_attn_fwd", "oracle_attn_bwd",
-                  "oracle_dense_causal", "oracle_route_groups"):
+                  "oracle_dense_causal", "oracle_route_groups", "oracle_route_causal"):
             getattr(_lib, f).restype = ctypes.c_int
     return _lib
 
@@ -104,6 +105,20 @@ def route(sh: Shape, q, summ, with_scores: bool = False):
     if scores is not None:
         scores = scores[..., :sh.n_hist_chunks]
     return idx, gap, scores
+
+
+def route_causal(sh: Shape, q, summ):
+    """Strictly causal routes, one per token: (idx int32 [B][Hkv][S][k], gap [B][Hkv][S]).
+
+    Token i routes by the mean of its block's queries up to itself; attend with
+    a copy of the shape whose q_block is 1.
+    """
+    q, summ = _f64(q), _f64(summ)
+    idx = np.zeros((sh.batch, sh.n_kv_heads, sh.seg_len, sh.topk), dtype=np.int32)
+    gap = np.zeros((sh.batch, sh.n_kv_heads, sh.seg_len), dtype=np.float64)
+    _check(lib().oracle_route_causal(ctypes.byref(sh), _p(q), _p(summ), idx.ctypes.data_as(_ip), _p(gap)),
+           "oracle_route_causal")
+    return idx, gap
 
 
 def route_groups(sh: Shape, q, gsumm, idx):

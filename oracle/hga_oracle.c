@@ -106,6 +106,45 @@ static int ranks_before(double sa, int a, double sb, int b)
     return a < b;
 }
 
+/* The selection step of a route, given the Nc scores s of one routing query:
+ * the sink chunks first, then the best remaining chunk until k_eff chunks
+ * (and one more, for the gap) are ranked.  out gets the chosen ids in
+ * ascending order, -1 padded to K; *gap (if given) the relative distance
+ * between the last chunk taken by score and the next one (+inf if none). */
+static void select_chunks(const double *s, int Nc, int K, int sink_chunks, int *order, char *taken, int *out,
+                          double *gap)
+{
+    const int keff = K < Nc ? K : Nc;
+    memset(taken, 0, Nc > 0 ? Nc : 1);
+    const int n_sink = sink_chunks < keff ? (sink_chunks > 0 ? sink_chunks : 0) : keff;
+    for (int r = 0; r < n_sink; ++r) {
+        order[r] = r;
+        taken[r] = 1;
+    }
+    int n_rank = keff + (Nc > keff ? 1 : 0);
+    for (int r = n_sink; r < n_rank; ++r) {
+        int best = -1;
+        for (int j = 0; j < Nc; ++j)
+            if (!taken[j] && (best < 0 || ranks_before(s[j], j, s[best], best))) best = j;
+        order[r] = best;
+        if (r < keff) taken[best] = 1;
+    }
+    int w = 0;
+    for (int j = 0; j < Nc; ++j)
+        if (taken[j]) out[w++] = j;
+    for (; w < K; ++w) out[w] = -1;
+    if (gap) {
+        double g_rel = INFINITY;
+        if (Nc > keff && keff > n_sink) {
+            double a = s[order[keff - 1]], c = s[order[keff]];
+            double den = fabs(a) > fabs(c) ? fabs(a) : fabs(c);
+            if (den < 1e-30) den = 1e-30;
+            g_rel = (a - c) / den;
+        }
+        *gap = g_rel;
+    }
+}
+
 /* [TS2.1] routing: score every closed history chunk against the query-block
  * summary and keep the k best.  idx gets the chosen chunk ids in ascending
  * order, padded with -1 when k > Nc.  gap (optional) gets, per query block,
@@ -126,7 +165,6 @@ int oracle_route(const oracle_shape_t *p, const double *q, const double *summ,
     int *order = (int *)malloc(sizeof(int) * (Nc > 0 ? Nc : 1));
     char *taken = (char *)malloc(Nc > 0 ? Nc : 1);
     if (!qbar || !s || !order || !taken) return -2;
-    const int keff = K < Nc ? K : Nc;
     for (int b = 0; b < B; ++b)
         for (int g = 0; g < Hkv; ++g)
             for (int m = 0; m < nqb; ++m) {
@@ -137,40 +175,52 @@ int oracle_route(const oracle_shape_t *p, const double *q, const double *summ,
                     s[j] = dot / sqrt((double)D);
                     if (scores) scores[ix4(b, Hkv, g, nqb, m, Nc, j)] = s[j];
                 }
-                /* plain selection: the sink chunks first, then the best remaining
-                 * chunk until k_eff chunks (and one more, for the gap) are ranked */
-                memset(taken, 0, Nc > 0 ? Nc : 1);
-                const int n_sink = p->sink_chunks < keff ? (p->sink_chunks > 0 ? p->sink_chunks : 0) : keff;
-                for (int r = 0; r < n_sink; ++r) {
-                    order[r] = r;
-                    taken[r] = 1;
-                }
-                int n_rank = keff + (Nc > keff ? 1 : 0);
-                for (int r = n_sink; r < n_rank; ++r) {
-                    int best = -1;
-                    for (int j = 0; j < Nc; ++j)
-                        if (!taken[j] && (best < 0 || ranks_before(s[j], j, s[best], best))) best = j;
-                    order[r] = best;
-                    if (r < keff) taken[best] = 1;
-                }
-                int *out = idx + ix4(b, Hkv, g, nqb, m, K, 0);
-                /* emit the chosen ids in ascending chunk order */
-                int w = 0;
-                for (int j = 0; j < Nc; ++j)
-                    if (taken[j]) out[w++] = j;
-                for (; w < K; ++w) out[w] = -1;
-                if (gap) {
-                    double g_rel = INFINITY;
-                    if (Nc > keff && keff > n_sink) {
-                        double a = s[order[keff - 1]], c = s[order[keff]];
-                        double den = fabs(a) > fabs(c) ? fabs(a) : fabs(c);
-                        if (den < 1e-30) den = 1e-30;
-                        g_rel = (a - c) / den;
-                    }
-                    gap[(b * Hkv + g) * nqb + m] = g_rel;
-                }
+                select_chunks(s, Nc, K, p->sink_chunks, order, taken, idx + ix4(b, Hkv, g, nqb, m, K, 0),
+                              gap ? gap + (b * Hkv + g) * nqb + m : NULL);
             }
     free(qbar); free(s); free(order); free(taken);
+    return 0;
+}
+
+/* [TS5, causal leakage; TS2.1] strictly causal routing: sharing one route
+ * among the tokens of a block lets a token's route depend on later tokens;
+ * here every token routes by the summary of its block's queries up to and
+ * including itself (the mean over the G heads of the group and the queries
+ * m*q_block .. i), so nothing after i can change the route of i.  The last
+ * token of a block gets the block's route; with q_block = 1 every token
+ * routes alone.  idx gets one route per token, [B][Hkv][S][k] (use it with
+ * q_block = 1 in the attention); gap, if given, [B][Hkv][S]; the sink rule
+ * applies as in oracle_route. */
+int oracle_route_causal(const oracle_shape_t *p, const double *q, const double *summ, int *idx, double *gap)
+{
+    const int B = p->batch, Hq = p->n_q_heads, Hkv = p->n_kv_heads, D = p->head_dim, S = p->seg_len;
+    const int Nc = p->n_hist_chunks, K = p->topk;
+    if (Hq % Hkv || S % p->q_block || K <= 0) return -1;
+    const int G = Hq / Hkv;
+    double *qsum = (double *)malloc(sizeof(double) * D);
+    double *s = (double *)malloc(sizeof(double) * (Nc > 0 ? Nc : 1));
+    int *order = (int *)malloc(sizeof(int) * (Nc > 0 ? Nc : 1));
+    char *taken = (char *)malloc(Nc > 0 ? Nc : 1);
+    if (!qsum || !s || !order || !taken) return -2;
+    for (int b = 0; b < B; ++b)
+        for (int g = 0; g < Hkv; ++g)
+            for (int i = 0; i < S; ++i) {
+                const int start = (i / p->q_block) * p->q_block;
+                /* prefix summary of the block: queries start .. i of the G heads */
+                for (int d = 0; d < D; ++d) qsum[d] = 0.0;
+                for (int hh = 0; hh < G; ++hh)
+                    for (int t = start; t <= i; ++t)
+                        for (int d = 0; d < D; ++d) qsum[d] += q[ix4(b, Hq, g * G + hh, S, t, D, d)];
+                const double cnt = (double)G * (i - start + 1);
+                for (int j = 0; j < Nc; ++j) {
+                    double dot = 0.0;
+                    for (int d = 0; d < D; ++d) dot += (qsum[d] / cnt) * summ[ix4(b, Hkv, g, Nc, j, D, d)];
+                    s[j] = dot / sqrt((double)D);
+                }
+                select_chunks(s, Nc, K, p->sink_chunks, order, taken, idx + ix4(b, Hkv, g, S, i, K, 0),
+                              gap ? gap + ((long long)b * Hkv + g) * S + i : NULL);
+            }
+    free(qsum); free(s); free(order); free(taken);
     return 0;
 }
 

@@ -610,3 +610,79 @@ def test_group_attended_count():
     for i in range(24):
         n_groups = (gidx[0, 0, i // 8] >= 0).sum()
         assert lse[0, 0, i] == pytest.approx(math.log(4 * n_groups + i + 1), rel=1e-14)
+
+
+# ------------------------------------------------------------ strictly causal routing
+
+def _causal_layer(seed, B=2, Hq=4, Hkv=2, D=8, c=8, qb=8, S=24, nc=9, k=3, sink=0):
+    rng = np.random.default_rng(seed)
+    sh = oracle.shape(B, Hq, Hkv, D, c, qb, k, S, nc, sink)
+    q = rng.standard_normal((B, Hq, S, D))
+    kh = rng.standard_normal((B, Hkv, nc * c, D))
+    return sh, q, kh, oracle.summaries(kh, c)
+
+
+def test_causal_route_matches_a_numpy_prefix_ranking():
+    """Token i routes by the mean of its block's queries start .. i over the G heads
+    (numpy prefix means, lexsort by score then index)."""
+    sh, q, _, summ = _causal_layer(71)
+    idx, _ = oracle.route_causal(sh, q, summ)
+    G = sh.n_q_heads // sh.n_kv_heads
+    for b, g, i in np.ndindex(sh.batch, sh.n_kv_heads, sh.seg_len):
+        start = (i // sh.q_block) * sh.q_block
+        qbar = q[b, g * G:(g + 1) * G, start:i + 1].mean(axis=(0, 1))
+        s = summ[b, g] @ qbar / np.sqrt(sh.head_dim)
+        want = sorted(np.lexsort((np.arange(sh.n_hist_chunks), -s))[:sh.topk].tolist())
+        assert list(idx[b, g, i]) == want
+
+
+def test_causal_route_of_a_block_end_is_the_block_route():
+    """The last token of a block summarises the whole block, so it gets the block's
+    route (also with a sink window)."""
+    for sink in (0, 1):
+        sh, q, _, summ = _causal_layer(72, sink=sink)
+        idx_tok, gap_tok = oracle.route_causal(sh, q, summ)
+        idx_blk, gap_blk, _ = oracle.route(sh, q, summ)
+        for m in range(sh.seg_len // sh.q_block):
+            i = m * sh.q_block + sh.q_block - 1
+            assert np.array_equal(idx_tok[:, :, i], idx_blk[:, :, m])
+            assert np.array_equal(gap_tok[:, :, i], gap_blk[:, :, m])
+
+
+def test_causal_route_ignores_later_queries():
+    """The point of the variant: changing queries after i leaves the routes of tokens
+    0..i unchanged, while the block route of i's block changes with them."""
+    sh, q, _, summ = _causal_layer(73)
+    idx0, _ = oracle.route_causal(sh, q, summ)
+    blk0, _, _ = oracle.route(sh, q, summ)
+    q2 = q.copy()
+    q2[:, :, 11:] = -5.0 * q2[:, :, 11:] + 3.0   # everything after token 10 (block 1 spans 8..15)
+    idx1, _ = oracle.route_causal(sh, q2, summ)
+    blk1, _, _ = oracle.route(sh, q2, summ)
+    assert np.array_equal(idx0[:, :, :11], idx1[:, :, :11])
+    assert not np.array_equal(idx0[:, :, 11:], idx1[:, :, 11:])
+    assert not np.array_equal(blk0[:, :, 1], blk1[:, :, 1])  # the shared block route leaks
+
+
+def test_causal_routes_with_one_token_blocks_equal_the_plain_route():
+    sh, q, _, summ = _causal_layer(74, qb=1)
+    idx_tok, _ = oracle.route_causal(sh, q, summ)
+    idx_blk, _, _ = oracle.route(sh, q, summ)
+    assert np.array_equal(idx_tok, idx_blk)
+
+
+def test_attention_with_causal_routes_equals_masked_attention():
+    """Per-token routes drive the attention through a one-token-block shape: exact
+    attention over each token's own routed chunks and the causal segment (torch, fp64)."""
+    sh, q, kh, summ = _causal_layer(75, B=1)
+    idx_tok, _ = oracle.route_causal(sh, q, summ)
+    rng = np.random.default_rng(76)
+    vh = rng.standard_normal(kh.shape)
+    ks = rng.standard_normal((1, sh.n_kv_heads, sh.seg_len, sh.head_dim))
+    vs = rng.standard_normal((1, sh.n_kv_heads, sh.seg_len, sh.head_dim))
+    sh1 = oracle.shape(1, sh.n_q_heads, sh.n_kv_heads, sh.head_dim, sh.chunk, 1, sh.topk, sh.seg_len,
+                       sh.n_hist_chunks)
+    out, lse = oracle.attn_fwd(sh1, q, kh, vh, ks, vs, idx_tok)
+    o_ref, lse_ref = _sdpa(sh1, q, kh, vh, ks, vs, _allowed_mask(sh1, idx_tok))
+    assert np.max(np.abs(out - o_ref)) < 1e-12
+    assert np.max(np.abs(lse - lse_ref)) < 1e-12
