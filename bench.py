@@ -426,6 +426,22 @@ def tokens_per_step(w):
     return w.batch if w.decode else w.seg_len * w.batch * len(w.seg_starts)
 
 
+def workload_config(w, world):
+    """The workload keys of the JSON line's `config`, the same for both arms."""
+    cfg = {"workload": w.name, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
+           "head_dim": w.head_dim, "context": w.seq_len}
+    if w.decode:
+        cfg.update({"history_tokens": w.seg_starts[0], "local_window": w.seg_len, "topk": w.topk,
+                    "sink_chunks": w.sink_chunks, "chunk": w.chunk, "decode": True,
+                    "tokens_per_step": tokens_per_step(w)})
+    else:
+        cfg.update({"seg_len": w.seg_len, "topk": w.topk, "sink_chunks": w.sink_chunks, "chunk": w.chunk,
+                    "q_block": w.q_block, "segments_per_step": len(w.seg_starts), "backward": w.backward,
+                    "tiered": w.tiered})
+    cfg["parallelism"] = f"one independent layer per GPU x{world}"
+    return cfg
+
+
 def decode_oracle_sample(w, target_seconds):
     """The oracle on the decode token of sequence 0 (its inputs drawn alone with the same
     generator): its route (the oracle routes every token of the local window as a one-token
@@ -523,7 +539,7 @@ def run_reference(args, rank):
     line = {"impl": "reference", "metric": METRIC, "value": v, "unit": UNIT, "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": args.workload},
+            "config": workload_config(w, args.gpus),
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -653,12 +669,7 @@ def run_hga(args, rank, world, local):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "batch": w.batch, "q_heads": w.n_q_heads, "kv_heads": w.n_kv_heads,
-                       "head_dim": w.head_dim, "context": w.seq_len, "seg_len": w.seg_len, "topk": w.topk,
-                       "sink_chunks": w.sink_chunks,
-                       "chunk": w.chunk, "q_block": w.q_block, "segments_per_step": len(w.seg_starts),
-                       "backward": w.backward, "tiered": w.tiered,
-                       "parallelism": f"one independent layer per GPU x{world}",
+            "config": {**workload_config(w, world),
                        "l2": "flushed before every timed step (256 MiB write)",
                        "launch": "one CUDA graph replay per step" if graph is not None else "eager",
                        "append": "side stream, overlapped with the route" if layer.side_append else "in order"},
@@ -846,11 +857,7 @@ def run_decode(args, rank, world, local):
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "batch": B, "q_heads": Hq, "kv_heads": Hkv, "head_dim": D,
-                       "context": w.seq_len, "history_tokens": layer.T, "local_window": layer.n_local,
-                       "topk": w.topk, "sink_chunks": w.sink_chunks, "chunk": w.chunk, "decode": True,
-                       "tokens_per_step": tokens_per_step(w),
-                       "parallelism": f"one independent layer per GPU x{world}",
+            "config": {**workload_config(w, world),
                        "l2": "flushed before every timed step (256 MiB write)",
                        "launch": "one CUDA graph replay per step"},
             "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,

@@ -50,3 +50,23 @@ def test_max_over_ranks_and_weak_scaling_with_two_gloo_ranks():
 def test_single_rank_needs_no_process_group():
     assert bench.max_over_ranks(3.0, 1, "cpu") == 3.0
     assert bench.job_throughput(100, 2, 1, 1000.0) == 200.0
+
+
+def test_reference_arm_line_carries_the_workload_config(capsys):
+    """bench.py --impl reference times the oracle on the host and prints one JSON line
+    with the same metric, unit and workload config as the GPU arm's line."""
+    import argparse
+    import json
+
+    from inputs import gen
+    args = argparse.Namespace(workload="tiny_fp32", steps=1, warmup=0, gpus=1, cpu_seconds=0.5)
+    bench.run_reference(args, 0)
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["metric"] == bench.METRIC and line["unit"] == bench.UNIT
+    assert line["higher_is_better"] is True and line["value"] > 0
+    assert line["config"] == bench.workload_config(gen.WORKLOADS["tiny_fp32"], 1)
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    # other ranks print nothing
+    bench.run_reference(args, 1)
+    assert capsys.readouterr().out == ""
