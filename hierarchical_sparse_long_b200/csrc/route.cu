@@ -11,11 +11,12 @@
 //
 // One CTA per (batch, kv head, query block); CL consecutive query blocks of
 // one (batch, kv head) form a thread-block cluster.
-//   1. Summary tiles start streaming at once by bulk copies into a 4-slot
-//      shared-memory ring, while every thread loads its share of the block's
-//      G x q_block query rows straight into registers (16-byte loads, all in
-//      flight together) and the CTA sums them in a fixed order: the block
-//      summary qbar (fp32).
+//   1. Summary tiles start streaming at once by bulk copies into a shared-
+//      memory ring (4 slots; 8 when the grid is under one CTA per SM, so the
+//      next round is in flight while one is scored), while every thread loads
+//      its share of the block's G x q_block query rows straight into
+//      registers (16-byte loads, all in flight together) and the CTA sums
+//      them in a fixed order: the block summary qbar (fp32).
 //   2. The cluster's CL summaries are exchanged through distributed shared
 //      memory; each CTA scores its 1/CL slice of the chunks against all CL
 //      of them, so every chunk summary crosses L2 -> SM once per cluster.
