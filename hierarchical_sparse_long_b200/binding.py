@@ -21,7 +21,7 @@ HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT = 1, 2
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3: "HGA_ERR_CUDA",
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
-EXPORTED = ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
+EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
             "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_fetch_tiered",
             "hga_get_device_status", "hga_selftest_wait_timeout", "hga_status_string", "hga_last_error")
 
@@ -83,6 +83,7 @@ def lib() -> ctypes.CDLL:
         pp = ctypes.POINTER(CParams)
         L.hga_build_summaries.argtypes = [vp, ll, i, i, i, i, i, i, i, vp, i, vp]
         L.hga_route.argtypes = [pp, vp, vp, i, vp, vp]
+        L.hga_route_causal.argtypes = [pp, vp, vp, i, vp, vp]
         L.hga_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_attn_bwd_workspace_size.argtypes = [pp]
         L.hga_attn_bwd_workspace_size.restype = sz
@@ -98,7 +99,7 @@ def lib() -> ctypes.CDLL:
         L.hga_status_string.argtypes = [i]
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
-        for f in ("hga_build_summaries", "hga_route", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
+        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
                   "hga_attn_decode", "hga_fetch_tiered", "hga_get_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -146,6 +147,13 @@ def hga_route(p: Params, q, summ, summ_cap_chunks: int, idx, stream=None):
     cp = p.c()
     _check(lib().hga_route(ctypes.byref(cp), _ptr(q), _ptr(summ), summ_cap_chunks, _ptr(idx), _stream(stream)),
            "hga_route")
+
+
+def hga_route_causal(p: Params, q, summ, summ_cap_chunks: int, idx, stream=None):
+    """Strictly causal routing: one route per token into idx [B][Hkv][S][k] (int32)."""
+    cp = p.c()
+    _check(lib().hga_route_causal(ctypes.byref(cp), _ptr(q), _ptr(summ), summ_cap_chunks, _ptr(idx),
+                                  _stream(stream)), "hga_route_causal")
 
 
 def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stream=None):

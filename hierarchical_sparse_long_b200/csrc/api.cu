@@ -118,6 +118,19 @@ hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, 
     return hga::launch_route(*p, q, summ, summ_cap_chunks, idx, status, stream);
 }
 
+hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
+                              int32_t *idx, cudaStream_t stream) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (summ_cap_chunks < p->n_hist_chunks) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 16384) return HGA_ERR_UNSUPPORTED;
+    if (!q || !idx || !aligned16(q)) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!summ || !aligned16(summ))) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    return hga::launch_route_causal(*p, q, summ, summ_cap_chunks, idx, status, stream);
+}
+
 hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                           const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
                           cudaStream_t stream) {

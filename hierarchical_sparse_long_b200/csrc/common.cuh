@@ -55,6 +55,9 @@ hga_status_t launch_summaries(const void *k, long long head_stride, int bh, int 
                               cudaStream_t stream);
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
                           unsigned *status, cudaStream_t stream);
+// Strictly causal routes, one per token: idx [B][Hkv][S][topk].
+hga_status_t launch_route_causal(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
+                          unsigned *status, cudaStream_t stream);
 hga_status_t launch_attn_fwd_simt(const hga_params_t &p, const void *q, const void *k_hist,
                                   const void *v_hist, const void *k_seg, const void *v_seg,
                                   const int32_t *idx, void *out, float *lse, unsigned *status,

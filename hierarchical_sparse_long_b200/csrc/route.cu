@@ -558,6 +558,125 @@ cudaError_t launch_t(const RouteArgs &a, int cl, bool split, unsigned grid, cuda
     }
 }
 
+// ---------------------------------------------------------------------------
+// Strictly causal routing (the technical summary's limits section proposes a
+// strictly causal variant of the block-shared route): token i of block m
+// routes by the mean over the G heads of the block's queries start .. i, so no
+// later query can change its route.  One CTA per (b, g, m):
+//   1. the block's G-head row sums (all threads, independent loads), then one
+//      thread per dimension turns them into prefix means in row order;
+//   2. passes of TP tokens (TP x Nc score images fit in shared memory): every
+//      32-row summary tile is loaded once per pass and scored against the
+//      pass's TP prefix summaries (thread = one chunk row x TP/8 tokens; fp32
+//      FFMA in a fixed order, like route_kernel);
+//   3. each warp selects its tokens' top-k with the sink chunks stamped first.
+constexpr int kCTile = 32;  // summary rows per tile
+
+struct CausalLayout {
+    int qpre, tile, sc, hist, total, tp;
+};
+
+CausalLayout causal_layout(int D, int q_block, int n) {
+    CausalLayout L{};
+    const int n4 = n > 4 ? round4(n) : 4;
+    L.qpre = 0;
+    L.tile = L.qpre + q_block * D * 4;
+    L.hist = L.tile + kCTile * (D + 4) * 4;
+    L.sc = L.hist + kWarps * 256 * 4;
+    const int room = kMaxSmem - L.sc;
+    int tp = room / (n4 * 4);
+    tp = tp >= q_block ? q_block : (tp / kWarps) * kWarps;
+    L.tp = tp;
+    L.total = L.sc + (tp > 0 ? tp : kWarps) * n4 * 4;
+    return L;
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1) route_causal_kernel(const RouteArgs a, int tp, CausalLayout L) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int QB = a.q_block, nqb = a.seg_len / QB;
+    const int m = (int)blockIdx.x % nqb, bg = (int)blockIdx.x / nqb;
+    const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    const int n = a.n, n4 = n > 4 ? (n + 3) & ~3 : 4;  // score row stride, as in causal_layout
+    constexpr int DP = D + 4;  // padded tile row (conflict-free 16-byte reads across rows)
+    float *qpre = reinterpret_cast<float *>(smem + L.qpre);
+    float *tile = reinterpret_cast<float *>(smem + L.tile);
+    uint32_t *sc = reinterpret_cast<uint32_t *>(smem + L.sc);
+    int *hist = reinterpret_cast<int *>(smem + L.hist);
+    int32_t *out = a.idx + ((long long)bg * a.seg_len + (long long)m * QB) * a.topk;
+    if (n <= a.topk) {  // every chunk is routed for every token (the same branch for the whole grid)
+        for (int e = tid; e < QB * a.topk; e += kThreads) {
+            const int t = e % a.topk;
+            out[e] = t < n ? t : -1;
+        }
+        return;
+    }
+
+    // 1. prefix summaries
+    const T *qb = static_cast<const T *>(a.q) +
+                  (((long long)b * a.n_q_heads + (long long)g * G) * a.seg_len + (long long)m * QB) * D;
+    for (int e = tid; e < QB * D; e += kThreads) {
+        const int r = e / D, d = e % D;
+        float rs = 0.f;
+        for (int hh = 0; hh < G; ++hh) rs += to_f32(qb[((long long)hh * a.seg_len + r) * D + d]);
+        qpre[e] = rs;
+    }
+    __syncthreads();
+    for (int d = tid; d < D; d += kThreads) {
+        float run = 0.f;
+        for (int r = 0; r < QB; ++r) {
+            run += qpre[r * D + d];
+            qpre[r * D + d] = run / static_cast<float>(G * (r + 1));
+        }
+    }
+    __syncthreads();
+
+    const float *sbase = a.summ + (long long)bg * a.cap * D;
+    const int jj = tid % kCTile, tg = tid / kCTile;  // chunk row of the tile, token group
+    for (int t0 = 0; t0 < QB; t0 += tp) {
+        const int ntp = min(tp, QB - t0);
+        // 2. scores of tokens t0 .. t0 + ntp - 1, tile by tile
+        for (int j0 = 0; j0 < n; j0 += kCTile) {
+            const int rows = min(kCTile, n - j0);
+            __syncthreads();  // the previous tile is consumed
+            for (int e = tid; e < rows * (D / 4); e += kThreads) {
+                const int r = e / (D / 4), c = e % (D / 4);
+                *reinterpret_cast<float4 *>(tile + r * DP + 4 * c) =
+                    *reinterpret_cast<const float4 *>(sbase + (long long)(j0 + r) * D + 4 * c);
+            }
+            __syncthreads();
+            if (jj < rows) {
+                const float4 *sv = reinterpret_cast<const float4 *>(tile + jj * DP);
+                for (int tk = tg; tk < ntp; tk += kThreads / kCTile) {  // warp-uniform
+                    const float4 *qv = reinterpret_cast<const float4 *>(qpre + (t0 + tk) * D);
+                    float acc = 0.f;
+#pragma unroll 8
+                    for (int u = 0; u < D / 4; ++u) {
+                        const float4 x = qv[u], y = sv[u];
+                        acc = fmaf(x.x, y.x, acc);
+                        acc = fmaf(x.y, y.y, acc);
+                        acc = fmaf(x.z, y.z, acc);
+                        acc = fmaf(x.w, y.w, acc);
+                    }
+                    sc[tk * n4 + j0 + jj] = ordered_bits(acc * a.inv_sqrt_d);
+                }
+            }
+        }
+        __syncthreads();
+        // 3. one warp per token: sink chunks first, then the radix select over the row
+        for (int tk = warp; tk < ntp; tk += kWarps) {
+            uint32_t *row = sc + tk * n4;
+            for (int j = lane; j < a.sink && j < n; j += 32) row[j] = 0xFFFFFFFFu;
+            __syncwarp();
+            select_warp_radix(row, n, a.topk, out + (long long)(t0 + tk) * a.topk, hist + warp * 256, lane);
+            __syncwarp();
+        }
+        __syncthreads();  // the score rows are reused by the next pass
+    }
+}
+
 }  // namespace
 
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
@@ -643,6 +762,45 @@ hga_status_t launch_route(const hga_params_t &p, const void *q, const float *sum
     else
         e = D == 128 ? launch_t<float, 128>(a, cl, split, grid, stream) : launch_t<float, 64>(a, cl, split, grid, stream);
     if (e == cudaSuccess) e = cudaGetLastError();
+    return record_cuda(e);
+}
+
+hga_status_t launch_route_causal(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
+                                 unsigned *status, cudaStream_t stream) {
+    const int n = p.n_hist_chunks, D = p.head_dim;
+    // one-token blocks: the block route is already per token
+    if (p.q_block == 1) return launch_route(p, q, summ, cap, idx, status, stream);
+    const CausalLayout L = causal_layout(D, p.q_block, n);
+    if (L.tp < 1 || L.total > kMaxSmem) {
+        record_error("hga_route_causal: shared-memory layout exceeds the per-CTA limit");
+        return HGA_ERR_UNSUPPORTED;
+    }
+    RouteArgs a{};
+    a.q = q;
+    a.summ = summ;
+    a.idx = idx;
+    a.status = status;
+    a.cap = cap;
+    a.n_q_heads = p.n_q_heads;
+    a.n_kv_heads = p.n_kv_heads;
+    a.seg_len = p.seg_len;
+    a.q_block = p.q_block;
+    a.n = n;
+    a.topk = p.topk;
+    a.sink = p.sink_chunks;
+    a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(D)));
+    const unsigned grid = static_cast<unsigned>(p.batch * p.n_kv_heads * (p.seg_len / p.q_block));
+    cudaError_t e;
+    auto go = [&](auto kern) {
+        cudaError_t err = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), L.total);
+        if (err != cudaSuccess) return err;
+        kern<<<grid, kThreads, L.total, stream>>>(a, L.tp, L);
+        return cudaGetLastError();
+    };
+    if (p.dtype == HGA_BF16)
+        e = D == 128 ? go(route_causal_kernel<__nv_bfloat16, 128>) : go(route_causal_kernel<__nv_bfloat16, 64>);
+    else
+        e = D == 128 ? go(route_causal_kernel<float, 128>) : go(route_causal_kernel<float, 64>);
     return record_cuda(e);
 }
 

@@ -133,6 +133,19 @@ hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch
 hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
                        int32_t *idx, cudaStream_t stream);
 
+/* Strictly causal routing (technical summary, limits section: sharing one
+ * route among the tokens of a block is a weak causal side channel; a strictly
+ * causal variant is proposed as future work).  Every token i of block m
+ * routes by qbar_i = fp32 mean over the G heads of group g and the queries
+ * m*q_block .. i of its block, with the score, selection, ties and sink rule
+ * of hga_route; the last token of a block gets the block's route.
+ *   idx: device int32 [B][Hkv][S][k], one route per token.  Other arguments
+ *   as hga_route.  q_block = 1 gives the plain per-token route.
+ * HGA_ERR_UNSUPPORTED when one token's score row set does not fit the CTA's
+ * shared memory (n_hist_chunks above about 5,000 for D = 128). */
+hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
+                              int32_t *idx, cudaStream_t stream);
+
 /* Exact-token attention forward (technical summary section 2.1; author
  * abstract: a bounded set of exact historical tokens per query block).  For
  * query (b, h, i) of a processed block m = i / q_block, g = h / G:

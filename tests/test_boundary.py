@@ -68,6 +68,20 @@ def test_bad_params_rejected_on_host(L, kw):
     assert rc == -1
     rc = L.hga_route(ctypes.byref(p), fake, fake, 64, fake, None)
     assert rc == -1
+    rc = L.hga_route_causal(ctypes.byref(p), fake, fake, 64, fake, None)
+    assert rc == -1
+
+
+def test_causal_route_checked_on_host(L):
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    p = _params().c()
+    assert L.hga_route_causal(ctypes.byref(p), fake, fake, 7, fake, None) == -1   # capacity < Nc
+    assert L.hga_route_causal(ctypes.byref(p), odd, fake, 8, fake, None) == -1    # misaligned q
+    assert L.hga_route_causal(ctypes.byref(p), fake, None, 8, fake, None) == -1   # no summaries
+    assert L.hga_route_causal(ctypes.byref(p), fake, fake, 8, None, None) == -1   # no route table
+    big = _params(n_hist_chunks=20000, hist_head_stride=20000 * 64).c()
+    assert L.hga_route_causal(ctypes.byref(big), fake, fake, 20000, fake, None) == -2
 
 
 def test_unsupported_shapes(L):
