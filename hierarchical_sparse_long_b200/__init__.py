@@ -6,7 +6,7 @@ segment-by-segment processing.
 """
 from .binding import (  # noqa: F401
     HGA_BF16, HGA_FP32, HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT, EXPORTED, HGAError, Params, lib,
-    hga_build_summaries, hga_route, hga_route_causal, hga_attn_fwd, hga_attn_bwd_workspace_size, hga_attn_bwd,
+    hga_build_summaries, hga_route, hga_route_causal, hga_route_groups, hga_attn_fwd, hga_attn_bwd_workspace_size, hga_attn_bwd,
     hga_attn_bwd_noalloc, hga_attn_decode_workspace_size, hga_attn_decode,
     hga_fetch_tiered, hga_get_device_status, hga_selftest_wait_timeout,
 )

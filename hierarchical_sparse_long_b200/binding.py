@@ -21,7 +21,7 @@ HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT = 1, 2
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3: "HGA_ERR_CUDA",
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
-EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
+EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
             "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_fetch_tiered",
             "hga_get_device_status", "hga_selftest_wait_timeout", "hga_status_string", "hga_last_error")
 
@@ -84,6 +84,7 @@ def lib() -> ctypes.CDLL:
         L.hga_build_summaries.argtypes = [vp, ll, i, i, i, i, i, i, i, vp, i, vp]
         L.hga_route.argtypes = [pp, vp, vp, i, vp, vp]
         L.hga_route_causal.argtypes = [pp, vp, vp, i, vp, vp]
+        L.hga_route_groups.argtypes = [pp, vp, vp, i, vp, i, i, vp, vp]
         L.hga_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_attn_bwd_workspace_size.argtypes = [pp]
         L.hga_attn_bwd_workspace_size.restype = sz
@@ -99,7 +100,7 @@ def lib() -> ctypes.CDLL:
         L.hga_status_string.argtypes = [i]
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
-        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
+        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
                   "hga_attn_decode", "hga_fetch_tiered", "hga_get_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
@@ -154,6 +155,14 @@ def hga_route_causal(p: Params, q, summ, summ_cap_chunks: int, idx, stream=None)
     cp = p.c()
     _check(lib().hga_route_causal(ctypes.byref(cp), _ptr(q), _ptr(summ), summ_cap_chunks, _ptr(idx),
                                   _stream(stream)), "hga_route_causal")
+
+
+def hga_route_groups(p: Params, q, gsumm, gsumm_cap_groups: int, idx, group: int, topg: int, gidx, stream=None):
+    """Second routing stage: the topg best groups of `group` tokens inside each block's
+    chosen chunks into gidx [B][Hkv][S/q_block][topg] (int32)."""
+    cp = p.c()
+    _check(lib().hga_route_groups(ctypes.byref(cp), _ptr(q), _ptr(gsumm), gsumm_cap_groups, _ptr(idx), group,
+                                  topg, _ptr(gidx), _stream(stream)), "hga_route_groups")
 
 
 def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stream=None):

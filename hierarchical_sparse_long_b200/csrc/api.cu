@@ -118,6 +118,19 @@ hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, 
     return hga::launch_route(*p, q, summ, summ_cap_chunks, idx, status, stream);
 }
 
+hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float *gsumm, int gsumm_cap_groups,
+                              const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (group != 8 && group != 16 && group != 32) return HGA_ERR_INVALID_ARG;
+    const int gpc = p->chunk / group;
+    if (topg < 1 || topg > p->topk * gpc) return HGA_ERR_INVALID_ARG;
+    if ((long long)gsumm_cap_groups < (long long)p->n_hist_chunks * gpc) return HGA_ERR_INVALID_ARG;
+    if (!q || !idx || !gidx || !aligned16(q)) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!gsumm || !aligned16(gsumm))) return HGA_ERR_INVALID_ARG;
+    return hga::launch_route_groups(*p, q, gsumm, gsumm_cap_groups, idx, group, topg, gidx, stream);
+}
+
 hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
                               int32_t *idx, cudaStream_t stream) {
     hga_status_t st = check_params(p);

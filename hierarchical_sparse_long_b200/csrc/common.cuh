@@ -55,6 +55,9 @@ hga_status_t launch_summaries(const void *k, long long head_stride, int bh, int 
                               cudaStream_t stream);
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
                           unsigned *status, cudaStream_t stream);
+// Group-stage routes (groups of `group` tokens in the chosen chunks): gidx [B][Hkv][S/q_block][topg].
+hga_status_t launch_route_groups(const hga_params_t &p, const void *q, const float *gsumm, long long cap,
+                                 const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream);
 // Strictly causal routes, one per token: idx [B][Hkv][S][topk].
 hga_status_t launch_route_causal(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
                           unsigned *status, cudaStream_t stream);

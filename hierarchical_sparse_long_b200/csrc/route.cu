@@ -677,6 +677,112 @@ __global__ void __launch_bounds__(kThreads, 1) route_causal_kernel(const RouteAr
     }
 }
 
+// ---------------------------------------------------------------------------
+// Group-level second stage (technical summary section 2.1, group selection):
+// the groups of `gs` tokens inside a block's chosen chunks are scored against
+// the same block summary with their group summaries (mean of the group's
+// keys) and the topg best are kept, by (score descending, group index
+// ascending), listed ascending and -1 padded.  One CTA per (b, g, m).
+constexpr int kMaxCand = 64 * 8;  // k <= 64 chosen chunks x up to 8 groups each
+
+struct GroupArgs {
+    const void *q;
+    const float *gsumm;
+    const int32_t *idx;
+    int32_t *gidx;
+    long long cap;  // group-summary rows per (b, g)
+    int n_q_heads, n_kv_heads, seg_len, q_block, n, topk, gpc, topg;
+    float inv_sqrt_d;
+};
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kThreads, 1) route_groups_kernel(const GroupArgs a) {
+    constexpr int NRS = kThreads / D;  // row slots of the block-summary sum
+    __shared__ float part[NRS][D];
+    __shared__ __align__(16) float qbar[D];
+    __shared__ uint32_t row[kMaxCand];
+    __shared__ int chunks[64], sel[kMaxCand], n_chunks;
+    __shared__ uint32_t s_tmax[kThreads];
+    __shared__ uint64_t s_key[kCandCap];
+    __shared__ int s_cj[kCandCap], s_hist[256], s_misc[16];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int nqb = a.seg_len / a.q_block;
+    const int m = (int)blockIdx.x % nqb, bg = (int)blockIdx.x / nqb;
+    const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+    const int G = a.n_q_heads / a.n_kv_heads;
+    int32_t *out = a.gidx + ((long long)bg * nqb + m) * a.topg;
+
+    // block summary: thread (rs, d) sums rows rs, rs + NRS, ... of the G x q_block
+    // rows (head-major) in order, then the NRS partials are added in order
+    {
+        const int d = tid % D, rs = tid / D;
+        const T *qb = static_cast<const T *>(a.q) +
+                      (((long long)b * a.n_q_heads + (long long)g * G) * a.seg_len + (long long)m * a.q_block) * D + d;
+        float acc = 0.f;
+        for (int r = rs; r < G * a.q_block; r += NRS) {
+            const int hh = r / a.q_block, i = r - hh * a.q_block;
+            acc += to_f32(qb[((long long)hh * a.seg_len + i) * D]);
+        }
+        part[rs][d] = acc;
+    }
+    if (tid == 0) {  // the block's chosen chunks, ascending (insertion sort of <= 64 ids)
+        const int32_t *selc = a.idx + ((long long)bg * nqb + m) * a.topk;
+        int nv = 0;
+        for (int t = 0; t < a.topk; ++t) {
+            const int j = selc[t];
+            if (j < 0 || j >= a.n) continue;
+            int p = nv++;
+            while (p > 0 && chunks[p - 1] > j) {
+                chunks[p] = chunks[p - 1];
+                --p;
+            }
+            chunks[p] = j;
+        }
+        n_chunks = nv;
+    }
+    __syncthreads();
+    if (tid < D) {
+        float s = 0.f;
+        for (int r = 0; r < NRS; ++r) s += part[r][tid];
+        qbar[tid] = s / static_cast<float>(G * a.q_block);
+    }
+    __syncthreads();
+
+    // scores of the candidate groups: one warp per candidate, D / 32 values per lane
+    const int ncand = n_chunks * a.gpc;
+    const float *gbase = a.gsumm + (long long)bg * a.cap * D;
+    constexpr int VPL = D / 32;
+    float qv[VPL];
+#pragma unroll
+    for (int e = 0; e < VPL; ++e) qv[e] = qbar[lane * VPL + e];
+    for (int c = warp; c < ncand; c += kWarps) {
+        const int gid = chunks[c / a.gpc] * a.gpc + c % a.gpc;
+        const float *gr = gbase + (long long)gid * D + lane * VPL;
+        float acc = 0.f;
+#pragma unroll
+        for (int e = 0; e < VPL; ++e) acc = fmaf(qv[e], gr[e], acc);
+#pragma unroll
+        for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(kFull, acc, o);
+        if (lane == 0) row[c] = ordered_bits(acc * a.inv_sqrt_d);
+    }
+    __syncthreads();
+
+    if (a.topg >= ncand) {  // every candidate is kept
+        for (int t = tid; t < a.topg; t += kThreads)
+            out[t] = t < ncand ? chunks[t / a.gpc] * a.gpc + t % a.gpc : -1;
+        return;
+    }
+    SelScratch ss;
+    ss.tmax = s_tmax;
+    ss.key = s_key;
+    ss.cj = s_cj;
+    ss.hist = s_hist;
+    ss.misc = s_misc;
+    select_cta(row, ncand, a.topg, sel, ss, tid);  // positions, ascending
+    __syncthreads();
+    for (int t = tid; t < a.topg; t += kThreads) out[t] = chunks[sel[t] / a.gpc] * a.gpc + sel[t] % a.gpc;
+}
+
 }  // namespace
 
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
@@ -802,6 +908,34 @@ hga_status_t launch_route_causal(const hga_params_t &p, const void *q, const flo
     else
         e = D == 128 ? go(route_causal_kernel<float, 128>) : go(route_causal_kernel<float, 64>);
     return record_cuda(e);
+}
+
+hga_status_t launch_route_groups(const hga_params_t &p, const void *q, const float *gsumm, long long cap,
+                                 const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream) {
+    GroupArgs a{};
+    a.q = q;
+    a.gsumm = gsumm;
+    a.idx = idx;
+    a.gidx = gidx;
+    a.cap = cap;
+    a.n_q_heads = p.n_q_heads;
+    a.n_kv_heads = p.n_kv_heads;
+    a.seg_len = p.seg_len;
+    a.q_block = p.q_block;
+    a.n = p.n_hist_chunks;
+    a.topk = p.topk;
+    a.gpc = p.chunk / group;
+    a.topg = topg;
+    a.inv_sqrt_d = static_cast<float>(1.0 / __builtin_sqrt(static_cast<double>(p.head_dim)));
+    const unsigned grid = static_cast<unsigned>(p.batch * p.n_kv_heads * (p.seg_len / p.q_block));
+    if (p.dtype == HGA_BF16) {
+        if (p.head_dim == 128) route_groups_kernel<__nv_bfloat16, 128><<<grid, kThreads, 0, stream>>>(a);
+        else route_groups_kernel<__nv_bfloat16, 64><<<grid, kThreads, 0, stream>>>(a);
+    } else {
+        if (p.head_dim == 128) route_groups_kernel<float, 128><<<grid, kThreads, 0, stream>>>(a);
+        else route_groups_kernel<float, 64><<<grid, kThreads, 0, stream>>>(a);
+    }
+    return record_cuda(cudaGetLastError());
 }
 
 }  // namespace hga

@@ -133,6 +133,23 @@ hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch
 hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
                        int32_t *idx, cudaStream_t stream);
 
+/* Group-level second routing stage (technical summary section 2.1, group
+ * selection: the chosen chunks are split into smaller groups, e.g. 8 tokens,
+ * and the router keeps the best groups inside the chosen chunks).  For every
+ * (b, g, query block m) with its chunk route idx (from hga_route):
+ *   candidates = the groups of `group` tokens of every valid chunk in
+ *                idx[b][g][m][*] (chunk j holds groups j*c/group .. +c/group-1);
+ *   s_u        = fp32 dot(qbar, gsumm[b][g][u]) / sqrt(D), qbar as in hga_route;
+ *   gidx[((b*Hkv + g)*nqb + m)*topg + a], a < topg: the topg candidates with the
+ *                largest s_u (ties: lower u), ascending, then -1 padding.
+ *   gsumm: device fp32 group summaries (the mean of each group's keys, e.g.
+ *     hga_build_summaries with chunk = group), gsumm_cap_groups rows per
+ *     (b, g) slice (>= Nc * c / group).
+ *   group: 8, 16 or 32 tokens.  topg: 1 .. topk * c / group.
+ *   gidx: device int32 [B][Hkv][S/q_block][topg]. */
+hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float *gsumm, int gsumm_cap_groups,
+                              const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream);
+
 /* Strictly causal routing (technical summary, limits section: sharing one
  * route among the tokens of a block is a weak causal side channel; a strictly
  * causal variant is proposed as future work).  Every token i of block m

@@ -72,6 +72,17 @@ def test_bad_params_rejected_on_host(L, kw):
     assert rc == -1
 
 
+def test_group_route_checked_on_host(L):
+    fake = ctypes.c_void_p(0x1000)
+    odd = ctypes.c_void_p(0x1008)
+    p = _params().c()  # Nc 8, k 4
+    for group, topg, cap in ((7, 4, 64), (64, 4, 64), (8, 0, 64), (8, 33, 64), (8, 4, 63), (16, 17, 32)):
+        assert L.hga_route_groups(ctypes.byref(p), fake, fake, cap, fake, group, topg, fake, None) == -1, (group, topg)
+    assert L.hga_route_groups(ctypes.byref(p), odd, fake, 64, fake, 8, 4, fake, None) == -1
+    assert L.hga_route_groups(ctypes.byref(p), fake, None, 64, fake, 8, 4, fake, None) == -1
+    assert L.hga_route_groups(ctypes.byref(p), fake, fake, 64, fake, 8, 4, None, None) == -1
+
+
 def test_causal_route_checked_on_host(L):
     fake = ctypes.c_void_p(0x1000)
     odd = ctypes.c_void_p(0x1008)
