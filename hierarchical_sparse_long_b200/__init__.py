@@ -1,8 +1,8 @@
 """B200-native Hierarchical Global Attention (HGA) layer.
 
 The compute lives in ``libhga.so`` (hand-written sm_100a CUDA, C ABI in
-include/hga.h); this package is its ctypes binding plus a small driver for
-segment-by-segment processing.
+include/hga.h); this package is its ctypes binding and the in-tree build
+script (``build.py``).
 """
 from .binding import (  # noqa: F401
     HGA_BF16, HGA_FP32, HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT, EXPORTED, HGAError, Params, lib,
