@@ -203,7 +203,7 @@ __device__ void select_warp_radix(const uint32_t *row, int n, int k, int32_t *ou
 }
 
 struct SelScratch {
-    uint32_t *tmax;  // [kThreads] per-thread maxima
+    uint32_t *tmax;  // [kThreads] per-thread maxima; 16-byte aligned (read as uint4)
     uint64_t *key;   // [kCandCap] candidate keys
     int *cj;         // [kCandCap] chosen candidates' chunk index, else INT_MAX
     int *hist;       // [256] (whole-row fallback)
@@ -702,7 +702,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_groups_kernel(const GroupAr
     __shared__ __align__(16) float qbar[D];
     __shared__ uint32_t row[kMaxCand];
     __shared__ int chunks[64], sel[kMaxCand], n_chunks;
-    __shared__ uint32_t s_tmax[kThreads];
+    __shared__ __align__(16) uint32_t s_tmax[kThreads];  // select_cta reads it as 16-byte vectors
     __shared__ uint64_t s_key[kCandCap];
     __shared__ int s_cj[kCandCap], s_hist[256], s_misc[16];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
