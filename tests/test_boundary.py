@@ -143,3 +143,18 @@ def test_decode_shape_checked_on_host(L):
     fake = ctypes.c_void_p(0x1000)
     # one-token segments are for hga_attn_decode only
     assert L.hga_attn_fwd(ctypes.byref(ok), fake, fake, fake, fake, fake, fake, fake, fake, None) == -2
+
+
+def test_decode_workspace_covers_every_partial(L):
+    """The decode workspace holds one (m, l, o[D]) fp32 partial per consumer warp (4),
+    split, (b, g) and query head of the group; the split count fills about two CTAs per
+    SM (148 here, where no device can be queried) without exceeding the unit count."""
+    for B, Hq, Hkv, D, k, nc, n_local in ((16, 32, 8, 128, 32, 2047, 64), (1, 8, 2, 64, 6, 5, 130),
+                                          (2, 4, 4, 128, 5, 20, 1)):
+        p = _params(batch=B, n_q_heads=Hq, n_kv_heads=Hkv, head_dim=D, topk=k, seg_len=1, q_block=1,
+                    n_hist_chunks=nc).c()
+        units = min(k, nc) + -(-n_local // 64)
+        n_split = max(1, min(units, 2 * 148 // (B * Hkv)))
+        floats = B * Hkv * n_split * 4 * (Hq // Hkv) * (D + 2)
+        want = (floats * 4 + 255) // 256 * 256
+        assert L.hga_attn_decode_workspace_size(ctypes.byref(p), n_local) == want, (B, Hq, Hkv, D)
