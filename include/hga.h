@@ -21,8 +21,16 @@
  *                         chunk index ascending), listed in ascending chunk
  *                         order and padded with -1;
  *   local window        = every active-segment token at or before the query;
- *   no attention sink and no 8-token group stage.
- * Query i of the active segment therefore attends exactly
+ *   attention sink      = with sink_chunks = s, history chunks 0 .. s-1 are
+ *                         always chosen, inside the k slots (hga_route);
+ *   group stage         = hga_route_groups: the best groups of 8, 16 or 32
+ *                         tokens inside the chosen chunks (a second routing
+ *                         stage; the attention entry points read chunk routes);
+ *   strictly causal     = hga_route_causal: token i routes by its block's
+ *                         queries up to i;
+ *   decode              = hga_attn_decode: one new token per sequence, routed
+ *                         as a one-token block.
+ * With chunk routes, query i of the active segment attends exactly
  * min(k, Nc) * chunk + i + 1 tokens.
  *
  * Conventions for every entry point:
