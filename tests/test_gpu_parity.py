@@ -32,6 +32,14 @@ EDGE = [
                n_q_heads=8, n_kv_heads=2, seed=14, backward=True),
     gen.custom("one_block", topk=1, seg_len=64, seq_len=192, seg_starts=(128,), dtype="bf16", head_dim=128,
                n_q_heads=4, n_kv_heads=1, seed=15, backward=True),
+    # tcgen05 head packing for other GQA groups: G = 1 (rows repeated, half written back),
+    # G = 8 (two CTAs of 4 heads per KV group), G = 6 (three CTAs of 2 heads)
+    gen.custom("g1_bf16", topk=3, seg_len=128, seq_len=640, seg_starts=(512,), dtype="bf16", head_dim=128,
+               n_q_heads=2, n_kv_heads=2, seed=16, backward=True),
+    gen.custom("g8_bf16", topk=4, seg_len=128, seq_len=640, seg_starts=(512,), dtype="bf16", head_dim=128,
+               n_q_heads=8, n_kv_heads=1, seed=17, backward=True),
+    gen.custom("g6_bf16", topk=2, seg_len=192, seq_len=576, seg_starts=(384,), dtype="bf16", head_dim=128,
+               n_q_heads=12, n_kv_heads=2, seed=18, backward=True),
 ]
 
 
@@ -316,8 +324,10 @@ def test_bwd_edge_cases(w):
 
 
 def test_bwd_full_size_sampled():
-    # the 16K training layer's last segment (T = 14,336): sampled dq rows and
-    # dk/dv rows of the last 64 active keys (every query that sees them is visited)
+    # the 16K training layer's last segment (T = 14,336): sampled dq rows of early,
+    # middle and late query blocks, and dk/dv rows of the first 128 active keys of KV
+    # head 0 (the dK/dV block every later query tile of the 4 heads reaches: 32 tiles x
+    # 4 heads = 128 accumulation steps) and of its last 64 keys
     w = W["qwen3_16k_train"]
     seg = 7
     arrs = hc.segment_arrays(w, seg)
@@ -328,7 +338,10 @@ def test_bwd_full_size_sampled():
     r = np.random.default_rng(3)
     for _ in range(64):
         q_need[0, r.integers(0, w.n_q_heads), r.integers(S - 256, S)] = 1
+    for m in (0, 1, 15):  # early blocks: every row of two heads of different groups
+        q_need[0, [1, 30], m * 64:(m + 1) * 64] = 1
     key_need = np.zeros((1, w.n_kv_heads, S), dtype=np.uint8)
+    key_need[0, 0, :128] = 1
     key_need[0, 0, S - 64:] = 1
     key_need[0, 5, [S - 1, S - 30]] = 1
     dq_o, dk_o, dv_o = oracle.attn_bwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
