@@ -5,15 +5,25 @@ Workloads (synthetic Qwen3-8B-shaped layers: 32 query heads, 8 KV heads,
 head_dim 128, bf16, chunk 64, query block 64; seeded inputs drawn on the GPU
 with the recipe of inputs/gen.py):
 
-* ``qwen3_16k_fwd`` (default): 14,336 detached history tokens + a 2,048-token
-  active segment, top-16 chunks.  One step = route the 32 query blocks,
-  exact-token attention forward over the routed chunks + the causal segment,
-  and the detach-time summary append of the segment's 32 chunks.
+* ``qwen3_16k_fwd`` (default headline): 14,336 detached history tokens + a
+  2,048-token active segment, top-16 chunks.  One step = route the 32 query
+  blocks, exact-token attention forward over the routed chunks + the causal
+  segment, and the detach-time summary append of the segment's 32 chunks.
 * ``qwen3_16k_train``: the same layer trained segment-wise: one step = 8
   consecutive 2,048-token segments, each route + forward + backward (dQ, and
   dK/dV of the segment) + summary append.
 * ``qwen3_128k_eval``: one step = a 131,072-token evaluation as 32 segments of
   4,096 tokens, top-32 chunks, each route + forward + summary append.
+* ``qwen3_128k_tiered``: the 128K evaluation with detached history K/V in
+  pinned host memory: each segment routes, then ``hga_attn_fwd_tiered`` fetches
+  the routed chunks wave by wave (32 query blocks per wave) into a device
+  staging cache on a side stream, overlapped with the attention of the
+  previous wave; the cache holds one segment's routing budget of chunk tiles
+  and keeps them from segment to segment (it is emptied when the 131,072-token
+  evaluation starts), so a routed chunk crosses the host link only when the
+  cache does not hold it; the segment's K/V are then offloaded to the host on
+  the copy stream (ordered before the next segment's fetches) and its
+  summaries appended.
 * ``qwen3_128k_decode``: generation at 128K context: 16 sequences each add one
   token after 131,008 detached history tokens; a step routes the 16 tokens
   (one-token query blocks) and runs the split-K decode attention over their 32
@@ -22,11 +32,11 @@ with the recipe of inputs/gen.py):
   decode grid of the 128K case on 2.1 GB of K/V; used for counter captures).
 * ``qwen3_16k_fwd_sink``: ``qwen3_16k_fwd`` with a one-chunk attention-sink
   window (history chunk 0 always routed, the other 15 slots by score).
-* ``qwen3_128k_tiered``: the 128K evaluation with detached history K/V in
-  pinned host memory: each segment routes, fetches only the routed chunks
-  (waves of 8 query blocks, double-buffered staging on a side stream
-  overlapped with attention), attends, copies the segment's K/V to the host
-  and appends its summaries.
+
+The default run prints one JSON line for the headline workload and measures
+``qwen3_16k_train``, ``qwen3_128k_eval`` and ``qwen3_128k_tiered`` too, each
+under ``workloads`` in the same line with its own roofline, kernels, e2e and
+CPU baseline (``--also none`` skips them).
 
 Metric: query tokens/s (active query tokens processed per second, all heads),
 device-timed with CUDA events, L2 flushed (256 MiB write) before every step.
@@ -53,16 +63,19 @@ sys.path.insert(0, ROOT)
 METRIC = "HGA attn query tok/s at 16K & 128K ctx; % of HBM / tensor-pipe roofline"
 UNIT = "query tok/s"
 CSRC = "hierarchical_sparse_long_b200/csrc/"
+# the translation unit of each kernel (and the PTX wrappers it inlines): a stored
+# ncu traffic figure stays valid while these sources are unchanged
 KERNEL_SOURCES = {
-    "attn_fwd": [CSRC + "attn_fwd_tc.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
-    "attn_bwd": [CSRC + "attn_bwd_tc.cu", CSRC + "attn_simt.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
-    "route": [CSRC + "route.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
-    "summaries": [CSRC + "summaries.cu", CSRC + "common.cuh"],
-    "fetch": [CSRC + "tiered.cu", CSRC + "common.cuh"],
-    "attn_decode": [CSRC + "decode.cu", CSRC + "tc_ptx.cuh", CSRC + "common.cuh"],
+    "attn_fwd": [CSRC + "attn_fwd_tc.cu", CSRC + "tc_ptx.cuh"],
+    "attn_bwd": [CSRC + "attn_bwd_tc.cu", CSRC + "tc_ptx.cuh"],
+    "route": [CSRC + "route.cu", CSRC + "tc_ptx.cuh"],
+    "summaries": [CSRC + "summaries.cu"],
+    "fetch": [CSRC + "tiered.cu"],
+    "attn_decode": [CSRC + "decode.cu", CSRC + "tc_ptx.cuh"],
 }
 WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_16k_fwd_sink",
              "qwen3_128k_decode", "qwen3_32k_decode")
+ALSO_DEFAULT = ("qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered")
 
 
 def parse():
@@ -72,11 +85,18 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="hga", choices=["hga", "reference"])
     ap.add_argument("--workload", default="qwen3_16k_fwd", choices=WORKLOADS)
+    ap.add_argument("--also", default="auto",
+                    help="comma-separated workloads measured after the headline one and reported under "
+                         "`workloads` ('none' for none; 'auto': the 16K training, 128K evaluation and 128K "
+                         "tiered workloads when the headline is the default)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--serial-append", action="store_true",
                     help="run each segment's summary append after its attention on the main stream "
                          "(default: on a side stream, overlapped with the route)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
+    ap.add_argument("--tier-wave", type=int, default=32, help="query blocks per fetch wave of the tiered workload")
+    ap.add_argument("--cpu-procs", type=int, default=0,
+                    help="oracle processes for the 128K samples (0: up to 8, bounded by the host's cores)")
     return ap.parse_args()
 
 
@@ -121,6 +141,23 @@ def kernel_traffic(kernel, workload):
     if not d or d.get("source_hash") != file_hash(KERNEL_SOURCES.get(kernel, [])):
         return None
     return d.get("bytes_per_launch")
+
+
+def cpu_info():
+    """Host CPU model, logical CPUs and the CPUs this process may run on."""
+    model = "unknown"
+    try:
+        for ln in open("/proc/cpuinfo"):
+            if ln.startswith("model name"):
+                model = ln.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:
+        usable = os.cpu_count() or 1
+    return {"cpu_model": model, "nproc": os.cpu_count() or 1, "usable_cpus": usable}
 
 
 class ClockSampler:
@@ -190,13 +227,16 @@ def summaries_bytes(w):
         w.batch * w.n_kv_heads * (w.seg_len // w.chunk) * w.head_dim * 4
 
 
+TILE_PAIR_BYTES = lambda w: 2 * w.chunk * w.head_dim * 2  # K and V of one chunk, bf16
+
+
 # ------------------------------------------------------------------ workload state
 class Layer:
     """Device state of one HGA layer: K/V of the whole sequence in one buffer per
     head (history and active segment are views), resident chunk summaries, and
     the queries (and upstream gradients) of every processed segment."""
 
-    WAVE = 8  # query blocks per tiered fetch wave
+    wave = 32  # query blocks per tiered fetch wave
 
     def __init__(self, w):
         import torch
@@ -283,7 +323,7 @@ class Layer:
             rec("attn_bwd")
             hga.hga_attn_bwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse,
                              self.do[T] if do is None else do, self.dq, self.dk, self.dv, self.ws)
-            launches += 3
+            launches += 2
         if self.side_append:
             rec(None)
             main.wait_stream(self.side)
@@ -295,82 +335,102 @@ class Layer:
         return launches + 1
 
     def _init_tiered(self):
-        torch, w = self.torch, self.w
+        """Pinned host copy of the whole sequence's K/V (the detached history is
+        read from there only) and the device staging cache: one segment's routing
+        budget of chunk tiles (as many tiles as the segment's blocks can route to)."""
+        torch, hga, w = self.torch, self.hga, self.w
         self.host_k = self.k.cpu().pin_memory()
         self.host_v = self.v.cpu().pin_memory()
-        self.slots = self.WAVE * w.batch * w.n_kv_heads * w.topk
-        self.stage = [(torch.empty(self.slots, w.chunk, w.head_dim, device="cuda", dtype=torch.bfloat16),
-                       torch.empty(self.slots, w.chunk, w.head_dim, device="cuda", dtype=torch.bfloat16))
-                      for _ in range(2)]
-        n_map = w.batch * w.n_kv_heads * self.nct + self.slots + 1
-        self.slot_map = [torch.empty(n_map, device="cuda", dtype=torch.int32) for _ in range(2)]
-        self.idx_r = [torch.empty_like(self.idx) for _ in range(2)]
-        self.n_fetched = torch.zeros(64, device="cuda", dtype=torch.int32)
+        nqb = w.seg_len // w.q_block
+        self.slots = w.batch * w.n_kv_heads * min(w.seg_starts[-1] // w.chunk, nqb * w.topk)
+        self.stage_k = torch.empty(self.slots, w.chunk, w.head_dim, device="cuda", dtype=torch.bfloat16)
+        self.stage_v = torch.empty_like(self.stage_k)
+        p0 = self.params(w.seg_starts[-1])
+        self.scratch = torch.empty(hga.hga_tier_scratch_size(p0, self.slots) // 4, device="cuda",
+                                   dtype=torch.int32)
+        self.idx_r = torch.empty_like(self.idx)
+        self.n_waves = -(-nqb // self.wave)
+        self.n_fetched = torch.zeros(len(w.seg_starts), self.n_waves, device="cuda", dtype=torch.int32)
         self.copy_stream = torch.cuda.Stream()
-        self.fetched_ev = [torch.cuda.Event() for _ in range(2)]
-        self.consumed_ev = [torch.cuda.Event() for _ in range(2)]
+        self.tier_events = [torch.cuda.Event() for _ in range(5)]
 
-    def segment_tiered(self, T, ev=None, q=None):
+    def segment_tiered(self, T, ev=None, q=None, si=0):
         """The same segment with the history only in pinned host memory: route,
-        fetch the routed chunks wave by wave on the copy stream (double-buffered
-        staging) while attention runs on the previous wave, then detach."""
+        then attention over the staging cache with the fetch waves overlapped
+        (hga_attn_fwd_tiered; the cache is emptied at the first segment only),
+        then detach: the segment's K/V go to the host on the copy stream, one
+        2-D copy for K and one for V, before any later fetch."""
         torch, hga, w = self.torch, self.hga, self.w
-        p = self.params(T, hist_head_stride=self.L)
+        p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
         rec = ev.record if ev is not None else (lambda name: None)
-        compute = torch.cuda.current_stream()
         rec("route")
         hga.hga_route(p, q, self.summ, self.nct, self.idx)
-        nqb = w.seg_len // w.q_block
-        waves = [(b0, min(b0 + self.WAVE, nqb)) for b0 in range(0, nqb, self.WAVE)]
-        launches = 1
         rec("attn_fwd")
-        if T == 0:
-            hga.hga_attn_fwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse)
-            launches += 1
-        else:
-            routed = torch.cuda.Event()
-            routed.record(compute)
-            self.copy_stream.wait_event(routed)
-
-            def fetch(wi):
-                b0, b1 = waves[wi]
-                buf = wi % 2
-                if wi >= 2:
-                    self.copy_stream.wait_event(self.consumed_ev[buf])
-                sk, sv = self.stage[buf]
-                hga.hga_fetch_tiered(p, self.host_k, self.host_v, self.idx, b0, b1, sk, sv, self.slots,
-                                     self.slot_map[buf], self.idx_r[buf], self.n_fetched[wi:wi + 1],
-                                     copy_stream=self.copy_stream)
-                self.fetched_ev[buf].record(self.copy_stream)
-
-            fetch(0)
-            for wi, (b0, b1) in enumerate(waves):
-                buf = wi % 2
-                if wi + 1 < len(waves):
-                    fetch(wi + 1)
-                compute.wait_event(self.fetched_ev[buf])
-                sk, sv = self.stage[buf]
-                pa = self.params(T, hist_head_stride=0, n_hist_chunks=self.slots, qblock_begin=b0, qblock_end=b1)
-                hga.hga_attn_fwd(pa, q, sk, sv, ks, vs, self.idx_r[buf], self.out, self.lse)
-                self.consumed_ev[buf].record(compute)
-                launches += 5
+        first = T == w.seg_starts[0]
+        hga.hga_attn_fwd_tiered(p, q, self.host_k, self.host_v, ks, vs, self.idx, self.out, self.lse, self.stage_k,
+                                self.stage_v, self.slots, self.scratch, self.idx_r, self.wave, self.tier_events,
+                                reset_cache=first, n_fetched=self.n_fetched[si], copy_stream=self.copy_stream)
+        launches = 1 + int(first) + (1 if T == 0 else 4 * self.n_waves)
         # detach: the segment's K/V join the host history, its chunks become routable
         rec("summaries")
-        self.host_k[:, :, T:T + w.seg_len].copy_(ks[:, :, :w.seg_len], non_blocking=True)
-        self.host_v[:, :, T:T + w.seg_len].copy_(vs[:, :, :w.seg_len], non_blocking=True)
+        self.copy_stream.wait_stream(torch.cuda.current_stream())
+        hga.hga_tier_offload(p, ks, vs, self.host_k, self.host_v, T, stream=self.copy_stream)
         hga.hga_build_summaries(self.k, self.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
                                 w.seg_len // w.chunk, self.summ, self.nct)
         rec(None)
         return launches + 1
 
+    def fetch_only_step(self):
+        """Route + every fetch wave of every segment on the copy stream, no attention
+        and no offload (the host-link side of the tiered step alone, the cache emptied
+        at the first segment as in the step); returns device ms."""
+        torch, hga, w = self.torch, self.hga, self.w
+        compute = torch.cuda.current_stream()
+        nqb = w.seg_len // w.q_block
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(compute)
+        for si, T in enumerate(w.seg_starts):
+            p = self.params(T)
+            hga.hga_route(p, self.q[T], self.summ, self.nct, self.idx)
+            if T == 0:
+                continue
+            self.copy_stream.wait_stream(compute)
+            if T == w.seg_starts[0] or (si == 1 and w.seg_starts[0] == 0):  # the step's first fetch
+                hga.hga_tier_reset(p, self.slots, self.scratch, stream=self.copy_stream)
+            for wi, b0 in enumerate(range(0, nqb, self.wave)):
+                hga.hga_fetch_tiered(p, self.host_k, self.host_v, self.idx, b0, min(b0 + self.wave, nqb),
+                                     self.stage_k, self.stage_v, self.slots, self.scratch, self.idx_r,
+                                     self.n_fetched[si, wi:wi + 1], copy_stream=self.copy_stream)
+            compute.wait_stream(self.copy_stream)
+        e.record(compute)
+        e.synchronize()
+        return s.elapsed_time(e)
+
+    def distinct_tiles(self):
+        """Distinct (b, g, chunk) tiles each segment routes to, summed over the
+        segments (what a cache emptied at every segment would fetch), and over the
+        whole step (what an unbounded cache would fetch).  Runs the routes again on
+        the same summaries; not timed."""
+        torch, hga, w = self.torch, self.hga, self.w
+        total, seen = 0, []
+        for T in w.seg_starts:
+            if T == 0:
+                continue
+            hga.hga_route(self.params(T), self.q[T], self.summ, self.nct, self.idx)
+            bg = torch.arange(w.batch * w.n_kv_heads, device="cuda").view(w.batch, w.n_kv_heads, 1, 1)
+            keys = torch.unique((bg * self.nct + self.idx.long())[self.idx >= 0])
+            total += int(keys.numel())
+            seen.append(keys)
+        return total, int(torch.unique(torch.cat(seen)).numel()) if seen else 0
+
     def step(self, ev=None):
         # the summaries of chunks >= T are never read by the route of a segment
         # starting at T, so each step simply re-appends every segment's chunks
         n = 0
-        for T in self.w.seg_starts:
-            n += self.segment_tiered(T, ev) if self.w.tiered else self.segment(T, ev)
+        for si, T in enumerate(self.w.seg_starts):
+            n += self.segment_tiered(T, ev, si=si) if self.w.tiered else self.segment(T, ev)
         return n
 
 
@@ -475,49 +535,127 @@ def decode_oracle_sample(w, target_seconds):
     return 1.0 / per_token, desc, 1
 
 
-def oracle_sample(w, target_seconds):
-    """Times the CPU oracle on a bounded sample of the workload; returns (tok/s, desc, cores)."""
+def _oracle_block_task(task):
+    """One sampled query block through the oracle (a worker of the CPU baseline):
+    forward of the block's rows for every head and, when dO is given, the backward's
+    dQ rows of the same block.  The routed chunks of the block arrive gathered in
+    route order, so the oracle runs the same arithmetic as on the whole history.
+    Returns (forward seconds, backward seconds)."""
+    import numpy as np
+
+    import oracle
+    shp, m, q_blk, kh, vh, ks, vs, idx, do_blk = task
+    B, Hq, _, D = q_blk.shape
+    S = ks.shape[2]
+    q = np.zeros((B, Hq, S, D), dtype=np.float32)
+    q[:, :, m * 64:(m + 1) * 64] = q_blk
+    rows = np.array([(b * Hq + h) * S + m * 64 + i for b in range(B) for h in range(Hq) for i in range(64)],
+                    dtype=np.int64)
+    sh = oracle.shape(*shp)
+    t0 = time.perf_counter()
+    oracle.attn_fwd(sh, q, kh, vh, ks, vs, idx, rows=rows)
+    t_f = time.perf_counter() - t0
+    t_b = 0.0
+    if do_blk is not None:
+        do = np.zeros_like(q)
+        do[:, :, m * 64:(m + 1) * 64] = do_blk
+        q_need = np.zeros((B, Hq, S), dtype=np.uint8)
+        q_need[:, :, m * 64:(m + 1) * 64] = 1
+        key_need = np.zeros((B, ks.shape[1], S), dtype=np.uint8)
+        t0 = time.perf_counter()
+        oracle.attn_bwd(sh, q, kh, vh, ks, vs, idx, do, q_need=q_need, key_need=key_need)
+        t_b = time.perf_counter() - t0
+    return t_f, t_b
+
+
+def oracle_sample(w, target_seconds, procs=1):
+    """Times the CPU oracle on a bounded sample of the workload and projects it to one
+    step; returns (tok/s, cpu_baseline dict)."""
+    info = cpu_info()
     if w.decode:
-        return decode_oracle_sample(w, target_seconds)
+        tok_s, desc, cores = decode_oracle_sample(w, target_seconds)
+        return tok_s, {"cores": cores, "sample": desc, **info}
     import numpy as np
 
     import oracle
     from inputs import gen
     T = w.seg_starts[-1]
-    S, D = w.seg_len, w.head_dim
-    # same recipe as inputs/gen.py, drawn with torch on the host (faster than numpy for 128K tokens)
+    S, D, B = w.seg_len, w.head_dim, w.batch
+    nqb = S // w.q_block
     q = gen.queries_torch(w, T, T + S, "cpu").float().numpy()
     k_all = gen.keys_torch(w, 0, T + S, "cpu").float().numpy()
     v_all = gen.values_torch(w, 0, T + S, "cpu").float().numpy()
-    sh = oracle.shape(w.batch, w.n_q_heads, w.n_kv_heads, D, w.chunk, w.q_block, w.topk, S, T // w.chunk,
-                      w.sink_chunks)
+    do = gen.grad_out_torch(w, T, T + S, "cpu").float().numpy() if w.backward else None
+    sh = oracle.shape(B, w.n_q_heads, w.n_kv_heads, D, w.chunk, w.q_block, w.topk, S, T // w.chunk, w.sink_chunks)
     t0 = time.perf_counter()
     oracle.summaries(k_all[:, :, T:], w.chunk)  # detach-time summaries of the segment
     t_summ = time.perf_counter() - t0
-    summ = oracle.summaries(k_all[:, :, :T], w.chunk) if T else np.zeros((w.batch, w.n_kv_heads, 0, D))
+    summ = oracle.summaries(k_all[:, :, :T], w.chunk) if T else np.zeros((B, w.n_kv_heads, 0, D))
     t0 = time.perf_counter()
     idx, _, _ = oracle.route(sh, q, summ)
     t_route = time.perf_counter() - t0
-    nqb = S // w.q_block
-    t_attn, blocks = 0.0, []
-    for m in range(nqb - 1, -1, -max(1, nqb // 8)):
-        rows = np.array([(b * w.n_q_heads + h) * S + m * w.q_block + i for b in range(w.batch)
-                         for h in range(w.n_q_heads) for i in range(w.q_block)], dtype=np.int64)
-        t0 = time.perf_counter()
-        oracle.attn_fwd(sh, q, k_all[:, :, :T], v_all[:, :, :T], k_all[:, :, T:], v_all[:, :, T:], idx, rows=rows)
-        t_attn += time.perf_counter() - t0
-        blocks.append(m)
-        if t_attn + t_route > target_seconds:
-            break
     keff = min(w.topk, T // w.chunk)
-    cost = lambda m: keff * w.chunk + m * w.q_block + (w.q_block + 1) / 2  # mean attended keys of block m
-    frac = sum(cost(m) for m in blocks) / sum(cost(m) for m in range(nqb))
-    seg_seconds = t_attn / frac + t_route + t_summ
-    tok_s = S * w.batch / seg_seconds
-    desc = (f"oracle fp64 single-thread on the last {S}-token segment (T={T}): summaries + route of the whole "
-            f"segment, attention forward of query blocks {sorted(blocks)} (all {w.n_q_heads} heads) scaled by "
-            f"attended-key count to the segment; {t_attn + t_route + t_summ:.1f} s CPU")
-    return tok_s, desc, 1
+    ks, vs = np.ascontiguousarray(k_all[:, :, T:]), np.ascontiguousarray(v_all[:, :, T:])
+
+    def task(m):
+        # the block's routed chunks gathered in route order: chunk slot a of head g
+        kh = np.zeros((B, w.n_kv_heads, max(keff, 1) * w.chunk, D), dtype=np.float32)
+        vh = np.zeros_like(kh)
+        ic = np.full(idx.shape, -1, dtype=np.int32)
+        for b in range(B):
+            for g in range(w.n_kv_heads):
+                for a, j in enumerate(idx[b, g, m]):
+                    if j >= 0:
+                        kh[b, g, a * w.chunk:(a + 1) * w.chunk] = k_all[b, g, j * w.chunk:(j + 1) * w.chunk]
+                        vh[b, g, a * w.chunk:(a + 1) * w.chunk] = v_all[b, g, j * w.chunk:(j + 1) * w.chunk]
+                        ic[b, g, m, a] = a
+        shp = (B, w.n_q_heads, w.n_kv_heads, D, w.chunk, w.q_block, w.topk, S, max(keff, 1), 0)
+        d_blk = do[:, :, m * 64:(m + 1) * 64] if do is not None else None
+        return shp, m, q[:, :, m * 64:(m + 1) * 64].copy(), kh, vh, ks, vs, ic, d_blk
+
+    # blocks spread over the segment, latest (most keys) first
+    order = list(range(nqb - 1, -1, -max(1, nqb // 8)))
+    times, blocks = [], []
+    t_wall0 = time.perf_counter()
+    if procs <= 1:
+        for m in order:
+            times.append(_oracle_block_task(task(m)))
+            blocks.append(m)
+            if sum(a + b for a, b in times) + t_route > target_seconds:
+                break
+    else:
+        import concurrent.futures
+        import multiprocessing
+        n_tasks = min(len(order), procs * max(1, int(target_seconds // 8)))
+        blocks = sorted({order[int(i * len(order) / n_tasks)] for i in range(n_tasks)}, reverse=True)
+        ctx = multiprocessing.get_context("spawn")  # never fork a process that has used the GPU
+        with concurrent.futures.ProcessPoolExecutor(max_workers=procs, mp_context=ctx) as ex:
+            t_wall0 = time.perf_counter()
+            times = list(ex.map(_oracle_block_task, [task(m) for m in blocks]))
+    t_wall = time.perf_counter() - t_wall0
+    t_fwd = sum(a for a, _ in times)
+    t_bwd = sum(b for _, b in times)
+    # attention work of a block ~ attended keys per row: k_eff*c + m*64 + 32.5
+    cost = lambda kf, m: kf * w.chunk + m * w.q_block + (w.q_block + 1) / 2
+    per_cost_f = t_fwd / sum(cost(keff, m) for m in blocks)
+    per_cost_b = t_bwd / sum(cost(keff, m) for m in blocks)
+    core_s = 0.0
+    route_s = 0.0
+    for Ts in w.seg_starts:  # project to every segment of the step
+        kf = min(w.topk, Ts // w.chunk)
+        core_s += sum(cost(kf, m) for m in range(nqb)) * (per_cost_f + per_cost_b)
+        route_s += t_route * (Ts / T if T else 0.0) + t_summ
+    cores = max(1, procs)
+    step_s = core_s / cores + route_s
+    tok_s = tokens_per_step(w) / step_s
+    what = "forward" + (" + backward dQ rows (dK/dV accumulation not timed)" if w.backward else "")
+    desc = (f"oracle fp64, {cores} process(es) of one thread: summaries + route of the last {S}-token segment "
+            f"(T={T}) and the {what} of query blocks {sorted(blocks)} (all {w.n_q_heads} heads), projected by "
+            f"attended-key count to all {len(w.seg_starts)} segment(s) of a step; blocks sharded over the "
+            f"processes, route and summaries on one; sample {sum(a + b for a, b in times) + t_route:.1f} "
+            f"core-s in {t_wall + t_route:.1f} s wall")
+    return tok_s, {"cores": cores, "sample": desc, "core_seconds_per_step": round(core_s + route_s, 2),
+                   "wall_seconds_per_step": round(step_s, 3), **info}
 
 
 # ------------------------------------------------------------------ arms
@@ -529,9 +667,11 @@ def run_reference(args, rank):
     import oracle
     oracle.build()
     budget = max(2.0, min(args.cpu_seconds, 150.0 / max(1, args.steps + args.warmup)))
-    per_step, desc = [], ""
+    per_step, cb, walls = [], {}, []
     for s in range(args.warmup + args.steps):
-        tok_s, desc, cores = oracle_sample(w, budget)
+        t0 = time.perf_counter()
+        tok_s, cb = oracle_sample(w, budget)
+        walls.append((time.perf_counter() - t0) * 1000)
         if s >= args.warmup:
             per_step.append(tok_s)
     v = statistics.median(per_step)
@@ -540,7 +680,10 @@ def run_reference(args, rank):
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, args.gpus),
-            "cpu_baseline": {"value": v, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": desc},
+            "step_is_sample": "each step times a bounded sample of the workload on the host cores; value and "
+                              "ms_per_step are that sample projected to a whole step",
+            "sample_wall_ms_per_step": round(statistics.median(walls[args.warmup:]), 1),
+            "cpu_baseline": {"value": v, "unit": UNIT, "kind": "oracle", **cb},
             "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -563,17 +706,11 @@ def host_link_gbs(nbytes=256 << 20):
     return best
 
 
-def run_hga(args, rank, world, local):
+def measure_layer(w, args, world, local):
+    """Times one device-resident or tiered workload; returns its JSON fields."""
     import torch
-    from inputs import gen
     import hierarchical_sparse_long_b200 as hga
-    from hierarchical_sparse_long_b200 import build
-    if rank == 0:
-        build.build()
-    if world > 1:
-        torch.distributed.barrier()
-    hga.lib()
-    w = gen.WORKLOADS[args.workload]
+    Layer.wave = args.tier_wave
     layer = Layer(w)
     layer.side_append = not args.serial_append and not w.tiered
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda", dtype=torch.float32)
@@ -582,7 +719,7 @@ def run_hga(args, rank, world, local):
         layer.step()
     torch.cuda.synchronize()
     if hga.hga_get_device_status() != 0:
-        raise RuntimeError("device status reported an error during warm-up")
+        raise RuntimeError(f"{w.name}: device status reported an error during warm-up")
     # Device-resident workloads replay one step captured as a CUDA graph (one
     # host launch per step, phase events recorded inside the graph); the tiered
     # workload drives its copy stream from the host and stays eager.
@@ -625,7 +762,7 @@ def run_hga(args, rank, world, local):
         torch.distributed.barrier()
     clocks = sampler.stop()
     total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, "cuda")
-    value = job_throughput(w.seg_len * w.batch * len(w.seg_starts), args.steps, world, total_ms)
+    value = job_throughput(tokens_per_step(w), args.steps, world, total_ms)
     status = hga.hga_get_device_status()
 
     # per-kernel device time over the timed steps (events on the launching stream)
@@ -648,7 +785,7 @@ def run_hga(args, rank, world, local):
     if layer.side_append:
         kernels["summaries"]["note"] = "on a side stream, timed while it overlaps the route"
     if w.tiered:
-        kernels["attn_fwd"]["note"] = "includes waits for the wave fetches it cannot hide"
+        kernels["attn_fwd"]["note"] = "hga_attn_fwd_tiered: includes the waits for the fetch waves it cannot hide"
         kernels["summaries"]["note"] = "includes the segment K/V copy to host memory"
     if w.backward:
         bwd_fl = sum(attn_bwd_flops(w, T) for T in w.seg_starts) * args.steps
@@ -666,27 +803,63 @@ def run_hga(args, rank, world, local):
             "peak_source": f"{peak_src}: MEASURED_PEAKS.json bf16_tflops (burst)",
             "units_per_launch": "4*D*(k_eff*64+i+1) flop per query row and head" if dom == "attn_fwd" else
             "dQ 6*D per attended key, dK/dV 8*D per causal segment pair, per row and head"}
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(w, world),
-                       "l2": "flushed before every timed step (256 MiB write)",
-                       "launch": "one CUDA graph replay per step" if graph is not None else "eager",
-                       "append": "side stream, overlapped with the route" if layer.side_append else "in order"},
-            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
-            "device_status": status}
+    res = {"value": value, "unit": UNIT, "ms_per_step": total_ms / args.steps,
+           "config": {**workload_config(w, world),
+                      "l2": "flushed before every timed step (256 MiB write)",
+                      "launch": "one CUDA graph replay per step" if graph is not None else "eager",
+                      "append": "side stream, overlapped with the route" if layer.side_append else "in order"},
+           "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
+           "device_status": status}
     if w.tiered:
-        fetched = int(layer.n_fetched.sum().item())
-        link = host_link_gbs()
-        nbytes = fetched * 2 * w.chunk * w.head_dim * 2
-        line["tiered"] = {"tiles_fetched_last_segment": fetched, "bytes_fetched_last_segment": nbytes,
-                          "host_link_gbs_measured": round(link, 2)}
-    line["e2e"] = e2e_measure(layer, max(2, min(args.steps, 5)))
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, desc, cores = oracle_sample(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+        res["tiered"] = tiered_report(layer, total_ms / args.steps, ph["attn_fwd"] / args.steps, flush)
+        # the step's dominant cost is the host link: its own roofline line
+        t = res["tiered"]
+        res["roofline_host_link"] = {"bound": "host link", "achieved": t["link_gbs_achieved"],
+                                     "peak": t["host_link_gbs_measured"], "unit": "GB/s",
+                                     "frac": round(t["link_gbs_achieved"] / t["host_link_gbs_measured"], 4),
+                                     "peak_source": "pinned host -> device cudaMemcpyAsync measured in this run"}
+    res["e2e"] = e2e_measure(layer, max(2, min(args.steps, 5)))
+    del layer, graph
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def tiered_report(layer, step_ms, attn_phase_ms, flush):
+    """Host-link accounting of the tiered step: tiles fetched per step against the
+    distinct tiles the segments route to, the fetch-only step and the resident
+    attention (no host link), and the share of the attention hidden under the
+    fetches: (fetch-only + resident attention - tiered attention phase) /
+    resident attention, the tiered phase being the fetch waves and attention of
+    every segment on the compute stream's timeline."""
+    import torch
+    w = layer.w
+    fetched = int(layer.n_fetched.sum().item())
+    per_segment, whole = layer.distinct_tiles()
+    flush_l2(flush)
+    t_fetch = layer.fetch_only_step()
+    # the attention alone with the history resident in device memory (no host link)
+    ev = PhaseEvents()
+    flush_l2(flush)
+    for T in w.seg_starts:
+        layer.segment(T, ev=ev)
+    torch.cuda.synchronize()
+    t_res = ev.totals()["attn_fwd"]
+    link = host_link_gbs()
+    tb = TILE_PAIR_BYTES(w)
+    hidden = (t_fetch + t_res - attn_phase_ms) / t_res if t_res > 0 else None
+    return {"staging_slots": layer.slots, "staging_mib": round(layer.slots * tb / 2**20, 1),
+            "cache_policy": "one segment's routing budget of chunk tiles, kept from segment to segment and "
+                            f"emptied when the evaluation starts; waves of {layer.wave} query blocks",
+            "tiles_fetched_per_step": fetched, "tiles_distinct_per_segment_summed": per_segment,
+            "tiles_distinct_per_step": whole,
+            "bytes_fetched_per_step": fetched * tb, "bytes_distinct_per_segment_summed": per_segment * tb,
+            "fetched_over_distinct_per_segment": round(fetched / per_segment, 4) if per_segment else None,
+            "ms_fetch_only_step": round(t_fetch, 3), "ms_attention_resident": round(t_res, 3),
+            "ms_attention_phase_tiered": round(attn_phase_ms, 3),
+            "attention_hidden_share": round(hidden, 4) if hidden is not None else None,
+            "link_gbs_achieved": round(fetched * tb / (step_ms / 1e3) / 1e9, 2),
+            "host_link_gbs_measured": round(link, 2)}
 
 
 def e2e_measure(layer, steps):
@@ -712,7 +885,7 @@ def e2e_measure(layer, steps):
     for it in range(steps + 1):
         torch.cuda.synchronize()
         s.record()
-        for T in w.seg_starts:
+        for si, T in enumerate(w.seg_starts):
             hi = host_in[T]
             q_d.copy_(hi[0], non_blocking=True)
             layer.k[:, :, T:T + S].copy_(hi[1], non_blocking=True)
@@ -720,7 +893,7 @@ def e2e_measure(layer, steps):
             if do_d is not None:
                 do_d.copy_(hi[3], non_blocking=True)
             if w.tiered:
-                layer.segment_tiered(T, q=q_d)
+                layer.segment_tiered(T, q=q_d, si=si)
             else:
                 layer.segment(T, q=q_d, do=do_d)
             for hbuf, t in zip(host_out, outs):
@@ -730,9 +903,54 @@ def e2e_measure(layer, steps):
         if it >= 1:
             times.append(s.elapsed_time(e))
     ms = statistics.mean(times)
-    return {"value": w.seg_len * w.batch * len(w.seg_starts) / (ms / 1000.0), "unit": UNIT,
+    return {"value": tokens_per_step(w) / (ms / 1000.0), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
             "scope": "every segment of the step through the C ABI from pinned host buffers"}
+
+
+def cpu_procs(args):
+    if args.cpu_procs > 0:
+        return args.cpu_procs
+    return max(1, min(8, cpu_info()["usable_cpus"]))
+
+
+def run_hga(args, rank, world, local):
+    import torch
+    from inputs import gen
+    import hierarchical_sparse_long_b200 as hga
+    from hierarchical_sparse_long_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    hga.lib()
+    w = gen.WORKLOADS[args.workload]
+    res = measure_layer(w, args, world, local)
+    line = {"metric": METRIC, "value": res.pop("value"), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", **res}
+    also = list(ALSO_DEFAULT) if (args.also == "auto" and args.workload == "qwen3_16k_fwd") else \
+        [a for a in args.also.split(",") if a and a not in ("auto", "none")]
+    nested = {}
+    for name in also:
+        wn = gen.WORKLOADS[name]
+        nested[name] = (run_decode_measure(wn, args, world, local) if wn.decode
+                        else measure_layer(wn, args, world, local))
+    baseline = rank == 0 and world == 1 and not args.no_cpu_baseline
+    if baseline:
+        import oracle
+        oracle.build()
+        tok_s, cb = oracle_sample(w, args.cpu_seconds, 1)
+        line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "kind": "oracle", **cb}
+        for name, r in nested.items():
+            wn = gen.WORKLOADS[name]
+            procs = cpu_procs(args) if wn.seq_len > 32768 else 1
+            tok_s, cb = oracle_sample(wn, min(args.cpu_seconds, 10.0), procs)
+            r["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "kind": "oracle", **cb}
+    if nested:
+        line["workloads"] = nested
+    if rank == 0:
+        print(json.dumps(line), flush=True)
 
 
 class DecodeLayer:
@@ -777,19 +995,11 @@ class DecodeLayer:
         return 3
 
 
-def run_decode(args, rank, world, local):
-    """bench.py for a decode workload: one step = route + decode attention of one new
-    token per sequence (query tok/s = tokens generated per second)."""
+def run_decode_measure(w, args, world, local):
+    """Times a decode workload: one step = route + decode attention of one new token
+    per sequence (query tok/s = tokens generated per second); returns its JSON fields."""
     import torch
-    from inputs import gen
     import hierarchical_sparse_long_b200 as hga
-    from hierarchical_sparse_long_b200 import build
-    if rank == 0:
-        build.build()
-    if world > 1:
-        torch.distributed.barrier()
-    hga.lib()
-    w = gen.WORKLOADS[args.workload]
     layer = DecodeLayer(w)
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda", dtype=torch.float32)
     for _ in range(args.warmup):
@@ -854,18 +1064,40 @@ def run_decode(args, rank, world, local):
             "peak_source": f"{peak_src}: MEASURED_PEAKS.json hbm_gbs",
             "units_per_launch": "K and V of the routed chunks and the local window once per (sequence, kv head), "
                                 "plus q, O and the route table"}
-    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": total_ms / args.steps, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {**workload_config(w, world),
-                       "l2": "flushed before every timed step (256 MiB write)",
-                       "launch": "one CUDA graph replay per step"},
-            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
-            "device_status": status}
-    line["e2e"] = decode_e2e(layer, max(2, min(args.steps, 5)))
+    res = {"value": value, "unit": UNIT, "ms_per_step": total_ms / args.steps,
+           "config": {**workload_config(w, world),
+                      "l2": "flushed before every timed step (256 MiB write)",
+                      "launch": "one CUDA graph replay per step"},
+           "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
+           "device_status": status}
+    res["e2e"] = decode_e2e(layer, max(2, min(args.steps, 5)))
+    del layer, graph
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode(args, rank, world, local):
+    """bench.py with a decode workload as the headline."""
+    import torch
+    from inputs import gen
+    import hierarchical_sparse_long_b200 as hga
+    from hierarchical_sparse_long_b200 import build
+    if rank == 0:
+        build.build()
+    if world > 1:
+        torch.distributed.barrier()
+    hga.lib()
+    w = gen.WORKLOADS[args.workload]
+    res = run_decode_measure(w, args, world, local)
+    line = {"metric": METRIC, "value": res.pop("value"), "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": res.pop("ms_per_step"), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic", **res}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tok_s, desc, cores = oracle_sample(w, args.cpu_seconds)
-        line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "cores": cores, "kind": "oracle", "sample": desc}
+        import oracle
+        oracle.build()
+        tok_s, cb = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {"value": tok_s, "unit": UNIT, "kind": "oracle", **cb}
     if rank == 0:
         print(json.dumps(line), flush=True)
 

@@ -17,12 +17,15 @@ _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libhga.so")
 
 HGA_BF16, HGA_FP32 = 0, 1
-HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT = 1, 2
+HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT, HGA_DEV_STAGE_FULL = 1, 2, 4
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3: "HGA_ERR_CUDA",
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
-EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd_workspace_size", "hga_attn_bwd",
-            "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_fetch_tiered",
+EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd",
+            "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_attn_fwd_groups", "hga_attn_bwd_groups",
+            "hga_attn_causal_workspace_size", "hga_attn_fwd_causal", "hga_attn_bwd_causal",
+            "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_tier_scratch_size",
+            "hga_tier_reset", "hga_fetch_tiered", "hga_tier_offload", "hga_attn_fwd_tiered",
             "hga_get_device_status", "hga_selftest_wait_timeout", "hga_status_string", "hga_last_error")
 
 
@@ -86,6 +89,12 @@ def lib() -> ctypes.CDLL:
         L.hga_route_causal.argtypes = [pp, vp, vp, i, vp, vp]
         L.hga_route_groups.argtypes = [pp, vp, vp, i, vp, i, i, vp, vp]
         L.hga_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.hga_attn_fwd_groups.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp]
+        L.hga_attn_bwd_groups.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.hga_attn_causal_workspace_size.argtypes = [pp, i]
+        L.hga_attn_causal_workspace_size.restype = sz
+        L.hga_attn_fwd_causal.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+        L.hga_attn_bwd_causal.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.hga_attn_bwd_workspace_size.argtypes = [pp]
         L.hga_attn_bwd_workspace_size.restype = sz
         L.hga_attn_bwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
@@ -93,15 +102,24 @@ def lib() -> ctypes.CDLL:
         L.hga_attn_decode_workspace_size.argtypes = [pp, i]
         L.hga_attn_decode_workspace_size.restype = sz
         L.hga_attn_decode.argtypes = [pp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, sz, vp]
+        L.hga_tier_scratch_size.argtypes = [pp, i]
+        L.hga_tier_scratch_size.restype = sz
+        L.hga_tier_reset.argtypes = [pp, i, vp, vp]
         L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
+        L.hga_tier_offload.argtypes = [pp, vp, vp, vp, vp, ll, vp]
+        L.hga_attn_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp, vp, vp,
+                                          ctypes.POINTER(vp)]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hga_selftest_wait_timeout.argtypes = [ll, vp]
         L.hga_selftest_wait_timeout.restype = ctypes.c_int
         L.hga_status_string.argtypes = [i]
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
-        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd", "hga_attn_bwd", "hga_attn_bwd_noalloc",
-                  "hga_attn_decode", "hga_fetch_tiered", "hga_get_device_status"):
+        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd",
+                  "hga_attn_bwd", "hga_attn_bwd_noalloc", "hga_attn_fwd_groups", "hga_attn_bwd_groups",
+                  "hga_attn_fwd_causal", "hga_attn_bwd_causal",
+                  "hga_attn_decode", "hga_tier_reset", "hga_fetch_tiered", "hga_tier_offload", "hga_attn_fwd_tiered",
+                  "hga_get_device_status"):
             getattr(L, f).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -172,6 +190,51 @@ def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stre
                               _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)), "hga_attn_fwd")
 
 
+def hga_attn_fwd_groups(p: Params, q, k_hist, v_hist, k_seg, v_seg, gidx, group: int, topg: int, out, lse,
+                        stream=None):
+    """Attention over the routed groups (hga_route_groups) + the causal segment."""
+    cp = p.c()
+    _check(lib().hga_attn_fwd_groups(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg),
+                                     _ptr(v_seg), _ptr(gidx), group, topg, _ptr(out), _ptr(lse), _stream(stream)),
+           "hga_attn_fwd_groups")
+
+
+def hga_attn_bwd_groups(p: Params, q, k_hist, v_hist, k_seg, v_seg, gidx, group: int, topg: int, out, lse, dout,
+                        dq, dk_seg, dv_seg, workspace, stream=None):
+    """Backward of hga_attn_fwd_groups: dq over routed groups and segment, dk/dv of the segment."""
+    cp = p.c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().hga_attn_bwd_groups(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg),
+                                     _ptr(v_seg), _ptr(gidx), group, topg, _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                     _ptr(dk_seg), _ptr(dv_seg), _ptr(workspace), nbytes, _stream(stream)),
+           "hga_attn_bwd_groups")
+
+
+def hga_attn_causal_workspace_size(p: Params, backward: bool = False) -> int:
+    cp = p.c()
+    return int(lib().hga_attn_causal_workspace_size(ctypes.byref(cp), 1 if backward else 0))
+
+
+def hga_attn_fwd_causal(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx_tok, out, lse, workspace, stream=None):
+    """Attention over per-token (strictly causal) routes [B][Hkv][S][k] + the causal segment."""
+    cp = p.c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().hga_attn_fwd_causal(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg),
+                                     _ptr(v_seg), _ptr(idx_tok), _ptr(out), _ptr(lse), _ptr(workspace), nbytes,
+                                     _stream(stream)), "hga_attn_fwd_causal")
+
+
+def hga_attn_bwd_causal(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx_tok, out, lse, dout, dq, dk_seg, dv_seg,
+                        workspace, stream=None):
+    """Backward of hga_attn_fwd_causal."""
+    cp = p.c()
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(lib().hga_attn_bwd_causal(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg),
+                                     _ptr(v_seg), _ptr(idx_tok), _ptr(out), _ptr(lse), _ptr(dout), _ptr(dq),
+                                     _ptr(dk_seg), _ptr(dv_seg), _ptr(workspace), nbytes, _stream(stream)),
+           "hga_attn_bwd_causal")
+
+
 def hga_attn_decode_workspace_size(p: Params, n_local: int) -> int:
     cp = p.c()
     return int(lib().hga_attn_decode_workspace_size(ctypes.byref(cp), n_local))
@@ -214,15 +277,52 @@ def hga_attn_bwd_noalloc(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, l
                                       _ptr(dk_seg), _ptr(dv_seg), _stream(stream)), "hga_attn_bwd_noalloc")
 
 
+def hga_tier_scratch_size(p: Params, stage_slots: int) -> int:
+    """Bytes of int32 scratch the tiered staging cache of stage_slots tiles needs."""
+    cp = p.c()
+    return int(lib().hga_tier_scratch_size(ctypes.byref(cp), stage_slots))
+
+
+def hga_tier_reset(p: Params, stage_slots: int, scratch, stream=None):
+    """Marks every slot of the staging cache empty."""
+    cp = p.c()
+    _check(lib().hga_tier_reset(ctypes.byref(cp), stage_slots, _ptr(scratch), _stream(stream)), "hga_tier_reset")
+
+
 def hga_fetch_tiered(p: Params, host_k, host_v, idx, qblock_begin: int, qblock_end: int, stage_k, stage_v,
-                     stage_slots: int, slot_map, idx_remapped, n_fetched=None, copy_stream=None, done=None):
-    """Copies only the routed chunks' K/V tiles from pinned host memory into staging slots."""
+                     stage_slots: int, scratch, idx_remapped, n_fetched=None, copy_stream=None, done=None):
+    """One fetch wave: the routed tiles of blocks [qblock_begin, qblock_end) the staging
+    cache does not hold are copied from pinned host memory; idx_remapped gets slots."""
     cp = p.c()
     ev = None if done is None else ctypes.c_void_p(done.cuda_event)
     _check(lib().hga_fetch_tiered(ctypes.byref(cp), _ptr(host_k), _ptr(host_v), _ptr(idx), qblock_begin,
-                                  qblock_end, _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(slot_map),
+                                  qblock_end, _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(scratch),
                                   _ptr(idx_remapped), _ptr(n_fetched), _stream(copy_stream), ev),
            "hga_fetch_tiered")
+
+
+def hga_tier_offload(p: Params, k_seg, v_seg, host_k, host_v, dst_token: int, stream=None):
+    """Copies the segment's K/V (every (b, g) slice) into the pinned host history at dst_token."""
+    cp = p.c()
+    _check(lib().hga_tier_offload(ctypes.byref(cp), _ptr(k_seg), _ptr(v_seg), _ptr(host_k), _ptr(host_v),
+                                  dst_token, _stream(stream)), "hga_tier_offload")
+
+
+def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v,
+                        stage_slots: int, scratch, idx_remapped, wave_blocks: int, events, reset_cache=False,
+                        n_fetched=None, stream=None, copy_stream=None):
+    """Attention over host-resident history: fetch waves on copy_stream overlapped with
+    the attention of the previous wave on stream (events: five torch.cuda.Event)."""
+    cp = p.c()
+    for e in events:
+        if not e.cuda_event:  # torch creates its CUDA event on the first record
+            e.record()
+    evs = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+    _check(lib().hga_attn_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(host_k), _ptr(host_v), _ptr(k_seg),
+                                     _ptr(v_seg), _ptr(idx), _ptr(out), _ptr(lse), _ptr(stage_k), _ptr(stage_v),
+                                     stage_slots, _ptr(scratch), _ptr(idx_remapped), wave_blocks,
+                                     1 if reset_cache else 0, _ptr(n_fetched), _stream(stream),
+                                     _stream(copy_stream), evs), "hga_attn_fwd_tiered")
 
 
 def hga_selftest_wait_timeout(wait_cycles: int, stream=None):

@@ -9,9 +9,21 @@
 #include <mutex>
 #include <string>
 
+#include <nvtx3/nvToolsExt.h>
+
 #include "common.cuh"
 
 namespace {
+
+// An NVTX range named after the entry point around every C-ABI call (the
+// host-side validation and the launches), for timelines taken with a
+// profiler; without one attached a push/pop is a call through a no-op stub.
+struct CallRange {
+    explicit CallRange(const char *name) { nvtxRangePushA(name); }
+    ~CallRange() { nvtxRangePop(); }
+    CallRange(const CallRange &) = delete;
+    CallRange &operator=(const CallRange &) = delete;
+};
 
 __device__ unsigned int g_status_word;
 
@@ -94,6 +106,7 @@ const char *hga_last_error(void) { return t_last_error.c_str(); }
 hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch, int n_kv_heads, int head_dim,
                                  int chunk, int first_chunk, int n_chunks, hga_dtype_t dtype, float *summ,
                                  int summ_cap_chunks, cudaStream_t stream) {
+    CallRange range("hga_build_summaries");
     if (batch < 1 || n_kv_heads < 1 || n_chunks < 0 || first_chunk < 0 || chunk < 1) return HGA_ERR_INVALID_ARG;
     if (dtype != HGA_BF16 && dtype != HGA_FP32) return HGA_ERR_INVALID_ARG;
     if (head_dim != 64 && head_dim != 128) return HGA_ERR_UNSUPPORTED;
@@ -107,6 +120,7 @@ hga_status_t hga_build_summaries(const void *k, long long head_stride, int batch
 
 hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks, int32_t *idx,
                        cudaStream_t stream) {
+    CallRange range("hga_route");
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (summ_cap_chunks < p->n_hist_chunks) return HGA_ERR_INVALID_ARG;
@@ -120,6 +134,7 @@ hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, 
 
 hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float *gsumm, int gsumm_cap_groups,
                               const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream) {
+    CallRange range("hga_route_groups");
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (group != 8 && group != 16 && group != 32) return HGA_ERR_INVALID_ARG;
@@ -133,6 +148,7 @@ hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float 
 
 hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
                               int32_t *idx, cudaStream_t stream) {
+    CallRange range("hga_route_causal");
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (summ_cap_chunks < p->n_hist_chunks) return HGA_ERR_INVALID_ARG;
@@ -147,6 +163,7 @@ hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float 
 hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                           const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
                           cudaStream_t stream) {
+    CallRange range("hga_attn_fwd");
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
@@ -156,8 +173,16 @@ hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hi
         if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
-    if (hga::attn_fwd_tc_supported(*p))
+    // bf16 with head_dim 128 runs on the tcgen05 kernel and nowhere else; fp32
+    // (and bf16 with head_dim 64) on the CUDA-core kernel
+    if (hga::attn_fwd_tc_shape(*p)) {
+        if (!hga::attn_fwd_tc_supported(*p)) {
+            hga::record_error("hga_attn_fwd: the tcgen05 kernel cannot take this call (no TMA tensor-map "
+                              "encoder in the driver, or a row coordinate beyond 32 bits)");
+            return HGA_ERR_UNSUPPORTED;
+        }
         return hga::launch_attn_fwd_tc(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status, stream);
+    }
     return hga::launch_attn_fwd_simt(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status, stream);
 }
 
@@ -171,6 +196,7 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
                           const void *k_seg, const void *v_seg, const int32_t *idx, const void *out,
                           const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg, void *workspace,
                           size_t workspace_bytes, cudaStream_t stream) {
+    CallRange range("hga_attn_bwd");
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
@@ -185,7 +211,12 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
     float *delta = static_cast<float *>(workspace);
-    if (hga::attn_bwd_tc_supported(*p)) {
+    if (hga::attn_fwd_tc_shape(*p)) {
+        if (!hga::attn_bwd_tc_supported(*p)) {
+            hga::record_error("hga_attn_bwd: the tcgen05 kernel cannot take this call (no TMA tensor-map "
+                              "encoder in the driver, or a row coordinate beyond 32 bits)");
+            return HGA_ERR_UNSUPPORTED;
+        }
         st = hga::launch_bwd_delta(*p, out, dout, delta, stream);
         if (st != HGA_OK) return st;
         return hga::launch_attn_bwd_tc(*p, q, k_hist, v_hist, k_seg, v_seg, idx, lse, delta, dout,
@@ -196,6 +227,138 @@ hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hi
                                      delta, status, stream);
 }
 
+namespace {
+
+// Checks shared by the group-routed and token-masked attention calls: the
+// tcgen05 shape only (bf16, head_dim 128), every block, pointers as in
+// hga_attn_fwd / hga_attn_bwd.
+hga_status_t check_routed_attn(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                               const void *k_seg, const void *v_seg, const void *routes, const void *out,
+                               const float *lse) {
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;
+    if (!hga::attn_fwd_tc_shape(*p)) {
+        hga::record_error("group-routed and token-masked attention run on the tcgen05 kernels only "
+                          "(bf16, head_dim 128)");
+        return HGA_ERR_UNSUPPORTED;
+    }
+    if (!hga::attn_fwd_tc_supported(*p)) {
+        hga::record_error("the tcgen05 kernel cannot take this call (no TMA tensor-map encoder in the "
+                          "driver, or a row coordinate beyond 32 bits)");
+        return HGA_ERR_UNSUPPORTED;
+    }
+    if (!q || !k_seg || !v_seg || !routes || !out || !lse) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {q, k_hist, v_hist, k_seg, v_seg, out})
+        if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    return HGA_OK;
+}
+
+hga_status_t check_group_args(const hga_params_t *p, int group, int topg) {
+    if (group != 8 && group != 16 && group != 32) return HGA_ERR_INVALID_ARG;
+    const int gpc = p->chunk / group;
+    if (topg < 1 || topg > p->topk * gpc || topg > 512) return HGA_ERR_INVALID_ARG;
+    return HGA_OK;
+}
+
+hga_status_t check_bwd_outputs(const hga_params_t *p, const void *dout, const void *dq, const void *dk,
+                               const void *dv) {
+    if (p->qblock_begin != 0 || p->qblock_end != 0) return HGA_ERR_INVALID_ARG;
+    if (!dout || !dq || !dk || !dv) return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {dout, dq, dk, dv})
+        if (!aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    return HGA_OK;
+}
+
+size_t delta_bytes(const hga_params_t &p) {
+    const size_t rows = (size_t)p.batch * p.n_q_heads * p.seg_len;
+    return ((rows * sizeof(float)) + 255) & ~(size_t)255;
+}
+
+}  // namespace
+
+hga_status_t hga_attn_fwd_groups(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *gidx, int group, int topg,
+                                 void *out, float *lse, cudaStream_t stream) {
+    CallRange range("hga_attn_fwd_groups");
+    hga_status_t st = check_routed_attn(p, q, k_hist, v_hist, k_seg, v_seg, gidx, out, lse);
+    if (st == HGA_OK) st = check_group_args(p, group, topg);
+    if (st != HGA_OK) return st;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    const hga::FwdRoutes rt{gidx, topg, group, nullptr, nullptr};
+    return hga::launch_attn_fwd_tc_routes(*p, q, k_hist, v_hist, k_seg, v_seg, rt, out, lse, status, stream);
+}
+
+hga_status_t hga_attn_bwd_groups(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *gidx, int group, int topg,
+                                 const void *out, const float *lse, const void *dout, void *dq, void *dk_seg,
+                                 void *dv_seg, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    CallRange range("hga_attn_bwd_groups");
+    hga_status_t st = check_routed_attn(p, q, k_hist, v_hist, k_seg, v_seg, gidx, out, lse);
+    if (st == HGA_OK) st = check_group_args(p, group, topg);
+    if (st == HGA_OK) st = check_bwd_outputs(p, dout, dq, dk_seg, dv_seg);
+    if (st != HGA_OK) return st;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < delta_bytes(*p)) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    float *delta = static_cast<float *>(workspace);
+    st = hga::launch_bwd_delta(*p, out, dout, delta, stream);
+    if (st != HGA_OK) return st;
+    const hga::FwdRoutes rt{gidx, topg, group, nullptr, nullptr};
+    return hga::launch_attn_bwd_tc_routes(*p, q, k_hist, v_hist, k_seg, v_seg, rt, lse, delta, dout,
+                                          static_cast<float *>(dq), static_cast<float *>(dk_seg),
+                                          static_cast<float *>(dv_seg), status, stream);
+}
+
+size_t hga_attn_causal_workspace_size(const hga_params_t *p, int backward) {
+    if (check_params(p) != HGA_OK || p->q_block != 64) return 0;
+    return hga::route_union_bytes(*p) + (backward ? delta_bytes(*p) : 0);
+}
+
+hga_status_t hga_attn_fwd_causal(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *idx_tok, void *out, float *lse,
+                                 void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    CallRange range("hga_attn_fwd_causal");
+    hga_status_t st = check_routed_attn(p, q, k_hist, v_hist, k_seg, v_seg, idx_tok, out, lse);
+    if (st != HGA_OK) return st;
+    if (p->n_hist_chunks > 16384) return HGA_ERR_UNSUPPORTED;
+    if (!workspace || !aligned16(workspace) || workspace_bytes < hga::route_union_bytes(*p))
+        return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    const hga::UnionView u = hga::route_union_view(*p, workspace);
+    st = hga::launch_route_union(*p, idx_tok, u, status, stream);
+    if (st != HGA_OK) return st;
+    const hga::FwdRoutes rt{u.list, u.cap, 0, u.count, u.mask};
+    return hga::launch_attn_fwd_tc_routes(*p, q, k_hist, v_hist, k_seg, v_seg, rt, out, lse, status, stream);
+}
+
+hga_status_t hga_attn_bwd_causal(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *idx_tok, const void *out,
+                                 const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg,
+                                 void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    CallRange range("hga_attn_bwd_causal");
+    hga_status_t st = check_routed_attn(p, q, k_hist, v_hist, k_seg, v_seg, idx_tok, out, lse);
+    if (st == HGA_OK) st = check_bwd_outputs(p, dout, dq, dk_seg, dv_seg);
+    if (st != HGA_OK) return st;
+    if (p->n_hist_chunks > 16384) return HGA_ERR_UNSUPPORTED;
+    const size_t ub = hga::route_union_bytes(*p);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < ub + delta_bytes(*p)) return HGA_ERR_INVALID_ARG;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    const hga::UnionView u = hga::route_union_view(*p, workspace);
+    float *delta = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + ub);
+    st = hga::launch_route_union(*p, idx_tok, u, status, stream);
+    if (st == HGA_OK) st = hga::launch_bwd_delta(*p, out, dout, delta, stream);
+    if (st != HGA_OK) return st;
+    const hga::FwdRoutes rt{u.list, u.cap, 0, u.count, u.mask};
+    return hga::launch_attn_bwd_tc_routes(*p, q, k_hist, v_hist, k_seg, v_seg, rt, lse, delta, dout,
+                                          static_cast<float *>(dq), static_cast<float *>(dk_seg),
+                                          static_cast<float *>(dv_seg), status, stream);
+}
+
 size_t hga_attn_decode_workspace_size(const hga_params_t *p, int n_local) {
     if (check_params(p) != HGA_OK || p->seg_len != 1 || n_local < 1) return 0;
     return hga::decode_workspace_bytes(*p, n_local);
@@ -204,6 +367,7 @@ size_t hga_attn_decode_workspace_size(const hga_params_t *p, int n_local) {
 hga_status_t hga_attn_decode(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                              const void *k_local, const void *v_local, int n_local, const int32_t *idx, void *out,
                              float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream) {
+    CallRange range("hga_attn_decode");
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (p->seg_len != 1 || p->q_block != 1 || n_local < 1 || p->seg_head_stride < n_local)
@@ -220,34 +384,154 @@ hga_status_t hga_attn_decode(const hga_params_t *p, const void *q, const void *k
                               static_cast<float *>(workspace), status, stream);
 }
 
-hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,
-                              int qblock_begin, int qblock_end, void *stage_k, void *stage_v, int stage_slots,
-                              int32_t *slot_map, int32_t *idx_remapped, int32_t *n_fetched, cudaStream_t copy_stream,
-                              cudaEvent_t done) {
+size_t hga_tier_scratch_size(const hga_params_t *p, int stage_slots) {
+    if (check_params(p) != HGA_OK || stage_slots < 1 || p->hist_head_stride < 1) return 0;
+    const size_t bytes = hga::tier_scratch_entries(*p, stage_slots) * sizeof(int32_t);
+    return (bytes + 255) & ~(size_t)255;
+}
+
+hga_status_t hga_tier_reset(const hga_params_t *p, int stage_slots, int32_t *scratch, cudaStream_t stream) {
+    CallRange range("hga_tier_reset");
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (stage_slots < 1 || p->hist_head_stride < 1 || !scratch) return HGA_ERR_INVALID_ARG;
+    return hga::launch_tier_reset(*p, stage_slots, scratch, stream);
+}
+
+namespace {
+
+// Argument checks shared by hga_fetch_tiered and hga_attn_fwd_tiered.  A
+// fetch of `blocks` query blocks may need every routed tile of those blocks,
+// and the tiles of the wave before it stay protected, so the cache must hold
+// twice that -- or every routable tile, after which nothing is ever evicted.
+hga_status_t check_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,
+                          const void *stage_k, const void *stage_v, int stage_slots, const int32_t *scratch,
+                          const int32_t *idx_remapped, int blocks) {
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
-    const int nqb = p->seg_len / p->q_block;
-    if (qblock_begin < 0 || qblock_end <= qblock_begin || qblock_end > nqb) return HGA_ERR_INVALID_ARG;
-    if (p->hist_head_stride < (long long)p->n_hist_chunks * p->chunk) return HGA_ERR_INVALID_ARG;
-    if (!host_k || !host_v || !idx || !stage_k || !stage_v || !slot_map || !idx_remapped || stage_slots < 0)
+    if (p->hist_head_stride < 1 || p->hist_head_stride < (long long)p->n_hist_chunks * p->chunk)
         return HGA_ERR_INVALID_ARG;
-    for (const void *ptr : {host_k, host_v, (const void *)stage_k, (const void *)stage_v})
+    if (!host_k || !host_v || !idx || !stage_k || !stage_v || !scratch || !idx_remapped || stage_slots < 1)
+        return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {host_k, host_v, stage_k, stage_v})
         if (!aligned16(ptr)) return HGA_ERR_INVALID_ARG;
     const int keff = p->topk < p->n_hist_chunks ? p->topk : p->n_hist_chunks;
-    const long long worst = (long long)(qblock_end - qblock_begin) * p->batch * p->n_kv_heads * keff;
+    const long long worst = 2ll * blocks * p->batch * p->n_kv_heads * keff;
     const long long distinct = (long long)p->batch * p->n_kv_heads * p->n_hist_chunks;
-    if ((worst < distinct ? worst : distinct) > stage_slots) return HGA_ERR_INVALID_ARG;
+    if ((worst < distinct ? worst : distinct) > stage_slots) {
+        hga::record_error("tiered: stage_slots below twice the tiles one wave can route (or every routable tile)");
+        return HGA_ERR_INVALID_ARG;
+    }
+    return HGA_OK;
+}
+
+}  // namespace
+
+hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,
+                              int qblock_begin, int qblock_end, void *stage_k, void *stage_v, int stage_slots,
+                              int32_t *scratch, int32_t *idx_remapped, int32_t *n_fetched, cudaStream_t copy_stream,
+                              cudaEvent_t done) {
+    CallRange range("hga_fetch_tiered");
+    if (!p) return HGA_ERR_INVALID_ARG;
+    const int nqb = p->q_block > 0 ? p->seg_len / p->q_block : 0;
+    if (qblock_begin < 0 || qblock_end <= qblock_begin || qblock_end > nqb) return HGA_ERR_INVALID_ARG;
+    hga_status_t st = check_tiered(p, host_k, host_v, idx, stage_k, stage_v, stage_slots, scratch, idx_remapped,
+                                   qblock_end - qblock_begin);
+    if (st != HGA_OK) return st;
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
     st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, qblock_begin, qblock_end, stage_k, stage_v, stage_slots,
-                                  slot_map, idx_remapped, n_fetched, status, copy_stream);
+                                  scratch, idx_remapped, n_fetched, status, copy_stream);
     if (st != HGA_OK) return st;
     if (done) return hga::record_cuda(cudaEventRecord(done, copy_stream));
     return HGA_OK;
 }
 
+hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const void *v_seg, void *host_k,
+                              void *host_v, long long dst_token, cudaStream_t stream) {
+    CallRange range("hga_tier_offload");
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (!k_seg || !v_seg || !host_k || !host_v || dst_token < 0 || p->hist_head_stride < 1 ||
+        dst_token + p->seg_len > p->hist_head_stride)
+        return HGA_ERR_INVALID_ARG;
+    for (void *hp : {host_k, host_v}) {
+        cudaPointerAttributes at;
+        if (cudaPointerGetAttributes(&at, hp) != cudaSuccess || at.type != cudaMemoryTypeHost) {
+            cudaGetLastError();
+            hga::record_error("hga_tier_offload: host_k / host_v must be page-locked host memory");
+            return HGA_ERR_INVALID_ARG;
+        }
+    }
+    const size_t esize = p->dtype == HGA_BF16 ? 2 : 4;
+    const size_t row = (size_t)p->head_dim * esize;
+    const size_t width = (size_t)p->seg_len * row;
+    const size_t rows = (size_t)p->batch * p->n_kv_heads;
+    const size_t spitch = (size_t)p->seg_head_stride * row, dpitch = (size_t)p->hist_head_stride * row;
+    for (int kv = 0; kv < 2; ++kv) {
+        const void *src = kv ? v_seg : k_seg;
+        uint8_t *dst = static_cast<uint8_t *>(kv ? host_v : host_k) + (size_t)dst_token * row;
+        const cudaError_t e = cudaMemcpy2DAsync(dst, dpitch, src, spitch, width, rows, cudaMemcpyDeviceToHost, stream);
+        if (e != cudaSuccess) return hga::record_cuda(e);
+    }
+    return HGA_OK;
+}
+
+hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const void *host_k, const void *host_v,
+                                 const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
+                                 void *stage_k, void *stage_v, int stage_slots, int32_t *scratch,
+                                 int32_t *idx_remapped, int wave_blocks, int reset_cache, int32_t *n_fetched,
+                                 cudaStream_t stream, cudaStream_t copy_stream, const cudaEvent_t *events) {
+    CallRange range("hga_attn_fwd_tiered");
+    if (!p || wave_blocks < 1 || !events) return HGA_ERR_INVALID_ARG;
+    for (int e = 0; e < 5; ++e)
+        if (!events[e]) return HGA_ERR_INVALID_ARG;
+    const int nqb = p->q_block > 0 ? p->seg_len / p->q_block : 0;
+    const int qb0 = (p->qblock_begin == 0 && p->qblock_end == 0) ? 0 : p->qblock_begin;
+    const int qb1 = (p->qblock_begin == 0 && p->qblock_end == 0) ? nqb : p->qblock_end;
+    hga_status_t st = check_tiered(p, host_k, host_v, idx, stage_k, stage_v, stage_slots, scratch, idx_remapped,
+                                   wave_blocks);
+    if (st != HGA_OK) return st;
+    if (!q || !k_seg || !v_seg || !out || !lse) return HGA_ERR_INVALID_ARG;
+    hga_params_t pa = *p;  // attention over the staging cache: route indices are slots
+    pa.hist_head_stride = 0;
+    pa.n_hist_chunks = stage_slots;
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    // the copy stream starts after everything already on the compute stream
+    // (the route that wrote idx, the attention of earlier calls over the cache)
+    cudaError_t e = cudaEventRecord(events[0], stream);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(copy_stream, events[0], 0);
+    if (e != cudaSuccess) return hga::record_cuda(e);
+    if (reset_cache) {
+        st = hga::launch_tier_reset(*p, stage_slots, scratch, copy_stream);
+        if (st != HGA_OK) return st;
+    }
+    if (p->n_hist_chunks == 0)  // nothing routable: plain attention over the segment
+        return hga_attn_fwd(p, q, stage_k, stage_v, k_seg, v_seg, idx, out, lse, stream);
+    for (int w = 0, b0 = qb0; b0 < qb1; ++w, b0 += wave_blocks) {
+        const int b1 = b0 + wave_blocks < qb1 ? b0 + wave_blocks : qb1;
+        cudaEvent_t fetched = events[1 + (w & 1)], consumed = events[3 + (w & 1)];
+        // the fetch of wave w may evict slots last read by wave w - 2: wait for that attention
+        if (w >= 2 && (e = cudaStreamWaitEvent(copy_stream, consumed, 0)) != cudaSuccess) return hga::record_cuda(e);
+        st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, b0, b1, stage_k, stage_v, stage_slots, scratch,
+                                      idx_remapped, n_fetched ? n_fetched + w : nullptr, status, copy_stream);
+        if (st != HGA_OK) return st;
+        if ((e = cudaEventRecord(fetched, copy_stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(stream, fetched, 0)) != cudaSuccess)
+            return hga::record_cuda(e);
+        pa.qblock_begin = b0;
+        pa.qblock_end = b1;
+        st = hga_attn_fwd(&pa, q, stage_k, stage_v, k_seg, v_seg, idx_remapped, out, lse, stream);
+        if (st != HGA_OK) return st;
+        if ((e = cudaEventRecord(consumed, stream)) != cudaSuccess) return hga::record_cuda(e);
+    }
+    return HGA_OK;
+}
+
 hga_status_t hga_selftest_wait_timeout(long long wait_cycles, cudaStream_t stream) {
+    CallRange range("hga_selftest_wait_timeout");
     if (wait_cycles < 1000 || wait_cycles > (1ll << 32)) return HGA_ERR_INVALID_ARG;
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);

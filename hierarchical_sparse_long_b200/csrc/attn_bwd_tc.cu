@@ -11,8 +11,9 @@
 //   dK_seg = dS^T Q / sqrt(D), dV_seg = P^T dO   over segment keys only
 //
 // Two block types in one launch, no atomics (results are deterministic):
-//   dQ blocks  : query-major, one CTA per (batch, kv head, query block) holding
-//                the G heads of the group as M=128 halves (like the forward);
+//   dQ blocks  : query-major, one CTA per (batch, kv head, query block, head
+//                sub-group) holding HC heads of the group (4, 2 or 1, as in the
+//                forward) as M=128 halves;
 //                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128), the
 //                dS rows in bf16 into shared memory, dQ += dS K (M128 N128 K64).
 //   dK/dV blocks: key-major over the active segment, one CTA per (batch, kv
@@ -26,6 +27,12 @@
 // thread.
 // Every wait is bounded and every warp-collective TMEM access is made from a
 // converged warp with warp-uniform decisions.
+//
+// The dQ blocks take the same three kinds of routes as the forward (template
+// MODE): whole routed chunks, routed groups of gs tokens (gs-row TMA boxes,
+// the unfilled slots of the last tile repeating a loaded group with their
+// columns masked), or the union of per-token routes with a token mask per
+// chunk.  A masked key gets P = 0, so it adds nothing to dQ.
 #include <cudaTypedefs.h>
 
 #include "tc_ptx.cuh"
@@ -41,9 +48,14 @@ constexpr uint32_t TILE_BYTES = TILE * D * 2;   // 16 KiB: [2 col halves][64 row
 constexpr uint32_t ROWS128_K64 = 128 * TILE * 2; // 16 KiB: [128 rows][128 B] bf16, K = 64
 constexpr uint32_t IDESC_N64 = tc::idesc_bf16(128, TILE, false, false);
 constexpr uint32_t IDESC_N128_BMN = tc::idesc_bf16(128, D, false, true);
+constexpr int kChunk = 0, kGroup = 1, kMasked = 2;
 
 struct BwdArgs {
     int batch, n_q_heads, n_kv_heads, seg_len, topk, n_hist_chunks;
+    int gs;                           // kGroup: tokens per group
+    const int32_t *ucount;            // kMasked: valid routes per block
+    const unsigned long long *umask;  // kMasked: token mask per route
+    int n_sub, hc;  // dQ CTAs per KV group, query heads per dQ CTA (4, 2 or 1)
     long long hist_stride, seg_stride;
     const int32_t *idx;
     const float *lse;
@@ -88,11 +100,12 @@ struct DqBars {
     uint32_t tmem_base;
     int abort;
     int n_hist;
+    int n_groups;  // kGroup: valid routed groups of the block
     int issued;
     int tiles[64];
 };
 
-template <int NH>
+template <int NH, int MODE>
 __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_q,
                                         const CUtensorMap &tm_do, const CUtensorMap &tm_kh, const CUtensorMap &tm_vh,
                                         const CUtensorMap &tm_ks, const CUtensorMap &tm_vs, const BwdArgs &a) {
@@ -102,12 +115,13 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
     DqBars *bars = reinterpret_cast<DqBars *>(smem + L::BAR);
     const uint32_t sbase = tc::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = 2 * NH;
     const int nqb = a.seg_len / TILE;
-    const int n_bg = a.batch * a.n_kv_heads;
-    const int m = nqb - 1 - blk / n_bg;
-    const int bg = blk % n_bg;
+    const int n_units = a.batch * a.n_kv_heads * a.n_sub;
+    const int m = nqb - 1 - blk / n_units;
+    const int unit = blk % n_units;
+    const int bg = unit / a.n_sub;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+    const int h0 = g * (a.n_q_heads / a.n_kv_heads) + (unit % a.n_sub) * a.hc;  // first query head of the CTA
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->q_full, 1);
@@ -127,12 +141,24 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         bars->issued = 0;
         tc::fence_mbar_init();
     }
+    const long long bgm = (long long)bg * nqb + m;
     if (warp == 2 && lane == 0) {
-        const int32_t *sel = a.idx + ((long long)bg * nqb + m) * a.topk;
+        const int32_t *sel = a.idx + bgm * a.topk;
         int n = 0;
-        for (int i = 0; i < a.topk; ++i) {
-            const int j = sel[i];
-            if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
+        if constexpr (MODE == kChunk) {
+            for (int i = 0; i < a.topk; ++i) {
+                const int j = sel[i];
+                if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
+            }
+        } else if constexpr (MODE == kGroup) {
+            const int n_all = a.n_hist_chunks * (TILE / a.gs);
+            int ng = 0;
+            for (int i = 0; i < a.topk; ++i) ng += (sel[i] >= 0 && sel[i] < n_all) ? 1 : 0;
+            bars->n_groups = ng;
+            n = (ng * a.gs + TILE - 1) / TILE;
+        } else {
+            const int cnt = a.ucount[bgm];
+            n = cnt < 0 ? 0 : (cnt > a.topk ? a.topk : cnt);
         }
         bars->n_hist = n;
     }
@@ -148,8 +174,8 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
     if (warp == 0) {
         if (lane == 0) {
             tc::mbar_arrive_expect_tx(&bars->q_full, 2 * NH * HALF_BYTES);
-            for (int hh = 0; hh < G; ++hh) {
-                const int qrow = (b * a.n_q_heads + g * G + hh) * a.seg_len + m * TILE;
+            for (int hh = 0; hh < 2 * NH; ++hh) {
+                const int qrow = (b * a.n_q_heads + h0 + (a.hc == 1 ? 0 : hh)) * a.seg_len + m * TILE;
                 const uint32_t off = (hh >> 1) * HALF_BYTES + (hh & 1) * (64 * 128);
                 tc::tma_load_2d(smem + L::Q + off, &tm_q, 0, qrow, &bars->q_full);
                 tc::tma_load_2d(smem + L::Q + off + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
@@ -157,21 +183,47 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                 tc::tma_load_2d(smem + L::DO + off + 128 * 128, &tm_do, 64, qrow, &bars->q_full);
             }
             int issued = 0;
+            // kGroup: the routed groups in list order (invalid entries skipped), 64 / gs per tile
+            const int32_t *gsel = a.idx + bgm * a.topk;
+            const int n_all = MODE == kGroup ? a.n_hist_chunks * (TILE / a.gs) : 0;
+            const int n_groups = MODE == kGroup ? bars->n_groups : 0;
+            int gcur = 0, gtaken = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int s = j % NST, u = j / NST;
                 if (j >= NST && !tc::mbar_wait(&bars->kv_empty[s], (u - 1) & 1, abort, a.status)) break;
-                const bool hist = j < n_hist;
-                const CUtensorMap *mk = hist ? &tm_kh : &tm_ks;
-                const CUtensorMap *mv = hist ? &tm_vh : &tm_vs;
-                const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
-                                     : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
                 uint8_t *kdst = smem + L::KV + s * 2 * TILE_BYTES;
                 uint8_t *vdst = kdst + TILE_BYTES;
                 tc::mbar_arrive_expect_tx(&bars->kv_full[s], 2 * TILE_BYTES);
-                tc::tma_load_2d(kdst, mk, 0, row, &bars->kv_full[s]);
-                tc::tma_load_2d(kdst + 64 * 128, mk, 64, row, &bars->kv_full[s]);
-                tc::tma_load_2d(vdst, mv, 0, row, &bars->kv_full[s]);
-                tc::tma_load_2d(vdst + 64 * 128, mv, 64, row, &bars->kv_full[s]);
+                if (j < n_hist && MODE == kGroup) {
+                    const int gpt = TILE / a.gs;
+                    int first = 0;
+                    for (int v = 0; v < gpt; ++v) {
+                        int grp = first;  // unfilled slots repeat the tile's first group
+                        if (gtaken < n_groups) {
+                            while (!(gsel[gcur] >= 0 && gsel[gcur] < n_all)) ++gcur;
+                            grp = gsel[gcur++];
+                            ++gtaken;
+                        }
+                        if (v == 0) first = grp;
+                        const int row = (int)((long long)bg * a.hist_stride + (long long)grp * a.gs);
+                        tc::tma_load_2d(kdst + v * a.gs * 128, &tm_kh, 0, row, &bars->kv_full[s]);
+                        tc::tma_load_2d(kdst + 64 * 128 + v * a.gs * 128, &tm_kh, 64, row, &bars->kv_full[s]);
+                        tc::tma_load_2d(vdst + v * a.gs * 128, &tm_vh, 0, row, &bars->kv_full[s]);
+                        tc::tma_load_2d(vdst + 64 * 128 + v * a.gs * 128, &tm_vh, 64, row, &bars->kv_full[s]);
+                    }
+                } else {
+                    const bool hist = j < n_hist;
+                    const CUtensorMap *mk = hist ? &tm_kh : &tm_ks;
+                    const CUtensorMap *mv = hist ? &tm_vh : &tm_vs;
+                    int chunk = 0;
+                    if (hist) chunk = MODE == kChunk ? bars->tiles[j] : a.idx[bgm * a.topk + j];
+                    const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)chunk * TILE)
+                                         : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+                    tc::tma_load_2d(kdst, mk, 0, row, &bars->kv_full[s]);
+                    tc::tma_load_2d(kdst + 64 * 128, mk, 64, row, &bars->kv_full[s]);
+                    tc::tma_load_2d(vdst, mv, 0, row, &bars->kv_full[s]);
+                    tc::tma_load_2d(vdst + 64 * 128, mv, 64, row, &bars->kv_full[s]);
+                }
                 ++issued;
             }
             bars->issued = issued;
@@ -225,13 +277,30 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         const int r = quad * 32 + lane;
         const int hh = 2 * h + (r >> 6);
         const int i = r & 63;
+        const bool write = hh < a.hc;  // rows 64..127 repeat the head when HC = 1
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        const long long row = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + m * TILE + i;
+        const long long row = ((long long)(b * a.n_q_heads + h0 + (write ? hh : 0))) * a.seg_len + m * TILE + i;
         const float lse2 = a.lse[row] * 1.4426950408889634f;
         const float dlt = a.delta[row];
         const uint32_t ds_row = sbase + L::DS + h * ROWS128_K64 + (r >> 3) * 1024 + (r & 7) * 128;
+        // kGroup: valid columns of the last history tile; kMasked: the row's token bit of
+        // the next tile's mask (read one tile ahead)
+        const int last_cols = MODE == kGroup ? bars->n_groups * a.gs - (n_hist - 1) * TILE : TILE;
+        unsigned long long mask_next = 0ull;
+        if (MODE == kMasked && n_hist > 0) mask_next = a.umask[bgm * a.topk];
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
+            // columns >= ncols of this tile are masked for this row
+            int ncols = TILE;
+            if constexpr (MODE == kGroup) {
+                if (j == n_hist - 1) ncols = last_cols;
+            }
+            if constexpr (MODE == kMasked) {
+                if (j < n_hist) {
+                    if (((mask_next >> i) & 1ull) == 0ull) ncols = 0;
+                    if (j + 1 < n_hist) mask_next = a.umask[bgm * a.topk + j + 1];
+                }
+            }
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[h], j & 1, abort, a.status))) {
                 ok = false;
                 break;
@@ -251,8 +320,8 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                     const int c0 = 32 * half + c;
                     float p0 = tc::ex2(__uint_as_float(sv[c]) * a.scale_log2 - lse2);
                     float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2);
-                    if (diag && c0 > i) p0 = 0.f;
-                    if (diag && c0 + 1 > i) p1 = 0.f;
+                    if ((diag && c0 > i) || c0 >= ncols) p0 = 0.f;
+                    if ((diag && c0 + 1 > i) || c0 + 1 >= ncols) p1 = 0.f;
                     pk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt),
                                                           p1 * (__uint_as_float(dpv[c + 1]) - dlt));
                 }
@@ -278,6 +347,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                 uint32_t o[32];
                 tc::tmem_ld32(tmem + lane_addr + 128 * h + c0, o);
                 tc::tmem_wait_ld();
+                if (!write) continue;
 #pragma unroll
                 for (int c = 0; c < 32; c += 4)
                     *reinterpret_cast<float4 *>(out + c0 + c) =
@@ -581,7 +651,7 @@ bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
 // key-major dK/dV body (most work first), the rest the query-major dQ body.
 // The causal dK/dV blocks are very uneven (the first key tile is seen by
 // every later query tile), so the dQ blocks fill the SMs around them.
-template <int NH>
+template <int NH, int MODE>
 __global__ void __launch_bounds__(128 + 128 * NH, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
@@ -591,20 +661,20 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
     if ((int)blockIdx.x < n_kv_ctas)
         dkdv_body((int)blockIdx.x, smem_raw, tm_q, tm_do, tm_ks, tm_vs, a);
     else
-        dq_body<NH>((int)blockIdx.x - n_kv_ctas, smem_raw, tm_q, tm_do, tm_kh, tm_vh, tm_ks, tm_vs, a);
+        dq_body<NH, MODE>((int)blockIdx.x - n_kv_ctas, smem_raw, tm_q, tm_do, tm_kh, tm_vh, tm_ks, tm_vs, a);
 }
 
-template <int NH>
+template <int NH, int MODE>
 hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUtensorMap &mdo,
                         const CUtensorMap &mkh, const CUtensorMap &mvh, const CUtensorMap &mks,
                         const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
-    auto kern = bwd_tc_kernel<NH>;
+    auto kern = bwd_tc_kernel<NH, MODE>;
     const size_t smem = DqSmem<NH>::ALLOC > DkvSmem::ALLOC ? DqSmem<NH>::ALLOC : DkvSmem::ALLOC;
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const int n_bg = p.batch * p.n_kv_heads;
     const int n_kv_ctas = ((p.seg_len + 127) / 128) * n_bg;
-    const unsigned grid = (unsigned)(n_kv_ctas + (p.seg_len / p.q_block) * n_bg);
+    const unsigned grid = (unsigned)(n_kv_ctas + (p.seg_len / p.q_block) * n_bg * a.n_sub);
     kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mdo, mkh, mvh, mks, mvs, a, n_kv_ctas);
     return record_cuda(cudaGetLastError());
 }
@@ -612,9 +682,7 @@ hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUte
 }  // namespace
 
 bool attn_bwd_tc_supported(const hga_params_t &p) {
-    const int G = p.n_q_heads / p.n_kv_heads;
-    if (p.dtype != HGA_BF16 || p.head_dim != 128 || p.chunk != 64 || p.q_block != 64) return false;
-    if (G != 2 && G != 4) return false;
+    if (!attn_fwd_tc_shape(p)) return false;
     const long long n_bg = (long long)p.batch * p.n_kv_heads;
     if (n_bg * (p.hist_head_stride > p.seg_head_stride ? p.hist_head_stride : p.seg_head_stride) >= (1ll << 31))
         return false;
@@ -622,10 +690,13 @@ bool attn_bwd_tc_supported(const hga_params_t &p) {
     return tma_encoder_available();
 }
 
-hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,
-                                const void *ks, const void *vs, const int32_t *idx, const float *lse,
-                                const float *delta, const void *dout, float *dq, float *dk, float *dv,
-                                unsigned *status, cudaStream_t stream) {
+namespace {
+
+template <int MODE>
+hga_status_t launch_bwd_mode(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
+                             const void *vs, const FwdRoutes &rt, const float *lse, const float *delta,
+                             const void *dout, float *dq, float *dk, float *dv, unsigned *status,
+                             cudaStream_t stream) {
     CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
     const long long n_bg = (long long)p.batch * p.n_kv_heads;
     const unsigned long long q_rows = (unsigned long long)p.batch * p.n_q_heads * p.seg_len;
@@ -637,7 +708,9 @@ hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void
         !make_map(&mvs, vs, seg_rows))
         return HGA_ERR_INVALID_ARG;
     if (hist_rows > 0) {
-        if (!make_map(&mkh, kh, (unsigned long long)hist_rows) || !make_map(&mvh, vh, (unsigned long long)hist_rows))
+        const unsigned box = MODE == kGroup ? (unsigned)rt.gs : 64u;  // group routes: one box per group
+        if (!tma_rows_map(&mkh, kh, (unsigned long long)hist_rows, box) ||
+            !tma_rows_map(&mvh, vh, (unsigned long long)hist_rows, box))
             return HGA_ERR_INVALID_ARG;
     } else {
         mkh = mks;
@@ -648,11 +721,14 @@ hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void
     a.n_q_heads = p.n_q_heads;
     a.n_kv_heads = p.n_kv_heads;
     a.seg_len = p.seg_len;
-    a.topk = p.topk;
+    a.topk = rt.per_block;
     a.n_hist_chunks = p.n_hist_chunks;
+    a.gs = rt.gs;
+    a.ucount = rt.ucount;
+    a.umask = rt.umask;
     a.hist_stride = p.hist_head_stride;
     a.seg_stride = p.seg_head_stride;
-    a.idx = idx;
+    a.idx = rt.list;
     a.lse = lse;
     a.delta = delta;
     a.dq = dq;
@@ -662,8 +738,31 @@ hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void
     a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
     a.scale = (float)(1.0 / __builtin_sqrt((double)D));
     const int G = p.n_q_heads / p.n_kv_heads;
-    return G == 4 ? launch_bwd<2>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream)
-                  : launch_bwd<1>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream);
+    a.hc = G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1);
+    a.n_sub = G / a.hc;
+    return G % 4 == 0 ? launch_bwd<2, MODE>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream)
+                      : launch_bwd<1, MODE>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream);
+}
+
+}  // namespace
+
+hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,
+                                const void *ks, const void *vs, const int32_t *idx, const float *lse,
+                                const float *delta, const void *dout, float *dq, float *dk, float *dv,
+                                unsigned *status, cudaStream_t stream) {
+    FwdRoutes rt{idx, p.topk, 0, nullptr, nullptr};
+    return launch_bwd_mode<kChunk>(p, q, kh, vh, ks, vs, rt, lse, delta, dout, dq, dk, dv, status, stream);
+}
+
+hga_status_t launch_attn_bwd_tc_routes(const hga_params_t &p, const void *q, const void *kh, const void *vh,
+                                       const void *ks, const void *vs, const FwdRoutes &rt, const float *lse,
+                                       const float *delta, const void *dout, float *dq, float *dk, float *dv,
+                                       unsigned *status, cudaStream_t stream) {
+    if (rt.gs > 0)
+        return launch_bwd_mode<kGroup>(p, q, kh, vh, ks, vs, rt, lse, delta, dout, dq, dk, dv, status, stream);
+    if (rt.umask)
+        return launch_bwd_mode<kMasked>(p, q, kh, vh, ks, vs, rt, lse, delta, dout, dq, dk, dv, status, stream);
+    return launch_bwd_mode<kChunk>(p, q, kh, vh, ks, vs, rt, lse, delta, dout, dq, dk, dv, status, stream);
 }
 
 }  // namespace hga

@@ -6,15 +6,18 @@
 // route only) and the author abstract (a bounded set of exact historical
 // tokens per query block).
 //
-// One CTA per (batch, kv head, query block).  The G query heads of the KV
-// group share every K/V tile, so the CTA holds all G*64 query rows as NH
-// M=128 halves (NH = G/2): each 64-token key tile (a routed history chunk,
-// then the active segment's causal tiles 0..m) is read once for G heads,
-// which is what lifts a history tile from 64 to 256 flop/byte.
+// One CTA per (batch, kv head, query block, head sub-group).  The query heads
+// of a KV group share every K/V tile, so a CTA holds HC of them (HC = 4 when
+// G % 4 == 0, else 2 when G is even, else 1) as NH M=128 halves of 64-row
+// head pairs: each 64-token key tile (a routed history chunk, then the active
+// segment's causal tiles 0..m) is read once for HC heads, which lifts a
+// history tile from 64 to 256 flop/byte at HC = 4.  G / HC CTAs share one KV
+// group (its tiles then come from L2).  With HC = 1 the second 64 rows of the
+// M=128 half repeat the head's rows and are not written back.
 //
-// Warp roles (NH = 2: 512 threads, warps 5-7 idle):
+// Warp roles (NH = 2: 672 threads):
 //   warp 0      TMA producer: Q once, then K and V of every tile, each into
-//               its own 5-stage ring (routed chunk j -> TMA row coordinate
+//               its own 4-stage ring (routed chunk j -> TMA row coordinate
 //               (b*Hkv+g)*stride + 64 j); a K stage is released as soon as
 //               QK^T of its tile completes, a V stage after PV.
 //   warps 1, 3  QK issuers, one thread per M half (warp 1 also owns TMEM):
@@ -26,14 +29,33 @@
 //               issued as soon as the softmax has written P.  One thread
 //               issues a tcgen05.mma only about every 100 cycles, so the four
 //               issue streams run in separate threads.
-//   warps 8+4h  softmax of half h: one TMEM lane (= query row) per thread;
-//               online softmax in the log2 domain, O rescaled in TMEM when
-//               the row max grows by more than 2^8, P written as bf16 pairs
-//               into the tile's S buffer, where the PV issue reads it.
+//   warps 5+8h+4c.. softmax of half h, columns 32c..32c+31 of every score
+//               tile: two threads per query row (TMEM lane), one per column
+//               half, exchanging the tile's row max through shared memory
+//               (an mbarrier per row quadrant); online softmax in the log2
+//               domain, O rescaled in TMEM (columns 64c..64c+63) when the row
+//               max grows by more than 2^8, P written as bf16 pairs into the
+//               tile's S buffer, where the PV issue reads it.  Two threads per
+//               row halve the serial per-tile chain of a thread (TMEM load,
+//               max, exponentials, sum, P store) and give each SM sub-partition
+//               four softmax warps to interleave on the exponential unit.
 // TMEM (512 columns): O_h at 128h, S_h double-buffered at 256 + 128h + 64b.
 // Every wait is bounded; a timeout sets HGA_DEV_TIMEOUT and the CTA unwinds.
+//
+// Three kinds of routes fill the history tiles (template MODE):
+//   kChunk   a block's routed 64-token chunks, one tile each (hga_attn_fwd);
+//   kGroup   a block's routed groups of gs = 8, 16 or 32 tokens (the group
+//            stage of the technical summary, section 2.1), packed 64 / gs to a
+//            tile, one TMA box of gs rows per group -- each box lands as whole
+//            128-byte swizzle atoms, so the MMA descriptors are unchanged; the
+//            unfilled slots of a block's last tile repeat a loaded group and
+//            their columns are masked;
+//   kMasked  the union of the per-token routes of a block's 64 tokens (the
+//            strictly causal variant of the technical summary's limits
+//            section), one tile per chunk of the union with a 64-bit mask of
+//            the block's tokens that route to it: rows whose bit is clear
+//            see the whole tile as masked.
 #include <cudaTypedefs.h>
-#include <cstdlib>
 
 #include "tc_ptx.cuh"
 
@@ -43,19 +65,23 @@ namespace {
 
 constexpr int D = 128;
 constexpr int TILE = 64;
-constexpr int NSTAGE = 5;
+constexpr int NSTAGE = 4;
 constexpr float kRescaleLog2 = 8.f;  // lazy-rescale threshold on the running max (log2 units)
 constexpr uint32_t Q_HALF_BYTES = 128 * D * 2;   // 32 KiB: [2 col halves][128 rows][128 B]
 constexpr uint32_t KV_TILE_BYTES = TILE * D * 2; // 16 KiB: [2 col halves][64 rows][128 B]
 constexpr uint32_t IDESC_QK = tc::idesc_bf16(128, TILE, false, false);
 constexpr uint32_t IDESC_PV = tc::idesc_bf16(128, D, false, true);
+constexpr int kChunk = 0, kGroup = 1, kMasked = 2;
+constexpr int kMaxGroups = 512;  // routed groups per block (k <= 64 chunks x 8 groups)
 
 template <int NH>
 struct Smem {
     static constexpr uint32_t Q = 0;
     static constexpr uint32_t K = Q + NH * Q_HALF_BYTES;      // K ring
     static constexpr uint32_t V = K + NSTAGE * KV_TILE_BYTES; // V ring
-    static constexpr uint32_t BAR = V + NSTAGE * KV_TILE_BYTES;
+    static constexpr uint32_t RED = V + NSTAGE * KV_TILE_BYTES;  // row max / sum exchange [2][2][128][2] fp32
+    static constexpr uint32_t GLIST = RED + 2 * 2 * 128 * 2 * 4;  // routed group ids (kGroup)
+    static constexpr uint32_t BAR = GLIST + kMaxGroups * 4;
     static constexpr uint32_t TOTAL = BAR + 1024;  // barriers, tile list, flags
     static constexpr uint32_t ALLOC = TOTAL + 1024; // + alignment slack
 };
@@ -80,6 +106,7 @@ struct Bars {
     uint64_t s_full[2][2];  // [half][S/P buffer]: S of the buffer's tile in TMEM
     uint64_t p_full[2][2];  // [half][S/P buffer]: P of the buffer's tile written to TMEM
     uint64_t o_done[2][2];  // [half][S/P buffer]: PV of the buffer's tile completed
+    uint64_t xchg[2][2][4]; // [parity][half][row quadrant]: both column halves posted their row values
     uint64_t drain[4];      // one per issuing thread (abort path)
     uint32_t tmem_base;
     int abort;
@@ -87,11 +114,20 @@ struct Bars {
     int issued_k;  // K / V tiles the producer issued
     int issued_v;
     int sm0_tiles;  // tiles whose softmax half 0 has finished (scheduling hint)
+    int n_groups;   // kGroup: routed groups of this block
     int tiles[64];
 };
 
+static_assert(sizeof(Bars) <= 1024, "barrier block must fit its region");
+
 struct FwdArgs {
     int batch, n_q_heads, n_kv_heads, seg_len, topk, n_hist_chunks;
+    // kGroup: tokens per group; kMasked: routes per block in idx (the union capacity),
+    // their count and the per-route token masks
+    int gs;
+    const int32_t *ucount;
+    const unsigned long long *umask;
+    int n_sub, hc;  // CTAs per KV group, query heads per CTA (4, 2 or 1)
     long long hist_stride, seg_stride;
     int qb0, n_blocks;
     const int32_t *idx;
@@ -101,10 +137,10 @@ struct FwdArgs {
     float scale_log2;  // log2(e) / sqrt(D)
 };
 
-// Two control warpgroups (producer, QK0, PV0, QK1, PV1, three idle warps) and
-// NH softmax warpgroups.  With NH = 2 the 512 threads launch at 128 registers
-// each; the control warpgroups give registers back and the softmax
-// warpgroups take them: 8 x 32 x 56 + 8 x 32 x 200 = 65,536, the launch total.
+// Five control warps (producer, QK0, PV0, QK1, PV1) and 8 NH softmax warps;
+// a softmax warp reads the TMEM lane quadrant (warp index % 4), so any four
+// consecutive softmax warps cover the 128 rows of a half.  With NH = 2 the
+// 672 threads launch at 96 registers each (64,512 of the SM's 65,536).
 // Bounded wait until the shared counter reaches `target` (same contract as mbar_wait).
 __device__ __forceinline__ bool wait_count(int *counter, int target, volatile int *abort, unsigned *status) {
     volatile int *c = counter;
@@ -121,13 +157,10 @@ __device__ __forceinline__ bool wait_count(int *counter, int target, volatile in
     return true;
 }
 
-constexpr int kCtrlWarps = 8;
-constexpr int kCtrlRegs = 56;
-constexpr int kSoftmaxRegs = 200;
-static_assert(8 * 32 * kCtrlRegs + 8 * 32 * kSoftmaxRegs == 512 * 128, "register split must match the launch");
+constexpr int kCtrlWarps = 5;
 
-template <int NH, int POLY>
-__global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
+template <int NH, int MODE>
+__global__ void __launch_bounds__(32 * kCtrlWarps + 256 * NH, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                        const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
                        const __grid_constant__ CUtensorMap tm_vs, const FwdArgs a) {
@@ -138,12 +171,14 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     const uint32_t sbase = tc::smem_u32(smem);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int G = 2 * NH;
     const int nqb = a.seg_len / TILE;
-    const int n_bg = a.batch * a.n_kv_heads;
-    const int m = a.qb0 + a.n_blocks - 1 - (int)blockIdx.x / n_bg;  // longest (latest) blocks first
-    const int bg = (int)blockIdx.x % n_bg;
+    const int n_units = a.batch * a.n_kv_heads * a.n_sub;
+    const int m = a.qb0 + a.n_blocks - 1 - (int)blockIdx.x / n_units;  // longest (latest) blocks first
+    const int unit = (int)blockIdx.x % n_units;
+    const int bg = unit / a.n_sub;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
+    // first query head of this CTA: the KV group's heads g*G .., HC per CTA
+    const int h0 = g * (a.n_q_heads / a.n_kv_heads) + (unit % a.n_sub) * a.hc;
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->q_full, 1);
@@ -156,8 +191,9 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
         for (int h = 0; h < 2; ++h)
             for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->s_full[h][bb], 1);
-                tc::mbar_init(&bars->p_full[h][bb], 4);
+                tc::mbar_init(&bars->p_full[h][bb], 8);  // every softmax warp of the half
                 tc::mbar_init(&bars->o_done[h][bb], 1);
+                for (int qd = 0; qd < 4; ++qd) tc::mbar_init(&bars->xchg[bb][h][qd], 2);
             }
         for (int d = 0; d < 4; ++d) tc::mbar_init(&bars->drain[d], 1);
         bars->issued_k = 0;
@@ -166,14 +202,32 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
         bars->abort = 0;
         tc::fence_mbar_init();
     }
+    int *glist = reinterpret_cast<int *>(smem + L::GLIST);
+    const long long bgm = (long long)bg * nqb + m;
     if (warp == 2 && lane == 0) {
-        // routed history chunks of this block; -1 is padding, anything else out of range is skipped
-        const int32_t *sel = a.idx + ((long long)bg * nqb + m) * a.topk;
+        const int32_t *sel = a.idx + bgm * a.topk;
         int n = 0;
-        for (int i = 0; i < a.topk; ++i) {
-            const int j = sel[i];
-            if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
-            else if (j != -1) atomicOr(a.status, kDevBadIndex);
+        if constexpr (MODE == kChunk) {
+            // routed history chunks of this block; -1 is padding, anything else out of range is skipped
+            for (int i = 0; i < a.topk; ++i) {
+                const int j = sel[i];
+                if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
+                else if (j != -1) atomicOr(a.status, kDevBadIndex);
+            }
+        } else if constexpr (MODE == kGroup) {
+            const int n_groups = a.n_hist_chunks * (TILE / a.gs);
+            int ng = 0;
+            for (int i = 0; i < a.topk && ng < kMaxGroups; ++i) {
+                const int u = sel[i];
+                if (u >= 0 && u < n_groups) glist[ng++] = u;
+                else if (u != -1) atomicOr(a.status, kDevBadIndex);
+            }
+            bars->n_groups = ng;
+            n = (ng * a.gs + TILE - 1) / TILE;
+        } else {
+            // the union list was validated when it was built
+            const int cnt = a.ucount[bgm];
+            n = cnt < 0 ? 0 : (cnt > a.topk ? a.topk : cnt);
         }
         bars->n_hist = n;
     }
@@ -187,7 +241,6 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     volatile int *abort = &bars->abort;
 
     if (warp < kCtrlWarps) {
-        if constexpr (NH == 2) asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kCtrlRegs));
     if (warp == 0) {
         if (lane == 0) {
             // ------------------------------------------------------------ TMA producer
@@ -197,31 +250,48 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
             tc::tma_prefetch_desc(&tm_vh);
             tc::tma_prefetch_desc(&tm_vs);
             tc::mbar_arrive_expect_tx(&bars->q_full, NH * Q_HALF_BYTES);
-            for (int hh = 0; hh < G; ++hh) {
-                const int qrow = (b * a.n_q_heads + g * G + hh) * a.seg_len + m * TILE;
+            for (int hh = 0; hh < 2 * NH; ++hh) {
+                const int qrow = (b * a.n_q_heads + h0 + (a.hc == 1 ? 0 : hh)) * a.seg_len + m * TILE;
                 uint8_t *dst = smem + L::Q + (hh >> 1) * Q_HALF_BYTES + (hh & 1) * (64 * 128);
                 tc::tma_load_2d(dst, &tm_q, 0, qrow, &bars->q_full);
                 tc::tma_load_2d(dst + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
             }
             // K(j), then V(j): a K stage frees once QK^T(j - NSTAGE) completes, a V
             // stage once PV(j - NSTAGE) does; routed chunk j is row (b*Hkv+g)*stride + 64 j
+            // a tile as TMA boxes: one 64-row box per column half, or (kGroup history
+            // tiles) 64 / gs boxes of gs rows per column half, group slot u at row u*gs
+            const int n_groups = MODE == kGroup ? bars->n_groups : 0;
+            auto load_tile = [&](uint8_t *dst, const CUtensorMap *mh, const CUtensorMap *ms, int j, uint64_t *bar) {
+                if (j >= n_hist) {
+                    const int row = (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+                    tc::tma_load_2d(dst, ms, 0, row, bar);
+                    tc::tma_load_2d(dst + 64 * 128, ms, 64, row, bar);
+                } else if constexpr (MODE == kGroup) {
+                    const int gpt = TILE / a.gs;
+                    for (int u = 0; u < gpt; ++u) {
+                        const int at = j * gpt + u;
+                        const int grp = glist[at < n_groups ? at : j * gpt];  // unfilled slots repeat a group
+                        const int row = (int)((long long)bg * a.hist_stride + (long long)grp * a.gs);
+                        tc::tma_load_2d(dst + u * a.gs * 128, mh, 0, row, bar);
+                        tc::tma_load_2d(dst + 64 * 128 + u * a.gs * 128, mh, 64, row, bar);
+                    }
+                } else {
+                    const int chunk = MODE == kChunk ? bars->tiles[j] : a.idx[bgm * a.topk + j];
+                    const int row = (int)((long long)bg * a.hist_stride + (long long)chunk * TILE);
+                    tc::tma_load_2d(dst, mh, 0, row, bar);
+                    tc::tma_load_2d(dst + 64 * 128, mh, 64, row, bar);
+                }
+            };
             int nk = 0, nv = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int s = j % NSTAGE, u = j / NSTAGE;
-                const bool hist = j < n_hist;
-                const int row = hist ? (int)((long long)bg * a.hist_stride + (long long)bars->tiles[j] * TILE)
-                                     : (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
                 if (j >= NSTAGE && !tc::mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort, a.status)) break;
-                uint8_t *kdst = smem + L::K + s * KV_TILE_BYTES;
                 tc::mbar_arrive_expect_tx(&bars->k_full[s], KV_TILE_BYTES);
-                tc::tma_load_2d(kdst, hist ? &tm_kh : &tm_ks, 0, row, &bars->k_full[s]);
-                tc::tma_load_2d(kdst + 64 * 128, hist ? &tm_kh : &tm_ks, 64, row, &bars->k_full[s]);
+                load_tile(smem + L::K + s * KV_TILE_BYTES, &tm_kh, &tm_ks, j, &bars->k_full[s]);
                 nk = j + 1;
                 if (j >= NSTAGE && !tc::mbar_wait(&bars->v_empty[s], (u - 1) & 1, abort, a.status)) break;
-                uint8_t *vdst = smem + L::V + s * KV_TILE_BYTES;
                 tc::mbar_arrive_expect_tx(&bars->v_full[s], KV_TILE_BYTES);
-                tc::tma_load_2d(vdst, hist ? &tm_vh : &tm_vs, 0, row, &bars->v_full[s]);
-                tc::tma_load_2d(vdst + 64 * 128, hist ? &tm_vh : &tm_vs, 64, row, &bars->v_full[s]);
+                load_tile(smem + L::V + s * KV_TILE_BYTES, &tm_vh, &tm_vs, j, &bars->v_full[s]);
                 nv = j + 1;
             }
             bars->issued_k = nk;
@@ -284,72 +354,112 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     }
     } else {
         // -------------------------------------------------------------- softmax / epilogue
-        if constexpr (NH == 2) asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kSoftmaxRegs));
-        const int h = (warp - kCtrlWarps) >> 2;  // M half
-        const int quad = warp & 3;               // TMEM lane quadrant this warp may access
-        const int r = quad * 32 + lane;          // row within the half = TMEM lane
-        const int hh = 2 * h + (r >> 6);         // head within the group
-        const int i = r & 63;                    // query row within the block
+        const int sg = (warp - kCtrlWarps) >> 2;  // softmax warp group (four consecutive warps)
+        const int h = sg >> 1;                    // M half
+        const int c = sg & 1;                     // column half of the score tile
+        const int quad = warp & 3;                // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;           // row within the half = TMEM lane
+        const int hh = 2 * h + (r >> 6);          // head within the CTA
+        const int i = r & 63;                     // query row within the block
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        const uint32_t o_addr = tmem + lane_addr + 128 * h;
+        const uint32_t o_addr = tmem + lane_addr + 128 * h + 64 * c;
+        // this thread's and its partner's slots of the row exchange, per tile parity
+        float *red = reinterpret_cast<float *>(smem + L::RED);
+        auto red_at = [&](int par, int cc) -> float * { return red + ((par * 2 + h) * 128 + r) * 2 + cc; };
+        // posts v for the partner thread (other column half, same row) and returns
+        // the partner's value; bounded wait, the same result across the warp
+        auto exchange = [&](int t, float v, float &other) -> bool {
+            const int par = t & 1;
+            *red_at(par, c) = v;
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->xchg[par][h][quad]);
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->xchg[par][h][quad], (t >> 1) & 1, abort, a.status)))
+                return false;
+            other = *reinterpret_cast<volatile float *>(red_at(par, c ^ 1));
+            return true;
+        };
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
+        // kGroup: valid columns of the last history tile; kMasked: this row's bit of the
+        // next tile's token mask (read one tile ahead)
+        const int last_cols = MODE == kGroup ? bars->n_groups * a.gs - (n_hist - 1) * TILE : TILE;
+        unsigned long long mask_next = 0ull;
+        if (MODE == kMasked && n_hist > 0) mask_next = a.umask[bgm * a.topk];
         for (int j = 0; j < n_tiles; ++j) {
             const int bb = j & 1;
+            bool row_off = false;  // kMasked: the whole tile is masked for this row
+            if constexpr (MODE == kMasked) {
+                if (j < n_hist) {
+                    row_off = ((mask_next >> i) & 1ull) == 0ull;
+                    if (j + 1 < n_hist) mask_next = a.umask[bgm * a.topk + j + 1];
+                }
+            }
             // tcgen05.ld/st below are warp-collective: keep every decision warp-uniform
             if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->s_full[h][bb], (j >> 1) & 1, abort, a.status))) {
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
-            uint32_t sr[64];
+            float x[32];
             {
-                uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
-                uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
-                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * h + 64 * bb;
-                tc::tmem_ld32(s_addr, lo);
-                tc::tmem_ld32(s_addr + 32, hi);
+                uint32_t sr[32];
+                tc::tmem_ld32(tmem + lane_addr + 256 + 128 * h + 64 * bb + 32 * c, sr);
                 tc::tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(sr[e]);
             }
-            float x[64];
-            const bool diag = (j == n_tiles - 1);  // the local tile of this block (warp-uniform)
+            if (j == n_tiles - 1) {  // the local tile of this block (warp-uniform)
 #pragma unroll
-            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
-            if (diag) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c > i) x[c] = -INFINITY;
+                for (int e = 0; e < 32; ++e)
+                    if (32 * c + e > i) x[e] = -INFINITY;
             }
-            // row max of the raw scores (the scale is positive), 8 independent chains
-            float mpart[8];
+            if constexpr (MODE == kGroup) {
+                if (j == n_hist - 1 && last_cols < TILE) {  // repeated groups past the routed ones
 #pragma unroll
-            for (int c = 0; c < 64; ++c) mpart[c & 7] = (c < 8) ? x[c] : fmaxf(mpart[c & 7], x[c]);
-            const float mx = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
-                                   fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7]))) *
-                             a.scale_log2;
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * c + e >= last_cols) x[e] = -INFINITY;
+                }
+            }
+            if constexpr (MODE == kMasked) {
+                if (row_off) {
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) x[e] = -INFINITY;
+                }
+            }
+            // row max of the raw scores (the scale is positive), 4 independent chains
+            float mpart[4];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) mpart[e & 3] = (e < 4) ? x[e] : fmaxf(mpart[e & 3], x[e]);
+            float mx = fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])) * a.scale_log2;
+            // both column halves have loaded their scores once the exchange completes, so
+            // P may overwrite the first 32 columns of the S buffer after it
+            float mo;
+            if (!exchange(j, mx, mo)) {
+                ok = false;
+                break;
+            }
+            mx = fmaxf(mx, mo);
             // Lazy rescaling: the reference max only moves when the row max grows by
             // more than kRescaleLog2, so P stays <= 2^kRescaleLog2 and O is rescaled
-            // in TMEM only on those (rare) tiles.
+            // in TMEM only on those (rare) tiles.  Both threads of a row take the
+            // same decision from the same exchanged max.
             const bool grow = mx > m_run + kRescaleLog2;
             const float m_use = grow ? mx : m_run;
             const float alpha = grow ? tc::ex2(m_run - m_use) : 1.f;
-            float spart[8];
+            // a row with no unmasked key yet keeps m = -inf; its p must come out 0, not NaN
+            const float m_sub = m_use == -INFINITY ? 0.f : m_use;
+            float spart[4];
+            uint32_t pk[16];
 #pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                // p = 2^(s * log2(e)/sqrt(D) - m); a share of them on the FMA pipe
-                const float arg = fmaf(x[c], a.scale_log2, -m_use);
-                const bool poly = (POLY == 1 && (c & 3) == 3) || (POLY == 2 && (c & 1));
-                x[c] = poly ? tc::ex2_poly(arg) : tc::ex2(arg);
-                spart[c & 7] = (c < 8) ? x[c] : spart[c & 7] + x[c];
+            for (int e = 0; e < 32; e += 2) {
+                // p = 2^(s * log2(e)/sqrt(D) - m)
+                const float p0 = tc::ex2(fmaf(x[e], a.scale_log2, -m_sub));
+                const float p1 = tc::ex2(fmaf(x[e + 1], a.scale_log2, -m_sub));
+                spart[e & 3] = (e < 4) ? p0 : spart[e & 3] + p0;
+                spart[(e + 1) & 3] = (e < 4) ? p1 : spart[(e + 1) & 3] + p1;
+                pk[e >> 1] = tc::pack_bf16(p0, p1);
             }
-            if (POLY != 0 && diag) {
-#pragma unroll
-                for (int c = 0; c < 64; ++c)
-                    if (c > i) x[c] = 0.f;  // the cubic maps -inf to ~2^-125, not 0
-            }
-            const float sum = ((spart[0] + spart[1]) + (spart[2] + spart[3])) +
-                              ((spart[4] + spart[5]) + (spart[6] + spart[7]));
-            l_run = l_run * alpha + sum;
+            l_run = l_run * alpha + ((spart[0] + spart[1]) + (spart[2] + spart[3]));
             const int pb = j & 1;
             // a rescale needs O complete up to tile j-1 (PV(j-1) done) before PV(j) adds to it;
             // rows that keep their reference max have alpha == 1, an exact no-op
@@ -361,53 +471,54 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
                 }
                 tc::fence_after_sync();
 #pragma unroll 1
-                for (int c0 = 0; c0 < D; c0 += 32) {
+                for (int c0 = 0; c0 < 64; c0 += 32) {
                     uint32_t o[32];
                     tc::tmem_ld32(o_addr + c0, o);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
+                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
                     tc::tmem_st32(o_addr + c0, o);
                 }
                 tc::tmem_wait_st();
             }
             m_run = m_use;
-            // P as bf16 pairs over the first 32 columns of this tile's S buffer (already
-            // read into registers); PV reads it from there as its A operand
-            {
-                uint32_t pk[32];
-#pragma unroll
-                for (int c = 0; c < 32; ++c) pk[c] = tc::pack_bf16(x[2 * c], x[2 * c + 1]);
-                tc::tmem_st32(tmem + lane_addr + 256 + 128 * h + 64 * pb, pk);
-                tc::tmem_wait_st();
-            }
+            // P as bf16 pairs: this thread's 16 of the first 32 columns of the tile's S
+            // buffer; PV reads them from there as its A operand
+            tc::tmem_st16(tmem + lane_addr + 256 + 128 * h + 64 * pb + 16 * c, pk);
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->p_full[h][pb]);
             if (NH == 2 && warp == kCtrlWarps && lane == 0) *reinterpret_cast<volatile int *>(&bars->sm0_tiles) = j + 1;
         }
+        // the row sum is split over the two column halves
+        float l_other = 0.f;
+        if (ok) ok = exchange(n_tiles, l_run, l_other);
         if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][(n_tiles - 1) & 1],
                                                         ((n_tiles - 1) >> 1) & 1, abort, a.status))) {
             tc::fence_after_sync();
-            const long long row = ((long long)(b * a.n_q_heads + g * G + hh)) * a.seg_len + m * TILE + i;
-            __nv_bfloat16 *orow = a.out + row * D;
-            const float inv_l = 1.f / l_run;
+            const float l_tot = l_run + l_other;
+            const bool write = hh < a.hc;  // rows 64..127 repeat the head when HC = 1
+            const long long row = ((long long)(b * a.n_q_heads + h0 + (write ? hh : 0))) * a.seg_len + m * TILE + i;
+            __nv_bfloat16 *orow = a.out + row * D + 64 * c;
+            const float inv_l = 1.f / l_tot;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 0; c0 < 64; c0 += 32) {
                 uint32_t o[32];
                 tc::tmem_ld32(o_addr + c0, o);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int c = 0; c < 32; c += 8) {
+                for (int e = 0; e < 32; e += 8) {
+                    if (!write) break;
                     uint4 v;
-                    v.x = tc::pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
-                    v.y = tc::pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
-                    v.z = tc::pack_bf16(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
-                    v.w = tc::pack_bf16(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
-                    *reinterpret_cast<uint4 *>(orow + c0 + c) = v;
+                    v.x = tc::pack_bf16(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
+                    v.y = tc::pack_bf16(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
+                    v.z = tc::pack_bf16(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
+                    v.w = tc::pack_bf16(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
+                    *reinterpret_cast<uint4 *>(orow + c0 + e) = v;
                 }
             }
-            a.lse[row] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
+            if (write && c == 0) a.lse[row] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
         }
     }
     tc::fence_before_sync();
@@ -444,9 +555,9 @@ bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
     return tma_rows_map(map, base, rows);
 }
 
-template <int NH>
+template <int NH, int MODE>
 hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
-                       const void *vs, const int32_t *idx, void *out, float *lse, unsigned *status,
+                       const void *vs, const FwdRoutes &rt, void *out, float *lse, unsigned *status,
                        cudaStream_t stream) {
     CUtensorMap mq, mkh, mvh, mks, mvs;
     const long long n_bg = (long long)p.batch * p.n_kv_heads;
@@ -458,7 +569,10 @@ hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, con
     if (!make_map(&mq, q, q_rows) || !make_map(&mks, ks, seg_rows) || !make_map(&mvs, vs, seg_rows))
         return HGA_ERR_INVALID_ARG;
     if (hist_rows > 0) {
-        if (!make_map(&mkh, kh, (unsigned long long)hist_rows) || !make_map(&mvh, vh, (unsigned long long)hist_rows))
+        // group routes read boxes of gs rows, one per routed group
+        const unsigned box = MODE == kGroup ? (unsigned)rt.gs : 64u;
+        if (!tma_rows_map(&mkh, kh, (unsigned long long)hist_rows, box) ||
+            !tma_rows_map(&mvh, vh, (unsigned long long)hist_rows, box))
             return HGA_ERR_INVALID_ARG;
     } else {
         mkh = mks;  // never read: no routable history
@@ -466,42 +580,54 @@ hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, con
     }
     const int nqb = p.seg_len / p.q_block;
     FwdArgs a;
+    const int G = p.n_q_heads / p.n_kv_heads;
+    a.hc = NH == 2 ? 4 : (G % 2 == 0 ? 2 : 1);
+    a.n_sub = G / a.hc;
     a.batch = p.batch;
     a.n_q_heads = p.n_q_heads;
     a.n_kv_heads = p.n_kv_heads;
     a.seg_len = p.seg_len;
-    a.topk = p.topk;
+    a.topk = rt.per_block;
     a.n_hist_chunks = p.n_hist_chunks;
+    a.gs = rt.gs;
+    a.ucount = rt.ucount;
+    a.umask = rt.umask;
     a.hist_stride = p.hist_head_stride;
     a.seg_stride = p.seg_head_stride;
     a.qb0 = p.qblock_end > 0 ? p.qblock_begin : 0;
     a.n_blocks = (p.qblock_end > 0 ? p.qblock_end : nqb) - a.qb0;
-    a.idx = idx;
+    a.idx = rt.list;
     a.out = static_cast<__nv_bfloat16 *>(out);
     a.lse = lse;
     a.status = status;
     a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
     const size_t smem = Smem<NH>::ALLOC;
-    static const int poly = [] {
-        const char *e = getenv("HGA_FWD_EXP2_POLY");
-        return e ? atoi(e) : 0;
-    }();
-    auto kern = poly == 2 ? attn_fwd_tc_kernel<NH, 2> : poly == 0 ? attn_fwd_tc_kernel<NH, 0>
-                                                                   : attn_fwd_tc_kernel<NH, 1>;
+    auto kern = attn_fwd_tc_kernel<NH, MODE>;
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
-    const unsigned grid = (unsigned)(a.n_blocks * n_bg);
+    const unsigned grid = (unsigned)(a.n_blocks * n_bg * a.n_sub);
     if (grid == 0) return HGA_OK;
-    kern<<<grid, 32 * kCtrlWarps + 128 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
+    kern<<<grid, 32 * kCtrlWarps + 256 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
     return record_cuda(cudaGetLastError());
+}
+
+template <int MODE>
+hga_status_t launch_mode(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
+                         const void *vs, const FwdRoutes &rt, void *out, float *lse, unsigned *status,
+                         cudaStream_t stream) {
+    const int G = p.n_q_heads / p.n_kv_heads;
+    if (G % 4 == 0) return launch_nh<2, MODE>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+    return launch_nh<1, MODE>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
 }
 
 }  // namespace
 
+bool attn_fwd_tc_shape(const hga_params_t &p) {
+    return p.dtype == HGA_BF16 && p.head_dim == 128 && p.chunk == 64 && p.q_block == 64;
+}
+
 bool attn_fwd_tc_supported(const hga_params_t &p) {
-    const int G = p.n_q_heads / p.n_kv_heads;
-    if (p.dtype != HGA_BF16 || p.head_dim != 128 || p.chunk != 64 || p.q_block != 64) return false;
-    if (G != 2 && G != 4) return false;
+    if (!attn_fwd_tc_shape(p)) return false;
     // TMA row coordinates are 32-bit
     const long long n_bg = (long long)p.batch * p.n_kv_heads;
     if (n_bg * (p.hist_head_stride > p.seg_head_stride ? p.hist_head_stride : p.seg_head_stride) >= (1ll << 31))
@@ -513,9 +639,16 @@ bool attn_fwd_tc_supported(const hga_params_t &p) {
 hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *kh, const void *vh,
                                 const void *ks, const void *vs, const int32_t *idx, void *out, float *lse,
                                 unsigned *status, cudaStream_t stream) {
-    const int G = p.n_q_heads / p.n_kv_heads;
-    if (G == 4) return launch_nh<2>(p, q, kh, vh, ks, vs, idx, out, lse, status, stream);
-    return launch_nh<1>(p, q, kh, vh, ks, vs, idx, out, lse, status, stream);
+    FwdRoutes rt{idx, p.topk, 0, nullptr, nullptr};
+    return launch_mode<kChunk>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+}
+
+hga_status_t launch_attn_fwd_tc_routes(const hga_params_t &p, const void *q, const void *kh, const void *vh,
+                                       const void *ks, const void *vs, const FwdRoutes &rt, void *out, float *lse,
+                                       unsigned *status, cudaStream_t stream) {
+    if (rt.gs > 0) return launch_mode<kGroup>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+    if (rt.umask) return launch_mode<kMasked>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+    return launch_mode<kChunk>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
 }
 
 }  // namespace hga

@@ -13,6 +13,7 @@ namespace hga {
 // Device status word bits (mirrors HGA_DEV_* in hga.h).
 constexpr unsigned kDevBadIndex = HGA_DEV_BAD_INDEX;
 constexpr unsigned kDevTimeout = HGA_DEV_TIMEOUT;
+constexpr unsigned kDevStageFull = HGA_DEV_STAGE_FULL;
 
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
@@ -77,7 +78,44 @@ hga_status_t launch_attn_bwd_tc(const hga_params_t &p, const void *q, const void
                                 const void *k_seg, const void *v_seg, const int32_t *idx, const float *lse,
                                 const float *delta, const void *dout, float *dq, float *dk, float *dv,
                                 unsigned *status, cudaStream_t stream);
+// bf16, head_dim 128, chunk 64, 64-query blocks: the shapes the tcgen05 kernels serve.
+bool attn_fwd_tc_shape(const hga_params_t &p);
+// attn_fwd_tc_shape and the TMA encoder is available and every row coordinate fits 32 bits.
 bool attn_fwd_tc_supported(const hga_params_t &p);
+// Routes that fill the history tiles of the tcgen05 attention kernels:
+//   chunk routes   list = idx [.][per_block = topk] chunk ids, gs = 0, no masks;
+//   group routes   list = gidx [.][per_block = topg] group ids of gs tokens;
+//   token-masked   list = the union of a block's per-token routes [.][per_block]
+//                  (ascending chunk ids), ucount entries valid per block, and
+//                  umask[.][per_block]: bit i set when token i of the block
+//                  routes to that chunk.
+struct FwdRoutes {
+    const int32_t *list;
+    int per_block;
+    int gs;
+    const int32_t *ucount;
+    const unsigned long long *umask;
+};
+hga_status_t launch_attn_fwd_tc_routes(const hga_params_t &p, const void *q, const void *k_hist, const void *v_hist,
+                                       const void *k_seg, const void *v_seg, const FwdRoutes &rt, void *out,
+                                       float *lse, unsigned *status, cudaStream_t stream);
+// Per-block unions of per-token routes (route_union.cu): ulist / umask [.][cap],
+// count [.] over the (b, g, block) triples, in a caller workspace.
+struct UnionView {
+    int cap;
+    int32_t *count;
+    int32_t *list;
+    unsigned long long *mask;
+};
+int route_union_cap(const hga_params_t &p);
+size_t route_union_bytes(const hga_params_t &p);
+UnionView route_union_view(const hga_params_t &p, void *ws);
+hga_status_t launch_route_union(const hga_params_t &p, const int32_t *idx_tok, const UnionView &v, unsigned *status,
+                                cudaStream_t stream);
+hga_status_t launch_attn_bwd_tc_routes(const hga_params_t &p, const void *q, const void *k_hist, const void *v_hist,
+                                       const void *k_seg, const void *v_seg, const FwdRoutes &rt, const float *lse,
+                                       const float *delta, const void *dout, float *dq, float *dk, float *dv,
+                                       unsigned *status, cudaStream_t stream);
 hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *k_hist,
                                 const void *v_hist, const void *k_seg, const void *v_seg,
                                 const int32_t *idx, void *out, float *lse, unsigned *status,
@@ -86,9 +124,13 @@ size_t decode_workspace_bytes(const hga_params_t &p, int n_local);
 hga_status_t launch_decode(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *kl,
                            const void *vl, int n_local, const int32_t *idx, void *out, float *lse, float *ws,
                            unsigned *status, cudaStream_t stream);
+// Tiered staging cache (tiered.cu): scratch entries, reset, and one fetch wave.
+long long tier_tile_cap(const hga_params_t &p);
+size_t tier_scratch_entries(const hga_params_t &p, int stage_slots);
+hga_status_t launch_tier_reset(const hga_params_t &p, int stage_slots, int32_t *scratch, cudaStream_t stream);
 hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
-                                 int stage_slots, int32_t *slot_map, int32_t *idx_remapped,
+                                 int stage_slots, int32_t *scratch, int32_t *idx_remapped,
                                  int32_t *n_fetched, unsigned *status, cudaStream_t stream);
 hga_status_t launch_selftest_wait_timeout(long long wait_cycles, unsigned *status, cudaStream_t stream);
 hga_status_t record_cuda(cudaError_t e);

@@ -52,7 +52,11 @@ extern "C" hga_status_t hga_attn_bwd_noalloc(const hga_params_t *p, const void *
                                              const void *dout, void *dq, void *dk_seg, void *dv_seg,
                                              cudaStream_t stream) {
     const size_t need = hga_attn_bwd_workspace_size(p);
-    if (need == 0) return HGA_ERR_INVALID_ARG;  // invalid shape
+    // a shape hga_attn_bwd rejects gets hga_attn_bwd's own status (its checks run
+    // before anything is enqueued)
+    if (need == 0)
+        return hga_attn_bwd(p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, dout, dq, dk_seg, dv_seg, nullptr, 0,
+                            stream);
     if (need > kScratchFloats * sizeof(float)) {
         hga::record_error("hga_attn_bwd_noalloc: batch * n_q_heads * seg_len exceeds the built-in "
                           "scratch of 1048576 rows; use hga_attn_bwd with a caller-allocated workspace");

@@ -218,25 +218,6 @@ __device__ __forceinline__ float ex2(float x) {
     return y;
 }
 
-// 2^x on the FMA pipe (no MUFU): x = n + f with n = round(x) and f in
-// [-1/2, 1/2]; 2^f by the cubic 1 + c1 f + c2 f^2 + c3 f^3 fitted to 2^f on
-// [-1/2, 1/2] in relative error (constant term fixed to 1 so 2^0 is exact;
-// Chebyshev-node least squares with Lawson reweighting; max relative error
-// 1.02e-4, below bf16 resolution); 2^n is added to the exponent field.
-// x is clamped to >= -125 so the exponent field stays that of a normal float
-// (results below 2^-125 read as about 2^-125, i.e. zero for attention).
-constexpr float kExp2C1 = 0.6932829273211771f;
-constexpr float kExp2C2 = 0.24221095962347064f;
-constexpr float kExp2C3 = 0.05500892999689336f;
-__device__ __forceinline__ float ex2_poly(float x) {
-    x = fmaxf(x, -125.f);
-    const float t = x + 12582912.f;  // 1.5 * 2^23: n sits in the low mantissa bits
-    const float n = t - 12582912.f;
-    const float f = x - n;
-    const float p = fmaf(fmaf(fmaf(kExp2C3, f, kExp2C2), f, kExp2C1), f, 1.0f);
-    return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t *>(&v);

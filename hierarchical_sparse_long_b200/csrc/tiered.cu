@@ -1,5 +1,5 @@
 // Tiered history: bring only the routed chunks' exact K/V from page-locked
-// host memory into a device staging buffer.
+// host memory into a device staging cache, and attend over it.
 //
 // "Long-Context Fine-Tuning with Limited VRAM", technical summary section 2.2
 // (tiered memory: detached history K/V in host RAM/NVMe; the GPU holds the
@@ -7,16 +7,30 @@
 // memory grows as O(S) + O(routing budget)) and the author abstract (HGA
 // loads a bounded set of exact historical tokens for each query block).
 //
-// Four kernels on the copy stream, for the query blocks [qb0, qb1):
-//   mark   : flag every (b, g, chunk) the blocks route to;
-//   scan   : number the flagged tiles -> slot_map[(b*Hkv+g)*Nc + j] = slot or -1,
-//            slot_src[slot] = (b*Hkv+g)*Nc + j, n_fetched;
-//   copy   : an SM copy of each needed 64 x D K and V tile straight from the
-//            mapped host pages into the staging slots (16-byte loads, many in
-//            flight, so the host link rather than the SMs is the bound);
+// The staging buffer is a cache of `slots` chunk tiles (64 x D keys and the
+// same values) shared by every (batch, kv head).  Its bookkeeping lives in a
+// caller-owned int32 scratch and persists from call to call:
+//   tile_slot[t]  slot holding tile t = (b*Hkv + g)*tile_cap + j, or -1
+//   tile_mark[t]  last wave that routed to tile t (de-duplicates a wave)
+//   slot_tile[s]  tile held by slot s, or -1
+//   slot_wave[s]  last wave whose attention reads slot s
+//   new_tile[], new_slot[]  this wave's fetch list
+//   ctl           wave counter, allocation cursor, fetch count
+// A fetch of query blocks [qb0, qb1) is one wave w, three kernels on the copy
+// stream:
+//   plan   (one CTA): the wave's distinct tiles; cached ones are re-stamped
+//          with w, the others get free slots -- slots whose last reader is
+//          wave w-2 or older, taken round-robin from a cursor, evicting their
+//          old tile -- and form the fetch list;
+//   copy   : an SM copy of each listed K and V tile straight from the mapped
+//          host pages into its slot (16-byte loads, many in flight, so the
+//          host link rather than the SMs is the bound);
 //   remap  : idx_remapped = slot of each routed chunk (-1 stays -1).
+// The caller guarantees that the attention of wave w-2 has finished before
+// the fetch of wave w starts (hga_attn_fwd_tiered orders its two streams so);
+// the attention of wave w-1 may still run, and its slots are never evicted.
 // The chunk order inside each block's route list is unchanged, so attention
-// over the staging buffer runs the same arithmetic in the same order as
+// over the staging cache runs the same arithmetic in the same order as
 // attention over resident history.
 #include "common.cuh"
 
@@ -24,75 +38,152 @@ namespace hga {
 
 namespace {
 
-__global__ void tier_mark_kernel(const int32_t *__restrict__ idx, int n_bg, int nqb, int topk, int qb0, int qb1,
-                                 int n_chunks, int32_t *__restrict__ slot_map, unsigned *status) {
+constexpr int kPlanThreads = 1024;
+constexpr int kFreeWave = -2;  // slot_wave of an empty slot: free for every wave >= 0
+
+struct TierScratch {
+    int32_t *tile_slot, *tile_mark, *slot_tile, *slot_wave, *new_tile, *new_slot, *ctl;
+};
+
+TierScratch tier_layout(int32_t *base, long long n_tiles, int slots) {
+    TierScratch s;
+    s.tile_slot = base;
+    s.tile_mark = s.tile_slot + n_tiles;
+    s.slot_tile = s.tile_mark + n_tiles;
+    s.slot_wave = s.slot_tile + slots;
+    s.new_tile = s.slot_wave + slots;
+    s.new_slot = s.new_tile + slots;
+    s.ctl = s.new_slot + slots;  // [0] last wave, [1] cursor, [2] tiles fetched by the last wave
+    return s;
+}
+
+__global__ void tier_reset_kernel(TierScratch s, long long n_tiles, int slots) {
+    const long long stride = (long long)gridDim.x * blockDim.x;
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < n_tiles; e += stride) {
+        s.tile_slot[e] = -1;
+        s.tile_mark[e] = -1;
+    }
+    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < slots; e += stride) {
+        s.slot_tile[e] = -1;
+        s.slot_wave[e] = kFreeWave;
+    }
+    if (blockIdx.x == 0 && threadIdx.x < 4) s.ctl[threadIdx.x] = 0;
+}
+
+// Block-wide exclusive scan of one flag per thread; returns the prefix and
+// writes the total to *total (every thread sees it after the call).
+__device__ int block_scan(int f, int *warp_sums, int *total) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int x = f;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int y = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += y;
+    }
+    if (lane == 31) warp_sums[warp] = x;
+    __syncthreads();
+    if (warp == 0) {
+        int v = lane < (int)(blockDim.x >> 5) ? warp_sums[lane] : 0;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += y;
+        }
+        warp_sums[lane] = v;
+        if (lane == 31) *total = v;
+    }
+    __syncthreads();
+    const int excl = (warp > 0 ? warp_sums[warp - 1] : 0) + x - f;
+    __syncthreads();  // warp_sums is reused by the next call
+    return excl;
+}
+
+__global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *__restrict__ idx, int n_bg, int nqb,
+                                                                 int topk, int qb0, int qb1, int n_chunks,
+                                                                 long long tile_cap, int slots, TierScratch s,
+                                                                 int32_t *n_fetched, unsigned *status) {
+    __shared__ int warp_sums[32];
+    __shared__ int n_new, total, taken_sh, cursor_sh;
+    const int tid = threadIdx.x;
+    const int w = s.ctl[0] + 1;
+    if (tid == 0) n_new = 0;
+    __syncthreads();
+    // 1. the wave's distinct tiles: cached ones are stamped with w, the others listed
     const long long per_bg = (long long)(qb1 - qb0) * topk;
-    const long long total = per_bg * n_bg;
-    for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
-         e += (long long)gridDim.x * blockDim.x) {
+    const long long total_e = per_bg * n_bg;
+    for (long long e = tid; e < total_e; e += kPlanThreads) {
         const int bg = (int)(e / per_bg);
         const long long r = e % per_bg;
         const int m = qb0 + (int)(r / topk), a = (int)(r % topk);
         const int j = idx[((long long)bg * nqb + m) * topk + a];
-        if (j >= 0 && j < n_chunks) slot_map[(long long)bg * n_chunks + j] = 1;
-        else if (j != -1) atomicOr(status, kDevBadIndex);
+        if (j < 0 || j >= n_chunks) {
+            if (j != -1) atomicOr(status, kDevBadIndex);
+            continue;
+        }
+        const long long t = (long long)bg * tile_cap + j;
+        if (atomicExch(&s.tile_mark[t], w) == w) continue;  // listed already by this wave
+        const int slot = s.tile_slot[t];
+        if (slot >= 0) {
+            s.slot_wave[slot] = w;
+        } else {
+            const int p = atomicAdd(&n_new, 1);
+            if (p < slots) s.new_tile[p] = (int32_t)t;
+        }
     }
-}
-
-// Single-CTA exclusive scan over the flags (entries are 0 / 1).
-__global__ void __launch_bounds__(1024) tier_scan_kernel(int32_t *__restrict__ slot_map, long long n,
-                                                         int32_t *__restrict__ slot_src, int32_t *__restrict__ n_out) {
-    __shared__ int warp_sums[32];
-    __shared__ int carry;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    if (tid == 0) carry = 0;
     __syncthreads();
-    for (long long base = 0; base < n; base += 1024) {
-        const long long e = base + tid;
-        const int f = (e < n) ? (slot_map[e] != 0) : 0;
-        int x = f;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const int y = __shfl_up_sync(0xffffffffu, x, off);
-            if (lane >= off) x += y;
+    const int need = n_new < slots ? n_new : slots;
+    // 2. free slots (last reader wave <= w - 2) round-robin from the cursor
+    if (tid == 0) {
+        taken_sh = 0;
+        cursor_sh = s.ctl[1];
+    }
+    __syncthreads();
+    const int cursor = cursor_sh;
+    int last = -1;
+    for (int base = 0; base < slots; base += kPlanThreads) {
+        if (taken_sh >= need) break;  // uniform: read after the barrier that ends the previous round
+        const int off = base + tid;
+        const int sl = off < slots ? (cursor + off) % slots : 0;
+        const int f = (off < slots && s.slot_wave[sl] <= w - 2) ? 1 : 0;
+        const int rank = taken_sh + block_scan(f, warp_sums, &total);
+        if (f && rank < need) {
+            const int t_new = s.new_tile[rank];
+            const int t_old = s.slot_tile[sl];
+            if (t_old >= 0) s.tile_slot[t_old] = -1;
+            s.slot_tile[sl] = t_new;
+            s.tile_slot[t_new] = sl;
+            s.slot_wave[sl] = w;
+            s.new_slot[rank] = sl;
+            if (rank == need - 1) last = off;
         }
-        if (lane == 31) warp_sums[warp] = x;
         __syncthreads();
-        if (warp == 0) {
-            int w = warp_sums[lane];
-#pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, w, off);
-                if (lane >= off) w += y;
-            }
-            warp_sums[lane] = w;
-        }
-        __syncthreads();
-        const int excl = carry + (warp > 0 ? warp_sums[warp - 1] : 0) + x - f;
-        if (e < n) {
-            slot_map[e] = f ? excl : -1;
-            if (f) slot_src[excl] = (int32_t)e;
-        }
-        __syncthreads();
-        if (tid == 1023) carry = excl + f;
+        if (tid == 0) taken_sh += total;
+        if (last >= 0) cursor_sh = (cursor + last + 1) % slots;
         __syncthreads();
     }
-    if (tid == 0 && n_out) *n_out = carry;
+    if (tid == 0) {
+        const int got = taken_sh < need ? taken_sh : need;
+        if (got < n_new) atomicOr(status, kDevStageFull);  // unfetched tiles stay -1 after the remap
+        s.ctl[0] = w;
+        s.ctl[1] = cursor_sh;
+        s.ctl[2] = got;
+        if (n_fetched) *n_fetched = got;
+    }
 }
 
 template <int ROW_BYTES>
 __global__ void __launch_bounds__(256) tier_copy_kernel(const uint4 *__restrict__ host_k, const uint4 *__restrict__ host_v,
-                                                        long long head_stride_bytes, int n_chunks, int chunk,
-                                                        const int32_t *__restrict__ slot_src,
-                                                        const int32_t *__restrict__ n_fetched, uint4 *__restrict__ stage_k,
+                                                        long long head_stride_bytes, long long tile_cap, int chunk,
+                                                        TierScratch s, uint4 *__restrict__ stage_k,
                                                         uint4 *__restrict__ stage_v) {
     constexpr int V_PER_ROW = ROW_BYTES / 16;
-    const int n = *n_fetched;
+    const int n = s.ctl[2];
     const int tile_vecs = chunk * V_PER_ROW;
-    for (int slot = blockIdx.x; slot < n; slot += gridDim.x) {
-        const int src = slot_src[slot];
-        const int bg = src / n_chunks, j = src % n_chunks;
-        const long long off = ((long long)bg * head_stride_bytes + (long long)j * chunk * ROW_BYTES) / 16;
+    for (int k = blockIdx.x; k < n; k += gridDim.x) {
+        const long long t = s.new_tile[k];
+        const int slot = s.new_slot[k];
+        const long long bg = t / tile_cap, j = t % tile_cap;
+        const long long off = (bg * head_stride_bytes + j * chunk * ROW_BYTES) / 16;
         const uint4 *sk = host_k + off, *sv = host_v + off;
         uint4 *dk = stage_k + (long long)slot * tile_vecs, *dv = stage_v + (long long)slot * tile_vecs;
         // issue every load of this thread before the stores (tile = 2 x chunk*ROW_BYTES)
@@ -116,7 +207,8 @@ __global__ void __launch_bounds__(256) tier_copy_kernel(const uint4 *__restrict_
 }
 
 __global__ void tier_remap_kernel(const int32_t *__restrict__ idx, int n_bg, int nqb, int topk, int qb0, int qb1,
-                                  int n_chunks, const int32_t *__restrict__ slot_map, int32_t *__restrict__ out) {
+                                  int n_chunks, long long tile_cap, const int32_t *__restrict__ tile_slot,
+                                  int32_t *__restrict__ out) {
     const long long per_bg = (long long)(qb1 - qb0) * topk;
     const long long total = per_bg * n_bg;
     for (long long e = (long long)blockIdx.x * blockDim.x + threadIdx.x; e < total;
@@ -126,55 +218,69 @@ __global__ void tier_remap_kernel(const int32_t *__restrict__ idx, int n_bg, int
         const int m = qb0 + (int)(r / topk), a = (int)(r % topk);
         const long long at = ((long long)bg * nqb + m) * topk + a;
         const int j = idx[at];
-        out[at] = (j >= 0 && j < n_chunks) ? slot_map[(long long)bg * n_chunks + j] : -1;
+        out[at] = (j >= 0 && j < n_chunks) ? tile_slot[(long long)bg * tile_cap + j] : -1;
     }
 }
 
 }  // namespace
 
+long long tier_tile_cap(const hga_params_t &p) { return p.hist_head_stride / p.chunk; }
+
+size_t tier_scratch_entries(const hga_params_t &p, int stage_slots) {
+    const long long n_tiles = (long long)p.batch * p.n_kv_heads * tier_tile_cap(p);
+    return (size_t)(2 * n_tiles + 4ll * stage_slots + 4);
+}
+
+hga_status_t launch_tier_reset(const hga_params_t &p, int stage_slots, int32_t *scratch, cudaStream_t stream) {
+    const long long n_tiles = (long long)p.batch * p.n_kv_heads * tier_tile_cap(p);
+    const TierScratch s = tier_layout(scratch, n_tiles, stage_slots);
+    const long long n = n_tiles > stage_slots ? n_tiles : stage_slots;
+    const unsigned grid = (unsigned)((n + 255) / 256 > 1184 ? 1184 : (n + 255) / 256 + 1);
+    tier_reset_kernel<<<grid, 256, 0, stream>>>(s, n_tiles, stage_slots);
+    return record_cuda(cudaGetLastError());
+}
+
 hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
-                                 int stage_slots, int32_t *slot_map, int32_t *idx_remapped, int32_t *n_fetched,
+                                 int stage_slots, int32_t *scratch, int32_t *idx_remapped, int32_t *n_fetched,
                                  unsigned *status, cudaStream_t stream) {
     const int n_bg = p.batch * p.n_kv_heads;
     const int nqb = p.seg_len / p.q_block;
-    const long long n_map = (long long)n_bg * p.n_hist_chunks;
-    int32_t *slot_src = slot_map + n_map;  // stage_slots entries after the map
+    const long long tile_cap = tier_tile_cap(p);
+    const TierScratch s = tier_layout(scratch, (long long)n_bg * tile_cap, stage_slots);
     void *dk = nullptr, *dv = nullptr;
     cudaError_t e = cudaHostGetDevicePointer(&dk, const_cast<void *>(host_k), 0);
-    if (e != cudaSuccess) { cudaGetLastError(); return HGA_ERR_INVALID_ARG; }
-    e = cudaHostGetDevicePointer(&dv, const_cast<void *>(host_v), 0);
-    if (e != cudaSuccess) { cudaGetLastError(); return HGA_ERR_INVALID_ARG; }
-    if (n_map > 0) {
-        e = cudaMemsetAsync(slot_map, 0, sizeof(int32_t) * n_map, stream);
-        if (e != cudaSuccess) return record_cuda(e);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        record_error("hga_fetch_tiered: host_k is not page-locked (mapped) host memory");
+        return HGA_ERR_INVALID_ARG;
     }
-    const long long marks = (long long)n_bg * (qb1 - qb0) * p.topk;
-    const unsigned g1 = (unsigned)((marks + 255) / 256 > 1184 ? 1184 : (marks + 255) / 256);
-    if (marks > 0 && n_map > 0)
-        tier_mark_kernel<<<g1, 256, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, slot_map, status);
-    // n_fetched doubles as the copy kernel's tile count; keep a device copy even when the caller passes none
-    int32_t *count = n_fetched ? n_fetched : slot_src + stage_slots;
-    tier_scan_kernel<<<1, 1024, 0, stream>>>(slot_map, n_map, slot_src, count);
+    e = cudaHostGetDevicePointer(&dv, const_cast<void *>(host_v), 0);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        record_error("hga_fetch_tiered: host_v is not page-locked (mapped) host memory");
+        return HGA_ERR_INVALID_ARG;
+    }
+    tier_plan_kernel<<<1, kPlanThreads, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, tile_cap,
+                                                     stage_slots, s, n_fetched, status);
     const int esize = p.dtype == HGA_BF16 ? 2 : 4;
     const long long head_stride_bytes = p.hist_head_stride * p.head_dim * esize;
     const int row_bytes = p.head_dim * esize;
-    const unsigned g3 = 148;
+    const unsigned g3 = (unsigned)sm_count();
     if (row_bytes == 128)
         tier_copy_kernel<128><<<g3, 256, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv, head_stride_bytes,
-                                                      p.n_hist_chunks, p.chunk, slot_src, count, (uint4 *)stage_k,
-                                                      (uint4 *)stage_v);
+                                                      tile_cap, p.chunk, s, (uint4 *)stage_k, (uint4 *)stage_v);
     else if (row_bytes == 256)
         tier_copy_kernel<256><<<g3, 256, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv, head_stride_bytes,
-                                                      p.n_hist_chunks, p.chunk, slot_src, count, (uint4 *)stage_k,
-                                                      (uint4 *)stage_v);
+                                                      tile_cap, p.chunk, s, (uint4 *)stage_k, (uint4 *)stage_v);
     else
         tier_copy_kernel<512><<<g3, 256, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv, head_stride_bytes,
-                                                      p.n_hist_chunks, p.chunk, slot_src, count, (uint4 *)stage_k,
-                                                      (uint4 *)stage_v);
+                                                      tile_cap, p.chunk, s, (uint4 *)stage_k, (uint4 *)stage_v);
+    const long long marks = (long long)n_bg * (qb1 - qb0) * p.topk;
+    const unsigned g1 = (unsigned)((marks + 255) / 256 > 1184 ? 1184 : (marks + 255) / 256);
     if (marks > 0)
-        tier_remap_kernel<<<g1, 256, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, slot_map,
-                                                  idx_remapped);
+        tier_remap_kernel<<<g1, 256, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, tile_cap,
+                                                  s.tile_slot, idx_remapped);
     return record_cuda(cudaGetLastError());
 }
 

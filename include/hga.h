@@ -25,9 +25,9 @@
  *                         always chosen, inside the k slots (hga_route);
  *   group stage         = hga_route_groups: the best groups of 8, 16 or 32
  *                         tokens inside the chosen chunks (a second routing
- *                         stage; the attention entry points read chunk routes);
+ *                         stage), attended by hga_attn_fwd/bwd_groups;
  *   strictly causal     = hga_route_causal: token i routes by its block's
- *                         queries up to i;
+ *                         queries up to i, attended by hga_attn_fwd/bwd_causal;
  *   decode              = hga_attn_decode: one new token per sequence, routed
  *                         as a one-token block.
  * With chunk routes, query i of the active segment attends exactly
@@ -75,6 +75,8 @@ typedef enum { HGA_BF16 = 0, HGA_FP32 = 1 } hga_dtype_t;
 /* Device status bits (hga_get_device_status). */
 #define HGA_DEV_BAD_INDEX 1u   /* a route index outside [-1, Nc) was skipped */
 #define HGA_DEV_TIMEOUT   2u   /* a pipeline wait gave up; results are invalid */
+#define HGA_DEV_STAGE_FULL 4u  /* a tiered fetch found too few free staging slots; the
+                                  tiles it could not place were not attended */
 
 /* Shape of one HGA attention layer call.
  *   batch B, n_q_heads Hq, n_kv_heads Hkv (Hq % Hkv == 0, G = Hq / Hkv),
@@ -163,7 +165,9 @@ hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float 
  * causal variant is proposed as future work).  Every token i of block m
  * routes by qbar_i = fp32 mean over the G heads of group g and the queries
  * m*q_block .. i of its block, with the score, selection, ties and sink rule
- * of hga_route; the last token of a block gets the block's route.
+ * of hga_route.  The last token of a block routes by the same block mean as
+ * hga_route, summed in another fp32 order, so its route equals the block's up
+ * to rounding (at near-ties of the k-th score the two may differ).
  *   idx: device int32 [B][Hkv][S][k], one route per token.  Other arguments
  *   as hga_route.  q_block = 1 gives the plain per-token route.
  * HGA_ERR_UNSUPPORTED when one token's score row set does not fit the CTA's
@@ -177,15 +181,69 @@ hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float 
  *   U = {history tokens of chunks idx[b][g][m][*] >= 0} u {segment tokens t <= i}
  *   z_t = q . k_t / sqrt(D),  out = sum_t softmax(z)_t v_t,  lse = ln sum_t exp(z_t)
  * History chunk j of head (b, g) is rows [j*c, j*c + c) of the slice at
- * k_hist + (b*Hkv + g)*hist_head_stride*D.  bf16 inputs use tcgen05 tensor
- * cores with fp32 accumulation (P is rounded to bf16 for the P.V product);
- * fp32 inputs use fp32 CUDA-core arithmetic.
+ * k_hist + (b*Hkv + g)*hist_head_stride*D.  Kernels by shape, never by
+ * environment: bf16 with head_dim 128 runs on tcgen05 tensor cores with fp32
+ * accumulation (P is rounded to bf16 for the P.V product; any GQA group size,
+ * packed 4, 2 or 1 query heads per CTA) and returns HGA_ERR_UNSUPPORTED when
+ * that kernel cannot run (no TMA tensor-map encoder in the driver, or a row
+ * coordinate beyond 32 bits); fp32 inputs run on fp32 CUDA cores (TF32 tensor
+ * cores would not meet fp32 accuracy), as does bf16 with head_dim 64.
  *   out: device [B][Hq][S][D] dtype; lse: device fp32 [B][Hq][S].  Rows of
  *   blocks outside [qblock_begin, qblock_end) are not written.
  * Route indices outside [-1, Nc) are skipped and flagged HGA_DEV_BAD_INDEX. */
 hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                           const void *k_seg, const void *v_seg, const int32_t *idx, void *out,
                           float *lse, cudaStream_t stream);
+
+/* Exact-token attention over group routes (technical summary section 2.1,
+ * group selection: only the exact K/V of the selected groups inside the chosen
+ * chunks are attended).  As hga_attn_fwd with the history part of U taken from
+ * gidx (hga_route_groups): for query (b, h, i) of block m,
+ *   U = {tokens u*group .. u*group + group - 1 of every u in gidx[b][g][m][*] >= 0}
+ *       u {segment tokens t <= i}
+ * so query i attends (valid groups) * group + i + 1 tokens.
+ *   gidx: device int32 [B][Hkv][S/q_block][topg], group ids < Nc * chunk / group
+ *   (others than -1 are skipped and flagged HGA_DEV_BAD_INDEX); group: 8, 16 or
+ *   32; topg: 1 .. min(topk * chunk / group, 512).  bf16 with head_dim 128 only
+ *   (tcgen05; anything else is HGA_ERR_UNSUPPORTED).  Groups are gathered as
+ *   group-row TMA boxes, 64 / group of them per 64-key tile. */
+hga_status_t hga_attn_fwd_groups(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *gidx, int group, int topg,
+                                 void *out, float *lse, cudaStream_t stream);
+
+/* Backward of hga_attn_fwd_groups (routes frozen): dq over the routed groups'
+ * and the segment's keys, dk_seg / dv_seg over the segment's keys; outputs and
+ * workspace (>= hga_attn_bwd_workspace_size(p) bytes) as hga_attn_bwd. */
+hga_status_t hga_attn_bwd_groups(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *gidx, int group, int topg,
+                                 const void *out, const float *lse, const void *dout, void *dq, void *dk_seg,
+                                 void *dv_seg, void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Exact-token attention over strictly causal routes (technical summary,
+ * limits section: the proposed strictly causal variant of block routing).
+ * idx_tok: device int32 [B][Hkv][S][topk], one route per token (from
+ * hga_route_causal).  Query (b, h, i) attends
+ *   U_i = {tokens of the chunks idx_tok[b][g][i][*] >= 0} u {segment tokens t <= i},
+ * i.e. min(k, Nc) * chunk + i + 1 tokens, equal to hga_attn_fwd with one-token
+ * query blocks.  The tcgen05 kernel keeps 64-query blocks: a first kernel
+ * builds, per block, the ascending union of its tokens' routed chunks and a
+ * 64-bit mask of the tokens routed to each (in workspace); the attention then
+ * masks, row by row, the union chunks a token did not route to.
+ *   workspace: device, >= hga_attn_causal_workspace_size(p, 0) bytes, 16-byte
+ *   aligned (the unions: B*Hkv*(S/64) * (4 + min(64 k, Nc) * 12) bytes).
+ *   Nc <= 16384; bf16 with head_dim 128 only (else HGA_ERR_UNSUPPORTED). */
+size_t hga_attn_causal_workspace_size(const hga_params_t *p, int backward);
+hga_status_t hga_attn_fwd_causal(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *idx_tok, void *out, float *lse,
+                                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Backward of hga_attn_fwd_causal (routes frozen): outputs as hga_attn_bwd;
+ * workspace >= hga_attn_causal_workspace_size(p, 1) bytes (the unions, then
+ * the fp32 row terms). */
+hga_status_t hga_attn_bwd_causal(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                                 const void *k_seg, const void *v_seg, const int32_t *idx_tok, const void *out,
+                                 const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg,
+                                 void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Bytes of device workspace hga_attn_bwd needs (fp32 row terms
  * delta = rowsum(dO * O), [B][Hq][S]).  Returns 0 for an invalid p. */
@@ -201,9 +259,11 @@ size_t hga_attn_bwd_workspace_size(const hga_params_t *p);
  *   dv_seg[b][g][t] = sum_{h in g, i >= t} P_t dO_i           (segment keys only)
  * History K/V get no gradient.  out / lse are the forward's outputs for
  * every block (qblock_begin/end must be 0/0).  dq [B][Hq][S][D], dk_seg and
- * dv_seg [B][Hkv][S][D]: device fp32 for every input dtype (gradients are
- * sums over many rows; fp32 keeps them within the tolerance a bf16 store
- * would exceed once |grad| >= 8), overwritten.  workspace: device, >=
+ * dv_seg [B][Hkv][S][D]: device fp32 for every input dtype, overwritten.  This
+ * is a deliberate departure from "gradients in the input dtype": gradients
+ * are sums over many rows, and one bf16 rounding of a value >= 8 is already
+ * off by up to 0.03, above the 2e-2 bf16 parity tolerance; the price is twice
+ * the bytes of a bf16 store.  Kernels by shape as for hga_attn_fwd.  workspace: device, >=
  * hga_attn_bwd_workspace_size(p) bytes, 16-byte aligned. */
 hga_status_t hga_attn_bwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
                           const void *k_seg, const void *v_seg, const int32_t *idx, const void *out,
@@ -259,27 +319,78 @@ hga_status_t hga_attn_decode(const hga_params_t *p, const void *q, const void *k
                              void *out, float *lse, void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /* Tiered history (technical summary section 2.2: detached K/V live in host
- * RAM, only the routed exact K/V are brought to the GPU).  For the query
- * blocks [qblock_begin, qblock_end) of idx, gathers the distinct (b, g, chunk)
- * tiles they route to, copies only those K and V tiles from page-locked host
- * memory (host_k / host_v: [B][Hkv][hist_head_stride][D], dtype) into the
- * device staging buffers stage_k / stage_v ([stage_slots][chunk][D]) and
- * writes idx_remapped (same shape as idx) with each index replaced by its
- * staging slot.  hga_attn_fwd over the same blocks with k_hist = stage_k,
- * v_hist = stage_v, hist_head_stride = 0 and idx = idx_remapped gives output
+ * RAM, only the routed exact K/V are brought to the GPU; device memory grows
+ * with the routing budget, not with the context).
+ *
+ * The device side is a staging cache of stage_slots chunk tiles (stage_k /
+ * stage_v: [stage_slots][chunk][D], dtype) shared by every (b, g), and its
+ * bookkeeping in a caller-owned int32 scratch of hga_tier_scratch_size bytes
+ * (tile -> slot map, slot -> tile map, the last wave reading each slot, the
+ * fetch list, a wave counter and an allocation cursor).  The cache persists
+ * from call to call: a tile fetched once is reused by every later wave that
+ * routes to it until it is evicted.  Tiles are (b, g, chunk j) of the host
+ * history host_k / host_v ([B][Hkv][hist_head_stride][D], page-locked), so the
+ * cache stays valid while the history only grows; reset it whenever the host
+ * history is replaced (or to start a segment with an empty cache).
+ *
+ * hga_tier_scratch_size: bytes of scratch for p (hist_head_stride tokens of
+ * host history per (b, g)) and stage_slots; 0 for invalid arguments.
+ * hga_tier_reset: marks every slot empty (one kernel on stream). */
+size_t hga_tier_scratch_size(const hga_params_t *p, int stage_slots);
+hga_status_t hga_tier_reset(const hga_params_t *p, int stage_slots, int32_t *scratch, cudaStream_t stream);
+
+/* One fetch wave: for the query blocks [qblock_begin, qblock_end) of idx, the
+ * distinct (b, g, chunk) tiles they route to that the cache does not hold are
+ * copied (K and V) from page-locked host memory into free slots -- slots whose
+ * last reading wave is two or more waves back, taken round-robin, evicting
+ * their old tile -- and idx_remapped (same shape as idx, rows of those blocks
+ * only) gets each index replaced by its slot.  hga_attn_fwd over the same
+ * blocks with k_hist = stage_k, v_hist = stage_v, hist_head_stride = 0,
+ * n_hist_chunks = stage_slots and idx = idx_remapped gives output
  * bit-identical to attending the history in device memory.
- *   slot_map: device int32 scratch of at least B*Hkv*Nc + stage_slots + 1
- *     entries (tile flags / slot numbers, then the slot -> tile list).
- *   n_fetched (device int32, may be NULL): number of tiles fetched.
- * The attention call over the staging buffer passes n_hist_chunks =
- * stage_slots (route indices are now slot numbers).
- * All work is enqueued on copy_stream; when done != NULL it is recorded on
- * copy_stream after the last kernel.  Returns HGA_ERR_INVALID_ARG when the
- * blocks can need more tiles than stage_slots. */
+ *   Ordering contract: the attention of the wave two fetches back must have
+ *   completed before this fetch starts (the previous wave's may still run);
+ *   hga_attn_fwd_tiered keeps it.
+ *   stage_slots >= min(2 * (blocks) * B * Hkv * min(k, Nc), B * Hkv * Nc),
+ *     else HGA_ERR_INVALID_ARG (the device flags HGA_DEV_STAGE_FULL if it
+ *     still runs out of free slots).
+ *   n_fetched (device int32, may be NULL): tiles copied by this wave.
+ *   host_k / host_v must be page-locked (mapped) host memory: anything else
+ *   returns HGA_ERR_INVALID_ARG before any launch.
+ * All work is enqueued on copy_stream; done (may be NULL) is recorded there
+ * after the last kernel. */
 hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const void *host_v,
                               const int32_t *idx, int qblock_begin, int qblock_end, void *stage_k,
-                              void *stage_v, int stage_slots, int32_t *slot_map, int32_t *idx_remapped,
+                              void *stage_v, int stage_slots, int32_t *scratch, int32_t *idx_remapped,
                               int32_t *n_fetched, cudaStream_t copy_stream, cudaEvent_t done);
+
+/* Detach into the host tier (technical summary section 2.2: the history K/V
+ * that leave the active segment live in host memory): copies tokens [0, S) of
+ * every (b, g) slice of k_seg / v_seg (device, seg_head_stride tokens apart)
+ * to tokens [dst_token, dst_token + S) of host_k / host_v (page-locked,
+ * [B][Hkv][hist_head_stride][D]), one 2-D copy each, on stream.  Later fetches
+ * of those chunks must be ordered after it (issue them on the same stream, or
+ * wait for it).  HGA_ERR_INVALID_ARG for pageable host memory or a range
+ * past hist_head_stride. */
+hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const void *v_seg, void *host_k,
+                              void *host_v, long long dst_token, cudaStream_t stream);
+
+/* hga_attn_fwd over host-resident history, overlapping fetch and attention:
+ * the blocks [qblock_begin, qblock_end) (0/0: all) are taken in waves of
+ * wave_blocks query blocks; wave w's fetch runs on copy_stream while wave
+ * w-1's attention runs on stream, and it starts only after wave w-2's
+ * attention has finished.  Output (out, lse) is bit-identical to hga_attn_fwd
+ * with the history resident.  The copy stream first waits for everything
+ * already enqueued on stream (the route that wrote idx); on return, stream is
+ * ordered after every fetch.  reset_cache != 0 empties the cache first.
+ *   events: 5 caller-created events (cudaEventDisableTiming is enough), used
+ *   as the cross-stream fences.  n_fetched (device int32, may be NULL): one
+ *   count per wave.  Other arguments as hga_fetch_tiered and hga_attn_fwd. */
+hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const void *host_k, const void *host_v,
+                                 const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
+                                 void *stage_k, void *stage_v, int stage_slots, int32_t *scratch,
+                                 int32_t *idx_remapped, int wave_blocks, int reset_cache, int32_t *n_fetched,
+                                 cudaStream_t stream, cudaStream_t copy_stream, const cudaEvent_t *events);
 
 /* Self-test of the bounded waits (the source pages have no counterpart): every
  * pipeline wait in the tensor-core kernels gives up after a cycle limit instead

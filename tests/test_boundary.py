@@ -100,6 +100,13 @@ def test_unsupported_shapes(L):
     for kw in (dict(head_dim=96), dict(chunk=32)):
         p = _params(**kw).c()
         assert L.hga_attn_fwd(ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, None) == -2
+        # the allocation-free backward reports the same status as hga_attn_bwd for a shape it has no kernel for
+        args = (ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake)
+        assert L.hga_attn_bwd(*args, fake, 1 << 20, None) == -2
+        assert L.hga_attn_bwd_noalloc(*args, None) == -2
+    bad = _params(topk=0).c()
+    args = (ctypes.byref(bad), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, fake)
+    assert L.hga_attn_bwd_noalloc(*args, None) == -1
 
 
 def test_null_and_misaligned_pointers(L):
@@ -116,13 +123,38 @@ def test_null_and_misaligned_pointers(L):
 
 
 def test_tiered_staging_capacity_checked_on_host(L):
-    p = _params(n_hist_chunks=32).c()
+    p = _params(n_hist_chunks=32, hist_head_stride=4096).c()
     fake = ctypes.c_void_p(0x1000)
-    # 2 blocks x 2 kv heads x 4 routes = 16 tiles may be needed
-    rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 0, 2, fake, fake, 15, fake, fake, None, None, None)
+    # 2 blocks x 2 kv heads x 4 routes = 16 tiles may be needed, and the 16 of the wave
+    # before stay protected: 32 slots (fewer than the 64 routable tiles) are required
+    rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 0, 2, fake, fake, 31, fake, fake, None, None, None)
     assert rc == -1
+    assert b"stage_slots" in L.hga_last_error()
     rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 1, 1, fake, fake, 64, fake, fake, None, None, None)
     assert rc == -1
+    rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 0, 2, fake, fake, 64, None, fake, None, None, None)
+    assert rc == -1  # no scratch
+    # the overlapped schedule: five events, waves of at least one block
+    evs = (ctypes.c_void_p * 5)(*([0x10] * 5))
+    args = [ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, 64, fake, fake]
+    assert L.hga_attn_fwd_tiered(*args, 0, 1, None, None, None, evs) == -1
+    assert L.hga_attn_fwd_tiered(*args, 1, 1, None, None, None, None) == -1
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, (ctypes.c_void_p * 5)(0x10, 0x10, 0, 0x10, 0x10)) == -1
+    args[11] = 31  # two waves of 2 blocks need 32 slots
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, evs) == -1
+
+
+def test_tiered_scratch_size(L):
+    # two int32 entries per (b, g, chunk) of the host history, four per slot, four control words
+    p = _params(n_hist_chunks=32, hist_head_stride=4096)
+    tiles = 1 * 2 * (4096 // 64)
+    want = ((2 * tiles + 4 * 100 + 4) * 4 + 255) // 256 * 256
+    assert hga.hga_tier_scratch_size(p, 100) == want
+    assert hga.hga_tier_scratch_size(p, 0) == 0
+    assert hga.hga_tier_scratch_size(_params(topk=0), 100) == 0
+    fake = ctypes.c_void_p(0x1000)
+    assert L.hga_tier_reset(ctypes.byref(p.c()), 0, fake, None) == -1
+    assert L.hga_tier_reset(ctypes.byref(p.c()), 100, None, None) == -1
 
 
 def test_workspace_size(L):

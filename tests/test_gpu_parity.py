@@ -390,7 +390,13 @@ def test_train_segments_route_and_summary_append():
 
 # ---------------------------------------------------------------- tiered history
 
-def _tiered_equals_resident(w, seg, wave):
+def _tiered_run(w, seg, wave, slots, reps=1):
+    """The segment's forward with the history only in pinned host memory, through
+    hga_attn_fwd_tiered: the overlapped schedule the benchmark runs (fetch waves on a
+    copy stream, attention of the previous wave on the compute stream, the staging
+    cache kept across waves, no host synchronisation between waves).  Returns the
+    resident forward, the tiered forward of every repetition (the cache is reset before
+    the first only), the fetched tiles per repetition, and the tiles routed."""
     import hierarchical_sparse_long_b200 as hga
     arrs = hc.segment_arrays(w, seg)
     g = hc.GpuSegment(w, arrs)
@@ -400,36 +406,99 @@ def _tiered_equals_resident(w, seg, wave):
     # history only in pinned host memory
     host_k = g.k_all[:, :, :T].contiguous().cpu().pin_memory()
     host_v = g.v_all[:, :, :T].contiguous().cpu().pin_memory()
-    nc = T // 64
     nqb = S // 64
-    keff = min(w.topk, nc)
-    slots = min(wave * w.batch * w.n_kv_heads * keff, w.batch * w.n_kv_heads * nc)
-    stage_k = torch.empty(max(slots, 1), 64, w.head_dim, device="cuda", dtype=g.q.dtype)
+    n_waves = -(-nqb // wave)
+    stage_k = torch.empty(slots, 64, w.head_dim, device="cuda", dtype=g.q.dtype)
     stage_v = torch.empty_like(stage_k)
-    slot_map = torch.empty(w.batch * w.n_kv_heads * nc + slots + 1, device="cuda", dtype=torch.int32)
-    idx_r = torch.full_like(idx, -1)
-    nf = torch.zeros(1, device="cuda", dtype=torch.int32)
-    out = torch.empty_like(out_res)
-    lse = torch.empty_like(lse_res)
     p = hc.params(w, T, hist_head_stride=T, seg_head_stride=T + S)
-    fetched = 0
-    for b0 in range(0, nqb, wave):
-        b1 = min(b0 + wave, nqb)
-        hga.hga_fetch_tiered(p, host_k, host_v, idx, b0, b1, stage_k, stage_v, slots, slot_map, idx_r, nf)
-        pa = hc.params(w, T, hist_head_stride=0, seg_head_stride=T + S, n_hist_chunks=slots,
-                       qblock_begin=b0, qblock_end=b1)
-        hga.hga_attn_fwd(pa, g.q, stage_k, stage_v, g.k_seg, g.v_seg, idx_r, out, lse)
-        torch.cuda.synchronize()
-        fetched += int(nf.item())
-    assert torch.equal(out, out_res) and torch.equal(lse, lse_res)
-    return fetched
+    scratch = torch.empty(hga.hga_tier_scratch_size(p, slots) // 4, device="cuda", dtype=torch.int32)
+    idx_r = torch.full_like(idx, -5)
+    events = [torch.cuda.Event() for _ in range(5)]
+    copy = torch.cuda.Stream()
+    results, fetched = [], []
+    for r in range(reps):
+        nf = torch.zeros(n_waves, device="cuda", dtype=torch.int32)
+        out = torch.full_like(out_res, float("nan"))
+        lse = torch.full_like(lse_res, float("nan"))
+        hga.hga_attn_fwd_tiered(p, g.q, host_k, host_v, g.k_seg, g.v_seg, idx, out, lse, stage_k, stage_v, slots,
+                                scratch, idx_r, wave, events, reset_cache=(r == 0), n_fetched=nf, copy_stream=copy)
+        results.append((out, lse))
+        fetched.append(nf)
+    torch.cuda.synchronize()
+    i = hc.f32(idx).astype(np.int64)
+    routed = {(b, gg, j) for b in range(w.batch) for gg in range(w.n_kv_heads) for j in i[b, gg].ravel() if j >= 0}
+    return arrs, idx, (out_res, lse_res), results, [int(f.sum().item()) for f in fetched], len(routed)
 
 
-def test_tiered_bitwise_small():
-    _tiered_equals_resident(MID, 0, wave=2)
+def _check_tiered(w, seg, wave, slots, sample_rows=None):
+    import hierarchical_sparse_long_b200 as hga
+    arrs, idx, (out_res, lse_res), results, fetched, distinct = _tiered_run(w, seg, wave, slots, reps=2)
+    for out, lse in results:
+        assert torch.equal(out, out_res) and torch.equal(lse, lse_res)
+    assert hga.hga_get_device_status() == 0
+    # against the oracle as well (the routes the GPU chose, attention in fp64)
+    T = arrs["T"]
+    sh = hc.oracle_shape(w, T)
+    rows = sample_rows
+    out_o, lse_o = oracle.attn_fwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                                   arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], hc.f32(idx).astype(np.int32),
+                                   rows=rows)
+    D = w.head_dim
+    out, lse = results[0]
+    if rows is None:
+        hc.compare(hc.f32(out), out_o, w.dtype, "tiered out")
+        hc.compare(hc.f32(lse), lse_o, w.dtype, "tiered lse")
+    else:
+        hc.compare(hc.f32(out).reshape(-1, D)[rows], out_o.reshape(-1, D)[rows], w.dtype, "tiered out")
+        hc.compare(hc.f32(lse).reshape(-1)[rows], lse_o.reshape(-1)[rows], w.dtype, "tiered lse")
+    return fetched, distinct
 
 
-def test_tiered_bitwise_128k_last_segment():
+def test_tiered_small_cache_evicts_and_matches():
+    # 13 history chunks x 2 kv heads; waves of 1 block route 2 x 4 tiles, so 16 slots
+    # (twice a wave) force evictions of tiles routed two waves back
+    fetched, distinct = _check_tiered(MID, 0, wave=1, slots=16)
+    assert fetched[0] >= distinct
+    print(f"small cache: fetched {fetched}, distinct {distinct}")
+
+
+def test_tiered_cache_fetches_each_tile_once():
+    # a cache that holds every routable tile: each routed tile crosses the host link
+    # once per reset, and a second pass over the same routes fetches nothing
+    fetched, distinct = _check_tiered(MID, 0, wave=2, slots=2 * 13)
+    assert fetched == [distinct, 0]
+
+
+def test_tiered_128k_last_segment():
     w = W["qwen3_128k_tiered"]
-    fetched = _tiered_equals_resident(w, 31, wave=8)
-    print(f"tiles fetched for the last 4,096-token segment: {fetched}")
+    nc = w.seg_starts[31] // 64
+    slots = w.batch * w.n_kv_heads * nc
+    fetched, distinct = _check_tiered(w, 31, wave=8, slots=slots, sample_rows=_sampled_rows(w, 96, seed=5))
+    assert fetched == [distinct, 0]
+    print(f"tiles fetched for the last 4,096-token segment: {fetched[0]} (distinct routed tiles {distinct})")
+
+
+def test_tiered_rejects_pageable_host_memory_before_any_launch():
+    import hierarchical_sparse_long_b200 as hga
+    w = MID
+    arrs = hc.segment_arrays(w, 0)
+    g = hc.GpuSegment(w, arrs)
+    T = arrs["T"]
+    idx = g.route(g.summaries())
+    host_k = g.k_all[:, :, :T].contiguous().cpu()  # pageable: not page-locked
+    host_v = g.v_all[:, :, :T].contiguous().cpu().pin_memory()
+    slots = 64
+    p = hc.params(w, T, hist_head_stride=T, seg_head_stride=T + w.seg_len)
+    stage_k = torch.zeros(slots, 64, w.head_dim, device="cuda", dtype=g.q.dtype)
+    stage_v = torch.zeros_like(stage_k)
+    scratch = torch.full((hga.hga_tier_scratch_size(p, slots) // 4,), 123, device="cuda", dtype=torch.int32)
+    idx_r = torch.full_like(idx, -5)
+    torch.cuda.synchronize()
+    with pytest.raises(hga.HGAError) as err:
+        hga.hga_fetch_tiered(p, host_k, host_v, idx, 0, 2, stage_k, stage_v, slots, scratch, idx_r)
+    assert err.value.code == -1
+    assert b"page-locked" in hga.lib().hga_last_error()
+    torch.cuda.synchronize()
+    # nothing was enqueued: scratch, staging and the remapped routes are untouched
+    assert torch.all(scratch == 123) and torch.all(idx_r == -5) and torch.all(stage_k == 0)
+    assert hga.hga_get_device_status() == 0
