@@ -15,7 +15,7 @@
 // group (its tiles then come from L2).  With HC = 1 the second 64 rows of the
 // M=128 half repeat the head's rows and are not written back.
 //
-// Warp roles (NH = 2: 672 threads):
+// Warp roles (NH = 2: 416 threads):
 //   warp 0      TMA producer: Q once, then K and V of every tile, each into
 //               its own 4-stage ring (routed chunk j -> TMA row coordinate
 //               (b*Hkv+g)*stride + 64 j); a K stage is released as soon as
@@ -29,16 +29,15 @@
 //               issued as soon as the softmax has written P.  One thread
 //               issues a tcgen05.mma only about every 100 cycles, so the four
 //               issue streams run in separate threads.
-//   warps 5+8h+4c.. softmax of half h, columns 32c..32c+31 of every score
-//               tile: two threads per query row (TMEM lane), one per column
-//               half, exchanging the tile's row max through shared memory
-//               (an mbarrier per row quadrant); online softmax in the log2
-//               domain, O rescaled in TMEM (columns 64c..64c+63) when the row
-//               max grows by more than 2^8, P written as bf16 pairs into the
-//               tile's S buffer, where the PV issue reads it.  Two threads per
-//               row halve the serial per-tile chain of a thread (TMEM load,
-//               max, exponentials, sum, P store) and give each SM sub-partition
-//               four softmax warps to interleave on the exponential unit.
+//   warps 5+4h.. softmax of half h: one TMEM lane (= query row) per thread
+//               (a warp reads the lane quadrant of its warp index % 4, so any
+//               four consecutive warps cover the half's 128 rows); online
+//               softmax in the log2 domain, O rescaled in TMEM when the row max
+//               grows by more than 2^8, P written as bf16 pairs into the tile's
+//               S buffer, where the PV issue reads it.  (Two threads per row,
+//               each with half of a tile's columns and a max exchange through
+//               shared memory, measured 7% slower on B200: the per-thread
+//               softmax chain is not what bounds a tile.)
 // TMEM (512 columns): O_h at 128h, S_h double-buffered at 256 + 128h + 64b.
 // Every wait is bounded; a timeout sets HGA_DEV_TIMEOUT and the CTA unwinds.
 //
@@ -79,8 +78,7 @@ struct Smem {
     static constexpr uint32_t Q = 0;
     static constexpr uint32_t K = Q + NH * Q_HALF_BYTES;      // K ring
     static constexpr uint32_t V = K + NSTAGE * KV_TILE_BYTES; // V ring
-    static constexpr uint32_t RED = V + NSTAGE * KV_TILE_BYTES;  // row max / sum exchange [2][2][128][2] fp32
-    static constexpr uint32_t GLIST = RED + 2 * 2 * 128 * 2 * 4;  // routed group ids (kGroup)
+    static constexpr uint32_t GLIST = V + NSTAGE * KV_TILE_BYTES;  // routed group ids (kGroup)
     static constexpr uint32_t BAR = GLIST + kMaxGroups * 4;
     static constexpr uint32_t TOTAL = BAR + 1024;  // barriers, tile list, flags
     static constexpr uint32_t ALLOC = TOTAL + 1024; // + alignment slack
@@ -106,7 +104,6 @@ struct Bars {
     uint64_t s_full[2][2];  // [half][S/P buffer]: S of the buffer's tile in TMEM
     uint64_t p_full[2][2];  // [half][S/P buffer]: P of the buffer's tile written to TMEM
     uint64_t o_done[2][2];  // [half][S/P buffer]: PV of the buffer's tile completed
-    uint64_t xchg[2][2][4]; // [parity][half][row quadrant]: both column halves posted their row values
     uint64_t drain[4];      // one per issuing thread (abort path)
     uint32_t tmem_base;
     int abort;
@@ -137,10 +134,8 @@ struct FwdArgs {
     float scale_log2;  // log2(e) / sqrt(D)
 };
 
-// Five control warps (producer, QK0, PV0, QK1, PV1) and 8 NH softmax warps;
-// a softmax warp reads the TMEM lane quadrant (warp index % 4), so any four
-// consecutive softmax warps cover the 128 rows of a half.  With NH = 2 the
-// 672 threads launch at 96 registers each (64,512 of the SM's 65,536).
+// Five control warps (producer, QK0, PV0, QK1, PV1) and 4 NH softmax warps.
+// With NH = 2 the 416 threads launch at up to 152 registers each.
 // Bounded wait until the shared counter reaches `target` (same contract as mbar_wait).
 __device__ __forceinline__ bool wait_count(int *counter, int target, volatile int *abort, unsigned *status) {
     volatile int *c = counter;
@@ -160,7 +155,7 @@ __device__ __forceinline__ bool wait_count(int *counter, int target, volatile in
 constexpr int kCtrlWarps = 5;
 
 template <int NH, int MODE>
-__global__ void __launch_bounds__(32 * kCtrlWarps + 256 * NH, 1)
+__global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                        const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
                        const __grid_constant__ CUtensorMap tm_vs, const FwdArgs a) {
@@ -191,9 +186,8 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 256 * NH, 1)
         for (int h = 0; h < 2; ++h)
             for (int bb = 0; bb < 2; ++bb) {
                 tc::mbar_init(&bars->s_full[h][bb], 1);
-                tc::mbar_init(&bars->p_full[h][bb], 8);  // every softmax warp of the half
+                tc::mbar_init(&bars->p_full[h][bb], 4);  // every softmax warp of the half
                 tc::mbar_init(&bars->o_done[h][bb], 1);
-                for (int qd = 0; qd < 4; ++qd) tc::mbar_init(&bars->xchg[bb][h][qd], 2);
             }
         for (int d = 0; d < 4; ++d) tc::mbar_init(&bars->drain[d], 1);
         bars->issued_k = 0;
@@ -354,30 +348,13 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 256 * NH, 1)
     }
     } else {
         // -------------------------------------------------------------- softmax / epilogue
-        const int sg = (warp - kCtrlWarps) >> 2;  // softmax warp group (four consecutive warps)
-        const int h = sg >> 1;                    // M half
-        const int c = sg & 1;                     // column half of the score tile
-        const int quad = warp & 3;                // TMEM lane quadrant this warp may access
-        const int r = quad * 32 + lane;           // row within the half = TMEM lane
-        const int hh = 2 * h + (r >> 6);          // head within the CTA
-        const int i = r & 63;                     // query row within the block
+        const int h = (warp - kCtrlWarps) >> 2;  // M half
+        const int quad = warp & 3;               // TMEM lane quadrant this warp may access
+        const int r = quad * 32 + lane;          // row within the half = TMEM lane
+        const int hh = 2 * h + (r >> 6);         // head within the group
+        const int i = r & 63;                    // query row within the block
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        const uint32_t o_addr = tmem + lane_addr + 128 * h + 64 * c;
-        // this thread's and its partner's slots of the row exchange, per tile parity
-        float *red = reinterpret_cast<float *>(smem + L::RED);
-        auto red_at = [&](int par, int cc) -> float * { return red + ((par * 2 + h) * 128 + r) * 2 + cc; };
-        // posts v for the partner thread (other column half, same row) and returns
-        // the partner's value; bounded wait, the same result across the warp
-        auto exchange = [&](int t, float v, float &other) -> bool {
-            const int par = t & 1;
-            *red_at(par, c) = v;
-            __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->xchg[par][h][quad]);
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->xchg[par][h][quad], (t >> 1) & 1, abort, a.status)))
-                return false;
-            other = *reinterpret_cast<volatile float *>(red_at(par, c ^ 1));
-            return true;
-        };
+        const uint32_t o_addr = tmem + lane_addr + 128 * h;
         float m_run = -INFINITY, l_run = 0.f;
         bool ok = true;
         // kGroup: valid columns of the last history tile; kMasked: this row's bit of the
@@ -400,66 +377,62 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 256 * NH, 1)
                 break;
             }
             tc::fence_after_sync();
-            float x[32];
+            uint32_t sr[64];
             {
-                uint32_t sr[32];
-                tc::tmem_ld32(tmem + lane_addr + 256 + 128 * h + 64 * bb + 32 * c, sr);
+                uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[0]);
+                uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sr[32]);
+                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * h + 64 * bb;
+                tc::tmem_ld32(s_addr, lo);
+                tc::tmem_ld32(s_addr + 32, hi);
                 tc::tmem_wait_ld();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) x[e] = __uint_as_float(sr[e]);
             }
-            if (j == n_tiles - 1) {  // the local tile of this block (warp-uniform)
+            float x[64];
+            const bool diag = (j == n_tiles - 1);  // the local tile of this block (warp-uniform)
 #pragma unroll
-                for (int e = 0; e < 32; ++e)
-                    if (32 * c + e > i) x[e] = -INFINITY;
+            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
+            if (diag) {
+#pragma unroll
+                for (int c = 0; c < 64; ++c)
+                    if (c > i) x[c] = -INFINITY;
             }
             if constexpr (MODE == kGroup) {
                 if (j == n_hist - 1 && last_cols < TILE) {  // repeated groups past the routed ones
 #pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * c + e >= last_cols) x[e] = -INFINITY;
+                    for (int c = 0; c < 64; ++c)
+                        if (c >= last_cols) x[c] = -INFINITY;
                 }
             }
             if constexpr (MODE == kMasked) {
                 if (row_off) {
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) x[e] = -INFINITY;
+                    for (int c = 0; c < 64; ++c) x[c] = -INFINITY;
                 }
             }
-            // row max of the raw scores (the scale is positive), 4 independent chains
-            float mpart[4];
+            // row max of the raw scores (the scale is positive), 8 independent chains
+            float mpart[8];
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mpart[e & 3] = (e < 4) ? x[e] : fmaxf(mpart[e & 3], x[e]);
-            float mx = fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])) * a.scale_log2;
-            // both column halves have loaded their scores once the exchange completes, so
-            // P may overwrite the first 32 columns of the S buffer after it
-            float mo;
-            if (!exchange(j, mx, mo)) {
-                ok = false;
-                break;
-            }
-            mx = fmaxf(mx, mo);
+            for (int c = 0; c < 64; ++c) mpart[c & 7] = (c < 8) ? x[c] : fmaxf(mpart[c & 7], x[c]);
+            const float mx = fmaxf(fmaxf(fmaxf(mpart[0], mpart[1]), fmaxf(mpart[2], mpart[3])),
+                                   fmaxf(fmaxf(mpart[4], mpart[5]), fmaxf(mpart[6], mpart[7]))) *
+                             a.scale_log2;
             // Lazy rescaling: the reference max only moves when the row max grows by
             // more than kRescaleLog2, so P stays <= 2^kRescaleLog2 and O is rescaled
-            // in TMEM only on those (rare) tiles.  Both threads of a row take the
-            // same decision from the same exchanged max.
+            // in TMEM only on those (rare) tiles.
             const bool grow = mx > m_run + kRescaleLog2;
             const float m_use = grow ? mx : m_run;
             const float alpha = grow ? tc::ex2(m_run - m_use) : 1.f;
             // a row with no unmasked key yet keeps m = -inf; its p must come out 0, not NaN
             const float m_sub = m_use == -INFINITY ? 0.f : m_use;
-            float spart[4];
-            uint32_t pk[16];
+            float spart[8];
 #pragma unroll
-            for (int e = 0; e < 32; e += 2) {
+            for (int c = 0; c < 64; ++c) {
                 // p = 2^(s * log2(e)/sqrt(D) - m)
-                const float p0 = tc::ex2(fmaf(x[e], a.scale_log2, -m_sub));
-                const float p1 = tc::ex2(fmaf(x[e + 1], a.scale_log2, -m_sub));
-                spart[e & 3] = (e < 4) ? p0 : spart[e & 3] + p0;
-                spart[(e + 1) & 3] = (e < 4) ? p1 : spart[(e + 1) & 3] + p1;
-                pk[e >> 1] = tc::pack_bf16(p0, p1);
+                x[c] = tc::ex2(fmaf(x[c], a.scale_log2, -m_sub));
+                spart[c & 7] = (c < 8) ? x[c] : spart[c & 7] + x[c];
             }
-            l_run = l_run * alpha + ((spart[0] + spart[1]) + (spart[2] + spart[3]));
+            const float sum = ((spart[0] + spart[1]) + (spart[2] + spart[3])) +
+                              ((spart[4] + spart[5]) + (spart[6] + spart[7]));
+            l_run = l_run * alpha + sum;
             const int pb = j & 1;
             // a rescale needs O complete up to tile j-1 (PV(j-1) done) before PV(j) adds to it;
             // rows that keep their reference max have alpha == 1, an exact no-op
@@ -471,54 +444,55 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 256 * NH, 1)
                 }
                 tc::fence_after_sync();
 #pragma unroll 1
-                for (int c0 = 0; c0 < 64; c0 += 32) {
+                for (int c0 = 0; c0 < D; c0 += 32) {
                     uint32_t o[32];
                     tc::tmem_ld32(o_addr + c0, o);
                     tc::tmem_wait_ld();
 #pragma unroll
-                    for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+                    for (int c = 0; c < 32; ++c) o[c] = __float_as_uint(__uint_as_float(o[c]) * alpha);
                     tc::tmem_st32(o_addr + c0, o);
                 }
                 tc::tmem_wait_st();
             }
             m_run = m_use;
-            // P as bf16 pairs: this thread's 16 of the first 32 columns of the tile's S
-            // buffer; PV reads them from there as its A operand
-            tc::tmem_st16(tmem + lane_addr + 256 + 128 * h + 64 * pb + 16 * c, pk);
-            tc::tmem_wait_st();
+            // P as bf16 pairs over the first 32 columns of this tile's S buffer (already
+            // read into registers); PV reads it from there as its A operand
+            {
+                uint32_t pk[32];
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = tc::pack_bf16(x[2 * c], x[2 * c + 1]);
+                tc::tmem_st32(tmem + lane_addr + 256 + 128 * h + 64 * pb, pk);
+                tc::tmem_wait_st();
+            }
             tc::fence_before_sync();
             __syncwarp();
             if (lane == 0) tc::mbar_arrive(&bars->p_full[h][pb]);
             if (NH == 2 && warp == kCtrlWarps && lane == 0) *reinterpret_cast<volatile int *>(&bars->sm0_tiles) = j + 1;
         }
-        // the row sum is split over the two column halves
-        float l_other = 0.f;
-        if (ok) ok = exchange(n_tiles, l_run, l_other);
         if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][(n_tiles - 1) & 1],
                                                         ((n_tiles - 1) >> 1) & 1, abort, a.status))) {
             tc::fence_after_sync();
-            const float l_tot = l_run + l_other;
             const bool write = hh < a.hc;  // rows 64..127 repeat the head when HC = 1
             const long long row = ((long long)(b * a.n_q_heads + h0 + (write ? hh : 0))) * a.seg_len + m * TILE + i;
-            __nv_bfloat16 *orow = a.out + row * D + 64 * c;
-            const float inv_l = 1.f / l_tot;
+            __nv_bfloat16 *orow = a.out + row * D;
+            const float inv_l = 1.f / l_run;
 #pragma unroll 1
-            for (int c0 = 0; c0 < 64; c0 += 32) {
+            for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
                 tc::tmem_ld32(o_addr + c0, o);
                 tc::tmem_wait_ld();
 #pragma unroll
-                for (int e = 0; e < 32; e += 8) {
+                for (int c = 0; c < 32; c += 8) {
                     if (!write) break;
                     uint4 v;
-                    v.x = tc::pack_bf16(__uint_as_float(o[e + 0]) * inv_l, __uint_as_float(o[e + 1]) * inv_l);
-                    v.y = tc::pack_bf16(__uint_as_float(o[e + 2]) * inv_l, __uint_as_float(o[e + 3]) * inv_l);
-                    v.z = tc::pack_bf16(__uint_as_float(o[e + 4]) * inv_l, __uint_as_float(o[e + 5]) * inv_l);
-                    v.w = tc::pack_bf16(__uint_as_float(o[e + 6]) * inv_l, __uint_as_float(o[e + 7]) * inv_l);
-                    *reinterpret_cast<uint4 *>(orow + c0 + e) = v;
+                    v.x = tc::pack_bf16(__uint_as_float(o[c + 0]) * inv_l, __uint_as_float(o[c + 1]) * inv_l);
+                    v.y = tc::pack_bf16(__uint_as_float(o[c + 2]) * inv_l, __uint_as_float(o[c + 3]) * inv_l);
+                    v.z = tc::pack_bf16(__uint_as_float(o[c + 4]) * inv_l, __uint_as_float(o[c + 5]) * inv_l);
+                    v.w = tc::pack_bf16(__uint_as_float(o[c + 6]) * inv_l, __uint_as_float(o[c + 7]) * inv_l);
+                    *reinterpret_cast<uint4 *>(orow + c0 + c) = v;
                 }
             }
-            if (write && c == 0) a.lse[row] = (m_run + __log2f(l_tot)) * 0.69314718055994530942f;
+            if (write) a.lse[row] = (m_run + __log2f(l_run)) * 0.69314718055994530942f;
         }
     }
     tc::fence_before_sync();
@@ -607,7 +581,7 @@ hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, con
     if (e != cudaSuccess) return record_cuda(e);
     const unsigned grid = (unsigned)(a.n_blocks * n_bg * a.n_sub);
     if (grid == 0) return HGA_OK;
-    kern<<<grid, 32 * kCtrlWarps + 256 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
+    kern<<<grid, 32 * kCtrlWarps + 128 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
     return record_cuda(cudaGetLastError());
 }
 
