@@ -39,9 +39,12 @@ under ``workloads`` in the same line with its own roofline, kernels, e2e and
 CPU baseline (``--also none`` skips them).
 
 Metric: query tokens/s (active query tokens processed per second, all heads),
-device-timed with CUDA events, L2 flushed (256 MiB write) before every step.
-Device-resident workloads capture one step as a CUDA graph and replay it (the
-phase events are recorded inside the graph); the tiered workload runs eagerly.
+device-timed with CUDA events around each step, L2 flushed (256 MiB write)
+before every step.  Device-resident workloads capture one step as a CUDA graph
+and replay it; the route and forward of a segment are one hga_route_attn_fwd
+call.  Per-kernel times come from a second graph of the same step with events
+between the library calls (route and forward then issued apart), replayed as
+many times after the timed region.  The tiered workload runs eagerly.
 Each segment's summary append, which reads only the segment's keys, runs on a
 side stream next to the segment's route (``--serial-append``: after attention).
 Rank 0 prints one JSON line.  ``--impl reference`` times the CPU oracle.
@@ -95,6 +98,9 @@ def parse():
                          "(default: on a side stream, overlapped with the route)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
     ap.add_argument("--tier-wave", type=int, default=32, help="query blocks per fetch wave of the tiered workload")
+    ap.add_argument("--only-last-segment", action="store_true",
+                    help="a step processes only the workload's last segment (its history summarised up "
+                         "front): for counter captures of the longest launches with few launches before them")
     ap.add_argument("--cpu-procs", type=int, default=0,
                     help="oracle processes for the 128K samples (0: up to 8, bounded by the host's cores)")
     return ap.parse_args()
@@ -293,7 +299,8 @@ class Layer:
 
     def segment(self, T, ev=None, q=None, do=None):
         """Route, attend [, backward], detach with history in device memory;
-        returns the number of library kernels launched.
+        returns the number of library kernels launched.  Uninstrumented (ev is
+        None), the route and the forward are one hga_route_attn_fwd call.
 
         With side_append the detach-time summary append (it reads only the
         segment's keys and writes summaries of chunks this segment's route
@@ -314,10 +321,13 @@ class Layer:
                                         w.seg_len // w.chunk, self.summ, self.nct)
                 if ev is not None:
                     ev.record(None)
-        rec("route")
-        hga.hga_route(p, q, self.summ, self.nct, self.idx)
-        rec("attn_fwd")
-        hga.hga_attn_fwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse)
+        if ev is None:
+            hga.hga_route_attn_fwd(p, q, self.summ, self.nct, self.idx, self.k, self.v, ks, vs, self.out, self.lse)
+        else:
+            rec("route")
+            hga.hga_route(p, q, self.summ, self.nct, self.idx)
+            rec("attn_fwd")
+            hga.hga_attn_fwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse)
         launches = 2
         if w.backward:
             rec("attn_bwd")
@@ -352,19 +362,26 @@ class Layer:
         self.n_waves = -(-nqb // self.wave)
         self.n_fetched = torch.zeros(len(w.seg_starts), self.n_waves, device="cuda", dtype=torch.int32)
         self.copy_stream = torch.cuda.Stream()
+        self.offload_stream = torch.cuda.Stream()
         self.tier_events = [torch.cuda.Event() for _ in range(5)]
 
     def segment_tiered(self, T, ev=None, q=None, si=0):
-        """The same segment with the history only in pinned host memory: route,
-        then attention over the staging cache with the fetch waves overlapped
+        """The same segment with the history only in pinned host memory: the
+        segment's K/V start their copy to the host history on an offload stream
+        (one 2-D copy each for K and V; only later segments read those rows, and
+        the next segment waits for it before it routes), then route, then
+        attention over the staging cache with the fetch waves overlapped
         (hga_attn_fwd_tiered; the cache is emptied at the first segment only),
-        then detach: the segment's K/V go to the host on the copy stream, one
-        2-D copy for K and one for V, before any later fetch."""
+        then the summary append."""
         torch, hga, w = self.torch, self.hga, self.w
         p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
         rec = ev.record if ev is not None else (lambda name: None)
+        compute = torch.cuda.current_stream()
+        compute.wait_stream(self.offload_stream)  # the previous segment is in the host history
+        self.offload_stream.wait_stream(compute)  # this segment's K/V are ready
+        hga.hga_tier_offload(p, ks, vs, self.host_k, self.host_v, T, stream=self.offload_stream)
         rec("route")
         hga.hga_route(p, q, self.summ, self.nct, self.idx)
         rec("attn_fwd")
@@ -373,10 +390,8 @@ class Layer:
                                 self.stage_v, self.slots, self.scratch, self.idx_r, self.wave, self.tier_events,
                                 reset_cache=first, n_fetched=self.n_fetched[si], copy_stream=self.copy_stream)
         launches = 1 + int(first) + (1 if T == 0 else 4 * self.n_waves)
-        # detach: the segment's K/V join the host history, its chunks become routable
+        # detach: the segment's chunks become routable
         rec("summaries")
-        self.copy_stream.wait_stream(torch.cuda.current_stream())
-        hga.hga_tier_offload(p, ks, vs, self.host_k, self.host_v, T, stream=self.copy_stream)
         hga.hga_build_summaries(self.k, self.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
                                 w.seg_len // w.chunk, self.summ, self.nct)
         rec(None)
@@ -431,6 +446,8 @@ class Layer:
         n = 0
         for si, T in enumerate(self.w.seg_starts):
             n += self.segment_tiered(T, ev, si=si) if self.w.tiered else self.segment(T, ev)
+        if self.w.tiered:  # the last offload belongs to the step
+            self.torch.cuda.current_stream().wait_stream(self.offload_stream)
         return n
 
 
@@ -711,6 +728,9 @@ def measure_layer(w, args, world, local):
     import torch
     import hierarchical_sparse_long_b200 as hga
     Layer.wave = args.tier_wave
+    if args.only_last_segment:
+        import dataclasses
+        w = dataclasses.replace(w, seg_starts=w.seg_starts[-1:])
     layer = Layer(w)
     layer.side_append = not args.serial_append and not w.tiered
     flush = torch.empty(256 * 1024 * 1024 // 4, device="cuda", dtype=torch.float32)
@@ -721,16 +741,24 @@ def measure_layer(w, args, world, local):
     if hga.hga_get_device_status() != 0:
         raise RuntimeError(f"{w.name}: device status reported an error during warm-up")
     # Device-resident workloads replay one step captured as a CUDA graph (one
-    # host launch per step, phase events recorded inside the graph); the tiered
-    # workload drives its copy stream from the host and stays eager.
-    graph, gev = None, None
+    # host launch per step; the route and the forward in one call, the forward
+    # overlapping the route's tail); the tiered workload drives its copy stream
+    # from the host and stays eager.  A second graph of the same step with CUDA
+    # events between the library calls (issued apart) gives the per-kernel
+    # times, replayed after the timed region: event nodes inside the timed
+    # graph would add their own gaps to the step.
+    graph, pgraph, gev = None, None, None
     if not w.tiered:
-        gev = PhaseEvents(external=True)
         graph = torch.cuda.CUDAGraph()
         with torch.cuda.graph(graph):
-            graph_launches = layer.step(ev=gev)
-        flush_l2(flush)
-        graph.replay()
+            graph_launches = layer.step()
+        gev = PhaseEvents(external=True)
+        pgraph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(pgraph):
+            layer.step(ev=gev)
+        for gr in (graph, pgraph):
+            flush_l2(flush)
+            gr.replay()
         torch.cuda.synchronize()
     sampler = ClockSampler(local)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -744,25 +772,31 @@ def measure_layer(w, args, world, local):
     time.sleep(0.3)
     for s in range(args.steps):
         flush_l2(flush)
+        starts[s].record()
         if graph is not None:
-            starts[s].record()
             graph.replay()
-            ends[s].record()
             launches += graph_launches
-            ends[s].synchronize()  # outside the timed window: read this replay's phase events
-            phases.append(gev.totals())
         else:
-            ev = PhaseEvents()
-            starts[s].record()
-            launches += layer.step(ev=ev)
-            ends[s].record()
-            phases.append(ev)
+            launches += layer.step()
+        ends[s].record()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
     total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, "cuda")
     value = job_throughput(tokens_per_step(w), args.steps, world, total_ms)
+    # per-kernel device times: the instrumented step, as many times as the timed one
+    for s in range(args.steps):
+        flush_l2(flush)
+        if pgraph is not None:
+            pgraph.replay()
+            torch.cuda.synchronize()
+            phases.append(gev.totals())
+        else:
+            ev = PhaseEvents()
+            layer.step(ev=ev)
+            phases.append(ev)
+    torch.cuda.synchronize()
     status = hga.hga_get_device_status()
 
     # per-kernel device time over the timed steps (events on the launching stream)
@@ -807,6 +841,12 @@ def measure_layer(w, args, world, local):
            "config": {**workload_config(w, world),
                       "l2": "flushed before every timed step (256 MiB write)",
                       "launch": "one CUDA graph replay per step" if graph is not None else "eager",
+                      "route_and_forward": "hga_route_attn_fwd (one call, the forward a programmatic "
+                                           "dependent of the route)" if not w.tiered else
+                                           "hga_route, then hga_attn_fwd_tiered",
+                      "kernel_times": "from as many replays of the same step with CUDA events between its "
+                                      "library calls (route and forward then issued apart), after the "
+                                      "timed region",
                       "append": "side stream, overlapped with the route" if layer.side_append else "in order"},
            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
            "device_status": status}
@@ -898,6 +938,8 @@ def e2e_measure(layer, steps):
                 layer.segment(T, q=q_d, do=do_d)
             for hbuf, t in zip(host_out, outs):
                 hbuf.copy_(t, non_blocking=True)
+        if w.tiered:
+            torch.cuda.current_stream().wait_stream(layer.offload_stream)
         e.record()
         e.synchronize()
         if it >= 1:
@@ -1008,12 +1050,18 @@ def run_decode_measure(w, args, world, local):
     torch.cuda.synchronize()
     if hga.hga_get_device_status() != 0:
         raise RuntimeError("device status reported an error during warm-up")
-    gev = PhaseEvents(external=True)
+    # the timed graph has no event nodes inside; a second graph of the same step with
+    # events between its calls gives the per-kernel times, replayed afterwards
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
-        graph_launches = layer.step(ev=gev)
-    flush_l2(flush)
-    graph.replay()
+        graph_launches = layer.step()
+    gev = PhaseEvents(external=True)
+    pgraph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(pgraph):
+        layer.step(ev=gev)
+    for gr in (graph, pgraph):
+        flush_l2(flush)
+        gr.replay()
     torch.cuda.synchronize()
     sampler = ClockSampler(local)
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
@@ -1030,14 +1078,17 @@ def run_decode_measure(w, args, world, local):
         graph.replay()
         ends[s_].record()
         launches += graph_launches
-        ends[s_].synchronize()  # outside the timed window: read this replay's phase events
-        phases.append(gev.totals())
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop()
     total_ms = max_over_ranks(sum(a.elapsed_time(b) for a, b in zip(starts, ends)), world, "cuda")
     value = job_throughput(tokens_per_step(w), args.steps, world, total_ms)
+    for s_ in range(args.steps):
+        flush_l2(flush)
+        pgraph.replay()
+        torch.cuda.synchronize()
+        phases.append(gev.totals())
     status = hga.hga_get_device_status()
     ph = {}
     for ev in phases:
@@ -1067,7 +1118,9 @@ def run_decode_measure(w, args, world, local):
     res = {"value": value, "unit": UNIT, "ms_per_step": total_ms / args.steps,
            "config": {**workload_config(w, world),
                       "l2": "flushed before every timed step (256 MiB write)",
-                      "launch": "one CUDA graph replay per step"},
+                      "launch": "one CUDA graph replay per step",
+                      "kernel_times": "from as many replays of the same step with CUDA events between its "
+                                      "library calls, after the timed region"},
            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
            "device_status": status}
     res["e2e"] = decode_e2e(layer, max(2, min(args.steps, 5)))

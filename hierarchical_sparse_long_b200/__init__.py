@@ -6,7 +6,8 @@ script (``build.py``).
 """
 from .binding import (  # noqa: F401
     HGA_BF16, HGA_FP32, HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT, HGA_DEV_STAGE_FULL, EXPORTED, HGAError, Params, lib,
-    hga_build_summaries, hga_route, hga_route_causal, hga_route_groups, hga_attn_fwd, hga_attn_bwd_workspace_size,
+    hga_build_summaries, hga_route, hga_route_causal, hga_route_groups, hga_attn_fwd, hga_route_attn_fwd,
+    hga_attn_bwd_workspace_size,
     hga_attn_bwd, hga_attn_bwd_noalloc, hga_attn_decode_workspace_size, hga_attn_decode,
     hga_attn_fwd_groups, hga_attn_bwd_groups, hga_attn_causal_workspace_size, hga_attn_fwd_causal,
     hga_attn_bwd_causal,

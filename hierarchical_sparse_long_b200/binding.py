@@ -22,6 +22,7 @@ STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3:
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
 EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd",
+            "hga_route_attn_fwd",
             "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_attn_fwd_groups", "hga_attn_bwd_groups",
             "hga_attn_causal_workspace_size", "hga_attn_fwd_causal", "hga_attn_bwd_causal",
             "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_tier_scratch_size",
@@ -89,6 +90,7 @@ def lib() -> ctypes.CDLL:
         L.hga_route_causal.argtypes = [pp, vp, vp, i, vp, vp]
         L.hga_route_groups.argtypes = [pp, vp, vp, i, vp, i, i, vp, vp]
         L.hga_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
+        L.hga_route_attn_fwd.argtypes = [pp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_attn_fwd_groups.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp]
         L.hga_attn_bwd_groups.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp, vp, vp, vp, vp, sz, vp]
         L.hga_attn_causal_workspace_size.argtypes = [pp, i]
@@ -117,6 +119,7 @@ def lib() -> ctypes.CDLL:
         L.hga_last_error.restype = ctypes.c_char_p
         for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd",
                   "hga_attn_bwd", "hga_attn_bwd_noalloc", "hga_attn_fwd_groups", "hga_attn_bwd_groups",
+                  "hga_route_attn_fwd",
                   "hga_attn_fwd_causal", "hga_attn_bwd_causal",
                   "hga_attn_decode", "hga_tier_reset", "hga_fetch_tiered", "hga_tier_offload", "hga_attn_fwd_tiered",
                   "hga_get_device_status"):
@@ -188,6 +191,16 @@ def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stre
     cp = p.c()
     _check(lib().hga_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg),
                               _ptr(idx), _ptr(out), _ptr(lse), _stream(stream)), "hga_attn_fwd")
+
+
+def hga_route_attn_fwd(p: Params, q, summ, summ_cap_chunks: int, idx, k_hist, v_hist, k_seg, v_seg, out, lse,
+                       stream=None):
+    """Route, then attend, in one call: the attention overlaps the route's tail
+    (routes into idx as hga_route; out/lse as hga_attn_fwd within rounding)."""
+    cp = p.c()
+    _check(lib().hga_route_attn_fwd(ctypes.byref(cp), _ptr(q), _ptr(summ), summ_cap_chunks, _ptr(idx),
+                                    _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg), _ptr(out), _ptr(lse),
+                                    _stream(stream)), "hga_route_attn_fwd")
 
 
 def hga_attn_fwd_groups(p: Params, q, k_hist, v_hist, k_seg, v_seg, gidx, group: int, topg: int, out, lse,

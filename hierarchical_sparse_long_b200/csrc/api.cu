@@ -186,6 +186,36 @@ hga_status_t hga_attn_fwd(const hga_params_t *p, const void *q, const void *k_hi
     return hga::launch_attn_fwd_simt(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status, stream);
 }
 
+hga_status_t hga_route_attn_fwd(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
+                                int32_t *idx, const void *k_hist, const void *v_hist, const void *k_seg,
+                                const void *v_seg, void *out, float *lse, cudaStream_t stream) {
+    CallRange range("hga_route_attn_fwd");
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
+    if (summ_cap_chunks < p->n_hist_chunks) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 16384) return HGA_ERR_UNSUPPORTED;
+    if (!q || !idx || !k_seg || !v_seg || !out || !lse) return HGA_ERR_INVALID_ARG;
+    if (p->n_hist_chunks > 0 && (!summ || !k_hist || !v_hist)) return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {q, (const void *)summ, k_hist, v_hist, k_seg, v_seg, (const void *)out})
+        if (ptr && !aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    const bool tc = hga::attn_fwd_tc_shape(*p);
+    if (tc && !hga::attn_fwd_tc_supported(*p)) {
+        hga::record_error("hga_route_attn_fwd: the tcgen05 kernel cannot take this call (no TMA tensor-map "
+                          "encoder in the driver, or a row coordinate beyond 32 bits)");
+        return HGA_ERR_UNSUPPORTED;
+    }
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    hga_params_t pr = *p;  // every block is routed
+    pr.qblock_begin = pr.qblock_end = 0;
+    st = hga::launch_route(pr, q, summ, summ_cap_chunks, idx, status, stream);
+    if (st != HGA_OK) return st;
+    if (tc) return hga::launch_attn_fwd_tc_after_route(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status,
+                                                        stream);
+    return hga::launch_attn_fwd_simt(*p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, status, stream);
+}
+
 size_t hga_attn_bwd_workspace_size(const hga_params_t *p) {
     if (check_params(p) != HGA_OK) return 0;
     const size_t rows = (size_t)p->batch * p->n_q_heads * p->seg_len;

@@ -54,6 +54,14 @@
 //            section), one tile per chunk of the union with a 64-bit mask of
 //            the block's tokens that route to it: rows whose bit is clear
 //            see the whole tile as masked.
+//
+// SEGF (chunk routes, hga_route_attn_fwd): the kernel is launched as a
+// programmatic dependent of the route kernel and takes the causal segment
+// tiles 0..m first -- they need no route -- so it runs while the route grid
+// finishes; the producer waits for the route grid (griddepcontrol.wait) only
+// before the first history tile, builds the tile list and publishes it to the
+// other roles through an mbarrier.  Everything else it reads was written
+// before the route kernel started.
 #include <cudaTypedefs.h>
 
 #include "tc_ptx.cuh"
@@ -105,6 +113,7 @@ struct Bars {
     uint64_t p_full[2][2];  // [half][S/P buffer]: P of the buffer's tile written to TMEM
     uint64_t o_done[2][2];  // [half][S/P buffer]: PV of the buffer's tile completed
     uint64_t drain[4];      // one per issuing thread (abort path)
+    uint64_t route_ready;   // SEGF: the history tile list is built
     uint32_t tmem_base;
     int abort;
     int n_hist;
@@ -154,7 +163,7 @@ __device__ __forceinline__ bool wait_count(int *counter, int target, volatile in
 
 constexpr int kCtrlWarps = 5;
 
-template <int NH, int MODE>
+template <int NH, int MODE, bool SEGF>
 __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     attn_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kh,
                        const __grid_constant__ CUtensorMap tm_vh, const __grid_constant__ CUtensorMap tm_ks,
@@ -190,6 +199,7 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
                 tc::mbar_init(&bars->o_done[h][bb], 1);
             }
         for (int d = 0; d < 4; ++d) tc::mbar_init(&bars->drain[d], 1);
+        tc::mbar_init(&bars->route_ready, 1);
         bars->issued_k = 0;
         bars->issued_v = 0;
         bars->sm0_tiles = 0;
@@ -198,16 +208,23 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     }
     int *glist = reinterpret_cast<int *>(smem + L::GLIST);
     const long long bgm = (long long)bg * nqb + m;
-    if (warp == 2 && lane == 0) {
+    // routed history chunks of this block; -1 is padding, anything else out of range is skipped
+    auto build_chunk_list = [&]() -> int {
+        const int32_t *sel = a.idx + bgm * a.topk;
+        int n = 0;
+        for (int i = 0; i < a.topk; ++i) {
+            const int j = sel[i];
+            if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
+            else if (j != -1) atomicOr(a.status, kDevBadIndex);
+        }
+        return n;
+    };
+    if (SEGF && warp == 2 && lane == 0) bars->n_hist = 0;  // published by the producer once routed
+    if (!SEGF && warp == 2 && lane == 0) {
         const int32_t *sel = a.idx + bgm * a.topk;
         int n = 0;
         if constexpr (MODE == kChunk) {
-            // routed history chunks of this block; -1 is padding, anything else out of range is skipped
-            for (int i = 0; i < a.topk; ++i) {
-                const int j = sel[i];
-                if (j >= 0 && j < a.n_hist_chunks) bars->tiles[n++] = j;
-                else if (j != -1) atomicOr(a.status, kDevBadIndex);
-            }
+            n = build_chunk_list();
         } else if constexpr (MODE == kGroup) {
             const int n_groups = a.n_hist_chunks * (TILE / a.gs);
             int ng = 0;
@@ -230,9 +247,20 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
     __syncthreads();
     tc::fence_after_sync();
     const uint32_t tmem = bars->tmem_base;
-    const int n_hist = bars->n_hist;
-    const int n_tiles = n_hist + m + 1;
     volatile int *abort = &bars->abort;
+    // Tile order: history tiles then segment tiles 0..m, or (SEGF) segment tiles
+    // then history tiles, whose count is known once the route is (resolve_tiles).
+    int n_hist = SEGF ? 0 : bars->n_hist;
+    int n_tiles = SEGF ? m + 2 : n_hist + m + 1;  // SEGF: provisional until tile m + 1
+    const int first_seg = SEGF ? 0 : n_hist;        // first segment tile (fixed once resolved)
+    // SEGF: at tile m + 1 every role waits for the producer's tile list
+    auto resolve_tiles = [&](int j) -> bool {
+        if (!SEGF || j != m + 1) return true;
+        if (!tc::mbar_wait(&bars->route_ready, 0, abort, a.status)) return false;
+        n_hist = *reinterpret_cast<volatile int *>(&bars->n_hist);
+        n_tiles = m + 1 + n_hist;
+        return true;
+    };
 
     if (warp < kCtrlWarps) {
     if (warp == 0) {
@@ -255,9 +283,12 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
             // a tile as TMA boxes: one 64-row box per column half, or (kGroup history
             // tiles) 64 / gs boxes of gs rows per column half, group slot u at row u*gs
             const int n_groups = MODE == kGroup ? bars->n_groups : 0;
-            auto load_tile = [&](uint8_t *dst, const CUtensorMap *mh, const CUtensorMap *ms, int j, uint64_t *bar) {
-                if (j >= n_hist) {
-                    const int row = (int)((long long)bg * a.seg_stride + (long long)(j - n_hist) * TILE);
+            auto load_tile = [&](uint8_t *dst, const CUtensorMap *mh, const CUtensorMap *ms, int jt, uint64_t *bar) {
+                // segment tile jt - first_seg (SEGF: jt <= m), else history tile j
+                const bool seg = SEGF ? jt <= m : jt >= n_hist;
+                const int j = SEGF ? jt - m - 1 : jt;
+                if (seg) {
+                    const int row = (int)((long long)bg * a.seg_stride + (long long)(jt - first_seg) * TILE);
                     tc::tma_load_2d(dst, ms, 0, row, bar);
                     tc::tma_load_2d(dst + 64 * 128, ms, 64, row, bar);
                 } else if constexpr (MODE == kGroup) {
@@ -279,6 +310,15 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
             int nk = 0, nv = 0;
             for (int j = 0; j < n_tiles; ++j) {
                 const int s = j % NSTAGE, u = j / NSTAGE;
+                if (SEGF && j == m + 1) {
+                    // the route grid has finished and its writes are visible after this
+                    asm volatile("griddepcontrol.wait;" ::: "memory");
+                    n_hist = build_chunk_list();
+                    bars->n_hist = n_hist;
+                    n_tiles = m + 1 + n_hist;
+                    tc::mbar_arrive(&bars->route_ready);
+                    if (j >= n_tiles) break;
+                }
                 if (j >= NSTAGE && !tc::mbar_wait(&bars->k_empty[s], (u - 1) & 1, abort, a.status)) break;
                 tc::mbar_arrive_expect_tx(&bars->k_full[s], KV_TILE_BYTES);
                 load_tile(smem + L::K + s * KV_TILE_BYTES, &tm_kh, &tm_ks, j, &bars->k_full[s]);
@@ -305,6 +345,8 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
                 ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
                 for (int j = 0; ok && j < n_tiles; ++j) {
                     const int s = j % NSTAGE, bb = j & 1;
+                    if (!resolve_tiles(j)) break;
+                    if (j >= n_tiles) break;
                     if (!tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)) break;
                     // S buffer bb is free once PV(j-2), which read P(j-2) from it, has completed
                     if (j >= 2 && !tc::mbar_wait(&bars->o_done[h][bb], ((j >> 1) - 1) & 1, abort, a.status))
@@ -330,6 +372,8 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
                 const uint32_t o_tmem = tmem + 128 * h;
                 for (int t = 0; t < n_tiles; ++t) {
                     const int s = t % NSTAGE, pb = t & 1;
+                    if (!resolve_tiles(t)) break;
+                    if (t >= n_tiles) break;
                     if (!tc::mbar_wait(&bars->v_full[s], (t / NSTAGE) & 1, abort, a.status)) break;
                     if (!tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort, a.status)) break;
                     tc::fence_after_sync();
@@ -364,6 +408,11 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
         if (MODE == kMasked && n_hist > 0) mask_next = a.umask[bgm * a.topk];
         for (int j = 0; j < n_tiles; ++j) {
             const int bb = j & 1;
+            if (!__all_sync(0xffffffffu, resolve_tiles(j))) {
+                ok = false;
+                break;
+            }
+            if (j >= n_tiles) break;
             bool row_off = false;  // kMasked: the whole tile is masked for this row
             if constexpr (MODE == kMasked) {
                 if (j < n_hist) {
@@ -387,7 +436,7 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
                 tc::tmem_wait_ld();
             }
             float x[64];
-            const bool diag = (j == n_tiles - 1);  // the local tile of this block (warp-uniform)
+            const bool diag = (j == (SEGF ? m : n_tiles - 1));  // the local tile of this block (warp-uniform)
 #pragma unroll
             for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(sr[c]);
             if (diag) {
@@ -529,7 +578,7 @@ bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
     return tma_rows_map(map, base, rows);
 }
 
-template <int NH, int MODE>
+template <int NH, int MODE, bool SEGF>
 hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
                        const void *vs, const FwdRoutes &rt, void *out, float *lse, unsigned *status,
                        cudaStream_t stream) {
@@ -576,22 +625,34 @@ hga_status_t launch_nh(const hga_params_t &p, const void *q, const void *kh, con
     a.status = status;
     a.scale_log2 = (float)(1.4426950408889634 / __builtin_sqrt((double)D));
     const size_t smem = Smem<NH>::ALLOC;
-    auto kern = attn_fwd_tc_kernel<NH, MODE>;
+    auto kern = attn_fwd_tc_kernel<NH, MODE, SEGF>;
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const unsigned grid = (unsigned)(a.n_blocks * n_bg * a.n_sub);
     if (grid == 0) return HGA_OK;
-    kern<<<grid, 32 * kCtrlWarps + 128 * NH, smem, stream>>>(mq, mkh, mvh, mks, mvs, a);
-    return record_cuda(cudaGetLastError());
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(32 * kCtrlWarps + 128 * NH);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    // SEGF: a programmatic dependent of the route kernel launched just before it
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = SEGF ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, kern, mq, mkh, mvh, mks, mvs, a);
+    if (e == cudaSuccess) e = cudaGetLastError();
+    return record_cuda(e);
 }
 
-template <int MODE>
+template <int MODE, bool SEGF = false>
 hga_status_t launch_mode(const hga_params_t &p, const void *q, const void *kh, const void *vh, const void *ks,
                          const void *vs, const FwdRoutes &rt, void *out, float *lse, unsigned *status,
                          cudaStream_t stream) {
     const int G = p.n_q_heads / p.n_kv_heads;
-    if (G % 4 == 0) return launch_nh<2, MODE>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
-    return launch_nh<1, MODE>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+    if (G % 4 == 0) return launch_nh<2, MODE, SEGF>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+    return launch_nh<1, MODE, SEGF>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
 }
 
 }  // namespace
@@ -615,6 +676,13 @@ hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void
                                 unsigned *status, cudaStream_t stream) {
     FwdRoutes rt{idx, p.topk, 0, nullptr, nullptr};
     return launch_mode<kChunk>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
+}
+
+hga_status_t launch_attn_fwd_tc_after_route(const hga_params_t &p, const void *q, const void *kh, const void *vh,
+                                            const void *ks, const void *vs, const int32_t *idx, void *out,
+                                            float *lse, unsigned *status, cudaStream_t stream) {
+    FwdRoutes rt{idx, p.topk, 0, nullptr, nullptr};
+    return launch_mode<kChunk, true>(p, q, kh, vh, ks, vs, rt, out, lse, status, stream);
 }
 
 hga_status_t launch_attn_fwd_tc_routes(const hga_params_t &p, const void *q, const void *kh, const void *vh,

@@ -116,6 +116,13 @@ hga_status_t launch_attn_bwd_tc_routes(const hga_params_t &p, const void *q, con
                                        const void *k_seg, const void *v_seg, const FwdRoutes &rt, const float *lse,
                                        const float *delta, const void *dout, float *dq, float *dk, float *dv,
                                        unsigned *status, cudaStream_t stream);
+// The tcgen05 forward as a programmatic dependent of the route kernel launched
+// just before it on the same stream (causal segment tiles first; the route is
+// waited for before the history tiles).
+hga_status_t launch_attn_fwd_tc_after_route(const hga_params_t &p, const void *q, const void *k_hist,
+                                            const void *v_hist, const void *k_seg, const void *v_seg,
+                                            const int32_t *idx, void *out, float *lse, unsigned *status,
+                                            cudaStream_t stream);
 hga_status_t launch_attn_fwd_tc(const hga_params_t &p, const void *q, const void *k_hist,
                                 const void *v_hist, const void *k_seg, const void *v_seg,
                                 const int32_t *idx, void *out, float *lse, unsigned *status,

@@ -290,6 +290,9 @@ __device__ void drain_ring(uint64_t *bar, int from, int to, int slots) {
 
 template <typename T, int D, int CL, bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 2) route_kernel(const RouteArgs a) {
+    // a forward launched as a programmatic dependent may start as soon as every
+    // CTA of this grid is running (it waits for this grid before reading idx)
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     constexpr int R = SPLIT ? 1 : CL;  // query blocks scored by this CTA
     extern __shared__ __align__(128) uint8_t smem[];
     __shared__ int abort_flag;

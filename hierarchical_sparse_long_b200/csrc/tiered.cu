@@ -24,7 +24,8 @@
 //          old tile -- and form the fetch list;
 //   copy   : an SM copy of each listed K and V tile straight from the mapped
 //          host pages into its slot (16-byte loads, many in flight, so the
-//          host link rather than the SMs is the bound);
+//          host link rather than the SMs is the bound; CTAs small enough to
+//          share an SM with an attention CTA);
 //   remap  : idx_remapped = slot of each routed chunk (-1 stays -1).
 // The caller guarantees that the attention of wave w-2 has finished before
 // the fetch of wave w starts (hga_attn_fwd_tiered orders its two streams so);
@@ -171,12 +172,18 @@ __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *
     }
 }
 
+// 128 threads and at most 64 registers a thread: small enough to share an SM with
+// an attention CTA (which leaves neither the registers nor the threads of a
+// larger copy CTA free), so a wave's fetch overlaps the previous wave's attention.
+constexpr int kCopyThreads = 128;
+
 template <int ROW_BYTES>
-__global__ void __launch_bounds__(256) tier_copy_kernel(const uint4 *__restrict__ host_k, const uint4 *__restrict__ host_v,
-                                                        long long head_stride_bytes, long long tile_cap, int chunk,
-                                                        TierScratch s, uint4 *__restrict__ stage_k,
-                                                        uint4 *__restrict__ stage_v) {
+__global__ void __launch_bounds__(kCopyThreads, 8)
+    tier_copy_kernel(const uint4 *__restrict__ host_k, const uint4 *__restrict__ host_v, long long head_stride_bytes,
+                     long long tile_cap, int chunk, TierScratch s, uint4 *__restrict__ stage_k,
+                     uint4 *__restrict__ stage_v) {
     constexpr int V_PER_ROW = ROW_BYTES / 16;
+    constexpr int PER = 4;  // vectors of K and of V a thread holds in flight
     const int n = s.ctl[2];
     const int tile_vecs = chunk * V_PER_ROW;
     for (int k = blockIdx.x; k < n; k += gridDim.x) {
@@ -186,22 +193,25 @@ __global__ void __launch_bounds__(256) tier_copy_kernel(const uint4 *__restrict_
         const long long off = (bg * head_stride_bytes + j * chunk * ROW_BYTES) / 16;
         const uint4 *sk = host_k + off, *sv = host_v + off;
         uint4 *dk = stage_k + (long long)slot * tile_vecs, *dv = stage_v + (long long)slot * tile_vecs;
-        // issue every load of this thread before the stores (tile = 2 x chunk*ROW_BYTES)
-        constexpr int MAXV = 8;
-        uint4 bk[MAXV], bv[MAXV];
-        int cnt = 0;
-        for (int e = threadIdx.x; e < tile_vecs && cnt < MAXV; e += blockDim.x, ++cnt) {
-            bk[cnt] = sk[e];
-            bv[cnt] = sv[e];
-        }
-        cnt = 0;
-        for (int e = threadIdx.x; e < tile_vecs && cnt < MAXV; e += blockDim.x, ++cnt) {
-            dk[e] = bk[cnt];
-            dv[e] = bv[cnt];
-        }
-        for (int e = threadIdx.x + MAXV * blockDim.x; e < tile_vecs; e += blockDim.x) {
-            dk[e] = sk[e];
-            dv[e] = sv[e];
+        // every load of a round is issued before its stores
+        for (int e0 = threadIdx.x; e0 < tile_vecs; e0 += PER * kCopyThreads) {
+            uint4 bk[PER], bv[PER];
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = e0 + u * kCopyThreads;
+                if (e < tile_vecs) {
+                    bk[u] = sk[e];
+                    bv[u] = sv[e];
+                }
+            }
+#pragma unroll
+            for (int u = 0; u < PER; ++u) {
+                const int e = e0 + u * kCopyThreads;
+                if (e < tile_vecs) {
+                    dk[e] = bk[u];
+                    dv[e] = bv[u];
+                }
+            }
         }
     }
 }
@@ -266,16 +276,19 @@ hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, cons
     const int esize = p.dtype == HGA_BF16 ? 2 : 4;
     const long long head_stride_bytes = p.hist_head_stride * p.head_dim * esize;
     const int row_bytes = p.head_dim * esize;
-    const unsigned g3 = (unsigned)sm_count();
+    const unsigned g3 = (unsigned)(2 * sm_count());
     if (row_bytes == 128)
-        tier_copy_kernel<128><<<g3, 256, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv, head_stride_bytes,
-                                                      tile_cap, p.chunk, s, (uint4 *)stage_k, (uint4 *)stage_v);
+        tier_copy_kernel<128><<<g3, kCopyThreads, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv,
+                                                               head_stride_bytes, tile_cap, p.chunk, s,
+                                                               (uint4 *)stage_k, (uint4 *)stage_v);
     else if (row_bytes == 256)
-        tier_copy_kernel<256><<<g3, 256, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv, head_stride_bytes,
-                                                      tile_cap, p.chunk, s, (uint4 *)stage_k, (uint4 *)stage_v);
+        tier_copy_kernel<256><<<g3, kCopyThreads, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv,
+                                                               head_stride_bytes, tile_cap, p.chunk, s,
+                                                               (uint4 *)stage_k, (uint4 *)stage_v);
     else
-        tier_copy_kernel<512><<<g3, 256, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv, head_stride_bytes,
-                                                      tile_cap, p.chunk, s, (uint4 *)stage_k, (uint4 *)stage_v);
+        tier_copy_kernel<512><<<g3, kCopyThreads, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv,
+                                                               head_stride_bytes, tile_cap, p.chunk, s,
+                                                               (uint4 *)stage_k, (uint4 *)stage_v);
     const long long marks = (long long)n_bg * (qb1 - qb0) * p.topk;
     const unsigned g1 = (unsigned)((marks + 255) / 256 > 1184 ? 1184 : (marks + 255) / 256);
     if (marks > 0)

@@ -245,6 +245,19 @@ hga_status_t hga_attn_bwd_causal(const hga_params_t *p, const void *q, const voi
                                  const float *lse, const void *dout, void *dq, void *dk_seg, void *dv_seg,
                                  void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* hga_route then hga_attn_fwd in one call, overlapped (technical summary
+ * section 2.1: the block routes, then attends its routed chunks and its local
+ * window).  idx gets the routes exactly as from hga_route.  The attention is
+ * launched as a programmatic dependent of the route kernel: it starts while
+ * the route grid is still running, takes the causal segment tiles first (they
+ * need no route) and waits for the route grid before the routed history
+ * tiles.  out / lse agree with hga_route + hga_attn_fwd within rounding (the
+ * tiles are summed in another order), not bit for bit.  Arguments and errors
+ * as the two calls; fp32 and bf16 head_dim 64 run the two calls in order. */
+hga_status_t hga_route_attn_fwd(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
+                                int32_t *idx, const void *k_hist, const void *v_hist, const void *k_seg,
+                                const void *v_seg, void *out, float *lse, cudaStream_t stream);
+
 /* Bytes of device workspace hga_attn_bwd needs (fp32 row terms
  * delta = rowsum(dO * O), [B][Hq][S]).  Returns 0 for an invalid p. */
 size_t hga_attn_bwd_workspace_size(const hga_params_t *p);

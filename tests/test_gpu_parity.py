@@ -502,3 +502,55 @@ def test_tiered_rejects_pageable_host_memory_before_any_launch():
     # nothing was enqueued: scratch, staging and the remapped routes are untouched
     assert torch.all(scratch == 123) and torch.all(idx_r == -5) and torch.all(stage_k == 0)
     assert hga.hga_get_device_status() == 0
+
+
+# ---------------------------------------------------------------- route + attention in one call
+
+@pytest.mark.parametrize("w", [MID, W["tiny_fp32"], *EDGE], ids=[w.name for w in [MID, W["tiny_fp32"], *EDGE]])
+def test_route_attn_fwd_matches_route_then_oracle(w):
+    """hga_route_attn_fwd writes the same routes as hga_route (bit for bit) and its
+    attention, which runs the causal segment tiles before the routed ones and
+    overlaps the route, matches the oracle on those routes."""
+    import hierarchical_sparse_long_b200 as hga
+    arrs = hc.segment_arrays(w, 0)
+    g = hc.GpuSegment(w, arrs)
+    summ = g.summaries()
+    idx_a = g.route(summ)
+    idx_b = torch.full_like(idx_a, -9)
+    out = torch.full_like(g.q, float("nan"))
+    lse = torch.full(g.q.shape[:3], float("nan"), device="cuda")
+    hga.hga_route_attn_fwd(g.p, g.q, summ, g.cap, idx_b, g.k_all, g.v_all, g.k_seg, g.v_seg, out, lse)
+    torch.cuda.synchronize()
+    assert torch.equal(idx_a, idx_b)
+    T = arrs["T"]
+    sh = hc.oracle_shape(w, T)
+    out_o, lse_o = oracle.attn_fwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                                   arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], hc.f32(idx_b).astype(np.int32))
+    hc.compare(hc.f32(out), out_o, w.dtype, f"{w.name} out")
+    hc.compare(hc.f32(lse), lse_o, "fp32" if w.dtype == "fp32" else "bf16", f"{w.name} lse")
+
+
+@pytest.mark.parametrize("name,seg,n", [("qwen3_16k_fwd", 0, 256), ("qwen3_128k_eval", 31, 128)])
+def test_route_attn_fwd_full_size_sampled(name, seg, n):
+    import hierarchical_sparse_long_b200 as hga
+    w = W[name]
+    arrs = hc.segment_arrays(w, seg)
+    g = hc.GpuSegment(w, arrs)
+    summ = g.summaries()
+    idx = torch.empty(w.batch, w.n_kv_heads, w.seg_len // 64, w.topk, device="cuda", dtype=torch.int32)
+    out = torch.empty_like(g.q)
+    lse = torch.empty(g.q.shape[:3], device="cuda")
+    hga.hga_route_attn_fwd(g.p, g.q, summ, g.cap, idx, g.k_all, g.v_all, g.k_seg, g.v_seg, out, lse)
+    torch.cuda.synchronize()
+    sh, _, idx_o, gap = hc.oracle_route(w, arrs)
+    hard, _ = hc.route_mismatches(hc.f32(idx).astype(np.int32), idx_o, gap)
+    assert hard == 0
+    T = arrs["T"]
+    rows = _sampled_rows(w, n, seed=seg + 100)
+    out_o, lse_o = oracle.attn_fwd(sh, arrs["q"], arrs["k_all"][:, :, :T], arrs["v_all"][:, :, :T],
+                                   arrs["k_all"][:, :, T:], arrs["v_all"][:, :, T:], hc.f32(idx).astype(np.int32),
+                                   rows=rows)
+    D = w.head_dim
+    hc.compare(hc.f32(out).reshape(-1, D)[rows], out_o.reshape(-1, D)[rows], "bf16", f"{name} out")
+    hc.compare(hc.f32(lse).reshape(-1)[rows], lse_o.reshape(-1)[rows], "bf16", f"{name} lse")
+    assert hga.hga_get_device_status() == 0
