@@ -15,15 +15,16 @@ with the recipe of inputs/gen.py):
 * ``qwen3_128k_eval``: one step = a 131,072-token evaluation as 32 segments of
   4,096 tokens, top-32 chunks, each route + forward + summary append.
 * ``qwen3_128k_tiered``: the 128K evaluation with detached history K/V in
-  pinned host memory: each segment routes, then ``hga_attn_fwd_tiered`` fetches
-  the routed chunks wave by wave (32 query blocks per wave) into a device
-  staging cache on a side stream, overlapped with the attention of the
-  previous wave; the cache holds one segment's routing budget of chunk tiles
-  and keeps them from segment to segment (it is emptied when the 131,072-token
-  evaluation starts), so a routed chunk crosses the host link only when the
-  cache does not hold it; the segment's K/V are then offloaded to the host on
-  the copy stream (ordered before the next segment's fetches) and its
-  summaries appended.
+  pinned host memory: each segment's route and the fetch of its routed chunks
+  into a device staging cache run on a copy stream, under the attention of
+  the segment before it (``hga_attn_fwd_tiered`` chained from segment to
+  segment, one fetch wave of 64 query blocks per segment by default); the
+  cache holds one segment's routing budget of chunk tiles and keeps them from
+  segment to segment (it is emptied when the 131,072-token evaluation
+  starts), so a routed chunk crosses the host link only when the cache does
+  not hold it; the segment's K/V are offloaded to the host on a third stream
+  (ordered before the next segment's fetches) and its summaries appended on
+  the copy stream.
 * ``qwen3_128k_decode``: generation at 128K context: 16 sequences each add one
   token after 131,008 detached history tokens; a step routes the 16 tokens
   (one-token query blocks) and runs the split-K decode attention over their 32
@@ -97,7 +98,9 @@ def parse():
                     help="run each segment's summary append after its attention on the main stream "
                          "(default: on a side stream, overlapped with the route)")
     ap.add_argument("--cpu-seconds", type=float, default=12.0, help="target CPU time of the oracle sample")
-    ap.add_argument("--tier-wave", type=int, default=32, help="query blocks per fetch wave of the tiered workload")
+    ap.add_argument("--tier-wave", type=int, default=64, help="query blocks per fetch wave of the tiered workload")
+    ap.add_argument("--tier-lag", type=int, default=2,
+                    help="a tiered fetch wave waits for the attention this many waves back (2..4)")
     ap.add_argument("--only-last-segment", action="store_true",
                     help="a step processes only the workload's last segment (its history summarised up "
                          "front): for counter captures of the longest launches with few launches before them")
@@ -242,7 +245,8 @@ class Layer:
     head (history and active segment are views), resident chunk summaries, and
     the queries (and upstream gradients) of every processed segment."""
 
-    wave = 32  # query blocks per tiered fetch wave
+    wave = 64  # query blocks per tiered fetch wave
+    lag = 2  # a tiered fetch waits for the attention this many waves back
 
     def __init__(self, w):
         import torch
@@ -358,44 +362,46 @@ class Layer:
         p0 = self.params(w.seg_starts[-1])
         self.scratch = torch.empty(hga.hga_tier_scratch_size(p0, self.slots) // 4, device="cuda",
                                    dtype=torch.int32)
-        self.idx_r = torch.empty_like(self.idx)
         self.n_waves = -(-nqb // self.wave)
+        # the fetch of a wave rewrites its blocks' remapped routes once the attention
+        # `lag` waves back is done: chained segments rotate enough buffers
+        self.idx_r = [torch.empty_like(self.idx) for _ in range(-(-self.lag // self.n_waves))]
         self.n_fetched = torch.zeros(len(w.seg_starts), self.n_waves, device="cuda", dtype=torch.int32)
         self.copy_stream = torch.cuda.Stream()
         self.offload_stream = torch.cuda.Stream()
-        self.tier_events = [torch.cuda.Event() for _ in range(5)]
+        self.sched = hga.TierSched(lag=self.lag)
 
     def segment_tiered(self, T, ev=None, q=None, si=0):
-        """The same segment with the history only in pinned host memory: the
-        segment's K/V start their copy to the host history on an offload stream
-        (one 2-D copy each for K and V; only later segments read those rows, and
-        the next segment waits for it before it routes), then route, then
-        attention over the staging cache with the fetch waves overlapped
-        (hga_attn_fwd_tiered; the cache is emptied at the first segment only),
-        then the summary append."""
-        torch, hga, w = self.torch, self.hga, self.w
+        """The same segment with the history only in pinned host memory, one
+        hga_segment_fwd_tiered call on three streams: the route, the fetch of the
+        routed tiles (chained from segment to segment over the staging cache, the
+        cache emptied at the first segment only) and the summary append on the
+        copy stream, the segment's K/V offload to the host history on a third,
+        the attention on the compute stream -- so a segment's route and fetches
+        run under the attention of the segment before it.  The segment's q, K and
+        V are resident, or were copied in on the copy stream."""
+        hga, w = self.hga, self.w
         p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
-        rec = ev.record if ev is not None else (lambda name: None)
-        compute = torch.cuda.current_stream()
-        compute.wait_stream(self.offload_stream)  # the previous segment is in the host history
-        self.offload_stream.wait_stream(compute)  # this segment's K/V are ready
-        hga.hga_tier_offload(p, ks, vs, self.host_k, self.host_v, T, stream=self.offload_stream)
-        rec("route")
-        hga.hga_route(p, q, self.summ, self.nct, self.idx)
-        rec("attn_fwd")
-        first = T == w.seg_starts[0]
-        hga.hga_attn_fwd_tiered(p, q, self.host_k, self.host_v, ks, vs, self.idx, self.out, self.lse, self.stage_k,
-                                self.stage_v, self.slots, self.scratch, self.idx_r, self.wave, self.tier_events,
-                                reset_cache=first, n_fetched=self.n_fetched[si], copy_stream=self.copy_stream)
-        launches = 1 + int(first) + (1 if T == 0 else 4 * self.n_waves)
-        # detach: the segment's chunks become routable
-        rec("summaries")
-        hga.hga_build_summaries(self.k, self.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
-                                w.seg_len // w.chunk, self.summ, self.nct)
-        rec(None)
-        return launches + 1
+        if ev is not None:
+            ev.record("attn_fwd")
+        first = si == 0
+        hga.hga_segment_fwd_tiered(p, q, ks, vs, self.summ, self.nct, self.idx, self.host_k, self.host_v, self.out,
+                                   self.lse, self.stage_k, self.stage_v, self.slots, self.scratch,
+                                   self.idx_r[si % len(self.idx_r)], self.wave, self.sched, reset=first,
+                                   n_fetched=self.n_fetched[si], copy_stream=self.copy_stream,
+                                   offload_stream=self.offload_stream)
+        if ev is not None:
+            ev.record(None)
+        # route, reset (first segment), fetch waves (plan, copy, remap) + attention, append
+        return 1 + int(first) + (1 if T == 0 else 4 * self.n_waves) + 1
+
+    def end_tiered_step(self):
+        """The step ends when the side streams' work (the last append and offload) has."""
+        compute = self.torch.cuda.current_stream()
+        compute.wait_stream(self.copy_stream)
+        compute.wait_stream(self.offload_stream)
 
     def fetch_only_step(self):
         """Route + every fetch wave of every segment on the copy stream, no attention
@@ -416,7 +422,7 @@ class Layer:
                 hga.hga_tier_reset(p, self.slots, self.scratch, stream=self.copy_stream)
             for wi, b0 in enumerate(range(0, nqb, self.wave)):
                 hga.hga_fetch_tiered(p, self.host_k, self.host_v, self.idx, b0, min(b0 + self.wave, nqb),
-                                     self.stage_k, self.stage_v, self.slots, self.scratch, self.idx_r,
+                                     self.stage_k, self.stage_v, self.slots, self.scratch, self.idx_r[0],
                                      self.n_fetched[si, wi:wi + 1], copy_stream=self.copy_stream)
             compute.wait_stream(self.copy_stream)
         e.record(compute)
@@ -446,8 +452,8 @@ class Layer:
         n = 0
         for si, T in enumerate(self.w.seg_starts):
             n += self.segment_tiered(T, ev, si=si) if self.w.tiered else self.segment(T, ev)
-        if self.w.tiered:  # the last offload belongs to the step
-            self.torch.cuda.current_stream().wait_stream(self.offload_stream)
+        if self.w.tiered:  # the last append and offload belong to the step
+            self.end_tiered_step()
         return n
 
 
@@ -728,6 +734,7 @@ def measure_layer(w, args, world, local):
     import torch
     import hierarchical_sparse_long_b200 as hga
     Layer.wave = args.tier_wave
+    Layer.lag = args.tier_lag
     if args.only_last_segment:
         import dataclasses
         w = dataclasses.replace(w, seg_starts=w.seg_starts[-1:])
@@ -738,8 +745,9 @@ def measure_layer(w, args, world, local):
         flush_l2(flush)
         layer.step()
     torch.cuda.synchronize()
-    if hga.hga_get_device_status() != 0:
-        raise RuntimeError(f"{w.name}: device status reported an error during warm-up")
+    bits = hga.hga_get_device_status()
+    if bits != 0:
+        raise RuntimeError(f"{w.name}: device status bits {bits:#x} during warm-up")
     # Device-resident workloads replay one step captured as a CUDA graph (one
     # host launch per step; the route and the forward in one call, the forward
     # overlapping the route's tail); the tiered workload drives its copy stream
@@ -810,17 +818,21 @@ def measure_layer(w, args, world, local):
     kernels = {
         "attn_fwd": {"bound": "tensor", "ms_per_launch": ph["attn_fwd"] / n_seg,
                      "achieved": fwd_fl / (ph["attn_fwd"] / 1e3) / 1e12, "unit": "TFLOP/s"},
-        "route": {"bound": "hbm", "ms_per_launch": ph["route"] / n_seg,
-                  "achieved": sum(route_bytes(w, T) for T in w.seg_starts) * args.steps / (ph["route"] / 1e3) / 1e9,
-                  "unit": "GB/s"},
-        "summaries": {"bound": "hbm", "ms_per_launch": ph["summaries"] / n_seg,
-                      "achieved": summaries_bytes(w) * n_seg / (ph["summaries"] / 1e3) / 1e9, "unit": "GB/s"},
     }
+    if "route" in ph:
+        kernels["route"] = {"bound": "hbm", "ms_per_launch": ph["route"] / n_seg,
+                            "achieved": sum(route_bytes(w, T) for T in w.seg_starts) * args.steps /
+                            (ph["route"] / 1e3) / 1e9, "unit": "GB/s"}
+    if "summaries" in ph:
+        kernels["summaries"] = {"bound": "hbm", "ms_per_launch": ph["summaries"] / n_seg,
+                                "achieved": summaries_bytes(w) * n_seg / (ph["summaries"] / 1e3) / 1e9,
+                                "unit": "GB/s"}
     if layer.side_append:
         kernels["summaries"]["note"] = "on a side stream, timed while it overlaps the route"
     if w.tiered:
-        kernels["attn_fwd"]["note"] = "hga_attn_fwd_tiered: includes the waits for the fetch waves it cannot hide"
-        kernels["summaries"]["note"] = "includes the segment K/V copy to host memory"
+        kernels["attn_fwd"]["note"] = "the compute stream's share of hga_segment_fwd_tiered: the attention " \
+                                      "waves and the waits for the fetches they cannot hide (the route, " \
+                                      "fetches, append and offload run on two side streams)"
     if w.backward:
         bwd_fl = sum(attn_bwd_flops(w, T) for T in w.seg_starts) * args.steps
         kernels["attn_bwd"] = {"bound": "tensor", "ms_per_launch": ph["attn_bwd"] / n_seg,
@@ -843,11 +855,13 @@ def measure_layer(w, args, world, local):
                       "launch": "one CUDA graph replay per step" if graph is not None else "eager",
                       "route_and_forward": "hga_route_attn_fwd (one call, the forward a programmatic "
                                            "dependent of the route)" if not w.tiered else
-                                           "hga_route, then hga_attn_fwd_tiered",
+                                           "hga_segment_fwd_tiered (route and fetches on a copy stream, "
+                                           "chained across segments)",
                       "kernel_times": "from as many replays of the same step with CUDA events between its "
                                       "library calls (route and forward then issued apart), after the "
                                       "timed region",
-                      "append": "side stream, overlapped with the route" if layer.side_append else "in order"},
+                      "append": "side stream, overlapped with the route" if layer.side_append else
+                                ("copy stream, overlapped with the attention" if w.tiered else "in order")},
            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
            "device_status": status}
     if w.tiered:
@@ -890,7 +904,8 @@ def tiered_report(layer, step_ms, attn_phase_ms, flush):
     hidden = (t_fetch + t_res - attn_phase_ms) / t_res if t_res > 0 else None
     return {"staging_slots": layer.slots, "staging_mib": round(layer.slots * tb / 2**20, 1),
             "cache_policy": "one segment's routing budget of chunk tiles, kept from segment to segment and "
-                            f"emptied when the evaluation starts; waves of {layer.wave} query blocks",
+                            f"emptied when the evaluation starts; waves of {layer.wave} query blocks, a fetch "
+                            f"after the attention {layer.lag} waves back",
             "tiles_fetched_per_step": fetched, "tiles_distinct_per_segment_summed": per_segment,
             "tiles_distinct_per_step": whole,
             "bytes_fetched_per_step": fetched * tb, "bytes_distinct_per_segment_summed": per_segment * tb,
@@ -916,7 +931,10 @@ def e2e_measure(layer, steps):
                      ([layer.do[T].cpu().pin_memory()] if w.backward else [])
     outs = [layer.out, layer.lse] + ([layer.dq, layer.dk, layer.dv] if w.backward else [])
     host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
-    q_d = torch.empty_like(layer.q[w.seg_starts[0]])
+    # the tiered step runs each segment's route and fetches under the attention of the
+    # segment before it: its inputs arrive on the copy stream, q in a ring of three
+    # buffers (the copy stream reaches segment s only after the attention of s - 3)
+    q_ring = [torch.empty_like(layer.q[w.seg_starts[0]]) for _ in range(3 if w.tiered else 1)]
     do_d = torch.empty_like(layer.do[w.seg_starts[0]]) if w.backward else None
     h2d = sum(t.numel() * t.element_size() for ts in host_in.values() for t in ts)
     d2h = sum(t.numel() * t.element_size() for t in outs) * len(w.seg_starts)
@@ -927,11 +945,15 @@ def e2e_measure(layer, steps):
         s.record()
         for si, T in enumerate(w.seg_starts):
             hi = host_in[T]
-            q_d.copy_(hi[0], non_blocking=True)
-            layer.k[:, :, T:T + S].copy_(hi[1], non_blocking=True)
-            layer.v[:, :, T:T + S].copy_(hi[2], non_blocking=True)
-            if do_d is not None:
-                do_d.copy_(hi[3], non_blocking=True)
+            q_d = q_ring[si % len(q_ring)]
+            if w.tiered and si == 0:
+                layer.copy_stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(layer.copy_stream if w.tiered else torch.cuda.current_stream()):
+                q_d.copy_(hi[0], non_blocking=True)
+                layer.k[:, :, T:T + S].copy_(hi[1], non_blocking=True)
+                layer.v[:, :, T:T + S].copy_(hi[2], non_blocking=True)
+                if do_d is not None:
+                    do_d.copy_(hi[3], non_blocking=True)
             if w.tiered:
                 layer.segment_tiered(T, q=q_d, si=si)
             else:
@@ -939,7 +961,7 @@ def e2e_measure(layer, steps):
             for hbuf, t in zip(host_out, outs):
                 hbuf.copy_(t, non_blocking=True)
         if w.tiered:
-            torch.cuda.current_stream().wait_stream(layer.offload_stream)
+            layer.end_tiered_step()
         e.record()
         e.synchronize()
         if it >= 1:

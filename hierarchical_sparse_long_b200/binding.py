@@ -18,15 +18,17 @@ LIB_PATH = os.path.join(_PKG, "libhga.so")
 
 HGA_BF16, HGA_FP32 = 0, 1
 HGA_DEV_BAD_INDEX, HGA_DEV_TIMEOUT, HGA_DEV_STAGE_FULL = 1, 2, 4
+HGA_TIER_RESET, HGA_TIER_CHAIN = 1, 2
 STATUS = {0: "HGA_OK", -1: "HGA_ERR_INVALID_ARG", -2: "HGA_ERR_UNSUPPORTED", -3: "HGA_ERR_CUDA",
           -4: "HGA_ERR_DEVICE_CHECK", -5: "HGA_ERR_TIMEOUT"}
 
-EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd",
+EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_route_groups_tiered",
+            "hga_attn_fwd",
             "hga_route_attn_fwd",
             "hga_attn_bwd_workspace_size", "hga_attn_bwd", "hga_attn_fwd_groups", "hga_attn_bwd_groups",
             "hga_attn_causal_workspace_size", "hga_attn_fwd_causal", "hga_attn_bwd_causal",
             "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_tier_scratch_size",
-            "hga_tier_reset", "hga_fetch_tiered", "hga_tier_offload", "hga_attn_fwd_tiered",
+            "hga_tier_reset", "hga_fetch_tiered", "hga_tier_offload", "hga_attn_fwd_tiered", "hga_segment_fwd_tiered",
             "hga_get_device_status", "hga_selftest_wait_timeout", "hga_status_string", "hga_last_error")
 
 
@@ -89,6 +91,7 @@ def lib() -> ctypes.CDLL:
         L.hga_route.argtypes = [pp, vp, vp, i, vp, vp]
         L.hga_route_causal.argtypes = [pp, vp, vp, i, vp, vp]
         L.hga_route_groups.argtypes = [pp, vp, vp, i, vp, i, i, vp, vp]
+        L.hga_route_groups_tiered.argtypes = [pp, vp, vp, i, vp, i, i, vp, vp, i, vp, vp, vp, vp]
         L.hga_attn_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_route_attn_fwd.argtypes = [pp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, vp]
         L.hga_attn_fwd_groups.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, i, vp, vp, vp]
@@ -110,14 +113,17 @@ def lib() -> ctypes.CDLL:
         L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
         L.hga_tier_offload.argtypes = [pp, vp, vp, vp, vp, ll, vp]
         L.hga_attn_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp, vp, vp,
-                                          ctypes.POINTER(vp)]
+                                          ctypes.POINTER(_TierSchedC)]
+        L.hga_segment_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp,
+                                             vp, vp, vp, ctypes.POINTER(_TierSchedC)]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hga_selftest_wait_timeout.argtypes = [ll, vp]
         L.hga_selftest_wait_timeout.restype = ctypes.c_int
         L.hga_status_string.argtypes = [i]
         L.hga_status_string.restype = ctypes.c_char_p
         L.hga_last_error.restype = ctypes.c_char_p
-        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups", "hga_attn_fwd",
+        for f in ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_groups",
+                  "hga_route_groups_tiered", "hga_attn_fwd",
                   "hga_attn_bwd", "hga_attn_bwd_noalloc", "hga_attn_fwd_groups", "hga_attn_bwd_groups",
                   "hga_route_attn_fwd",
                   "hga_attn_fwd_causal", "hga_attn_bwd_causal",
@@ -184,6 +190,17 @@ def hga_route_groups(p: Params, q, gsumm, gsumm_cap_groups: int, idx, group: int
     cp = p.c()
     _check(lib().hga_route_groups(ctypes.byref(cp), _ptr(q), _ptr(gsumm), gsumm_cap_groups, _ptr(idx), group,
                                   topg, _ptr(gidx), _stream(stream)), "hga_route_groups")
+
+
+def hga_route_groups_tiered(p: Params, q, host_gsumm, gsumm_cap_groups: int, idx, group: int, topg: int, gidx,
+                            stage_gsumm, stage_slots: int, scratch, idx_remapped, n_fetched=None, stream=None):
+    """hga_route_groups from a device cache of group summaries whose misses are
+    fetched from pinned host memory (p.hist_head_stride = gsumm_cap_groups * group)."""
+    cp = p.c()
+    _check(lib().hga_route_groups_tiered(ctypes.byref(cp), _ptr(q), _ptr(host_gsumm), gsumm_cap_groups, _ptr(idx),
+                                         group, topg, _ptr(gidx), _ptr(stage_gsumm), stage_slots, _ptr(scratch),
+                                         _ptr(idx_remapped), _ptr(n_fetched), _stream(stream)),
+           "hga_route_groups_tiered")
 
 
 def hga_attn_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stream=None):
@@ -321,21 +338,77 @@ def hga_tier_offload(p: Params, k_seg, v_seg, host_k, host_v, dst_token: int, st
                                   dst_token, _stream(stream)), "hga_tier_offload")
 
 
-def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v,
-                        stage_slots: int, scratch, idx_remapped, wave_blocks: int, events, reset_cache=False,
-                        n_fetched=None, stream=None, copy_stream=None):
-    """Attention over host-resident history: fetch waves on copy_stream overlapped with
-    the attention of the previous wave on stream (events: five torch.cuda.Event)."""
-    cp = p.c()
-    for e in events:
-        if not e.cuda_event:  # torch creates its CUDA event on the first record
+class _TierSchedC(ctypes.Structure):
+    _fields_ = [("start", ctypes.c_void_p), ("fetched", ctypes.c_void_p), ("consumed", ctypes.c_void_p * 4),
+                ("inputs", ctypes.c_void_p), ("offloaded", ctypes.c_void_p * 2), ("lag", ctypes.c_int),
+                ("wave", ctypes.c_longlong), ("segment", ctypes.c_longlong)]
+
+
+class TierSched:
+    """hga_tier_sched_t: the cross-stream schedule of hga_attn_fwd_tiered over one
+    staging cache -- torch events the library records, the lag (the fetch of wave h
+    waits for the attention of wave h - lag) and the wave counter it advances."""
+
+    MAX_LAG = 4
+
+    def __init__(self, lag: int = 2):
+        import torch
+        if not 2 <= lag <= self.MAX_LAG:
+            raise ValueError(f"lag must be in 2..{self.MAX_LAG}")
+        self.events = [torch.cuda.Event() for _ in range(5 + lag)]
+        for e in self.events:  # torch creates its CUDA event on the first record
             e.record()
-    evs = (ctypes.c_void_p * 5)(*[e.cuda_event for e in events])
+        h = [e.cuda_event for e in self.events]
+        self.c = _TierSchedC()
+        self.c.start, self.c.fetched, self.c.inputs = h[0], h[1], h[2]
+        self.c.offloaded[0], self.c.offloaded[1] = h[3], h[4]
+        for i in range(lag):
+            self.c.consumed[i] = h[5 + i]
+        self.c.lag = lag
+        self.c.wave = 0
+        self.c.segment = 0
+
+    @property
+    def lag(self) -> int:
+        return self.c.lag
+
+    @property
+    def wave(self) -> int:
+        return self.c.wave
+
+    @property
+    def segment(self) -> int:
+        return self.c.segment
+
+
+def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v,
+                        stage_slots: int, scratch, idx_remapped, wave_blocks: int, sched: TierSched,
+                        reset_cache=False, chain=False, n_fetched=None, stream=None, copy_stream=None):
+    """Attention over host-resident history: fetch waves on copy_stream overlapped with
+    earlier waves' attention on stream, ordered by sched (a TierSched)."""
+    cp = p.c()
+    flags = (HGA_TIER_RESET if reset_cache else 0) | (HGA_TIER_CHAIN if chain else 0)
     _check(lib().hga_attn_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(host_k), _ptr(host_v), _ptr(k_seg),
                                      _ptr(v_seg), _ptr(idx), _ptr(out), _ptr(lse), _ptr(stage_k), _ptr(stage_v),
-                                     stage_slots, _ptr(scratch), _ptr(idx_remapped), wave_blocks,
-                                     1 if reset_cache else 0, _ptr(n_fetched), _stream(stream),
-                                     _stream(copy_stream), evs), "hga_attn_fwd_tiered")
+                                     stage_slots, _ptr(scratch), _ptr(idx_remapped), wave_blocks, flags,
+                                     _ptr(n_fetched), _stream(stream), _stream(copy_stream), ctypes.byref(sched.c)),
+           "hga_attn_fwd_tiered")
+
+
+def hga_segment_fwd_tiered(p: Params, q, k_seg, v_seg, summ, summ_cap_chunks: int, idx, host_k, host_v, out, lse,
+                           stage_k, stage_v, stage_slots: int, scratch, idx_remapped, wave_blocks: int,
+                           sched: TierSched, reset=False, n_fetched=None, stream=None, copy_stream=None,
+                           offload_stream=None):
+    """One segment of a tiered evaluation: route, fetches and summary append on
+    copy_stream, the K/V offload on offload_stream, attention on stream."""
+    cp = p.c()
+    _check(lib().hga_segment_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(summ),
+                                        summ_cap_chunks, _ptr(idx), _ptr(host_k), _ptr(host_v), _ptr(out), _ptr(lse),
+                                        _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(scratch),
+                                        _ptr(idx_remapped), wave_blocks, HGA_TIER_RESET if reset else 0,
+                                        _ptr(n_fetched), _stream(stream), _stream(copy_stream),
+                                        _stream(offload_stream), ctypes.byref(sched.c)),
+           "hga_segment_fwd_tiered")
 
 
 def hga_selftest_wait_timeout(wait_cycles: int, stream=None):

@@ -146,6 +146,46 @@ hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float 
     return hga::launch_route_groups(*p, q, gsumm, gsumm_cap_groups, idx, group, topg, gidx, stream);
 }
 
+hga_status_t hga_route_groups_tiered(const hga_params_t *p, const void *q, const float *host_gsumm,
+                                     int gsumm_cap_groups, const int32_t *idx, int group, int topg, int32_t *gidx,
+                                     float *stage_gsumm, int stage_slots, int32_t *scratch, int32_t *idx_remapped,
+                                     int32_t *n_fetched, cudaStream_t stream) {
+    CallRange range("hga_route_groups_tiered");
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;
+    if (group != 8 && group != 16 && group != 32) return HGA_ERR_INVALID_ARG;
+    const int gpc = p->chunk / group;
+    if (topg < 1 || topg > p->topk * gpc) return HGA_ERR_INVALID_ARG;
+    if ((long long)gsumm_cap_groups < (long long)p->n_hist_chunks * gpc) return HGA_ERR_INVALID_ARG;
+    // the cache's tiles are (b, g, chunk) of the group-summary history
+    if (p->hist_head_stride != (long long)gsumm_cap_groups * group || gsumm_cap_groups % gpc) {
+        hga::record_error("hga_route_groups_tiered: hist_head_stride must be gsumm_cap_groups * group "
+                          "(a whole number of chunks)");
+        return HGA_ERR_INVALID_ARG;
+    }
+    if (!q || !idx || !gidx || !host_gsumm || !stage_gsumm || !scratch || !idx_remapped || stage_slots < 1)
+        return HGA_ERR_INVALID_ARG;
+    for (const void *ptr : {q, (const void *)host_gsumm, (const void *)stage_gsumm})
+        if (!aligned16(ptr)) return HGA_ERR_INVALID_ARG;
+    const int keff = p->topk < p->n_hist_chunks ? p->topk : p->n_hist_chunks;
+    const long long worst = 2ll * (p->seg_len / p->q_block) * p->batch * p->n_kv_heads * keff;
+    const long long distinct = (long long)p->batch * p->n_kv_heads * p->n_hist_chunks;
+    if ((worst < distinct ? worst : distinct) > stage_slots) {
+        hga::record_error("hga_route_groups_tiered: stage_slots below twice the chunks one call can route "
+                          "(or every routable chunk)");
+        return HGA_ERR_INVALID_ARG;
+    }
+    unsigned *status = status_ptr();
+    if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
+    if (p->n_hist_chunks > 0) {
+        st = hga::launch_fetch_group_summaries(*p, host_gsumm, group, idx, stage_gsumm, stage_slots, scratch,
+                                               idx_remapped, n_fetched, status, stream);
+        if (st != HGA_OK) return st;
+    }
+    return hga::launch_route_groups(*p, q, stage_gsumm, 0, idx, group, topg, gidx, stream, idx_remapped);
+}
+
 hga_status_t hga_route_causal(const hga_params_t *p, const void *q, const float *summ, int summ_cap_chunks,
                               int32_t *idx, cudaStream_t stream) {
     CallRange range("hga_route_causal");
@@ -432,11 +472,12 @@ namespace {
 
 // Argument checks shared by hga_fetch_tiered and hga_attn_fwd_tiered.  A
 // fetch of `blocks` query blocks may need every routed tile of those blocks,
-// and the tiles of the wave before it stay protected, so the cache must hold
-// twice that -- or every routable tile, after which nothing is ever evicted.
+// and the tiles of the lag - 1 waves before it stay protected, so the cache
+// must hold lag times that -- or every routable tile, after which nothing is
+// ever evicted.
 hga_status_t check_tiered(const hga_params_t *p, const void *host_k, const void *host_v, const int32_t *idx,
                           const void *stage_k, const void *stage_v, int stage_slots, const int32_t *scratch,
-                          const int32_t *idx_remapped, int blocks) {
+                          const int32_t *idx_remapped, int blocks, int lag) {
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
     if (p->q_block != 64) return HGA_ERR_UNSUPPORTED;  // one-token segments go through hga_attn_decode
@@ -447,10 +488,10 @@ hga_status_t check_tiered(const hga_params_t *p, const void *host_k, const void 
     for (const void *ptr : {host_k, host_v, stage_k, stage_v})
         if (!aligned16(ptr)) return HGA_ERR_INVALID_ARG;
     const int keff = p->topk < p->n_hist_chunks ? p->topk : p->n_hist_chunks;
-    const long long worst = 2ll * blocks * p->batch * p->n_kv_heads * keff;
+    const long long worst = (long long)lag * blocks * p->batch * p->n_kv_heads * keff;
     const long long distinct = (long long)p->batch * p->n_kv_heads * p->n_hist_chunks;
     if ((worst < distinct ? worst : distinct) > stage_slots) {
-        hga::record_error("tiered: stage_slots below twice the tiles one wave can route (or every routable tile)");
+        hga::record_error("tiered: stage_slots below lag times the tiles one wave can route (or every routable tile)");
         return HGA_ERR_INVALID_ARG;
     }
     return HGA_OK;
@@ -467,12 +508,12 @@ hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const v
     const int nqb = p->q_block > 0 ? p->seg_len / p->q_block : 0;
     if (qblock_begin < 0 || qblock_end <= qblock_begin || qblock_end > nqb) return HGA_ERR_INVALID_ARG;
     hga_status_t st = check_tiered(p, host_k, host_v, idx, stage_k, stage_v, stage_slots, scratch, idx_remapped,
-                                   qblock_end - qblock_begin);
+                                   qblock_end - qblock_begin, 2);
     if (st != HGA_OK) return st;
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
     st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, qblock_begin, qblock_end, stage_k, stage_v, stage_slots,
-                                  scratch, idx_remapped, n_fetched, status, copy_stream);
+                                  2, scratch, idx_remapped, n_fetched, status, copy_stream);
     if (st != HGA_OK) return st;
     if (done) return hga::record_cuda(cudaEventRecord(done, copy_stream));
     return HGA_OK;
@@ -511,17 +552,20 @@ hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const vo
 hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const void *host_k, const void *host_v,
                                  const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
                                  void *stage_k, void *stage_v, int stage_slots, int32_t *scratch,
-                                 int32_t *idx_remapped, int wave_blocks, int reset_cache, int32_t *n_fetched,
-                                 cudaStream_t stream, cudaStream_t copy_stream, const cudaEvent_t *events) {
+                                 int32_t *idx_remapped, int wave_blocks, int flags, int32_t *n_fetched,
+                                 cudaStream_t stream, cudaStream_t copy_stream, hga_tier_sched_t *sched) {
     CallRange range("hga_attn_fwd_tiered");
-    if (!p || wave_blocks < 1 || !events) return HGA_ERR_INVALID_ARG;
-    for (int e = 0; e < 5; ++e)
-        if (!events[e]) return HGA_ERR_INVALID_ARG;
+    if (!p || wave_blocks < 1 || !sched || (flags & ~(HGA_TIER_RESET | HGA_TIER_CHAIN))) return HGA_ERR_INVALID_ARG;
+    const int lag = sched->lag;
+    if (lag < 2 || lag > HGA_TIER_MAX_LAG || sched->wave < 0 || !sched->start || !sched->fetched)
+        return HGA_ERR_INVALID_ARG;
+    for (int i = 0; i < lag; ++i)
+        if (!sched->consumed[i]) return HGA_ERR_INVALID_ARG;
     const int nqb = p->q_block > 0 ? p->seg_len / p->q_block : 0;
     const int qb0 = (p->qblock_begin == 0 && p->qblock_end == 0) ? 0 : p->qblock_begin;
     const int qb1 = (p->qblock_begin == 0 && p->qblock_end == 0) ? nqb : p->qblock_end;
     hga_status_t st = check_tiered(p, host_k, host_v, idx, stage_k, stage_v, stage_slots, scratch, idx_remapped,
-                                   wave_blocks);
+                                   wave_blocks, lag);
     if (st != HGA_OK) return st;
     if (!q || !k_seg || !v_seg || !out || !lse) return HGA_ERR_INVALID_ARG;
     hga_params_t pa = *p;  // attention over the staging cache: route indices are slots
@@ -529,34 +573,101 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
     pa.n_hist_chunks = stage_slots;
     unsigned *status = status_ptr();
     if (!status) return hga::record_cuda(cudaErrorInvalidDevice);
-    // the copy stream starts after everything already on the compute stream
-    // (the route that wrote idx, the attention of earlier calls over the cache)
-    cudaError_t e = cudaEventRecord(events[0], stream);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(copy_stream, events[0], 0);
-    if (e != cudaSuccess) return hga::record_cuda(e);
-    if (reset_cache) {
+    const bool reset = (flags & HGA_TIER_RESET) != 0;
+    cudaError_t e = cudaSuccess;
+    if (reset || !(flags & HGA_TIER_CHAIN) || sched->wave == 0) {
+        // the copy stream starts after everything already on the compute stream
+        // (the route that wrote idx, the attention of earlier calls over the cache)
+        e = cudaEventRecord(sched->start, stream);
+        if (e == cudaSuccess) e = cudaStreamWaitEvent(copy_stream, sched->start, 0);
+        if (e != cudaSuccess) return hga::record_cuda(e);
+    }
+    if (reset) {
         st = hga::launch_tier_reset(*p, stage_slots, scratch, copy_stream);
         if (st != HGA_OK) return st;
+        sched->wave = 0;
     }
-    if (p->n_hist_chunks == 0)  // nothing routable: plain attention over the segment
+    if (p->n_hist_chunks == 0) {
+        // nothing routable: plain attention over the segment, after whatever the copy
+        // stream holds (the caller may have written idx or the inputs there)
+        if ((e = cudaEventRecord(sched->fetched, copy_stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(stream, sched->fetched, 0)) != cudaSuccess)
+            return hga::record_cuda(e);
         return hga_attn_fwd(p, q, stage_k, stage_v, k_seg, v_seg, idx, out, lse, stream);
-    for (int w = 0, b0 = qb0; b0 < qb1; ++w, b0 += wave_blocks) {
+    }
+    for (int b0 = qb0; b0 < qb1; b0 += wave_blocks) {
         const int b1 = b0 + wave_blocks < qb1 ? b0 + wave_blocks : qb1;
-        cudaEvent_t fetched = events[1 + (w & 1)], consumed = events[3 + (w & 1)];
-        // the fetch of wave w may evict slots last read by wave w - 2: wait for that attention
-        if (w >= 2 && (e = cudaStreamWaitEvent(copy_stream, consumed, 0)) != cudaSuccess) return hga::record_cuda(e);
-        st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, b0, b1, stage_k, stage_v, stage_slots, scratch,
-                                      idx_remapped, n_fetched ? n_fetched + w : nullptr, status, copy_stream);
+        const long long h = sched->wave;
+        cudaEvent_t consumed = sched->consumed[h % lag];
+        // the fetch of wave h may evict the slots wave h - lag read: wait for that attention
+        if (h >= lag && (e = cudaStreamWaitEvent(copy_stream, consumed, 0)) != cudaSuccess)
+            return hga::record_cuda(e);
+        st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, b0, b1, stage_k, stage_v, stage_slots, lag, scratch,
+                                      idx_remapped, n_fetched ? n_fetched + (b0 - qb0) / wave_blocks : nullptr,
+                                      status, copy_stream);
         if (st != HGA_OK) return st;
-        if ((e = cudaEventRecord(fetched, copy_stream)) != cudaSuccess ||
-            (e = cudaStreamWaitEvent(stream, fetched, 0)) != cudaSuccess)
+        if ((e = cudaEventRecord(sched->fetched, copy_stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(stream, sched->fetched, 0)) != cudaSuccess)
             return hga::record_cuda(e);
         pa.qblock_begin = b0;
         pa.qblock_end = b1;
         st = hga_attn_fwd(&pa, q, stage_k, stage_v, k_seg, v_seg, idx_remapped, out, lse, stream);
         if (st != HGA_OK) return st;
         if ((e = cudaEventRecord(consumed, stream)) != cudaSuccess) return hga::record_cuda(e);
+        sched->wave = h + 1;
     }
+    return HGA_OK;
+}
+
+hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const void *k_seg, const void *v_seg,
+                                    float *summ, int summ_cap_chunks, int32_t *idx, void *host_k, void *host_v,
+                                    void *out, float *lse, void *stage_k, void *stage_v, int stage_slots,
+                                    int32_t *scratch, int32_t *idx_remapped, int wave_blocks, int flags,
+                                    int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,
+                                    cudaStream_t offload_stream, hga_tier_sched_t *sched) {
+    CallRange range("hga_segment_fwd_tiered");
+    if (!p || !sched || (flags & ~HGA_TIER_RESET)) return HGA_ERR_INVALID_ARG;
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (!sched->inputs || !sched->offloaded[0] || !sched->offloaded[1] || sched->segment < 0)
+        return HGA_ERR_INVALID_ARG;
+    if (p->seg_len % p->chunk != 0) return HGA_ERR_INVALID_ARG;
+    const int seg_chunks = p->seg_len / p->chunk;
+    const long long T = (long long)p->n_hist_chunks * p->chunk;
+    if ((long long)p->n_hist_chunks + seg_chunks > summ_cap_chunks || T + p->seg_len > p->hist_head_stride)
+        return HGA_ERR_INVALID_ARG;
+    if (!summ || !aligned16(summ) || !k_seg || !aligned16(k_seg)) return HGA_ERR_INVALID_ARG;
+    const bool reset = (flags & HGA_TIER_RESET) != 0;
+    cudaError_t e = cudaSuccess;
+    if (reset) {  // the evaluation starts: the side streams after whatever came before it
+        if ((e = cudaEventRecord(sched->start, stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(copy_stream, sched->start, 0)) != cudaSuccess)
+            return hga::record_cuda(e);
+        sched->segment = 0;
+    }
+    const long long seg = sched->segment;
+    // detach into the host tier once the segment's K/V are there
+    if ((e = cudaEventRecord(sched->inputs, copy_stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(offload_stream, sched->inputs, 0)) != cudaSuccess)
+        return hga::record_cuda(e);
+    st = hga_tier_offload(p, k_seg, v_seg, host_k, host_v, T, offload_stream);
+    if (st != HGA_OK) return st;
+    if ((e = cudaEventRecord(sched->offloaded[seg & 1], offload_stream)) != cudaSuccess) return hga::record_cuda(e);
+    st = hga_route(p, q, summ, summ_cap_chunks, idx, copy_stream);
+    if (st != HGA_OK) return st;
+    // this segment's fetches read the rows the previous segment offloaded
+    if (seg > 0 && (e = cudaStreamWaitEvent(copy_stream, sched->offloaded[(seg - 1) & 1], 0)) != cudaSuccess)
+        return hga::record_cuda(e);
+    st = hga_attn_fwd_tiered(p, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v, stage_slots,
+                             scratch, idx_remapped, wave_blocks, reset ? HGA_TIER_RESET : HGA_TIER_CHAIN, n_fetched,
+                             stream, copy_stream, sched);
+    if (st != HGA_OK) return st;
+    // detach: the segment's chunks become routable for the next segment
+    st = hga::launch_summaries(k_seg, p->seg_head_stride, p->batch * p->n_kv_heads, p->head_dim, p->chunk,
+                               p->n_hist_chunks, seg_chunks, p->dtype, summ, summ_cap_chunks, copy_stream,
+                               p->n_hist_chunks);
+    if (st != HGA_OK) return st;
+    sched->segment = seg + 1;
     return HGA_OK;
 }
 

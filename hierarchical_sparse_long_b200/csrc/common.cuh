@@ -51,14 +51,24 @@ template <> struct Vec16<__nv_bfloat16> {
 // Host-side launchers (one translation unit each); all validate nothing --
 // the C ABI layer has already checked every argument.
 namespace hga {
+// k_first_chunk: the chunk index of k's first row (0: k is the start of each slice)
 hga_status_t launch_summaries(const void *k, long long head_stride, int bh, int head_dim, int chunk,
                               int first_chunk, int n_chunks, hga_dtype_t dtype, float *summ, int cap,
-                              cudaStream_t stream);
+                              cudaStream_t stream, int k_first_chunk = 0);
 hga_status_t launch_route(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
                           unsigned *status, cudaStream_t stream);
 // Group-stage routes (groups of `group` tokens in the chosen chunks): gidx [B][Hkv][S/q_block][topg].
+// slot_idx (may be null): the chunk routes remapped to staging slots of gsumm (one
+// shared slice of staged group summaries, chunk / group rows per slot).
 hga_status_t launch_route_groups(const hga_params_t &p, const void *q, const float *gsumm, long long cap,
-                                 const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream);
+                                 const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream,
+                                 const int32_t *slot_idx = nullptr);
+// One fetch of the group summaries of every block's routed chunks into a staging
+// cache (hga_route_groups_tiered); p.hist_head_stride = group summaries per (b, g) * group.
+hga_status_t launch_fetch_group_summaries(const hga_params_t &p, const float *host_gsumm, int group,
+                                          const int32_t *idx, float *stage, int stage_slots, int32_t *scratch,
+                                          int32_t *idx_remapped, int32_t *n_fetched, unsigned *status,
+                                          cudaStream_t stream);
 // Strictly causal routes, one per token: idx [B][Hkv][S][topk].
 hga_status_t launch_route_causal(const hga_params_t &p, const void *q, const float *summ, int cap, int32_t *idx,
                           unsigned *status, cudaStream_t stream);
@@ -137,7 +147,7 @@ size_t tier_scratch_entries(const hga_params_t &p, int stage_slots);
 hga_status_t launch_tier_reset(const hga_params_t &p, int stage_slots, int32_t *scratch, cudaStream_t stream);
 hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
-                                 int stage_slots, int32_t *scratch, int32_t *idx_remapped,
+                                 int stage_slots, int lag, int32_t *scratch, int32_t *idx_remapped,
                                  int32_t *n_fetched, unsigned *status, cudaStream_t stream);
 hga_status_t launch_selftest_wait_timeout(long long wait_cycles, unsigned *status, cudaStream_t stream);
 hga_status_t record_cuda(cudaError_t e);

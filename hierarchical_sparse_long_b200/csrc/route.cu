@@ -692,6 +692,9 @@ struct GroupArgs {
     const void *q;
     const float *gsumm;
     const int32_t *idx;
+    // staged group summaries: when set, chunk j = idx[.][a] has its groups at rows
+    // slot_idx[.][a] * gpc .. of one shared slice (cap = 0); ids and order still follow idx
+    const int32_t *slot_idx;
     int32_t *gidx;
     long long cap;  // group-summary rows per (b, g)
     int n_q_heads, n_kv_heads, seg_len, q_block, n, topk, gpc, topg;
@@ -704,7 +707,7 @@ __global__ void __launch_bounds__(kThreads, 1) route_groups_kernel(const GroupAr
     __shared__ float part[NRS][D];
     __shared__ __align__(16) float qbar[D];
     __shared__ uint32_t row[kMaxCand];
-    __shared__ int chunks[64], sel[kMaxCand], n_chunks;
+    __shared__ int chunks[64], rows[64], sel[kMaxCand], n_chunks;
     __shared__ __align__(16) uint32_t s_tmax[kThreads];  // select_cta reads it as 16-byte vectors
     __shared__ uint64_t s_key[kCandCap];
     __shared__ int s_cj[kCandCap], s_hist[256], s_misc[16];
@@ -730,16 +733,21 @@ __global__ void __launch_bounds__(kThreads, 1) route_groups_kernel(const GroupAr
     }
     if (tid == 0) {  // the block's chosen chunks, ascending (insertion sort of <= 64 ids)
         const int32_t *selc = a.idx + ((long long)bg * nqb + m) * a.topk;
+        const int32_t *slc = a.slot_idx ? a.slot_idx + ((long long)bg * nqb + m) * a.topk : nullptr;
         int nv = 0;
         for (int t = 0; t < a.topk; ++t) {
             const int j = selc[t];
             if (j < 0 || j >= a.n) continue;
+            if (slc && slc[t] < 0) continue;  // not staged
+            const int row = slc ? slc[t] : j;  // first summary row of the chunk's groups / gpc
             int p = nv++;
             while (p > 0 && chunks[p - 1] > j) {
                 chunks[p] = chunks[p - 1];
+                rows[p] = rows[p - 1];
                 --p;
             }
             chunks[p] = j;
+            rows[p] = row;
         }
         n_chunks = nv;
     }
@@ -753,14 +761,14 @@ __global__ void __launch_bounds__(kThreads, 1) route_groups_kernel(const GroupAr
 
     // scores of the candidate groups: one warp per candidate, D / 32 values per lane
     const int ncand = n_chunks * a.gpc;
-    const float *gbase = a.gsumm + (long long)bg * a.cap * D;
+    const float *gbase = a.gsumm + (a.slot_idx ? 0ll : (long long)bg * a.cap * D);
     constexpr int VPL = D / 32;
     float qv[VPL];
 #pragma unroll
     for (int e = 0; e < VPL; ++e) qv[e] = qbar[lane * VPL + e];
     for (int c = warp; c < ncand; c += kWarps) {
-        const int gid = chunks[c / a.gpc] * a.gpc + c % a.gpc;
-        const float *gr = gbase + (long long)gid * D + lane * VPL;
+        const int grow = rows[c / a.gpc] * a.gpc + c % a.gpc;  // summary row (slot-based when staged)
+        const float *gr = gbase + (long long)grow * D + lane * VPL;
         float acc = 0.f;
 #pragma unroll
         for (int e = 0; e < VPL; ++e) acc = fmaf(qv[e], gr[e], acc);
@@ -914,11 +922,13 @@ hga_status_t launch_route_causal(const hga_params_t &p, const void *q, const flo
 }
 
 hga_status_t launch_route_groups(const hga_params_t &p, const void *q, const float *gsumm, long long cap,
-                                 const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream) {
+                                 const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream,
+                                 const int32_t *slot_idx) {
     GroupArgs a{};
     a.q = q;
     a.gsumm = gsumm;
     a.idx = idx;
+    a.slot_idx = slot_idx;
     a.gidx = gidx;
     a.cap = cap;
     a.n_q_heads = p.n_q_heads;

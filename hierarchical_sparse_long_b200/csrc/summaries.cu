@@ -18,7 +18,8 @@ namespace hga {
 template <typename T, int D>
 __global__ void __launch_bounds__(256) summaries_kernel(const T *__restrict__ k, long long head_stride,
                                                         int n_slices, int chunk, int first_chunk,
-                                                        int n_chunks, float *__restrict__ summ, int cap) {
+                                                        int n_chunks, int k_first_chunk,
+                                                        float *__restrict__ summ, int cap) {
     constexpr int VEC = Vec16<T>::N;
     constexpr int LPR = D / VEC;     // threads per row
     constexpr int NSLOT = 256 / LPR; // row slots
@@ -29,7 +30,7 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T *__restrict__ k,
     const int j = first_chunk + (int)(blockIdx.x % n_chunks);
     const int col = (tid % LPR) * VEC;
     const int rslot = tid / LPR;
-    const T *base = k + ((long long)slice * head_stride + (long long)j * chunk) * D + col;
+    const T *base = k + ((long long)slice * head_stride + (long long)(j - k_first_chunk) * chunk) * D + col;
 
     float acc[VEC];
 #pragma unroll
@@ -63,25 +64,28 @@ __global__ void __launch_bounds__(256) summaries_kernel(const T *__restrict__ k,
 
 template <typename T, int D>
 static hga_status_t launch_t(const void *k, long long head_stride, int bh, int chunk, int first_chunk,
-                             int n_chunks, float *summ, int cap, cudaStream_t stream) {
+                             int n_chunks, int k_first_chunk, float *summ, int cap, cudaStream_t stream) {
     const long long blocks = (long long)bh * n_chunks;
     summaries_kernel<T, D><<<(unsigned)blocks, 256, 0, stream>>>(static_cast<const T *>(k), head_stride, bh,
-                                                                 chunk, first_chunk, n_chunks, summ, cap);
+                                                                 chunk, first_chunk, n_chunks, k_first_chunk,
+                                                                 summ, cap);
     return record_cuda(cudaGetLastError());
 }
 
 hga_status_t launch_summaries(const void *k, long long head_stride, int bh, int head_dim, int chunk,
                               int first_chunk, int n_chunks, hga_dtype_t dtype, float *summ, int cap,
-                              cudaStream_t stream) {
+                              cudaStream_t stream, int k_first_chunk) {
     if (n_chunks == 0 || bh == 0) return HGA_OK;
+    const int k0 = k_first_chunk;
     if (dtype == HGA_BF16) {
         if (head_dim == 128)
-            return launch_t<__nv_bfloat16, 128>(k, head_stride, bh, chunk, first_chunk, n_chunks, summ, cap, stream);
-        return launch_t<__nv_bfloat16, 64>(k, head_stride, bh, chunk, first_chunk, n_chunks, summ, cap, stream);
+            return launch_t<__nv_bfloat16, 128>(k, head_stride, bh, chunk, first_chunk, n_chunks, k0, summ, cap,
+                                                stream);
+        return launch_t<__nv_bfloat16, 64>(k, head_stride, bh, chunk, first_chunk, n_chunks, k0, summ, cap, stream);
     }
     if (head_dim == 128)
-        return launch_t<float, 128>(k, head_stride, bh, chunk, first_chunk, n_chunks, summ, cap, stream);
-    return launch_t<float, 64>(k, head_stride, bh, chunk, first_chunk, n_chunks, summ, cap, stream);
+        return launch_t<float, 128>(k, head_stride, bh, chunk, first_chunk, n_chunks, k0, summ, cap, stream);
+    return launch_t<float, 64>(k, head_stride, bh, chunk, first_chunk, n_chunks, k0, summ, cap, stream);
 }
 
 }  // namespace hga

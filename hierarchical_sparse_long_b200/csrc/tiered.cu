@@ -20,16 +20,18 @@
 // stream:
 //   plan   (one CTA): the wave's distinct tiles; cached ones are re-stamped
 //          with w, the others get free slots -- slots whose last reader is
-//          wave w-2 or older, taken round-robin from a cursor, evicting their
+//          wave w-lag or older, taken round-robin from a cursor, evicting their
 //          old tile -- and form the fetch list;
 //   copy   : an SM copy of each listed K and V tile straight from the mapped
 //          host pages into its slot (16-byte loads, many in flight, so the
 //          host link rather than the SMs is the bound; CTAs small enough to
 //          share an SM with an attention CTA);
 //   remap  : idx_remapped = slot of each routed chunk (-1 stays -1).
-// The caller guarantees that the attention of wave w-2 has finished before
+// The caller guarantees that the attention of wave w-lag has finished before
 // the fetch of wave w starts (hga_attn_fwd_tiered orders its two streams so);
-// the attention of wave w-1 may still run, and its slots are never evicted.
+// the attention of waves w-lag+1 .. w-1 may still run, and their slots are
+// never evicted.  lag is 2 for the single fetches (hga_fetch_tiered, the
+// group-summary cache).
 // The chunk order inside each block's route list is unchanged, so attention
 // over the staging cache runs the same arithmetic in the same order as
 // attention over resident history.
@@ -40,7 +42,7 @@ namespace hga {
 namespace {
 
 constexpr int kPlanThreads = 1024;
-constexpr int kFreeWave = -2;  // slot_wave of an empty slot: free for every wave >= 0
+constexpr int kFreeWave = -(1 << 30);  // slot_wave of an empty slot: free for every wave and lag
 
 struct TierScratch {
     int32_t *tile_slot, *tile_mark, *slot_tile, *slot_wave, *new_tile, *new_slot, *ctl;
@@ -101,8 +103,9 @@ __device__ int block_scan(int f, int *warp_sums, int *total) {
 
 __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *__restrict__ idx, int n_bg, int nqb,
                                                                  int topk, int qb0, int qb1, int n_chunks,
-                                                                 long long tile_cap, int slots, TierScratch s,
-                                                                 int32_t *n_fetched, unsigned *status) {
+                                                                 long long tile_cap, int slots, int lag,
+                                                                 TierScratch s, int32_t *n_fetched,
+                                                                 unsigned *status) {
     __shared__ int warp_sums[32];
     __shared__ int n_new, total, taken_sh, cursor_sh;
     const int tid = threadIdx.x;
@@ -133,7 +136,7 @@ __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *
     }
     __syncthreads();
     const int need = n_new < slots ? n_new : slots;
-    // 2. free slots (last reader wave <= w - 2) round-robin from the cursor
+    // 2. free slots (last reader wave <= w - lag) round-robin from the cursor
     if (tid == 0) {
         taken_sh = 0;
         cursor_sh = s.ctl[1];
@@ -145,7 +148,7 @@ __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *
         if (taken_sh >= need) break;  // uniform: read after the barrier that ends the previous round
         const int off = base + tid;
         const int sl = off < slots ? (cursor + off) % slots : 0;
-        const int f = (off < slots && s.slot_wave[sl] <= w - 2) ? 1 : 0;
+        const int f = (off < slots && s.slot_wave[sl] <= w - lag) ? 1 : 0;
         const int rank = taken_sh + block_scan(f, warp_sums, &total);
         if (f && rank < need) {
             const int t_new = s.new_tile[rank];
@@ -191,8 +194,10 @@ __global__ void __launch_bounds__(kCopyThreads, 8)
         const int slot = s.new_slot[k];
         const long long bg = t / tile_cap, j = t % tile_cap;
         const long long off = (bg * head_stride_bytes + j * chunk * ROW_BYTES) / 16;
-        const uint4 *sk = host_k + off, *sv = host_v + off;
-        uint4 *dk = stage_k + (long long)slot * tile_vecs, *dv = stage_v + (long long)slot * tile_vecs;
+        // host_v / stage_v are null when one tensor is staged (group summaries)
+        const bool two = host_v != nullptr;
+        const uint4 *sk = host_k + off, *sv = two ? host_v + off : nullptr;
+        uint4 *dk = stage_k + (long long)slot * tile_vecs, *dv = two ? stage_v + (long long)slot * tile_vecs : nullptr;
         // every load of a round is issued before its stores
         for (int e0 = threadIdx.x; e0 < tile_vecs; e0 += PER * kCopyThreads) {
             uint4 bk[PER], bv[PER];
@@ -201,7 +206,7 @@ __global__ void __launch_bounds__(kCopyThreads, 8)
                 const int e = e0 + u * kCopyThreads;
                 if (e < tile_vecs) {
                     bk[u] = sk[e];
-                    bv[u] = sv[e];
+                    if (two) bv[u] = sv[e];
                 }
             }
 #pragma unroll
@@ -209,7 +214,7 @@ __global__ void __launch_bounds__(kCopyThreads, 8)
                 const int e = e0 + u * kCopyThreads;
                 if (e < tile_vecs) {
                     dk[e] = bk[u];
-                    dv[e] = bv[u];
+                    if (two) dv[e] = bv[u];
                 }
             }
         }
@@ -250,51 +255,71 @@ hga_status_t launch_tier_reset(const hga_params_t &p, int stage_slots, int32_t *
     return record_cuda(cudaGetLastError());
 }
 
-hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
-                                 const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
-                                 int stage_slots, int32_t *scratch, int32_t *idx_remapped, int32_t *n_fetched,
-                                 unsigned *status, cudaStream_t stream) {
+namespace {
+
+// One fetch wave of tiles of tile_rows rows of row_bytes bytes (K and V of a
+// chunk, or one chunk's group summaries when host_v is null), tile j of (b, g)
+// starting at row j * tile_rows of a slice of head_stride_rows rows.
+hga_status_t fetch_wave(const hga_params_t &p, const void *host_k, const void *host_v, int tile_rows, int row_bytes,
+                        long long head_stride_rows, long long tile_cap, const int32_t *idx, int qb0, int qb1,
+                        void *stage_k, void *stage_v, int stage_slots, int lag, int32_t *scratch,
+                        int32_t *idx_remapped, int32_t *n_fetched, unsigned *status, cudaStream_t stream) {
     const int n_bg = p.batch * p.n_kv_heads;
     const int nqb = p.seg_len / p.q_block;
-    const long long tile_cap = tier_tile_cap(p);
     const TierScratch s = tier_layout(scratch, (long long)n_bg * tile_cap, stage_slots);
     void *dk = nullptr, *dv = nullptr;
     cudaError_t e = cudaHostGetDevicePointer(&dk, const_cast<void *>(host_k), 0);
+    if (e == cudaSuccess && host_v) e = cudaHostGetDevicePointer(&dv, const_cast<void *>(host_v), 0);
     if (e != cudaSuccess) {
         cudaGetLastError();
-        record_error("hga_fetch_tiered: host_k is not page-locked (mapped) host memory");
-        return HGA_ERR_INVALID_ARG;
-    }
-    e = cudaHostGetDevicePointer(&dv, const_cast<void *>(host_v), 0);
-    if (e != cudaSuccess) {
-        cudaGetLastError();
-        record_error("hga_fetch_tiered: host_v is not page-locked (mapped) host memory");
+        record_error("tiered fetch: the host history is not page-locked (mapped) host memory");
         return HGA_ERR_INVALID_ARG;
     }
     tier_plan_kernel<<<1, kPlanThreads, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, tile_cap,
-                                                     stage_slots, s, n_fetched, status);
-    const int esize = p.dtype == HGA_BF16 ? 2 : 4;
-    const long long head_stride_bytes = p.hist_head_stride * p.head_dim * esize;
-    const int row_bytes = p.head_dim * esize;
+                                                     stage_slots, lag, s, n_fetched, status);
+    const long long head_stride_bytes = head_stride_rows * row_bytes;
     const unsigned g3 = (unsigned)(2 * sm_count());
+    const uint4 *hk = static_cast<const uint4 *>(dk), *hv = static_cast<const uint4 *>(dv);
+    uint4 *sk = static_cast<uint4 *>(stage_k), *sv = static_cast<uint4 *>(stage_v);
     if (row_bytes == 128)
-        tier_copy_kernel<128><<<g3, kCopyThreads, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv,
-                                                               head_stride_bytes, tile_cap, p.chunk, s,
-                                                               (uint4 *)stage_k, (uint4 *)stage_v);
+        tier_copy_kernel<128><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, sk,
+                                                               sv);
     else if (row_bytes == 256)
-        tier_copy_kernel<256><<<g3, kCopyThreads, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv,
-                                                               head_stride_bytes, tile_cap, p.chunk, s,
-                                                               (uint4 *)stage_k, (uint4 *)stage_v);
+        tier_copy_kernel<256><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, sk,
+                                                               sv);
     else
-        tier_copy_kernel<512><<<g3, kCopyThreads, 0, stream>>>((const uint4 *)dk, (const uint4 *)dv,
-                                                               head_stride_bytes, tile_cap, p.chunk, s,
-                                                               (uint4 *)stage_k, (uint4 *)stage_v);
+        tier_copy_kernel<512><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, sk,
+                                                               sv);
     const long long marks = (long long)n_bg * (qb1 - qb0) * p.topk;
     const unsigned g1 = (unsigned)((marks + 255) / 256 > 1184 ? 1184 : (marks + 255) / 256);
     if (marks > 0)
         tier_remap_kernel<<<g1, 256, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, tile_cap,
                                                   s.tile_slot, idx_remapped);
     return record_cuda(cudaGetLastError());
+}
+
+}  // namespace
+
+hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
+                                 const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
+                                 int stage_slots, int lag, int32_t *scratch, int32_t *idx_remapped,
+                                 int32_t *n_fetched, unsigned *status, cudaStream_t stream) {
+    const int esize = p.dtype == HGA_BF16 ? 2 : 4;
+    return fetch_wave(p, host_k, host_v, p.chunk, p.head_dim * esize, p.hist_head_stride, tier_tile_cap(p), idx, qb0,
+                      qb1, stage_k, stage_v, stage_slots, lag, scratch, idx_remapped, n_fetched, status, stream);
+}
+
+hga_status_t launch_fetch_group_summaries(const hga_params_t &p, const float *host_gsumm, int group,
+                                          const int32_t *idx, float *stage, int stage_slots, int32_t *scratch,
+                                          int32_t *idx_remapped, int32_t *n_fetched, unsigned *status,
+                                          cudaStream_t stream) {
+    // a tile = the chunk / group fp32 summaries of one chunk's groups; the slice of
+    // (b, g) holds hist_head_stride / group of them
+    const int gpc = p.chunk / group;
+    const long long rows = p.hist_head_stride / group;
+    return fetch_wave(p, host_gsumm, nullptr, gpc, p.head_dim * 4, rows, tier_tile_cap(p), idx, 0,
+                      p.seg_len / p.q_block, stage, nullptr, stage_slots, 2, scratch, idx_remapped, n_fetched,
+                      status, stream);
 }
 
 }  // namespace hga

@@ -160,6 +160,26 @@ hga_status_t hga_route(const hga_params_t *p, const void *q, const float *summ, 
 hga_status_t hga_route_groups(const hga_params_t *p, const void *q, const float *gsumm, int gsumm_cap_groups,
                               const int32_t *idx, int group, int topg, int32_t *gidx, cudaStream_t stream);
 
+/* hga_route_groups with the group summaries kept in page-locked host memory
+ * and a device cache of them (technical summary section 2.2: group summaries
+ * are cached on the GPU and misses are fetched from the host).  For every
+ * block's routed chunks, the chunk's chunk/group group summaries (one cache
+ * tile) are copied from host_gsumm ([B][Hkv][gsumm_cap_groups][D] fp32) into
+ * stage_gsumm ([stage_slots][chunk/group][D] fp32) unless the cache already
+ * holds them -- the staging cache, its scratch, eviction rule and device
+ * status bits are those of hga_fetch_tiered, one fetch wave per call, all on
+ * stream -- and the routes are then computed from the cache: gidx equals
+ * hga_route_groups' over the same values, bit for bit.
+ *   p->hist_head_stride must be gsumm_cap_groups * group (the history tokens the
+ *   group summaries cover; hga_tier_scratch_size / hga_tier_reset with this p
+ *   size and empty the cache); idx_remapped (same shape as idx) receives the
+ *   routed chunks' cache slots; n_fetched (may be NULL): tiles copied.
+ *   stage_slots >= min(2 * (S/q_block) * B * Hkv * min(k, Nc), B * Hkv * Nc). */
+hga_status_t hga_route_groups_tiered(const hga_params_t *p, const void *q, const float *host_gsumm,
+                                     int gsumm_cap_groups, const int32_t *idx, int group, int topg, int32_t *gidx,
+                                     float *stage_gsumm, int stage_slots, int32_t *scratch, int32_t *idx_remapped,
+                                     int32_t *n_fetched, cudaStream_t stream);
+
 /* Strictly causal routing (technical summary, limits section: sharing one
  * route among the tokens of a block is a weak causal side channel; a strictly
  * causal variant is proposed as future work).  Every token i of block m
@@ -388,22 +408,95 @@ hga_status_t hga_fetch_tiered(const hga_params_t *p, const void *host_k, const v
 hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const void *v_seg, void *host_k,
                               void *host_v, long long dst_token, cudaStream_t stream);
 
+/* Cross-stream schedule of hga_attn_fwd_tiered, owned by the caller and kept
+ * from call to call over one staging cache.  Wave h of the schedule is one
+ * fetch (on the copy stream) and the attention that reads it (on the compute
+ * stream); the fetch of wave h may evict the slots that wave h - lag read, so
+ * it starts only after that attention (consumed[h % lag]) and may overlap the
+ * attention of the lag - 1 waves before it.  The cache then holds the tiles of
+ * lag waves: stage_slots >= min(lag * wave_blocks * B * Hkv * min(k, Nc),
+ * B * Hkv * Nc).
+ *   Create the events (cudaEventDisableTiming is enough; inputs and
+ *   offloaded only for hga_segment_fwd_tiered), set lag (2 ..
+ *   HGA_TIER_MAX_LAG), wave = 0 and segment = 0; the library records the
+ *   events and advances the counters.  Use one compute stream and one copy stream for all calls of
+ *   a schedule, and no other fetch into its cache (hga_fetch_tiered,
+ *   hga_route_groups_tiered) between them.  A schedule's first call (wave 0)
+ *   is never chained. */
+#define HGA_TIER_MAX_LAG 4
+typedef struct {
+    cudaEvent_t start;                       /* unchained calls: the copy stream after the compute stream */
+    cudaEvent_t fetched;                     /* attention of wave h after the fetch of wave h */
+    cudaEvent_t consumed[HGA_TIER_MAX_LAG];  /* fetch of wave h after the attention of wave h - lag */
+    cudaEvent_t inputs;                      /* hga_segment_fwd_tiered: the offload after the segment's inputs */
+    cudaEvent_t offloaded[2];                /* hga_segment_fwd_tiered: fetches after the previous offload */
+    int lag;
+    long long wave;                          /* waves issued through the schedule since its cache was emptied */
+    long long segment;                       /* segments through hga_segment_fwd_tiered since then */
+} hga_tier_sched_t;
+
 /* hga_attn_fwd over host-resident history, overlapping fetch and attention:
  * the blocks [qblock_begin, qblock_end) (0/0: all) are taken in waves of
- * wave_blocks query blocks; wave w's fetch runs on copy_stream while wave
- * w-1's attention runs on stream, and it starts only after wave w-2's
- * attention has finished.  Output (out, lse) is bit-identical to hga_attn_fwd
- * with the history resident.  The copy stream first waits for everything
- * already enqueued on stream (the route that wrote idx); on return, stream is
- * ordered after every fetch.  reset_cache != 0 empties the cache first.
- *   events: 5 caller-created events (cudaEventDisableTiming is enough), used
- *   as the cross-stream fences.  n_fetched (device int32, may be NULL): one
- *   count per wave.  Other arguments as hga_fetch_tiered and hga_attn_fwd. */
+ * wave_blocks query blocks; the fetch of each wave runs on copy_stream while
+ * earlier waves' attention runs on stream, ordered by sched (above).  Output
+ * (out, lse) is bit-identical to hga_attn_fwd with the history resident.  On
+ * return, stream is ordered after every fetch of the call (with Nc = 0, after
+ * all work then on copy_stream).
+ *   flags: HGA_TIER_RESET empties the cache first (and sets sched->wave = 0).
+ *   Without HGA_TIER_CHAIN, and always with HGA_TIER_RESET, the copy stream
+ *   first waits for everything already enqueued on stream (the route that
+ *   wrote idx, earlier attention over the cache).  With HGA_TIER_CHAIN alone
+ *   the call continues the schedule of the previous call (the next segment of
+ *   an evaluation): the copy stream does not wait for stream -- the caller
+ *   orders it after whatever wrote idx and after the host rows the fetches
+ *   read -- so the first fetches overlap the previous call's last attention.
+ *   Chained calls need a non-decreasing Nc, and idx_remapped must not be a
+ *   buffer that an attention still in flight reads: the fetch of wave h
+ *   writes its blocks' rows once wave h - lag is done, so chained calls of n
+ *   waves each rotate ceil(lag / n) idx_remapped buffers.
+ *   n_fetched (device int32, may be NULL): one count per wave.  Other
+ *   arguments as hga_fetch_tiered and hga_attn_fwd.  HGA_ERR_INVALID_ARG for
+ *   a null event, a lag outside 2 .. HGA_TIER_MAX_LAG or unknown flags. */
+#define HGA_TIER_RESET 1
+#define HGA_TIER_CHAIN 2
 hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const void *host_k, const void *host_v,
                                  const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
                                  void *stage_k, void *stage_v, int stage_slots, int32_t *scratch,
-                                 int32_t *idx_remapped, int wave_blocks, int reset_cache, int32_t *n_fetched,
-                                 cudaStream_t stream, cudaStream_t copy_stream, const cudaEvent_t *events);
+                                 int32_t *idx_remapped, int wave_blocks, int flags, int32_t *n_fetched,
+                                 cudaStream_t stream, cudaStream_t copy_stream, hga_tier_sched_t *sched);
+
+/* One segment of an evaluation whose detached history lives in page-locked
+ * host memory (technical summary section 2.2, tiered memory; section 2.1 for
+ * the route and the exact-token attention; the segment detaches at its end),
+ * on three streams, so that a segment's route and fetches run under the
+ * previous segment's attention:
+ *   copy_stream   : hga_route of the segment into idx; the fetch waves of
+ *                   hga_attn_fwd_tiered, chained from the previous segment,
+ *                   the first after the previous segment's offload; then the
+ *                   detach-time append of the segment's S / chunk summaries
+ *                   to chunks [Nc, Nc + S / chunk) of summ.
+ *   offload_stream: k_seg / v_seg copied to tokens [T, T + S) of host_k /
+ *                   host_v (T = Nc * chunk) once the inputs are ready.
+ *   stream        : the attention waves, writing out and lse.
+ * q, k_seg and v_seg must be ready in copy_stream's order (the caller copies
+ * them in there, or orders copy_stream after their producer).  flags:
+ * HGA_TIER_RESET for the evaluation's first segment (copy_stream first waits
+ * for stream; the cache is emptied; sched->wave and sched->segment restart);
+ * 0 continues the evaluation.  On return stream is ordered after the
+ * segment's fetches; the append and the offload are ordered before the next
+ * call's fetches, and the caller orders stream after copy_stream and
+ * offload_stream before it reads summ or the host history itself.
+ * idx_remapped as in hga_attn_fwd_tiered (rotate ceil(lag / waves per
+ * segment) buffers over the segments).  HGA_ERR_INVALID_ARG when
+ * summ_cap_chunks < Nc + S / chunk, T + S > hist_head_stride, the host
+ * history is not page-locked, or an event of sched is null; other arguments
+ * and checks as hga_route, hga_attn_fwd_tiered and hga_tier_offload. */
+hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const void *k_seg, const void *v_seg,
+                                    float *summ, int summ_cap_chunks, int32_t *idx, void *host_k, void *host_v,
+                                    void *out, float *lse, void *stage_k, void *stage_v, int stage_slots,
+                                    int32_t *scratch, int32_t *idx_remapped, int wave_blocks, int flags,
+                                    int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,
+                                    cudaStream_t offload_stream, hga_tier_sched_t *sched);
 
 /* Self-test of the bounded waits (the source pages have no counterpart): every
  * pipeline wait in the tensor-core kernels gives up after a cycle limit instead

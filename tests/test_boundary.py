@@ -83,6 +83,20 @@ def test_group_route_checked_on_host(L):
     assert L.hga_route_groups(ctypes.byref(p), fake, fake, 64, fake, 8, 4, None, None) == -1
 
 
+def test_tiered_group_route_checked_on_host(L):
+    fake = ctypes.c_void_p(0x1000)
+    # Nc 8, k 4, groups of 8: the group-summary history is 64 groups per (b, g)
+    p = _params(hist_head_stride=64 * 8).c()
+    args = lambda cap, grp, topg, slots: (ctypes.byref(p), fake, fake, cap, fake, grp, topg, fake, fake, slots, fake,
+                                          fake, None, None)
+    assert L.hga_route_groups_tiered(*args(64, 7, 4, 16)) == -1       # group size
+    assert L.hga_route_groups_tiered(*args(64, 8, 33, 16)) == -1      # topg above k * chunk / group
+    assert L.hga_route_groups_tiered(*args(32, 8, 4, 16)) == -1       # capacity below Nc * 8
+    assert L.hga_route_groups_tiered(*args(128, 8, 4, 16)) == -1      # hist_head_stride != cap * group
+    assert L.hga_route_groups_tiered(*args(64, 8, 4, 15)) == -1       # stage below 2 x 2 blocks x 2 heads x 4
+    assert b"stage_slots" in L.hga_last_error()
+
+
 def test_causal_route_checked_on_host(L):
     fake = ctypes.c_void_p(0x1000)
     odd = ctypes.c_void_p(0x1008)
@@ -134,14 +148,59 @@ def test_tiered_staging_capacity_checked_on_host(L):
     assert rc == -1
     rc = L.hga_fetch_tiered(ctypes.byref(p), fake, fake, fake, 0, 2, fake, fake, 64, None, fake, None, None, None)
     assert rc == -1  # no scratch
-    # the overlapped schedule: five events, waves of at least one block
-    evs = (ctypes.c_void_p * 5)(*([0x10] * 5))
+    # the overlapped schedule: every event set, lag in 2..4, known flags, waves of at
+    # least one block, and slots for lag waves
+    sc = hga.binding._TierSchedC()
+    sc.start = sc.fetched = 0x10
+    sc.consumed[0] = sc.consumed[1] = sc.consumed[2] = 0x10
+    sc.lag = 2
     args = [ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, 64, fake, fake]
-    assert L.hga_attn_fwd_tiered(*args, 0, 1, None, None, None, evs) == -1
+    assert L.hga_attn_fwd_tiered(*args, 0, 1, None, None, None, ctypes.byref(sc)) == -1
     assert L.hga_attn_fwd_tiered(*args, 1, 1, None, None, None, None) == -1
-    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, (ctypes.c_void_p * 5)(0x10, 0x10, 0, 0x10, 0x10)) == -1
+    assert L.hga_attn_fwd_tiered(*args, 2, 4, None, None, None, ctypes.byref(sc)) == -1  # unknown flag
+    for lag in (1, 5):
+        sc.lag = lag
+        assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
+    sc.lag = 4  # consumed[3] unset
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
+    sc.lag = 2
+    sc.fetched = 0
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
+    sc.fetched = 0x10
     args[11] = 31  # two waves of 2 blocks need 32 slots
-    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, evs) == -1
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
+    sc.lag = 3
+    args[11] = 47  # lag 3: 48 slots (fewer than the 64 routable tiles)
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
+    assert b"stage_slots" in L.hga_last_error()
+
+
+def test_segment_tiered_checked_on_host(L):
+    # one tiered evaluation segment: summaries room for the segment's chunks, the
+    # segment inside the host history, the offload events, flags
+    p = _params(n_hist_chunks=32, hist_head_stride=4096)
+    fake = ctypes.c_void_p(0x1000)
+    sc = hga.binding._TierSchedC()
+    sc.start = sc.fetched = sc.inputs = 0x10
+    sc.consumed[0] = sc.consumed[1] = 0x10
+    sc.offloaded[0] = sc.offloaded[1] = 0x10
+    sc.lag = 2
+    seg_chunks = p.seg_len // 64
+
+    def call(pp, cap, flags=0, sched=sc):
+        return L.hga_segment_fwd_tiered(ctypes.byref(pp.c()), fake, fake, fake, fake, cap, fake, fake, fake, fake,
+                                        fake, fake, fake, 64, fake, fake, 2, flags, None, None, None, None,
+                                        ctypes.byref(sched) if sched is not None else None)
+
+    assert call(p, 32 + seg_chunks - 1) == -1  # no room to append the segment's summaries
+    assert call(_params(n_hist_chunks=32, hist_head_stride=32 * 64 + p.seg_len - 1), 4096) == -1
+    assert call(p, 4096, flags=2) == -1  # only HGA_TIER_RESET is a flag here
+    assert call(p, 4096, sched=None) == -1
+    sc.offloaded[1] = 0
+    assert call(p, 4096) == -1
+    sc.offloaded[1] = 0x10
+    sc.inputs = 0
+    assert call(p, 4096) == -1
 
 
 def test_tiered_scratch_size(L):

@@ -413,7 +413,7 @@ def _tiered_run(w, seg, wave, slots, reps=1):
     p = hc.params(w, T, hist_head_stride=T, seg_head_stride=T + S)
     scratch = torch.empty(hga.hga_tier_scratch_size(p, slots) // 4, device="cuda", dtype=torch.int32)
     idx_r = torch.full_like(idx, -5)
-    events = [torch.cuda.Event() for _ in range(5)]
+    sched = hga.TierSched(lag=2)
     copy = torch.cuda.Stream()
     results, fetched = [], []
     for r in range(reps):
@@ -421,7 +421,7 @@ def _tiered_run(w, seg, wave, slots, reps=1):
         out = torch.full_like(out_res, float("nan"))
         lse = torch.full_like(lse_res, float("nan"))
         hga.hga_attn_fwd_tiered(p, g.q, host_k, host_v, g.k_seg, g.v_seg, idx, out, lse, stage_k, stage_v, slots,
-                                scratch, idx_r, wave, events, reset_cache=(r == 0), n_fetched=nf, copy_stream=copy)
+                                scratch, idx_r, wave, sched, reset_cache=(r == 0), n_fetched=nf, copy_stream=copy)
         results.append((out, lse))
         fetched.append(nf)
     torch.cuda.synchronize()
@@ -476,6 +476,93 @@ def test_tiered_128k_last_segment():
     fetched, distinct = _check_tiered(w, 31, wave=8, slots=slots, sample_rows=_sampled_rows(w, 96, seed=5))
     assert fetched == [distinct, 0]
     print(f"tiles fetched for the last 4,096-token segment: {fetched[0]} (distinct routed tiles {distinct})")
+
+
+# six consecutive 256-token segments of one sequence, for the chained tiered schedule
+CHAIN = gen.custom("chain_bf16", n_q_heads=8, n_kv_heads=2, head_dim=128, topk=4, seg_len=256, seq_len=6 * 256,
+                   seg_starts=tuple(range(0, 6 * 256, 256)), dtype="bf16", seed=23)
+
+
+@pytest.mark.parametrize("wave,lag,slots", [(4, 2, 40), (1, 4, 32), (1, 3, 24), (2, 2, 32), (1, 2, 16)],
+                         ids=["segment_waves_lag2", "block_waves_lag4", "block_waves_lag3", "two_block_waves_lag2",
+                              "block_waves_lag2"])
+def test_tiered_chained_segments_match_resident(wave, lag, slots):
+    """An evaluation of six segments with the history only in pinned host memory,
+    through hga_segment_fwd_tiered as the benchmark runs it: each segment's K/V
+    offloaded to the host history on a third stream, its route, fetch waves and
+    summary append on the copy stream, its attention waves on the compute stream,
+    chained from segment to segment (no host synchronisation anywhere), so fetches of
+    a segment run under the attention of the one before it.  The host history starts as NaN, so a
+    fetch that overtook an offload, or an eviction of a slot still being read, changes
+    the output.  Every segment's out and lse equal the resident forward on the same
+    routes bit for bit.  Slots: the least the schedule accepts, min(lag x wave x B x
+    Hkv x k, B x Hkv x Nc); all but the segment-wave case hold fewer than the last
+    segment's 40 routable tiles, so the cache evicts."""
+    import hierarchical_sparse_long_b200 as hga
+    w = CHAIN
+    L, S, D = w.seq_len, w.seg_len, w.head_dim
+    nqb = S // 64
+    k_all = hc.to_dev(gen.keys(w, 0, L), w)
+    v_all = hc.to_dev(gen.values(w, 0, L), w)
+    qs = {T: hc.to_dev(gen.queries(w, T, T + S), w) for T in w.seg_starts}
+    nct = L // 64
+    # resident reference: routes and forward per segment, history in device memory
+    full = torch.zeros(w.batch, w.n_kv_heads, nct, D, device="cuda")
+    hga.hga_build_summaries(k_all, L, w.batch, w.n_kv_heads, D, 64, 0, nct, full, nct)
+    ref = {}
+    for T in w.seg_starts:
+        p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
+        idx = torch.empty(w.batch, w.n_kv_heads, nqb, w.topk, device="cuda", dtype=torch.int32)
+        hga.hga_route(p, qs[T], full, nct, idx)
+        out = torch.empty_like(qs[T])
+        lse = torch.empty(qs[T].shape[:3], device="cuda")
+        hga.hga_attn_fwd(p, qs[T], k_all, v_all, k_all[:, :, T:], v_all[:, :, T:], idx, out, lse)
+        ref[T] = (out, lse, idx)
+    torch.cuda.synchronize()
+    # the chained tiered evaluation
+    host_k = torch.full((w.batch, w.n_kv_heads, L, D), float("nan"), dtype=k_all.dtype).pin_memory()
+    host_v = torch.full_like(host_k, float("nan")).pin_memory()
+    summ = torch.zeros_like(full)
+    stage_k = torch.empty(slots, 64, D, device="cuda", dtype=k_all.dtype)
+    stage_v = torch.empty_like(stage_k)
+    p_last = hc.params(w, w.seg_starts[-1], hist_head_stride=L, seg_head_stride=L)
+    scratch = torch.empty(hga.hga_tier_scratch_size(p_last, slots) // 4, device="cuda", dtype=torch.int32)
+    n_waves = -(-nqb // wave)
+    idx_r = [torch.full((w.batch, w.n_kv_heads, nqb, w.topk), -5, device="cuda", dtype=torch.int32)
+             for _ in range(-(-lag // n_waves))]
+    idx = torch.full_like(idx_r[0], 7)  # stale routes: read before the first route, they would be flagged
+    sched = hga.TierSched(lag=lag)
+    compute, copy, off = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    nf = torch.zeros(len(w.seg_starts), n_waves, device="cuda", dtype=torch.int32)
+    got = {}
+    for si, T in enumerate(w.seg_starts):
+        p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
+        out = torch.full_like(qs[T], float("nan"))
+        lse = torch.full(qs[T].shape[:3], float("nan"), device="cuda")
+        hga.hga_segment_fwd_tiered(p, qs[T], k_all[:, :, T:], v_all[:, :, T:], summ, nct, idx, host_k, host_v, out,
+                                   lse, stage_k, stage_v, slots, scratch, idx_r[si % len(idx_r)], wave, sched,
+                                   reset=si == 0, n_fetched=nf[si], copy_stream=copy, offload_stream=off)
+        got[T] = (out, lse)
+    compute.wait_stream(copy)
+    compute.wait_stream(off)
+    torch.cuda.synchronize()
+    assert hga.hga_get_device_status() == 0
+    for T in w.seg_starts:
+        assert torch.equal(got[T][0], ref[T][0]), f"segment at {T}: out"
+        assert torch.equal(got[T][1], ref[T][1]), f"segment at {T}: lse"
+    assert sched.segment == len(w.seg_starts)
+    # the host history holds every segment's K/V
+    assert torch.equal(host_k, k_all.cpu()) and torch.equal(host_v, v_all.cpu())
+    assert torch.equal(summ, full)
+    assert sched.wave == n_waves * (len(w.seg_starts) - 1)  # the first segment has no history: no wave
+    fetched = int(nf.sum().item())
+    union = {(b, g, int(j)) for T in w.seg_starts for b in range(w.batch) for g in range(w.n_kv_heads)
+             for j in ref[T][2][b, g].flatten().tolist() if j >= 0}
+    print(f"wave {wave}, lag {lag}, {slots} slots: fetched {fetched} tiles over {len(w.seg_starts)} segments, "
+          f"{len(union)} distinct")
+    assert fetched >= len(union)
+    if len(union) > slots:
+        assert fetched > slots  # the cache evicted
 
 
 def test_tiered_rejects_pageable_host_memory_before_any_launch():

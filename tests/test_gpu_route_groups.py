@@ -101,3 +101,75 @@ def test_group_route_full_size_16k():
     hard, exempt = hc.route_mismatches(got, want, gap)
     print(f"16K groups of 8, topg 64: near-tie exemptions {exempt}")
     assert hard == 0
+
+
+def _tiered_group_route(w, T, group, topg, q, kh, idx_list, slots):
+    """hga_route_groups_tiered (group summaries in pinned host memory, a device cache of
+    them) against hga_route_groups on the same summaries resident on the device, one
+    call per chunk-route table of idx_list (the cache is kept between calls).  Returns
+    the tiles fetched by each call and the distinct routed chunks of each table."""
+    import hierarchical_sparse_long_b200 as hga
+    nc = T // 64
+    gpc = 64 // group
+    ng = nc * gpc
+    gsumm = torch.zeros(w.batch, w.n_kv_heads, ng, w.head_dim, device="cuda")
+    hga.hga_build_summaries(hc.to_dev(kh, w), T, w.batch, w.n_kv_heads, w.head_dim, group, 0, ng, gsumm, ng)
+    nqb = w.seg_len // 64
+    p = hc.params(w, T, hist_head_stride=ng * group)
+    qd = hc.to_dev(q, w)
+    host = gsumm.cpu().pin_memory()
+    stage = torch.empty(slots, gpc, w.head_dim, device="cuda")
+    scratch = torch.empty(hga.hga_tier_scratch_size(p, slots) // 4, device="cuda", dtype=torch.int32)
+    hga.hga_tier_reset(p, slots, scratch)
+    fetched, distinct = [], []
+    for idx_o in idx_list:
+        idx = torch.from_numpy(np.ascontiguousarray(idx_o)).cuda()
+        want = torch.full((w.batch, w.n_kv_heads, nqb, topg), -7, device="cuda", dtype=torch.int32)
+        hga.hga_route_groups(p, qd, gsumm, ng, idx, group, topg, want)
+        idx_r = torch.full_like(idx, -5)
+        got = torch.full_like(want, -9)
+        nf = torch.zeros(1, device="cuda", dtype=torch.int32)
+        hga.hga_route_groups_tiered(p, qd, host, ng, idx, group, topg, got, stage, slots, scratch, idx_r, nf)
+        torch.cuda.synchronize()
+        assert torch.equal(got, want)
+        fetched.append(int(nf.item()))
+        i = np.asarray(idx_o).astype(np.int64)
+        distinct.append(len({(b, g, j) for b in range(w.batch) for g in range(w.n_kv_heads)
+                             for j in i[b, g].ravel() if j >= 0}))
+    assert hga.hga_get_device_status() == 0
+    return fetched, distinct
+
+
+def test_group_route_from_host_cache_equals_resident():
+    # a cache holding every routable chunk's groups: each routed chunk's summaries are
+    # fetched once, the second call over the same routes fetches nothing
+    w = gen.custom("grp_tier", dtype="bf16", head_dim=128, n_q_heads=8, n_kv_heads=2, topk=6, seg_len=192,
+                   seq_len=40 * 64 + 192, seg_starts=(40 * 64,), seed=98)
+    T = 40 * 64
+    q = gen.queries(w, T, T + w.seg_len)
+    kh = gen.keys(w, 0, T)
+    _, _, idx_o, _ = hc.oracle_route(w, dict(T=T, q=q, k_all=kh))
+    fetched, distinct = _tiered_group_route(w, T, 8, 20, q, kh, [idx_o, idx_o], slots=2 * 40)
+    assert fetched == [distinct[0], 0]
+
+
+def test_group_route_from_small_host_cache_evicts():
+    # 3 blocks x 2 heads x 6 chunks = at most 36 routed chunks per call, 72 slots (< 80
+    # routable): calls over five route tables (four of random chunks) fetch more tiles than the cache
+    # holds, so the round-robin eviction reaches the first table's slots, and a last call
+    # over the first table fetches some of them back; every call's routes equal the
+    # resident ones
+    w = gen.custom("grp_tier_small", dtype="fp32", head_dim=64, n_q_heads=4, n_kv_heads=2, topk=6, seg_len=192,
+                   seq_len=40 * 64 + 192, seg_starts=(40 * 64,), seed=99)
+    T = 40 * 64
+    q = gen.queries(w, T, T + w.seg_len)
+    kh = gen.keys(w, 0, T)
+    _, _, idx_o, _ = hc.oracle_route(w, dict(T=T, q=q, k_all=kh))
+    rng = np.random.default_rng(7)
+    others = [np.sort(np.stack([[[rng.choice(40, 6, replace=False) for _ in range(3)] for _ in range(2)]]), axis=-1)
+              .astype(np.int32) for _ in range(4)]
+    fetched, distinct = _tiered_group_route(w, T, 16, 9, q, kh, [idx_o, *others, idx_o], slots=72)
+    assert fetched[0] == distinct[0]
+    assert sum(fetched[:5]) > 72  # more tiles than slots: the cache evicted
+    assert fetched[5] > 0  # the first table's tiles were among them
+    print(f"small group-summary cache: fetched {fetched}, distinct {distinct}")
