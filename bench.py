@@ -366,20 +366,25 @@ class Layer:
         # the fetch of a wave rewrites its blocks' remapped routes once the attention
         # `lag` waves back is done: chained segments rotate enough buffers
         self.idx_r = [torch.empty_like(self.idx) for _ in range(-(-self.lag // self.n_waves))]
+        # a route may run a segment ahead of the fetches that read the one before it
+        self.idx_ring = [self.idx, torch.empty_like(self.idx)]
         self.n_fetched = torch.zeros(len(w.seg_starts), self.n_waves, device="cuda", dtype=torch.int32)
-        self.copy_stream = torch.cuda.Stream()
-        self.offload_stream = torch.cuda.Stream()
+        # the side streams' kernels are small; at high priority they take SMs as the
+        # attention's CTAs retire instead of waiting behind the whole attention grid
+        self.copy_stream = torch.cuda.Stream(priority=-1)
+        self.route_stream = torch.cuda.Stream(priority=-1)
+        self.offload_stream = torch.cuda.Stream(priority=-1)
         self.sched = hga.TierSched(lag=self.lag)
 
     def segment_tiered(self, T, ev=None, q=None, si=0):
         """The same segment with the history only in pinned host memory, one
-        hga_segment_fwd_tiered call on three streams: the route, the fetch of the
-        routed tiles (chained from segment to segment over the staging cache, the
-        cache emptied at the first segment only) and the summary append on the
-        copy stream, the segment's K/V offload to the host history on a third,
-        the attention on the compute stream -- so a segment's route and fetches
-        run under the attention of the segment before it.  The segment's q, K and
-        V are resident, or were copied in on the copy stream."""
+        hga_segment_fwd_tiered call on four streams: the route and the summary
+        append on a route stream, the fetch of the routed tiles on a copy stream
+        (chained from segment to segment over the staging cache, the cache emptied
+        at the first segment only), the segment's K/V offload to the host history
+        on a third, the attention on the compute stream -- so a segment's route
+        and fetches run under the attention of the segments before it.  The
+        segment's q, K and V are resident, or were copied in on the route stream."""
         hga, w = self.hga, self.w
         p = self.params(T)
         q = self.q[T] if q is None else q
@@ -387,11 +392,11 @@ class Layer:
         if ev is not None:
             ev.record("attn_fwd")
         first = si == 0
-        hga.hga_segment_fwd_tiered(p, q, ks, vs, self.summ, self.nct, self.idx, self.host_k, self.host_v, self.out,
-                                   self.lse, self.stage_k, self.stage_v, self.slots, self.scratch,
-                                   self.idx_r[si % len(self.idx_r)], self.wave, self.sched, reset=first,
-                                   n_fetched=self.n_fetched[si], copy_stream=self.copy_stream,
-                                   offload_stream=self.offload_stream)
+        hga.hga_segment_fwd_tiered(p, q, ks, vs, self.summ, self.nct, self.idx_ring[si % 2], self.host_k,
+                                   self.host_v, self.out, self.lse, self.stage_k, self.stage_v, self.slots,
+                                   self.scratch, self.idx_r[si % len(self.idx_r)], self.wave, self.sched,
+                                   reset=first, n_fetched=self.n_fetched[si], copy_stream=self.copy_stream,
+                                   route_stream=self.route_stream, offload_stream=self.offload_stream)
         if ev is not None:
             ev.record(None)
         # route, reset (first segment), fetch waves (plan, copy, remap) + attention, append
@@ -401,6 +406,7 @@ class Layer:
         """The step ends when the side streams' work (the last append and offload) has."""
         compute = self.torch.cuda.current_stream()
         compute.wait_stream(self.copy_stream)
+        compute.wait_stream(self.route_stream)
         compute.wait_stream(self.offload_stream)
 
     def fetch_only_step(self):
@@ -932,9 +938,10 @@ def e2e_measure(layer, steps):
     outs = [layer.out, layer.lse] + ([layer.dq, layer.dk, layer.dv] if w.backward else [])
     host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
     # the tiered step runs each segment's route and fetches under the attention of the
-    # segment before it: its inputs arrive on the copy stream, q in a ring of three
-    # buffers (the copy stream reaches segment s only after the attention of s - 3)
-    q_ring = [torch.empty_like(layer.q[w.seg_starts[0]]) for _ in range(3 if w.tiered else 1)]
+    # segments before it: its inputs arrive on the route stream, q in a ring of five
+    # buffers (the route stream reaches segment s only after the fetches of s - 3, which
+    # come after the attention of s - 5)
+    q_ring = [torch.empty_like(layer.q[w.seg_starts[0]]) for _ in range(5 if w.tiered else 1)]
     do_d = torch.empty_like(layer.do[w.seg_starts[0]]) if w.backward else None
     h2d = sum(t.numel() * t.element_size() for ts in host_in.values() for t in ts)
     d2h = sum(t.numel() * t.element_size() for t in outs) * len(w.seg_starts)
@@ -947,8 +954,8 @@ def e2e_measure(layer, steps):
             hi = host_in[T]
             q_d = q_ring[si % len(q_ring)]
             if w.tiered and si == 0:
-                layer.copy_stream.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(layer.copy_stream if w.tiered else torch.cuda.current_stream()):
+                layer.route_stream.wait_stream(torch.cuda.current_stream())
+            with torch.cuda.stream(layer.route_stream if w.tiered else torch.cuda.current_stream()):
                 q_d.copy_(hi[0], non_blocking=True)
                 layer.k[:, :, T:T + S].copy_(hi[1], non_blocking=True)
                 layer.v[:, :, T:T + S].copy_(hi[2], non_blocking=True)

@@ -115,7 +115,7 @@ def lib() -> ctypes.CDLL:
         L.hga_attn_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp, vp, vp,
                                           ctypes.POINTER(_TierSchedC)]
         L.hga_segment_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp,
-                                             vp, vp, vp, ctypes.POINTER(_TierSchedC)]
+                                             vp, vp, vp, vp, ctypes.POINTER(_TierSchedC)]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hga_selftest_wait_timeout.argtypes = [ll, vp]
         L.hga_selftest_wait_timeout.restype = ctypes.c_int
@@ -340,7 +340,8 @@ def hga_tier_offload(p: Params, k_seg, v_seg, host_k, host_v, dst_token: int, st
 
 class _TierSchedC(ctypes.Structure):
     _fields_ = [("start", ctypes.c_void_p), ("fetched", ctypes.c_void_p), ("consumed", ctypes.c_void_p * 4),
-                ("inputs", ctypes.c_void_p), ("offloaded", ctypes.c_void_p * 2), ("lag", ctypes.c_int),
+                ("inputs", ctypes.c_void_p), ("offloaded", ctypes.c_void_p * 2), ("routed", ctypes.c_void_p),
+                ("idx_free", ctypes.c_void_p * 2), ("lag", ctypes.c_int),
                 ("wave", ctypes.c_longlong), ("segment", ctypes.c_longlong)]
 
 
@@ -355,15 +356,16 @@ class TierSched:
         import torch
         if not 2 <= lag <= self.MAX_LAG:
             raise ValueError(f"lag must be in 2..{self.MAX_LAG}")
-        self.events = [torch.cuda.Event() for _ in range(5 + lag)]
+        self.events = [torch.cuda.Event() for _ in range(8 + lag)]
         for e in self.events:  # torch creates its CUDA event on the first record
             e.record()
         h = [e.cuda_event for e in self.events]
         self.c = _TierSchedC()
-        self.c.start, self.c.fetched, self.c.inputs = h[0], h[1], h[2]
-        self.c.offloaded[0], self.c.offloaded[1] = h[3], h[4]
+        self.c.start, self.c.fetched, self.c.inputs, self.c.routed = h[0], h[1], h[2], h[3]
+        self.c.offloaded[0], self.c.offloaded[1] = h[4], h[5]
+        self.c.idx_free[0], self.c.idx_free[1] = h[6], h[7]
         for i in range(lag):
-            self.c.consumed[i] = h[5 + i]
+            self.c.consumed[i] = h[8 + i]
         self.c.lag = lag
         self.c.wave = 0
         self.c.segment = 0
@@ -398,16 +400,16 @@ def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, ls
 def hga_segment_fwd_tiered(p: Params, q, k_seg, v_seg, summ, summ_cap_chunks: int, idx, host_k, host_v, out, lse,
                            stage_k, stage_v, stage_slots: int, scratch, idx_remapped, wave_blocks: int,
                            sched: TierSched, reset=False, n_fetched=None, stream=None, copy_stream=None,
-                           offload_stream=None):
-    """One segment of a tiered evaluation: route, fetches and summary append on
-    copy_stream, the K/V offload on offload_stream, attention on stream."""
+                           route_stream=None, offload_stream=None):
+    """One segment of a tiered evaluation: route and summary append on route_stream,
+    fetches on copy_stream, the K/V offload on offload_stream, attention on stream."""
     cp = p.c()
     _check(lib().hga_segment_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(summ),
                                         summ_cap_chunks, _ptr(idx), _ptr(host_k), _ptr(host_v), _ptr(out), _ptr(lse),
                                         _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(scratch),
                                         _ptr(idx_remapped), wave_blocks, HGA_TIER_RESET if reset else 0,
                                         _ptr(n_fetched), _stream(stream), _stream(copy_stream),
-                                        _stream(offload_stream), ctypes.byref(sched.c)),
+                                        _stream(route_stream), _stream(offload_stream), ctypes.byref(sched.c)),
            "hga_segment_fwd_tiered")
 
 

@@ -589,11 +589,17 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
     }
     if (p->n_hist_chunks == 0) {
         // nothing routable: plain attention over the segment, after whatever the copy
-        // stream holds (the caller may have written idx or the inputs there)
+        // stream holds (the caller may have written idx or the inputs there); it reads
+        // idx itself, so the copy stream's later work waits for it
         if ((e = cudaEventRecord(sched->fetched, copy_stream)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(stream, sched->fetched, 0)) != cudaSuccess)
             return hga::record_cuda(e);
-        return hga_attn_fwd(p, q, stage_k, stage_v, k_seg, v_seg, idx, out, lse, stream);
+        st = hga_attn_fwd(p, q, stage_k, stage_v, k_seg, v_seg, idx, out, lse, stream);
+        if (st != HGA_OK) return st;
+        if ((e = cudaEventRecord(sched->start, stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(copy_stream, sched->start, 0)) != cudaSuccess)
+            return hga::record_cuda(e);
+        return HGA_OK;
     }
     for (int b0 = qb0; b0 < qb1; b0 += wave_blocks) {
         const int b1 = b0 + wave_blocks < qb1 ? b0 + wave_blocks : qb1;
@@ -624,12 +630,13 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
                                     void *out, float *lse, void *stage_k, void *stage_v, int stage_slots,
                                     int32_t *scratch, int32_t *idx_remapped, int wave_blocks, int flags,
                                     int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,
-                                    cudaStream_t offload_stream, hga_tier_sched_t *sched) {
+                                    cudaStream_t route_stream, cudaStream_t offload_stream, hga_tier_sched_t *sched) {
     CallRange range("hga_segment_fwd_tiered");
     if (!p || !sched || (flags & ~HGA_TIER_RESET)) return HGA_ERR_INVALID_ARG;
     hga_status_t st = check_params(p);
     if (st != HGA_OK) return st;
-    if (!sched->inputs || !sched->offloaded[0] || !sched->offloaded[1] || sched->segment < 0)
+    if (!sched->inputs || !sched->offloaded[0] || !sched->offloaded[1] || !sched->routed || !sched->idx_free[0] ||
+        !sched->idx_free[1] || !sched->start || sched->segment < 0)
         return HGA_ERR_INVALID_ARG;
     if (p->seg_len % p->chunk != 0) return HGA_ERR_INVALID_ARG;
     const int seg_chunks = p->seg_len / p->chunk;
@@ -641,30 +648,38 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
     cudaError_t e = cudaSuccess;
     if (reset) {  // the evaluation starts: the side streams after whatever came before it
         if ((e = cudaEventRecord(sched->start, stream)) != cudaSuccess ||
-            (e = cudaStreamWaitEvent(copy_stream, sched->start, 0)) != cudaSuccess)
+            (e = cudaStreamWaitEvent(copy_stream, sched->start, 0)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(route_stream, sched->start, 0)) != cudaSuccess)
             return hga::record_cuda(e);
         sched->segment = 0;
     }
     const long long seg = sched->segment;
     // detach into the host tier once the segment's K/V are there
-    if ((e = cudaEventRecord(sched->inputs, copy_stream)) != cudaSuccess ||
+    if ((e = cudaEventRecord(sched->inputs, route_stream)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(offload_stream, sched->inputs, 0)) != cudaSuccess)
         return hga::record_cuda(e);
     st = hga_tier_offload(p, k_seg, v_seg, host_k, host_v, T, offload_stream);
     if (st != HGA_OK) return st;
     if ((e = cudaEventRecord(sched->offloaded[seg & 1], offload_stream)) != cudaSuccess) return hga::record_cuda(e);
-    st = hga_route(p, q, summ, summ_cap_chunks, idx, copy_stream);
+    // the route; its idx buffer was last read by the fetches of segment seg - 2
+    if (seg >= 2 && (e = cudaStreamWaitEvent(route_stream, sched->idx_free[seg & 1], 0)) != cudaSuccess)
+        return hga::record_cuda(e);
+    st = hga_route(p, q, summ, summ_cap_chunks, idx, route_stream);
     if (st != HGA_OK) return st;
-    // this segment's fetches read the rows the previous segment offloaded
+    // this segment's fetches: after its route and after the rows the previous segment offloaded
+    if ((e = cudaEventRecord(sched->routed, route_stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(copy_stream, sched->routed, 0)) != cudaSuccess)
+        return hga::record_cuda(e);
     if (seg > 0 && (e = cudaStreamWaitEvent(copy_stream, sched->offloaded[(seg - 1) & 1], 0)) != cudaSuccess)
         return hga::record_cuda(e);
     st = hga_attn_fwd_tiered(p, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v, stage_slots,
                              scratch, idx_remapped, wave_blocks, reset ? HGA_TIER_RESET : HGA_TIER_CHAIN, n_fetched,
                              stream, copy_stream, sched);
     if (st != HGA_OK) return st;
+    if ((e = cudaEventRecord(sched->idx_free[seg & 1], copy_stream)) != cudaSuccess) return hga::record_cuda(e);
     // detach: the segment's chunks become routable for the next segment
     st = hga::launch_summaries(k_seg, p->seg_head_stride, p->batch * p->n_kv_heads, p->head_dim, p->chunk,
-                               p->n_hist_chunks, seg_chunks, p->dtype, summ, summ_cap_chunks, copy_stream,
+                               p->n_hist_chunks, seg_chunks, p->dtype, summ, summ_cap_chunks, route_stream,
                                p->n_hist_chunks);
     if (st != HGA_OK) return st;
     sched->segment = seg + 1;

@@ -416,8 +416,8 @@ hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const vo
  * attention of the lag - 1 waves before it.  The cache then holds the tiles of
  * lag waves: stage_slots >= min(lag * wave_blocks * B * Hkv * min(k, Nc),
  * B * Hkv * Nc).
- *   Create the events (cudaEventDisableTiming is enough; inputs and
- *   offloaded only for hga_segment_fwd_tiered), set lag (2 ..
+ *   Create the events (cudaEventDisableTiming is enough; inputs, offloaded,
+ *   routed and idx_free only for hga_segment_fwd_tiered), set lag (2 ..
  *   HGA_TIER_MAX_LAG), wave = 0 and segment = 0; the library records the
  *   events and advances the counters.  Use one compute stream and one copy stream for all calls of
  *   a schedule, and no other fetch into its cache (hga_fetch_tiered,
@@ -430,6 +430,8 @@ typedef struct {
     cudaEvent_t consumed[HGA_TIER_MAX_LAG];  /* fetch of wave h after the attention of wave h - lag */
     cudaEvent_t inputs;                      /* hga_segment_fwd_tiered: the offload after the segment's inputs */
     cudaEvent_t offloaded[2];                /* hga_segment_fwd_tiered: fetches after the previous offload */
+    cudaEvent_t routed;                      /* hga_segment_fwd_tiered: fetches after the segment's route */
+    cudaEvent_t idx_free[2];                 /* hga_segment_fwd_tiered: a route after the last reader of its idx */
     int lag;
     long long wave;                          /* waves issued through the schedule since its cache was emptied */
     long long segment;                       /* segments through hga_segment_fwd_tiered since then */
@@ -441,7 +443,8 @@ typedef struct {
  * earlier waves' attention runs on stream, ordered by sched (above).  Output
  * (out, lse) is bit-identical to hga_attn_fwd with the history resident.  On
  * return, stream is ordered after every fetch of the call (with Nc = 0, after
- * all work then on copy_stream).
+ * all work then on copy_stream, and copy_stream after the attention, which
+ * reads idx).
  *   flags: HGA_TIER_RESET empties the cache first (and sets sched->wave = 0).
  *   Without HGA_TIER_CHAIN, and always with HGA_TIER_RESET, the copy stream
  *   first waits for everything already enqueued on stream (the route that
@@ -468,26 +471,28 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
 /* One segment of an evaluation whose detached history lives in page-locked
  * host memory (technical summary section 2.2, tiered memory; section 2.1 for
  * the route and the exact-token attention; the segment detaches at its end),
- * on three streams, so that a segment's route and fetches run under the
- * previous segment's attention:
- *   copy_stream   : hga_route of the segment into idx; the fetch waves of
- *                   hga_attn_fwd_tiered, chained from the previous segment,
- *                   the first after the previous segment's offload; then the
- *                   detach-time append of the segment's S / chunk summaries
- *                   to chunks [Nc, Nc + S / chunk) of summ.
+ * on four streams, so that a segment's route and fetches run under the
+ * attention of the segments before it:
+ *   route_stream  : hga_route of the segment into idx, then the detach-time
+ *                   append of the segment's S / chunk summaries to chunks
+ *                   [Nc, Nc + S / chunk) of summ.
+ *   copy_stream   : the fetch waves of hga_attn_fwd_tiered, chained from the
+ *                   previous segment, after the segment's route and the
+ *                   previous segment's offload.
  *   offload_stream: k_seg / v_seg copied to tokens [T, T + S) of host_k /
  *                   host_v (T = Nc * chunk) once the inputs are ready.
  *   stream        : the attention waves, writing out and lse.
- * q, k_seg and v_seg must be ready in copy_stream's order (the caller copies
- * them in there, or orders copy_stream after their producer).  flags:
- * HGA_TIER_RESET for the evaluation's first segment (copy_stream first waits
- * for stream; the cache is emptied; sched->wave and sched->segment restart);
- * 0 continues the evaluation.  On return stream is ordered after the
- * segment's fetches; the append and the offload are ordered before the next
- * call's fetches, and the caller orders stream after copy_stream and
- * offload_stream before it reads summ or the host history itself.
- * idx_remapped as in hga_attn_fwd_tiered (rotate ceil(lag / waves per
- * segment) buffers over the segments).  HGA_ERR_INVALID_ARG when
+ * q, k_seg and v_seg must be ready in route_stream's order (the caller copies
+ * them in there, or orders route_stream after their producer).  idx: the
+ * segment's route table; the route of segment s + 2 waits until the fetches
+ * of segment s have read theirs, so rotate two buffers (a route may then run
+ * a segment ahead).  flags: HGA_TIER_RESET for the evaluation's first segment
+ * (the side streams first wait for stream; the cache is emptied;
+ * sched->wave and sched->segment restart); 0 continues the evaluation.  On
+ * return stream is ordered after the segment's fetches; the caller orders
+ * stream after route_stream and offload_stream before it reads summ or the
+ * host history itself.  idx_remapped as in hga_attn_fwd_tiered (rotate
+ * ceil(lag / waves per segment) buffers).  HGA_ERR_INVALID_ARG when
  * summ_cap_chunks < Nc + S / chunk, T + S > hist_head_stride, the host
  * history is not page-locked, or an event of sched is null; other arguments
  * and checks as hga_route, hga_attn_fwd_tiered and hga_tier_offload. */
@@ -496,7 +501,7 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
                                     void *out, float *lse, void *stage_k, void *stage_v, int stage_slots,
                                     int32_t *scratch, int32_t *idx_remapped, int wave_blocks, int flags,
                                     int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,
-                                    cudaStream_t offload_stream, hga_tier_sched_t *sched);
+                                    cudaStream_t route_stream, cudaStream_t offload_stream, hga_tier_sched_t *sched);
 
 /* Self-test of the bounded waits (the source pages have no counterpart): every
  * pipeline wait in the tensor-core kernels gives up after a cycle limit instead

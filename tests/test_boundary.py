@@ -184,12 +184,13 @@ def test_segment_tiered_checked_on_host(L):
     sc.start = sc.fetched = sc.inputs = 0x10
     sc.consumed[0] = sc.consumed[1] = 0x10
     sc.offloaded[0] = sc.offloaded[1] = 0x10
+    sc.routed = sc.idx_free[0] = sc.idx_free[1] = 0x10
     sc.lag = 2
     seg_chunks = p.seg_len // 64
 
     def call(pp, cap, flags=0, sched=sc):
         return L.hga_segment_fwd_tiered(ctypes.byref(pp.c()), fake, fake, fake, fake, cap, fake, fake, fake, fake,
-                                        fake, fake, fake, 64, fake, fake, 2, flags, None, None, None, None,
+                                        fake, fake, fake, 64, fake, fake, 2, flags, None, None, None, None, None,
                                         ctypes.byref(sched) if sched is not None else None)
 
     assert call(p, 32 + seg_chunks - 1) == -1  # no room to append the segment's summaries
@@ -200,6 +201,9 @@ def test_segment_tiered_checked_on_host(L):
     assert call(p, 4096) == -1
     sc.offloaded[1] = 0x10
     sc.inputs = 0
+    assert call(p, 4096) == -1
+    sc.inputs = 0x10
+    sc.idx_free[0] = 0
     assert call(p, 4096) == -1
 
 

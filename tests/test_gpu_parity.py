@@ -489,10 +489,11 @@ CHAIN = gen.custom("chain_bf16", n_q_heads=8, n_kv_heads=2, head_dim=128, topk=4
 def test_tiered_chained_segments_match_resident(wave, lag, slots):
     """An evaluation of six segments with the history only in pinned host memory,
     through hga_segment_fwd_tiered as the benchmark runs it: each segment's K/V
-    offloaded to the host history on a third stream, its route, fetch waves and
-    summary append on the copy stream, its attention waves on the compute stream,
-    chained from segment to segment (no host synchronisation anywhere), so fetches of
-    a segment run under the attention of the one before it.  The host history starts as NaN, so a
+    offloaded to the host history on one stream, its route and summary append on a
+    second, its fetch waves on a third (all three at high priority), its attention
+    waves on the compute stream, chained from segment to segment (no host
+    synchronisation anywhere), so a segment's route and fetches run under the
+    attention of the segments before it.  The host history starts as NaN, so a
     fetch that overtook an offload, or an eviction of a slot still being read, changes
     the output.  Every segment's out and lse equal the resident forward on the same
     routes bit for bit.  Slots: the least the schedule accepts, min(lag x wave x B x
@@ -530,21 +531,24 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots):
     n_waves = -(-nqb // wave)
     idx_r = [torch.full((w.batch, w.n_kv_heads, nqb, w.topk), -5, device="cuda", dtype=torch.int32)
              for _ in range(-(-lag // n_waves))]
-    idx = torch.full_like(idx_r[0], 7)  # stale routes: read before the first route, they would be flagged
+    # stale routes: read before the route that rewrites them, they would be flagged
+    idx = [torch.full_like(idx_r[0], 7) for _ in range(2)]
     sched = hga.TierSched(lag=lag)
-    compute, copy, off = torch.cuda.current_stream(), torch.cuda.Stream(), torch.cuda.Stream()
+    compute = torch.cuda.current_stream()
+    copy, route_s, off = (torch.cuda.Stream(priority=-1) for _ in range(3))
     nf = torch.zeros(len(w.seg_starts), n_waves, device="cuda", dtype=torch.int32)
     got = {}
     for si, T in enumerate(w.seg_starts):
         p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
         out = torch.full_like(qs[T], float("nan"))
         lse = torch.full(qs[T].shape[:3], float("nan"), device="cuda")
-        hga.hga_segment_fwd_tiered(p, qs[T], k_all[:, :, T:], v_all[:, :, T:], summ, nct, idx, host_k, host_v, out,
-                                   lse, stage_k, stage_v, slots, scratch, idx_r[si % len(idx_r)], wave, sched,
-                                   reset=si == 0, n_fetched=nf[si], copy_stream=copy, offload_stream=off)
+        hga.hga_segment_fwd_tiered(p, qs[T], k_all[:, :, T:], v_all[:, :, T:], summ, nct, idx[si % 2], host_k,
+                                   host_v, out, lse, stage_k, stage_v, slots, scratch, idx_r[si % len(idx_r)], wave,
+                                   sched, reset=si == 0, n_fetched=nf[si], copy_stream=copy, route_stream=route_s,
+                                   offload_stream=off)
         got[T] = (out, lse)
-    compute.wait_stream(copy)
-    compute.wait_stream(off)
+    for st in (copy, route_s, off):
+        compute.wait_stream(st)
     torch.cuda.synchronize()
     assert hga.hga_get_device_status() == 0
     for T in w.seg_starts:
