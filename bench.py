@@ -101,6 +101,9 @@ def parse():
     ap.add_argument("--tier-wave", type=int, default=64, help="query blocks per fetch wave of the tiered workload")
     ap.add_argument("--tier-lag", type=int, default=2,
                     help="a tiered fetch wave waits for the attention this many waves back (2..4)")
+    ap.add_argument("--tier-host-only", action="store_true",
+                    help="tiered fetches read every chunk from the host history (default: the previous "
+                         "segment's chunks from its K/V still in device memory)")
     ap.add_argument("--only-last-segment", action="store_true",
                     help="a step processes only the workload's last segment (its history summarised up "
                          "front): for counter captures of the longest launches with few launches before them")
@@ -247,6 +250,7 @@ class Layer:
 
     wave = 64  # query blocks per tiered fetch wave
     lag = 2  # a tiered fetch waits for the attention this many waves back
+    prev_source = True  # tiered fetches copy the previous segment's chunks from its device K/V
 
     def __init__(self, w):
         import torch
@@ -389,6 +393,11 @@ class Layer:
         p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
+        # the previous segment's K/V are still in device memory: its chunks are
+        # copied from there rather than back across the host link
+        prev = si > 0 and self.prev_source and T >= w.seg_len
+        pk = self.k[:, :, T - w.seg_len:] if prev else None
+        pv = self.v[:, :, T - w.seg_len:] if prev else None
         if ev is not None:
             ev.record("attn_fwd")
         first = si == 0
@@ -396,7 +405,8 @@ class Layer:
                                    self.host_v, self.out, self.lse, self.stage_k, self.stage_v, self.slots,
                                    self.scratch, self.idx_r[si % len(self.idx_r)], self.wave, self.sched,
                                    reset=first, n_fetched=self.n_fetched[si], copy_stream=self.copy_stream,
-                                   route_stream=self.route_stream, offload_stream=self.offload_stream)
+                                   route_stream=self.route_stream, offload_stream=self.offload_stream,
+                                   prev_k_seg=pk, prev_v_seg=pv)
         if ev is not None:
             ev.record(None)
         # route, reset (first segment), fetch waves (plan, copy, remap) + attention, append
@@ -718,21 +728,38 @@ def run_reference(args, rank):
 
 
 def host_link_gbs(nbytes=256 << 20):
-    """Pinned host -> device copy bandwidth measured here (the tiered path's roofline)."""
+    """Pinned host <-> device copy bandwidth measured here (the tiered path's roofline):
+    host -> device alone, device -> host alone, and both directions at once (two
+    streams; the sum of the bytes over the time of the pair), each the best of five."""
     import torch
-    h = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
-    d = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
-    d.copy_(h, non_blocking=True)
-    torch.cuda.synchronize()
-    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    best = 0.0
-    for _ in range(5):
-        s.record()
-        d.copy_(h, non_blocking=True)
-        e.record()
-        e.synchronize()
-        best = max(best, nbytes / (s.elapsed_time(e) / 1000) / 1e9)
-    return best
+    h_in = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h_out = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d_in = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    d_out = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    main = torch.cuda.current_stream()
+
+    def best(h2d, d2h):
+        top = 0.0
+        for _ in range(6):
+            s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            s.record(main)
+            s_in.wait_stream(main)
+            s_out.wait_stream(main)
+            if h2d:
+                with torch.cuda.stream(s_in):
+                    d_in.copy_(h_in, non_blocking=True)
+            if d2h:
+                with torch.cuda.stream(s_out):
+                    h_out.copy_(d_out, non_blocking=True)
+            main.wait_stream(s_in)
+            main.wait_stream(s_out)
+            e.record(main)
+            e.synchronize()
+            top = max(top, (int(h2d) + int(d2h)) * nbytes / (s.elapsed_time(e) / 1000) / 1e9)
+        return top
+
+    return {"h2d": best(True, False), "d2h": best(False, True), "both": best(True, True)}
 
 
 def measure_layer(w, args, world, local):
@@ -741,6 +768,7 @@ def measure_layer(w, args, world, local):
     import hierarchical_sparse_long_b200 as hga
     Layer.wave = args.tier_wave
     Layer.lag = args.tier_lag
+    Layer.prev_source = not args.tier_host_only
     if args.only_last_segment:
         import dataclasses
         w = dataclasses.replace(w, seg_starts=w.seg_starts[-1:])
@@ -874,10 +902,15 @@ def measure_layer(w, args, world, local):
         res["tiered"] = tiered_report(layer, total_ms / args.steps, ph["attn_fwd"] / args.steps, flush)
         # the step's dominant cost is the host link: its own roofline line
         t = res["tiered"]
-        res["roofline_host_link"] = {"bound": "host link", "achieved": t["link_gbs_achieved"],
-                                     "peak": t["host_link_gbs_measured"], "unit": "GB/s",
-                                     "frac": round(t["link_gbs_achieved"] / t["host_link_gbs_measured"], 4),
-                                     "peak_source": "pinned host -> device cudaMemcpyAsync measured in this run"}
+        # the fetches (host -> device) and the detach copies (device -> host) share the
+        # link: both directions' bytes over the step against both directions at once
+        pk = t["host_link_gbs_measured"]["both"]
+        res["roofline_host_link"] = {"bound": "host link", "achieved": t["link_both_gbs_achieved"],
+                                     "peak": pk, "unit": "GB/s",
+                                     "frac": round(t["link_both_gbs_achieved"] / pk, 4),
+                                     "traffic": t["bytes_fetched_per_step"] + t["bytes_offloaded_per_step"],
+                                     "peak_source": "pinned cudaMemcpyAsync host -> device and device -> host "
+                                                    "at once on two streams, measured in this run"}
     res["e2e"] = e2e_measure(layer, max(2, min(args.steps, 5)))
     del layer, graph
     torch.cuda.synchronize()
@@ -886,8 +919,10 @@ def measure_layer(w, args, world, local):
 
 
 def tiered_report(layer, step_ms, attn_phase_ms, flush):
-    """Host-link accounting of the tiered step: tiles fetched per step against the
-    distinct tiles the segments route to, the fetch-only step and the resident
+    """Host-link accounting of the tiered step: tiles fetched from the host per step
+    (the previous segment's chunks come from device memory unless --tier-host-only)
+    against the distinct tiles the segments route to, the fetch-only step (every
+    chunk from the host) and the resident
     attention (no host link), and the share of the attention hidden under the
     fetches: (fetch-only + resident attention - tiered attention phase) /
     resident attention, the tiered phase being the fetch waves and attention of
@@ -907,11 +942,15 @@ def tiered_report(layer, step_ms, attn_phase_ms, flush):
     t_res = ev.totals()["attn_fwd"]
     link = host_link_gbs()
     tb = TILE_PAIR_BYTES(w)
+    # the detach copies every segment's K/V to the host history: device -> host bytes
+    off_b = len(w.seg_starts) * w.batch * w.n_kv_heads * w.seg_len * w.head_dim * 2 * 2
     hidden = (t_fetch + t_res - attn_phase_ms) / t_res if t_res > 0 else None
     return {"staging_slots": layer.slots, "staging_mib": round(layer.slots * tb / 2**20, 1),
             "cache_policy": "one segment's routing budget of chunk tiles, kept from segment to segment and "
                             f"emptied when the evaluation starts; waves of {layer.wave} query blocks, a fetch "
                             f"after the attention {layer.lag} waves back",
+            "fetch_source": "host history; the previous segment's chunks from its K/V still in device memory"
+                            if layer.prev_source else "host history for every chunk",
             "tiles_fetched_per_step": fetched, "tiles_distinct_per_segment_summed": per_segment,
             "tiles_distinct_per_step": whole,
             "bytes_fetched_per_step": fetched * tb, "bytes_distinct_per_segment_summed": per_segment * tb,
@@ -919,8 +958,10 @@ def tiered_report(layer, step_ms, attn_phase_ms, flush):
             "ms_fetch_only_step": round(t_fetch, 3), "ms_attention_resident": round(t_res, 3),
             "ms_attention_phase_tiered": round(attn_phase_ms, 3),
             "attention_hidden_share": round(hidden, 4) if hidden is not None else None,
+            "bytes_offloaded_per_step": off_b,
             "link_gbs_achieved": round(fetched * tb / (step_ms / 1e3) / 1e9, 2),
-            "host_link_gbs_measured": round(link, 2)}
+            "link_both_gbs_achieved": round((fetched * tb + off_b) / (step_ms / 1e3) / 1e9, 2),
+            "host_link_gbs_measured": {k: round(v, 2) for k, v in link.items()}}
 
 
 def e2e_measure(layer, steps):

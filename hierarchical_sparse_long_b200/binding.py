@@ -112,10 +112,10 @@ def lib() -> ctypes.CDLL:
         L.hga_tier_reset.argtypes = [pp, i, vp, vp]
         L.hga_fetch_tiered.argtypes = [pp, vp, vp, vp, i, i, vp, vp, i, vp, vp, vp, vp, vp]
         L.hga_tier_offload.argtypes = [pp, vp, vp, vp, vp, ll, vp]
-        L.hga_attn_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp, vp, vp,
-                                          ctypes.POINTER(_TierSchedC)]
-        L.hga_segment_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp,
-                                             vp, vp, vp, vp, ctypes.POINTER(_TierSchedC)]
+        L.hga_attn_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp, vp,
+                                          vp, ctypes.POINTER(_TierSchedC)]
+        L.hga_segment_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i,
+                                             i, vp, vp, vp, vp, vp, ctypes.POINTER(_TierSchedC)]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
         L.hga_selftest_wait_timeout.argtypes = [ll, vp]
         L.hga_selftest_wait_timeout.restype = ctypes.c_int
@@ -385,13 +385,16 @@ class TierSched:
 
 def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v,
                         stage_slots: int, scratch, idx_remapped, wave_blocks: int, sched: TierSched,
-                        reset_cache=False, chain=False, n_fetched=None, stream=None, copy_stream=None):
+                        reset_cache=False, chain=False, n_fetched=None, stream=None, copy_stream=None,
+                        prev_k_seg=None, prev_v_seg=None):
     """Attention over host-resident history: fetch waves on copy_stream overlapped with
-    earlier waves' attention on stream, ordered by sched (a TierSched)."""
+    earlier waves' attention on stream, ordered by sched (a TierSched); the previous
+    segment's chunks are copied from prev_k_seg / prev_v_seg when given."""
     cp = p.c()
     flags = (HGA_TIER_RESET if reset_cache else 0) | (HGA_TIER_CHAIN if chain else 0)
     _check(lib().hga_attn_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(host_k), _ptr(host_v), _ptr(k_seg),
-                                     _ptr(v_seg), _ptr(idx), _ptr(out), _ptr(lse), _ptr(stage_k), _ptr(stage_v),
+                                     _ptr(v_seg), _ptr(prev_k_seg), _ptr(prev_v_seg), _ptr(idx), _ptr(out),
+                                     _ptr(lse), _ptr(stage_k), _ptr(stage_v),
                                      stage_slots, _ptr(scratch), _ptr(idx_remapped), wave_blocks, flags,
                                      _ptr(n_fetched), _stream(stream), _stream(copy_stream), ctypes.byref(sched.c)),
            "hga_attn_fwd_tiered")
@@ -400,11 +403,13 @@ def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, ls
 def hga_segment_fwd_tiered(p: Params, q, k_seg, v_seg, summ, summ_cap_chunks: int, idx, host_k, host_v, out, lse,
                            stage_k, stage_v, stage_slots: int, scratch, idx_remapped, wave_blocks: int,
                            sched: TierSched, reset=False, n_fetched=None, stream=None, copy_stream=None,
-                           route_stream=None, offload_stream=None):
+                           route_stream=None, offload_stream=None, prev_k_seg=None, prev_v_seg=None):
     """One segment of a tiered evaluation: route and summary append on route_stream,
-    fetches on copy_stream, the K/V offload on offload_stream, attention on stream."""
+    fetches on copy_stream (the previous segment's chunks from prev_k_seg / prev_v_seg
+    when given), the K/V offload on offload_stream, attention on stream."""
     cp = p.c()
-    _check(lib().hga_segment_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(summ),
+    _check(lib().hga_segment_fwd_tiered(ctypes.byref(cp), _ptr(q), _ptr(k_seg), _ptr(v_seg), _ptr(prev_k_seg),
+                                        _ptr(prev_v_seg), _ptr(summ),
                                         summ_cap_chunks, _ptr(idx), _ptr(host_k), _ptr(host_v), _ptr(out), _ptr(lse),
                                         _ptr(stage_k), _ptr(stage_v), stage_slots, _ptr(scratch),
                                         _ptr(idx_remapped), wave_blocks, HGA_TIER_RESET if reset else 0,

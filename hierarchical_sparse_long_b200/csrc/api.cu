@@ -550,7 +550,8 @@ hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const vo
 }
 
 hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const void *host_k, const void *host_v,
-                                 const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
+                                 const void *k_seg, const void *v_seg, const void *prev_k_seg,
+                                 const void *prev_v_seg, const int32_t *idx, void *out, float *lse,
                                  void *stage_k, void *stage_v, int stage_slots, int32_t *scratch,
                                  int32_t *idx_remapped, int wave_blocks, int flags, int32_t *n_fetched,
                                  cudaStream_t stream, cudaStream_t copy_stream, hga_tier_sched_t *sched) {
@@ -568,6 +569,9 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
                                    wave_blocks, lag);
     if (st != HGA_OK) return st;
     if (!q || !k_seg || !v_seg || !out || !lse) return HGA_ERR_INVALID_ARG;
+    if ((prev_k_seg == nullptr) != (prev_v_seg == nullptr)) return HGA_ERR_INVALID_ARG;
+    if (prev_k_seg && (p->n_hist_chunks < p->seg_len / p->chunk || !aligned16(prev_k_seg) || !aligned16(prev_v_seg)))
+        return HGA_ERR_INVALID_ARG;
     hga_params_t pa = *p;  // attention over the staging cache: route indices are slots
     pa.hist_head_stride = 0;
     pa.n_hist_chunks = stage_slots;
@@ -610,7 +614,7 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
             return hga::record_cuda(e);
         st = hga::launch_fetch_tiered(*p, host_k, host_v, idx, b0, b1, stage_k, stage_v, stage_slots, lag, scratch,
                                       idx_remapped, n_fetched ? n_fetched + (b0 - qb0) / wave_blocks : nullptr,
-                                      status, copy_stream);
+                                      status, copy_stream, prev_k_seg, prev_v_seg);
         if (st != HGA_OK) return st;
         if ((e = cudaEventRecord(sched->fetched, copy_stream)) != cudaSuccess ||
             (e = cudaStreamWaitEvent(stream, sched->fetched, 0)) != cudaSuccess)
@@ -626,7 +630,8 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
 }
 
 hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const void *k_seg, const void *v_seg,
-                                    float *summ, int summ_cap_chunks, int32_t *idx, void *host_k, void *host_v,
+                                    const void *prev_k_seg, const void *prev_v_seg, float *summ,
+                                    int summ_cap_chunks, int32_t *idx, void *host_k, void *host_v,
                                     void *out, float *lse, void *stage_k, void *stage_v, int stage_slots,
                                     int32_t *scratch, int32_t *idx_remapped, int wave_blocks, int flags,
                                     int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,
@@ -654,6 +659,12 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
         sched->segment = 0;
     }
     const long long seg = sched->segment;
+    // this segment's fetches read host rows the previous segment offloaded, or with
+    // prev_k_seg (whose chunks come from device memory) the one before; waited for
+    // here, before the offload below re-records the event of the ring
+    const long long need = seg - (prev_k_seg ? 2 : 1);
+    if (need >= 0 && (e = cudaStreamWaitEvent(copy_stream, sched->offloaded[need & 1], 0)) != cudaSuccess)
+        return hga::record_cuda(e);
     // detach into the host tier once the segment's K/V are there
     if ((e = cudaEventRecord(sched->inputs, route_stream)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(offload_stream, sched->inputs, 0)) != cudaSuccess)
@@ -666,15 +677,13 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
         return hga::record_cuda(e);
     st = hga_route(p, q, summ, summ_cap_chunks, idx, route_stream);
     if (st != HGA_OK) return st;
-    // this segment's fetches: after its route and after the rows the previous segment offloaded
+    // this segment's fetches: after its route
     if ((e = cudaEventRecord(sched->routed, route_stream)) != cudaSuccess ||
         (e = cudaStreamWaitEvent(copy_stream, sched->routed, 0)) != cudaSuccess)
         return hga::record_cuda(e);
-    if (seg > 0 && (e = cudaStreamWaitEvent(copy_stream, sched->offloaded[(seg - 1) & 1], 0)) != cudaSuccess)
-        return hga::record_cuda(e);
-    st = hga_attn_fwd_tiered(p, q, host_k, host_v, k_seg, v_seg, idx, out, lse, stage_k, stage_v, stage_slots,
-                             scratch, idx_remapped, wave_blocks, reset ? HGA_TIER_RESET : HGA_TIER_CHAIN, n_fetched,
-                             stream, copy_stream, sched);
+    st = hga_attn_fwd_tiered(p, q, host_k, host_v, k_seg, v_seg, prev_k_seg, prev_v_seg, idx, out, lse, stage_k,
+                             stage_v, stage_slots, scratch, idx_remapped, wave_blocks,
+                             reset ? HGA_TIER_RESET : HGA_TIER_CHAIN, n_fetched, stream, copy_stream, sched);
     if (st != HGA_OK) return st;
     if ((e = cudaEventRecord(sched->idx_free[seg & 1], copy_stream)) != cudaSuccess) return hga::record_cuda(e);
     // detach: the segment's chunks become routable for the next segment

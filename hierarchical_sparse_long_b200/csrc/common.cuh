@@ -148,7 +148,8 @@ hga_status_t launch_tier_reset(const hga_params_t &p, int stage_slots, int32_t *
 hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
                                  int stage_slots, int lag, int32_t *scratch, int32_t *idx_remapped,
-                                 int32_t *n_fetched, unsigned *status, cudaStream_t stream);
+                                 int32_t *n_fetched, unsigned *status, cudaStream_t stream,
+                                 const void *prev_k = nullptr, const void *prev_v = nullptr);
 hga_status_t launch_selftest_wait_timeout(long long wait_cycles, unsigned *status, cudaStream_t stream);
 hga_status_t record_cuda(cudaError_t e);
 void record_error(const char *msg);

@@ -25,7 +25,10 @@
 //   copy   : an SM copy of each listed K and V tile straight from the mapped
 //          host pages into its slot (16-byte loads, many in flight, so the
 //          host link rather than the SMs is the bound; CTAs small enough to
-//          share an SM with an attention CTA);
+//          share an SM with an attention CTA) -- or, for the chunks of the
+//          segment that detached last, from its K/V still in device memory
+//          (the same bytes the host history received), so a chunk crosses
+//          the host link only when it is older than that;
 //   remap  : idx_remapped = slot of each routed chunk (-1 stays -1).
 // The caller guarantees that the attention of wave w-lag has finished before
 // the fetch of wave w starts (hga_attn_fwd_tiered orders its two streams so);
@@ -46,6 +49,14 @@ constexpr int kFreeWave = -(1 << 30);  // slot_wave of an empty slot: free for e
 
 struct TierScratch {
     int32_t *tile_slot, *tile_mark, *slot_tile, *slot_wave, *new_tile, *new_slot, *ctl;
+};
+
+// Chunks [j0, j0 + nj) of every (b, g) read from device memory instead of the
+// host (k == nullptr: none); slice bg starts bg * head_stride_bytes in.
+struct DevSource {
+    const uint4 *k, *v;
+    long long head_stride_bytes, j0, nj;
+    __device__ bool holds(long long j) const { return k != nullptr && j >= j0 && j < j0 + nj; }
 };
 
 TierScratch tier_layout(int32_t *base, long long n_tiles, int slots) {
@@ -104,13 +115,16 @@ __device__ int block_scan(int f, int *warp_sums, int *total) {
 __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *__restrict__ idx, int n_bg, int nqb,
                                                                  int topk, int qb0, int qb1, int n_chunks,
                                                                  long long tile_cap, int slots, int lag,
-                                                                 TierScratch s, int32_t *n_fetched,
+                                                                 TierScratch s, DevSource dev, int32_t *n_fetched,
                                                                  unsigned *status) {
     __shared__ int warp_sums[32];
-    __shared__ int n_new, total, taken_sh, cursor_sh;
+    __shared__ int n_new, n_host, total, taken_sh, cursor_sh;
     const int tid = threadIdx.x;
     const int w = s.ctl[0] + 1;
-    if (tid == 0) n_new = 0;
+    if (tid == 0) {
+        n_new = 0;
+        n_host = 0;
+    }
     __syncthreads();
     // 1. the wave's distinct tiles: cached ones are stamped with w, the others listed
     const long long per_bg = (long long)(qb1 - qb0) * topk;
@@ -132,6 +146,7 @@ __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *
         } else {
             const int p = atomicAdd(&n_new, 1);
             if (p < slots) s.new_tile[p] = (int32_t)t;
+            if (!dev.holds(j)) atomicAdd(&n_host, 1);
         }
     }
     __syncthreads();
@@ -171,7 +186,7 @@ __global__ void __launch_bounds__(kPlanThreads) tier_plan_kernel(const int32_t *
         s.ctl[0] = w;
         s.ctl[1] = cursor_sh;
         s.ctl[2] = got;
-        if (n_fetched) *n_fetched = got;
+        if (n_fetched) *n_fetched = got < n_host ? got : n_host;  // the tiles that cross the host link
     }
 }
 
@@ -183,7 +198,7 @@ constexpr int kCopyThreads = 128;
 template <int ROW_BYTES>
 __global__ void __launch_bounds__(kCopyThreads, 8)
     tier_copy_kernel(const uint4 *__restrict__ host_k, const uint4 *__restrict__ host_v, long long head_stride_bytes,
-                     long long tile_cap, int chunk, TierScratch s, uint4 *__restrict__ stage_k,
+                     long long tile_cap, int chunk, TierScratch s, DevSource dev, uint4 *__restrict__ stage_k,
                      uint4 *__restrict__ stage_v) {
     constexpr int V_PER_ROW = ROW_BYTES / 16;
     constexpr int PER = 4;  // vectors of K and of V a thread holds in flight
@@ -193,10 +208,18 @@ __global__ void __launch_bounds__(kCopyThreads, 8)
         const long long t = s.new_tile[k];
         const int slot = s.new_slot[k];
         const long long bg = t / tile_cap, j = t % tile_cap;
-        const long long off = (bg * head_stride_bytes + j * chunk * ROW_BYTES) / 16;
         // host_v / stage_v are null when one tensor is staged (group summaries)
         const bool two = host_v != nullptr;
-        const uint4 *sk = host_k + off, *sv = two ? host_v + off : nullptr;
+        const uint4 *sk, *sv;
+        if (dev.holds(j)) {
+            const long long off = (bg * dev.head_stride_bytes + (j - dev.j0) * chunk * ROW_BYTES) / 16;
+            sk = dev.k + off;
+            sv = two ? dev.v + off : nullptr;
+        } else {
+            const long long off = (bg * head_stride_bytes + j * chunk * ROW_BYTES) / 16;
+            sk = host_k + off;
+            sv = two ? host_v + off : nullptr;
+        }
         uint4 *dk = stage_k + (long long)slot * tile_vecs, *dv = two ? stage_v + (long long)slot * tile_vecs : nullptr;
         // every load of a round is issued before its stores
         for (int e0 = threadIdx.x; e0 < tile_vecs; e0 += PER * kCopyThreads) {
@@ -263,7 +286,8 @@ namespace {
 hga_status_t fetch_wave(const hga_params_t &p, const void *host_k, const void *host_v, int tile_rows, int row_bytes,
                         long long head_stride_rows, long long tile_cap, const int32_t *idx, int qb0, int qb1,
                         void *stage_k, void *stage_v, int stage_slots, int lag, int32_t *scratch,
-                        int32_t *idx_remapped, int32_t *n_fetched, unsigned *status, cudaStream_t stream) {
+                        int32_t *idx_remapped, int32_t *n_fetched, unsigned *status, cudaStream_t stream,
+                        const DevSource &dev) {
     const int n_bg = p.batch * p.n_kv_heads;
     const int nqb = p.seg_len / p.q_block;
     const TierScratch s = tier_layout(scratch, (long long)n_bg * tile_cap, stage_slots);
@@ -276,20 +300,20 @@ hga_status_t fetch_wave(const hga_params_t &p, const void *host_k, const void *h
         return HGA_ERR_INVALID_ARG;
     }
     tier_plan_kernel<<<1, kPlanThreads, 0, stream>>>(idx, n_bg, nqb, p.topk, qb0, qb1, p.n_hist_chunks, tile_cap,
-                                                     stage_slots, lag, s, n_fetched, status);
+                                                     stage_slots, lag, s, dev, n_fetched, status);
     const long long head_stride_bytes = head_stride_rows * row_bytes;
     const unsigned g3 = (unsigned)(2 * sm_count());
     const uint4 *hk = static_cast<const uint4 *>(dk), *hv = static_cast<const uint4 *>(dv);
     uint4 *sk = static_cast<uint4 *>(stage_k), *sv = static_cast<uint4 *>(stage_v);
     if (row_bytes == 128)
-        tier_copy_kernel<128><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, sk,
-                                                               sv);
+        tier_copy_kernel<128><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, dev,
+                                                               sk, sv);
     else if (row_bytes == 256)
-        tier_copy_kernel<256><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, sk,
-                                                               sv);
+        tier_copy_kernel<256><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, dev,
+                                                               sk, sv);
     else
-        tier_copy_kernel<512><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, sk,
-                                                               sv);
+        tier_copy_kernel<512><<<g3, kCopyThreads, 0, stream>>>(hk, hv, head_stride_bytes, tile_cap, tile_rows, s, dev,
+                                                               sk, sv);
     const long long marks = (long long)n_bg * (qb1 - qb0) * p.topk;
     const unsigned g1 = (unsigned)((marks + 255) / 256 > 1184 ? 1184 : (marks + 255) / 256);
     if (marks > 0)
@@ -303,10 +327,19 @@ hga_status_t fetch_wave(const hga_params_t &p, const void *host_k, const void *h
 hga_status_t launch_fetch_tiered(const hga_params_t &p, const void *host_k, const void *host_v,
                                  const int32_t *idx, int qb0, int qb1, void *stage_k, void *stage_v,
                                  int stage_slots, int lag, int32_t *scratch, int32_t *idx_remapped,
-                                 int32_t *n_fetched, unsigned *status, cudaStream_t stream) {
+                                 int32_t *n_fetched, unsigned *status, cudaStream_t stream, const void *prev_k,
+                                 const void *prev_v) {
     const int esize = p.dtype == HGA_BF16 ? 2 : 4;
+    DevSource dev{nullptr, nullptr, 0, 0, 0};
+    if (prev_k && prev_v) {  // the segment before this one: chunks [Nc - S / chunk, Nc)
+        dev.k = static_cast<const uint4 *>(prev_k);
+        dev.v = static_cast<const uint4 *>(prev_v);
+        dev.head_stride_bytes = p.seg_head_stride * p.head_dim * esize;
+        dev.nj = p.seg_len / p.chunk;
+        dev.j0 = p.n_hist_chunks - dev.nj;
+    }
     return fetch_wave(p, host_k, host_v, p.chunk, p.head_dim * esize, p.hist_head_stride, tier_tile_cap(p), idx, qb0,
-                      qb1, stage_k, stage_v, stage_slots, lag, scratch, idx_remapped, n_fetched, status, stream);
+                      qb1, stage_k, stage_v, stage_slots, lag, scratch, idx_remapped, n_fetched, status, stream, dev);
 }
 
 hga_status_t launch_fetch_group_summaries(const hga_params_t &p, const float *host_gsumm, int group,
@@ -319,7 +352,7 @@ hga_status_t launch_fetch_group_summaries(const hga_params_t &p, const float *ho
     const long long rows = p.hist_head_stride / group;
     return fetch_wave(p, host_gsumm, nullptr, gpc, p.head_dim * 4, rows, tier_tile_cap(p), idx, 0,
                       p.seg_len / p.q_block, stage, nullptr, stage_slots, 2, scratch, idx_remapped, n_fetched,
-                      status, stream);
+                      status, stream, DevSource{nullptr, nullptr, 0, 0, 0});
 }
 
 }  // namespace hga

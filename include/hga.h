@@ -457,13 +457,20 @@ typedef struct {
  *   buffer that an attention still in flight reads: the fetch of wave h
  *   writes its blocks' rows once wave h - lag is done, so chained calls of n
  *   waves each rotate ceil(lag / n) idx_remapped buffers.
- *   n_fetched (device int32, may be NULL): one count per wave.  Other
- *   arguments as hga_fetch_tiered and hga_attn_fwd.  HGA_ERR_INVALID_ARG for
- *   a null event, a lag outside 2 .. HGA_TIER_MAX_LAG or unknown flags. */
+ *   prev_k_seg / prev_v_seg (may be NULL): the K/V of the segment that
+ *   detached last, tokens [T - S, T) (T = Nc * chunk), laid out like k_seg /
+ *   v_seg and still in device memory until the call's fetches are done; its
+ *   chunks are then copied from there instead of across the host link (the
+ *   host history holds the same bytes, so the output does not change).
+ *   n_fetched (device int32, may be NULL): one count per wave, of the tiles
+ *   copied from the host.  Other arguments as hga_fetch_tiered and
+ *   hga_attn_fwd.  HGA_ERR_INVALID_ARG for a null event, a lag outside 2 ..
+ *   HGA_TIER_MAX_LAG, unknown flags, or prev_k_seg with Nc < S / chunk. */
 #define HGA_TIER_RESET 1
 #define HGA_TIER_CHAIN 2
 hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const void *host_k, const void *host_v,
-                                 const void *k_seg, const void *v_seg, const int32_t *idx, void *out, float *lse,
+                                 const void *k_seg, const void *v_seg, const void *prev_k_seg,
+                                 const void *prev_v_seg, const int32_t *idx, void *out, float *lse,
                                  void *stage_k, void *stage_v, int stage_slots, int32_t *scratch,
                                  int32_t *idx_remapped, int wave_blocks, int flags, int32_t *n_fetched,
                                  cudaStream_t stream, cudaStream_t copy_stream, hga_tier_sched_t *sched);
@@ -478,7 +485,9 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
  *                   [Nc, Nc + S / chunk) of summ.
  *   copy_stream   : the fetch waves of hga_attn_fwd_tiered, chained from the
  *                   previous segment, after the segment's route and the
- *                   previous segment's offload.
+ *                   previous segment's offload -- or, given prev_k_seg /
+ *                   prev_v_seg (the previous segment's K/V, which its chunks
+ *                   are then copied from), the offload of the one before.
  *   offload_stream: k_seg / v_seg copied to tokens [T, T + S) of host_k /
  *                   host_v (T = Nc * chunk) once the inputs are ready.
  *   stream        : the attention waves, writing out and lse.
@@ -497,7 +506,8 @@ hga_status_t hga_attn_fwd_tiered(const hga_params_t *p, const void *q, const voi
  * history is not page-locked, or an event of sched is null; other arguments
  * and checks as hga_route, hga_attn_fwd_tiered and hga_tier_offload. */
 hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const void *k_seg, const void *v_seg,
-                                    float *summ, int summ_cap_chunks, int32_t *idx, void *host_k, void *host_v,
+                                    const void *prev_k_seg, const void *prev_v_seg, float *summ,
+                                    int summ_cap_chunks, int32_t *idx, void *host_k, void *host_v,
                                     void *out, float *lse, void *stage_k, void *stage_v, int stage_slots,
                                     int32_t *scratch, int32_t *idx_remapped, int wave_blocks, int flags,
                                     int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,

@@ -154,7 +154,9 @@ def test_tiered_staging_capacity_checked_on_host(L):
     sc.start = sc.fetched = 0x10
     sc.consumed[0] = sc.consumed[1] = sc.consumed[2] = 0x10
     sc.lag = 2
-    args = [ctypes.byref(p), fake, fake, fake, fake, fake, fake, fake, fake, fake, fake, 64, fake, fake]
+    # p, q, host_k, host_v, k_seg, v_seg, prev_k_seg, prev_v_seg, idx, out, lse, stage_k, stage_v, slots,
+    # scratch, idx_remapped
+    args = [ctypes.byref(p), fake, fake, fake, fake, fake, None, None, fake, fake, fake, fake, fake, 64, fake, fake]
     assert L.hga_attn_fwd_tiered(*args, 0, 1, None, None, None, ctypes.byref(sc)) == -1
     assert L.hga_attn_fwd_tiered(*args, 1, 1, None, None, None, None) == -1
     assert L.hga_attn_fwd_tiered(*args, 2, 4, None, None, None, ctypes.byref(sc)) == -1  # unknown flag
@@ -167,12 +169,20 @@ def test_tiered_staging_capacity_checked_on_host(L):
     sc.fetched = 0
     assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
     sc.fetched = 0x10
-    args[11] = 31  # two waves of 2 blocks need 32 slots
+    args[13] = 31  # two waves of 2 blocks need 32 slots
     assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
     sc.lag = 3
-    args[11] = 47  # lag 3: 48 slots (fewer than the 64 routable tiles)
+    args[13] = 47  # lag 3: 48 slots (fewer than the 64 routable tiles)
     assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
     assert b"stage_slots" in L.hga_last_error()
+    # the previous segment's K/V come as a pair, and only with a segment's worth of history
+    sc.lag = 2
+    args[13] = 64
+    args[6] = fake
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
+    short = _params(n_hist_chunks=1, hist_head_stride=4096).c()  # Nc = 1 < S / chunk = 2
+    args[0], args[7] = ctypes.byref(short), fake
+    assert L.hga_attn_fwd_tiered(*args, 2, 1, None, None, None, ctypes.byref(sc)) == -1
 
 
 def test_segment_tiered_checked_on_host(L):
@@ -189,7 +199,8 @@ def test_segment_tiered_checked_on_host(L):
     seg_chunks = p.seg_len // 64
 
     def call(pp, cap, flags=0, sched=sc):
-        return L.hga_segment_fwd_tiered(ctypes.byref(pp.c()), fake, fake, fake, fake, cap, fake, fake, fake, fake,
+        return L.hga_segment_fwd_tiered(ctypes.byref(pp.c()), fake, fake, fake, None, None, fake, cap, fake, fake,
+                                        fake, fake,
                                         fake, fake, fake, 64, fake, fake, 2, flags, None, None, None, None, None,
                                         ctypes.byref(sched) if sched is not None else None)
 

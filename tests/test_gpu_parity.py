@@ -483,10 +483,13 @@ CHAIN = gen.custom("chain_bf16", n_q_heads=8, n_kv_heads=2, head_dim=128, topk=4
                    seg_starts=tuple(range(0, 6 * 256, 256)), dtype="bf16", seed=23)
 
 
-@pytest.mark.parametrize("wave,lag,slots", [(4, 2, 40), (1, 4, 32), (1, 3, 24), (2, 2, 32), (1, 2, 16)],
+@pytest.mark.parametrize("wave,lag,slots,prev", [(4, 2, 40, False), (1, 4, 32, False), (1, 3, 24, False),
+                                                 (2, 2, 32, False), (1, 2, 16, False), (4, 2, 40, True),
+                                                 (1, 2, 16, True), (2, 3, 48, True)],
                          ids=["segment_waves_lag2", "block_waves_lag4", "block_waves_lag3", "two_block_waves_lag2",
-                              "block_waves_lag2"])
-def test_tiered_chained_segments_match_resident(wave, lag, slots):
+                              "block_waves_lag2", "segment_waves_lag2_prev", "block_waves_lag2_prev",
+                              "two_block_waves_lag3_prev"])
+def test_tiered_chained_segments_match_resident(wave, lag, slots, prev):
     """An evaluation of six segments with the history only in pinned host memory,
     through hga_segment_fwd_tiered as the benchmark runs it: each segment's K/V
     offloaded to the host history on one stream, its route and summary append on a
@@ -497,8 +500,11 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots):
     fetch that overtook an offload, or an eviction of a slot still being read, changes
     the output.  Every segment's out and lse equal the resident forward on the same
     routes bit for bit.  Slots: the least the schedule accepts, min(lag x wave x B x
-    Hkv x k, B x Hkv x Nc); all but the segment-wave case hold fewer than the last
-    segment's 40 routable tiles, so the cache evicts."""
+    Hkv x k, B x Hkv x Nc); all but the segment-wave cases hold fewer than the last
+    segment's 40 routable tiles, so the cache evicts.  With prev, each segment's
+    fetches copy the previous segment's chunks from its K/V in device memory (and
+    wait only for the offload of the segment before that): the outputs are the same
+    and fewer tiles cross the host link."""
     import hierarchical_sparse_long_b200 as hga
     w = CHAIN
     L, S, D = w.seq_len, w.seg_len, w.head_dim
@@ -542,10 +548,12 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots):
         p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
         out = torch.full_like(qs[T], float("nan"))
         lse = torch.full(qs[T].shape[:3], float("nan"), device="cuda")
+        use_prev = prev and si > 0
         hga.hga_segment_fwd_tiered(p, qs[T], k_all[:, :, T:], v_all[:, :, T:], summ, nct, idx[si % 2], host_k,
                                    host_v, out, lse, stage_k, stage_v, slots, scratch, idx_r[si % len(idx_r)], wave,
                                    sched, reset=si == 0, n_fetched=nf[si], copy_stream=copy, route_stream=route_s,
-                                   offload_stream=off)
+                                   offload_stream=off, prev_k_seg=k_all[:, :, T - S:] if use_prev else None,
+                                   prev_v_seg=v_all[:, :, T - S:] if use_prev else None)
         got[T] = (out, lse)
     for st in (copy, route_s, off):
         compute.wait_stream(st)
@@ -562,11 +570,17 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots):
     fetched = int(nf.sum().item())
     union = {(b, g, int(j)) for T in w.seg_starts for b in range(w.batch) for g in range(w.n_kv_heads)
              for j in ref[T][2][b, g].flatten().tolist() if j >= 0}
-    print(f"wave {wave}, lag {lag}, {slots} slots: fetched {fetched} tiles over {len(w.seg_starts)} segments, "
-          f"{len(union)} distinct")
-    assert fetched >= len(union)
-    if len(union) > slots:
-        assert fetched > slots  # the cache evicted
+    print(f"wave {wave}, lag {lag}, {slots} slots, prev {prev}: fetched from the host {fetched} tiles over "
+          f"{len(w.seg_starts)} segments, {len(union)} distinct")
+    if not prev:
+        assert fetched >= len(union)
+        if len(union) > slots:
+            assert fetched > slots  # the cache evicted
+    elif slots >= 2 * (w.seq_len - S) // 64:
+        # a cache that never evicts: a segment's chunks are first routable by the next
+        # segment, whose fetches take them from device memory, so only the chunks first
+        # routed later than that cross the host link
+        assert fetched < len(union)
 
 
 def test_tiered_rejects_pageable_host_memory_before_any_launch():
