@@ -282,6 +282,13 @@ class Layer:
                                   device=dev)
         self.side = torch.cuda.Stream()
         self.side_append = False
+        # a multi-segment forward-only evaluation: each segment's route (and append) on a
+        # route stream, under the attention of the segment before it (hga_segment_fwd)
+        self.pipelined = not w.backward and not w.tiered and len(w.seg_starts) > 1
+        if self.pipelined:
+            self.route_stream = torch.cuda.Stream(priority=-1)
+            self.idx_ring = [self.idx, torch.empty_like(self.idx)]
+            self.sched = hga.TierSched(lag=2)
         if w.tiered:
             self._init_tiered()
         self.reset()
@@ -305,10 +312,14 @@ class Layer:
             setattr(p, k, v)
         return p
 
-    def segment(self, T, ev=None, q=None, do=None):
+    def segment(self, T, ev=None, q=None, do=None, si=0):
         """Route, attend [, backward], detach with history in device memory;
         returns the number of library kernels launched.  Uninstrumented (ev is
-        None), the route and the forward are one hga_route_attn_fwd call.
+        None), the route and the forward are one hga_route_attn_fwd call, or,
+        in a multi-segment forward-only evaluation, one hga_segment_fwd call
+        whose route runs on a route stream under the previous segment's
+        attention (its q, K and V are then resident or were copied in on the
+        route stream).
 
         With side_append the detach-time summary append (it reads only the
         segment's keys and writes summaries of chunks this segment's route
@@ -318,6 +329,10 @@ class Layer:
         p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
+        if ev is None and self.pipelined:
+            hga.hga_segment_fwd(p, q, self.k, self.v, ks, vs, self.summ, self.nct, self.idx_ring[si % 2], self.out,
+                                self.lse, self.sched, reset=si == 0, route_stream=self.route_stream)
+            return 3  # route, forward, append
         rec = ev.record if ev is not None else (lambda name: None)
         main = torch.cuda.current_stream()
         if self.side_append:
@@ -467,9 +482,11 @@ class Layer:
         # starting at T, so each step simply re-appends every segment's chunks
         n = 0
         for si, T in enumerate(self.w.seg_starts):
-            n += self.segment_tiered(T, ev, si=si) if self.w.tiered else self.segment(T, ev)
+            n += self.segment_tiered(T, ev, si=si) if self.w.tiered else self.segment(T, ev, si=si)
         if self.w.tiered:  # the last append and offload belong to the step
             self.end_tiered_step()
+        elif self.pipelined and ev is None:  # the last append belongs to the step
+            self.torch.cuda.current_stream().wait_stream(self.route_stream)
         return n
 
 
@@ -887,15 +904,18 @@ def measure_layer(w, args, world, local):
            "config": {**workload_config(w, world),
                       "l2": "flushed before every timed step (256 MiB write)",
                       "launch": "one CUDA graph replay per step" if graph is not None else "eager",
-                      "route_and_forward": "hga_route_attn_fwd (one call, the forward a programmatic "
-                                           "dependent of the route)" if not w.tiered else
-                                           "hga_segment_fwd_tiered (route and fetches on a copy stream, "
-                                           "chained across segments)",
+                      "route_and_forward": ("hga_segment_fwd_tiered (route on a route stream, fetches on a "
+                                            "copy stream, chained across segments)" if w.tiered else
+                                            "hga_segment_fwd (each segment's route on a route stream under "
+                                            "the previous segment's attention)" if layer.pipelined else
+                                            "hga_route_attn_fwd (one call, the forward a programmatic "
+                                            "dependent of the route)"),
                       "kernel_times": "from as many replays of the same step with CUDA events between its "
                                       "library calls (route and forward then issued apart), after the "
                                       "timed region",
-                      "append": "side stream, overlapped with the route" if layer.side_append else
-                                ("copy stream, overlapped with the attention" if w.tiered else "in order")},
+                      "append": ("route stream, overlapped with the attention" if w.tiered or layer.pipelined
+                                 else "side stream, overlapped with the route" if layer.side_append
+                                 else "in order")},
            "roofline": roof, "kernels": kernels, "clocks": clocks, "gpu_launches": launches,
            "device_status": status}
     if w.tiered:
@@ -982,7 +1002,9 @@ def e2e_measure(layer, steps):
     # segments before it: its inputs arrive on the route stream, q in a ring of five
     # buffers (the route stream reaches segment s only after the fetches of s - 3, which
     # come after the attention of s - 5)
-    q_ring = [torch.empty_like(layer.q[w.seg_starts[0]]) for _ in range(5 if w.tiered else 1)]
+    # (a pipelined evaluation's route stream runs a segment ahead: a ring of three)
+    q_ring = [torch.empty_like(layer.q[w.seg_starts[0]]) for _ in range(5 if w.tiered else
+                                                                        3 if layer.pipelined else 1)]
     do_d = torch.empty_like(layer.do[w.seg_starts[0]]) if w.backward else None
     h2d = sum(t.numel() * t.element_size() for ts in host_in.values() for t in ts)
     d2h = sum(t.numel() * t.element_size() for t in outs) * len(w.seg_starts)
@@ -994,9 +1016,10 @@ def e2e_measure(layer, steps):
         for si, T in enumerate(w.seg_starts):
             hi = host_in[T]
             q_d = q_ring[si % len(q_ring)]
-            if w.tiered and si == 0:
+            side_in = w.tiered or layer.pipelined
+            if side_in and si == 0:
                 layer.route_stream.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(layer.route_stream if w.tiered else torch.cuda.current_stream()):
+            with torch.cuda.stream(layer.route_stream if side_in else torch.cuda.current_stream()):
                 q_d.copy_(hi[0], non_blocking=True)
                 layer.k[:, :, T:T + S].copy_(hi[1], non_blocking=True)
                 layer.v[:, :, T:T + S].copy_(hi[2], non_blocking=True)
@@ -1005,11 +1028,13 @@ def e2e_measure(layer, steps):
             if w.tiered:
                 layer.segment_tiered(T, q=q_d, si=si)
             else:
-                layer.segment(T, q=q_d, do=do_d)
+                layer.segment(T, q=q_d, do=do_d, si=si)
             for hbuf, t in zip(host_out, outs):
                 hbuf.copy_(t, non_blocking=True)
         if w.tiered:
             layer.end_tiered_step()
+        elif layer.pipelined:
+            torch.cuda.current_stream().wait_stream(layer.route_stream)
         e.record()
         e.synchronize()
         if it >= 1:

@@ -14,6 +14,6 @@ from .binding import (  # noqa: F401
     hga_attn_fwd_groups, hga_attn_bwd_groups, hga_attn_causal_workspace_size, hga_attn_fwd_causal,
     hga_attn_bwd_causal,
     hga_tier_scratch_size, hga_tier_reset, hga_fetch_tiered, hga_tier_offload, hga_attn_fwd_tiered,
-    hga_segment_fwd_tiered,
+    hga_segment_fwd_tiered, hga_segment_fwd,
     hga_get_device_status, hga_selftest_wait_timeout,
 )

@@ -29,6 +29,7 @@ EXPORTED = ("hga_build_summaries", "hga_route", "hga_route_causal", "hga_route_g
             "hga_attn_causal_workspace_size", "hga_attn_fwd_causal", "hga_attn_bwd_causal",
             "hga_attn_bwd_noalloc", "hga_attn_decode_workspace_size", "hga_attn_decode", "hga_tier_scratch_size",
             "hga_tier_reset", "hga_fetch_tiered", "hga_tier_offload", "hga_attn_fwd_tiered", "hga_segment_fwd_tiered",
+            "hga_segment_fwd",
             "hga_get_device_status", "hga_selftest_wait_timeout", "hga_status_string", "hga_last_error")
 
 
@@ -114,6 +115,8 @@ def lib() -> ctypes.CDLL:
         L.hga_tier_offload.argtypes = [pp, vp, vp, vp, vp, ll, vp]
         L.hga_attn_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i, i, vp, vp,
                                           vp, ctypes.POINTER(_TierSchedC)]
+        L.hga_segment_fwd.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, i, vp, vp,
+                                      ctypes.POINTER(_TierSchedC)]
         L.hga_segment_fwd_tiered.argtypes = [pp, vp, vp, vp, vp, vp, vp, i, vp, vp, vp, vp, vp, vp, vp, i, vp, vp, i,
                                              i, vp, vp, vp, vp, vp, ctypes.POINTER(_TierSchedC)]
         L.hga_get_device_status.argtypes = [vp, ctypes.POINTER(ctypes.c_uint)]
@@ -398,6 +401,18 @@ def hga_attn_fwd_tiered(p: Params, q, host_k, host_v, k_seg, v_seg, idx, out, ls
                                      stage_slots, _ptr(scratch), _ptr(idx_remapped), wave_blocks, flags,
                                      _ptr(n_fetched), _stream(stream), _stream(copy_stream), ctypes.byref(sched.c)),
            "hga_attn_fwd_tiered")
+
+
+def hga_segment_fwd(p: Params, q, k_hist, v_hist, k_seg, v_seg, summ, summ_cap_chunks: int, idx, out, lse,
+                    sched: TierSched, reset=False, stream=None, route_stream=None):
+    """One segment of an evaluation over resident history: route and summary append on
+    route_stream, attention on stream (a segment's route runs under the previous
+    segment's attention)."""
+    cp = p.c()
+    _check(lib().hga_segment_fwd(ctypes.byref(cp), _ptr(q), _ptr(k_hist), _ptr(v_hist), _ptr(k_seg), _ptr(v_seg),
+                                 _ptr(summ), summ_cap_chunks, _ptr(idx), _ptr(out), _ptr(lse),
+                                 HGA_TIER_RESET if reset else 0, _stream(stream), _stream(route_stream),
+                                 ctypes.byref(sched.c)), "hga_segment_fwd")
 
 
 def hga_segment_fwd_tiered(p: Params, q, k_seg, v_seg, summ, summ_cap_chunks: int, idx, host_k, host_v, out, lse,

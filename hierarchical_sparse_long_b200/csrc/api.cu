@@ -695,6 +695,48 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
     return HGA_OK;
 }
 
+hga_status_t hga_segment_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                             const void *k_seg, const void *v_seg, float *summ, int summ_cap_chunks, int32_t *idx,
+                             void *out, float *lse, int flags, cudaStream_t stream, cudaStream_t route_stream,
+                             hga_tier_sched_t *sched) {
+    CallRange range("hga_segment_fwd");
+    if (!p || !sched || (flags & ~HGA_TIER_RESET)) return HGA_ERR_INVALID_ARG;
+    hga_status_t st = check_params(p);
+    if (st != HGA_OK) return st;
+    if (!sched->start || !sched->routed || !sched->idx_free[0] || !sched->idx_free[1] || sched->segment < 0)
+        return HGA_ERR_INVALID_ARG;
+    if (p->seg_len % p->chunk != 0) return HGA_ERR_INVALID_ARG;
+    const int seg_chunks = p->seg_len / p->chunk;
+    if ((long long)p->n_hist_chunks + seg_chunks > summ_cap_chunks) return HGA_ERR_INVALID_ARG;
+    if (!summ || !aligned16(summ) || !k_seg || !aligned16(k_seg)) return HGA_ERR_INVALID_ARG;
+    cudaError_t e = cudaSuccess;
+    if (flags & HGA_TIER_RESET) {  // the evaluation starts: the route stream after whatever came before it
+        if ((e = cudaEventRecord(sched->start, stream)) != cudaSuccess ||
+            (e = cudaStreamWaitEvent(route_stream, sched->start, 0)) != cudaSuccess)
+            return hga::record_cuda(e);
+        sched->segment = 0;
+    }
+    const long long seg = sched->segment;
+    // the route; its idx buffer was last read by the attention of segment seg - 2
+    if (seg >= 2 && (e = cudaStreamWaitEvent(route_stream, sched->idx_free[seg & 1], 0)) != cudaSuccess)
+        return hga::record_cuda(e);
+    st = hga_route(p, q, summ, summ_cap_chunks, idx, route_stream);
+    if (st != HGA_OK) return st;
+    if ((e = cudaEventRecord(sched->routed, route_stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(stream, sched->routed, 0)) != cudaSuccess)
+        return hga::record_cuda(e);
+    st = hga_attn_fwd(p, q, k_hist, v_hist, k_seg, v_seg, idx, out, lse, stream);
+    if (st != HGA_OK) return st;
+    if ((e = cudaEventRecord(sched->idx_free[seg & 1], stream)) != cudaSuccess) return hga::record_cuda(e);
+    // detach: the segment's chunks become routable for the next segment
+    st = hga::launch_summaries(k_seg, p->seg_head_stride, p->batch * p->n_kv_heads, p->head_dim, p->chunk,
+                               p->n_hist_chunks, seg_chunks, p->dtype, summ, summ_cap_chunks, route_stream,
+                               p->n_hist_chunks);
+    if (st != HGA_OK) return st;
+    sched->segment = seg + 1;
+    return HGA_OK;
+}
+
 hga_status_t hga_selftest_wait_timeout(long long wait_cycles, cudaStream_t stream) {
     CallRange range("hga_selftest_wait_timeout");
     if (wait_cycles < 1000 || wait_cycles > (1ll << 32)) return HGA_ERR_INVALID_ARG;

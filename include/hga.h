@@ -513,6 +513,31 @@ hga_status_t hga_segment_fwd_tiered(const hga_params_t *p, const void *q, const 
                                     int32_t *n_fetched, cudaStream_t stream, cudaStream_t copy_stream,
                                     cudaStream_t route_stream, cudaStream_t offload_stream, hga_tier_sched_t *sched);
 
+/* One segment of an evaluation with the history resident in device memory
+ * (technical summary section 2.1: route, then exact-token attention; the
+ * segment detaches at its end), on two streams, so that a segment's route runs
+ * under the attention of the segment before it:
+ *   route_stream: hga_route of the segment into idx, then the detach-time
+ *                 append of the segment's S / chunk summaries to chunks
+ *                 [Nc, Nc + S / chunk) of summ (read from k_seg).
+ *   stream      : hga_attn_fwd of the segment, once its route is done.
+ * The inputs (q, k_seg, v_seg and the history) must be ready in route_stream's
+ * order (the caller copies them in there, or orders route_stream after their
+ * producer).  idx: the segment's route table; the route of segment s + 2 waits
+ * until the attention of segment s has read its buffer, so rotate two buffers.
+ * flags: HGA_TIER_RESET for the evaluation's first segment (route_stream first
+ * waits for stream; sched->segment restarts); 0 continues the evaluation.
+ * sched: a schedule object as for hga_segment_fwd_tiered, of which this call
+ * uses start, routed, idx_free and segment.  On return stream is ordered after
+ * the segment's route; the caller orders stream after route_stream before it
+ * reads summ itself.  Other arguments and checks as hga_route and hga_attn_fwd;
+ * HGA_ERR_INVALID_ARG when summ_cap_chunks < Nc + S / chunk or an event is
+ * null. */
+hga_status_t hga_segment_fwd(const hga_params_t *p, const void *q, const void *k_hist, const void *v_hist,
+                             const void *k_seg, const void *v_seg, float *summ, int summ_cap_chunks, int32_t *idx,
+                             void *out, float *lse, int flags, cudaStream_t stream, cudaStream_t route_stream,
+                             hga_tier_sched_t *sched);
+
 /* Self-test of the bounded waits (the source pages have no counterpart): every
  * pipeline wait in the tensor-core kernels gives up after a cycle limit instead
  * of hanging, sets HGA_DEV_TIMEOUT and lets the kernel end.  This launches one

@@ -218,6 +218,26 @@ def test_segment_tiered_checked_on_host(L):
     assert call(p, 4096) == -1
 
 
+def test_segment_fwd_checked_on_host(L):
+    p = _params(n_hist_chunks=32, hist_head_stride=4096)
+    fake = ctypes.c_void_p(0x1000)
+    sc = hga.binding._TierSchedC()
+    sc.start = sc.routed = sc.idx_free[0] = sc.idx_free[1] = 0x10
+    sc.lag = 2
+
+    def call(pp, cap, flags=0, sched=sc):
+        return L.hga_segment_fwd(ctypes.byref(pp.c()), fake, fake, fake, fake, fake, fake, cap, fake, fake, fake,
+                                 flags, None, None, ctypes.byref(sched) if sched is not None else None)
+
+    assert call(p, 32 + p.seg_len // 64 - 1) == -1  # no room to append the segment's summaries
+    assert call(p, 4096, flags=2) == -1
+    assert call(p, 4096, sched=None) == -1
+    sc.routed = 0
+    assert call(p, 4096) == -1
+    sc.routed = 0x10
+    assert call(_params(topk=0), 4096) == -1
+
+
 def test_tiered_scratch_size(L):
     # two int32 entries per (b, g, chunk) of the host history, four per slot, four control words
     p = _params(n_hist_chunks=32, hist_head_stride=4096)

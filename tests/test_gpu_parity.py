@@ -583,6 +583,57 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots, prev):
         assert fetched < len(union)
 
 
+def test_segment_fwd_pipelined_matches_resident():
+    """The same six-segment evaluation with the history resident, through
+    hga_segment_fwd on two streams (each segment's route and summary append on a
+    high-priority route stream, running under the previous segment's attention, two
+    rotating route tables, no host synchronisation): every segment's out and lse equal
+    hga_route + hga_attn_fwd on the full summaries bit for bit, and the appended
+    summaries equal a rebuild."""
+    import hierarchical_sparse_long_b200 as hga
+    w = CHAIN
+    L, S, D = w.seq_len, w.seg_len, w.head_dim
+    nqb = S // 64
+    k_all = hc.to_dev(gen.keys(w, 0, L), w)
+    v_all = hc.to_dev(gen.values(w, 0, L), w)
+    qs = {T: hc.to_dev(gen.queries(w, T, T + S), w) for T in w.seg_starts}
+    nct = L // 64
+    full = torch.zeros(w.batch, w.n_kv_heads, nct, D, device="cuda")
+    hga.hga_build_summaries(k_all, L, w.batch, w.n_kv_heads, D, 64, 0, nct, full, nct)
+    ref = {}
+    for T in w.seg_starts:
+        p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
+        idx = torch.empty(w.batch, w.n_kv_heads, nqb, w.topk, device="cuda", dtype=torch.int32)
+        hga.hga_route(p, qs[T], full, nct, idx)
+        out = torch.empty_like(qs[T])
+        lse = torch.empty(qs[T].shape[:3], device="cuda")
+        hga.hga_attn_fwd(p, qs[T], k_all, v_all, k_all[:, :, T:], v_all[:, :, T:], idx, out, lse)
+        ref[T] = (out, lse)
+    torch.cuda.synchronize()
+    summ = torch.zeros_like(full)
+    idx = [torch.full((w.batch, w.n_kv_heads, nqb, w.topk), 7, device="cuda", dtype=torch.int32) for _ in range(2)]
+    sched = hga.TierSched(lag=2)
+    compute, route_s = torch.cuda.current_stream(), torch.cuda.Stream(priority=-1)
+    got = {}
+    for rep in range(2):  # a second evaluation restarts the schedule over the same buffers
+        summ.zero_()
+        for si, T in enumerate(w.seg_starts):
+            p = hc.params(w, T, hist_head_stride=L, seg_head_stride=L)
+            out = torch.full_like(qs[T], float("nan"))
+            lse = torch.full(qs[T].shape[:3], float("nan"), device="cuda")
+            hga.hga_segment_fwd(p, qs[T], k_all, v_all, k_all[:, :, T:], v_all[:, :, T:], summ, nct, idx[si % 2],
+                                out, lse, sched, reset=si == 0, route_stream=route_s)
+            got[(rep, T)] = (out, lse)
+        compute.wait_stream(route_s)
+    torch.cuda.synchronize()
+    assert hga.hga_get_device_status() == 0
+    for (rep, T), (out, lse) in got.items():
+        assert torch.equal(out, ref[T][0]), f"evaluation {rep}, segment at {T}: out"
+        assert torch.equal(lse, ref[T][1]), f"evaluation {rep}, segment at {T}: lse"
+    assert torch.equal(summ, full)
+    assert sched.segment == len(w.seg_starts)
+
+
 def test_tiered_rejects_pageable_host_memory_before_any_launch():
     import hierarchical_sparse_long_b200 as hga
     w = MID
