@@ -312,7 +312,7 @@ class Layer:
             setattr(p, k, v)
         return p
 
-    def segment(self, T, ev=None, q=None, do=None, si=0):
+    def segment(self, T, ev=None, q=None, do=None, si=0, outs=None):
         """Route, attend [, backward], detach with history in device memory;
         returns the number of library kernels launched.  Uninstrumented (ev is
         None), the route and the forward are one hga_route_attn_fwd call, or,
@@ -329,9 +329,12 @@ class Layer:
         p = self.params(T)
         q = self.q[T] if q is None else q
         ks, vs = self.k[:, :, T:], self.v[:, :, T:]
+        # the segment's outputs: O, LSE [, dQ, dK, dV]
+        o_out, o_lse, o_dq, o_dk, o_dv = outs if outs is not None else (
+            self.out, self.lse, getattr(self, "dq", None), getattr(self, "dk", None), getattr(self, "dv", None))
         if ev is None and self.pipelined:
-            hga.hga_segment_fwd(p, q, self.k, self.v, ks, vs, self.summ, self.nct, self.idx_ring[si % 2], self.out,
-                                self.lse, self.sched, reset=si == 0, route_stream=self.route_stream)
+            hga.hga_segment_fwd(p, q, self.k, self.v, ks, vs, self.summ, self.nct, self.idx_ring[si % 2], o_out,
+                                o_lse, self.sched, reset=si == 0, route_stream=self.route_stream)
             return 3  # route, forward, append
         rec = ev.record if ev is not None else (lambda name: None)
         main = torch.cuda.current_stream()
@@ -345,17 +348,17 @@ class Layer:
                 if ev is not None:
                     ev.record(None)
         if ev is None:
-            hga.hga_route_attn_fwd(p, q, self.summ, self.nct, self.idx, self.k, self.v, ks, vs, self.out, self.lse)
+            hga.hga_route_attn_fwd(p, q, self.summ, self.nct, self.idx, self.k, self.v, ks, vs, o_out, o_lse)
         else:
             rec("route")
             hga.hga_route(p, q, self.summ, self.nct, self.idx)
             rec("attn_fwd")
-            hga.hga_attn_fwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse)
+            hga.hga_attn_fwd(p, q, self.k, self.v, ks, vs, self.idx, o_out, o_lse)
         launches = 2
         if w.backward:
             rec("attn_bwd")
-            hga.hga_attn_bwd(p, q, self.k, self.v, ks, vs, self.idx, self.out, self.lse,
-                             self.do[T] if do is None else do, self.dq, self.dk, self.dv, self.ws)
+            hga.hga_attn_bwd(p, q, self.k, self.v, ks, vs, self.idx, o_out, o_lse,
+                             self.do[T] if do is None else do, o_dq, o_dk, o_dv, self.ws)
             launches += 2
         if self.side_append:
             rec(None)
@@ -395,7 +398,7 @@ class Layer:
         self.offload_stream = torch.cuda.Stream(priority=-1)
         self.sched = hga.TierSched(lag=self.lag)
 
-    def segment_tiered(self, T, ev=None, q=None, si=0):
+    def segment_tiered(self, T, ev=None, q=None, si=0, outs=None):
         """The same segment with the history only in pinned host memory, one
         hga_segment_fwd_tiered call on four streams: the route and the summary
         append on a route stream, the fetch of the routed tiles on a copy stream
@@ -417,7 +420,8 @@ class Layer:
             ev.record("attn_fwd")
         first = si == 0
         hga.hga_segment_fwd_tiered(p, q, ks, vs, self.summ, self.nct, self.idx_ring[si % 2], self.host_k,
-                                   self.host_v, self.out, self.lse, self.stage_k, self.stage_v, self.slots,
+                                   self.host_v, self.out if outs is None else outs[0],
+                                   self.lse if outs is None else outs[1], self.stage_k, self.stage_v, self.slots,
                                    self.scratch, self.idx_r[si % len(self.idx_r)], self.wave, self.sched,
                                    reset=first, n_fetched=self.n_fetched[si], copy_stream=self.copy_stream,
                                    route_stream=self.route_stream, offload_stream=self.offload_stream,
@@ -931,7 +935,9 @@ def measure_layer(w, args, world, local):
                                      "traffic": t["bytes_fetched_per_step"] + t["bytes_offloaded_per_step"],
                                      "peak_source": "pinned cudaMemcpyAsync host -> device and device -> host "
                                                     "at once on two streams, measured in this run"}
-    res["e2e"] = e2e_measure(layer, max(2, min(args.steps, 5)))
+    single = len(w.seg_starts) == 1 and not w.backward and not w.tiered
+    res["e2e"] = e2e_stream_measure(layer, max(10, args.steps)) if single else \
+        e2e_measure(layer, max(2, min(args.steps, 5)))
     del layer, graph
     torch.cuda.synchronize()
     torch.cuda.empty_cache()
@@ -984,10 +990,90 @@ def tiered_report(layer, step_ms, attn_phase_ms, flush):
             "host_link_gbs_measured": {k: round(v, 2) for k, v in link.items()}}
 
 
+def e2e_stream_measure(layer, steps):
+    """A single-segment forward step through the C ABI from pinned host buffers,
+    streamed: each step's q and segment K/V are copied host -> device on an input
+    stream, its route + forward + append run on the compute stream, and its O and
+    LSE are copied back on an output stream, over two device slots, so the copies
+    of one step overlap the compute of its neighbours (every step still moves all
+    of its own bytes, inside the timed region)."""
+    import torch
+    hga, w = layer.hga, layer.w
+    S, T = w.seg_len, w.seg_starts[0]
+    p = layer.params(T)
+    host_in = [layer.q[T].cpu().pin_memory(), layer.k[:, :, T:T + S].cpu().pin_memory(),
+               layer.v[:, :, T:T + S].cpu().pin_memory()]
+
+    class Slot:
+        pass
+
+    slots = []
+    for n in range(2):
+        sl = Slot()
+        sl.q = torch.empty_like(layer.q[T])
+        sl.k = layer.k if n == 0 else layer.k.clone()
+        sl.v = layer.v if n == 0 else layer.v.clone()
+        sl.summ = layer.summ if n == 0 else layer.summ.clone()
+        sl.idx = torch.empty_like(layer.idx)
+        sl.out = torch.empty_like(layer.out)
+        sl.lse = torch.empty_like(layer.lse)
+        sl.host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (sl.out, sl.lse)]
+        sl.in_ready, sl.computed, sl.out_read = (torch.cuda.Event() for _ in range(3))
+        slots.append(sl)
+    h2d = sum(t.numel() * t.element_size() for t in host_in)
+    d2h = sum(t.numel() * t.element_size() for t in (layer.out, layer.lse))
+    main = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    torch.cuda.synchronize()
+
+    def run(n_steps):
+        for i in range(n_steps):
+            sl = slots[i % 2]
+            if i >= 2:
+                s_in.wait_event(sl.computed)  # step i - 2 has read this slot's inputs
+            with torch.cuda.stream(s_in):
+                sl.q.copy_(host_in[0], non_blocking=True)
+                sl.k[:, :, T:T + S].copy_(host_in[1], non_blocking=True)
+                sl.v[:, :, T:T + S].copy_(host_in[2], non_blocking=True)
+            sl.in_ready.record(s_in)
+            main.wait_event(sl.in_ready)
+            if i >= 2:
+                main.wait_event(sl.out_read)  # step i - 2's outputs have left this slot
+            ks, vs = sl.k[:, :, T:], sl.v[:, :, T:]
+            hga.hga_route_attn_fwd(p, sl.q, sl.summ, layer.nct, sl.idx, sl.k, sl.v, ks, vs, sl.out, sl.lse)
+            hga.hga_build_summaries(sl.k, layer.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
+                                    S // w.chunk, sl.summ, layer.nct)
+            sl.computed.record(main)
+            s_out.wait_event(sl.computed)
+            with torch.cuda.stream(s_out):
+                for hbuf, t in zip(sl.host_out, (sl.out, sl.lse)):
+                    hbuf.copy_(t, non_blocking=True)
+            sl.out_read.record(s_out)
+        main.wait_stream(s_out)
+
+    run(4)  # warm-up
+    torch.cuda.synchronize()
+    st, en = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.record(main)
+    s_in.wait_stream(main)
+    s_out.wait_stream(main)
+    run(steps)
+    en.record(main)
+    en.synchronize()
+    ms = st.elapsed_time(en) / steps
+    return {"value": tokens_per_step(w) / (ms / 1000.0), "unit": UNIT,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
+            "scope": f"{steps} steps through the C ABI from pinned host buffers, streamed over two device slots: "
+                     "a step's inputs in and outputs out on their own streams, overlapping the compute of the "
+                     "steps next to it"}
+
+
 def e2e_measure(layer, steps):
     """The whole step through the C ABI from pinned host buffers: every segment's
     inputs (q, segment K/V [, dO]) copied host -> device before its compute and
-    its outputs (O, LSE [, dQ, dK, dV]) copied back, all inside the timed region."""
+    its outputs (O, LSE [, dQ, dK, dV]) copied back, all inside the timed region.
+    The outputs leave on their own stream from two alternating output sets, so a
+    segment's copy-out overlaps the compute of the next."""
     import torch
     w = layer.w
     S = w.seg_len
@@ -996,8 +1082,12 @@ def e2e_measure(layer, steps):
         host_in[T] = [layer.q[T].cpu().pin_memory(), layer.k[:, :, T:T + S].cpu().pin_memory(),
                       layer.v[:, :, T:T + S].cpu().pin_memory()] + \
                      ([layer.do[T].cpu().pin_memory()] if w.backward else [])
-    outs = [layer.out, layer.lse] + ([layer.dq, layer.dk, layer.dv] if w.backward else [])
-    host_out = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+    outs0 = [layer.out, layer.lse] + ([layer.dq, layer.dk, layer.dv] if w.backward else [])
+    out_sets = [outs0, [torch.empty_like(t) for t in outs0]]
+    host_out = [[torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs0] for _ in range(2)]
+    computed = [torch.cuda.Event() for _ in range(2)]
+    out_read = [torch.cuda.Event() for _ in range(2)]
+    s_out = torch.cuda.Stream()
     # the tiered step runs each segment's route and fetches under the attention of the
     # segments before it: its inputs arrive on the route stream, q in a ring of five
     # buffers (the route stream reaches segment s only after the fetches of s - 3, which
@@ -1007,34 +1097,45 @@ def e2e_measure(layer, steps):
                                                                         3 if layer.pipelined else 1)]
     do_d = torch.empty_like(layer.do[w.seg_starts[0]]) if w.backward else None
     h2d = sum(t.numel() * t.element_size() for ts in host_in.values() for t in ts)
-    d2h = sum(t.numel() * t.element_size() for t in outs) * len(w.seg_starts)
+    d2h = sum(t.numel() * t.element_size() for t in outs0) * len(w.seg_starts)
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     times = []
     for it in range(steps + 1):
         torch.cuda.synchronize()
+        main = torch.cuda.current_stream()
         s.record()
+        s_out.wait_stream(main)
         for si, T in enumerate(w.seg_starts):
             hi = host_in[T]
             q_d = q_ring[si % len(q_ring)]
             side_in = w.tiered or layer.pipelined
             if side_in and si == 0:
-                layer.route_stream.wait_stream(torch.cuda.current_stream())
-            with torch.cuda.stream(layer.route_stream if side_in else torch.cuda.current_stream()):
+                layer.route_stream.wait_stream(main)
+            with torch.cuda.stream(layer.route_stream if side_in else main):
                 q_d.copy_(hi[0], non_blocking=True)
                 layer.k[:, :, T:T + S].copy_(hi[1], non_blocking=True)
                 layer.v[:, :, T:T + S].copy_(hi[2], non_blocking=True)
                 if do_d is not None:
                     do_d.copy_(hi[3], non_blocking=True)
+            o = si % 2
+            if si >= 2:
+                main.wait_event(out_read[o])  # the output set's previous segment has left
             if w.tiered:
-                layer.segment_tiered(T, q=q_d, si=si)
+                layer.segment_tiered(T, q=q_d, si=si, outs=out_sets[o])
             else:
-                layer.segment(T, q=q_d, do=do_d, si=si)
-            for hbuf, t in zip(host_out, outs):
-                hbuf.copy_(t, non_blocking=True)
+                layer.segment(T, q=q_d, do=do_d, si=si,
+                              outs=out_sets[o] + [None] * (5 - len(out_sets[o])))
+            computed[o].record(main)
+            s_out.wait_event(computed[o])
+            with torch.cuda.stream(s_out):
+                for hbuf, t in zip(host_out[o], out_sets[o]):
+                    hbuf.copy_(t, non_blocking=True)
+            out_read[o].record(s_out)
         if w.tiered:
             layer.end_tiered_step()
         elif layer.pipelined:
-            torch.cuda.current_stream().wait_stream(layer.route_stream)
+            main.wait_stream(layer.route_stream)
+        main.wait_stream(s_out)
         e.record()
         e.synchronize()
         if it >= 1:
@@ -1042,7 +1143,8 @@ def e2e_measure(layer, steps):
     ms = statistics.mean(times)
     return {"value": tokens_per_step(w) / (ms / 1000.0), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "scope": "every segment of the step through the C ABI from pinned host buffers"}
+            "scope": "every segment of the step through the C ABI from pinned host buffers (outputs copied out "
+                     "on their own stream from two alternating output sets)"}
 
 
 def cpu_procs(args):
