@@ -490,6 +490,29 @@ CHAIN = gen.custom("chain_bf16", n_q_heads=8, n_kv_heads=2, head_dim=128, topk=4
                               "block_waves_lag2", "segment_waves_lag2_prev", "block_waves_lag2_prev",
                               "two_block_waves_lag3_prev"])
 def test_tiered_chained_segments_match_resident(wave, lag, slots, prev):
+    _chained_tiered(CHAIN, wave, lag, slots, prev)
+
+
+# other tile layouts of the staging copy: 128-byte rows (bf16, D = 64; two batches,
+# G = 1, the SIMT attention) and 512-byte rows (fp32, D = 128)
+CHAIN_LAYOUTS = [
+    gen.custom("chain_bf16_d64_b2", batch=2, n_q_heads=2, n_kv_heads=2, head_dim=64, topk=3, seg_len=128,
+               seq_len=6 * 128, seg_starts=tuple(range(0, 6 * 128, 128)), dtype="bf16", seed=24),
+    gen.custom("chain_fp32_d128", n_q_heads=4, n_kv_heads=2, head_dim=128, topk=3, seg_len=128, seq_len=6 * 128,
+               seg_starts=tuple(range(0, 6 * 128, 128)), dtype="fp32", seed=25),
+]
+
+
+@pytest.mark.parametrize("w", CHAIN_LAYOUTS, ids=[w.name for w in CHAIN_LAYOUTS])
+@pytest.mark.parametrize("prev", [False, True], ids=["host_only", "prev"])
+def test_tiered_chained_other_layouts(w, prev):
+    """The chained tiered evaluation with 128- and 512-byte rows, two batches and
+    G = 1: bitwise equal to the resident forward, with a cache that evicts."""
+    n_bg = w.batch * w.n_kv_heads
+    _chained_tiered(w, 1, 2, 2 * n_bg * w.topk, prev)
+
+
+def _chained_tiered(w, wave, lag, slots, prev):
     """An evaluation of six segments with the history only in pinned host memory,
     through hga_segment_fwd_tiered as the benchmark runs it: each segment's K/V
     offloaded to the host history on one stream, its route and summary append on a
@@ -500,13 +523,13 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots, prev):
     fetch that overtook an offload, or an eviction of a slot still being read, changes
     the output.  Every segment's out and lse equal the resident forward on the same
     routes bit for bit.  Slots: the least the schedule accepts, min(lag x wave x B x
-    Hkv x k, B x Hkv x Nc); all but the segment-wave cases hold fewer than the last
-    segment's 40 routable tiles, so the cache evicts.  With prev, each segment's
+    Hkv x k, B x Hkv x Nc); on the 256-token segments all but the segment-wave cases
+    hold fewer than the last segment's 40 routable tiles, so the cache evicts (the
+    other layouts' caches evict too).  With prev, each segment's
     fetches copy the previous segment's chunks from its K/V in device memory (and
     wait only for the offload of the segment before that): the outputs are the same
     and fewer tiles cross the host link."""
     import hierarchical_sparse_long_b200 as hga
-    w = CHAIN
     L, S, D = w.seq_len, w.seg_len, w.head_dim
     nqb = S // 64
     k_all = hc.to_dev(gen.keys(w, 0, L), w)
@@ -576,7 +599,7 @@ def test_tiered_chained_segments_match_resident(wave, lag, slots, prev):
         assert fetched >= len(union)
         if len(union) > slots:
             assert fetched > slots  # the cache evicted
-    elif slots >= 2 * (w.seq_len - S) // 64:
+    elif slots >= w.batch * w.n_kv_heads * ((w.seq_len - S) // 64):
         # a cache that never evicts: a segment's chunks are first routable by the next
         # segment, whose fetches take them from device memory, so only the chunks first
         # routed later than that cross the host link
