@@ -419,10 +419,10 @@ hga_status_t hga_tier_offload(const hga_params_t *p, const void *k_seg, const vo
  *   Create the events (cudaEventDisableTiming is enough; inputs, offloaded,
  *   routed and idx_free only for hga_segment_fwd_tiered), set lag (2 ..
  *   HGA_TIER_MAX_LAG), wave = 0 and segment = 0; the library records the
- *   events and advances the counters.  Use one compute stream and one copy stream for all calls of
- *   a schedule, and no other fetch into its cache (hga_fetch_tiered,
- *   hga_route_groups_tiered) between them.  A schedule's first call (wave 0)
- *   is never chained. */
+ *   events and advances the counters.  Use one compute stream and one copy
+ *   stream for all calls of a schedule, and no other fetch into its cache
+ *   (hga_fetch_tiered, hga_route_groups_tiered) between them.  A schedule's
+ *   first call (wave 0) is never chained. */
 #define HGA_TIER_MAX_LAG 4
 typedef struct {
     cudaEvent_t start;                       /* unchained calls: the copy stream after the compute stream */
