@@ -35,9 +35,9 @@ with the recipe of inputs/gen.py):
   window (history chunk 0 always routed, the other 15 slots by score).
 
 The default run prints one JSON line for the headline workload and measures
-``qwen3_16k_train``, ``qwen3_128k_eval`` and ``qwen3_128k_tiered`` too, each
-under ``workloads`` in the same line with its own roofline, kernels, e2e and
-CPU baseline (``--also none`` skips them).
+``qwen3_16k_train``, ``qwen3_128k_eval``, ``qwen3_128k_tiered`` and
+``qwen3_128k_decode`` too, each under ``workloads`` in the same line with its own
+roofline, kernels, e2e and CPU baseline (``--also none`` skips them).
 
 Metric: query tokens/s (active query tokens processed per second, all heads),
 device-timed with CUDA events around each step, L2 flushed (256 MiB write)
@@ -79,7 +79,7 @@ KERNEL_SOURCES = {
 }
 WORKLOADS = ("qwen3_16k_fwd", "qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_16k_fwd_sink",
              "qwen3_128k_decode", "qwen3_32k_decode")
-ALSO_DEFAULT = ("qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered")
+ALSO_DEFAULT = ("qwen3_16k_train", "qwen3_128k_eval", "qwen3_128k_tiered", "qwen3_128k_decode")
 
 
 def parse():
