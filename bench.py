@@ -990,11 +990,11 @@ def tiered_report(layer, step_ms, attn_phase_ms, flush):
             "host_link_gbs_measured": {k: round(v, 2) for k, v in link.items()}}
 
 
-def e2e_stream_measure(layer, steps):
+def e2e_stream_measure(layer, steps, n_slots=2):
     """A single-segment forward step through the C ABI from pinned host buffers,
     streamed: each step's q and segment K/V are copied host -> device on an input
     stream, its route + forward + append run on the compute stream, and its O and
-    LSE are copied back on an output stream, over two device slots, so the copies
+    LSE are copied back on an output stream, over n_slots device slots, so the copies
     of one step overlap the compute of its neighbours (every step still moves all
     of its own bytes, inside the timed region)."""
     import torch
@@ -1008,7 +1008,7 @@ def e2e_stream_measure(layer, steps):
         pass
 
     slots = []
-    for n in range(2):
+    for n in range(n_slots):
         sl = Slot()
         sl.q = torch.empty_like(layer.q[T])
         sl.k = layer.k if n == 0 else layer.k.clone()
@@ -1028,17 +1028,17 @@ def e2e_stream_measure(layer, steps):
 
     def run(n_steps):
         for i in range(n_steps):
-            sl = slots[i % 2]
-            if i >= 2:
-                s_in.wait_event(sl.computed)  # step i - 2 has read this slot's inputs
+            sl = slots[i % n_slots]
+            if i >= n_slots:
+                s_in.wait_event(sl.computed)  # the slot's previous step has read its inputs
             with torch.cuda.stream(s_in):
                 sl.q.copy_(host_in[0], non_blocking=True)
                 sl.k[:, :, T:T + S].copy_(host_in[1], non_blocking=True)
                 sl.v[:, :, T:T + S].copy_(host_in[2], non_blocking=True)
             sl.in_ready.record(s_in)
             main.wait_event(sl.in_ready)
-            if i >= 2:
-                main.wait_event(sl.out_read)  # step i - 2's outputs have left this slot
+            if i >= n_slots:
+                main.wait_event(sl.out_read)  # the slot's previous step's outputs have left it
             ks, vs = sl.k[:, :, T:], sl.v[:, :, T:]
             hga.hga_route_attn_fwd(p, sl.q, sl.summ, layer.nct, sl.idx, sl.k, sl.v, ks, vs, sl.out, sl.lse)
             hga.hga_build_summaries(sl.k, layer.L, w.batch, w.n_kv_heads, w.head_dim, w.chunk, T // w.chunk,
@@ -1063,7 +1063,8 @@ def e2e_stream_measure(layer, steps):
     ms = st.elapsed_time(en) / steps
     return {"value": tokens_per_step(w) / (ms / 1000.0), "unit": UNIT,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": ms,
-            "scope": f"{steps} steps through the C ABI from pinned host buffers, streamed over two device slots: "
+            "scope": f"{steps} steps through the C ABI from pinned host buffers, streamed over {n_slots} device "
+                     "slots: "
                      "a step's inputs in and outputs out on their own streams, overlapping the compute of the "
                      "steps next to it"}
 
