@@ -10,21 +10,24 @@
 //   dQ = dS K / sqrt(D)                      over routed history and segment keys
 //   dK_seg = dS^T Q / sqrt(D), dV_seg = P^T dO   over segment keys only
 //
-// Two block types in one launch, no atomics (results are deterministic):
-//   dQ blocks  : query-major, one CTA per (batch, kv head, query block, head
-//                sub-group) holding HC heads of the group (4, 2 or 1, as in the
-//                forward) as M=128 halves;
-//                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128), the
-//                dS rows in bf16 into shared memory, dQ += dS K (M128 N128 K64).
+// Two block types in one launch of 256-thread blocks, no atomics (results are
+// deterministic):
+//   dQ blocks  : query-major, one CTA per M=128 tile of query rows: HC heads of the
+//                group (4, 2 or 1, as in the forward) x 128 / HC rows of one query
+//                block (two CTAs per block when HC = 4);
+//                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128) into one
+//                of two TMEM buffers, the dS rows in bf16 into one of two shared-
+//                memory buffers, dQ += dS K (M128 N128 K64); warp 0 loads, warps 1,
+//                2 and 3 issue S, dP and dQ, warps 4-7 take one row each.
 //   dK/dV blocks: key-major over the active segment, one CTA per (batch, kv
 //                head, 128 segment keys); for every later 64-query tile of
 //                every head of the group: S^T = K Q^T and dP^T = V dO^T
 //                (M128 N64 K128), P^T and dS^T in bf16 into shared memory,
-//                dV += P^T dO and dK += dS^T Q (M128 N128 K64).
-// Warp 0 issues TMA loads, warps 1 and 3 issue the UMMAs (one thread each:
-// a single thread can issue a tcgen05.mma only every ~100 cycles), warp 1
-// owns TMEM, and the remaining warpgroups handle one TMEM lane (row) per
-// thread.
+//                dV += P^T dO and dK += dS^T Q (M128 N128 K64); warp 0 loads,
+//                warps 1 and 3 issue (S^T + dV, dP^T + dK), warps 4-7 take one
+//                key row each.
+// A single thread can issue a tcgen05.mma only about every 110-120 cycles, so the
+// tensor pipe is kept busy by several issuing threads.  Warp 1 owns TMEM.
 // Every wait is bounded and every warp-collective TMEM access is made from a
 // converged warp with warp-uniform decisions.
 //
@@ -56,6 +59,7 @@ struct BwdArgs {
     const int32_t *ucount;            // kMasked: valid routes per block
     const unsigned long long *umask;  // kMasked: token mask per route
     int n_sub, hc;  // dQ CTAs per KV group, query heads per dQ CTA (4, 2 or 1)
+    int rph;        // query rows per head in a dQ CTA (32 when hc = 4, else 64)
     long long hist_stride, seg_stride;
     const int32_t *idx;
     const float *lse;
@@ -76,27 +80,45 @@ __device__ __forceinline__ void store_row_sw128(uint32_t row_addr, int r, const 
                          pk[4 * cc + 3]);
 }
 
+// One thread can issue a tcgen05.mma only about every 110-120 cycles, while an
+// M128 N64 K16 MMA with both operands in shared memory occupies the tensor pipe for
+// ~55 cycles: the pipe is fed only by several threads issuing at once.  An issuing
+// warp runs its loop converged and elects one lane per MMA (the same lane, which also
+// commits).
+__device__ __forceinline__ bool elect_one() {
+    uint32_t pred = 0;
+    asm volatile("{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\telect.sync rx|px, %1;\n\t@px mov.s32 %0, 1;\n\t}"
+                 : "+r"(pred)
+                 : "r"(0xffffffffu));
+    return pred != 0;
+}
+
 // ============================================================ dQ kernel
-template <int NH>
+// A dQ CTA holds one M=128 tile of query rows: HC heads x RPH rows of one query block
+// (4 x 32, two CTAs per block, when HC = 4; 2 x 64 when HC = 2; 64 rows repeated when
+// HC = 1).  Per key tile j: S_j = Q K_j^T and dP_j = dO V_j^T (M128 N64 K128, each from
+// its own issuing warp) into one of two TMEM buffers, dS_j in bf16 into one of two
+// shared-memory buffers, dQ += dS_j K_j (M128 N128 K64, a third issuing warp).  With
+// both buffers doubled, the MMAs of tile j+1 run while the softmax warps work on tile j.
 struct DqSmem {
-    static constexpr int NSTAGE = 2;
-    static constexpr uint32_t Q = 0;
-    static constexpr uint32_t DO = Q + NH * HALF_BYTES;
-    static constexpr uint32_t KV = DO + NH * HALF_BYTES;
-    static constexpr uint32_t DS = KV + NSTAGE * 2 * TILE_BYTES;
-    static constexpr uint32_t BAR = DS + NH * ROWS128_K64;
+    static constexpr int NSTAGE = 4;
+    static constexpr uint32_t Q = 0;                                // [2 col halves][128 rows][128 B]
+    static constexpr uint32_t DO = Q + HALF_BYTES;
+    static constexpr uint32_t KV = DO + HALF_BYTES;                 // per stage: K tile, V tile
+    static constexpr uint32_t DS = KV + NSTAGE * 2 * TILE_BYTES;    // 2 x [128 rows][128 B]
+    static constexpr uint32_t BAR = DS + 2 * ROWS128_K64;
     static constexpr uint32_t ALLOC = BAR + 1024 + 1024;
 };
 
 struct DqBars {
     uint64_t q_full;
-    uint64_t kv_full[2];
-    uint64_t kv_empty[2];
-    uint64_t sdp_full[2];
-    uint64_t sdp_free[2];
-    uint64_t ds_full[2];
-    uint64_t dq_done[2];
-    uint64_t drain[2];
+    uint64_t kv_full[DqSmem::NSTAGE];
+    uint64_t kv_empty[DqSmem::NSTAGE];  // dP issuer (V read) + dQ issuer (K read)
+    uint64_t sdp_full[2];               // S issuer + dP issuer
+    uint64_t sdp_free[2];               // 4 softmax warps have read S, dP
+    uint64_t ds_full[2];                // 4 softmax warps have stored dS
+    uint64_t ds_free[2];                // dQ += dS K of that buffer done
+    uint64_t drain[3];
     uint32_t tmem_base;
     int abort;
     int n_hist;
@@ -105,38 +127,43 @@ struct DqBars {
     int tiles[64];
 };
 
-template <int NH, int MODE>
-__device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_q,
-                                        const CUtensorMap &tm_do, const CUtensorMap &tm_kh, const CUtensorMap &tm_vh,
+// TMEM columns of a dQ CTA: dQ accumulator [0, 128); S/dP buffer b at 128 + 128 b
+// (S in its first 64 columns, dP in the next 64).
+template <int MODE>
+__device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_qd,
+                                        const CUtensorMap &tm_dod, const CUtensorMap &tm_kh, const CUtensorMap &tm_vh,
                                         const CUtensorMap &tm_ks, const CUtensorMap &tm_vs, const BwdArgs &a) {
-    using L = DqSmem<NH>;
+    using L = DqSmem;
     constexpr int NST = L::NSTAGE;
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     DqBars *bars = reinterpret_cast<DqBars *>(smem + L::BAR);
     const uint32_t sbase = tc::smem_u32(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nqb = a.seg_len / TILE;
-    const int n_units = a.batch * a.n_kv_heads * a.n_sub;
-    const int m = nqb - 1 - blk / n_units;
-    const int unit = blk % n_units;
-    const int bg = unit / a.n_sub;
+    const int n_slices = TILE / a.rph;
+    const int n_units = a.batch * a.n_kv_heads * a.n_sub * n_slices;
+    const int m = nqb - 1 - blk / n_units;  // longest blocks first
+    int rem = blk % n_units;
+    const int slice = rem % n_slices;
+    rem /= n_slices;
+    const int bg = rem / a.n_sub;
     const int b = bg / a.n_kv_heads, g = bg % a.n_kv_heads;
-    const int h0 = g * (a.n_q_heads / a.n_kv_heads) + (unit % a.n_sub) * a.hc;  // first query head of the CTA
+    const int h0 = g * (a.n_q_heads / a.n_kv_heads) + (rem % a.n_sub) * a.hc;  // first query head of the CTA
+    const int row0 = m * TILE + slice * a.rph;                                // first query row of the slice
 
     if (threadIdx.x == 0) {
         tc::mbar_init(&bars->q_full, 1);
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(&bars->kv_full[s], 1);
-            tc::mbar_init(&bars->kv_empty[s], NH);
+            tc::mbar_init(&bars->kv_empty[s], 2);
         }
-        for (int h = 0; h < 2; ++h) {
-            tc::mbar_init(&bars->sdp_full[h], 1);
-            tc::mbar_init(&bars->sdp_free[h], 4);
-            tc::mbar_init(&bars->ds_full[h], 4);
-            tc::mbar_init(&bars->dq_done[h], 1);
+        for (int bb = 0; bb < 2; ++bb) {
+            tc::mbar_init(&bars->sdp_full[bb], 2);
+            tc::mbar_init(&bars->sdp_free[bb], 4);
+            tc::mbar_init(&bars->ds_full[bb], 4);
+            tc::mbar_init(&bars->ds_free[bb], 1);
         }
-        tc::mbar_init(&bars->drain[0], 1);
-        tc::mbar_init(&bars->drain[1], 1);
+        for (int d = 0; d < 3; ++d) tc::mbar_init(&bars->drain[d], 1);
         bars->abort = 0;
         bars->issued = 0;
         tc::fence_mbar_init();
@@ -173,14 +200,15 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
 
     if (warp == 0) {
         if (lane == 0) {
-            tc::mbar_arrive_expect_tx(&bars->q_full, 2 * NH * HALF_BYTES);
-            for (int hh = 0; hh < 2 * NH; ++hh) {
-                const int qrow = (b * a.n_q_heads + h0 + (a.hc == 1 ? 0 : hh)) * a.seg_len + m * TILE;
-                const uint32_t off = (hh >> 1) * HALF_BYTES + (hh & 1) * (64 * 128);
-                tc::tma_load_2d(smem + L::Q + off, &tm_q, 0, qrow, &bars->q_full);
-                tc::tma_load_2d(smem + L::Q + off + 128 * 128, &tm_q, 64, qrow, &bars->q_full);
-                tc::tma_load_2d(smem + L::DO + off, &tm_do, 0, qrow, &bars->q_full);
-                tc::tma_load_2d(smem + L::DO + off + 128 * 128, &tm_do, 64, qrow, &bars->q_full);
+            // Q and dO: TMEM lane r holds head r / RPH (repeating head 0 when HC = 1), row row0 + r % RPH
+            tc::mbar_arrive_expect_tx(&bars->q_full, 2 * HALF_BYTES);
+            for (int hh = 0; hh < 128 / a.rph; ++hh) {
+                const int qrow = (b * a.n_q_heads + h0 + (hh < a.hc ? hh : 0)) * a.seg_len + row0;
+                const uint32_t off = hh * a.rph * 128;
+                tc::tma_load_2d(smem + L::Q + off, &tm_qd, 0, qrow, &bars->q_full);
+                tc::tma_load_2d(smem + L::Q + off + 128 * 128, &tm_qd, 64, qrow, &bars->q_full);
+                tc::tma_load_2d(smem + L::DO + off, &tm_dod, 0, qrow, &bars->q_full);
+                tc::tma_load_2d(smem + L::DO + off + 128 * 128, &tm_dod, 64, qrow, &bars->q_full);
             }
             int issued = 0;
             // kGroup: the routed groups in list order (invalid entries skipped), 64 / gs per tile
@@ -228,61 +256,68 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             }
             bars->issued = issued;
         }
-    } else if (warp == 1 || warp == 3) {
-        // one UMMA issuing thread per 128-row half (a thread issues one MMA per ~100 cycles)
-        const int h = warp == 1 ? 0 : 1;
-        if (lane == 0 && h < NH) {
-            const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * HALF_BYTES, 16, 1024);
-            const uint64_t do_desc = tc::desc_sw128(sbase + L::DO + h * HALF_BYTES, 16, 1024);
-            const uint64_t kv_desc = tc::desc_sw128(sbase + L::KV, 16, 1024);
-            const uint64_t kmn_desc = tc::desc_sw128(sbase + L::KV, 8192, 1024);
-            const uint64_t ds_desc = tc::desc_sw128(sbase + L::DS + h * ROWS128_K64, 16, 1024);
-            auto issue_dq = [&](int t) -> bool {
-                const int s = t % NST;
-                if (!tc::mbar_wait(&bars->ds_full[h], t & 1, abort, a.status)) return false;
-                tc::fence_after_sync();
-                const uint64_t kd = kmn_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
+    } else if (warp == 1 || warp == 2) {
+        // warp 1: S_j = Q K_j^T; warp 2: dP_j = dO V_j^T (and the V half of the stage's release)
+        const bool is_s = warp == 1;
+        const uint64_t a_desc = tc::desc_sw128(sbase + (is_s ? L::Q : L::DO), 16, 1024);
+        const uint64_t kv_desc = tc::desc_sw128(sbase + L::KV + (is_s ? 0u : TILE_BYTES), 16, 1024);
+        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->q_full, 0, abort, a.status));
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            const int s = j % NST, bb = j & 1;
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->kv_full[s], (j / NST) & 1, abort, a.status) &&
+                                             (j < 2 || tc::mbar_wait(&bars->sdp_free[bb], ((j >> 1) - 1) & 1, abort,
+                                                                     a.status)));
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint64_t kd = kv_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
+            const uint32_t d = tmem + 128 + 128 * bb + (is_s ? 0u : 64u);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    tc::mma_f16(tmem + 128 * h, ds_desc + (kk * 32 >> 4), kd + (kk * 2048 >> 4), IDESC_N128_BMN,
-                                (t > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&bars->dq_done[h]);
-                tc::mma_commit(&bars->kv_empty[s]);  // one arrival per half
-                return true;
-            };
-            bool ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
-            for (int j = 0; ok && j < n_tiles; ++j) {
-                const int s = j % NST;
-                if (!tc::mbar_wait(&bars->kv_full[s], (j / NST) & 1, abort, a.status)) { ok = false; break; }
-                if (j >= 1 && !tc::mbar_wait(&bars->sdp_free[h], (j - 1) & 1, abort, a.status)) { ok = false; break; }
-                tc::fence_after_sync();
-                const uint64_t kd = kv_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
-                const uint64_t vd = kd + (uint64_t)(TILE_BYTES >> 4);
-                // S = Q K^T and dP = dO V^T: two independent accumulators, interleaved
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                    const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
-                    tc::mma_f16(tmem + 256 + 128 * h, q_desc + aoff, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
-                    tc::mma_f16(tmem + 256 + 128 * h + 64, do_desc + aoff, vd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(&bars->sdp_full[h]);
-                if (j >= 1 && !issue_dq(j - 1)) { ok = false; break; }
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+                if (elect_one()) tc::mma_f16(d, a_desc + aoff, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                __syncwarp();
             }
-            if (ok) issue_dq(n_tiles - 1);
+            if (elect_one()) {
+                tc::mma_commit(&bars->sdp_full[bb]);
+                if (!is_s) tc::mma_commit(&bars->kv_empty[s]);
+            }
+            __syncwarp();
+        }
+    } else if (warp == 3) {
+        // dQ += dS_j K_j (K MN-major), then the K half of the stage's release
+        const uint64_t kmn_desc = tc::desc_sw128(sbase + L::KV, 8192, 1024);
+        const uint64_t ds_desc = tc::desc_sw128(sbase + L::DS, 16, 1024);
+        for (int j = 0; j < n_tiles; ++j) {
+            const int s = j % NST, bb = j & 1;
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->ds_full[bb], (j >> 1) & 1, abort, a.status))) break;
+            tc::fence_after_sync();
+            const uint64_t kd = kmn_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
+            const uint64_t dd = ds_desc + (uint64_t)((bb * ROWS128_K64) >> 4);
+#pragma unroll
+            for (int kk = 0; kk < TILE / 16; ++kk) {
+                if (elect_one())
+                    tc::mma_f16(tmem, dd + (kk * 32 >> 4), kd + (kk * 2048 >> 4), IDESC_N128_BMN,
+                                (j > 0 || kk > 0) ? 1u : 0u);
+                __syncwarp();
+            }
+            if (elect_one()) {
+                tc::mma_commit(&bars->ds_free[bb]);
+                tc::mma_commit(&bars->kv_empty[s]);
+            }
+            __syncwarp();
         }
     } else if (warp >= 4) {
-        const int h = (warp - 4) >> 2;
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
-        const int hh = 2 * h + (r >> 6);
-        const int i = r & 63;
-        const bool write = hh < a.hc;  // rows 64..127 repeat the head when HC = 1
+        const int hh = r / a.rph;
+        const int i = slice * a.rph + r % a.rph;  // row within the query block
+        const bool write = hh < a.hc;             // rows 64..127 repeat the head when HC = 1
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
         const long long row = ((long long)(b * a.n_q_heads + h0 + (write ? hh : 0))) * a.seg_len + m * TILE + i;
         const float lse2 = a.lse[row] * 1.4426950408889634f;
         const float dlt = a.delta[row];
-        const uint32_t ds_row = sbase + L::DS + h * ROWS128_K64 + (r >> 3) * 1024 + (r & 7) * 128;
+        const uint32_t ds_row = sbase + L::DS + (r >> 3) * 1024 + (r & 7) * 128;
         // kGroup: valid columns of the last history tile; kMasked: the row's token bit of
         // the next tile's mask (read one tile ahead)
         const int last_cols = MODE == kGroup ? bars->n_groups * a.gs - (n_hist - 1) * TILE : TILE;
@@ -290,6 +325,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         if (MODE == kMasked && n_hist > 0) mask_next = a.umask[bgm * a.topk];
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
+            const int bb = j & 1;
             // columns >= ncols of this tile are masked for this row
             int ncols = TILE;
             if constexpr (MODE == kGroup) {
@@ -301,7 +337,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                     if (j + 1 < n_hist) mask_next = a.umask[bgm * a.topk + j + 1];
                 }
             }
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[h], j & 1, abort, a.status))) {
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[bb], (j >> 1) & 1, abort, a.status))) {
                 ok = false;
                 break;
             }
@@ -311,7 +347,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t sv[32], dpv[32];
-                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * h + 32 * half;
+                const uint32_t s_addr = tmem + lane_addr + 128 + 128 * bb + 32 * half;
                 tc::tmem_ld32(s_addr, sv);
                 tc::tmem_ld32(s_addr + 64, dpv);
                 tc::tmem_wait_ld();
@@ -328,24 +364,27 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             }
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[h]);
-            if (j >= 1 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->dq_done[h], (j - 1) & 1, abort, a.status))) {
+            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[bb]);
+            // dS buffer bb is free once dQ += dS K of tile j - 2 has read it
+            if (j >= 2 &&
+                !__all_sync(0xffffffffu, tc::mbar_wait(&bars->ds_free[bb], ((j >> 1) - 1) & 1, abort, a.status))) {
                 ok = false;
                 break;
             }
-            store_row_sw128(ds_row, r, pk);
+            store_row_sw128(ds_row + bb * ROWS128_K64, r, pk);
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->ds_full[h]);
+            if (lane == 0) tc::mbar_arrive(&bars->ds_full[bb]);
         }
-        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->dq_done[h], (n_tiles - 1) & 1, abort, a.status))) {
+        const int jl = n_tiles - 1;
+        if (ok && __all_sync(0xffffffffu, tc::mbar_wait(&bars->ds_free[jl & 1], (jl >> 1) & 1, abort, a.status))) {
             tc::fence_after_sync();
             float *out = a.dq + row * D;
 #pragma unroll 1
             for (int c0 = 0; c0 < D; c0 += 32) {
                 uint32_t o[32];
-                tc::tmem_ld32(tmem + lane_addr + 128 * h + c0, o);
+                tc::tmem_ld32(tmem + lane_addr + c0, o);
                 tc::tmem_wait_ld();
                 if (!write) continue;
 #pragma unroll
@@ -367,9 +406,12 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                 tc::mbar_wait(&bars->kv_full[j % NST], (j / NST) & 1, &never, a.status, 1ll << 28);
             tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
         }
-        if ((warp == 1 || (warp == 3 && NH == 2)) && lane == 0) {
-            tc::mma_commit(&bars->drain[warp == 3]);
-            tc::mbar_wait(&bars->drain[warp == 3], 0, &never, a.status, 1ll << 28);
+        if (warp >= 1 && warp <= 3) {
+            // the lane that issued this warp's MMAs commits and waits for them
+            if (elect_one()) {
+                tc::mma_commit(&bars->drain[warp - 1]);
+                tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
+            }
         }
         __syncwarp();
         tc::fence_after_sync();
@@ -651,9 +693,12 @@ bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
 // key-major dK/dV body (most work first), the rest the query-major dQ body.
 // The causal dK/dV blocks are very uneven (the first key tile is seen by
 // every later query tile), so the dQ blocks fill the SMs around them.
-template <int NH, int MODE>
-__global__ void __launch_bounds__(128 + 128 * NH, 1)
+// tm_q / tm_do have 64-row boxes (dK/dV query tiles), tm_qd / tm_dod boxes of
+// RPH rows (a dQ CTA's rows of one head).
+template <int MODE>
+__global__ void __launch_bounds__(256, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_qd, const __grid_constant__ CUtensorMap tm_dod,
                   const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
                   const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                   const BwdArgs a, const int n_kv_ctas) {
@@ -661,21 +706,21 @@ __global__ void __launch_bounds__(128 + 128 * NH, 1)
     if ((int)blockIdx.x < n_kv_ctas)
         dkdv_body((int)blockIdx.x, smem_raw, tm_q, tm_do, tm_ks, tm_vs, a);
     else
-        dq_body<NH, MODE>((int)blockIdx.x - n_kv_ctas, smem_raw, tm_q, tm_do, tm_kh, tm_vh, tm_ks, tm_vs, a);
+        dq_body<MODE>((int)blockIdx.x - n_kv_ctas, smem_raw, tm_qd, tm_dod, tm_kh, tm_vh, tm_ks, tm_vs, a);
 }
 
-template <int NH, int MODE>
-hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUtensorMap &mdo,
-                        const CUtensorMap &mkh, const CUtensorMap &mvh, const CUtensorMap &mks,
-                        const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
-    auto kern = bwd_tc_kernel<NH, MODE>;
-    const size_t smem = DqSmem<NH>::ALLOC > DkvSmem::ALLOC ? DqSmem<NH>::ALLOC : DkvSmem::ALLOC;
+template <int MODE>
+hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUtensorMap &mdo, const CUtensorMap &mqd,
+                        const CUtensorMap &mdod, const CUtensorMap &mkh, const CUtensorMap &mvh,
+                        const CUtensorMap &mks, const CUtensorMap &mvs, const BwdArgs &a, cudaStream_t stream) {
+    auto kern = bwd_tc_kernel<MODE>;
+    const size_t smem = DqSmem::ALLOC > DkvSmem::ALLOC ? DqSmem::ALLOC : DkvSmem::ALLOC;
     cudaError_t e = set_max_dynamic_smem(reinterpret_cast<const void *>(kern), (int)smem);
     if (e != cudaSuccess) return record_cuda(e);
     const int n_bg = p.batch * p.n_kv_heads;
     const int n_kv_ctas = ((p.seg_len + 127) / 128) * n_bg;
-    const unsigned grid = (unsigned)(n_kv_ctas + (p.seg_len / p.q_block) * n_bg * a.n_sub);
-    kern<<<grid, 128 + 128 * NH, smem, stream>>>(mq, mdo, mkh, mvh, mks, mvs, a, n_kv_ctas);
+    const unsigned grid = (unsigned)(n_kv_ctas + (p.seg_len / p.q_block) * n_bg * a.n_sub * (TILE / a.rph));
+    kern<<<grid, 256, smem, stream>>>(mq, mdo, mqd, mdod, mkh, mvh, mks, mvs, a, n_kv_ctas);
     return record_cuda(cudaGetLastError());
 }
 
@@ -697,7 +742,7 @@ hga_status_t launch_bwd_mode(const hga_params_t &p, const void *q, const void *k
                              const void *vs, const FwdRoutes &rt, const float *lse, const float *delta,
                              const void *dout, float *dq, float *dk, float *dv, unsigned *status,
                              cudaStream_t stream) {
-    CUtensorMap mq, mdo, mkh, mvh, mks, mvs;
+    CUtensorMap mq, mdo, mqd, mdod, mkh, mvh, mks, mvs;
     const long long n_bg = (long long)p.batch * p.n_kv_heads;
     const unsigned long long q_rows = (unsigned long long)p.batch * p.n_q_heads * p.seg_len;
     const long long hist_rows =
@@ -740,8 +785,14 @@ hga_status_t launch_bwd_mode(const hga_params_t &p, const void *q, const void *k
     const int G = p.n_q_heads / p.n_kv_heads;
     a.hc = G % 4 == 0 ? 4 : (G % 2 == 0 ? 2 : 1);
     a.n_sub = G / a.hc;
-    return G % 4 == 0 ? launch_bwd<2, MODE>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream)
-                      : launch_bwd<1, MODE>(p, mq, mdo, mkh, mvh, mks, mvs, a, stream);
+    a.rph = a.hc == 4 ? 32 : 64;
+    if (a.rph == 64) {
+        mqd = mq;
+        mdod = mdo;
+    } else if (!tma_rows_map(&mqd, q, q_rows, (unsigned)a.rph) || !tma_rows_map(&mdod, dout, q_rows, (unsigned)a.rph)) {
+        return HGA_ERR_INVALID_ARG;
+    }
+    return launch_bwd<MODE>(p, mq, mdo, mqd, mdod, mkh, mvh, mks, mvs, a, stream);
 }
 
 }  // namespace
