@@ -423,33 +423,50 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
 }
 
 // ============================================================ dK/dV kernel
+// A dK/dV CTA holds 128 segment keys (TMEM lanes) and walks the (head, later query
+// tile) steps of its KV group.  Per step t: S^T = K Q_t^T (warp 1) and dP^T = V dO_t^T
+// (warp 2) into one of two TMEM buffers; the softmax warps write P^T and dS^T as bf16
+// pairs back into the same buffer (over the S^T and dP^T columns they have read), and
+// warp 3 issues dV += P^T dO_t and dK += dS^T Q_t with A read from TMEM.  So the next
+// step's S^T / dP^T run while the softmax works on this one.
 struct DkvSmem {
-    static constexpr int NSTAGE = 3;
+    static constexpr int NSTAGE = 4;
     static constexpr uint32_t K = 0;                          // 128 keys, K-major
     static constexpr uint32_t V = K + HALF_BYTES;
     static constexpr uint32_t RING = V + HALF_BYTES;          // per stage: Q tile, dO tile
     static constexpr uint32_t STAGE_BYTES = 2 * TILE_BYTES;
-    static constexpr uint32_t PT = RING + NSTAGE * STAGE_BYTES;  // P^T  [128 keys][64 q] bf16
-    static constexpr uint32_t DST = PT + ROWS128_K64;          // dS^T
-    static constexpr uint32_t ROWT = DST + ROWS128_K64;        // per stage: lse2[64], delta[64]
+    static constexpr uint32_t ROWT = RING + NSTAGE * STAGE_BYTES;  // per stage: lse[64], delta[64]
     static constexpr uint32_t BAR = ROWT + NSTAGE * 512;
     static constexpr uint32_t ALLOC = BAR + 1024 + 1024;
 };
 
 struct DkvBars {
     uint64_t kv_full;
-    uint64_t ring_full[3];
-    uint64_t ring_empty[3];
-    uint64_t sdp_full[2];
-    uint64_t sdp_free[2];
-    uint64_t pds_full;
-    uint64_t pds_free;
-    uint64_t drain[2];
+    uint64_t ring_full[DkvSmem::NSTAGE];
+    uint64_t ring_empty[DkvSmem::NSTAGE];  // dV / dK of the step done (the last readers of Q_t, dO_t)
+    uint64_t sdp_full[2];                  // S^T issuer + dP^T issuer
+    uint64_t pds_full[2];                  // 4 softmax warps have stored P^T, dS^T
+    uint64_t buf_free[2];                  // dV / dK of that buffer done
+    uint64_t drain[3];
     uint32_t tmem_base;
     int abort;
     int issued;
 };
 
+// D[tmem] (+)= A[tmem] * B[smem] for one K=16 step of kind::f16 (A read from TMEM:
+// lane = row, 8 columns of bf16 pairs per K step).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// TMEM columns of a dK/dV CTA: dV [0, 128), dK [128, 256), step buffer b at 256 + 128 b
+// (S^T then P^T in its first 64 columns, dP^T then dS^T in the next 64).
 __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_q,
                                           const CUtensorMap &tm_do, const CUtensorMap &tm_ks,
                                           const CUtensorMap &tm_vs, const BwdArgs &a) {
@@ -473,16 +490,14 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
         tc::mbar_init(&bars->kv_full, 1);
         for (int s = 0; s < NST; ++s) {
             tc::mbar_init(&bars->ring_full[s], 1);
-            tc::mbar_init(&bars->ring_empty[s], 2);
+            tc::mbar_init(&bars->ring_empty[s], 1);
         }
         for (int bb = 0; bb < 2; ++bb) {
-            tc::mbar_init(&bars->sdp_full[bb], 2);  // S^T and dP^T issuers
-            tc::mbar_init(&bars->sdp_free[bb], 4);
+            tc::mbar_init(&bars->sdp_full[bb], 2);
+            tc::mbar_init(&bars->pds_full[bb], 4);
+            tc::mbar_init(&bars->buf_free[bb], 1);
         }
-        tc::mbar_init(&bars->pds_full, 4);
-        tc::mbar_init(&bars->pds_free, 2);  // dV and dK issuers
-        tc::mbar_init(&bars->drain[0], 1);
-        tc::mbar_init(&bars->drain[1], 1);
+        for (int d = 0; d < 3; ++d) tc::mbar_init(&bars->drain[d], 1);
         bars->abort = 0;
         bars->issued = 0;
         tc::fence_mbar_init();
@@ -525,71 +540,73 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             }
             bars->issued = issued;
         }
-    } else if (warp == 1 || warp == 3) {
-        // two UMMA issuing threads (a thread issues one MMA per ~100 cycles):
-        // warp 1 issues S^T = K Q^T and dV += P^T dO, warp 3 dP^T = V dO^T and dK += dS^T Q
-        const bool first = warp == 1;
-        if (lane == 0) {
-            const uint64_t kv_desc = tc::desc_sw128(sbase + (first ? L::K : L::V), 16, 1024);
-            const uint64_t ring_desc = tc::desc_sw128(sbase + L::RING, 16, 1024);
-            const uint64_t ring_mn_desc = tc::desc_sw128(sbase + L::RING, 8192, 1024);
-            const uint64_t a_desc = tc::desc_sw128(sbase + (first ? L::PT : L::DST), 16, 1024);
-            // stage operand of each issuer: Q tile for S^T / dK, dO tile for dP^T / dV
-            const uint32_t s_op = first ? 0u : TILE_BYTES;     // S^T uses Q, dP^T uses dO
-            const uint32_t g_op = first ? TILE_BYTES : 0u;     // dV uses dO, dK uses Q
-            const uint32_t acc = first ? 0u : 128u;            // dV at 0, dK at 128
-            auto issue_grads = [&](int t) -> bool {
-                const int s = t % NST;
-                if (!tc::mbar_wait(&bars->pds_full, t & 1, abort, a.status)) return false;
-                tc::fence_after_sync();
-                const uint64_t bd = ring_mn_desc + (uint64_t)((s * L::STAGE_BYTES + g_op) >> 4);
+    } else if (warp == 1 || warp == 2) {
+        // warp 1: S^T = K Q_t^T; warp 2: dP^T = V dO_t^T
+        const bool is_s = warp == 1;
+        const uint64_t a_desc = tc::desc_sw128(sbase + (is_s ? L::K : L::V), 16, 1024);
+        const uint64_t ring_desc = tc::desc_sw128(sbase + L::RING + (is_s ? 0u : TILE_BYTES), 16, 1024);
+        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->kv_full, 0, abort, a.status));
+        for (int t = 0; ok && t < n_steps; ++t) {
+            const int s = t % NST, bb = t & 1;
+            ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status) &&
+                                             (t < 2 || tc::mbar_wait(&bars->buf_free[bb], ((t >> 1) - 1) & 1, abort,
+                                                                     a.status)));
+            if (!ok) break;
+            tc::fence_after_sync();
+            const uint64_t bd = ring_desc + (uint64_t)((s * L::STAGE_BYTES) >> 4);
+            const uint32_t d = tmem + 256 + 128 * bb + (is_s ? 0u : 64u);
 #pragma unroll
-                for (int kk = 0; kk < TILE / 16; ++kk)
-                    tc::mma_f16(tmem + acc, a_desc + (kk * 32 >> 4), bd + (kk * 2048 >> 4), IDESC_N128_BMN,
-                                (t > 0 || kk > 0) ? 1u : 0u);
-                tc::mma_commit(&bars->pds_free);       // one arrival per issuer
-                tc::mma_commit(&bars->ring_empty[s]);  // one arrival per issuer
-                return true;
-            };
-            bool ok = tc::mbar_wait(&bars->kv_full, 0, abort, a.status);
-            for (int t = 0; ok && t < n_steps; ++t) {
-                const int s = t % NST, bb = t & 1;
-                if (!tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status)) { ok = false; break; }
-                if (t >= 2 && !tc::mbar_wait(&bars->sdp_free[bb], ((t >> 1) - 1) & 1, abort, a.status)) {
-                    ok = false;
-                    break;
-                }
-                tc::fence_after_sync();
-                const uint64_t bd = ring_desc + (uint64_t)((s * L::STAGE_BYTES + s_op) >> 4);
-                const uint32_t d = tmem + 256 + 128 * bb + (first ? 0u : 64u);
-#pragma unroll
-                for (int kk = 0; kk < D / 16; ++kk) {
-                    const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                    const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
-                    tc::mma_f16(d, kv_desc + aoff, bd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
-                }
-                tc::mma_commit(&bars->sdp_full[bb]);  // one arrival per issuer
-                if (t >= 1 && !issue_grads(t - 1)) { ok = false; break; }
+            for (int kk = 0; kk < D / 16; ++kk) {
+                const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
+                const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
+                if (elect_one()) tc::mma_f16(d, a_desc + aoff, bd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                __syncwarp();
             }
-            if (ok && n_steps > 0) issue_grads(n_steps - 1);
+            if (elect_one()) tc::mma_commit(&bars->sdp_full[bb]);
+            __syncwarp();
+        }
+    } else if (warp == 3) {
+        // dV += P^T dO_t and dK += dS^T Q_t (A from TMEM, B MN-major in the ring stage)
+        const uint64_t ring_mn_desc = tc::desc_sw128(sbase + L::RING, 8192, 1024);
+        for (int t = 0; t < n_steps; ++t) {
+            const int s = t % NST, bb = t & 1;
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->pds_full[bb], (t >> 1) & 1, abort, a.status))) break;
+            tc::fence_after_sync();
+            const uint64_t qd = ring_mn_desc + (uint64_t)((s * L::STAGE_BYTES) >> 4);
+            const uint64_t gd = qd + (uint64_t)(TILE_BYTES >> 4);
+            const uint32_t pa = tmem + 256 + 128 * bb;
+#pragma unroll
+            for (int kk = 0; kk < TILE / 16; ++kk) {
+                if (elect_one())
+                    mma_f16_ts(tmem, pa + 8 * kk, gd + (kk * 2048 >> 4), IDESC_N128_BMN, (t > 0 || kk > 0) ? 1u : 0u);
+                __syncwarp();
+            }
+#pragma unroll
+            for (int kk = 0; kk < TILE / 16; ++kk) {
+                if (elect_one())
+                    mma_f16_ts(tmem + 128, pa + 64 + 8 * kk, qd + (kk * 2048 >> 4), IDESC_N128_BMN,
+                               (t > 0 || kk > 0) ? 1u : 0u);
+                __syncwarp();
+            }
+            if (elect_one()) {
+                tc::mma_commit(&bars->buf_free[bb]);
+                tc::mma_commit(&bars->ring_empty[s]);
+            }
+            __syncwarp();
         }
     } else if (warp >= 4 && warp < 8) {
         const int quad = warp & 3;
         const int r = quad * 32 + lane;  // key row = TMEM lane
         const int key = key0 + r;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
-        const uint32_t pt_row = sbase + L::PT + (r >> 3) * 1024 + (r & 7) * 128;
-        const uint32_t dst_row = sbase + L::DST + (r >> 3) * 1024 + (r & 7) * 128;
         bool ok = true;
         for (int t = 0; t < n_steps; ++t) {
             const int s = t % NST, bb = t & 1;
             const int mq = m0 + t % (nqb - m0);
-            // the stage's lse / delta rows (TMA-written), this step's S^T, dP^T in TMEM,
-            // and the P^T / dS^T buffers free again (the previous step's dV, dK done)
+            // the stage's lse / delta rows (TMA-written) and this step's S^T, dP^T in TMEM
             if (!__all_sync(0xffffffffu,
                             tc::mbar_wait(&bars->ring_full[s], (t / NST) & 1, abort, a.status) &&
-                                tc::mbar_wait(&bars->sdp_full[bb], (t >> 1) & 1, abort, a.status) &&
-                                (t == 0 || tc::mbar_wait(&bars->pds_free, (t - 1) & 1, abort, a.status)))) {
+                                tc::mbar_wait(&bars->sdp_full[bb], (t >> 1) & 1, abort, a.status))) {
                 ok = false;
                 break;
             }
@@ -597,14 +614,14 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             const float *lse2 = reinterpret_cast<const float *>(smem + L::ROWT + s * 512);
             const float *dlt = lse2 + 64;
             const int q0 = mq * TILE;  // first query position of the tile
+            const uint32_t buf = tmem + lane_addr + 256 + 128 * bb;
+            uint32_t ppk[32], dpk[32];
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t sv[32], dpv[32];
-                const uint32_t s_addr = tmem + lane_addr + 256 + 128 * bb + 32 * half;
-                tc::tmem_ld32(s_addr, sv);
-                tc::tmem_ld32(s_addr + 64, dpv);
+                tc::tmem_ld32(buf + 32 * half, sv);
+                tc::tmem_ld32(buf + 64 + 32 * half, dpv);
                 tc::tmem_wait_ld();
-                uint32_t ppk[16], dpk[16];
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
                     const int c0 = 32 * half + c;
@@ -612,31 +629,24 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
                     float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2[c0 + 1] * 1.4426950408889634f);
                     if (key > q0 + c0) p0 = 0.f;      // causal: the key comes after the query
                     if (key > q0 + c0 + 1) p1 = 0.f;
-                    ppk[c / 2] = tc::pack_bf16(p0, p1);
-                    dpk[c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
-                                               p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
-                }
-#pragma unroll
-                for (int cc = 0; cc < 4; ++cc) {
-                    const int chunk = 4 * half + cc;
-                    tc::st_shared_v4(pt_row + ((chunk ^ (r & 7)) << 4), ppk[4 * cc], ppk[4 * cc + 1], ppk[4 * cc + 2],
-                                     ppk[4 * cc + 3]);
-                    tc::st_shared_v4(dst_row + ((chunk ^ (r & 7)) << 4), dpk[4 * cc], dpk[4 * cc + 1],
-                                     dpk[4 * cc + 2], dpk[4 * cc + 3]);
+                    ppk[16 * half + c / 2] = tc::pack_bf16(p0, p1);
+                    dpk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
+                                                           p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
                 }
             }
-            tc::fence_proxy_async();
+            // P^T over the S^T columns, dS^T over the dP^T columns (both read above)
+            tc::tmem_st32(buf, ppk);
+            tc::tmem_st32(buf + 64, dpk);
+            tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) {
-                tc::mbar_arrive(&bars->sdp_free[bb]);
-                tc::mbar_arrive(&bars->pds_full);
-            }
+            if (lane == 0) tc::mbar_arrive(&bars->pds_full[bb]);
         }
-        const bool done = ok && (n_steps == 0 ||
-                                 __all_sync(0xffffffffu, tc::mbar_wait(&bars->pds_free, (n_steps - 1) & 1, abort,
-                                                                       a.status)));
-        if (done && n_steps > 0) {
+        const int tl = n_steps - 1;
+        const bool done = ok && n_steps > 0 &&
+                          __all_sync(0xffffffffu, tc::mbar_wait(&bars->buf_free[tl & 1], (tl >> 1) & 1, abort,
+                                                                a.status));
+        if (done) {
             tc::fence_after_sync();
             const bool valid = key < a.seg_len;
             const long long orow = (long long)bg * a.seg_len + key;
@@ -671,9 +681,12 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
                 tc::mbar_wait(&bars->ring_full[t % NST], (t / NST) & 1, &never, a.status, 1ll << 28);
             tc::mbar_wait(&bars->kv_full, 0, &never, a.status, 1ll << 28);
         }
-        if ((warp == 1 || warp == 3) && lane == 0) {
-            tc::mma_commit(&bars->drain[warp == 3]);
-            tc::mbar_wait(&bars->drain[warp == 3], 0, &never, a.status, 1ll << 28);
+        if (warp >= 1 && warp <= 3) {
+            // the lane that issued this warp's MMAs commits and waits for them
+            if (elect_one()) {
+                tc::mma_commit(&bars->drain[warp - 1]);
+                tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
+            }
         }
         __syncwarp();
         tc::fence_after_sync();
