@@ -80,19 +80,6 @@ __device__ __forceinline__ void store_row_sw128(uint32_t row_addr, int r, const 
                          pk[4 * cc + 3]);
 }
 
-// One thread can issue a tcgen05.mma only about every 110-120 cycles, while an
-// M128 N64 K16 MMA with both operands in shared memory occupies the tensor pipe for
-// ~55 cycles: the pipe is fed only by several threads issuing at once.  An issuing
-// warp runs its loop converged and elects one lane per MMA (the same lane, which also
-// commits).
-__device__ __forceinline__ bool elect_one() {
-    uint32_t pred = 0;
-    asm volatile("{\n\t.reg .b32 rx;\n\t.reg .pred px;\n\telect.sync rx|px, %1;\n\t@px mov.s32 %0, 1;\n\t}"
-                 : "+r"(pred)
-                 : "r"(0xffffffffu));
-    return pred != 0;
-}
-
 // ============================================================ dQ kernel
 // A dQ CTA holds one M=128 tile of query rows: HC heads x RPH rows of one query block
 // (4 x 32, two CTAs per block, when HC = 4; 2 x 64 when HC = 2; 64 rows repeated when
@@ -275,10 +262,10 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
                 const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
-                if (elect_one()) tc::mma_f16(d, a_desc + aoff, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                if (tc::elect_one()) tc::mma_f16(d, a_desc + aoff, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
                 __syncwarp();
             }
-            if (elect_one()) {
+            if (tc::elect_one()) {
                 tc::mma_commit(&bars->sdp_full[bb]);
                 if (!is_s) tc::mma_commit(&bars->kv_empty[s]);
             }
@@ -296,12 +283,12 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             const uint64_t dd = ds_desc + (uint64_t)((bb * ROWS128_K64) >> 4);
 #pragma unroll
             for (int kk = 0; kk < TILE / 16; ++kk) {
-                if (elect_one())
+                if (tc::elect_one())
                     tc::mma_f16(tmem, dd + (kk * 32 >> 4), kd + (kk * 2048 >> 4), IDESC_N128_BMN,
                                 (j > 0 || kk > 0) ? 1u : 0u);
                 __syncwarp();
             }
-            if (elect_one()) {
+            if (tc::elect_one()) {
                 tc::mma_commit(&bars->ds_free[bb]);
                 tc::mma_commit(&bars->kv_empty[s]);
             }
@@ -408,7 +395,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         }
         if (warp >= 1 && warp <= 3) {
             // the lane that issued this warp's MMAs commits and waits for them
-            if (elect_one()) {
+            if (tc::elect_one()) {
                 tc::mma_commit(&bars->drain[warp - 1]);
                 tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
             }
@@ -559,10 +546,10 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
                 const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
-                if (elect_one()) tc::mma_f16(d, a_desc + aoff, bd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                if (tc::elect_one()) tc::mma_f16(d, a_desc + aoff, bd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
                 __syncwarp();
             }
-            if (elect_one()) tc::mma_commit(&bars->sdp_full[bb]);
+            if (tc::elect_one()) tc::mma_commit(&bars->sdp_full[bb]);
             __syncwarp();
         }
     } else if (warp == 3) {
@@ -577,18 +564,18 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             const uint32_t pa = tmem + 256 + 128 * bb;
 #pragma unroll
             for (int kk = 0; kk < TILE / 16; ++kk) {
-                if (elect_one())
+                if (tc::elect_one())
                     mma_f16_ts(tmem, pa + 8 * kk, gd + (kk * 2048 >> 4), IDESC_N128_BMN, (t > 0 || kk > 0) ? 1u : 0u);
                 __syncwarp();
             }
 #pragma unroll
             for (int kk = 0; kk < TILE / 16; ++kk) {
-                if (elect_one())
+                if (tc::elect_one())
                     mma_f16_ts(tmem + 128, pa + 64 + 8 * kk, qd + (kk * 2048 >> 4), IDESC_N128_BMN,
                                (t > 0 || kk > 0) ? 1u : 0u);
                 __syncwarp();
             }
-            if (elect_one()) {
+            if (tc::elect_one()) {
                 tc::mma_commit(&bars->buf_free[bb]);
                 tc::mma_commit(&bars->ring_empty[s]);
             }
@@ -683,7 +670,7 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
         }
         if (warp >= 1 && warp <= 3) {
             // the lane that issued this warp's MMAs commits and waits for them
-            if (elect_one()) {
+            if (tc::elect_one()) {
                 tc::mma_commit(&bars->drain[warp - 1]);
                 tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
             }

@@ -335,57 +335,74 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
         // ------------------------------------------------------------ UMMA issuers
         const int h = (warp - 1) >> 1;      // M half
         const bool qk = (warp & 1) != 0;    // warps 1, 3: QK^T; warps 2, 4: PV
-        if (lane == 0 && warp <= 4 && h < NH) {
+        if (warp <= 4 && h < NH) {
+            // The whole warp runs the loop (waits included) and elects one lane per MMA.
             // Descriptors are built once; a K-step, stage or buffer offset is added
             // to the start-address field (addresses stay below 2^18, so no carry).
             bool ok = true;
             if (qk) {
                 const uint64_t q_desc = tc::desc_sw128(sbase + L::Q + h * Q_HALF_BYTES, 16, 1024);
                 const uint64_t k_desc = tc::desc_sw128(sbase + L::K, 16, 1024);
-                ok = tc::mbar_wait(&bars->q_full, 0, abort, a.status);
+                ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->q_full, 0, abort, a.status));
                 for (int j = 0; ok && j < n_tiles; ++j) {
                     const int s = j % NSTAGE, bb = j & 1;
-                    if (!resolve_tiles(j)) break;
+                    if (!__all_sync(0xffffffffu, resolve_tiles(j))) break;
                     if (j >= n_tiles) break;
-                    if (!tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)) break;
+                    if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->k_full[s], (j / NSTAGE) & 1, abort, a.status)))
+                        break;
                     // S buffer bb is free once PV(j-2), which read P(j-2) from it, has completed
-                    if (j >= 2 && !tc::mbar_wait(&bars->o_done[h][bb], ((j >> 1) - 1) & 1, abort, a.status))
+                    if (j >= 2 && !__all_sync(0xffffffffu, tc::mbar_wait(&bars->o_done[h][bb], ((j >> 1) - 1) & 1,
+                                                                         abort, a.status)))
                         break;
                     // half 1 runs half a tile behind half 0: its S(j) lands while half 0
                     // is in the exp phase of tile j, so the two softmax groups take
                     // turns on the MUFU instead of stalling on it together
-                    if (h == 1 && j >= 1 && !wait_count(&bars->sm0_tiles, j, abort, a.status)) break;
+                    if (h == 1 && j >= 1 && !__all_sync(0xffffffffu, wait_count(&bars->sm0_tiles, j, abort, a.status)))
+                        break;
                     tc::fence_after_sync();
                     const uint64_t kd = k_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
 #pragma unroll
                     for (int kk = 0; kk < D / 16; ++kk) {
                         const uint32_t koff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
                         const uint32_t qoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
-                        tc::mma_f16(tmem + 256 + 128 * h + 64 * bb, q_desc + qoff, kd + koff, IDESC_QK,
-                                    kk > 0 ? 1u : 0u);
+                        if (tc::elect_one())
+                            tc::mma_f16(tmem + 256 + 128 * h + 64 * bb, q_desc + qoff, kd + koff, IDESC_QK,
+                                        kk > 0 ? 1u : 0u);
+                        __syncwarp();
                     }
-                    tc::mma_commit(&bars->s_full[h][bb]);
-                    tc::mma_commit(&bars->k_empty[s]);  // one arrival per half
+                    if (tc::elect_one()) {
+                        tc::mma_commit(&bars->s_full[h][bb]);
+                        tc::mma_commit(&bars->k_empty[s]);  // one arrival per half
+                    }
+                    __syncwarp();
                 }
             } else {
                 const uint64_t v_desc = tc::desc_sw128(sbase + L::V, 8192, 1024);
                 const uint32_t o_tmem = tmem + 128 * h;
                 for (int t = 0; t < n_tiles; ++t) {
                     const int s = t % NSTAGE, pb = t & 1;
-                    if (!resolve_tiles(t)) break;
+                    if (!__all_sync(0xffffffffu, resolve_tiles(t))) break;
                     if (t >= n_tiles) break;
-                    if (!tc::mbar_wait(&bars->v_full[s], (t / NSTAGE) & 1, abort, a.status)) break;
-                    if (!tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort, a.status)) break;
+                    if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->v_full[s], (t / NSTAGE) & 1, abort, a.status) &&
+                                                     tc::mbar_wait(&bars->p_full[h][pb], (t >> 1) & 1, abort,
+                                                                   a.status)))
+                        break;
                     tc::fence_after_sync();
                     const uint64_t vd = v_desc + (uint64_t)((s * KV_TILE_BYTES) >> 4);
                     // P(t) as bf16 pairs in the first 32 columns of S buffer pb: 8 columns per K step
                     const uint32_t pa = tmem + 256 + 128 * h + 64 * pb;
 #pragma unroll
-                    for (int kk = 0; kk < TILE / 16; ++kk)
-                        mma_f16_ts(o_tmem, pa + 8 * kk, vd + (kk * 2048 >> 4), IDESC_PV,
-                                   (t > 0 || kk > 0) ? 1u : 0u);
-                    tc::mma_commit(&bars->o_done[h][pb]);
-                    tc::mma_commit(&bars->v_empty[s]);  // one arrival per half
+                    for (int kk = 0; kk < TILE / 16; ++kk) {
+                        if (tc::elect_one())
+                            mma_f16_ts(o_tmem, pa + 8 * kk, vd + (kk * 2048 >> 4), IDESC_PV,
+                                       (t > 0 || kk > 0) ? 1u : 0u);
+                        __syncwarp();
+                    }
+                    if (tc::elect_one()) {
+                        tc::mma_commit(&bars->o_done[h][pb]);
+                        tc::mma_commit(&bars->v_empty[s]);  // one arrival per half
+                    }
+                    __syncwarp();
                 }
             }
         }
@@ -560,9 +577,12 @@ __global__ void __launch_bounds__(32 * kCtrlWarps + 128 * NH, 1)
             }
             tc::mbar_wait(&bars->q_full, 0, &never, a.status, 1ll << 28);
         }
-        if (warp >= 1 && warp <= 4 && lane == 0 && ((warp - 1) >> 1) < NH) {
-            tc::mma_commit(&bars->drain[warp - 1]);
-            tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
+        if (warp >= 1 && warp <= 4 && ((warp - 1) >> 1) < NH) {
+            // the lane that issued this warp's MMAs commits and waits for them
+            if (tc::elect_one()) {
+                tc::mma_commit(&bars->drain[warp - 1]);
+                tc::mbar_wait(&bars->drain[warp - 1], 0, &never, a.status, 1ll << 28);
+            }
         }
         __syncwarp();
         tc::fence_after_sync();
