@@ -70,8 +70,8 @@ CSRC = "hierarchical_sparse_long_b200/csrc/"
 # the translation unit of each kernel (and the PTX wrappers it inlines): a stored
 # ncu traffic figure stays valid while these sources are unchanged
 KERNEL_SOURCES = {
-    "attn_fwd": [CSRC + "attn_fwd_tc.cu", CSRC + "tc_ptx.cuh"],
-    "attn_bwd": [CSRC + "attn_bwd_tc.cu", CSRC + "tc_ptx.cuh"],
+    "attn_fwd": [CSRC + "attn_fwd_tc.cu", CSRC + "tc_ptx.cuh", CSRC + "tc_issue.cuh"],
+    "attn_bwd": [CSRC + "attn_bwd_tc.cu", CSRC + "tc_ptx.cuh", CSRC + "tc_issue.cuh"],
     "route": [CSRC + "route.cu", CSRC + "tc_ptx.cuh"],
     "summaries": [CSRC + "summaries.cu"],
     "fetch": [CSRC + "tiered.cu"],

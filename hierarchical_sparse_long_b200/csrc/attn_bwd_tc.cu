@@ -38,6 +38,7 @@
 // chunk.  A masked key gets P = 0, so it adds nothing to dQ.
 #include <cudaTypedefs.h>
 
+#include "tc_issue.cuh"
 #include "tc_ptx.cuh"
 
 namespace hga {

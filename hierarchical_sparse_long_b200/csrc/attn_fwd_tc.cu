@@ -64,6 +64,7 @@
 // before the route kernel started.
 #include <cudaTypedefs.h>
 
+#include "tc_issue.cuh"
 #include "tc_ptx.cuh"
 
 namespace hga {
