@@ -10,24 +10,25 @@
 //   dQ = dS K / sqrt(D)                      over routed history and segment keys
 //   dK_seg = dS^T Q / sqrt(D), dV_seg = P^T dO   over segment keys only
 //
-// Two block types in one launch of 256-thread blocks, no atomics (results are
+// Two block types in one launch of 384-thread blocks, no atomics (results are
 // deterministic):
 //   dQ blocks  : query-major, one CTA per M=128 tile of query rows: HC heads of the
 //                group (4, 2 or 1, as in the forward) x 128 / HC rows of one query
 //                block (two CTAs per block when HC = 4);
 //                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128) into one
-//                of two TMEM buffers, the dS rows in bf16 into one of two shared-
+//                of three TMEM buffers, the dS rows in bf16 into one of two shared-
 //                memory buffers, dQ += dS K (M128 N128 K64); warp 0 loads, warps 1,
 //                2 and 3 issue S, dP and dQ, warps 4-7 take one row each.
 //   dK/dV blocks: key-major over the active segment, one CTA per (batch, kv
 //                head, 128 segment keys); for every later 64-query tile of
 //                every head of the group: S^T = K Q^T and dP^T = V dO^T
-//                (M128 N64 K128), P^T and dS^T in bf16 into shared memory,
-//                dV += P^T dO and dK += dS^T Q (M128 N128 K64); warp 0 loads,
-//                warps 1 and 3 issue (S^T + dV, dP^T + dK), warps 4-7 take one
-//                key row each.
-// A single thread can issue a tcgen05.mma only about every 110-120 cycles, so the
-// tensor pipe is kept busy by several issuing threads.  Warp 1 owns TMEM.
+//                (M128 N64 K128) into one of two TMEM buffers, P^T and dS^T in
+//                bf16 written back into that buffer, dV += P^T dO and dK += dS^T Q
+//                (M128 N128 K64, A from TMEM); warp 0 loads, warps 1 and 2 issue
+//                S^T and dP^T, warp 3 dV and dK, warps 4-11 take half a key row
+//                each (32 query columns).
+// Each MMA-issuing warp runs its loop converged and elects one lane per MMA and for
+// the commits that track them; warp 1 owns TMEM.
 // Every wait is bounded and every warp-collective TMEM access is made from a
 // converged warp with warp-uniform decisions.
 //
@@ -85,9 +86,10 @@ __device__ __forceinline__ void store_row_sw128(uint32_t row_addr, int r, const 
 // A dQ CTA holds one M=128 tile of query rows: HC heads x RPH rows of one query block
 // (4 x 32, two CTAs per block, when HC = 4; 2 x 64 when HC = 2; 64 rows repeated when
 // HC = 1).  Per key tile j: S_j = Q K_j^T and dP_j = dO V_j^T (M128 N64 K128, each from
-// its own issuing warp) into one of two TMEM buffers, dS_j in bf16 into one of two
-// shared-memory buffers, dQ += dS_j K_j (M128 N128 K64, a third issuing warp).  With
-// both buffers doubled, the MMAs of tile j+1 run while the softmax warps work on tile j.
+// its own issuing warp) into one of three TMEM buffers, dS_j in bf16 into one of two
+// shared-memory buffers, dQ += dS_j K_j (M128 N128 K64, a third issuing warp).  The MMAs
+// of tiles j+1 and j+2 run while the softmax warps work on tile j: issuing and running
+// S and dP of a tile takes longer than the softmax of one.
 struct DqSmem {
     static constexpr int NSTAGE = 4;
     static constexpr uint32_t Q = 0;                                // [2 col halves][128 rows][128 B]
@@ -102,8 +104,8 @@ struct DqBars {
     uint64_t q_full;
     uint64_t kv_full[DqSmem::NSTAGE];
     uint64_t kv_empty[DqSmem::NSTAGE];  // dP issuer (V read) + dQ issuer (K read)
-    uint64_t sdp_full[2];               // S issuer + dP issuer
-    uint64_t sdp_free[2];               // 4 softmax warps have read S, dP
+    uint64_t sdp_full[3];               // S issuer + dP issuer
+    uint64_t sdp_free[3];               // 4 softmax warps have read S, dP
     uint64_t ds_full[2];                // 4 softmax warps have stored dS
     uint64_t ds_free[2];                // dQ += dS K of that buffer done
     uint64_t drain[3];
@@ -115,8 +117,8 @@ struct DqBars {
     int tiles[64];
 };
 
-// TMEM columns of a dQ CTA: dQ accumulator [0, 128); S/dP buffer b at 128 + 128 b
-// (S in its first 64 columns, dP in the next 64).
+// TMEM columns of a dQ CTA: dQ accumulator [0, 128); S/dP buffer b (b < 3) at
+// 128 + 128 b (S in its first 64 columns, dP in the next 64).
 template <int MODE>
 __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_qd,
                                         const CUtensorMap &tm_dod, const CUtensorMap &tm_kh, const CUtensorMap &tm_vh,
@@ -145,9 +147,11 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             tc::mbar_init(&bars->kv_full[s], 1);
             tc::mbar_init(&bars->kv_empty[s], 2);
         }
-        for (int bb = 0; bb < 2; ++bb) {
+        for (int bb = 0; bb < 3; ++bb) {
             tc::mbar_init(&bars->sdp_full[bb], 2);
             tc::mbar_init(&bars->sdp_free[bb], 4);
+        }
+        for (int bb = 0; bb < 2; ++bb) {
             tc::mbar_init(&bars->ds_full[bb], 4);
             tc::mbar_init(&bars->ds_free[bb], 1);
         }
@@ -251,14 +255,14 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         const uint64_t kv_desc = tc::desc_sw128(sbase + L::KV + (is_s ? 0u : TILE_BYTES), 16, 1024);
         bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->q_full, 0, abort, a.status));
         for (int j = 0; ok && j < n_tiles; ++j) {
-            const int s = j % NST, bb = j & 1;
+            const int s = j % NST, sb = j % 3;
             ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->kv_full[s], (j / NST) & 1, abort, a.status) &&
-                                             (j < 2 || tc::mbar_wait(&bars->sdp_free[bb], ((j >> 1) - 1) & 1, abort,
+                                             (j < 3 || tc::mbar_wait(&bars->sdp_free[sb], ((j / 3) - 1) & 1, abort,
                                                                      a.status)));
             if (!ok) break;
             tc::fence_after_sync();
             const uint64_t kd = kv_desc + (uint64_t)((s * 2 * TILE_BYTES) >> 4);
-            const uint32_t d = tmem + 128 + 128 * bb + (is_s ? 0u : 64u);
+            const uint32_t d = tmem + 128 + 128 * sb + (is_s ? 0u : 64u);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
                 const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
@@ -267,7 +271,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                 __syncwarp();
             }
             if (tc::elect_one()) {
-                tc::mma_commit(&bars->sdp_full[bb]);
+                tc::mma_commit(&bars->sdp_full[sb]);
                 if (!is_s) tc::mma_commit(&bars->kv_empty[s]);
             }
             __syncwarp();
@@ -295,7 +299,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             }
             __syncwarp();
         }
-    } else if (warp >= 4) {
+    } else if (warp >= 4 && warp < 8) {
         const int quad = warp & 3;
         const int r = quad * 32 + lane;
         const int hh = r / a.rph;
@@ -313,7 +317,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         if (MODE == kMasked && n_hist > 0) mask_next = a.umask[bgm * a.topk];
         bool ok = true;
         for (int j = 0; j < n_tiles; ++j) {
-            const int bb = j & 1;
+            const int bb = j & 1, sb = j % 3;
             // columns >= ncols of this tile are masked for this row
             int ncols = TILE;
             if constexpr (MODE == kGroup) {
@@ -325,7 +329,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                     if (j + 1 < n_hist) mask_next = a.umask[bgm * a.topk + j + 1];
                 }
             }
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[bb], (j >> 1) & 1, abort, a.status))) {
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[sb], (j / 3) & 1, abort, a.status))) {
                 ok = false;
                 break;
             }
@@ -335,7 +339,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
 #pragma unroll
             for (int half = 0; half < 2; ++half) {
                 uint32_t sv[32], dpv[32];
-                const uint32_t s_addr = tmem + lane_addr + 128 + 128 * bb + 32 * half;
+                const uint32_t s_addr = tmem + lane_addr + 128 + 128 * sb + 32 * half;
                 tc::tmem_ld32(s_addr, sv);
                 tc::tmem_ld32(s_addr + 64, dpv);
                 tc::tmem_wait_ld();
@@ -352,7 +356,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             }
             tc::fence_before_sync();
             __syncwarp();
-            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[bb]);
+            if (lane == 0) tc::mbar_arrive(&bars->sdp_free[sb]);
             // dS buffer bb is free once dQ += dS K of tile j - 2 has read it
             if (j >= 2 &&
                 !__all_sync(0xffffffffu, tc::mbar_wait(&bars->ds_free[bb], ((j >> 1) - 1) & 1, abort, a.status))) {
@@ -413,10 +417,11 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
 // ============================================================ dK/dV kernel
 // A dK/dV CTA holds 128 segment keys (TMEM lanes) and walks the (head, later query
 // tile) steps of its KV group.  Per step t: S^T = K Q_t^T (warp 1) and dP^T = V dO_t^T
-// (warp 2) into one of two TMEM buffers; the softmax warps write P^T and dS^T as bf16
-// pairs back into the same buffer (over the S^T and dP^T columns they have read), and
-// warp 3 issues dV += P^T dO_t and dK += dS^T Q_t with A read from TMEM.  So the next
-// step's S^T / dP^T run while the softmax works on this one.
+// (warp 2) into one of two TMEM buffers; two warps per key row (warps 4-7: query columns
+// 0..31, warps 8-11: 32..63) write P^T and dS^T as bf16 pairs back into the same buffer,
+// each over the first half of the S^T / dP^T columns it has read, and warp 3 issues
+// dV += P^T dO_t and dK += dS^T Q_t with A read from TMEM.  So the next step's S^T /
+// dP^T run while the softmax works on this one.
 struct DkvSmem {
     static constexpr int NSTAGE = 4;
     static constexpr uint32_t K = 0;                          // 128 keys, K-major
@@ -453,8 +458,18 @@ __device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uin
         : "memory");
 }
 
-// TMEM columns of a dK/dV CTA: dV [0, 128), dK [128, 256), step buffer b at 256 + 128 b
-// (S^T then P^T in its first 64 columns, dP^T then dS^T in the next 64).
+// 32 lanes x 16 consecutive 32-bit columns from registers.
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+        "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
+        "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+        : "memory");
+}
+
+// TMEM columns of a dK/dV CTA: dV [0, 128), dK [128, 256), step buffer b at 256 + 128 b:
+// S^T in its first 64 columns, dP^T in the next 64; P^T of query columns 0..31 / 32..63
+// lands in columns 0..15 / 32..47 of the buffer, dS^T in 64..79 / 96..111.
 __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_q,
                                           const CUtensorMap &tm_do, const CUtensorMap &tm_ks,
                                           const CUtensorMap &tm_vs, const BwdArgs &a) {
@@ -482,7 +497,7 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
         }
         for (int bb = 0; bb < 2; ++bb) {
             tc::mbar_init(&bars->sdp_full[bb], 2);
-            tc::mbar_init(&bars->pds_full[bb], 4);
+            tc::mbar_init(&bars->pds_full[bb], 8);
             tc::mbar_init(&bars->buf_free[bb], 1);
         }
         for (int d = 0; d < 3; ++d) tc::mbar_init(&bars->drain[d], 1);
@@ -562,17 +577,20 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             tc::fence_after_sync();
             const uint64_t qd = ring_mn_desc + (uint64_t)((s * L::STAGE_BYTES) >> 4);
             const uint64_t gd = qd + (uint64_t)(TILE_BYTES >> 4);
+            // P^T (dS^T) of query columns 0..31 at columns 0..15 (64..79), of 32..63 at 32..47 (96..111)
             const uint32_t pa = tmem + 256 + 128 * bb;
 #pragma unroll
             for (int kk = 0; kk < TILE / 16; ++kk) {
+                const uint32_t ka = (kk & 1) * 8 + (kk >> 1) * 32;
                 if (tc::elect_one())
-                    mma_f16_ts(tmem, pa + 8 * kk, gd + (kk * 2048 >> 4), IDESC_N128_BMN, (t > 0 || kk > 0) ? 1u : 0u);
+                    mma_f16_ts(tmem, pa + ka, gd + (kk * 2048 >> 4), IDESC_N128_BMN, (t > 0 || kk > 0) ? 1u : 0u);
                 __syncwarp();
             }
 #pragma unroll
             for (int kk = 0; kk < TILE / 16; ++kk) {
+                const uint32_t ka = (kk & 1) * 8 + (kk >> 1) * 32;
                 if (tc::elect_one())
-                    mma_f16_ts(tmem + 128, pa + 64 + 8 * kk, qd + (kk * 2048 >> 4), IDESC_N128_BMN,
+                    mma_f16_ts(tmem + 128, pa + 64 + ka, qd + (kk * 2048 >> 4), IDESC_N128_BMN,
                                (t > 0 || kk > 0) ? 1u : 0u);
                 __syncwarp();
             }
@@ -582,8 +600,9 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             }
             __syncwarp();
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4) {
         const int quad = warp & 3;
+        const int part = (warp - 4) >> 2;  // query columns 32 part .. 32 part + 31 of each step
         const int r = quad * 32 + lane;  // key row = TMEM lane
         const int key = key0 + r;
         const uint32_t lane_addr = (uint32_t)(quad * 32) << 16;
@@ -602,29 +621,28 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             const float *lse2 = reinterpret_cast<const float *>(smem + L::ROWT + s * 512);
             const float *dlt = lse2 + 64;
             const int q0 = mq * TILE;  // first query position of the tile
-            const uint32_t buf = tmem + lane_addr + 256 + 128 * bb;
-            uint32_t ppk[32], dpk[32];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            const uint32_t buf = tmem + lane_addr + 256 + 128 * bb + 32 * part;
+            uint32_t ppk[16], dpk[16];
+            {
                 uint32_t sv[32], dpv[32];
-                tc::tmem_ld32(buf + 32 * half, sv);
-                tc::tmem_ld32(buf + 64 + 32 * half, dpv);
+                tc::tmem_ld32(buf, sv);
+                tc::tmem_ld32(buf + 64, dpv);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const int c0 = 32 * half + c;
+                    const int c0 = 32 * part + c;
                     float p0 = tc::ex2(__uint_as_float(sv[c]) * a.scale_log2 - lse2[c0] * 1.4426950408889634f);
                     float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2[c0 + 1] * 1.4426950408889634f);
                     if (key > q0 + c0) p0 = 0.f;      // causal: the key comes after the query
                     if (key > q0 + c0 + 1) p1 = 0.f;
-                    ppk[16 * half + c / 2] = tc::pack_bf16(p0, p1);
-                    dpk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
-                                                           p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
+                    ppk[c / 2] = tc::pack_bf16(p0, p1);
+                    dpk[c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt[c0]),
+                                               p1 * (__uint_as_float(dpv[c + 1]) - dlt[c0 + 1]));
                 }
             }
-            // P^T over the S^T columns, dS^T over the dP^T columns (both read above)
-            tc::tmem_st32(buf, ppk);
-            tc::tmem_st32(buf + 64, dpk);
+            // P^T / dS^T over the first 16 of the 32 S^T / dP^T columns this warp has read
+            tmem_st16(buf, ppk);
+            tmem_st16(buf + 64, dpk);
             tc::tmem_wait_st();
             tc::fence_before_sync();
             __syncwarp();
@@ -638,8 +656,8 @@ __device__ __forceinline__ void dkdv_body(const int blk, uint8_t *smem_raw, cons
             tc::fence_after_sync();
             const bool valid = key < a.seg_len;
             const long long orow = (long long)bg * a.seg_len + key;
-#pragma unroll 1
-            for (int which = 0; which < 2; ++which) {  // 0: dV, 1: dK
+            {
+                const int which = part;  // part 0 writes dV, part 1 dK
                 float *out = (which ? a.dk : a.dv) + orow * D;
                 const float sc = which ? a.scale : 1.f;
 #pragma unroll 1
@@ -697,7 +715,7 @@ bool make_map(CUtensorMap *map, const void *base, unsigned long long rows) {
 // tm_q / tm_do have 64-row boxes (dK/dV query tiles), tm_qd / tm_dod boxes of
 // RPH rows (a dQ CTA's rows of one head).
 template <int MODE>
-__global__ void __launch_bounds__(256, 1)
+__global__ void __launch_bounds__(384, 1)
     bwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_do,
                   const __grid_constant__ CUtensorMap tm_qd, const __grid_constant__ CUtensorMap tm_dod,
                   const __grid_constant__ CUtensorMap tm_kh, const __grid_constant__ CUtensorMap tm_vh,
@@ -721,7 +739,7 @@ hga_status_t launch_bwd(const hga_params_t &p, const CUtensorMap &mq, const CUte
     const int n_bg = p.batch * p.n_kv_heads;
     const int n_kv_ctas = ((p.seg_len + 127) / 128) * n_bg;
     const unsigned grid = (unsigned)(n_kv_ctas + (p.seg_len / p.q_block) * n_bg * a.n_sub * (TILE / a.rph));
-    kern<<<grid, 256, smem, stream>>>(mq, mdo, mqd, mdod, mkh, mvh, mks, mvs, a, n_kv_ctas);
+    kern<<<grid, 384, smem, stream>>>(mq, mdo, mqd, mdod, mkh, mvh, mks, mvs, a, n_kv_ctas);
     return record_cuda(cudaGetLastError());
 }
 

@@ -26,9 +26,9 @@
 //               stored there.
 //   warps 2, 4  PV issuers, one thread per M half:
 //               O_h += P_h V    (M128 N128 K64, P from TMEM, V MN-major),
-//               issued as soon as the softmax has written P.  One thread
-//               issues a tcgen05.mma only about every 100 cycles, so the four
-//               issue streams run in separate threads.
+//               issued as soon as the softmax has written P.  The four issue
+//               streams run in separate warps, each converged with one lane
+//               elected per MMA.
 //   warps 5+4h.. softmax of half h: one TMEM lane (= query row) per thread
 //               (a warp reads the lane quadrant of its warp index % 4, so any
 //               four consecutive warps cover the half's 128 rows); online
