@@ -74,22 +74,27 @@ struct BwdArgs {
     float scale;       // 1 / sqrt(D)
 };
 
-// Writes 32 packed bf16 pairs (64 values) of row r as a 128-byte SW128 row.
-__device__ __forceinline__ void store_row_sw128(uint32_t row_addr, int r, const uint32_t (&pk)[32]) {
-#pragma unroll
-    for (int cc = 0; cc < 8; ++cc)
-        tc::st_shared_v4(row_addr + ((cc ^ (r & 7)) << 4), pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2],
-                         pk[4 * cc + 3]);
+// D[tmem] (+)= A[tmem] * B[smem] for one K=16 step of kind::f16 (A read from TMEM:
+// lane = row, 8 columns of bf16 pairs per K step).
+__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
+                                           uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
+        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
 }
 
 // ============================================================ dQ kernel
 // A dQ CTA holds one M=128 tile of query rows: HC heads x RPH rows of one query block
 // (4 x 32, two CTAs per block, when HC = 4; 2 x 64 when HC = 2; 64 rows repeated when
-// HC = 1).  Per key tile j: S_j = Q K_j^T and dP_j = dO V_j^T (M128 N64 K128, each from
-// its own issuing warp) into one of three TMEM buffers, dS_j in bf16 into one of two
-// shared-memory buffers, dQ += dS_j K_j (M128 N128 K64, a third issuing warp).  The MMAs
-// of tiles j+1 and j+2 run while the softmax warps work on tile j: issuing and running
-// S and dP of a tile takes longer than the softmax of one.
+// HC = 1).  Q and dO are copied once into TMEM, so S_j = Q K_j^T and dP_j = dO V_j^T
+// (M128 N64 K128, each from its own issuing warp) read only K_j / V_j from shared memory
+// (an MMA with both operands there re-reads 4 KiB of A for every 2 KiB of B, and shared-
+// memory operand bandwidth bounds the tile); they land in one of two TMEM buffers, dS_j
+// goes in bf16 into one of two shared-memory buffers, dQ += dS_j K_j (M128 N128 K64, a
+// third issuing warp).  Two warps per row (32 key columns each) form dS.
 struct DqSmem {
     static constexpr int NSTAGE = 4;
     static constexpr uint32_t Q = 0;                                // [2 col halves][128 rows][128 B]
@@ -104,9 +109,10 @@ struct DqBars {
     uint64_t q_full;
     uint64_t kv_full[DqSmem::NSTAGE];
     uint64_t kv_empty[DqSmem::NSTAGE];  // dP issuer (V read) + dQ issuer (K read)
-    uint64_t sdp_full[3];               // S issuer + dP issuer
-    uint64_t sdp_free[3];               // 4 softmax warps have read S, dP
-    uint64_t ds_full[2];                // 4 softmax warps have stored dS
+    uint64_t qt_full;                   // Q and dO copied into TMEM (8 row warps)
+    uint64_t sdp_full[2];               // S issuer + dP issuer
+    uint64_t sdp_free[2];               // 8 row warps have read S, dP
+    uint64_t ds_full[2];                // 8 row warps have stored dS
     uint64_t ds_free[2];                // dQ += dS K of that buffer done
     uint64_t drain[3];
     uint32_t tmem_base;
@@ -117,8 +123,9 @@ struct DqBars {
     int tiles[64];
 };
 
-// TMEM columns of a dQ CTA: dQ accumulator [0, 128); S/dP buffer b (b < 3) at
-// 128 + 128 b (S in its first 64 columns, dP in the next 64).
+// TMEM columns of a dQ CTA: dQ accumulator [0, 128); S/dP buffer b (b < 2) at
+// 128 + 128 b (S in its first 64 columns, dP in the next 64); Q as bf16 pairs at
+// [384, 448), dO at [448, 512).
 template <int MODE>
 __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const CUtensorMap &tm_qd,
                                         const CUtensorMap &tm_dod, const CUtensorMap &tm_kh, const CUtensorMap &tm_vh,
@@ -147,12 +154,13 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             tc::mbar_init(&bars->kv_full[s], 1);
             tc::mbar_init(&bars->kv_empty[s], 2);
         }
-        for (int bb = 0; bb < 3; ++bb) {
+        tc::mbar_init(&bars->qt_full, 8);
+        for (int bb = 0; bb < 2; ++bb) {
             tc::mbar_init(&bars->sdp_full[bb], 2);
-            tc::mbar_init(&bars->sdp_free[bb], 4);
+            tc::mbar_init(&bars->sdp_free[bb], 8);
         }
         for (int bb = 0; bb < 2; ++bb) {
-            tc::mbar_init(&bars->ds_full[bb], 4);
+            tc::mbar_init(&bars->ds_full[bb], 8);
             tc::mbar_init(&bars->ds_free[bb], 1);
         }
         for (int d = 0; d < 3; ++d) tc::mbar_init(&bars->drain[d], 1);
@@ -251,13 +259,13 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
     } else if (warp == 1 || warp == 2) {
         // warp 1: S_j = Q K_j^T; warp 2: dP_j = dO V_j^T (and the V half of the stage's release)
         const bool is_s = warp == 1;
-        const uint64_t a_desc = tc::desc_sw128(sbase + (is_s ? L::Q : L::DO), 16, 1024);
+        const uint32_t a_tmem = tmem + (is_s ? 384u : 448u);  // Q or dO as bf16 pairs, 8 columns per K step
         const uint64_t kv_desc = tc::desc_sw128(sbase + L::KV + (is_s ? 0u : TILE_BYTES), 16, 1024);
-        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->q_full, 0, abort, a.status));
+        bool ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->qt_full, 0, abort, a.status));
         for (int j = 0; ok && j < n_tiles; ++j) {
-            const int s = j % NST, sb = j % 3;
+            const int s = j % NST, sb = j & 1;
             ok = __all_sync(0xffffffffu, tc::mbar_wait(&bars->kv_full[s], (j / NST) & 1, abort, a.status) &&
-                                             (j < 3 || tc::mbar_wait(&bars->sdp_free[sb], ((j / 3) - 1) & 1, abort,
+                                             (j < 2 || tc::mbar_wait(&bars->sdp_free[sb], ((j >> 1) - 1) & 1, abort,
                                                                      a.status)));
             if (!ok) break;
             tc::fence_after_sync();
@@ -265,9 +273,8 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             const uint32_t d = tmem + 128 + 128 * sb + (is_s ? 0u : 64u);
 #pragma unroll
             for (int kk = 0; kk < D / 16; ++kk) {
-                const uint32_t aoff = ((kk >> 2) * (128 * 128) + (kk & 3) * 32) >> 4;
                 const uint32_t boff = ((kk >> 2) * (64 * 128) + (kk & 3) * 32) >> 4;
-                if (tc::elect_one()) tc::mma_f16(d, a_desc + aoff, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
+                if (tc::elect_one()) mma_f16_ts(d, a_tmem + 8 * kk, kd + boff, IDESC_N64, kk > 0 ? 1u : 0u);
                 __syncwarp();
             }
             if (tc::elect_one()) {
@@ -299,8 +306,9 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             }
             __syncwarp();
         }
-    } else if (warp >= 4 && warp < 8) {
+    } else if (warp >= 4) {
         const int quad = warp & 3;
+        const int part = (warp - 4) >> 2;  // key columns 32 part .. 32 part + 31 of each tile
         const int r = quad * 32 + lane;
         const int hh = r / a.rph;
         const int i = slice * a.rph + r % a.rph;  // row within the query block
@@ -310,14 +318,38 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
         const float lse2 = a.lse[row] * 1.4426950408889634f;
         const float dlt = a.delta[row];
         const uint32_t ds_row = sbase + L::DS + (r >> 3) * 1024 + (r & 7) * 128;
+        bool ok = true;
+        // Q (part 0) or dO (part 1) row r from its 128-byte-swizzled shared-memory tile into
+        // TMEM lane r as 64 columns of bf16 pairs
+        if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->q_full, 0, abort, a.status))) {
+            ok = false;
+        } else {
+            const uint8_t *src = smem + (part ? L::DO : L::Q) + (r >> 3) * 1024 + (r & 7) * 128;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf) {
+                uint32_t v[32];
+#pragma unroll
+                for (int c = 0; c < 8; ++c) {
+                    const uint4 w = *reinterpret_cast<const uint4 *>(src + hf * 16384 + ((c ^ (r & 7)) << 4));
+                    v[4 * c] = w.x;
+                    v[4 * c + 1] = w.y;
+                    v[4 * c + 2] = w.z;
+                    v[4 * c + 3] = w.w;
+                }
+                tc::tmem_st32(tmem + lane_addr + (part ? 448u : 384u) + 32 * hf, v);
+            }
+            tc::tmem_wait_st();
+            tc::fence_before_sync();
+            __syncwarp();
+            if (lane == 0) tc::mbar_arrive(&bars->qt_full);
+        }
         // kGroup: valid columns of the last history tile; kMasked: the row's token bit of
         // the next tile's mask (read one tile ahead)
         const int last_cols = MODE == kGroup ? bars->n_groups * a.gs - (n_hist - 1) * TILE : TILE;
         unsigned long long mask_next = 0ull;
         if (MODE == kMasked && n_hist > 0) mask_next = a.umask[bgm * a.topk];
-        bool ok = true;
-        for (int j = 0; j < n_tiles; ++j) {
-            const int bb = j & 1, sb = j % 3;
+        for (int j = 0; ok && j < n_tiles; ++j) {
+            const int bb = j & 1, sb = j & 1;
             // columns >= ncols of this tile are masked for this row
             int ncols = TILE;
             if constexpr (MODE == kGroup) {
@@ -329,29 +361,28 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                     if (j + 1 < n_hist) mask_next = a.umask[bgm * a.topk + j + 1];
                 }
             }
-            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[sb], (j / 3) & 1, abort, a.status))) {
+            if (!__all_sync(0xffffffffu, tc::mbar_wait(&bars->sdp_full[sb], (j >> 1) & 1, abort, a.status))) {
                 ok = false;
                 break;
             }
             tc::fence_after_sync();
             const bool diag = (j == n_tiles - 1);
-            uint32_t pk[32];
-#pragma unroll
-            for (int half = 0; half < 2; ++half) {
+            uint32_t pk[16];
+            {
                 uint32_t sv[32], dpv[32];
-                const uint32_t s_addr = tmem + lane_addr + 128 + 128 * sb + 32 * half;
+                const uint32_t s_addr = tmem + lane_addr + 128 + 128 * sb + 32 * part;
                 tc::tmem_ld32(s_addr, sv);
                 tc::tmem_ld32(s_addr + 64, dpv);
                 tc::tmem_wait_ld();
 #pragma unroll
                 for (int c = 0; c < 32; c += 2) {
-                    const int c0 = 32 * half + c;
+                    const int c0 = 32 * part + c;
                     float p0 = tc::ex2(__uint_as_float(sv[c]) * a.scale_log2 - lse2);
                     float p1 = tc::ex2(__uint_as_float(sv[c + 1]) * a.scale_log2 - lse2);
                     if ((diag && c0 > i) || c0 >= ncols) p0 = 0.f;
                     if ((diag && c0 + 1 > i) || c0 + 1 >= ncols) p1 = 0.f;
-                    pk[16 * half + c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt),
-                                                          p1 * (__uint_as_float(dpv[c + 1]) - dlt));
+                    pk[c / 2] = tc::pack_bf16(p0 * (__uint_as_float(dpv[c]) - dlt),
+                                              p1 * (__uint_as_float(dpv[c + 1]) - dlt));
                 }
             }
             tc::fence_before_sync();
@@ -363,7 +394,11 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
                 ok = false;
                 break;
             }
-            store_row_sw128(ds_row + bb * ROWS128_K64, r, pk);
+            // this warp's 64 bytes of the row: 16-byte chunks 4 part .. 4 part + 3 (128-byte swizzle)
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc)
+                tc::st_shared_v4(ds_row + bb * ROWS128_K64 + (((4 * part + cc) ^ (r & 7)) << 4), pk[4 * cc],
+                                 pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
             tc::fence_proxy_async();
             tc::fence_before_sync();
             __syncwarp();
@@ -374,7 +409,7 @@ __device__ __forceinline__ void dq_body(const int blk, uint8_t *smem_raw, const 
             tc::fence_after_sync();
             float *out = a.dq + row * D;
 #pragma unroll 1
-            for (int c0 = 0; c0 < D; c0 += 32) {
+            for (int c0 = 64 * part; c0 < 64 * part + 64; c0 += 32) {
                 uint32_t o[32];
                 tc::tmem_ld32(tmem + lane_addr + c0, o);
                 tc::tmem_wait_ld();
@@ -445,18 +480,6 @@ struct DkvBars {
     int abort;
     int issued;
 };
-
-// D[tmem] (+)= A[tmem] * B[smem] for one K=16 step of kind::f16 (A read from TMEM:
-// lane = row, 8 columns of bf16 pairs per K step).
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "setp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-        ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
 
 // 32 lanes x 16 consecutive 32-bit columns from registers.
 __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
