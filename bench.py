@@ -128,12 +128,40 @@ def dist_setup():
     return rank, world, local
 
 
+def code_text(src):
+    """C/C++/CUDA source with its comments removed and blank or trailing space dropped:
+    what the compiler sees, so an edit of comments alone keeps a kernel's stored counters.
+    String and character literals are kept whole (an inline-asm string may hold '//')."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            j = src.find("\n", i)
+            i = n if j < 0 else j
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            out.append(" ")
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    lines = (ln.rstrip() for ln in "".join(out).splitlines())
+    return "\n".join(ln for ln in lines if ln)
+
+
 def file_hash(paths):
+    """Hash of the code (comments and blank lines dropped) of the given source files."""
     h = hashlib.sha256()
     for p in paths:
         fp = os.path.join(ROOT, p)
         if os.path.exists(fp):
-            h.update(open(fp, "rb").read())
+            h.update(code_text(open(fp, encoding="utf-8").read()).encode())
     return h.hexdigest()[:16]
 
 
