@@ -15,10 +15,11 @@
 //   dQ blocks  : query-major, one CTA per M=128 tile of query rows: HC heads of the
 //                group (4, 2 or 1, as in the forward) x 128 / HC rows of one query
 //                block (two CTAs per block when HC = 4);
-//                per key tile: S = Q K^T and dP = dO V^T (M128 N64 K128) into one
-//                of three TMEM buffers, the dS rows in bf16 into one of two shared-
-//                memory buffers, dQ += dS K (M128 N128 K64); warp 0 loads, warps 1,
-//                2 and 3 issue S, dP and dQ, warps 4-7 take one row each.
+//                Q and dO copied once into TMEM; per key tile: S = Q K^T and
+//                dP = dO V^T (M128 N64 K128, A from TMEM) into one of two TMEM
+//                buffers, the dS rows in bf16 into one of two shared-memory buffers,
+//                dQ += dS K (M128 N128 K64); warp 0 loads, warps 1, 2 and 3 issue S,
+//                dP and dQ, warps 4-11 take half a row each (32 key columns).
 //   dK/dV blocks: key-major over the active segment, one CTA per (batch, kv
 //                head, 128 segment keys); for every later 64-query tile of
 //                every head of the group: S^T = K Q^T and dP^T = V dO^T
