@@ -474,7 +474,7 @@ struct DkvBars {
     uint64_t ring_full[DkvSmem::NSTAGE];
     uint64_t ring_empty[DkvSmem::NSTAGE];  // dV / dK of the step done (the last readers of Q_t, dO_t)
     uint64_t sdp_full[2];                  // S^T issuer + dP^T issuer
-    uint64_t pds_full[2];                  // 4 softmax warps have stored P^T, dS^T
+    uint64_t pds_full[2];                  // 8 row warps have stored P^T, dS^T
     uint64_t buf_free[2];                  // dV / dK of that buffer done
     uint64_t drain[3];
     uint32_t tmem_base;
