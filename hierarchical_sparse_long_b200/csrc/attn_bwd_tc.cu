@@ -124,6 +124,9 @@ struct DqBars {
     int tiles[64];
 };
 
+static_assert(sizeof(DqBars) <= 1024, "dQ barrier block must fit its region");
+static_assert(DqSmem::ALLOC <= 227 * 1024, "dQ shared memory must fit one block's 227 KiB");
+
 // TMEM columns of a dQ CTA: dQ accumulator [0, 128); S/dP buffer b (b < 2) at
 // 128 + 128 b (S in its first 64 columns, dP in the next 64); Q as bf16 pairs at
 // [384, 448), dO at [448, 512).
@@ -490,6 +493,9 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16
         "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
         : "memory");
 }
+
+static_assert(sizeof(DkvBars) <= 1024, "dK/dV barrier block must fit its region");
+static_assert(DkvSmem::ALLOC <= 227 * 1024, "dK/dV shared memory must fit one block's 227 KiB");
 
 // TMEM columns of a dK/dV CTA: dV [0, 128), dK [128, 256), step buffer b at 256 + 128 b:
 // S^T in its first 64 columns, dP^T in the next 64; P^T of query columns 0..31 / 32..63
